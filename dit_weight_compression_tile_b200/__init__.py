@@ -1,0 +1,16 @@
+"""B200-native fused decode of lattice-rANS compressed weights.
+
+The library (``libeptile.so``, C ABI in ``include/eptile.h``) holds the host compressor,
+the stream parser and the sm_100a decode kernel; ``binding`` marshals torch tensors to
+it.  Importing the package loads nothing; the first use of a binding name imports
+``binding``, whose ``lib()`` fails loudly when the built library is missing.
+"""
+_BINDING_NAMES = ("BF16", "FP16", "FP32", "INT8", "FP8E4M3", "EpError", "compress", "decompress",
+                  "stream_info", "lib", "StreamInfo")
+
+
+def __getattr__(name):
+    if name in _BINDING_NAMES:
+        from . import binding
+        return getattr(binding, name)
+    raise AttributeError(name)

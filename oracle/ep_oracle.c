@@ -1,0 +1,1286 @@
+/*
+ * Oracle for the lattice-rANS tile stream -- TEST INFRASTRUCTURE ONLY.
+ * See ep_oracle.h for scope.  Build: gcc -std=c99 -O2 -ffp-contract=off -fPIC -shared.
+ *
+ * Sources followed (page title, section):
+ *   [ABS]  "EntroPack: Fast and Accurate Entropy-Coded Weight Compression at Arbitrary
+ *          Bitrates", Abstract -- row-normalized E8 lattice quantization, conditional
+ *          model of lattice coordinates, sampled storage estimates pick the resolution,
+ *          entropy coding in independently decodable tiles, fused decode + reconstruction,
+ *          BF16 / FP16 / FP8 / INT8 containers.
+ *   [API]  "EntroPack API reference", compress / CompressedTensor -- non-empty 2-D finite
+ *          input, actual_bpp = 8 * storage_nbytes / numel including metadata.
+ *   [README] "EntroPack README", Get started / Configuration -- target range [0.001, 11].
+ *   [LIN]  "Compressed Linear usage", Combine compression with FP8 or INT8 computation --
+ *          lossy compression applied to FP8/INT8 weight codes, target < 8, per-row scales
+ *          counted in storage.
+ * Textbook material restated here (not from the pages):
+ *   Conway & Sloane, "Fast quantizing and decoding algorithms for lattice quantizers and
+ *   codes" (IEEE Trans. IT, 1982): nearest point of D_n and of E8 = D8 u (D8 + 1/2).
+ *   Duda, "Asymmetric numeral systems" (2013): range variant rANS.
+ *   Giesen, "Interleaved entropy coders" (2014): several rANS states sharing one stream.
+ *   Micikevicius et al., "FP8 Formats for Deep Learning" (2022): E4M3 encoding.
+ */
+#include "ep_oracle.h"
+
+#include <float.h>
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------------------
+ * Stream constants (format version 1).  These are the build's readings of what the
+ * pages leave open: 11-bit frequency tables, 32-bit states with 16-bit renormalisation
+ * words, 32 interleaved states per tile, seven coding contexts.
+ * ---------------------------------------------------------------------------------- */
+#define MAGIC 0x31545045u /* bytes 'E','P','T','1' */
+#define VERSION 1
+#define PROB_BITS 11
+#define PROB_M 2048u
+#define STATE_L 65536u
+#define LANES 32
+#define NCTX 7
+#define MAX_SPLIT 7
+#define CHUNK_BITS 11
+#define HEADER_BYTES 64
+#define NQ 1280
+#define SAMPLE_TARGET 65536
+
+static size_t al16(size_t n) { return (n + 15) & ~(size_t)15; }
+
+/* ---------------------------------- scalar decode of inputs -------------------------- */
+static double half_to_double(uint16_t h)
+{
+    int s = h >> 15, e = (h >> 10) & 31, m = h & 1023;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + m), e - 25);
+    return s ? -v : v;
+}
+
+static double src_value(const void *src, int32_t dt, int64_t i)
+{
+    if (dt == ORD_BF16) {
+        uint32_t b = (uint32_t)((const uint16_t *)src)[i] << 16;
+        float f;
+        memcpy(&f, &b, 4);
+        return (double)f;
+    }
+    if (dt == ORD_FP16)
+        return half_to_double(((const uint16_t *)src)[i]);
+    return (double)((const float *)src)[i];
+}
+
+/* ---------------------------------- container conversions --------------------------- */
+/* fp32 -> bf16, round to nearest even (finite inputs; overflow rounds to infinity) */
+uint16_t or_bf16_from_float(float w)
+{
+    uint32_t b;
+    memcpy(&b, &w, 4);
+    if ((b & 0x7fffffffu) > 0x7f800000u)
+        return (uint16_t)((b >> 16) | 0x40);
+    b += 0x7fffu + ((b >> 16) & 1u);
+    return (uint16_t)(b >> 16);
+}
+
+/* fp32 -> IEEE binary16, round to nearest even, subnormals kept, overflow to infinity.
+ * Written from the binary16 definition: value = (-1)^s * 2^(e-15) * 1.m, e in [1,30]. */
+uint16_t or_fp16_from_float(float w)
+{
+    double a = fabs((double)w);
+    uint16_t s = signbit(w) ? 0x8000 : 0;
+    if (isnan(w))
+        return 0x7e00;
+    if (a < ldexp(1.0, -14)) { /* subnormal range: multiples of 2^-24 */
+        double q = nearbyint(a * ldexp(1.0, 24)); /* exact scaling, then RNE */
+        return (uint16_t)(s | (uint16_t)q);        /* q == 1024 is the smallest normal */
+    }
+    int e;
+    double fr = frexp(a, &e); /* a = fr * 2^e, fr in [0.5, 1) */
+    double mant = nearbyint(fr * 2048.0);  /* 11 significant bits, RNE */
+    if (mant == 2048.0) {
+        mant = 1024.0;
+        e += 1;
+    }
+    int be = e - 1 + 15;
+    if (be >= 31)
+        return (uint16_t)(s | 0x7c00);
+    return (uint16_t)(s | (uint16_t)(be << 10) | (uint16_t)((int)mant - 1024));
+}
+
+/* fp32 -> FP8 E4M3 (the "FN" variant: no infinities, S.1111.111 is NaN, max 448),
+ * round to nearest even, saturating to +-448.  Exponent bias 7, smallest normal 2^-6,
+ * subnormal step 2^-9. */
+uint8_t or_e4m3_from_float(float w)
+{
+    double a = fabs((double)w);
+    uint8_t s = signbit(w) ? 0x80 : 0;
+    if (isnan(w))
+        return 0x7f;
+    if (a < ldexp(1.0, -6)) {
+        double q = nearbyint(a * 512.0); /* multiples of 2^-9 */
+        return (uint8_t)(s | (uint8_t)q); /* q == 8 encodes 2^-6 exactly */
+    }
+    int e;
+    double fr = frexp(a, &e);
+    double mant = nearbyint(fr * 16.0); /* 4 significant bits */
+    if (mant == 16.0) {
+        mant = 8.0;
+        e += 1;
+    }
+    int be = e - 1 + 7;
+    int mm = (int)mant - 8;
+    if (be > 15 || (be == 15 && mm == 7))
+        return (uint8_t)(s | 0x7e); /* saturate to 448 */
+    return (uint8_t)(s | (uint8_t)(be << 3) | (uint8_t)mm);
+}
+
+/* fp32 -> int8 code: round to nearest even, clamp to the symmetric range [-127, 127] */
+int8_t or_int8_from_float(float w)
+{
+    if (w >= 127.0f)
+        return 127;
+    if (w <= -127.0f)
+        return -127;
+    return (int8_t)(int)nearbyintf(w);
+}
+
+static double e4m3_value(uint8_t c)
+{
+    int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v = e ? ldexp(8.0 + m, e - 10) : ldexp((double)m, -9);
+    return s ? -v : v;
+}
+
+void or_convert_batch(const float *w, int64_t n, int32_t dt, void *out)
+{
+    for (int64_t i = 0; i < n; i++) {
+        if (dt == ORD_BF16)
+            ((uint16_t *)out)[i] = or_bf16_from_float(w[i]);
+        else if (dt == ORD_FP16)
+            ((uint16_t *)out)[i] = or_fp16_from_float(w[i]);
+        else if (dt == ORD_FP32)
+            ((float *)out)[i] = w[i];
+        else if (dt == ORD_INT8)
+            ((int8_t *)out)[i] = or_int8_from_float(w[i]);
+        else
+            ((uint8_t *)out)[i] = or_e4m3_from_float(w[i]);
+    }
+}
+
+static int elt_size(int32_t dt)
+{
+    return dt == ORD_FP32 ? 4 : (dt == ORD_BF16 || dt == ORD_FP16) ? 2 : 1;
+}
+
+/* ---------------------------------- resolution grid ---------------------------------- */
+/* Reading: the "quantization resolution" is a lattice scale q on a fixed grid that is
+ * exact in binary floating point: q(k) = (64 + k mod 64) / 64 * 2^(floor(k/64) - 8),
+ * k in [0, 1280), i.e. q from 2^-8 to just under 2^12 with 64 linear steps per octave. */
+double or_q_of_k(int32_t k)
+{
+    return (double)(64 + (k & 63)) * ldexp(1.0, (k >> 6) - 14);
+}
+
+/* Largest admissible k for a row length: |v| stays below 2^21 so that every coordinate
+ * is exact in fp32 and its token input stays below 2^22. */
+int32_t or_k_max(int64_t cols)
+{
+    double lim = ldexp(1.0, 20) / (sqrt((double)cols) + 1.0);
+    int32_t k = NQ - 1;
+    while (k > 0 && or_q_of_k(k) > lim)
+        k--;
+    return k;
+}
+
+/* ---------------------------------- lattice quantizer -------------------------------- */
+/* Nearest point of D8 = {r in Z^8 : sum r even} (Conway & Sloane): round every
+ * coordinate to the nearest integer (ties to even); if the sum is odd, move the
+ * coordinate with the largest rounding error (lowest index on ties) to its other
+ * neighbouring integer (upwards when that coordinate was already an integer). */
+void or_d8_nearest(const double *y, double *r)
+{
+    long long sum = 0;
+    for (int i = 0; i < 8; i++) {
+        r[i] = nearbyint(y[i]);
+        sum += (long long)r[i];
+    }
+    if (sum % 2 != 0) {
+        int j = 0;
+        double worst = -1.0;
+        for (int i = 0; i < 8; i++) {
+            double d = fabs(y[i] - r[i]);
+            if (d > worst) {
+                worst = d;
+                j = i;
+            }
+        }
+        if (y[j] < r[j])
+            r[j] -= 1.0;
+        else
+            r[j] += 1.0;
+    }
+}
+
+/* Nearest point of E8 = D8 u (D8 + 1/2): decode x in D8 and x - 1/2 in D8 (+1/2),
+ * keep the closer (squared errors summed in coordinate order; a tie keeps the integer
+ * coset).  Returns v = 2z so that both cosets are integers: all v_i even (integer
+ * coset) or all odd, and sum v = 0 mod 4. */
+void or_e8_nearest(const double *x, int32_t *v)
+{
+    double ya[8], yb[8], ra[8], rb[8], da = 0.0, db = 0.0;
+    for (int i = 0; i < 8; i++) {
+        ya[i] = x[i];
+        yb[i] = x[i] - 0.5;
+    }
+    or_d8_nearest(ya, ra);
+    or_d8_nearest(yb, rb);
+    for (int i = 0; i < 8; i++) {
+        double e = ya[i] - ra[i];
+        da += e * e;
+    }
+    for (int i = 0; i < 8; i++) {
+        double e = yb[i] - rb[i];
+        db += e * e;
+    }
+    if (db < da)
+        for (int i = 0; i < 8; i++)
+            v[i] = 2 * (int32_t)rb[i] + 1;
+    else
+        for (int i = 0; i < 8; i++)
+            v[i] = 2 * (int32_t)ra[i];
+}
+
+void or_e8_nearest_batch(const double *x, int64_t nblocks, int32_t *v)
+{
+    for (int64_t b = 0; b < nblocks; b++)
+        or_e8_nearest(x + 8 * b, v + 8 * b);
+}
+
+/* ---------------------------------- symbols ------------------------------------------ */
+uint32_t or_zigzag(int32_t y) { return y >= 0 ? 2u * (uint32_t)y : 2u * (uint32_t)(-(int64_t)y) - 1u; }
+
+int32_t or_unzigzag(uint32_t u) { return (u & 1u) ? -(int32_t)((u + 1u) / 2u) : (int32_t)(u / 2u); }
+
+/* Conditional model (reading of [ABS] "conditional probability model of lattice
+ * coordinates"): the coordinates of one block are coded in order 0..7.
+ *   coordinate 0: context 0, symbol zigzag(v0); its parity is the coset c.
+ *   coordinates 1..6: context 1 + c, symbol zigzag(y_i) with y_i = (v_i - c) / 2.
+ *   coordinate 7: context 3 + 2c + p, p = (y_0 + ... + y_6) mod 2.  E8 forces
+ *     y_7 = p (mod 2), so the symbol is zigzag((y_7 - p) / 2). */
+static void block_symbols(const int32_t *v, uint32_t *ctx, uint32_t *u)
+{
+    int32_t c = (v[0] % 2 != 0) ? 1 : 0;
+    int32_t y[8], p = 0;
+    for (int i = 0; i < 8; i++)
+        y[i] = (v[i] - c) / 2; /* exact: v_i - c is even */
+    for (int i = 0; i < 7; i++)
+        p ^= (y[i] % 2 != 0) ? 1 : 0;
+    ctx[0] = 0;
+    u[0] = or_zigzag(v[0]);
+    for (int i = 1; i < 7; i++) {
+        ctx[i] = 1u + (uint32_t)c;
+        u[i] = or_zigzag(y[i]);
+    }
+    ctx[7] = 3u + 2u * (uint32_t)c + (uint32_t)p;
+    u[7] = or_zigzag((y[7] - p) / 2);
+}
+
+/* Token binarization ("hybrid integer"): with split m and h = min(m, 2), a value
+ * u < 2^m is its own token; otherwise, with n = floor(log2 u), the token carries n and
+ * the h bits below the leading one, and the remaining n - h low bits travel as raw
+ * extra bits. */
+void or_tokenize(uint32_t u, int32_t m, uint32_t *tok, uint32_t *nbits, uint32_t *extra)
+{
+    uint32_t h = (uint32_t)(m < 2 ? m : 2);
+    if (u < (1u << m)) {
+        *tok = u;
+        *nbits = 0;
+        *extra = 0;
+        return;
+    }
+    uint32_t n = 0;
+    while ((u >> (n + 1)) != 0)
+        n++;
+    uint32_t top = (u >> (n - h)) & ((1u << h) - 1u);
+    *tok = (1u << m) + ((n - (uint32_t)m) << h) + top;
+    *nbits = n - h;
+    *extra = u & ((1u << (n - h)) - 1u);
+}
+
+uint32_t or_detokenize(uint32_t tok, int32_t m, uint32_t extra)
+{
+    uint32_t h = (uint32_t)(m < 2 ? m : 2);
+    if (tok < (1u << m))
+        return tok;
+    uint32_t d = tok - (1u << m);
+    uint32_t n = (uint32_t)m + (d >> h);
+    uint32_t top = (1u << h) | (d & ((1u << h) - 1u));
+    return (top << (n - h)) | extra;
+}
+
+void or_detokenize_batch(const uint32_t *tok, int64_t n, int32_t m, const uint32_t *extra, uint32_t *u)
+{
+    for (int64_t i = 0; i < n; i++)
+        u[i] = or_detokenize(tok[i], m, extra[i]);
+}
+
+static void token_bits(uint32_t tok, int32_t m, uint32_t *nbits)
+{
+    uint32_t h = (uint32_t)(m < 2 ? m : 2);
+    if (tok < (1u << m)) {
+        *nbits = 0;
+        return;
+    }
+    uint32_t n = (uint32_t)m + ((tok - (1u << m)) >> h);
+    *nbits = n - h;
+}
+
+/* number of tokens a split can produce for values below 2^22 */
+static uint32_t max_tokens(int32_t m)
+{
+    uint32_t h = (uint32_t)(m < 2 ? m : 2);
+    return (1u << m) + ((22u - (uint32_t)m) << h);
+}
+
+void or_tokenize_batch(const uint32_t *u, int64_t n, int32_t m, uint32_t *tok, uint32_t *nbits, uint32_t *extra)
+{
+    for (int64_t i = 0; i < n; i++)
+        or_tokenize(u[i], m, tok + i, nbits + i, extra + i);
+}
+
+/* split: smallest m in [0, 7] with at least 99% of the context's values below 2^m */
+static int32_t choose_split(const uint64_t *bitlen_hist /* [24]: count by bit length */)
+{
+    uint64_t n = 0;
+    for (int i = 0; i < 24; i++)
+        n += bitlen_hist[i];
+    if (n == 0)
+        return 0;
+    uint64_t below = 0;
+    for (int32_t m = 0; m <= MAX_SPLIT; m++) {
+        below += bitlen_hist[m]; /* values with bit length m are below 2^m */
+        if (below * 100u >= n * 99u)
+            return m;
+    }
+    return MAX_SPLIT;
+}
+
+static int bit_length(uint32_t u)
+{
+    int n = 0;
+    while (u) {
+        n++;
+        u >>= 1;
+    }
+    return n;
+}
+
+/* ---------------------------------- frequency tables --------------------------------- */
+/* Counts -> frequencies summing to M = 2^11 by largest remainders: f_i = floor(c_i M / n);
+ * the M - sum f_i leftover units go one each to the largest remainders (c_i M mod n),
+ * lower index first on ties; then every seen token left at 0 is raised to 1 by taking a
+ * unit from the currently largest frequency (lower index first on ties).  A context
+ * with one token gets f = M.  Returns the table length (last seen token + 1). */
+int32_t or_normalize_freqs(const uint64_t *counts, int32_t n, uint32_t *f)
+{
+    uint64_t total = 0;
+    int32_t len = 0;
+    for (int32_t i = 0; i < n; i++) {
+        total += counts[i];
+        if (counts[i])
+            len = i + 1;
+        f[i] = 0;
+    }
+    if (total == 0)
+        return 0;
+    uint64_t *rem = (uint64_t *)calloc((size_t)n, sizeof(uint64_t));
+    uint32_t sum = 0;
+    for (int32_t i = 0; i < n; i++) {
+        if (!counts[i])
+            continue;
+        /* c * M < 2^64 for any realistic count (c < 2^53) */
+        f[i] = (uint32_t)((counts[i] * PROB_M) / total);
+        rem[i] = (counts[i] * PROB_M) % total;
+        sum += f[i];
+    }
+    uint32_t left = PROB_M - sum;
+    unsigned char *given = (unsigned char *)calloc((size_t)n, 1);
+    for (uint32_t r = 0; r < left; r++) {
+        int32_t best = -1;
+        for (int32_t i = 0; i < n; i++)
+            if (counts[i] && !given[i] && (best < 0 || rem[i] > rem[best]))
+                best = i;
+        given[best] = 1;
+        f[best] += 1;
+    }
+    for (int32_t i = 0; i < n; i++) {
+        if (counts[i] && f[i] == 0) {
+            int32_t big = 0;
+            for (int32_t j = 1; j < n; j++)
+                if (f[j] > f[big])
+                    big = j;
+            f[big] -= 1;
+            f[i] = 1;
+        }
+    }
+    free(rem);
+    free(given);
+    return len;
+}
+
+/* ---------------------------------- tiles -------------------------------------------- */
+/* Reading of "independently decodable tiles" ([ABS]): a tile is 32 lanes x K blocks;
+ * lane l of tile t owns blocks t*32K + 32k + l, k = 0..K-1.  K is set by the block count
+ * alone: K = 16 below 2^20 blocks, else the power of two at or below nb / 2^16, capped
+ * at 256, which keeps the tile count near 2048 for mid-sized matrices. */
+uint32_t or_choose_blocks_per_lane(int64_t nb)
+{
+    int64_t q = nb / 65536;
+    if (q < 16)
+        return 16;
+    uint32_t k = 16;
+    while ((int64_t)k * 2 <= q && k < 256)
+        k *= 2;
+    return k;
+}
+
+/* ---------------------------------- value preparation -------------------------------- */
+static int is_code_container(int32_t c) { return c == ORD_INT8 || c == ORD_FP8E4M3; }
+
+/* Per-row absmax INT8 / FP8 codes ([LIN], "lossy compression to the quantized weights";
+ * readings: INT8 uses the symmetric range [-127, 127]; an all-zero row gets scale 1). */
+int or_prequant(const void *src, int32_t sdt, int64_t rows, int64_t cols, int32_t container, double *codes,
+                float *scales)
+{
+    for (int64_t r = 0; r < rows; r++) {
+        double amax = 0.0;
+        for (int64_t j = 0; j < cols; j++) {
+            double a = fabs(src_value(src, sdt, r * cols + j));
+            if (a > amax)
+                amax = a;
+        }
+        float s = 1.0f;
+        if (amax > 0.0)
+            s = (float)(amax / (container == ORD_INT8 ? 127.0 : 448.0));
+        if (s == 0.0f) /* amax so small that the scale underflows */
+            s = FLT_MIN;
+        scales[r] = s;
+        for (int64_t j = 0; j < cols; j++) {
+            double w = src_value(src, sdt, r * cols + j);
+            double c;
+            if (amax == 0.0)
+                c = 0.0;
+            else if (container == ORD_INT8) {
+                c = nearbyint(w / (double)s);
+                if (c > 127.0)
+                    c = 127.0;
+                if (c < -127.0)
+                    c = -127.0;
+            } else {
+                float t = (float)(w / (double)s);
+                c = e4m3_value(or_e4m3_from_float(t));
+            }
+            codes[r * cols + j] = c;
+        }
+    }
+    return OR_OK;
+}
+
+/* values the lattice stage sees: the source itself, or the INT8/FP8 codes */
+static double *lattice_input(const void *src, int32_t sdt, int64_t rows, int64_t cols, int32_t container,
+                             float *scales_out)
+{
+    double *w = (double *)malloc((size_t)(rows * cols) * sizeof(double));
+    if (!w)
+        return NULL;
+    if (is_code_container(container)) {
+        float *sc = scales_out ? scales_out : (float *)malloc((size_t)rows * sizeof(float));
+        or_prequant(src, sdt, rows, cols, container, w, sc);
+        if (!scales_out)
+            free(sc);
+    } else {
+        for (int64_t i = 0; i < rows * cols; i++)
+            w[i] = src_value(src, sdt, i);
+    }
+    return w;
+}
+
+/* "Row-normalized" (reading): each row is divided by its RMS s_r; the resolution q then
+ * scales it, so the lattice input is x = w / (2 f_r) with f_r = s_r / (2q) rounded to
+ * fp32 -- the same fp32 factor the decoder multiplies by.  s_r is the fp32 rounding of
+ * sqrt(sum_j w_j^2 / C) with the sum taken left to right in double.  A row whose s_r is
+ * 0 has f_r = 0 and all-zero lattice points; a factor that overflows fp32 is clamped to
+ * FLT_MAX. */
+static void row_rms(const double *w, int64_t rows, int64_t cols, float *s)
+{
+    for (int64_t r = 0; r < rows; r++) {
+        double acc = 0.0;
+        for (int64_t j = 0; j < cols; j++) {
+            double a = w[r * cols + j];
+            acc += a * a;
+        }
+        s[r] = (float)sqrt(acc / (double)cols);
+    }
+}
+
+static float row_factor(float s, int32_t k)
+{
+    if (s == 0.0f)
+        return 0.0f;
+    float f = (float)((double)s / (2.0 * or_q_of_k(k)));
+    if (isinf(f))
+        f = FLT_MAX;
+    return f;
+}
+
+static void quantize_block(const double *w, float f, int32_t *v)
+{
+    if (f == 0.0f) {
+        for (int i = 0; i < 8; i++)
+            v[i] = 0;
+        return;
+    }
+    double x[8];
+    for (int i = 0; i < 8; i++)
+        x[i] = w[i] / (2.0 * (double)f);
+    or_e8_nearest(x, v);
+}
+
+void or_row_factors(const void *src, int32_t sdt, int64_t rows, int64_t cols, int32_t container, int32_t k,
+                    float *s_out, float *f_out)
+{
+    double *w = lattice_input(src, sdt, rows, cols, container, NULL);
+    row_rms(w, rows, cols, s_out);
+    for (int64_t r = 0; r < rows; r++)
+        f_out[r] = row_factor(s_out[r], k);
+    free(w);
+}
+
+int or_quantize(const void *src, int32_t sdt, int64_t rows, int64_t cols, int32_t container, int32_t k,
+                int32_t *v)
+{
+    double *w = lattice_input(src, sdt, rows, cols, container, NULL);
+    float *s = (float *)malloc((size_t)rows * sizeof(float));
+    row_rms(w, rows, cols, s);
+    int64_t cb = cols / 8;
+    for (int64_t b = 0; b < rows * cb; b++)
+        quantize_block(w + 8 * b, row_factor(s[b / cb], k), v + 8 * b);
+    free(s);
+    free(w);
+    return OR_OK;
+}
+
+/* ---------------------------------- storage estimate --------------------------------- */
+static size_t meta_bytes(int64_t rows, int32_t container, uint64_t total_tokens, uint32_t ntiles)
+{
+    size_t m = HEADER_BYTES + al16((size_t)rows * 4);
+    if (is_code_container(container))
+        m += al16((size_t)rows * 4);
+    m += al16((size_t)total_tokens * 2);
+    m += al16((size_t)(ntiles + 1) * 4);
+    return m;
+}
+
+/* Sampled storage estimate ([ABS]: "sampled storage estimates select the quantization
+ * resolution without repeated full-stream encoding").  Every S-th block (S = ceil(nb /
+ * 65536)) is quantized at k; its symbols are tokenized with splits chosen on the sample,
+ * and the payload is estimated as the sample's empirical conditional entropy of tokens
+ * plus its raw extra bits, scaled by nb / n_sample.  Exact metadata is added, the table
+ * length taken from the sample, plus 104 bytes per tile: a final state holds about 24 bits
+ * that carry no payload (32 lanes x 3 bytes) and a tile pads to 16 bytes (8 on average). */
+static double estimate_bpp(const double *w, const float *s, int64_t rows, int64_t cols, int32_t container,
+                           int32_t k, uint32_t K)
+{
+    int64_t cb = cols / 8, nb = rows * cb;
+    int64_t S = (nb + SAMPLE_TARGET - 1) / SAMPLE_TARGET;
+    if (S < 1)
+        S = 1;
+    int64_t ns = (nb + S - 1) / S;
+    uint32_t *ctx = (uint32_t *)malloc((size_t)ns * 8 * sizeof(uint32_t));
+    uint32_t *u = (uint32_t *)malloc((size_t)ns * 8 * sizeof(uint32_t));
+    uint64_t hist[NCTX][24];
+    memset(hist, 0, sizeof hist);
+    for (int64_t j = 0; j < ns; j++) {
+        int64_t b = j * S;
+        int32_t v[8];
+        quantize_block(w + 8 * b, row_factor(s[b / cb], k), v);
+        block_symbols(v, ctx + 8 * j, u + 8 * j);
+        for (int i = 0; i < 8; i++)
+            hist[ctx[8 * j + i]][bit_length(u[8 * j + i])]++;
+    }
+    int32_t m[NCTX];
+    uint64_t *cnt[NCTX];
+    for (int c = 0; c < NCTX; c++) {
+        m[c] = choose_split(hist[c]);
+        cnt[c] = (uint64_t *)calloc(max_tokens(m[c]), sizeof(uint64_t));
+    }
+    double extra = 0.0;
+    for (int64_t i = 0; i < ns * 8; i++) {
+        uint32_t t, nbits, ex;
+        or_tokenize(u[i], m[ctx[i]], &t, &nbits, &ex);
+        cnt[ctx[i]][t]++;
+        extra += (double)nbits;
+    }
+    double bits = 0.0;
+    uint64_t total_tokens = 0;
+    for (int c = 0; c < NCTX; c++) {
+        uint64_t n = 0;
+        uint32_t len = 0;
+        for (uint32_t t = 0; t < max_tokens(m[c]); t++) {
+            n += cnt[c][t];
+            if (cnt[c][t])
+                len = t + 1;
+        }
+        total_tokens += len;
+        if (n == 0)
+            continue;
+        bits += (double)n * log2((double)n);
+        for (uint32_t t = 0; t < max_tokens(m[c]); t++)
+            if (cnt[c][t])
+                bits -= (double)cnt[c][t] * log2((double)cnt[c][t]);
+    }
+    bits += extra;
+    uint32_t ntiles = (uint32_t)((nb + (int64_t)LANES * K - 1) / ((int64_t)LANES * K));
+    double bytes = (double)meta_bytes(rows, container, total_tokens, ntiles) + 104.0 * (double)ntiles +
+                   bits * ((double)nb / (double)ns) / 8.0;
+    for (int c = 0; c < NCTX; c++)
+        free(cnt[c]);
+    free(ctx);
+    free(u);
+    return 8.0 * bytes / (double)(rows * cols);
+}
+
+double or_estimate_bpp(const void *src, int32_t sdt, int64_t rows, int64_t cols, int32_t container, int32_t k,
+                       uint32_t K)
+{
+    double *w = lattice_input(src, sdt, rows, cols, container, NULL);
+    float *s = (float *)malloc((size_t)rows * sizeof(float));
+    row_rms(w, rows, cols, s);
+    if (K == 0)
+        K = or_choose_blocks_per_lane(rows * (cols / 8));
+    double e = estimate_bpp(w, s, rows, cols, container, k, K);
+    free(s);
+    free(w);
+    return e;
+}
+
+/* ---------------------------------- byte helpers ------------------------------------- */
+static void put16(uint8_t *p, uint32_t v)
+{
+    p[0] = (uint8_t)v;
+    p[1] = (uint8_t)(v >> 8);
+}
+static void put32(uint8_t *p, uint32_t v)
+{
+    for (int i = 0; i < 4; i++)
+        p[i] = (uint8_t)(v >> (8 * i));
+}
+static void put64(uint8_t *p, uint64_t v)
+{
+    for (int i = 0; i < 8; i++)
+        p[i] = (uint8_t)(v >> (8 * i));
+}
+static uint32_t get16(const uint8_t *p) { return (uint32_t)p[0] | ((uint32_t)p[1] << 8); }
+static uint32_t get32(const uint8_t *p)
+{
+    return (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) | ((uint32_t)p[3] << 24);
+}
+static uint64_t get64(const uint8_t *p) { return (uint64_t)get32(p) | ((uint64_t)get32(p + 4) << 32); }
+
+/* ---------------------------------- tile encoder ------------------------------------- */
+typedef struct {
+    uint8_t lane;
+    uint16_t f, cum;
+} event;
+
+typedef struct {
+    uint8_t *p;
+    size_t n, cap;
+} bytes;
+
+static void bytes_put(bytes *b, const void *src, size_t n)
+{
+    if (b->n + n > b->cap) {
+        size_t c = b->cap ? b->cap : 1024;
+        while (c < b->n + n)
+            c *= 2;
+        b->p = (uint8_t *)realloc(b->p, c);
+        b->cap = c;
+    }
+    memcpy(b->p + b->n, src, n);
+    b->n += n;
+}
+
+/* Decode order inside a tile (the interleaving rule both sides follow): for k = 0..K-1,
+ * for coordinate i = 0..7: one step in which every lane that owns block t*32K + 32k + l
+ * decodes the token of coordinate i; then, for j = 0, 1, ..., one step in which every
+ * lane whose token left more than j chunks of extra bits decodes chunk j (chunks of at
+ * most 11 bits, least significant first, each a uniform symbol).  After each step the
+ * lanes that fell below L read one 16-bit word each, lower lanes first.
+ * The encoder runs these events in reverse, emitting words in reverse; the tile stores
+ * the final encoder states (= initial decoder states) and the words in decode order. */
+static void encode_tile(const uint32_t *ctx, const uint32_t *u, int64_t nb, int64_t t, uint32_t K,
+                        const int32_t *m, uint32_t *const *freq, uint32_t *const *cum, bytes *out)
+{
+    int64_t base = t * (int64_t)LANES * K;
+    size_t cap = (size_t)LANES * K * 8 * 3, ne = 0;
+    event *ev = (event *)malloc(cap * sizeof(event));
+    for (uint32_t k = 0; k < K; k++) {
+        int64_t b0 = base + (int64_t)k * LANES;
+        if (b0 >= nb)
+            break;
+        for (int i = 0; i < 8; i++) {
+            uint32_t nbits[LANES], extra[LANES];
+            for (int l = 0; l < LANES; l++) {
+                nbits[l] = 0;
+                int64_t b = b0 + l;
+                if (b >= nb)
+                    continue;
+                uint32_t c = ctx[8 * b + i], tok;
+                or_tokenize(u[8 * b + i], m[c], &tok, &nbits[l], &extra[l]);
+                ev[ne].lane = (uint8_t)l;
+                ev[ne].f = (uint16_t)freq[c][tok];
+                ev[ne].cum = (uint16_t)cum[c][tok];
+                ne++;
+            }
+            for (uint32_t j = 0;; j++) {
+                int any = 0;
+                for (int l = 0; l < LANES; l++) {
+                    if (nbits[l] <= CHUNK_BITS * j)
+                        continue;
+                    uint32_t left = nbits[l] - CHUNK_BITS * j;
+                    uint32_t bits = left < CHUNK_BITS ? left : CHUNK_BITS;
+                    uint32_t val = (extra[l] >> (CHUNK_BITS * j)) & ((1u << bits) - 1u);
+                    ev[ne].lane = (uint8_t)l;
+                    ev[ne].f = (uint16_t)(1u << (PROB_BITS - bits));
+                    ev[ne].cum = (uint16_t)(val << (PROB_BITS - bits));
+                    ne++;
+                    any = 1;
+                }
+                if (!any)
+                    break;
+            }
+        }
+    }
+    uint32_t x[LANES];
+    for (int l = 0; l < LANES; l++)
+        x[l] = STATE_L;
+    uint16_t *words = (uint16_t *)malloc((ne + 1) * sizeof(uint16_t));
+    size_t nw = 0;
+    for (size_t e = ne; e-- > 0;) {
+        uint32_t l = ev[e].lane, f = ev[e].f;
+        uint32_t s = x[l];
+        /* renormalise so that the encoded state stays below 2^32: x_max = (L >> 11) << 16 * f */
+        if ((uint64_t)s >= ((uint64_t)f << 21)) {
+            words[nw++] = (uint16_t)(s & 0xffffu);
+            s >>= 16;
+        }
+        x[l] = ((s / f) << PROB_BITS) + (s % f) + ev[e].cum;
+    }
+    uint8_t st[LANES * 4];
+    for (int l = 0; l < LANES; l++)
+        put32(st + 4 * l, x[l]);
+    bytes_put(out, st, sizeof st);
+    for (size_t i = 0; i < nw; i++) {
+        uint8_t w2[2];
+        put16(w2, words[nw - 1 - i]);
+        bytes_put(out, w2, 2);
+    }
+    static const uint8_t zeros[16] = {0};
+    size_t pad = al16(out->n) - out->n;
+    bytes_put(out, zeros, pad);
+    free(words);
+    free(ev);
+}
+
+/* ---------------------------------- full encode at one k ----------------------------- */
+static int encode_at(const double *w, const float *s, const float *scales, int64_t rows, int64_t cols,
+                     int32_t sdt, int32_t container, int32_t k, uint32_t K, uint8_t *out, size_t cap,
+                     size_t *out_n)
+{
+    int64_t cb = cols / 8, nb = rows * cb;
+    uint32_t *ctx = (uint32_t *)malloc((size_t)nb * 8 * sizeof(uint32_t));
+    uint32_t *u = (uint32_t *)malloc((size_t)nb * 8 * sizeof(uint32_t));
+    float *f = (float *)malloc((size_t)rows * sizeof(float));
+    if (!ctx || !u || !f)
+        return OR_ERR_INVALID_ARG;
+    for (int64_t r = 0; r < rows; r++)
+        f[r] = row_factor(s[r], k);
+    uint64_t hist[NCTX][24];
+    memset(hist, 0, sizeof hist);
+    for (int64_t b = 0; b < nb; b++) {
+        int32_t v[8];
+        quantize_block(w + 8 * b, f[b / cb], v);
+        block_symbols(v, ctx + 8 * b, u + 8 * b);
+        for (int i = 0; i < 8; i++)
+            hist[ctx[8 * b + i]][bit_length(u[8 * b + i])]++;
+    }
+    int32_t m[NCTX];
+    uint32_t *freq[NCTX], *cum[NCTX];
+    uint64_t *cnt[NCTX];
+    uint32_t ntok[NCTX];
+    uint64_t total_tokens = 0;
+    for (int c = 0; c < NCTX; c++) {
+        m[c] = choose_split(hist[c]);
+        cnt[c] = (uint64_t *)calloc(max_tokens(m[c]), sizeof(uint64_t));
+        freq[c] = (uint32_t *)calloc(max_tokens(m[c]), sizeof(uint32_t));
+        cum[c] = (uint32_t *)calloc(max_tokens(m[c]), sizeof(uint32_t));
+    }
+    for (int64_t i = 0; i < nb * 8; i++) {
+        uint32_t t, nbits, ex;
+        or_tokenize(u[i], m[ctx[i]], &t, &nbits, &ex);
+        cnt[ctx[i]][t]++;
+    }
+    for (int c = 0; c < NCTX; c++) {
+        ntok[c] = (uint32_t)or_normalize_freqs(cnt[c], (int32_t)max_tokens(m[c]), freq[c]);
+        uint32_t a = 0;
+        for (uint32_t t = 0; t < max_tokens(m[c]); t++) {
+            cum[c][t] = a;
+            a += freq[c][t];
+        }
+        total_tokens += ntok[c];
+    }
+    uint32_t T = (uint32_t)((nb + (int64_t)LANES * K - 1) / ((int64_t)LANES * K));
+    bytes tiles = {0, 0, 0};
+    uint32_t *dir = (uint32_t *)malloc(((size_t)T + 1) * sizeof(uint32_t));
+    for (uint32_t t = 0; t < T; t++) {
+        dir[t] = (uint32_t)(tiles.n / 16);
+        encode_tile(ctx, u, nb, t, K, m, freq, cum, &tiles);
+    }
+    dir[T] = (uint32_t)(tiles.n / 16);
+
+    size_t off_rowf = HEADER_BYTES;
+    size_t off_scales = off_rowf + al16((size_t)rows * 4);
+    size_t off_freq = off_scales + (is_code_container(container) ? al16((size_t)rows * 4) : 0);
+    size_t off_dir = off_freq + al16((size_t)total_tokens * 2);
+    size_t off_tiles = off_dir + al16(((size_t)T + 1) * 4);
+    size_t total = off_tiles + tiles.n;
+    int rc = OR_OK;
+    *out_n = total;
+    if (total > cap || !out) {
+        rc = OR_ERR_BUFFER_TOO_SMALL;
+    } else {
+        memset(out, 0, total);
+        put32(out, MAGIC);
+        put16(out + 4, VERSION);
+        out[6] = (uint8_t)sdt;
+        out[7] = (uint8_t)container;
+        put64(out + 8, (uint64_t)rows);
+        put64(out + 16, (uint64_t)cols);
+        put32(out + 24, T);
+        put32(out + 28, K);
+        put16(out + 32, (uint32_t)k);
+        out[34] = PROB_BITS;
+        out[35] = NCTX;
+        for (int c = 0; c < NCTX; c++) {
+            out[36 + c] = (uint8_t)m[c];
+            put16(out + 44 + 2 * c, ntok[c]);
+        }
+        for (int64_t r = 0; r < rows; r++) {
+            uint32_t b;
+            memcpy(&b, &f[r], 4);
+            put32(out + off_rowf + 4 * r, b);
+        }
+        if (is_code_container(container))
+            for (int64_t r = 0; r < rows; r++) {
+                uint32_t b;
+                memcpy(&b, &scales[r], 4);
+                put32(out + off_scales + 4 * r, b);
+            }
+        size_t p = off_freq;
+        for (int c = 0; c < NCTX; c++)
+            for (uint32_t t = 0; t < ntok[c]; t++, p += 2)
+                put16(out + p, freq[c][t]);
+        for (uint32_t t = 0; t <= T; t++)
+            put32(out + off_dir + 4 * t, dir[t]);
+        memcpy(out + off_tiles, tiles.p, tiles.n);
+    }
+    for (int c = 0; c < NCTX; c++) {
+        free(cnt[c]);
+        free(freq[c]);
+        free(cum[c]);
+    }
+    free(tiles.p);
+    free(dir);
+    free(f);
+    free(u);
+    free(ctx);
+    return rc;
+}
+
+/* ---------------------------------- compress ----------------------------------------- */
+int or_compress(const void *src, int32_t sdt, int64_t rows, int64_t cols, double target, int32_t container,
+                uint32_t K, int32_t q_override, uint8_t *out, size_t cap, size_t *out_n)
+{
+    if (!src || !out_n || rows <= 0 || cols <= 0)
+        return OR_ERR_INVALID_ARG;
+    if (sdt != ORD_BF16 && sdt != ORD_FP16 && sdt != ORD_FP32)
+        return OR_ERR_UNSUPPORTED;
+    if (container == 0)
+        container = sdt;
+    if (container < ORD_BF16 || container > ORD_FP8E4M3)
+        return OR_ERR_INVALID_ARG;
+    if (cols % 8 != 0)
+        return OR_ERR_UNSUPPORTED;
+    if (K > 4096)
+        return OR_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < rows * cols; i++)
+        if (!isfinite(src_value(src, sdt, i)))
+            return OR_ERR_NONFINITE;
+    if (!(target >= 0.001) || !(target <= 11.0) || (is_code_container(container) && !(target < 8.0)))
+        return OR_ERR_TARGET_RANGE;
+    float *scales = (float *)malloc((size_t)rows * sizeof(float));
+    double *w = lattice_input(src, sdt, rows, cols, container, scales);
+    float *s = (float *)malloc((size_t)rows * sizeof(float));
+    row_rms(w, rows, cols, s);
+    int64_t nb = rows * (cols / 8);
+    if (K == 0)
+        K = or_choose_blocks_per_lane(nb);
+    int32_t kmax = or_k_max(cols);
+    int32_t k;
+    if (q_override >= 0) {
+        k = q_override > kmax ? kmax : q_override;
+    } else {
+        double budget = 0.995 * target;
+        int32_t lo = 0, hi = kmax;
+        while (lo < hi) {
+            int32_t mid = lo + (hi - lo + 1) / 2;
+            if (estimate_bpp(w, s, rows, cols, container, mid, K) <= budget)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        k = lo;
+    }
+    int rc;
+    for (;;) {
+        size_t n = 0;
+        rc = encode_at(w, s, scales, rows, cols, sdt, container, k, K, NULL, 0, &n);
+        if (q_override >= 0 || 8.0 * (double)n <= target * (double)(rows * cols)) {
+            rc = encode_at(w, s, scales, rows, cols, sdt, container, k, K, out, cap, out_n);
+            break;
+        }
+        if (k == 0) {
+            *out_n = n;
+            rc = OR_ERR_TARGET_UNREACHABLE;
+            break;
+        }
+        k--;
+    }
+    free(s);
+    free(w);
+    free(scales);
+    return rc;
+}
+
+/* ---------------------------------- parse -------------------------------------------- */
+int or_parse(const uint8_t *p, size_t n, or_info *info)
+{
+    if (!p || !info || n < HEADER_BYTES)
+        return OR_ERR_CORRUPT;
+    if (get32(p) != MAGIC || get16(p + 4) != VERSION || p[34] != PROB_BITS || p[35] != NCTX)
+        return OR_ERR_CORRUPT;
+    memset(info, 0, sizeof *info);
+    info->src_dtype = p[6];
+    info->container_dtype = p[7];
+    info->rows = (int64_t)get64(p + 8);
+    info->cols = (int64_t)get64(p + 16);
+    info->n_tiles = get32(p + 24);
+    info->blocks_per_lane = get32(p + 28);
+    info->q_index = (int32_t)get16(p + 32);
+    if (info->src_dtype < ORD_BF16 || info->src_dtype > ORD_FP32 || info->container_dtype < ORD_BF16 ||
+        info->container_dtype > ORD_FP8E4M3)
+        return OR_ERR_CORRUPT;
+    if (info->rows <= 0 || info->cols <= 0 || info->cols % 8 != 0 || info->rows > ((int64_t)1 << 40) ||
+        info->cols > ((int64_t)1 << 40) || info->blocks_per_lane == 0 || info->blocks_per_lane > 4096)
+        return OR_ERR_CORRUPT;
+    int64_t nb = info->rows * (info->cols / 8);
+    int64_t T = (nb + (int64_t)LANES * info->blocks_per_lane - 1) / ((int64_t)LANES * info->blocks_per_lane);
+    if (T != (int64_t)info->n_tiles)
+        return OR_ERR_CORRUPT;
+    uint64_t total_tokens = 0;
+    for (int c = 0; c < NCTX; c++) {
+        info->split[c] = p[36 + c];
+        info->ntok[c] = (uint16_t)get16(p + 44 + 2 * c);
+        if (info->split[c] > MAX_SPLIT || info->ntok[c] > max_tokens(info->split[c]))
+            return OR_ERR_CORRUPT;
+        total_tokens += info->ntok[c];
+    }
+    info->off_rowf = HEADER_BYTES;
+    info->off_scales = info->off_rowf + al16((size_t)info->rows * 4);
+    info->off_freq = info->off_scales + (is_code_container(info->container_dtype) ? al16((size_t)info->rows * 4) : 0);
+    info->off_dir = info->off_freq + al16((size_t)total_tokens * 2);
+    info->off_tiles = info->off_dir + al16(((size_t)T + 1) * 4);
+    if (info->off_tiles > n)
+        return OR_ERR_CORRUPT;
+    /* tables sum to M */
+    size_t q = info->off_freq;
+    for (int c = 0; c < NCTX; c++) {
+        uint32_t sum = 0;
+        for (uint32_t t = 0; t < info->ntok[c]; t++, q += 2)
+            sum += get16(p + q);
+        if (info->ntok[c] && sum != PROB_M)
+            return OR_ERR_CORRUPT;
+    }
+    /* directory: starts at 0, each tile holds at least its states, ends at the blob end */
+    const uint8_t *d = p + info->off_dir;
+    if (get32(d) != 0)
+        return OR_ERR_CORRUPT;
+    for (int64_t t = 0; t < T; t++)
+        if (get32(d + 4 * (t + 1)) < get32(d + 4 * t) + 8)
+            return OR_ERR_CORRUPT;
+    if (info->off_tiles + 16 * (uint64_t)get32(d + 4 * T) != n)
+        return OR_ERR_CORRUPT;
+    info->storage_nbytes = n;
+    info->header_nbytes = HEADER_BYTES;
+    info->actual_bpp = 8.0 * (double)n / (double)(info->rows * info->cols);
+    return OR_OK;
+}
+
+/* ---------------------------------- decode ------------------------------------------- */
+typedef struct {
+    or_info in;
+    const uint8_t *p;
+    uint16_t *slot_tok[NCTX]; /* slot -> token (0xffff: slot outside the table) */
+    uint32_t *freq[NCTX], *cum[NCTX];
+    const uint8_t *rowf;
+} dec_ctx;
+
+static int dec_open(dec_ctx *D, const uint8_t *p, size_t n)
+{
+    int rc = or_parse(p, n, &D->in);
+    if (rc)
+        return rc;
+    D->p = p;
+    D->rowf = p + D->in.off_rowf;
+    size_t q = D->in.off_freq;
+    for (int c = 0; c < NCTX; c++) {
+        uint32_t nt = D->in.ntok[c];
+        D->slot_tok[c] = (uint16_t *)malloc(PROB_M * sizeof(uint16_t));
+        D->freq[c] = (uint32_t *)calloc(nt + 1, sizeof(uint32_t));
+        D->cum[c] = (uint32_t *)calloc(nt + 1, sizeof(uint32_t));
+        for (uint32_t s = 0; s < PROB_M; s++)
+            D->slot_tok[c][s] = 0xffff;
+        uint32_t a = 0;
+        for (uint32_t t = 0; t < nt; t++, q += 2) {
+            D->freq[c][t] = get16(p + q);
+            D->cum[c][t] = a;
+            for (uint32_t s = a; s < a + D->freq[c][t]; s++)
+                D->slot_tok[c][s] = (uint16_t)t;
+            a += D->freq[c][t];
+        }
+    }
+    return OR_OK;
+}
+
+static void dec_close(dec_ctx *D)
+{
+    for (int c = 0; c < NCTX; c++) {
+        free(D->slot_tok[c]);
+        free(D->freq[c]);
+        free(D->cum[c]);
+    }
+}
+
+/* one lane's rANS step for a table symbol; returns the token */
+static uint32_t dec_token(dec_ctx *D, uint32_t c, uint32_t *x, uint32_t *status, double *ideal)
+{
+    uint32_t slot = *x & (PROB_M - 1);
+    uint32_t t = D->slot_tok[c][slot];
+    if (t == 0xffff) {
+        *status |= OR_DEC_BAD_TOKEN;
+        return 0;
+    }
+    uint32_t f = D->freq[c][t];
+    *x = f * (*x >> PROB_BITS) + slot - D->cum[c][t];
+    if (ideal)
+        *ideal += -log2((double)f / (double)PROB_M);
+    return t;
+}
+
+typedef struct {
+    uint64_t *tokcount[NCTX];
+    double ideal, extra;
+    uint64_t nsym;
+} code_stats;
+
+static void decode_tile(dec_ctx *D, int64_t t, int32_t *vout, void *out, uint32_t *status, code_stats *cs)
+{
+    const or_info *I = &D->in;
+    int64_t cb = I->cols / 8, nb = I->rows * cb;
+    uint32_t K = I->blocks_per_lane;
+    const uint8_t *dir = D->p + I->off_dir;
+    const uint8_t *tp = D->p + I->off_tiles + 16 * (uint64_t)get32(dir + 4 * t);
+    uint64_t tile_bytes = 16 * (uint64_t)(get32(dir + 4 * (t + 1)) - get32(dir + 4 * t));
+    uint64_t nwords = (tile_bytes - 4 * LANES) / 2, pos = 0;
+    const uint8_t *wp = tp + 4 * LANES;
+    uint32_t x[LANES];
+    for (int l = 0; l < LANES; l++)
+        x[l] = get32(tp + 4 * l);
+    int64_t base = t * (int64_t)LANES * K;
+    int esz = elt_size(I->container_dtype);
+    for (uint32_t k = 0; k < K; k++) {
+        int64_t b0 = base + (int64_t)k * LANES;
+        if (b0 >= nb)
+            break;
+        int32_t v[LANES][8], y[LANES][8], c[LANES], p[LANES];
+        for (int i = 0; i < 8; i++) {
+            uint32_t tok[LANES], nbits[LANES], extra[LANES], ctx[LANES];
+            /* token step */
+            for (int l = 0; l < LANES; l++) {
+                nbits[l] = 0;
+                extra[l] = 0;
+                if (b0 + l >= nb)
+                    continue;
+                ctx[l] = i == 0 ? 0u : i < 7 ? 1u + (uint32_t)c[l] : 3u + 2u * (uint32_t)c[l] + (uint32_t)p[l];
+                tok[l] = dec_token(D, ctx[l], &x[l], status, cs ? &cs->ideal : NULL);
+                token_bits(tok[l], I->split[ctx[l]], &nbits[l]);
+                if (cs) {
+                    cs->tokcount[ctx[l]][tok[l]]++;
+                    cs->extra += nbits[l];
+                    cs->nsym++;
+                }
+                if (x[l] < STATE_L) {
+                    uint32_t wd = 0;
+                    if (pos < nwords)
+                        wd = get16(wp + 2 * pos);
+                    else
+                        *status |= OR_DEC_WORD_OVERRUN;
+                    pos++;
+                    x[l] = (x[l] << 16) | wd;
+                }
+            }
+            /* chunk steps */
+            for (uint32_t j = 0;; j++) {
+                int any = 0;
+                for (int l = 0; l < LANES; l++) {
+                    if (nbits[l] <= CHUNK_BITS * j)
+                        continue;
+                    any = 1;
+                    uint32_t left = nbits[l] - CHUNK_BITS * j;
+                    uint32_t bits = left < CHUNK_BITS ? left : CHUNK_BITS;
+                    uint32_t f = 1u << (PROB_BITS - bits);
+                    uint32_t slot = x[l] & (PROB_M - 1);
+                    uint32_t val = slot >> (PROB_BITS - bits);
+                    x[l] = f * (x[l] >> PROB_BITS) + slot - val * f;
+                    extra[l] |= val << (CHUNK_BITS * j);
+                    if (x[l] < STATE_L) {
+                        uint32_t wd = 0;
+                        if (pos < nwords)
+                            wd = get16(wp + 2 * pos);
+                        else
+                            *status |= OR_DEC_WORD_OVERRUN;
+                        pos++;
+                        x[l] = (x[l] << 16) | wd;
+                    }
+                }
+                if (!any)
+                    break;
+            }
+            /* inverse symbolization */
+            for (int l = 0; l < LANES; l++) {
+                if (b0 + l >= nb)
+                    continue;
+                uint32_t uu = or_detokenize(tok[l], I->split[ctx[l]], extra[l]);
+                if (tok[l] >= I->ntok[ctx[l]])
+                    *status |= OR_DEC_BAD_TOKEN;
+                if (i == 0) {
+                    v[l][0] = or_unzigzag(uu);
+                    c[l] = (v[l][0] % 2 != 0) ? 1 : 0;
+                    y[l][0] = (v[l][0] - c[l]) / 2;
+                    p[l] = (y[l][0] % 2 != 0) ? 1 : 0;
+                } else if (i < 7) {
+                    y[l][i] = or_unzigzag(uu);
+                    v[l][i] = 2 * y[l][i] + c[l];
+                    p[l] ^= (y[l][i] % 2 != 0) ? 1 : 0;
+                } else {
+                    y[l][7] = 2 * or_unzigzag(uu) + p[l];
+                    v[l][7] = 2 * y[l][7] + c[l];
+                }
+            }
+        }
+        /* reconstruction: w = f_r * v in fp32, then the container conversion */
+        for (int l = 0; l < LANES; l++) {
+            int64_t b = b0 + l;
+            if (b >= nb)
+                continue;
+            int64_t r = b / cb;
+            uint32_t fb = get32(D->rowf + 4 * r);
+            float fr;
+            memcpy(&fr, &fb, 4);
+            if (vout)
+                memcpy(vout + 8 * b, v[l], 8 * sizeof(int32_t));
+            if (out) {
+                float wv[8];
+                for (int i = 0; i < 8; i++)
+                    wv[i] = fr * (float)v[l][i];
+                or_convert_batch(wv, 8, I->container_dtype, (uint8_t *)out + (size_t)(8 * b) * (size_t)esz);
+            }
+        }
+    }
+    for (int l = 0; l < LANES; l++)
+        if (x[l] != STATE_L)
+            *status |= OR_DEC_BAD_END;
+    if (pos > nwords || nwords - pos >= 8)
+        *status |= OR_DEC_WORD_COUNT;
+}
+
+int or_decode(const uint8_t *blob, size_t n, uint32_t t0, uint32_t t1, int32_t *v, void *out,
+              uint32_t *status)
+{
+    dec_ctx D;
+    uint32_t st = 0;
+    int rc = dec_open(&D, blob, n);
+    if (rc)
+        return rc;
+    if (t1 > D.in.n_tiles)
+        t1 = D.in.n_tiles;
+    for (uint32_t t = t0; t < t1; t++)
+        decode_tile(&D, t, v, out, &st, NULL);
+    dec_close(&D);
+    if (status)
+        *status |= st;
+    return OR_OK;
+}
+
+int or_code_stats(const uint8_t *blob, size_t n, double *ideal_bits, double *emp_entropy_bits, double *extra_bits,
+                  uint64_t *n_symbols, uint64_t *payload_bytes)
+{
+    dec_ctx D;
+    uint32_t st = 0;
+    int rc = dec_open(&D, blob, n);
+    if (rc)
+        return rc;
+    code_stats cs;
+    memset(&cs, 0, sizeof cs);
+    for (int c = 0; c < NCTX; c++)
+        cs.tokcount[c] = (uint64_t *)calloc(D.in.ntok[c] + 1, sizeof(uint64_t));
+    for (uint32_t t = 0; t < D.in.n_tiles; t++)
+        decode_tile(&D, t, NULL, NULL, &st, &cs);
+    double H = 0.0;
+    for (int c = 0; c < NCTX; c++) {
+        uint64_t tot = 0;
+        for (uint32_t t = 0; t < D.in.ntok[c]; t++)
+            tot += cs.tokcount[c][t];
+        for (uint32_t t = 0; t < D.in.ntok[c]; t++)
+            if (cs.tokcount[c][t])
+                H += (double)cs.tokcount[c][t] * log2((double)tot / (double)cs.tokcount[c][t]);
+        free(cs.tokcount[c]);
+    }
+    const uint8_t *dir = blob + D.in.off_dir;
+    uint64_t pb = 0;
+    for (uint32_t t = 0; t < D.in.n_tiles; t++)
+        pb += 16 * (uint64_t)(get32(dir + 4 * (t + 1)) - get32(dir + 4 * t)) - 4 * LANES;
+    *ideal_bits = cs.ideal;
+    *emp_entropy_bits = H;
+    *extra_bits = cs.extra;
+    *n_symbols = cs.nsym;
+    *payload_bytes = pb;
+    dec_close(&D);
+    return st ? OR_ERR_CORRUPT : OR_OK;
+}

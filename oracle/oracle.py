@@ -1,0 +1,257 @@
+"""ctypes binding of the C oracle (oracle/ep_oracle.c) -- test infrastructure only.
+
+Argument marshalling between numpy arrays and the C functions; no arithmetic of the
+method lives here.  Only tests/, __graft_entry__.smoke() and bench.py's CPU-baseline
+leg may import this module.
+"""
+import ctypes as C
+
+import numpy as np
+
+from . import build as _build
+
+BF16, FP16, FP32, INT8, FP8E4M3 = 1, 2, 3, 4, 5
+OK, ERR_INVALID_ARG, ERR_NONFINITE, ERR_TARGET_RANGE, ERR_TARGET_UNREACHABLE = 0, -1, -2, -3, -4
+ERR_BUFFER_TOO_SMALL, ERR_CORRUPT, ERR_UNSUPPORTED = -5, -6, -8
+ELT = {BF16: 2, FP16: 2, FP32: 4, INT8: 1, FP8E4M3: 1}
+NP_DTYPE = {BF16: np.uint16, FP16: np.uint16, FP32: np.float32, INT8: np.int8, FP8E4M3: np.uint8}
+
+
+class Info(C.Structure):
+    _fields_ = [
+        ("rows", C.c_int64), ("cols", C.c_int64),
+        ("src_dtype", C.c_int32), ("container_dtype", C.c_int32),
+        ("storage_nbytes", C.c_uint64), ("header_nbytes", C.c_uint64),
+        ("actual_bpp", C.c_double), ("q_index", C.c_int32),
+        ("n_tiles", C.c_uint32), ("blocks_per_lane", C.c_uint32),
+        ("split", C.c_uint8 * 7), ("ntok", C.c_uint16 * 7),
+        ("off_rowf", C.c_uint64), ("off_scales", C.c_uint64), ("off_freq", C.c_uint64),
+        ("off_dir", C.c_uint64), ("off_tiles", C.c_uint64),
+    ]
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = C.CDLL(_build.build())
+        p = C.c_void_p
+        L.or_q_of_k.restype = C.c_double
+        L.or_q_of_k.argtypes = [C.c_int32]
+        L.or_k_max.restype = C.c_int32
+        L.or_k_max.argtypes = [C.c_int64]
+        L.or_d8_nearest.argtypes = [p, p]
+        L.or_e8_nearest.argtypes = [p, p]
+        L.or_e8_nearest_batch.argtypes = [p, C.c_int64, p]
+        L.or_zigzag.restype = C.c_uint32
+        L.or_zigzag.argtypes = [C.c_int32]
+        L.or_unzigzag.restype = C.c_int32
+        L.or_unzigzag.argtypes = [C.c_uint32]
+        L.or_tokenize_batch.argtypes = [p, C.c_int64, C.c_int32, p, p, p]
+        L.or_detokenize.restype = C.c_uint32
+        L.or_detokenize.argtypes = [C.c_uint32, C.c_int32, C.c_uint32]
+        L.or_detokenize_batch.argtypes = [p, C.c_int64, C.c_int32, p, p]
+        L.or_normalize_freqs.restype = C.c_int32
+        L.or_normalize_freqs.argtypes = [p, C.c_int32, p]
+        L.or_choose_blocks_per_lane.restype = C.c_uint32
+        L.or_choose_blocks_per_lane.argtypes = [C.c_int64]
+        L.or_convert_batch.argtypes = [p, C.c_int64, C.c_int32, p]
+        L.or_prequant.restype = C.c_int
+        L.or_prequant.argtypes = [p, C.c_int32, C.c_int64, C.c_int64, C.c_int32, p, p]
+        L.or_row_factors.argtypes = [p, C.c_int32, C.c_int64, C.c_int64, C.c_int32, C.c_int32, p, p]
+        L.or_quantize.restype = C.c_int
+        L.or_quantize.argtypes = [p, C.c_int32, C.c_int64, C.c_int64, C.c_int32, C.c_int32, p]
+        L.or_estimate_bpp.restype = C.c_double
+        L.or_estimate_bpp.argtypes = [p, C.c_int32, C.c_int64, C.c_int64, C.c_int32, C.c_int32, C.c_uint32]
+        L.or_compress.restype = C.c_int
+        L.or_compress.argtypes = [p, C.c_int32, C.c_int64, C.c_int64, C.c_double, C.c_int32, C.c_uint32,
+                                  C.c_int32, p, C.c_size_t, C.POINTER(C.c_size_t)]
+        L.or_parse.restype = C.c_int
+        L.or_parse.argtypes = [p, C.c_size_t, C.POINTER(Info)]
+        L.or_decode.restype = C.c_int
+        L.or_decode.argtypes = [p, C.c_size_t, C.c_uint32, C.c_uint32, p, p, C.POINTER(C.c_uint32)]
+        L.or_code_stats.restype = C.c_int
+        L.or_code_stats.argtypes = [p, C.c_size_t, C.POINTER(C.c_double), C.POINTER(C.c_double),
+                                    C.POINTER(C.c_double), C.POINTER(C.c_uint64), C.POINTER(C.c_uint64)]
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return a.ctypes.data_as(C.c_void_p)
+
+
+def _src(src):
+    """(pointer-able contiguous array, dtype code) for a numpy array or a CPU torch tensor."""
+    try:
+        import torch
+        if isinstance(src, torch.Tensor):
+            if src.dtype == torch.bfloat16:
+                return src.contiguous().view(torch.int16).numpy().view(np.uint16), BF16
+            if src.dtype == torch.float16:
+                return src.contiguous().view(torch.int16).numpy().view(np.uint16), FP16
+            if src.dtype == torch.float32:
+                return src.contiguous().numpy(), FP32
+            raise TypeError(f"unsupported dtype {src.dtype}")
+    except ImportError:
+        pass
+    a = np.ascontiguousarray(src)
+    if a.dtype == np.float32:
+        return a, FP32
+    raise TypeError("pass a torch tensor (bf16/fp16/fp32) or a float32 array")
+
+
+# ---- scalar pieces ----
+def q_of_k(k):
+    return lib().or_q_of_k(int(k))
+
+
+def k_max(cols):
+    return lib().or_k_max(int(cols))
+
+
+def d8_nearest(y):
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    r = np.zeros(8, np.float64)
+    lib().or_d8_nearest(_ptr(y), _ptr(r))
+    return r
+
+
+def e8_nearest(x):
+    """Lattice points v = 2z for blocks x of shape (..., 8)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    shp = x.shape
+    x2 = x.reshape(-1, 8)
+    v = np.zeros(x2.shape, np.int32)
+    lib().or_e8_nearest_batch(_ptr(x2), x2.shape[0], _ptr(v))
+    return v.reshape(shp)
+
+
+def zigzag(y):
+    return lib().or_zigzag(int(y))
+
+
+def unzigzag(u):
+    return lib().or_unzigzag(int(u))
+
+
+def tokenize(u, m):
+    u = np.ascontiguousarray(u, dtype=np.uint32)
+    tok = np.zeros_like(u)
+    nb = np.zeros_like(u)
+    ex = np.zeros_like(u)
+    lib().or_tokenize_batch(_ptr(u), u.size, int(m), _ptr(tok), _ptr(nb), _ptr(ex))
+    return tok, nb, ex
+
+
+def detokenize(tok, m, extra):
+    return lib().or_detokenize(int(tok), int(m), int(extra))
+
+
+def detokenize_batch(tok, m, extra):
+    tok = np.ascontiguousarray(tok, dtype=np.uint32)
+    extra = np.ascontiguousarray(extra, dtype=np.uint32)
+    u = np.zeros_like(tok)
+    lib().or_detokenize_batch(_ptr(tok), tok.size, int(m), _ptr(extra), _ptr(u))
+    return u
+
+
+def normalize_freqs(counts):
+    c = np.ascontiguousarray(counts, dtype=np.uint64)
+    f = np.zeros(c.size, np.uint32)
+    n = lib().or_normalize_freqs(_ptr(c), c.size, _ptr(f))
+    return f, n
+
+
+def blocks_per_lane(nblocks):
+    return lib().or_choose_blocks_per_lane(int(nblocks))
+
+
+def convert(w, dtype):
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    out = np.zeros(w.shape, NP_DTYPE[dtype])
+    lib().or_convert_batch(_ptr(w), w.size, dtype, _ptr(out))
+    return out
+
+
+def prequant(src, container):
+    a, dt = _src(src)
+    R, Cc = a.shape
+    codes = np.zeros((R, Cc), np.float64)
+    scales = np.zeros(R, np.float32)
+    lib().or_prequant(_ptr(a), dt, R, Cc, container, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def row_factors(src, k, container=0):
+    a, dt = _src(src)
+    R, Cc = a.shape
+    s = np.zeros(R, np.float32)
+    f = np.zeros(R, np.float32)
+    lib().or_row_factors(_ptr(a), dt, R, Cc, container or dt, int(k), _ptr(s), _ptr(f))
+    return s, f
+
+
+def quantize(src, k, container=0):
+    a, dt = _src(src)
+    R, Cc = a.shape
+    v = np.zeros((R, Cc), np.int32)
+    lib().or_quantize(_ptr(a), dt, R, Cc, container or dt, int(k), _ptr(v))
+    return v
+
+
+def estimate_bpp(src, k, container=0, blocks_per_lane=0):
+    a, dt = _src(src)
+    R, Cc = a.shape
+    return lib().or_estimate_bpp(_ptr(a), dt, R, Cc, container or dt, int(k), blocks_per_lane)
+
+
+# ---- the stream ----
+def compress(src, target_bpp, container=0, blocks_per_lane=0, q_override=-1):
+    """Returns (rc, blob as a uint8 numpy array)."""
+    a, dt = _src(src)
+    R, Cc = a.shape
+    n = C.c_size_t(0)
+    rc = lib().or_compress(_ptr(a), dt, R, Cc, float(target_bpp), container, blocks_per_lane, q_override,
+                           None, 0, C.byref(n))
+    if rc not in (OK, ERR_BUFFER_TOO_SMALL):
+        return rc, None
+    out = np.zeros(n.value, np.uint8)
+    rc = lib().or_compress(_ptr(a), dt, R, Cc, float(target_bpp), container, blocks_per_lane, q_override,
+                           _ptr(out), out.size, C.byref(n))
+    return rc, (out[: n.value] if rc == OK else None)
+
+
+def parse(blob):
+    blob = np.ascontiguousarray(blob, dtype=np.uint8)
+    info = Info()
+    rc = lib().or_parse(_ptr(blob), blob.size, C.byref(info))
+    return rc, info
+
+
+def decode(blob, t0=0, t1=None, want_v=True, want_out=True):
+    """Returns (rc, status, v (rows, cols) int32 or None, out (rows, cols) container array or None)."""
+    blob = np.ascontiguousarray(blob, dtype=np.uint8)
+    rc, info = parse(blob)
+    if rc != OK:
+        return rc, 0, None, None
+    R, Cc = info.rows, info.cols
+    v = np.zeros((R, Cc), np.int32) if want_v else None
+    out = np.zeros((R, Cc), NP_DTYPE[info.container_dtype]) if want_out else None
+    st = C.c_uint32(0)
+    t1 = info.n_tiles if t1 is None else t1
+    rc = lib().or_decode(_ptr(blob), blob.size, t0, t1, _ptr(v) if v is not None else None,
+                         _ptr(out) if out is not None else None, C.byref(st))
+    return rc, st.value, v, out
+
+
+def code_stats(blob):
+    blob = np.ascontiguousarray(blob, dtype=np.uint8)
+    ideal, H, extra = C.c_double(), C.c_double(), C.c_double()
+    ns, pb = C.c_uint64(), C.c_uint64()
+    rc = lib().or_code_stats(_ptr(blob), blob.size, C.byref(ideal), C.byref(H), C.byref(extra),
+                             C.byref(ns), C.byref(pb))
+    return rc, dict(ideal_bits=ideal.value, entropy_bits=H.value, extra_bits=extra.value,
+                    n_symbols=ns.value, payload_bytes=pb.value)
