@@ -1,0 +1,159 @@
+"""Thin ctypes binding of libeptile.so (include/eptile.h): argument marshalling only.
+
+Every step of compression runs in the library's C++ and every step of decompression in
+its sm_100a kernel; this module passes torch tensors' pointers, sizes and streams.
+There is no fallback: a missing library or a missing GPU raises ``EpError``.
+"""
+import ctypes as C
+import os
+import re
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libeptile.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "eptile.h")
+
+BF16, FP16, FP32, INT8, FP8E4M3, LATTICE_I32 = 1, 2, 3, 4, 5, 6
+TORCH_DTYPE = {BF16: torch.bfloat16, FP16: torch.float16, FP32: torch.float32, INT8: torch.int8,
+               FP8E4M3: torch.float8_e4m3fn}
+CODE_OF = {v: k for k, v in TORCH_DTYPE.items()}
+NAMES = {"bf16": BF16, "fp16": FP16, "fp32": FP32, "int8": INT8, "fp8_e4m3": FP8E4M3}
+
+
+class EpError(RuntimeError):
+    def __init__(self, status, what=""):
+        self.status = status
+        msg = lib().ep_status_string(status).decode() if _lib is not None else str(status)
+        super().__init__(f"{what}: {msg} ({status})" if what else f"{msg} ({status})")
+
+
+class Config(C.Structure):
+    _fields_ = [("target_bpp", C.c_double), ("container_dtype", C.c_int32), ("blocks_per_lane", C.c_uint32),
+                ("q_index", C.c_int32), ("n_threads", C.c_int32)]
+
+
+class StreamInfo(C.Structure):
+    _fields_ = [
+        ("rows", C.c_int64), ("cols", C.c_int64),
+        ("src_dtype", C.c_int32), ("container_dtype", C.c_int32),
+        ("storage_nbytes", C.c_uint64), ("header_nbytes", C.c_uint64),
+        ("actual_bpp", C.c_double), ("q_index", C.c_int32),
+        ("n_tiles", C.c_uint32), ("blocks_per_lane", C.c_uint32),
+        ("split", C.c_uint8 * 8), ("ntok", C.c_uint16 * 8),
+        ("off_rowf", C.c_uint64), ("off_scales", C.c_uint64), ("off_freq", C.c_uint64),
+        ("off_dir", C.c_uint64), ("off_tiles", C.c_uint64), ("out_nbytes", C.c_uint64),
+    ]
+
+    @property
+    def shape(self):
+        return (self.rows, self.cols)
+
+    @property
+    def dtype(self):
+        return TORCH_DTYPE[self.container_dtype]
+
+    def storage_nbytes_(self, include_header=True):
+        return self.storage_nbytes - (0 if include_header else self.header_nbytes)
+
+
+_lib = None
+
+
+def declared_functions():
+    """names of the functions include/eptile.h declares"""
+    text = open(HEADER).read()
+    return re.findall(r"^(?:int|size_t|const char \*)\s*\*?\s*(ep_\w+)\(", text, flags=re.M)
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m dit_weight_compression_tile_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        p = C.c_void_p
+        L.ep_compress_bound.restype = C.c_size_t
+        L.ep_compress_bound.argtypes = [C.c_int64, C.c_int64, C.POINTER(Config)]
+        L.ep_compress_host.restype = C.c_int
+        L.ep_compress_host.argtypes = [p, C.c_int32, C.c_int64, C.c_int64, C.POINTER(Config), p, C.c_size_t,
+                                       C.POINTER(C.c_size_t)]
+        L.ep_stream_info.restype = C.c_int
+        L.ep_stream_info.argtypes = [p, C.c_size_t, C.POINTER(StreamInfo)]
+        L.ep_decompress.restype = C.c_int
+        L.ep_decompress.argtypes = [C.POINTER(StreamInfo), p, p, C.c_int32, p, p]
+        L.ep_status_string.restype = C.c_char_p
+        L.ep_status_string.argtypes = [C.c_int]
+        _lib = L
+    return _lib
+
+
+def _config(target_bpp, container=0, blocks_per_lane=0, q_index=-1, n_threads=0):
+    if isinstance(container, str):
+        container = NAMES[container]
+    if isinstance(container, torch.dtype):
+        container = CODE_OF[container]
+    return Config(float(target_bpp), int(container or 0), int(blocks_per_lane), int(q_index), int(n_threads))
+
+
+def compress(tensor, target_bpp, container=0, blocks_per_lane=0, q_index=-1, n_threads=0):
+    """compress(tensor, config) on the host: returns the stream as a CPU uint8 tensor.
+
+    ``tensor``: 2-D BF16/FP16/FP32 (moved to the CPU if needed).  ``container``: 0 (same as
+    the source), a dtype code / name / torch dtype; INT8 and FP8 store per-row absmax codes."""
+    if tensor.dim() != 2 or tensor.numel() == 0:
+        raise EpError(-1, "compress needs a non-empty 2-D tensor")
+    src = tensor.detach().to("cpu").contiguous()
+    if src.dtype not in (torch.bfloat16, torch.float16, torch.float32):
+        raise EpError(-8, f"source dtype {src.dtype}")
+    cfg = _config(target_bpp, container, blocks_per_lane, q_index, n_threads)
+    L = lib()
+    cap = L.ep_compress_bound(src.shape[0], src.shape[1], C.byref(cfg))
+    out = torch.empty(max(cap, 64), dtype=torch.uint8)
+    n = C.c_size_t(0)
+    rc = L.ep_compress_host(src.data_ptr(), CODE_OF[src.dtype], src.shape[0], src.shape[1], C.byref(cfg),
+                            out.data_ptr(), out.numel(), C.byref(n))
+    if rc == -5:  # the bound is a guarantee; this is a second chance, not the normal path
+        out = torch.empty(n.value, dtype=torch.uint8)
+        rc = L.ep_compress_host(src.data_ptr(), CODE_OF[src.dtype], src.shape[0], src.shape[1], C.byref(cfg),
+                                out.data_ptr(), out.numel(), C.byref(n))
+    if rc != 0:
+        raise EpError(rc, "ep_compress_host")
+    return out[: n.value].clone()
+
+
+def stream_info(blob):
+    """CompressedTensor properties from a host copy of the stream (CPU uint8 tensor)."""
+    b = blob.detach().to("cpu").contiguous()
+    info = StreamInfo()
+    rc = lib().ep_stream_info(b.data_ptr(), b.numel(), C.byref(info))
+    if rc != 0:
+        raise EpError(rc, "ep_stream_info")
+    return info
+
+
+def decompress(d_blob, info=None, out=None, status=None, stream=None, lattice=False):
+    """decompress(compressed): the fused GPU decode of a device-resident stream.
+
+    ``d_blob``: CUDA uint8 tensor holding the whole stream.  ``info``: from ``stream_info``
+    (parsed from ``d_blob`` through a host copy when omitted).  ``out``: optional CUDA tensor
+    of ``info.shape`` / ``info.dtype``.  ``status``: optional CUDA int32 tensor of one element
+    into which damage flags are ORed.  Launches on ``stream`` (default: the current stream).
+    ``lattice=True`` returns the decoded lattice points v = 2z (int32) instead of weights."""
+    if not d_blob.is_cuda:
+        raise EpError(-1, "decompress needs the stream in device memory")
+    if info is None:
+        info = stream_info(d_blob.cpu())
+    want = torch.int32 if lattice else info.dtype
+    if out is None:
+        out = torch.empty(info.shape, dtype=want, device=d_blob.device)
+    if not out.is_cuda or out.dtype != want or tuple(out.shape) != info.shape or not out.is_contiguous():
+        raise EpError(-1, "output tensor does not match the stream")
+    st = status.data_ptr() if status is not None else None
+    s = (stream or torch.cuda.current_stream(d_blob.device)).cuda_stream
+    dt = LATTICE_I32 if lattice else info.container_dtype
+    rc = lib().ep_decompress(C.byref(info), d_blob.data_ptr(), out.data_ptr(), dt, st, s)
+    if rc != 0:
+        raise EpError(rc, "ep_decompress")
+    return out

@@ -1,0 +1,60 @@
+// Stream format v1 constants and small helpers shared by the library's host encoder, the
+// stream parser and the decode kernel.  The byte layout is fixed by the library (the pages
+// give none): a 64-byte header, per-row factors, optional per-row code scales, per-context
+// frequency tables, a tile directory and the tiles.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+namespace ep {
+
+constexpr uint32_t kMagic = 0x31545045u;  // "EPT1"
+constexpr uint32_t kVersion = 1;
+constexpr uint32_t kProbBits = 11;         // frequency precision: tables sum to 2^11
+constexpr uint32_t kProbScale = 1u << kProbBits;
+constexpr uint32_t kStateLow = 1u << 16;   // rANS state interval [2^16, 2^32), 16-bit words
+constexpr int kLanes = 32;                 // interleaved states per tile = warp lanes
+constexpr int kContexts = 7;
+constexpr int kMaxSplit = 7;
+constexpr uint32_t kChunkBits = 11;        // extra bits travel in uniform chunks of <= 11 bits
+constexpr size_t kHeaderBytes = 64;
+constexpr int kNumQ = 1280;                // resolution indices
+constexpr int64_t kSampleBlocks = 65536;   // blocks sampled by the storage estimate
+constexpr double kTileOverheadBytes = 104.0;  // per tile in the estimate
+constexpr double kTargetMargin = 0.995;
+
+inline size_t align16(size_t n) { return (n + 15) & ~size_t(15); }
+
+inline uint32_t split_h(uint32_t m) { return m < 2 ? m : 2; }
+
+// tokens a split can produce for values below 2^22
+inline uint32_t split_alphabet(uint32_t m) { return (1u << m) + ((22u - m) << split_h(m)); }
+
+inline int elt_bytes(int dt) { return dt == 3 ? 4 : (dt == 1 || dt == 2) ? 2 : 1; }
+
+inline bool is_code_container(int dt) { return dt == 4 || dt == 5; }
+
+struct Layout {
+    size_t rowf, scales, freq, dir, tiles;
+};
+
+inline Layout layout_for(int64_t rows, int container, uint64_t total_tokens, uint64_t ntiles) {
+    Layout L;
+    L.rowf = kHeaderBytes;
+    L.scales = L.rowf + align16(size_t(rows) * 4);
+    L.freq = L.scales + (is_code_container(container) ? align16(size_t(rows) * 4) : 0);
+    L.dir = L.freq + align16(size_t(total_tokens) * 2);
+    L.tiles = L.dir + align16(size_t(ntiles + 1) * 4);
+    return L;
+}
+
+// K (blocks per lane) from the block count: 16 below 2^20 blocks, else the power of two at
+// or below nb / 2^16, at most 256.
+inline uint32_t auto_blocks_per_lane(int64_t nb) {
+    int64_t target = nb >> 16;
+    uint32_t k = 16;
+    while (k < 256 && int64_t(k) * 2 <= target) k <<= 1;
+    return k;
+}
+
+}  // namespace ep

@@ -1,0 +1,639 @@
+// Host compressor: ep_compress_host / ep_compress_bound.
+//
+// compress(tensor, config) of the "EntroPack API reference", following the pipeline of the
+// "EntroPack: Fast and Accurate Entropy-Coded Weight Compression at Arbitrary Bitrates"
+// Abstract: row-normalized E8 lattice quantization, a conditional model of the lattice
+// coordinates, a resolution picked by sampled storage estimates (no repeated full-stream
+// encoding in the normal case), and entropy coding in independently decodable tiles.
+// Multithreaded over rows, blocks and tiles; the output bytes do not depend on the thread
+// count (every floating-point reduction keeps a fixed order).
+#include <algorithm>
+#include <cfloat>
+#include <cmath>
+#include <cstring>
+#include <functional>
+#include <thread>
+#include <vector>
+
+#include "../../include/eptile.h"
+#include "format.h"
+
+namespace ep {
+namespace {
+
+// ------------------------------------------------------------------ threading
+void parallel_for(int64_t n, int threads, const std::function<void(int64_t, int64_t)> &fn) {
+    if (n <= 0) return;
+    int64_t nt = std::max<int64_t>(1, std::min<int64_t>(threads, (n + 1023) / 1024));
+    if (nt == 1) {
+        fn(0, n);
+        return;
+    }
+    std::vector<std::thread> pool;
+    int64_t chunk = (n + nt - 1) / nt;
+    for (int64_t t = 0; t < nt; ++t) {
+        int64_t b = t * chunk, e = std::min(n, b + chunk);
+        if (b < e) pool.emplace_back(fn, b, e);
+    }
+    for (auto &th : pool) th.join();
+}
+
+// ------------------------------------------------------------------ source values
+// fp16 -> float through a table built from the bit fields (exact)
+const float *half_table() {
+    static std::vector<float> tab = [] {
+        std::vector<float> t(65536);
+        for (uint32_t h = 0; h < 65536; ++h) {
+            uint32_t sign = (h & 0x8000u) << 16, exp = (h >> 10) & 31, man = h & 1023;
+            float v;
+            if (exp == 0) {
+                v = std::ldexp(float(man), -24);
+            } else if (exp == 31) {
+                v = man ? NAN : INFINITY;
+            } else {
+                v = std::ldexp(float(man | 1024u), int(exp) - 25);
+            }
+            uint32_t b;
+            std::memcpy(&b, &v, 4);
+            b |= sign;
+            std::memcpy(&v, &b, 4);
+            t[h] = v;
+        }
+        return t;
+    }();
+    return tab.data();
+}
+
+struct Source {
+    const void *p;
+    int dt;
+    float at(int64_t i) const {
+        if (dt == EP_BF16) {
+            uint32_t b = uint32_t(static_cast<const uint16_t *>(p)[i]) << 16;
+            float f;
+            std::memcpy(&f, &b, 4);
+            return f;
+        }
+        if (dt == EP_FP16) return half_table()[static_cast<const uint16_t *>(p)[i]];
+        return static_cast<const float *>(p)[i];
+    }
+};
+
+// ------------------------------------------------------------------ FP8 E4M3 codes
+// The 127 non-negative finite E4M3 values in increasing order (code = index).
+const std::vector<double> &e4m3_values() {
+    static std::vector<double> vals = [] {
+        std::vector<double> v;
+        for (int code = 0; code <= 0x7e; ++code) {
+            int e = code >> 3, m = code & 7;
+            v.push_back(e == 0 ? m / 512.0 : std::ldexp(1.0 + m / 8.0, e - 7));
+        }
+        return v;
+    }();
+    return vals;
+}
+
+// round |t| to the E4M3 grid, nearest with ties to the even code, saturating at 448
+double e4m3_round(float t) {
+    const auto &vals = e4m3_values();
+    double a = std::fabs(double(t));
+    double r;
+    if (a >= vals.back()) {
+        r = vals.back();
+    } else {
+        size_t hi = size_t(std::upper_bound(vals.begin(), vals.end(), a) - vals.begin());  // vals[hi] > a
+        size_t lo = hi - 1;                                                                  // vals[lo] <= a
+        double dlo = a - vals[lo], dhi = vals[hi] - a;
+        if (dlo < dhi)
+            r = vals[lo];
+        else if (dhi < dlo)
+            r = vals[hi];
+        else
+            r = (lo % 2 == 0) ? vals[lo] : vals[hi];
+    }
+    return std::signbit(t) ? -r : r;
+}
+
+// ------------------------------------------------------------------ quantizer
+double q_value(int k) { return std::ldexp(double(64 + (k % 64)), k / 64 - 14); }
+
+int max_q_index(int64_t cols) {
+    double lim = std::ldexp(1.0, 20) / (std::sqrt(double(cols)) + 1.0);
+    int k = kNumQ - 1;
+    while (k > 0 && q_value(k) > lim) --k;
+    return k;
+}
+
+float factor_of(float rms, int k) {
+    if (rms == 0.0f) return 0.0f;
+    float f = float(double(rms) / (2.0 * q_value(k)));
+    return std::isinf(f) ? FLT_MAX : f;
+}
+
+// nearest point of D8 (Conway & Sloane): round, then repair an odd coordinate sum at the
+// coordinate with the largest rounding error
+inline void nearest_d8(const double *y, double *r) {
+    long long s = 0;
+    for (int i = 0; i < 8; ++i) {
+        r[i] = std::nearbyint(y[i]);
+        s += static_cast<long long>(r[i]);
+    }
+    if (s & 1) {
+        int worst = 0;
+        double werr = std::fabs(y[0] - r[0]);
+        for (int i = 1; i < 8; ++i) {
+            double e = std::fabs(y[i] - r[i]);
+            if (e > werr) {
+                werr = e;
+                worst = i;
+            }
+        }
+        r[worst] += (y[worst] < r[worst]) ? -1.0 : 1.0;
+    }
+}
+
+// v = 2 * nearest point of E8 = D8 u (D8 + 1/2); ties keep the integer coset
+inline void quantize_e8(const double *x, int32_t *v) {
+    double a[8], b[8], ra[8], rb[8];
+    for (int i = 0; i < 8; ++i) {
+        a[i] = x[i];
+        b[i] = x[i] - 0.5;
+    }
+    nearest_d8(a, ra);
+    nearest_d8(b, rb);
+    double da = 0.0, db = 0.0;
+    for (int i = 0; i < 8; ++i) da += (a[i] - ra[i]) * (a[i] - ra[i]);
+    for (int i = 0; i < 8; ++i) db += (b[i] - rb[i]) * (b[i] - rb[i]);
+    if (db < da) {
+        for (int i = 0; i < 8; ++i) v[i] = int32_t(rb[i]) * 2 + 1;
+    } else {
+        for (int i = 0; i < 8; ++i) v[i] = int32_t(ra[i]) * 2;
+    }
+}
+
+// ------------------------------------------------------------------ symbols
+inline uint32_t zz(int32_t y) { return y < 0 ? uint32_t(-int64_t(y)) * 2u - 1u : uint32_t(y) * 2u; }
+
+inline int bitlen(uint32_t u) { return u ? 32 - __builtin_clz(u) : 0; }
+
+// contexts and values of one block: 0 for coordinate 0 (zz v0), 1 + c for coordinates 1..6
+// (zz y_i), 3 + 2c + p for coordinate 7 (zz of (y7 - p) / 2)
+inline void symbols_of(const int32_t *v, uint8_t *ctx, uint32_t *u) {
+    int32_t c = v[0] & 1;
+    int32_t par = 0;
+    ctx[0] = 0;
+    u[0] = zz(v[0]);
+    par ^= ((v[0] - c) >> 1) & 1;
+    for (int i = 1; i < 7; ++i) {
+        int32_t y = (v[i] - c) >> 1;
+        par ^= y & 1;
+        ctx[i] = uint8_t(1 + c);
+        u[i] = zz(y);
+    }
+    int32_t y7 = (v[7] - c) >> 1;
+    ctx[7] = uint8_t(3 + 2 * c + par);
+    u[7] = zz((y7 - par) >> 1);
+}
+
+struct Token {
+    uint32_t tok, nbits, extra;
+};
+
+inline Token token_of(uint32_t u, uint32_t m) {
+    if (u < (1u << m)) return {u, 0, 0};
+    uint32_t h = split_h(m);
+    uint32_t n = uint32_t(bitlen(u)) - 1;
+    uint32_t low = n - h;
+    return {(1u << m) + ((n - m) << h) + ((u >> low) & ((1u << h) - 1u)), low, u & ((1u << low) - 1u)};
+}
+
+// smallest m in [0, 7] with >= 99% of the values below 2^m (bit length <= m)
+uint32_t pick_split(const uint64_t *by_len) {
+    uint64_t n = 0;
+    for (int i = 0; i <= 32; ++i) n += by_len[i];
+    if (!n) return 0;
+    uint64_t acc = 0;
+    for (uint32_t m = 0; m <= uint32_t(kMaxSplit); ++m) {
+        acc += by_len[m];
+        if (acc * 100u >= n * 99u) return m;
+    }
+    return kMaxSplit;
+}
+
+// largest remainders to a sum of 2^11, then every seen token raised to >= 1 from the
+// currently largest frequency (lowest index on ties)
+uint32_t build_freqs(const std::vector<uint64_t> &cnt, std::vector<uint32_t> &f) {
+    size_t n = cnt.size();
+    f.assign(n, 0);
+    uint64_t total = 0;
+    uint32_t len = 0;
+    for (size_t i = 0; i < n; ++i) {
+        total += cnt[i];
+        if (cnt[i]) len = uint32_t(i + 1);
+    }
+    if (!total) return 0;
+    std::vector<std::pair<uint64_t, uint32_t>> rems;  // (remainder, index)
+    uint32_t used = 0;
+    for (size_t i = 0; i < n; ++i) {
+        if (!cnt[i]) continue;
+        uint64_t scaled = cnt[i] * kProbScale;
+        f[i] = uint32_t(scaled / total);
+        used += f[i];
+        rems.emplace_back(scaled % total, uint32_t(i));
+    }
+    std::stable_sort(rems.begin(), rems.end(),
+                     [](const auto &a, const auto &b) { return a.first > b.first; });
+    for (uint32_t r = 0; r < kProbScale - used; ++r) f[rems[r].second] += 1;
+    for (size_t i = 0; i < n; ++i) {
+        if (cnt[i] && !f[i]) {
+            size_t big = size_t(std::max_element(f.begin(), f.end()) - f.begin());
+            f[big] -= 1;
+            f[i] = 1;
+        }
+    }
+    return len;
+}
+
+// ------------------------------------------------------------------ the encoder
+struct Encoder {
+    Source src;
+    int64_t rows, cols, nb;
+    int container;
+    int threads;
+    uint32_t K;
+    std::vector<float> codes;   // INT8/FP8 code matrix (exact in fp32), empty otherwise
+    std::vector<float> scales;  // INT8/FP8 per-row scales
+    std::vector<float> rms;     // per-row RMS s_r
+
+    double value(int64_t i) const { return codes.empty() ? double(src.at(i)) : double(codes[size_t(i)]); }
+
+    void quantize_block(int64_t b, float f, int32_t *v) const {
+        if (f == 0.0f) {
+            std::fill(v, v + 8, 0);
+            return;
+        }
+        double x[8], two_f = 2.0 * double(f);
+        for (int i = 0; i < 8; ++i) x[i] = value(8 * b + i) / two_f;
+        quantize_e8(x, v);
+    }
+
+    void prepare() {
+        int64_t cb = cols / 8;
+        nb = rows * cb;
+        if (is_code_container(container)) {
+            codes.resize(size_t(rows * cols));
+            scales.resize(size_t(rows));
+            double bound = container == EP_INT8 ? 127.0 : 448.0;
+            parallel_for(rows, threads, [&](int64_t r0, int64_t r1) {
+                for (int64_t r = r0; r < r1; ++r) {
+                    double amax = 0.0;
+                    for (int64_t j = 0; j < cols; ++j) amax = std::max(amax, std::fabs(double(src.at(r * cols + j))));
+                    float s = amax > 0.0 ? float(amax / bound) : 1.0f;
+                    if (s == 0.0f) s = FLT_MIN;
+                    scales[size_t(r)] = s;
+                    for (int64_t j = 0; j < cols; ++j) {
+                        double w = src.at(r * cols + j);
+                        double c;
+                        if (amax == 0.0) {
+                            c = 0.0;
+                        } else if (container == EP_INT8) {
+                            c = std::min(127.0, std::max(-127.0, std::nearbyint(w / double(s))));
+                        } else {
+                            c = e4m3_round(float(w / double(s)));
+                        }
+                        codes[size_t(r * cols + j)] = float(c);
+                    }
+                }
+            });
+        }
+        rms.resize(size_t(rows));
+        parallel_for(rows, threads, [&](int64_t r0, int64_t r1) {
+            for (int64_t r = r0; r < r1; ++r) {
+                double acc = 0.0;
+                for (int64_t j = 0; j < cols; ++j) {
+                    double a = value(r * cols + j);
+                    acc += a * a;
+                }
+                rms[size_t(r)] = float(std::sqrt(acc / double(cols)));
+            }
+        });
+    }
+
+    uint32_t tile_count() const { return uint32_t((nb + int64_t(kLanes) * K - 1) / (int64_t(kLanes) * K)); }
+
+    // ---- sampled storage estimate (bits per weight at resolution index k)
+    double estimate(int k) const {
+        int64_t cb = cols / 8;
+        int64_t step = std::max<int64_t>(1, (nb + kSampleBlocks - 1) / kSampleBlocks);
+        int64_t ns = (nb + step - 1) / step;
+        std::vector<uint8_t> ctx(static_cast<size_t>(ns) * 8);
+        std::vector<uint32_t> val(static_cast<size_t>(ns) * 8);
+        parallel_for(ns, threads, [&](int64_t j0, int64_t j1) {
+            for (int64_t j = j0; j < j1; ++j) {
+                int64_t b = j * step;
+                int32_t v[8];
+                quantize_block(b, factor_of(rms[size_t(b / cb)], k), v);
+                symbols_of(v, &ctx[size_t(8 * j)], &val[size_t(8 * j)]);
+            }
+        });
+        uint64_t by_len[kContexts][33] = {};
+        for (size_t i = 0; i < val.size(); ++i) by_len[ctx[i]][bitlen(val[i])]++;
+        uint32_t m[kContexts];
+        std::vector<uint64_t> cnt[kContexts];
+        for (int c = 0; c < kContexts; ++c) {
+            m[c] = pick_split(by_len[c]);
+            cnt[c].assign(split_alphabet(m[c]), 0);
+        }
+        uint64_t extra = 0;
+        for (size_t i = 0; i < val.size(); ++i) {
+            Token t = token_of(val[i], m[ctx[i]]);
+            cnt[ctx[i]][t.tok]++;
+            extra += t.nbits;
+        }
+        double bits = 0.0;
+        uint64_t tokens = 0;
+        for (int c = 0; c < kContexts; ++c) {
+            uint64_t n = 0;
+            uint32_t len = 0;
+            for (size_t t = 0; t < cnt[c].size(); ++t) {
+                n += cnt[c][t];
+                if (cnt[c][t]) len = uint32_t(t + 1);
+            }
+            tokens += len;
+            if (!n) continue;
+            bits += double(n) * std::log2(double(n));
+            for (size_t t = 0; t < cnt[c].size(); ++t)
+                if (cnt[c][t]) bits -= double(cnt[c][t]) * std::log2(double(cnt[c][t]));
+        }
+        bits += double(extra);
+        uint32_t T = tile_count();
+        Layout L = layout_for(rows, container, tokens, T);
+        double bytes = double(L.tiles) + kTileOverheadBytes * double(T) + bits * (double(nb) / double(ns)) / 8.0;
+        return 8.0 * bytes / double(rows * cols);
+    }
+
+    // ---- one tile: events in decode order, encoded in reverse
+    struct Event {
+        uint16_t f, cum;
+        uint8_t lane;
+    };
+
+    static void encode_tile(const uint8_t *ctx, const uint32_t *val, int64_t nb, int64_t t, uint32_t K,
+                            const uint32_t *m, const std::vector<uint32_t> *freq, const std::vector<uint32_t> *cum,
+                            std::vector<Event> &ev, std::vector<uint16_t> &words, std::vector<uint8_t> &out) {
+        ev.clear();
+        words.clear();
+        int64_t first = t * int64_t(kLanes) * K;
+        for (uint32_t k = 0; k < K; ++k) {
+            int64_t b0 = first + int64_t(k) * kLanes;
+            if (b0 >= nb) break;
+            int lanes = int(std::min<int64_t>(kLanes, nb - b0));
+            for (int i = 0; i < 8; ++i) {
+                Token tk[kLanes];
+                uint32_t maxbits = 0;
+                for (int l = 0; l < lanes; ++l) {
+                    size_t s = size_t(8 * (b0 + l) + i);
+                    uint8_t c = ctx[s];
+                    tk[l] = token_of(val[s], m[c]);
+                    ev.push_back({uint16_t(freq[c][tk[l].tok]), uint16_t(cum[c][tk[l].tok]), uint8_t(l)});
+                    maxbits = std::max(maxbits, tk[l].nbits);
+                }
+                for (uint32_t j = 0; j * kChunkBits < maxbits; ++j) {
+                    for (int l = 0; l < lanes; ++l) {
+                        if (tk[l].nbits <= j * kChunkBits) continue;
+                        uint32_t bits = std::min(kChunkBits, tk[l].nbits - j * kChunkBits);
+                        uint32_t chunk = (tk[l].extra >> (j * kChunkBits)) & ((1u << bits) - 1u);
+                        uint32_t f = 1u << (kProbBits - bits);
+                        ev.push_back({uint16_t(f), uint16_t(chunk * f), uint8_t(l)});
+                    }
+                }
+            }
+        }
+        uint32_t x[kLanes];
+        std::fill(x, x + kLanes, kStateLow);
+        for (size_t e = ev.size(); e-- > 0;) {
+            uint32_t &s = x[ev[e].lane];
+            uint32_t f = ev[e].f;
+            if (uint64_t(s) >= (uint64_t(f) << (32 - kProbBits))) {  // keep the next state below 2^32
+                words.push_back(uint16_t(s));
+                s >>= 16;
+            }
+            s = (s / f) * kProbScale + (s % f) + ev[e].cum;
+        }
+        size_t base = out.size();
+        size_t bytes = align16(4 * kLanes + 2 * words.size());
+        out.resize(base + bytes, 0);
+        uint8_t *p = out.data() + base;
+        for (int l = 0; l < kLanes; ++l)
+            for (int b = 0; b < 4; ++b) p[4 * l + b] = uint8_t(x[l] >> (8 * b));
+        p += 4 * kLanes;
+        for (size_t i = 0; i < words.size(); ++i) {
+            uint16_t w = words[words.size() - 1 - i];
+            p[2 * i] = uint8_t(w);
+            p[2 * i + 1] = uint8_t(w >> 8);
+        }
+    }
+
+    // ---- full stream at resolution index k
+    std::vector<uint8_t> encode(int k) const {
+        int64_t cb = cols / 8;
+        std::vector<uint8_t> ctx(static_cast<size_t>(nb) * 8);
+        std::vector<uint32_t> val(static_cast<size_t>(nb) * 8);
+        std::vector<float> fac(static_cast<size_t>(rows));
+        for (int64_t r = 0; r < rows; ++r) fac[size_t(r)] = factor_of(rms[size_t(r)], k);
+        int nchunks = int(std::max<int64_t>(1, std::min<int64_t>(threads, (nb + 1023) / 1024)));
+        std::vector<std::vector<uint64_t>> part_len(size_t(nchunks), std::vector<uint64_t>(kContexts * 33, 0));
+        int64_t per = (nb + nchunks - 1) / nchunks;
+        parallel_for(nchunks, nchunks, [&](int64_t c0, int64_t c1) {
+            for (int64_t c = c0; c < c1; ++c) {
+                auto &hist = part_len[size_t(c)];
+                for (int64_t b = c * per; b < std::min(nb, (c + 1) * per); ++b) {
+                    int32_t v[8];
+                    quantize_block(b, fac[size_t(b / cb)], v);
+                    symbols_of(v, &ctx[size_t(8 * b)], &val[size_t(8 * b)]);
+                    for (int i = 0; i < 8; ++i) hist[size_t(ctx[size_t(8 * b + i)] * 33 + bitlen(val[size_t(8 * b + i)]))]++;
+                }
+            }
+        });
+        uint64_t by_len[kContexts][33] = {};
+        for (auto &h : part_len)
+            for (int c = 0; c < kContexts; ++c)
+                for (int i = 0; i < 33; ++i) by_len[c][i] += h[size_t(c * 33 + i)];
+        uint32_t m[kContexts];
+        for (int c = 0; c < kContexts; ++c) m[c] = pick_split(by_len[c]);
+        // token counts
+        std::vector<std::vector<uint64_t>> part_cnt(static_cast<size_t>(nchunks));
+        parallel_for(nchunks, nchunks, [&](int64_t c0, int64_t c1) {
+            for (int64_t c = c0; c < c1; ++c) {
+                auto &cnt = part_cnt[size_t(c)];
+                cnt.assign(kContexts * 256, 0);
+                for (int64_t s = 8 * c * per; s < 8 * std::min(nb, (c + 1) * per); ++s)
+                    cnt[size_t(ctx[size_t(s)]) * 256 + token_of(val[size_t(s)], m[ctx[size_t(s)]]).tok]++;
+            }
+        });
+        std::vector<uint32_t> freq[kContexts], cum[kContexts];
+        uint32_t ntok[kContexts];
+        uint64_t tokens = 0;
+        for (int c = 0; c < kContexts; ++c) {
+            std::vector<uint64_t> cnt(split_alphabet(m[c]), 0);
+            for (auto &pc : part_cnt)
+                for (size_t t = 0; t < cnt.size(); ++t) cnt[t] += pc[size_t(c) * 256 + t];
+            ntok[c] = build_freqs(cnt, freq[c]);
+            cum[c].assign(freq[c].size(), 0);
+            for (size_t t = 1; t < freq[c].size(); ++t) cum[c][t] = cum[c][t - 1] + freq[c][t - 1];
+            tokens += ntok[c];
+        }
+        // tiles, encoded in parallel into per-range buffers
+        uint32_t T = tile_count();
+        int tchunks = int(std::max<int64_t>(1, std::min<int64_t>(threads, T)));
+        std::vector<std::vector<uint8_t>> part_tiles(static_cast<size_t>(tchunks));
+        std::vector<std::vector<uint32_t>> part_sizes(static_cast<size_t>(tchunks));
+        int64_t tper = (int64_t(T) + tchunks - 1) / tchunks;
+        parallel_for(tchunks, tchunks, [&](int64_t c0, int64_t c1) {
+            std::vector<Event> ev;
+            std::vector<uint16_t> words;
+            for (int64_t c = c0; c < c1; ++c)
+                for (int64_t t = c * tper; t < std::min<int64_t>(T, (c + 1) * tper); ++t) {
+                    size_t before = part_tiles[size_t(c)].size();
+                    encode_tile(ctx.data(), val.data(), nb, t, K, m, freq, cum, ev, words, part_tiles[size_t(c)]);
+                    part_sizes[size_t(c)].push_back(uint32_t((part_tiles[size_t(c)].size() - before) / 16));
+                }
+        });
+        Layout L = layout_for(rows, container, tokens, T);
+        size_t tile_bytes = 0;
+        for (auto &pt : part_tiles) tile_bytes += pt.size();
+        std::vector<uint8_t> out(L.tiles + tile_bytes, 0);
+        uint8_t *h = out.data();
+        auto put = [](uint8_t *p, uint64_t v, int n) {
+            for (int i = 0; i < n; ++i) p[i] = uint8_t(v >> (8 * i));
+        };
+        put(h, kMagic, 4);
+        put(h + 4, kVersion, 2);
+        h[6] = uint8_t(src.dt);
+        h[7] = uint8_t(container);
+        put(h + 8, uint64_t(rows), 8);
+        put(h + 16, uint64_t(cols), 8);
+        put(h + 24, T, 4);
+        put(h + 28, K, 4);
+        put(h + 32, uint32_t(k), 2);
+        h[34] = uint8_t(kProbBits);
+        h[35] = uint8_t(kContexts);
+        for (int c = 0; c < kContexts; ++c) {
+            h[36 + c] = uint8_t(m[c]);
+            put(h + 44 + 2 * c, ntok[c], 2);
+        }
+        std::memcpy(h + L.rowf, fac.data(), size_t(rows) * 4);
+        if (is_code_container(container)) std::memcpy(h + L.scales, scales.data(), size_t(rows) * 4);
+        size_t q = L.freq;
+        for (int c = 0; c < kContexts; ++c)
+            for (uint32_t t = 0; t < ntok[c]; ++t, q += 2) put(h + q, freq[c][t], 2);
+        uint32_t at = 0;
+        size_t d = L.dir, o = L.tiles;
+        for (int c = 0; c < tchunks; ++c) {
+            for (uint32_t sz : part_sizes[size_t(c)]) {
+                put(h + d, at, 4);
+                d += 4;
+                at += sz;
+            }
+            std::memcpy(h + o, part_tiles[size_t(c)].data(), part_tiles[size_t(c)].size());
+            o += part_tiles[size_t(c)].size();
+        }
+        put(h + d, at, 4);
+        return out;
+    }
+};
+
+bool little_endian_host() {
+    uint32_t one = 1;
+    uint8_t b;
+    std::memcpy(&b, &one, 1);
+    return b == 1;
+}
+
+}  // namespace
+}  // namespace ep
+
+extern "C" size_t ep_compress_bound(int64_t rows, int64_t cols, const ep_config *cfg) {
+    if (rows <= 0 || cols <= 0 || !cfg) return 0;
+    double n = double(rows) * double(cols);
+    if (cfg->q_index < 0) return size_t(std::floor(cfg->target_bpp * n / 8.0));
+    int64_t nb = rows * (cols / 8);
+    uint32_t K = cfg->blocks_per_lane ? cfg->blocks_per_lane : ep::auto_blocks_per_lane(nb);
+    uint64_t T = uint64_t((nb + 32 * int64_t(K) - 1) / (32 * int64_t(K)));
+    return ep::layout_for(rows, ep::is_code_container(cfg->container_dtype) ? cfg->container_dtype : 0,
+                          7 * 256, T)
+               .tiles +
+           size_t(T) * (128 + 16) + size_t(5.0 * n);
+}
+
+extern "C" int ep_compress_host(const void *src, int32_t src_dtype, int64_t rows, int64_t cols, const ep_config *cfg,
+                                void *out, size_t out_cap, size_t *out_nbytes) {
+    using namespace ep;
+    if (!src || !cfg || !out_nbytes || rows <= 0 || cols <= 0) return EP_ERR_INVALID_ARG;
+    *out_nbytes = 0;
+    if (!little_endian_host()) return EP_ERR_UNSUPPORTED;
+    if (src_dtype != EP_BF16 && src_dtype != EP_FP16 && src_dtype != EP_FP32) return EP_ERR_UNSUPPORTED;
+    int container = cfg->container_dtype ? cfg->container_dtype : src_dtype;
+    if (container < EP_BF16 || container > EP_FP8_E4M3) return EP_ERR_INVALID_ARG;
+    if (cols % 8) return EP_ERR_UNSUPPORTED;
+    if (cfg->blocks_per_lane > 4096) return EP_ERR_INVALID_ARG;
+    if ((rows * (cols / 8)) >> 32) return EP_ERR_UNSUPPORTED;
+
+    Encoder E;
+    E.src = Source{src, src_dtype};
+    E.rows = rows;
+    E.cols = cols;
+    E.container = container;
+    E.threads = cfg->n_threads > 0 ? cfg->n_threads : int(std::max(1u, std::thread::hardware_concurrency()));
+    // finite check
+    {
+        int64_t n = rows * cols;
+        std::vector<char> bad(static_cast<size_t>(E.threads), 0);
+        int64_t per = (n + E.threads - 1) / E.threads;
+        parallel_for(E.threads, E.threads, [&](int64_t t0, int64_t t1) {
+            for (int64_t t = t0; t < t1; ++t)
+                for (int64_t i = t * per; i < std::min(n, (t + 1) * per); ++i)
+                    if (!std::isfinite(E.src.at(i))) {
+                        bad[size_t(t)] = 1;
+                        break;
+                    }
+        });
+        for (char b : bad)
+            if (b) return EP_ERR_NONFINITE;
+    }
+    double target = cfg->target_bpp;
+    if (!(target >= 0.001) || !(target <= 11.0) || (is_code_container(container) && !(target < 8.0)))
+        return EP_ERR_TARGET_RANGE;
+    E.prepare();
+    E.K = cfg->blocks_per_lane ? cfg->blocks_per_lane : auto_blocks_per_lane(E.nb);
+    int kmax = max_q_index(cols);
+    int k;
+    if (cfg->q_index >= 0) {
+        k = std::min(cfg->q_index, kmax);
+    } else {
+        double budget = kTargetMargin * target;
+        int lo = 0, hi = kmax;
+        while (lo < hi) {
+            int mid = lo + (hi - lo + 1) / 2;
+            if (E.estimate(mid) <= budget)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        k = lo;
+    }
+    std::vector<uint8_t> blob;
+    for (;;) {
+        blob = E.encode(k);
+        if (cfg->q_index >= 0 || 8.0 * double(blob.size()) <= target * double(rows * cols)) break;
+        if (k == 0) {
+            *out_nbytes = blob.size();
+            return EP_ERR_TARGET_UNREACHABLE;
+        }
+        --k;
+    }
+    *out_nbytes = blob.size();
+    if (!out || blob.size() > out_cap) return EP_ERR_BUFFER_TOO_SMALL;
+    std::memcpy(out, blob.data(), blob.size());
+    return EP_OK;
+}

@@ -1,0 +1,96 @@
+// Stream parser: ep_stream_info and ep_status_string.
+//
+// The CompressedTensor properties of the "EntroPack API reference" (shape, dtype,
+// actual_bpp = 8 * storage_nbytes / numel, storage_nbytes with and without the header)
+// read from a host copy of a format-v1 stream, which is validated before any decode.
+#include <cstring>
+
+#include "../../include/eptile.h"
+#include "format.h"
+
+namespace {
+
+uint64_t rd(const uint8_t *p, int n) {
+    uint64_t v = 0;
+    for (int i = n - 1; i >= 0; --i) v = (v << 8) | p[i];
+    return v;
+}
+
+}  // namespace
+
+extern "C" int ep_stream_info(const void *blob, size_t nbytes, ep_info *info) {
+    using namespace ep;
+    if (!blob || !info) return EP_ERR_INVALID_ARG;
+    const uint8_t *p = static_cast<const uint8_t *>(blob);
+    if (nbytes < kHeaderBytes) return EP_ERR_CORRUPT;
+    if (rd(p, 4) != kMagic || rd(p + 4, 2) != kVersion || p[34] != kProbBits || p[35] != kContexts)
+        return EP_ERR_CORRUPT;
+    ep_info I;
+    std::memset(&I, 0, sizeof I);
+    I.src_dtype = p[6];
+    I.container_dtype = p[7];
+    I.rows = int64_t(rd(p + 8, 8));
+    I.cols = int64_t(rd(p + 16, 8));
+    I.n_tiles = uint32_t(rd(p + 24, 4));
+    I.blocks_per_lane = uint32_t(rd(p + 28, 4));
+    I.q_index = int32_t(rd(p + 32, 2));
+    if (I.src_dtype < EP_BF16 || I.src_dtype > EP_FP32 || I.container_dtype < EP_BF16 ||
+        I.container_dtype > EP_FP8_E4M3)
+        return EP_ERR_CORRUPT;
+    if (I.rows <= 0 || I.cols <= 0 || I.cols % 8 || I.rows >= (int64_t(1) << 40) || I.cols >= (int64_t(1) << 40) ||
+        I.blocks_per_lane == 0 || I.blocks_per_lane > 4096 || I.q_index >= kNumQ)
+        return EP_ERR_CORRUPT;
+    int64_t nb = I.rows * (I.cols / 8);
+    int64_t per_tile = int64_t(kLanes) * I.blocks_per_lane;
+    if ((nb + per_tile - 1) / per_tile != int64_t(I.n_tiles)) return EP_ERR_CORRUPT;
+    uint64_t tokens = 0;
+    for (int c = 0; c < kContexts; ++c) {
+        I.split[c] = p[36 + c];
+        I.ntok[c] = uint16_t(rd(p + 44 + 2 * c, 2));
+        if (I.split[c] > kMaxSplit || I.ntok[c] > split_alphabet(I.split[c])) return EP_ERR_CORRUPT;
+        tokens += I.ntok[c];
+    }
+    Layout L = layout_for(I.rows, I.container_dtype, tokens, I.n_tiles);
+    if (L.tiles > nbytes) return EP_ERR_CORRUPT;
+    I.off_rowf = L.rowf;
+    I.off_scales = L.scales;
+    I.off_freq = L.freq;
+    I.off_dir = L.dir;
+    I.off_tiles = L.tiles;
+    size_t q = L.freq;
+    for (int c = 0; c < kContexts; ++c) {
+        uint32_t sum = 0;
+        for (uint32_t t = 0; t < I.ntok[c]; ++t, q += 2) sum += uint32_t(rd(p + q, 2));
+        if (I.ntok[c] && sum != kProbScale) return EP_ERR_CORRUPT;
+    }
+    const uint8_t *d = p + L.dir;
+    uint64_t prev = rd(d, 4);
+    if (prev != 0) return EP_ERR_CORRUPT;
+    for (uint32_t t = 1; t <= I.n_tiles; ++t) {
+        uint64_t cur = rd(d + 4 * t, 4);
+        if (cur < prev + 8) return EP_ERR_CORRUPT;  // a tile holds at least its 32 states
+        prev = cur;
+    }
+    if (L.tiles + 16 * prev != nbytes) return EP_ERR_CORRUPT;
+    I.storage_nbytes = nbytes;
+    I.header_nbytes = kHeaderBytes;
+    I.actual_bpp = 8.0 * double(nbytes) / double(I.rows * I.cols);
+    I.out_nbytes = uint64_t(I.rows * I.cols) * uint64_t(elt_bytes(I.container_dtype));
+    *info = I;
+    return EP_OK;
+}
+
+extern "C" const char *ep_status_string(int s) {
+    switch (s) {
+    case EP_OK: return "ok";
+    case EP_ERR_INVALID_ARG: return "invalid argument";
+    case EP_ERR_NONFINITE: return "tensor holds NaN or Inf";
+    case EP_ERR_TARGET_RANGE: return "target_bpp outside the supported range";
+    case EP_ERR_TARGET_UNREACHABLE: return "target_bpp below what the metadata alone needs";
+    case EP_ERR_BUFFER_TOO_SMALL: return "output buffer too small";
+    case EP_ERR_CORRUPT: return "stream fails validation";
+    case EP_ERR_CUDA: return "CUDA runtime error";
+    case EP_ERR_UNSUPPORTED: return "not supported by stream format v1";
+    default: return "unknown status";
+    }
+}

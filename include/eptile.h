@@ -1,0 +1,137 @@
+/*
+ * eptile -- lattice-rANS weight streams with a fused B200 (sm_100a) decode.
+ *
+ * C ABI of libeptile.so.  Plain pointers and sizes only; no exceptions cross it; every
+ * call returns an ep_status (0 = EP_OK, negative = error).  The library never allocates
+ * device memory and never synchronises a stream: the caller owns every buffer.
+ *
+ * Sources (EntroPack pages, by title and section):
+ *   "EntroPack API reference" -- compress(tensor, config) -> CompressedTensor,
+ *       decompress(compressed) -> tensor with the same shape and dtype, CompressedTensor
+ *       actual_bpp = 8 * storage_nbytes / numel and storage_nbytes(include_header).
+ *   "EntroPack: Fast and Accurate Entropy-Coded Weight Compression at Arbitrary Bitrates",
+ *       Abstract -- row-normalized E8 lattice quantization, a conditional model of the
+ *       lattice coordinates, resolution chosen by sampled storage estimates, entropy coding
+ *       in independently decodable tiles, fused GPU symbol decode and reconstruction,
+ *       BF16 / FP16 / FP8 / INT8 containers.
+ *   "EntroPack README", Configuration -- 0.001 <= target_bpp <= 11.
+ *   "Compressed Linear usage", Combine compression with FP8 or INT8 computation -- lossy
+ *       compression of FP8 / INT8 weight codes, 0.001 <= target_bpp < 8, per-row scales
+ *       counted in storage.
+ * The byte layout of the stream (format version 1) is this library's own; it is written
+ * out in the repository's design notes.
+ */
+#ifndef EPTILE_H
+#define EPTILE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* same type as cudaStream_t; NULL is the legacy default stream */
+typedef struct CUstream_st *ep_stream_t;
+
+/* element types: source tensors (BF16, FP16, FP32) and containers (the first five).
+ * EP_LATTICE_I32 is an output form only: the decoded lattice points v = 2z as int32. */
+enum ep_dtype { EP_BF16 = 1, EP_FP16 = 2, EP_FP32 = 3, EP_INT8 = 4, EP_FP8_E4M3 = 5, EP_LATTICE_I32 = 6 };
+
+enum ep_status {
+    EP_OK = 0,
+    EP_ERR_INVALID_ARG = -1,        /* null pointer, empty or non-2-D shape, bad dtype/config */
+    EP_ERR_NONFINITE = -2,          /* NaN or Inf in the source ("finite values", API reference) */
+    EP_ERR_TARGET_RANGE = -3,       /* target_bpp outside [0.001, 11], or >= 8 for INT8/FP8 codes */
+    EP_ERR_TARGET_UNREACHABLE = -4, /* even the coarsest resolution (metadata alone) exceeds the target */
+    EP_ERR_BUFFER_TOO_SMALL = -5,   /* out_cap too small; *out_nbytes holds the size needed */
+    EP_ERR_CORRUPT = -6,            /* the stream fails validation */
+    EP_ERR_CUDA = -7,               /* a CUDA runtime call failed (launch, attribute) */
+    EP_ERR_UNSUPPORTED = -8         /* valid but outside format v1: cols % 8 != 0, > 2^32 blocks */
+};
+
+/* bits the decode kernel ORs into *d_status when a stream is damaged */
+enum ep_decode_flags {
+    EP_DEC_WORD_OVERRUN = 1u, /* a renormalisation read ran past the tile's words */
+    EP_DEC_BAD_TOKEN = 2u,    /* a token outside its table (reported by the oracle; the
+                                 kernel reports such damage through the two flags below) */
+    EP_DEC_BAD_END = 4u,      /* a lane's state did not return to 2^16 at the end of its tile */
+    EP_DEC_WORD_COUNT = 8u,   /* the tile has unread words beyond its 16-byte padding */
+    EP_DEC_BAD_TILE = 16u     /* a tile directory entry points outside the tile section */
+};
+
+typedef struct {
+    double target_bpp;        /* bits per weight, including all metadata ("actual_bpp", API ref.) */
+    int32_t container_dtype;  /* 0 = the source dtype; EP_INT8 / EP_FP8_E4M3 = per-row absmax codes */
+    uint32_t blocks_per_lane; /* tile size K (blocks per lane); 0 = chosen from the shape */
+    int32_t q_index;          /* -1 = search the resolution; >= 0 = encode at this resolution index */
+    int32_t n_threads;        /* host encoder threads; 0 = all hardware threads */
+} ep_config;
+
+typedef struct {
+    int64_t rows, cols;
+    int32_t src_dtype, container_dtype;
+    uint64_t storage_nbytes;  /* total stream bytes = storage_nbytes(include_header=True) */
+    uint64_t header_nbytes;   /* 64; storage_nbytes - header_nbytes = include_header=False */
+    double actual_bpp;        /* 8 * storage_nbytes / (rows * cols) */
+    int32_t q_index;          /* resolution index k: lattice scale q = (64 + k%64) * 2^(k/64 - 14) */
+    uint32_t n_tiles, blocks_per_lane;
+    uint8_t split[8];         /* per-context token split m (7 contexts) */
+    uint16_t ntok[8];         /* per-context table length */
+    uint64_t off_rowf;        /* byte offsets of the sections inside the stream */
+    uint64_t off_scales;      /* INT8/FP8: per-row dequantization scales (fp32), for a GEMM consumer */
+    uint64_t off_freq, off_dir, off_tiles;
+    uint64_t out_nbytes;      /* rows * cols * container element size */
+} ep_info;
+
+/* Upper bound of the stream size for ep_compress_host: with a searched resolution the
+ * stream never exceeds floor(target_bpp * rows * cols / 8); with a fixed q_index the bound
+ * is loose (metadata + 5 bytes per weight).  Returns 0 for invalid arguments. */
+size_t ep_compress_bound(int64_t rows, int64_t cols, const ep_config *cfg);
+
+/* compress(tensor, config) of the API reference, on the host.
+ *   src        host pointer, row-major rows x cols elements of src_dtype (BF16/FP16/FP32),
+ *              read only.
+ *   cfg        target_bpp etc. (see ep_config); not retained.
+ *   out        host buffer of out_cap bytes that receives the stream; caller-owned.
+ *   out_nbytes receives the stream size (also on EP_ERR_BUFFER_TOO_SMALL: the size needed).
+ * Steps (Abstract): optional per-row INT8/FP8 code preparation, row normalisation, a
+ * resolution search on sampled storage estimates, E8 nearest-point quantization, per-context
+ * frequency tables, tile-wise interleaved rANS.  The result satisfies actual_bpp <=
+ * target_bpp or the call fails with EP_ERR_TARGET_UNREACHABLE.  Deterministic: the bytes do
+ * not depend on n_threads.  Thread-safe (no global state). */
+int ep_compress_host(const void *src, int32_t src_dtype, int64_t rows, int64_t cols, const ep_config *cfg,
+                     void *out, size_t out_cap, size_t *out_nbytes);
+
+/* CompressedTensor's properties (API reference) from a HOST copy of the stream.
+ *   blob   host pointer to the first nbytes of the stream; nbytes must be the whole stream
+ *          (the tile directory is checked against the stream end).
+ *   info   filled on success.
+ * Validates magic, version, shape, dtypes, table sums (each used context sums to 2048) and
+ * the tile directory; returns EP_ERR_CORRUPT otherwise. */
+int ep_stream_info(const void *blob, size_t nbytes, ep_info *info);
+
+/* decompress(compressed) of the API reference: the fused decode on the GPU.
+ *   info      from ep_stream_info on a host copy of the same stream.
+ *   d_blob    device pointer to the whole stream (info->storage_nbytes bytes), 16-byte aligned.
+ *   d_out     device pointer to rows * cols elements of out_dtype, row-major, 16-byte aligned.
+ *   out_dtype info->container_dtype (the reconstructed weights or codes), or EP_LATTICE_I32 for
+ *             the decoded lattice points v = 2z (int32) before scaling; no other conversion.
+ *   d_status  nullable device pointer to one uint32; the kernel ORs EP_DEC_* bits into it
+ *             when it meets a damaged tile (clear it before the call to read it per call).
+ *   stream    CUDA stream of the launch.
+ * One kernel launch (sm_100a): a persistent grid in which each warp decodes whole tiles with
+ * its 32 lanes as interleaved rANS states, rebuilds the E8 coset in registers, scales by the
+ * row factor in fp32 and stores the container with coalesced vector stores.  Asynchronous:
+ * errors of the launch itself are returned; stream damage goes to d_status.  The library
+ * allocates nothing and keeps a per-device cache of the SM count only. */
+int ep_decompress(const ep_info *info, const void *d_blob, void *d_out, int32_t out_dtype, uint32_t *d_status,
+                  ep_stream_t stream);
+
+/* static string for a status code */
+const char *ep_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -231,15 +231,19 @@ def parse(blob):
     return rc, info
 
 
-def decode(blob, t0=0, t1=None, want_v=True, want_out=True):
-    """Returns (rc, status, v (rows, cols) int32 or None, out (rows, cols) container array or None)."""
+def decode(blob, t0=0, t1=None, want_v=True, want_out=True, out_buf=None):
+    """Returns (rc, status, v (rows, cols) int32 or None, out (rows, cols) container array or None).
+    ``out_buf``: optional preallocated container array to decode into."""
     blob = np.ascontiguousarray(blob, dtype=np.uint8)
     rc, info = parse(blob)
     if rc != OK:
         return rc, 0, None, None
     R, Cc = info.rows, info.cols
     v = np.zeros((R, Cc), np.int32) if want_v else None
-    out = np.zeros((R, Cc), NP_DTYPE[info.container_dtype]) if want_out else None
+    if out_buf is not None:
+        out = out_buf
+    else:
+        out = np.zeros((R, Cc), NP_DTYPE[info.container_dtype]) if want_out else None
     st = C.c_uint32(0)
     t1 = info.n_tiles if t1 is None else t1
     rc = lib().or_decode(_ptr(blob), blob.size, t0, t1, _ptr(v) if v is not None else None,

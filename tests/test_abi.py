@@ -1,0 +1,100 @@
+"""The C-ABI library loads without a GPU and exports every function include/eptile.h
+declares; the host-side calls (compressor, parser) behave as documented."""
+import ctypes as C
+
+import numpy as np
+import pytest
+import torch
+
+from dit_weight_compression_tile_b200 import binding as B
+from dit_weight_compression_tile_b200 import synth
+
+
+def test_exports_every_declared_symbol():
+    names = B.declared_functions()
+    assert set(names) == {"ep_compress_bound", "ep_compress_host", "ep_stream_info", "ep_decompress",
+                          "ep_status_string"}
+    lib = B.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    # the symbols are plain C (unmangled) in the shared object's dynamic table
+    raw = C.CDLL(B.LIB_PATH)
+    for n in names:
+        assert C.cast(getattr(raw, n), C.c_void_p).value
+
+
+def test_status_strings():
+    lib = B.lib()
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, 99):
+        assert lib.ep_status_string(code)
+
+
+def test_info_fields_and_storage():
+    w = synth.gaussian(256, 256, 0.02, 0)
+    blob = B.compress(w, 3.5)
+    info = B.stream_info(blob)
+    assert info.shape == (256, 256) and info.dtype == torch.bfloat16
+    assert info.storage_nbytes == blob.numel()
+    assert info.actual_bpp == 8.0 * blob.numel() / w.numel() <= 3.5  # "actual_bpp" of the API reference
+    assert info.storage_nbytes_(include_header=False) == blob.numel() - 64
+    assert info.out_nbytes == 2 * w.numel()
+
+
+def test_errors():
+    w = synth.gaussian(8, 64, 0.02, 1)
+    with pytest.raises(B.EpError) as e:
+        bad = w.clone()
+        bad[0, 0] = float("nan")
+        B.compress(bad, 4.0)
+    assert e.value.status == -2
+    with pytest.raises(B.EpError) as e:
+        B.compress(w, 12.0)
+    assert e.value.status == -3
+    with pytest.raises(B.EpError) as e:
+        B.compress(w, 8.0, container="int8")
+    assert e.value.status == -3
+    with pytest.raises(B.EpError) as e:
+        B.compress(w, 0.01)
+    assert e.value.status == -4
+    with pytest.raises(B.EpError) as e:
+        B.compress(synth.gaussian(8, 12, 0.02, 1), 4.0)
+    assert e.value.status == -8
+    with pytest.raises(B.EpError):
+        B.compress(torch.zeros(0, 8), 4.0)
+    with pytest.raises(B.EpError):
+        B.stream_info(torch.zeros(10, dtype=torch.uint8))
+
+
+def test_corrupt_streams_rejected():
+    w = synth.gaussian(64, 512, 0.02, 2)
+    blob = B.compress(w, 4.0)
+    info = B.stream_info(blob)
+    with pytest.raises(B.EpError):
+        B.stream_info(blob[:-16])
+    # (a moved inner directory entry passes the parser; the decoder flags it)
+    for off in (0, 4, 7, 34, info.off_freq, info.off_dir):
+        bad = blob.clone()
+        bad[off] ^= 0x5A
+        with pytest.raises(B.EpError) as e:
+            B.stream_info(bad)
+        assert e.value.status == -6, off
+
+
+def test_decompress_needs_device_memory():
+    blob = B.compress(synth.gaussian(16, 64, 0.02, 3), 11.0, q_index=600)
+    with pytest.raises(B.EpError):
+        B.decompress(blob)
+
+
+def test_compress_bound_holds():
+    w = synth.gaussian(64, 256, 0.02, 4)
+    for target in (0.5, 2.0, 4.0, 8.0):
+        cfg = B._config(target)
+        bound = B.lib().ep_compress_bound(64, 256, C.byref(cfg))
+        try:
+            blob = B.compress(w, target)
+        except B.EpError:
+            continue
+        assert blob.numel() <= bound
+    cfg = B._config(4.0, q_index=900)
+    assert B.compress(w, 4.0, q_index=900).numel() <= B.lib().ep_compress_bound(64, 256, C.byref(cfg))
