@@ -230,10 +230,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_
     const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
 
     // ---- tables: sentinel everywhere (token 255, f = 2^11: an identity step), then the
-    // cumulative frequencies per context (one warp each), then the slots of every token
+    // cumulative frequencies per context (warps take contexts round robin), then the slots of
+    // every token
     for (uint32_t i = threadIdx.x; i < kLutEntries; i += blockDim.x) lut[i] = (255u << 24) | (kProbScale << 12) | (i & (kProbScale - 1));
-    if (warp < uint32_t(kContexts)) {
-        uint32_t c = warp, n = p.tab_off[c + 1] - p.tab_off[c], run = 0;
+    for (uint32_t c = warp; c < uint32_t(kContexts); c += nwarps) {  // small CTAs take several contexts
+        uint32_t n = p.tab_off[c + 1] - p.tab_off[c], run = 0;
         for (uint32_t base = 0; base < n; base += 32) {
             uint32_t t = base + lane;
             uint32_t f = t < n ? uint32_t(p.freq[p.tab_off[c] + t]) : 0u;
