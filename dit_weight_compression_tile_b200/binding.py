@@ -43,6 +43,7 @@ class StreamInfo(C.Structure):
         ("split", C.c_uint8 * 8), ("ntok", C.c_uint16 * 8),
         ("off_rowf", C.c_uint64), ("off_scales", C.c_uint64), ("off_freq", C.c_uint64),
         ("off_dir", C.c_uint64), ("off_tiles", C.c_uint64), ("out_nbytes", C.c_uint64),
+        ("max_tile_nbytes", C.c_uint64),
     ]
 
     @property

@@ -9,7 +9,7 @@
 namespace ep {
 
 constexpr uint32_t kMagic = 0x31545045u;  // "EPT1"
-constexpr uint32_t kVersion = 1;
+constexpr uint32_t kVersion = 2;
 constexpr uint32_t kProbBits = 11;         // frequency precision: tables sum to 2^11
 constexpr uint32_t kProbScale = 1u << kProbBits;
 constexpr uint32_t kStateLow = 1u << 16;   // rANS state interval [2^16, 2^32), 16-bit words
@@ -18,9 +18,11 @@ constexpr int kContexts = 7;
 constexpr int kMaxSplit = 7;
 constexpr uint32_t kChunkBits = 11;        // extra bits travel in uniform chunks of <= 11 bits
 constexpr size_t kHeaderBytes = 64;
+constexpr size_t kTileHead = 192;            // per tile: 32 initial states (u32) + 32 word counts (u16)
+constexpr double kTileBudget = 5952.0;       // expected payload bytes per tile (6 KB staging buffer)
 constexpr int kNumQ = 1280;                // resolution indices
 constexpr int64_t kSampleBlocks = 65536;   // blocks sampled by the storage estimate
-constexpr double kTileOverheadBytes = 104.0;  // per tile in the estimate
+constexpr double kTileOverheadBytes = 168.0;  // per tile in the estimate
 constexpr double kTargetMargin = 0.995;
 
 inline size_t align16(size_t n) { return (n + 15) & ~size_t(15); }
@@ -48,12 +50,14 @@ inline Layout layout_for(int64_t rows, int container, uint64_t total_tokens, uin
     return L;
 }
 
-// K (blocks per lane) from the block count: 16 below 2^20 blocks, else the power of two at
-// or below nb / 2^16, at most 256.
-inline uint32_t auto_blocks_per_lane(int64_t nb) {
-    int64_t target = nb >> 16;
+// K (blocks per lane) from the block count and the target rate: the power of two at or below
+// nb / 2^16 (at least 16, at most 256), halved while a tile's expected payload (32 K blocks x 8
+// coordinates x target bits, plus a tenth) exceeds the staging budget.
+inline uint32_t auto_blocks_per_lane(int64_t nb, double target_bpp) {
+    int64_t want = nb >> 16;
     uint32_t k = 16;
-    while (k < 256 && int64_t(k) * 2 <= target) k <<= 1;
+    while (k < 256 && int64_t(k) * 2 <= want) k <<= 1;
+    while (k > 1 && 32.0 * double(k) * target_bpp * 1.1 > kTileBudget) k >>= 1;
     return k;
 }
 

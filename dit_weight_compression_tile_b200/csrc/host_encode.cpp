@@ -207,7 +207,7 @@ inline Token token_of(uint32_t u, uint32_t m) {
     return {(1u << m) + ((n - m) << h) + ((u >> low) & ((1u << h) - 1u)), low, u & ((1u << low) - 1u)};
 }
 
-// smallest m in [0, 7] with >= 99% of the values below 2^m (bit length <= m)
+// smallest m in [0, 7] with >= 99.9% of the values below 2^m (bit length <= m)
 uint32_t pick_split(const uint64_t *by_len) {
     uint64_t n = 0;
     for (int i = 0; i <= 32; ++i) n += by_len[i];
@@ -215,7 +215,7 @@ uint32_t pick_split(const uint64_t *by_len) {
     uint64_t acc = 0;
     for (uint32_t m = 0; m <= uint32_t(kMaxSplit); ++m) {
         acc += by_len[m];
-        if (acc * 100u >= n * 99u) return m;
+        if (acc * 1000u >= n * 999u) return m;
     }
     return kMaxSplit;
 }
@@ -372,65 +372,64 @@ struct Encoder {
         return 8.0 * bytes / double(rows * cols);
     }
 
-    // ---- one tile: events in decode order, encoded in reverse
+    // ---- one tile: 32 independent lanes, each its symbols in decode order encoded in reverse
     struct Event {
         uint16_t f, cum;
-        uint8_t lane;
     };
 
     static void encode_tile(const uint8_t *ctx, const uint32_t *val, int64_t nb, int64_t t, uint32_t K,
                             const uint32_t *m, const std::vector<uint32_t> *freq, const std::vector<uint32_t> *cum,
                             std::vector<Event> &ev, std::vector<uint16_t> &words, std::vector<uint8_t> &out) {
-        ev.clear();
-        words.clear();
         int64_t first = t * int64_t(kLanes) * K;
-        for (uint32_t k = 0; k < K; ++k) {
-            int64_t b0 = first + int64_t(k) * kLanes;
-            if (b0 >= nb) break;
-            int lanes = int(std::min<int64_t>(kLanes, nb - b0));
-            for (int i = 0; i < 8; ++i) {
-                Token tk[kLanes];
-                uint32_t maxbits = 0;
-                for (int l = 0; l < lanes; ++l) {
-                    size_t s = size_t(8 * (b0 + l) + i);
+        uint32_t state[kLanes];
+        uint32_t count[kLanes];
+        words.clear();
+        std::vector<size_t> lane_end(kLanes);
+        for (int l = 0; l < kLanes; ++l) {
+            ev.clear();
+            for (uint32_t k = 0; k < K; ++k) {
+                int64_t b = first + int64_t(k) * kLanes + l;
+                if (b >= nb) break;
+                for (int i = 0; i < 8; ++i) {
+                    size_t s = size_t(8 * b + i);
                     uint8_t c = ctx[s];
-                    tk[l] = token_of(val[s], m[c]);
-                    ev.push_back({uint16_t(freq[c][tk[l].tok]), uint16_t(cum[c][tk[l].tok]), uint8_t(l)});
-                    maxbits = std::max(maxbits, tk[l].nbits);
-                }
-                for (uint32_t j = 0; j * kChunkBits < maxbits; ++j) {
-                    for (int l = 0; l < lanes; ++l) {
-                        if (tk[l].nbits <= j * kChunkBits) continue;
-                        uint32_t bits = std::min(kChunkBits, tk[l].nbits - j * kChunkBits);
-                        uint32_t chunk = (tk[l].extra >> (j * kChunkBits)) & ((1u << bits) - 1u);
+                    Token tk = token_of(val[s], m[c]);
+                    ev.push_back({uint16_t(freq[c][tk.tok]), uint16_t(cum[c][tk.tok])});
+                    for (uint32_t j = 0; j * kChunkBits < tk.nbits; ++j) {
+                        uint32_t bits = std::min(kChunkBits, tk.nbits - j * kChunkBits);
+                        uint32_t chunk = (tk.extra >> (j * kChunkBits)) & ((1u << bits) - 1u);
                         uint32_t f = 1u << (kProbBits - bits);
-                        ev.push_back({uint16_t(f), uint16_t(chunk * f), uint8_t(l)});
+                        ev.push_back({uint16_t(f), uint16_t(chunk * f)});
                     }
                 }
             }
-        }
-        uint32_t x[kLanes];
-        std::fill(x, x + kLanes, kStateLow);
-        for (size_t e = ev.size(); e-- > 0;) {
-            uint32_t &s = x[ev[e].lane];
-            uint32_t f = ev[e].f;
-            if (uint64_t(s) >= (uint64_t(f) << (32 - kProbBits))) {  // keep the next state below 2^32
-                words.push_back(uint16_t(s));
-                s >>= 16;
+            uint32_t x = kStateLow;
+            size_t before = words.size();
+            for (size_t e = ev.size(); e-- > 0;) {
+                uint32_t f = ev[e].f;
+                if (uint64_t(x) >= (uint64_t(f) << (32 - kProbBits))) {  // keep the next state below 2^32
+                    words.push_back(uint16_t(x));
+                    x >>= 16;
+                }
+                x = (x / f) * kProbScale + (x % f) + ev[e].cum;
             }
-            s = (s / f) * kProbScale + (s % f) + ev[e].cum;
+            std::reverse(words.begin() + long(before), words.end());  // decode order
+            state[l] = x;
+            count[l] = uint32_t(words.size() - before);
         }
         size_t base = out.size();
-        size_t bytes = align16(4 * kLanes + 2 * words.size());
+        size_t bytes = align16(kTileHead + 2 * words.size());
         out.resize(base + bytes, 0);
         uint8_t *p = out.data() + base;
-        for (int l = 0; l < kLanes; ++l)
-            for (int b = 0; b < 4; ++b) p[4 * l + b] = uint8_t(x[l] >> (8 * b));
-        p += 4 * kLanes;
+        for (int l = 0; l < kLanes; ++l) {
+            for (int b = 0; b < 4; ++b) p[4 * l + b] = uint8_t(state[l] >> (8 * b));
+            p[4 * kLanes + 2 * l] = uint8_t(count[l]);
+            p[4 * kLanes + 2 * l + 1] = uint8_t(count[l] >> 8);
+        }
+        p += kTileHead;
         for (size_t i = 0; i < words.size(); ++i) {
-            uint16_t w = words[words.size() - 1 - i];
-            p[2 * i] = uint8_t(w);
-            p[2 * i + 1] = uint8_t(w >> 8);
+            p[2 * i] = uint8_t(words[i]);
+            p[2 * i + 1] = uint8_t(words[i] >> 8);
         }
     }
 
@@ -558,12 +557,12 @@ extern "C" size_t ep_compress_bound(int64_t rows, int64_t cols, const ep_config 
     double n = double(rows) * double(cols);
     if (cfg->q_index < 0) return size_t(std::floor(cfg->target_bpp * n / 8.0));
     int64_t nb = rows * (cols / 8);
-    uint32_t K = cfg->blocks_per_lane ? cfg->blocks_per_lane : ep::auto_blocks_per_lane(nb);
+    uint32_t K = cfg->blocks_per_lane ? cfg->blocks_per_lane : ep::auto_blocks_per_lane(nb, cfg->target_bpp);
     uint64_t T = uint64_t((nb + 32 * int64_t(K) - 1) / (32 * int64_t(K)));
     return ep::layout_for(rows, ep::is_code_container(cfg->container_dtype) ? cfg->container_dtype : 0,
                           7 * 256, T)
                .tiles +
-           size_t(T) * (128 + 16) + size_t(5.0 * n);
+           size_t(T) * (ep::kTileHead + 16) + size_t(5.0 * n);
 }
 
 extern "C" int ep_compress_host(const void *src, int32_t src_dtype, int64_t rows, int64_t cols, const ep_config *cfg,
@@ -605,7 +604,7 @@ extern "C" int ep_compress_host(const void *src, int32_t src_dtype, int64_t rows
     if (!(target >= 0.001) || !(target <= 11.0) || (is_code_container(container) && !(target < 8.0)))
         return EP_ERR_TARGET_RANGE;
     E.prepare();
-    E.K = cfg->blocks_per_lane ? cfg->blocks_per_lane : auto_blocks_per_lane(E.nb);
+    E.K = cfg->blocks_per_lane ? cfg->blocks_per_lane : auto_blocks_per_lane(E.nb, target);
     int kmax = max_q_index(cols);
     int k;
     if (cfg->q_index >= 0) {

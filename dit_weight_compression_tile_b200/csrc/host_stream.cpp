@@ -64,13 +64,15 @@ extern "C" int ep_stream_info(const void *blob, size_t nbytes, ep_info *info) {
         if (I.ntok[c] && sum != kProbScale) return EP_ERR_CORRUPT;
     }
     const uint8_t *d = p + L.dir;
-    uint64_t prev = rd(d, 4);
+    uint64_t prev = rd(d, 4), largest = 0;
     if (prev != 0) return EP_ERR_CORRUPT;
     for (uint32_t t = 1; t <= I.n_tiles; ++t) {
         uint64_t cur = rd(d + 4 * t, 4);
-        if (cur < prev + 8) return EP_ERR_CORRUPT;  // a tile holds at least its 32 states
+        if (cur < prev + kTileHead / 16) return EP_ERR_CORRUPT;  // a tile holds at least its head
+        if (cur - prev > largest) largest = cur - prev;
         prev = cur;
     }
+    I.max_tile_nbytes = 16 * largest;
     if (L.tiles + 16 * prev != nbytes) return EP_ERR_CORRUPT;
     I.storage_nbytes = nbytes;
     I.header_nbytes = kHeaderBytes;

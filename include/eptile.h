@@ -82,6 +82,7 @@ typedef struct {
     uint64_t off_scales;      /* INT8/FP8: per-row dequantization scales (fp32), for a GEMM consumer */
     uint64_t off_freq, off_dir, off_tiles;
     uint64_t out_nbytes;      /* rows * cols * container element size */
+    uint64_t max_tile_nbytes; /* largest tile in the stream (sizes the decoder's staging buffers) */
 } ep_info;
 
 /* Upper bound of the stream size for ep_compress_host: with a searched resolution the

@@ -34,7 +34,7 @@
  * words, 32 interleaved states per tile, seven coding contexts.
  * ---------------------------------------------------------------------------------- */
 #define MAGIC 0x31545045u /* bytes 'E','P','T','1' */
-#define VERSION 1
+#define VERSION 2
 #define PROB_BITS 11
 #define PROB_M 2048u
 #define STATE_L 65536u
@@ -43,6 +43,8 @@
 #define MAX_SPLIT 7
 #define CHUNK_BITS 11
 #define HEADER_BYTES 64
+#define TILE_HEAD 192        /* 32 states (u32) + 32 word counts (u16) */
+#define TILE_BUDGET 5952.0   /* expected payload bytes a tile may hold (a 6 KB staging buffer) */
 #define NQ 1280
 #define SAMPLE_TARGET 65536
 
@@ -353,7 +355,7 @@ void or_tokenize_batch(const uint32_t *u, int64_t n, int32_t m, uint32_t *tok, u
         or_tokenize(u[i], m, tok + i, nbits + i, extra + i);
 }
 
-/* split: smallest m in [0, 7] with at least 99% of the context's values below 2^m */
+/* split: smallest m in [0, 7] with at least 99.9% of the context's values below 2^m */
 static int32_t choose_split(const uint64_t *bitlen_hist /* [24]: count by bit length */)
 {
     uint64_t n = 0;
@@ -364,7 +366,7 @@ static int32_t choose_split(const uint64_t *bitlen_hist /* [24]: count by bit le
     uint64_t below = 0;
     for (int32_t m = 0; m <= MAX_SPLIT; m++) {
         below += bitlen_hist[m]; /* values with bit length m are below 2^m */
-        if (below * 100u >= n * 99u)
+        if (below * 1000u >= n * 999u)
             return m;
     }
     return MAX_SPLIT;
@@ -435,17 +437,18 @@ int32_t or_normalize_freqs(const uint64_t *counts, int32_t n, uint32_t *f)
 
 /* ---------------------------------- tiles -------------------------------------------- */
 /* Reading of "independently decodable tiles" ([ABS]): a tile is 32 lanes x K blocks;
- * lane l of tile t owns blocks t*32K + 32k + l, k = 0..K-1.  K is set by the block count
- * alone: K = 16 below 2^20 blocks, else the power of two at or below nb / 2^16, capped
- * at 256, which keeps the tile count near 2048 for mid-sized matrices. */
-uint32_t or_choose_blocks_per_lane(int64_t nb)
+ * lane l of tile t owns blocks t*32K + 32k + l, k = 0..K-1.  K comes from the block count and
+ * the target rate: the power of two at or below nb / 2^16 (at least 16, at most 256), which
+ * keeps mid-sized matrices near 2048 tiles, then halved (down to 1) while the tile's expected
+ * payload, 32 K blocks x 8 coordinates x target bits plus a tenth, exceeds 5952 bytes. */
+uint32_t or_choose_blocks_per_lane(int64_t nb, double target)
 {
     int64_t q = nb / 65536;
-    if (q < 16)
-        return 16;
     uint32_t k = 16;
     while ((int64_t)k * 2 <= q && k < 256)
         k *= 2;
+    while (k > 1 && 32.0 * (double)k * target * 1.1 > TILE_BUDGET)
+        k /= 2;
     return k;
 }
 
@@ -591,8 +594,9 @@ static size_t meta_bytes(int64_t rows, int32_t container, uint64_t total_tokens,
  * 65536)) is quantized at k; its symbols are tokenized with splits chosen on the sample,
  * and the payload is estimated as the sample's empirical conditional entropy of tokens
  * plus its raw extra bits, scaled by nb / n_sample.  Exact metadata is added, the table
- * length taken from the sample, plus 104 bytes per tile: a final state holds about 24 bits
- * that carry no payload (32 lanes x 3 bytes) and a tile pads to 16 bytes (8 on average). */
+ * length taken from the sample, plus 168 bytes per tile: a final state holds about 24 bits
+ * that carry no payload (32 lanes x 3 bytes), the 32 word counts take 64 bytes and a tile
+ * pads to 16 bytes (8 on average). */
 static double estimate_bpp(const double *w, const float *s, int64_t rows, int64_t cols, int32_t container,
                            int32_t k, uint32_t K)
 {
@@ -646,7 +650,7 @@ static double estimate_bpp(const double *w, const float *s, int64_t rows, int64_
     }
     bits += extra;
     uint32_t ntiles = (uint32_t)((nb + (int64_t)LANES * K - 1) / ((int64_t)LANES * K));
-    double bytes = (double)meta_bytes(rows, container, total_tokens, ntiles) + 104.0 * (double)ntiles +
+    double bytes = (double)meta_bytes(rows, container, total_tokens, ntiles) + 168.0 * (double)ntiles +
                    bits * ((double)nb / (double)ns) / 8.0;
     for (int c = 0; c < NCTX; c++)
         free(cnt[c]);
@@ -662,7 +666,7 @@ double or_estimate_bpp(const void *src, int32_t sdt, int64_t rows, int64_t cols,
     float *s = (float *)malloc((size_t)rows * sizeof(float));
     row_rms(w, rows, cols, s);
     if (K == 0)
-        K = or_choose_blocks_per_lane(rows * (cols / 8));
+        K = or_choose_blocks_per_lane(rows * (cols / 8), 4.0);
     double e = estimate_bpp(w, s, rows, cols, container, k, K);
     free(s);
     free(w);
@@ -716,85 +720,79 @@ static void bytes_put(bytes *b, const void *src, size_t n)
     b->n += n;
 }
 
-/* Decode order inside a tile (the interleaving rule both sides follow): for k = 0..K-1,
- * for coordinate i = 0..7: one step in which every lane that owns block t*32K + 32k + l
- * decodes the token of coordinate i; then, for j = 0, 1, ..., one step in which every
- * lane whose token left more than j chunks of extra bits decodes chunk j (chunks of at
- * most 11 bits, least significant first, each a uniform symbol).  After each step the
- * lanes that fell below L read one 16-bit word each, lower lanes first.
- * The encoder runs these events in reverse, emitting words in reverse; the tile stores
- * the final encoder states (= initial decoder states) and the words in decode order. */
+/* Decode order inside a tile (the rule both sides follow): the 32 lanes are independent
+ * rANS coders, each with its own word stream.  Lane l decodes its blocks t*32K + 32k + l in
+ * order of k; per block the 8 coordinates in order; per coordinate its token, then the chunks
+ * of its raw extra bits (at most 11 bits each, least significant first, each a uniform
+ * symbol).  After every symbol the lane reads one 16-bit word from its own stream if its
+ * state fell below L.  The encoder runs a lane's symbols in reverse, emitting words in
+ * reverse.  A tile stores the 32 final encoder states (= initial decoder states, u32), the
+ * 32 word counts (u16), then the word streams of lanes 0..31 one after another, each in the
+ * order the decoder reads it, zero padded to 16 bytes. */
 static void encode_tile(const uint32_t *ctx, const uint32_t *u, int64_t nb, int64_t t, uint32_t K,
                         const int32_t *m, uint32_t *const *freq, uint32_t *const *cum, bytes *out)
 {
     int64_t base = t * (int64_t)LANES * K;
-    size_t cap = (size_t)LANES * K * 8 * 3, ne = 0;
+    size_t cap = (size_t)K * 8 * 3;
     event *ev = (event *)malloc(cap * sizeof(event));
-    for (uint32_t k = 0; k < K; k++) {
-        int64_t b0 = base + (int64_t)k * LANES;
-        if (b0 >= nb)
-            break;
-        for (int i = 0; i < 8; i++) {
-            uint32_t nbits[LANES], extra[LANES];
-            for (int l = 0; l < LANES; l++) {
-                nbits[l] = 0;
-                int64_t b = b0 + l;
-                if (b >= nb)
-                    continue;
-                uint32_t c = ctx[8 * b + i], tok;
-                or_tokenize(u[8 * b + i], m[c], &tok, &nbits[l], &extra[l]);
+    uint16_t *words[LANES];
+    size_t nw[LANES];
+    uint32_t x[LANES];
+    for (int l = 0; l < LANES; l++) {
+        size_t ne = 0;
+        for (uint32_t k = 0; k < K; k++) {
+            int64_t b = base + (int64_t)k * LANES + l;
+            if (b >= nb)
+                break;
+            for (int i = 0; i < 8; i++) {
+                uint32_t c = ctx[8 * b + i], tok, nbits, extra;
+                or_tokenize(u[8 * b + i], m[c], &tok, &nbits, &extra);
                 ev[ne].lane = (uint8_t)l;
                 ev[ne].f = (uint16_t)freq[c][tok];
                 ev[ne].cum = (uint16_t)cum[c][tok];
                 ne++;
-            }
-            for (uint32_t j = 0;; j++) {
-                int any = 0;
-                for (int l = 0; l < LANES; l++) {
-                    if (nbits[l] <= CHUNK_BITS * j)
-                        continue;
-                    uint32_t left = nbits[l] - CHUNK_BITS * j;
+                for (uint32_t j = 0; CHUNK_BITS * j < nbits; j++) {
+                    uint32_t left = nbits - CHUNK_BITS * j;
                     uint32_t bits = left < CHUNK_BITS ? left : CHUNK_BITS;
-                    uint32_t val = (extra[l] >> (CHUNK_BITS * j)) & ((1u << bits) - 1u);
+                    uint32_t val = (extra >> (CHUNK_BITS * j)) & ((1u << bits) - 1u);
                     ev[ne].lane = (uint8_t)l;
                     ev[ne].f = (uint16_t)(1u << (PROB_BITS - bits));
                     ev[ne].cum = (uint16_t)(val << (PROB_BITS - bits));
                     ne++;
-                    any = 1;
                 }
-                if (!any)
-                    break;
             }
         }
-    }
-    uint32_t x[LANES];
-    for (int l = 0; l < LANES; l++)
-        x[l] = STATE_L;
-    uint16_t *words = (uint16_t *)malloc((ne + 1) * sizeof(uint16_t));
-    size_t nw = 0;
-    for (size_t e = ne; e-- > 0;) {
-        uint32_t l = ev[e].lane, f = ev[e].f;
-        uint32_t s = x[l];
-        /* renormalise so that the encoded state stays below 2^32: x_max = (L >> 11) << 16 * f */
-        if ((uint64_t)s >= ((uint64_t)f << 21)) {
-            words[nw++] = (uint16_t)(s & 0xffffu);
-            s >>= 16;
+        words[l] = (uint16_t *)malloc((ne + 1) * sizeof(uint16_t));
+        nw[l] = 0;
+        uint32_t s = STATE_L;
+        for (size_t e = ne; e-- > 0;) {
+            uint32_t f = ev[e].f;
+            /* renormalise so that the encoded state stays below 2^32: x_max = (L >> 11) << 16 * f */
+            if ((uint64_t)s >= ((uint64_t)f << 21)) {
+                words[l][nw[l]++] = (uint16_t)(s & 0xffffu);
+                s >>= 16;
+            }
+            s = ((s / f) << PROB_BITS) + (s % f) + ev[e].cum;
         }
-        x[l] = ((s / f) << PROB_BITS) + (s % f) + ev[e].cum;
+        x[l] = s;
     }
-    uint8_t st[LANES * 4];
-    for (int l = 0; l < LANES; l++)
-        put32(st + 4 * l, x[l]);
-    bytes_put(out, st, sizeof st);
-    for (size_t i = 0; i < nw; i++) {
-        uint8_t w2[2];
-        put16(w2, words[nw - 1 - i]);
-        bytes_put(out, w2, 2);
+    uint8_t head[TILE_HEAD];
+    for (int l = 0; l < LANES; l++) {
+        put32(head + 4 * l, x[l]);
+        put16(head + 4 * LANES + 2 * l, (uint32_t)nw[l]);
+    }
+    bytes_put(out, head, sizeof head);
+    for (int l = 0; l < LANES; l++) {
+        for (size_t i = 0; i < nw[l]; i++) {
+            uint8_t w2[2];
+            put16(w2, words[l][nw[l] - 1 - i]);
+            bytes_put(out, w2, 2);
+        }
+        free(words[l]);
     }
     static const uint8_t zeros[16] = {0};
     size_t pad = al16(out->n) - out->n;
     bytes_put(out, zeros, pad);
-    free(words);
     free(ev);
 }
 
@@ -940,7 +938,7 @@ int or_compress(const void *src, int32_t sdt, int64_t rows, int64_t cols, double
     row_rms(w, rows, cols, s);
     int64_t nb = rows * (cols / 8);
     if (K == 0)
-        K = or_choose_blocks_per_lane(nb);
+        K = or_choose_blocks_per_lane(nb, target);
     int32_t kmax = or_k_max(cols);
     int32_t k;
     if (q_override >= 0) {
@@ -1032,7 +1030,7 @@ int or_parse(const uint8_t *p, size_t n, or_info *info)
     if (get32(d) != 0)
         return OR_ERR_CORRUPT;
     for (int64_t t = 0; t < T; t++)
-        if (get32(d + 4 * (t + 1)) < get32(d + 4 * t) + 8)
+        if (get32(d + 4 * (t + 1)) < get32(d + 4 * t) + TILE_HEAD / 16)
             return OR_ERR_CORRUPT;
     if (info->off_tiles + 16 * (uint64_t)get32(d + 4 * T) != n)
         return OR_ERR_CORRUPT;
@@ -1109,6 +1107,22 @@ typedef struct {
     uint64_t nsym;
 } code_stats;
 
+/* one lane's renormalisation: below L it reads the next word of its own stream */
+static void dec_renorm(uint32_t *x, const uint8_t *wp, uint64_t nwords, uint64_t *pos, uint32_t *status)
+{
+    if (*x >= STATE_L)
+        return;
+    uint32_t wd = 0;
+    if (*pos < nwords)
+        wd = get16(wp + 2 * *pos);
+    else
+        *status |= OR_DEC_WORD_OVERRUN;
+    (*pos)++;
+    *x = (*x << 16) | wd;
+}
+
+/* Decodes tile t lane by lane, each lane an independent coder over its own word stream
+ * (the order written down at encode_tile). */
 static void decode_tile(dec_ctx *D, int64_t t, int32_t *vout, void *out, uint32_t *status, code_stats *cs)
 {
     const or_info *I = &D->in;
@@ -1117,116 +1131,81 @@ static void decode_tile(dec_ctx *D, int64_t t, int32_t *vout, void *out, uint32_
     const uint8_t *dir = D->p + I->off_dir;
     const uint8_t *tp = D->p + I->off_tiles + 16 * (uint64_t)get32(dir + 4 * t);
     uint64_t tile_bytes = 16 * (uint64_t)(get32(dir + 4 * (t + 1)) - get32(dir + 4 * t));
-    uint64_t nwords = (tile_bytes - 4 * LANES) / 2, pos = 0;
-    const uint8_t *wp = tp + 4 * LANES;
-    uint32_t x[LANES];
-    for (int l = 0; l < LANES; l++)
-        x[l] = get32(tp + 4 * l);
+    uint64_t capacity = (tile_bytes - TILE_HEAD) / 2, start = 0;
     int64_t base = t * (int64_t)LANES * K;
     int esz = elt_size(I->container_dtype);
-    for (uint32_t k = 0; k < K; k++) {
-        int64_t b0 = base + (int64_t)k * LANES;
-        if (b0 >= nb)
-            break;
-        int32_t v[LANES][8], y[LANES][8], c[LANES], p[LANES];
-        for (int i = 0; i < 8; i++) {
-            uint32_t tok[LANES], nbits[LANES], extra[LANES], ctx[LANES];
-            /* token step */
-            for (int l = 0; l < LANES; l++) {
-                nbits[l] = 0;
-                extra[l] = 0;
-                if (b0 + l >= nb)
-                    continue;
-                ctx[l] = i == 0 ? 0u : i < 7 ? 1u + (uint32_t)c[l] : 3u + 2u * (uint32_t)c[l] + (uint32_t)p[l];
-                tok[l] = dec_token(D, ctx[l], &x[l], status, cs ? &cs->ideal : NULL);
-                token_bits(tok[l], I->split[ctx[l]], &nbits[l]);
+    for (int l = 0; l < LANES; l++) {
+        uint32_t x = get32(tp + 4 * l);
+        uint64_t nwords = get16(tp + 4 * LANES + 2 * l), pos = 0;
+        const uint8_t *wp = tp + TILE_HEAD + 2 * start;
+        if (start + nwords > capacity) {
+            *status |= OR_DEC_WORD_OVERRUN;
+            nwords = start < capacity ? capacity - start : 0;
+        }
+        start += get16(tp + 4 * LANES + 2 * l);
+        for (uint32_t k = 0; k < K; k++) {
+            int64_t b = base + (int64_t)k * LANES + l;
+            if (b >= nb)
+                break;
+            int32_t v[8], y[8], c = 0, p = 0;
+            for (int i = 0; i < 8; i++) {
+                uint32_t ctx = i == 0 ? 0u : i < 7 ? 1u + (uint32_t)c : 3u + 2u * (uint32_t)c + (uint32_t)p;
+                uint32_t tok = dec_token(D, ctx, &x, status, cs ? &cs->ideal : NULL), nbits, extra = 0;
+                dec_renorm(&x, wp, nwords, &pos, status);
+                token_bits(tok, I->split[ctx], &nbits);
                 if (cs) {
-                    cs->tokcount[ctx[l]][tok[l]]++;
-                    cs->extra += nbits[l];
+                    cs->tokcount[ctx][tok]++;
+                    cs->extra += nbits;
                     cs->nsym++;
                 }
-                if (x[l] < STATE_L) {
-                    uint32_t wd = 0;
-                    if (pos < nwords)
-                        wd = get16(wp + 2 * pos);
-                    else
-                        *status |= OR_DEC_WORD_OVERRUN;
-                    pos++;
-                    x[l] = (x[l] << 16) | wd;
-                }
-            }
-            /* chunk steps */
-            for (uint32_t j = 0;; j++) {
-                int any = 0;
-                for (int l = 0; l < LANES; l++) {
-                    if (nbits[l] <= CHUNK_BITS * j)
-                        continue;
-                    any = 1;
-                    uint32_t left = nbits[l] - CHUNK_BITS * j;
+                for (uint32_t j = 0; CHUNK_BITS * j < nbits; j++) {
+                    uint32_t left = nbits - CHUNK_BITS * j;
                     uint32_t bits = left < CHUNK_BITS ? left : CHUNK_BITS;
                     uint32_t f = 1u << (PROB_BITS - bits);
-                    uint32_t slot = x[l] & (PROB_M - 1);
+                    uint32_t slot = x & (PROB_M - 1);
                     uint32_t val = slot >> (PROB_BITS - bits);
-                    x[l] = f * (x[l] >> PROB_BITS) + slot - val * f;
-                    extra[l] |= val << (CHUNK_BITS * j);
-                    if (x[l] < STATE_L) {
-                        uint32_t wd = 0;
-                        if (pos < nwords)
-                            wd = get16(wp + 2 * pos);
-                        else
-                            *status |= OR_DEC_WORD_OVERRUN;
-                        pos++;
-                        x[l] = (x[l] << 16) | wd;
-                    }
+                    x = f * (x >> PROB_BITS) + slot - val * f;
+                    extra |= val << (CHUNK_BITS * j);
+                    dec_renorm(&x, wp, nwords, &pos, status);
                 }
-                if (!any)
-                    break;
-            }
-            /* inverse symbolization */
-            for (int l = 0; l < LANES; l++) {
-                if (b0 + l >= nb)
-                    continue;
-                uint32_t uu = or_detokenize(tok[l], I->split[ctx[l]], extra[l]);
-                if (tok[l] >= I->ntok[ctx[l]])
+                /* inverse symbolization */
+                uint32_t uu = or_detokenize(tok, I->split[ctx], extra);
+                if (tok >= I->ntok[ctx])
                     *status |= OR_DEC_BAD_TOKEN;
                 if (i == 0) {
-                    v[l][0] = or_unzigzag(uu);
-                    c[l] = (v[l][0] % 2 != 0) ? 1 : 0;
-                    y[l][0] = (v[l][0] - c[l]) / 2;
-                    p[l] = (y[l][0] % 2 != 0) ? 1 : 0;
+                    v[0] = or_unzigzag(uu);
+                    c = (v[0] % 2 != 0) ? 1 : 0;
+                    y[0] = (v[0] - c) / 2;
+                    p = (y[0] % 2 != 0) ? 1 : 0;
                 } else if (i < 7) {
-                    y[l][i] = or_unzigzag(uu);
-                    v[l][i] = 2 * y[l][i] + c[l];
-                    p[l] ^= (y[l][i] % 2 != 0) ? 1 : 0;
+                    y[i] = or_unzigzag(uu);
+                    v[i] = 2 * y[i] + c;
+                    p ^= (y[i] % 2 != 0) ? 1 : 0;
                 } else {
-                    y[l][7] = 2 * or_unzigzag(uu) + p[l];
-                    v[l][7] = 2 * y[l][7] + c[l];
+                    y[7] = 2 * or_unzigzag(uu) + p;
+                    v[7] = 2 * y[7] + c;
                 }
             }
-        }
-        /* reconstruction: w = f_r * v in fp32, then the container conversion */
-        for (int l = 0; l < LANES; l++) {
-            int64_t b = b0 + l;
-            if (b >= nb)
-                continue;
+            /* reconstruction: w = f_r * v in fp32, then the container conversion */
             int64_t r = b / cb;
             uint32_t fb = get32(D->rowf + 4 * r);
             float fr;
             memcpy(&fr, &fb, 4);
             if (vout)
-                memcpy(vout + 8 * b, v[l], 8 * sizeof(int32_t));
+                memcpy(vout + 8 * b, v, 8 * sizeof(int32_t));
             if (out) {
                 float wv[8];
                 for (int i = 0; i < 8; i++)
-                    wv[i] = fr * (float)v[l][i];
+                    wv[i] = fr * (float)v[i];
                 or_convert_batch(wv, 8, I->container_dtype, (uint8_t *)out + (size_t)(8 * b) * (size_t)esz);
             }
         }
-    }
-    for (int l = 0; l < LANES; l++)
-        if (x[l] != STATE_L)
+        if (x != STATE_L)
             *status |= OR_DEC_BAD_END;
-    if (pos > nwords || nwords - pos >= 8)
+        if (pos != nwords)
+            *status |= pos > nwords ? OR_DEC_WORD_OVERRUN : OR_DEC_WORD_COUNT;
+    }
+    if (start > capacity || capacity - start >= 8)
         *status |= OR_DEC_WORD_COUNT;
 }
 
@@ -1275,7 +1254,7 @@ int or_code_stats(const uint8_t *blob, size_t n, double *ideal_bits, double *emp
     const uint8_t *dir = blob + D.in.off_dir;
     uint64_t pb = 0;
     for (uint32_t t = 0; t < D.in.n_tiles; t++)
-        pb += 16 * (uint64_t)(get32(dir + 4 * (t + 1)) - get32(dir + 4 * t)) - 4 * LANES;
+        pb += 16 * (uint64_t)(get32(dir + 4 * (t + 1)) - get32(dir + 4 * t)) - TILE_HEAD;
     *ideal_bits = cs.ideal;
     *emp_entropy_bits = H;
     *extra_bits = cs.extra;

@@ -79,7 +79,7 @@ uint32_t or_detokenize(uint32_t tok, int32_t m, uint32_t extra);
 void or_detokenize_batch(const uint32_t *tok, int64_t n, int32_t m, const uint32_t *extra, uint32_t *u);
 void or_tokenize_batch(const uint32_t *u, int64_t n, int32_t m, uint32_t *tok, uint32_t *nbits, uint32_t *extra);
 int32_t or_normalize_freqs(const uint64_t *counts, int32_t n, uint32_t *freqs);
-uint32_t or_choose_blocks_per_lane(int64_t nblocks);
+uint32_t or_choose_blocks_per_lane(int64_t nblocks, double target_bpp);
 uint16_t or_bf16_from_float(float w);
 uint16_t or_fp16_from_float(float w);
 uint8_t or_e4m3_from_float(float w);
@@ -95,7 +95,8 @@ void or_row_factors(const void *src, int32_t src_dtype, int64_t rows, int64_t co
 /* lattice points v = 2z (int32, rows*cols) at resolution index k */
 int or_quantize(const void *src, int32_t src_dtype, int64_t rows, int64_t cols, int32_t container,
                 int32_t k, int32_t *v);
-/* sampled storage estimate (bits per weight) at resolution index k */
+/* sampled storage estimate (bits per weight) at resolution index k; blocks_per_lane 0 takes
+ * the automatic tile size for a 4 bpp target */
 double or_estimate_bpp(const void *src, int32_t src_dtype, int64_t rows, int64_t cols, int32_t container,
                        int32_t k, uint32_t blocks_per_lane);
 

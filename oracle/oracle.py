@@ -56,7 +56,7 @@ def lib():
         L.or_normalize_freqs.restype = C.c_int32
         L.or_normalize_freqs.argtypes = [p, C.c_int32, p]
         L.or_choose_blocks_per_lane.restype = C.c_uint32
-        L.or_choose_blocks_per_lane.argtypes = [C.c_int64]
+        L.or_choose_blocks_per_lane.argtypes = [C.c_int64, C.c_double]
         L.or_convert_batch.argtypes = [p, C.c_int64, C.c_int32, p]
         L.or_prequant.restype = C.c_int
         L.or_prequant.argtypes = [p, C.c_int32, C.c_int64, C.c_int64, C.c_int32, p, p]
@@ -165,8 +165,8 @@ def normalize_freqs(counts):
     return f, n
 
 
-def blocks_per_lane(nblocks):
-    return lib().or_choose_blocks_per_lane(int(nblocks))
+def blocks_per_lane(nblocks, target_bpp):
+    return lib().or_choose_blocks_per_lane(int(nblocks), float(target_bpp))
 
 
 def convert(w, dtype):

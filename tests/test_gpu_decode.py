@@ -150,3 +150,15 @@ def test_damaged_streams_flagged(oracle):
     B.decompress(d, host_info, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) != 0
+
+
+@pytest.mark.parametrize("K,q", [(64, 900), (256, 760), (128, 1000)])
+def test_tiles_larger_than_staging_buffer(oracle, K, q):
+    """tiles above the kernel's 6 KB per-warp buffer are decoded in place from global memory"""
+    w = synth.gaussian_outliers(96, 4096, seed=K)
+    rc, blob = oracle.compress(w, 11.0, blocks_per_lane=K, q_override=q)
+    assert rc == 0
+    rc, info = oracle.parse(blob)
+    sizes = np.diff(np.frombuffer(blob[info.off_dir: info.off_dir + 4 * (info.n_tiles + 1)].tobytes(), np.uint32))
+    assert (16 * sizes > 6144).any()
+    check_parity(oracle, blob)

@@ -21,8 +21,8 @@ CASES = [
     ("fp32_src", lambda: synth.row_lognormal(128, 1024, 4, dtype=torch.float32), 5.0, 0, 0),
     ("fp32_to_bf16", lambda: synth.row_lognormal(128, 1024, 4, dtype=torch.float32), 5.0, B.BF16, 0),
     ("dit_out_rows", lambda: synth.dit_layer(3, 1)[:512], 2.5, 0, 0),
-    ("K1", lambda: synth.gaussian(40, 256, 0.02, 5), 6.0, 0, 1),
-    ("K5", lambda: synth.gaussian(40, 256, 0.02, 5), 6.0, 0, 5),
+    ("K1", lambda: synth.gaussian(40, 256, 0.02, 5), 11.0, 0, 1),
+    ("K5", lambda: synth.gaussian(40, 256, 0.02, 5), 8.0, 0, 5),
     ("zero_rows", lambda: torch.cat([synth.gaussian(30, 512, 0.02, 6), torch.zeros(2, 512, dtype=torch.bfloat16)]),
      4.0, 0, 0),
 ]

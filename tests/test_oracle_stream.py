@@ -33,7 +33,7 @@ def to_f32(out, container):
 
 
 def tile_states(blob, info):
-    """initial decoder states of every tile (the documented tile layout)"""
+    """initial decoder states of every tile (the documented tile layout: 32 u32 states first)"""
     b = blob.tobytes()
     d0 = info.off_dir
     states = []
@@ -121,7 +121,7 @@ def test_rate_control(oracle, target):
     assert info.actual_bpp == 8.0 * blob.size / w.numel()
     # the search lands close below the target: one grid step is ~0.016 bits per weight
     assert info.actual_bpp >= target - 0.15
-    est = oracle.estimate_bpp(w, info.q_index)
+    est = oracle.estimate_bpp(w, info.q_index, blocks_per_lane=info.blocks_per_lane)
     assert abs(est - info.actual_bpp) < 0.05 + 0.02 * target
 
 
@@ -140,7 +140,7 @@ def test_rate_distortion_closed_form(oracle, target):
 def test_estimate_monotone(oracle):
     w = synth.row_lognormal(128, 1024, seed=9)
     ks = list(range(300, 900, 40))
-    est = [oracle.estimate_bpp(w, k) for k in ks]
+    est = [oracle.estimate_bpp(w, k, blocks_per_lane=16) for k in ks]
     assert all(b > a for a, b in zip(est, est[1:]))
 
 
@@ -164,7 +164,7 @@ def test_code_containers(oracle, container, target):
 
 def test_tiles_independent(oracle):
     w = synth.gaussian(64, 2048, 0.02, seed=12)
-    blob, info, v, out = roundtrip(oracle, w, 3.0, K=2)
+    blob, info, v, out = roundtrip(oracle, w, 6.0, K=2)  # tiny tiles: 2.6 bpp of tile heads
     assert info.n_tiles > 4
     for t0, t1 in [(0, 1), (1, 3), (info.n_tiles - 1, info.n_tiles)]:
         rc, st, v2, out2 = oracle.decode(blob, t0, t1)
@@ -179,7 +179,7 @@ def test_zero_rows(oracle):
     w[5, :8] = 0
     blob, info, v, out = roundtrip(oracle, w, 4.0)
     assert not v[2].any()
-    z = torch.zeros(8, 64, dtype=torch.bfloat16)
+    z = torch.zeros(32, 64, dtype=torch.bfloat16)
     rc, blob = oracle.compress(z, 4.0)
     assert rc == 0
     rc, st, v, out = oracle.decode(blob)

@@ -54,8 +54,17 @@ def test_resolution_grid(oracle):
 
 
 def test_blocks_per_lane_rule(oracle):
-    assert oracle.blocks_per_lane(1) == 16
-    assert oracle.blocks_per_lane(2 ** 20) == 16
-    assert oracle.blocks_per_lane(4096 * 4096 // 8) == 32
-    assert oracle.blocks_per_lane(8192 * 28672 // 8) == 256
-    assert oracle.blocks_per_lane(10 ** 12) == 256
+    """tiles near 2048 for mid-size matrices, at most 256 blocks per lane, and a tile's
+    expected payload (32 K x 8 coordinates x target bits, +10%) within 5952 bytes"""
+    assert oracle.blocks_per_lane(1, 4.0) == 16
+    assert oracle.blocks_per_lane(2 ** 20, 4.0) == 16
+    assert oracle.blocks_per_lane(4096 * 4096 // 8, 4.0) == 32
+    assert oracle.blocks_per_lane(8192 * 28672 // 8, 0.5) == 256
+    assert oracle.blocks_per_lane(8192 * 28672 // 8, 4.0) == 32
+    assert oracle.blocks_per_lane(8192 * 28672 // 8, 8.0) == 16
+    assert oracle.blocks_per_lane(10 ** 12, 11.0) == 8
+    for nb in (10, 10 ** 5, 10 ** 7, 10 ** 9):
+        for t in (0.001, 0.5, 2.0, 4.0, 8.0, 11.0):
+            k = oracle.blocks_per_lane(nb, t)
+            assert k & (k - 1) == 0 and 1 <= k <= 256
+            assert k == 1 or 32 * k * t * 1.1 <= 5952
