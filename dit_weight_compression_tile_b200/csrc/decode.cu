@@ -167,9 +167,6 @@ struct Packer<EP_LATTICE_I32> {
 __device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void *gsrc) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_dst), "l"(gsrc) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit_wait_all() {
-    asm volatile("cp.async.commit_group;\ncp.async.wait_all;\n" ::: "memory");
-}
 
 // ------------------------------------------------------------------ a lane's word stream
 // The tile's words live either in the warp's shared-memory buffer (SMEM) or, for a tile larger
@@ -198,6 +195,7 @@ struct Lane {
     uint32_t x;     // rANS state
     uint32_t idx;   // index (in the tile's word area) of the next word this lane would read
     uint32_t last;  // last word index of the tile
+    uint32_t w;     // that word, fetched as soon as the previous one was consumed
 };
 
 __device__ __forceinline__ int32_t unzigzag(uint32_t u) { return int32_t(u >> 1) ^ -int32_t(u & 1u); }
@@ -210,15 +208,14 @@ __device__ __forceinline__ int32_t unzigzag(uint32_t u) { return int32_t(u >> 1)
 template <bool SMEM, bool ACT>
 __device__ __forceinline__ int32_t step(Lane &s, bool act, const uint32_t *lut, const uint32_t *tinfo,
                                         const Words<SMEM> &W) {
-    uint32_t w = W.at(min(s.idx, s.last));
     uint32_t e = lut[s.x & (kProbScale - 1)];
     uint32_t x = (e >> 20) * (s.x >> kProbBits) + (e & 0x7ffu);
-    bool need = x < kStateLow;
-    x = need ? __byte_perm(w, x, 0x5410) : x;  // (x << 16) | w for x < 2^16
-    if (!ACT || act) {
-        s.x = x;
-        s.idx += need ? 1u : 0u;
+    bool need = x < kStateLow && (!ACT || act);
+    if (need) {
+        x = __byte_perm(s.w, x, 0x5410);  // (x << 16) | w for x < 2^16
+        s.w = W.at(min(++s.idx, s.last));
     }
+    if (!ACT || act) s.x = x;
     int32_t val = int32_t(e << 13) >> 24;  // bits [11, 19): the signed value of a direct token
     bool esc = (e & kEsc) && (!ACT || act);
     if (__any_sync(0xffffffffu, esc)) {
@@ -226,18 +223,17 @@ __device__ __forceinline__ int32_t step(Lane &s, bool act, const uint32_t *lut, 
         uint32_t u = ti >> 5, nbits = ti & 31u, shift = 0;
 #pragma unroll 1
         for (int j = 0; j < 2 && __any_sync(0xffffffffu, nbits != 0); ++j) {
-            bool a = nbits != 0;
-            uint32_t bits = nbits < kChunkBits ? nbits : kChunkBits;
-            uint32_t keep = kProbBits - bits;
-            uint32_t slot = s.x & (kProbScale - 1);
-            uint32_t xc = ((s.x >> kProbBits) << keep) | (slot & ((1u << keep) - 1u));
-            uint32_t wc = W.at(min(s.idx, s.last));
-            bool nd = xc < kStateLow;
-            xc = nd ? __byte_perm(wc, xc, 0x5410) : xc;
-            if (a) {
+            if (nbits != 0) {
+                uint32_t bits = nbits < kChunkBits ? nbits : kChunkBits;
+                uint32_t keep = kProbBits - bits;
+                uint32_t slot = s.x & (kProbScale - 1);
+                uint32_t xc = ((s.x >> kProbBits) << keep) | (slot & ((1u << keep) - 1u));
+                if (xc < kStateLow) {
+                    xc = __byte_perm(s.w, xc, 0x5410);
+                    s.w = W.at(min(++s.idx, s.last));
+                }
                 u |= (slot >> keep) << shift;
                 s.x = xc;
-                s.idx += nd ? 1u : 0u;
                 shift += bits;
                 nbits -= bits;
             }
@@ -317,6 +313,7 @@ __device__ __forceinline__ uint32_t decode_tile(const Params &p, const uint32_t 
     uint32_t start = incl - n;
     s.idx = start;
     s.last = capacity ? capacity - 1u : 0u;
+    s.w = W.at(min(s.idx, s.last));
     if (uint64_t(t + 1) * 32u * p.K <= p.nb)
         decode_blocks<DT, SMEM, false>(p, s, lut, tinfo, W, t, lane);
     else
@@ -338,6 +335,20 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_
     uint32_t *tinfo = smem + kLutEntries;                            // [ctx][token]
     uint32_t *cum = tinfo + kContexts * 256;                         // [ctx][257]
     uint8_t *buf = reinterpret_cast<uint8_t *>(smem) + kFixedBytes + size_t(warp) * p.tile_buf;
+
+    // ---- this warp's first tile starts loading now, behind the table set-up
+    uint32_t t_begin = uint32_t(uint64_t(blockIdx.x) * p.T / gridDim.x);
+    uint32_t t_end = uint32_t(uint64_t(blockIdx.x + 1) * p.T / gridDim.x);
+    const uint32_t buf_s = static_cast<uint32_t>(__cvta_generic_to_shared(buf));
+    auto stage = [&](uint32_t t) {  // tile t into the buffer if it is valid and fits; no wait
+        uint32_t beg = __ldg(p.dir + t), end = __ldg(p.dir + t + 1);
+        if (end >= beg + uint32_t(kTileHead / 16) && uint64_t(end) <= p.tile_units && (end - beg) * 16u <= p.tile_buf) {
+            const uint8_t *tp = p.tiles + size_t(beg) * 16;
+            for (uint32_t i = lane; i < end - beg; i += 32u) cp_async16(buf_s + 16u * i, tp + 16u * i);
+        }
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+    };
+    if (t_begin + warp < t_end) stage(t_begin + warp);
 
     // ---- tables.  Every slot starts as an escape to token 255 with f = 2^11 and bias = slot
     // (an identity step that decodes nothing: a damaged stream then fails its end checks);
@@ -391,10 +402,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_
     __syncthreads();
 
     // ---- tiles of this CTA: a contiguous range, warps round robin
-    uint32_t t_begin = uint32_t(uint64_t(blockIdx.x) * p.T / gridDim.x);
-    uint32_t t_end = uint32_t(uint64_t(blockIdx.x + 1) * p.T / gridDim.x);
-    const uint32_t buf_s = static_cast<uint32_t>(__cvta_generic_to_shared(buf));
     for (uint32_t t = t_begin + warp; t < t_end; t += nwarps) {
+        if (t != t_begin + warp) {
+            __syncwarp();  // the previous tile's reads of the buffer are done
+            stage(t);
+        }
         uint32_t beg = __ldg(p.dir + t), end = __ldg(p.dir + t + 1);
         uint32_t err;
         if (end < beg + uint32_t(kTileHead / 16) || uint64_t(end) > p.tile_units) {
@@ -403,9 +415,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_
             const uint8_t *tp = p.tiles + size_t(beg) * 16;
             uint32_t tile_bytes = (end - beg) * 16u;
             if (tile_bytes <= p.tile_buf) {
-                __syncwarp();  // the previous tile's reads of the buffer are done
-                for (uint32_t i = lane; i < tile_bytes / 16u; i += 32u) cp_async16(buf_s + 16u * i, tp + 16u * i);
-                cp_async_commit_wait_all();
+                asm volatile("cp.async.wait_all;\n" ::: "memory");
                 __syncwarp();
                 Words<true> W{buf_s + uint32_t(kTileHead)};
                 err = decode_tile<DT, true>(p, lut, tinfo, buf, W, tile_bytes, t, lane);
