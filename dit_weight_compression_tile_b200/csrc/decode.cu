@@ -1,20 +1,26 @@
 // Fused tile decode for sm_100a: ep_decompress.
 //
-// "The final coordinates are entropy-coded in independently decodable tiles, enabling fast,
-// fused symbol decoding and numerical weight reconstruction on the GPU" ("EntroPack: Fast and
-// Accurate Entropy-Coded Weight Compression at Arbitrary Bitrates", Abstract).  One kernel:
-//   * each CTA turns the stream's frequency tables into seven 2048-slot tables in shared
-//     memory; a slot's 32-bit entry holds the symbol's frequency, the slot's offset inside the
-//     symbol, an escape flag and, for direct tokens, the decoded signed coordinate value;
-//   * each warp decodes whole tiles: the tile is staged into the warp's shared-memory buffer
-//     with 16-byte async copies, and lane l runs the rANS coder of lane l over its own word
-//     stream, so a step needs no warp-wide exchange and its word address is known before the
-//     state update that decides whether to consume it;
-//   * the 8 coordinates of a lane's block are rebuilt in registers (coset from coordinate 0,
-//     parity-forced coordinate 7), scaled by the row factor with one fp32 multiply and
-//     converted to the container (BF16 / FP16 / FP32 / INT8 / FP8-E4M3) with round to nearest
-//     even; a warp writes 32 consecutive blocks with one 16-byte (8-byte for codes) store per
-//     lane.
+// The pages' pipeline ends in entropy coding "in independently decodable tiles" with "fused
+// symbol decoding and numerical weight reconstruction on the GPU" ("EntroPack: Fast and
+// Accurate Entropy-Coded Weight Compression at Arbitrary Bitrates", Abstract).  One kernel, one
+// CTA per SM:
+//   * prologue: the frequency tables reach shared memory with one bulk (TMA) copy; the CTA turns
+//     them into seven 2048-slot tables.  A slot's 32-bit entry holds the token's frequency
+//     (11 bits), the slot's offset inside the token (11 bits), an escape flag and, for a
+//     direct token, the lattice coordinate v + 256 (9 bits);
+//   * each warp decodes whole tiles.  A tile (32 initial states, 32 word counts, the lanes'
+//     16-bit word streams, the raw extra bits) is brought into the warp's shared-memory buffer
+//     by one bulk copy completing on an mbarrier, two tiles in flight per warp.  Lane l runs the
+//     rANS coder of lane l over its own word stream, so a step is a table lookup, a
+//     multiply-add and a predicated word read, with no warp-wide exchange;
+//   * the coset c and the parity of y0..y6 that pick the contexts of coordinates 1..7 are bits
+//     of the table entries, so a block's 8 tokens decode without a branch; the rare escape
+//     tokens (at most a few per thousand) are resolved after the block from the tile's raw bit
+//     stream;
+//   * reconstruction stays in registers: the entry's value field becomes an exact float with
+//     one logic op and one fused multiply-add, w = fp32(f_r * v) is one multiply, and the
+//     container conversion rounds to nearest even; a warp stores 32 consecutive blocks with
+//     one 16-byte (BF16 / FP16) or 8-byte (INT8 / FP8) store per lane.
 // The path is a scan over compressed bytes, bound by HBM bandwidth and instruction issue; it
 // uses no tensor cores because nothing in it is a dense contraction.
 #include <cuda_bf16.h>
@@ -31,24 +37,33 @@ namespace ep {
 namespace {
 
 constexpr int kMaxWarps = 32;
-constexpr uint32_t kLutEntries = kContexts * kProbScale;
-constexpr uint32_t kTileBufMax = 16384;  // largest per-warp tile buffer; larger tiles are read in place
-constexpr size_t kSmemLimit = 232448;    // shared memory one CTA may use on sm_100
-constexpr size_t kLutBytes = size_t(kLutEntries) * 4;
-constexpr size_t kTinfoBytes = size_t(kContexts) * 256 * 4;
-constexpr size_t kCumBytes = (size_t(kContexts) * 257 * 4 + 15) & ~size_t(15);  // keeps the tile buffers 16-byte aligned
-constexpr size_t kFixedBytes = kLutBytes + kTinfoBytes + kCumBytes;
+constexpr uint32_t kSlotBytes = kProbScale * 4;                   // one context's slot table
+constexpr size_t kLutBytes = size_t(kContexts) * kSlotBytes;      // 56 KB
+constexpr uint32_t kCumStride = kMaxAlphabet + 8;                 // u16 per context (freqs, then their prefix sums)
+constexpr size_t kCumBytes = (size_t(kContexts) * kCumStride * 2 + 15) & ~size_t(15);
+constexpr uint32_t kSegs = kProbScale / 32;                       // 32-slot segments per context
+constexpr size_t kSegBytes = (size_t(kContexts) * kSegs * 2 + 15) & ~size_t(15);
+constexpr size_t kBarBytes = size_t(kMaxWarps) * 2 * 8 + 16;      // two mbarriers per warp + one for the tables
+constexpr size_t kFixedBytes = kLutBytes + kCumBytes + kSegBytes + kBarBytes;
+constexpr uint32_t kSlack = 64;       // bytes past a tile that a lane's bounded over-read may touch
+constexpr size_t kSmemLimit = 232448; // shared memory one CTA may use on sm_100
+constexpr uint32_t kWaitLimit = 1u << 22;  // mbarrier polls before a copy is declared lost
 static_assert(kFixedBytes % 16 == 0, "tile buffers must start 16-byte aligned");
-constexpr size_t smem_bytes(uint32_t warps, uint32_t tile_buf) { return kFixedBytes + size_t(warps) * tile_buf; }
 
-// slot entry: bias [0,11) | value or token [11,19) | escape [19] | frequency [20,32)
-constexpr uint32_t kEsc = 1u << 19;
+// slot entry: bias [0,11) | value field [11,20) | escape [20] | frequency [21,32)
+constexpr uint32_t kEscBit = 1u << 20;
+constexpr uint32_t kFieldMask = 0x1ffu << 11;
+// a direct token's entry becomes the float 2^34 + (v + 256) 2^22 with one OR; one FMA with
+// 2^-22 and -(2^12 + 256) then gives v exactly
+constexpr uint32_t kMagic = 0x50800000u;
+constexpr float kInvScale = 1.0f / 4194304.0f;
+constexpr float kBias = 4352.0f;
 
 struct Params {
     const uint32_t *dir;     // tile directory, 16-byte units (T + 1 entries)
     const uint8_t *tiles;    // tile section
     const float *rowf;       // per-row factors f_r
-    const uint16_t *freq;    // frequency tables, contexts in order
+    const uint8_t *freq;     // frequency tables (u16), contexts in order; 16-byte aligned
     void *out;               // container, row-major
     uint32_t *status;        // nullable
     uint64_t tile_units;     // size of the tile section in 16-byte units
@@ -56,22 +71,76 @@ struct Params {
     uint32_t cb;             // blocks per row
     uint32_t K;              // blocks per lane
     uint32_t T;              // tiles
-    uint32_t tile_buf;       // bytes of each warp's tile buffer (multiple of 16)
-    uint32_t splits;         // 3 bits per context
+    uint32_t tile_buf;       // bytes of each tile buffer (multiple of 16, includes kSlack)
+    uint32_t nbuf;           // tile buffers per warp (1 or 2); 0: tiles are read from global memory
+    uint32_t freq_bytes;     // bytes of the frequency section to stage (multiple of 16)
+    uint32_t splits;         // 4 bits per context
     uint32_t tab_off[kContexts + 1];  // table start of each context (prefix sum of ntok)
 };
 
+__device__ __forceinline__ uint32_t split_of(const Params &p, uint32_t c) { return (p.splits >> (4 * c)) & 15u; }
+
+__device__ __forceinline__ int32_t unzigzag(uint32_t u) { return int32_t(u >> 1) ^ -int32_t(u & 1u); }
+
+// ------------------------------------------------------------------ shared memory, mbarriers, bulk copies
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void sts32(uint32_t a, uint32_t v) { asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v)); }
+__device__ __forceinline__ void sts16(uint32_t a, uint32_t v) { asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "r"(v)); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+// the issuing thread's arrival, announcing the bytes the copy will deliver
+__device__ __forceinline__ void mbar_expect(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// bounded wait for a phase; false when the limit ran out
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kWaitLimit; ++i)
+        if (mbar_try(bar, parity)) return true;
+    return false;
+}
+// one bulk copy global -> this CTA's shared memory, completing on an mbarrier (TMA, no tensor map)
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+// orders this thread's earlier generic-proxy accesses of shared memory before later async-proxy ones
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // ------------------------------------------------------------------ containers
+// put(i, v, fr): coordinate i of the block, v the exact lattice value as a float, fr the row
+// factor; the weight is fp32(fr * v), one correctly rounded multiply.
 template <int DT>
 struct Packer;
 
-__device__ __forceinline__ float reconstruct(int32_t v, float fr) { return __fmul_rn(fr, __int2float_rn(v)); }
+__device__ __forceinline__ float reconstruct(float v, float fr) { return __fmul_rn(fr, v); }
 
 template <>
 struct Packer<EP_BF16> {
     uint32_t o[4];
     float lo;
-    __device__ __forceinline__ void put(int i, int32_t v, float fr) {
+    __device__ __forceinline__ void put(int i, float v, float fr) {
         float w = reconstruct(v, fr);
         if (i & 1) {
             __nv_bfloat162 h = __floats2bfloat162_rn(lo, w);
@@ -89,7 +158,7 @@ template <>
 struct Packer<EP_FP16> {
     uint32_t o[4];
     float lo;
-    __device__ __forceinline__ void put(int i, int32_t v, float fr) {
+    __device__ __forceinline__ void put(int i, float v, float fr) {
         float w = reconstruct(v, fr);
         if (i & 1) {
             __half2 h = __floats2half2_rn(lo, w);
@@ -106,7 +175,7 @@ struct Packer<EP_FP16> {
 template <>
 struct Packer<EP_FP32> {
     float o[8];
-    __device__ __forceinline__ void put(int i, int32_t v, float fr) { o[i] = reconstruct(v, fr); }
+    __device__ __forceinline__ void put(int i, float v, float fr) { o[i] = reconstruct(v, fr); }
     __device__ __forceinline__ void store(void *out, uint32_t b) {
         float4 *p = reinterpret_cast<float4 *>(out) + 2 * size_t(b);
         p[0] = make_float4(o[0], o[1], o[2], o[3]);
@@ -117,7 +186,7 @@ struct Packer<EP_FP32> {
 template <>
 struct Packer<EP_INT8> {
     uint32_t o[2];
-    __device__ __forceinline__ void put(int i, int32_t v, float fr) {
+    __device__ __forceinline__ void put(int i, float v, float fr) {
         int q = min(127, max(-127, __float2int_rn(reconstruct(v, fr))));
         uint32_t byte = uint32_t(q) & 0xffu;
         if ((i & 3) == 0)
@@ -134,7 +203,7 @@ template <>
 struct Packer<EP_FP8_E4M3> {
     uint32_t o[2];
     float lo;
-    __device__ __forceinline__ void put(int i, int32_t v, float fr) {
+    __device__ __forceinline__ void put(int i, float v, float fr) {
         float w = reconstruct(v, fr);
         if (i & 1) {
             uint32_t pair = __nv_cvt_float2_to_fp8x2(make_float2(lo, w), __NV_SATFINITE, __NV_E4M3);
@@ -155,7 +224,7 @@ struct Packer<EP_FP8_E4M3> {
 template <>
 struct Packer<EP_LATTICE_I32> {
     int32_t o[8];
-    __device__ __forceinline__ void put(int i, int32_t v, float) { o[i] = v; }
+    __device__ __forceinline__ void put(int i, float v, float) { o[i] = __float2int_rn(v); }
     __device__ __forceinline__ void store(void *out, uint32_t b) {
         int4 *p = reinterpret_cast<int4 *>(out) + 2 * size_t(b);
         p[0] = make_int4(o[0], o[1], o[2], o[3]);
@@ -163,145 +232,177 @@ struct Packer<EP_LATTICE_I32> {
     }
 };
 
-// ------------------------------------------------------------------ async copies (16 B per lane)
-__device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void *gsrc) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_dst), "l"(gsrc) : "memory");
+// ------------------------------------------------------------------ a lane's words
+// The tile's word area sits either in the warp's shared-memory buffer (SMEM) or, for a tile
+// larger than any buffer, in global memory.  A lane keeps its state x, the next word w of its
+// region (read ahead) and that word's address.  Raw extra bits are read from the back of the
+// region.  Every address stays inside the buffer (shared memory: tile + slack) or the tile
+// (global memory), whatever the stream holds.
+template <bool SMEM>
+struct Lane;
+
+template <>
+struct Lane<true> {
+    uint32_t x, w;
+    uint32_t wp;      // shared address of w
+    uint32_t area;    // shared address of word 0 of the tile's word area
+    uint32_t end;     // index one past the lane's region
+    __device__ __forceinline__ void advance() {
+        wp += 2;
+        w = lds16(wp);
+    }
+    __device__ __forceinline__ bool past(uint32_t lim) const { return wp > lim; }
+    __device__ __forceinline__ uint32_t word(int32_t i) const { return lds16(area + 2u * uint32_t(i)); }
+    __device__ __forceinline__ uint32_t consumed(uint32_t start) const { return (wp - area) / 2u - start; }
+};
+
+template <>
+struct Lane<false> {
+    uint32_t x, w;
+    const uint16_t *wp, *wlim;  // w's address; the last word this lane may touch
+    const uint16_t *area;
+    uint32_t end;
+    __device__ __forceinline__ void advance() {
+        wp = wp < wlim ? wp + 1 : wp;
+        w = __ldg(wp);
+    }
+    // reads here are clamped to the tile one by one, so no block-level stop is needed
+    __device__ __forceinline__ bool past(const uint16_t *) const { return false; }
+    __device__ __forceinline__ uint32_t word(int32_t i) const { return __ldg(area + i); }
+    __device__ __forceinline__ uint32_t consumed(uint32_t start) const { return uint32_t(wp - area) - start; }
+};
+
+// One token of one lane: a lookup in the context's slot table and the rANS update
+// x' = f (x >> 11) + (slot - cum); below 2^16 the state takes the next word of the region.
+template <bool SMEM, bool ACT>
+__device__ __forceinline__ uint32_t step(Lane<SMEM> &L, bool act, uint32_t lut) {
+    if (ACT && !act) return 0u;
+    uint32_t e = lds32(lut + ((L.x & (kProbScale - 1u)) << 2));
+    uint32_t xn = (e >> 21) * (L.x >> kProbBits) + (e & (kProbScale - 1u));
+    if (xn < kStateLow) {
+        xn = (xn << 16) | L.w;
+        L.advance();
+    }
+    L.x = xn;
+    return e;
 }
 
-// ------------------------------------------------------------------ a lane's word stream
-// The tile's words live either in the warp's shared-memory buffer (SMEM) or, for a tile larger
-// than the buffer, in global memory.  Indices are clamped to the tile's last word, so a damaged
-// stream can only read inside its own tile.
+// `nbits` raw bits at raw-bit position rb of the lane (the region's last word holds bits
+// 0..15), least significant first; nbits <= 24
 template <bool SMEM>
-struct Words;
+__device__ __forceinline__ uint32_t raw_bits(const Lane<SMEM> &L, uint32_t rb, uint32_t nbits) {
+    int32_t j = int32_t(L.end) - 1 - int32_t(rb >> 4);
+    int32_t lo = SMEM ? -3 : -int32_t(kTileHead / 2);  // stays inside the buffer / the tile
+    uint32_t w0 = L.word(max(j, lo)), w1 = L.word(max(j - 1, lo)), w2 = L.word(max(j - 2, lo));
+    uint64_t win = uint64_t(w0) | (uint64_t(w1) << 16) | (uint64_t(w2) << 32);
+    return uint32_t(win >> (rb & 15u)) & ((1u << nbits) - 1u);
+}
 
-template <>
-struct Words<true> {
-    uint32_t base;  // shared-memory address of word 0
-    __device__ __forceinline__ uint32_t at(uint32_t i) const {
-        uint32_t w;
-        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(w) : "r"(base + 2u * i));
-        return w;
-    }
-};
-
-template <>
-struct Words<false> {
-    const uint16_t *base;
-    __device__ __forceinline__ uint32_t at(uint32_t i) const { return __ldg(base + i); }
-};
-
-struct Lane {
-    uint32_t x;     // rANS state
-    uint32_t idx;   // index (in the tile's word area) of the next word this lane would read
-    uint32_t last;  // last word index of the tile
-    uint32_t w;     // that word, fetched as soon as the previous one was consumed
-};
-
-__device__ __forceinline__ int32_t unzigzag(uint32_t u) { return int32_t(u >> 1) ^ -int32_t(u & 1u); }
-
-// One coordinate of one lane: a rANS step through the context's slot table.  The word the
-// lane would read is fetched before the state update so the load overlaps the table lookup.
-// An escape token (rare: the token split keeps 99.9% of values direct) is followed by chunks of
-// raw extra bits, at most 11 bits each, least significant first, each a uniform symbol taking
-// the top bits of the slot; the warp runs them together, masked per lane.
-template <bool SMEM, bool ACT>
-__device__ __forceinline__ int32_t step(Lane &s, bool act, const uint32_t *lut, const uint32_t *tinfo,
-                                        const Words<SMEM> &W) {
-    uint32_t e = lut[s.x & (kProbScale - 1)];
-    uint32_t x = (e >> 20) * (s.x >> kProbBits) + (e & 0x7ffu);
-    bool need = x < kStateLow && (!ACT || act);
-    if (need) {
-        x = __byte_perm(s.w, x, 0x5410);  // (x << 16) | w for x < 2^16
-        s.w = W.at(min(++s.idx, s.last));
-    }
-    if (!ACT || act) s.x = x;
-    int32_t val = int32_t(e << 13) >> 24;  // bits [11, 19): the signed value of a direct token
-    bool esc = (e & kEsc) && (!ACT || act);
-    if (__any_sync(0xffffffffu, esc)) {
-        uint32_t ti = esc ? tinfo[(e >> 11) & 0xffu] : 0u;  // (value base << 5) | raw extra bits
-        uint32_t u = ti >> 5, nbits = ti & 31u, shift = 0;
-#pragma unroll 1
-        for (int j = 0; j < 2 && __any_sync(0xffffffffu, nbits != 0); ++j) {
-            if (nbits != 0) {
-                uint32_t bits = nbits < kChunkBits ? nbits : kChunkBits;
-                uint32_t keep = kProbBits - bits;
-                uint32_t slot = s.x & (kProbScale - 1);
-                uint32_t xc = ((s.x >> kProbBits) << keep) | (slot & ((1u << keep) - 1u));
-                if (xc < kStateLow) {
-                    xc = __byte_perm(s.w, xc, 0x5410);
-                    s.w = W.at(min(++s.idx, s.last));
-                }
-                u |= (slot >> keep) << shift;
-                s.x = xc;
-                shift += bits;
-                nbits -= bits;
+// Escape tokens of a block (the warp has at least one).  Token layout (split m, `low` kept
+// bits, 2 bits below the leading one): d = token - 2^m = ((n - m) << 2 | top) << low | lo; the
+// value is s = (4 | top) << (n - 2) | extra << low | lo with n - 2 - low raw extra bits.
+template <bool SMEM>
+__device__ __forceinline__ void resolve_escapes(const Params &p, const uint32_t (&e)[8], uint32_t (&F)[8],
+                                                uint32_t c, uint32_t par, Lane<SMEM> &L, uint32_t &rb) {
+    uint32_t lm = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) lm |= ((e[i] >> 20) & 1u) << i;
+    uint32_t M = __reduce_or_sync(0xffffffffu, lm);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        if (M & (1u << i)) {
+            if (lm & (1u << i)) {
+                uint32_t ctx = i == 0 ? 0u : (i < 7 ? 1u + c : 3u + 2u * c + par);
+                uint32_t low = i == 0 ? 2u : (i < 7 ? 1u : 0u);
+                uint32_t m = split_of(p, ctx);
+                uint32_t fld = (e[i] >> 11) & 0x1ffu;
+                uint32_t d = (i >= 1 && i <= 6) ? fld >> 1 : fld;
+                uint32_t q = d >> low;
+                uint32_t n = min(m + (q >> 2), kValueBits - 1u);
+                uint32_t nbits = n - 2u - low;
+                uint32_t extra = raw_bits(L, rb, nbits);
+                rb += nbits;
+                uint32_t s = ((4u | (q & 3u)) << (n - 2u)) | (extra << low) | (d & ((1u << low) - 1u));
+                int32_t v;
+                if (i == 0)
+                    v = 4 * unzigzag(s >> 2) + int32_t(s & 3u);
+                else if (i < 7)
+                    v = 2 * (2 * unzigzag(s >> 1) + int32_t(s & 1u)) + int32_t(c);
+                else
+                    v = 2 * (2 * unzigzag(s) + int32_t(par)) + int32_t(c);
+                F[i] = __float_as_uint(__int2float_rn(v + 4352) * 4194304.0f);
             }
         }
-        if (esc) val = unzigzag(u);
     }
-    return val;
 }
 
-// ------------------------------------------------------------------ one tile
-template <int DT, bool SMEM, bool ACT>
-__device__ __forceinline__ void decode_blocks(const Params &p, Lane &s, const uint32_t *lut, const uint32_t *tinfo,
-                                              const Words<SMEM> &W, uint32_t t, uint32_t lane) {
+// ------------------------------------------------------------------ the blocks of one tile
+// Lane l decodes blocks t*32K + 32k + l, k = 0..K-1.  ACT: the last tile, where lanes run out
+// of blocks.  Returns EP_DEC_* bits.
+template <int DT, bool SMEM, bool ACT, typename Lim>
+__device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L, uint32_t &rb, uint32_t lut,
+                                                  Lim wlim, uint32_t t, uint32_t lane) {
     uint32_t b = t * 32u * p.K + lane;
     uint32_t row = b / p.cb, col = b - row * p.cb;
-    float fr = b < p.nb ? __ldg(p.rowf + row) : 0.0f;  // row factor, loaded one block ahead
+    float fr = (!ACT || b < p.nb) ? __ldg(p.rowf + row) : 0.0f;
+    uint32_t err = 0;
     for (uint32_t k = 0; k < p.K; ++k, b += 32u) {
-        if (ACT && b - lane >= p.nb) break;
         bool act = !ACT || b < p.nb;
+        if (ACT && !__any_sync(0xffffffffu, act)) break;
+        // a damaged stream may drive a lane's reads ahead; stop before they leave the buffer
+        if (__any_sync(0xffffffffu, L.past(wlim))) {
+            err |= EP_DEC_WORD_OVERRUN;
+            break;
+        }
         uint32_t col_n = col + 32u, row_n = row;
         while (col_n >= p.cb) {
             col_n -= p.cb;
             ++row_n;
         }
         float fr_n = (k + 1 < p.K && b + 32u < p.nb) ? __ldg(p.rowf + row_n) : 0.0f;
-        Packer<DT> pk;
-        // coordinate 0 carries the coset c = v0 mod 2; y0 = floor(v0 / 2)
-        int32_t v = step<SMEM, ACT>(s, act, lut, tinfo, W);
-        int32_t c = v & 1;
-        int32_t par = v >> 1;
-        pk.put(0, v, fr);
-        const uint32_t *lb = lut + (1u + uint32_t(c)) * kProbScale;
-        const uint32_t *tb = tinfo + (1u + uint32_t(c)) * 256u;
+        uint32_t e[8];
+        // coordinate 0 (context 0) carries the coset c in bit 11 of its entry
+        e[0] = step<SMEM, ACT>(L, act, lut);
+        uint32_t lutc = lut + kSlotBytes + ((e[0] & 0x800u) << 2);  // context 1 + c
 #pragma unroll
-        for (int i = 1; i < 7; ++i) {
-            int32_t y = step<SMEM, ACT>(s, act, lb, tb, W);
-            par ^= y;
-            pk.put(i, 2 * y + c, fr);
-        }
-        // coordinate 7: E8 forces y7 = y0 + ... + y6 (mod 2)
-        par &= 1;
-        uint32_t c7 = 3u + 2u * uint32_t(c) + uint32_t(par);
-        int32_t t7 = step<SMEM, ACT>(s, act, lut + c7 * kProbScale, tinfo + c7 * 256u, W);
-        pk.put(7, 2 * (2 * t7 + par) + c, fr);
+        for (int i = 1; i < 7; ++i) e[i] = step<SMEM, ACT>(L, act, lutc);
+        // bit 12 of an entry is the parity of y_i: coordinate 7 takes context 3 + 2c + p
+        uint32_t X = e[0] ^ e[1] ^ e[2] ^ e[3] ^ e[4] ^ e[5] ^ e[6];
+        uint32_t lut7 = lut + 3u * kSlotBytes + ((e[0] & 0x800u) << 3) + ((X & 0x1000u) << 1);
+        e[7] = step<SMEM, ACT>(L, act, lut7);
+        uint32_t F[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) F[i] = (e[i] & kFieldMask) | kMagic;
+        uint32_t O = e[0] | e[1] | e[2] | e[3] | e[4] | e[5] | e[6] | e[7];
+        if (__any_sync(0xffffffffu, O & kEscBit))
+            resolve_escapes<SMEM>(p, e, F, (e[0] >> 11) & 1u, (X >> 12) & 1u, L, rb);
+        Packer<DT> pk;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pk.put(i, __fmaf_rn(__uint_as_float(F[i]), kInvScale, -kBias), fr);
         if (act) pk.store(p.out, b);
         col = col_n;
         row = row_n;
         fr = fr_n;
     }
+    return err;
 }
 
-// Decodes tile t with one warp.  Returns the EP_DEC_* bits of this lane.
-template <int DT, bool SMEM>
-__device__ __forceinline__ uint32_t decode_tile(const Params &p, const uint32_t *lut, const uint32_t *tinfo,
-                                                const uint8_t *head, const Words<SMEM> &W, uint32_t tile_bytes,
+// Decodes tile t with one warp.  `head` points at the tile (states, region lengths, word area):
+// a shared address (SMEM) or a global pointer.  Returns the EP_DEC_* bits of this lane.
+template <int DT, bool SMEM, typename Ptr>
+__device__ __forceinline__ uint32_t decode_tile(const Params &p, uint32_t lut, Ptr head, uint32_t tile_bytes,
                                                 uint32_t t, uint32_t lane) {
-    // the 32 initial states and word counts; each lane's stream starts after the lower lanes'
-    Lane s;
-    uint32_t n;
-    if (SMEM) {
-        uint32_t h = static_cast<uint32_t>(__cvta_generic_to_shared(head));
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(s.x) : "r"(h + 4u * lane));
-        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(n) : "r"(h + 128u + 2u * lane));
+    Lane<SMEM> L;
+    uint32_t len;
+    if constexpr (SMEM) {
+        L.x = lds32(head + 4u * lane);
+        len = lds16(head + 128u + 2u * lane);
     } else {
-        s.x = __ldg(reinterpret_cast<const uint32_t *>(head) + lane);
-        n = __ldg(reinterpret_cast<const uint16_t *>(head + 128) + lane);
+        L.x = __ldg(reinterpret_cast<const uint32_t *>(head) + lane);
+        len = __ldg(reinterpret_cast<const uint16_t *>(head + 128) + lane);
     }
-    uint32_t incl = n;
+    // each lane's region starts after the lower lanes' regions
+    uint32_t incl = len;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
         uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
@@ -309,122 +410,214 @@ __device__ __forceinline__ uint32_t decode_tile(const Params &p, const uint32_t 
     }
     uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
     uint32_t capacity = (tile_bytes - uint32_t(kTileHead)) / 2u;
-    if (total > capacity) return EP_DEC_WORD_OVERRUN;  // warp-uniform: the counts overrun the tile
-    uint32_t start = incl - n;
-    s.idx = start;
-    s.last = capacity ? capacity - 1u : 0u;
-    s.w = W.at(min(s.idx, s.last));
-    if (uint64_t(t + 1) * 32u * p.K <= p.nb)
-        decode_blocks<DT, SMEM, false>(p, s, lut, tinfo, W, t, lane);
-    else
-        decode_blocks<DT, SMEM, true>(p, s, lut, tinfo, W, t, lane);
-    uint32_t err = 0;
-    if (s.x != kStateLow) err |= EP_DEC_BAD_END;
-    uint32_t used = s.idx - start;
-    if (used != n) err |= used > n ? EP_DEC_WORD_OVERRUN : EP_DEC_WORD_COUNT;
+    if (total > capacity) return EP_DEC_WORD_OVERRUN;  // warp-uniform: the regions overrun the tile
+    uint32_t start = incl - len;
+    L.end = incl;
+    uint32_t rb = 0, err;
+    if constexpr (SMEM) {
+        L.area = head + uint32_t(kTileHead);
+        L.wp = L.area + 2u * start;
+        L.w = lds16(L.wp);
+        uint32_t wlim = L.area + 2u * capacity;
+        if (uint64_t(t + 1) * 32u * p.K <= p.nb)
+            err = decode_blocks<DT, SMEM, false>(p, L, rb, lut, wlim, t, lane);
+        else
+            err = decode_blocks<DT, SMEM, true>(p, L, rb, lut, wlim, t, lane);
+    } else {
+        L.area = reinterpret_cast<const uint16_t *>(head + kTileHead);
+        L.wlim = L.area + (capacity ? capacity - 1u : 0u);
+        L.wp = L.area + start < L.wlim ? L.area + start : L.wlim;
+        L.w = __ldg(L.wp);
+        if (uint64_t(t + 1) * 32u * p.K <= p.nb)
+            err = decode_blocks<DT, SMEM, false>(p, L, rb, lut, L.wlim, t, lane);
+        else
+            err = decode_blocks<DT, SMEM, true>(p, L, rb, lut, L.wlim, t, lane);
+    }
+    if (L.x != kStateLow) err |= EP_DEC_BAD_END;
+    // the front (rANS words) and the back (raw bits) cover the region exactly
+    uint32_t used = L.consumed(start) + (rb + 15u) / 16u;
+    if (used != len) err |= used > len ? EP_DEC_WORD_OVERRUN : EP_DEC_WORD_COUNT;
     if (capacity - total >= 8u) err |= EP_DEC_WORD_COUNT;
     return err;
 }
 
+// ------------------------------------------------------------------ slot tables
+// Entry of token t of context c with frequency f: frequency, escape flag and value field (the
+// offset of the slot inside the token is added per slot).  A direct token stores v + 256 of
+// the coordinate it stands for; an escape token stores its index past 2^m (for coordinates
+// 1..6 as 2 d + c, so that bits 0 and 1 of the field are the coset and the parity of y in
+// every entry of contexts 0..2).
+__device__ __forceinline__ uint32_t token_head(uint32_t c, uint32_t t, uint32_t f, uint32_t m) {
+    uint32_t field;
+    if (t < (1u << m)) {
+        int32_t v;
+        if (c == 0)
+            v = 4 * unzigzag(t >> 2) + int32_t(t & 3u);
+        else if (c < 3)
+            v = 2 * (2 * unzigzag(t >> 1) + int32_t(t & 1u)) + int32_t(c - 1);
+        else
+            v = 2 * (2 * unzigzag(t) + int32_t((c - 3) & 1u)) + int32_t((c - 3) >> 1);
+        field = (uint32_t(v + 256) & 0x1ffu) << 11;
+    } else {
+        uint32_t d = t - (1u << m);
+        uint32_t fv = (c == 1 || c == 2) ? 2u * d + (c - 1) : d;
+        field = kEscBit | ((fv & 0x1ffu) << 11);
+    }
+    return (min(f, kProbScale - 1u) << 21) | field;
+}
+
 // ------------------------------------------------------------------ kernel
+// Shared memory: slot tables (the frequency section is first staged here), per-context
+// prefix sums, per-segment first tokens, mbarriers, then nbuf tile buffers per warp.
 template <int DT>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_constant__ Params p) {
-    extern __shared__ __align__(16) uint32_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    uint32_t *lut = smem;                                            // [ctx][slot]
-    uint32_t *tinfo = smem + kLutEntries;                            // [ctx][token]
-    uint32_t *cum = tinfo + kContexts * 256;                         // [ctx][257]
-    uint8_t *buf = reinterpret_cast<uint8_t *>(smem) + kFixedBytes + size_t(warp) * p.tile_buf;
+    const uint32_t lut = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    const uint32_t cum = lut + uint32_t(kLutBytes);
+    const uint32_t seg = cum + uint32_t(kCumBytes);
+    const uint32_t bars = seg + uint32_t(kSegBytes);
+    const uint32_t tbar = bars + uint32_t(kMaxWarps) * 16u;  // the tables' mbarrier
+    const uint32_t nbuf = p.nbuf;
+    const uint32_t bufs = bars + uint32_t(kBarBytes) + warp * (nbuf ? nbuf : 1u) * p.tile_buf;
+    const uint32_t t_begin = uint32_t(uint64_t(blockIdx.x) * p.T / gridDim.x);
+    const uint32_t t_end = uint32_t(uint64_t(blockIdx.x + 1) * p.T / gridDim.x);
 
-    // ---- this warp's first tile starts loading now, behind the table set-up
-    uint32_t t_begin = uint32_t(uint64_t(blockIdx.x) * p.T / gridDim.x);
-    uint32_t t_end = uint32_t(uint64_t(blockIdx.x + 1) * p.T / gridDim.x);
-    const uint32_t buf_s = static_cast<uint32_t>(__cvta_generic_to_shared(buf));
-    auto stage = [&](uint32_t t) {  // tile t into the buffer if it is valid and fits; no wait
-        uint32_t beg = __ldg(p.dir + t), end = __ldg(p.dir + t + 1);
-        if (end >= beg + uint32_t(kTileHead / 16) && uint64_t(end) <= p.tile_units && (end - beg) * 16u <= p.tile_buf) {
-            const uint8_t *tp = p.tiles + size_t(beg) * 16;
-            for (uint32_t i = lane; i < end - beg; i += 32u) cp_async16(buf_s + 16u * i, tp + 16u * i);
+    if (threadIdx.x == 0) {
+        for (uint32_t w = 0; w < nwarps; ++w) {
+            mbar_init(bars + 16u * w, 1);
+            mbar_init(bars + 16u * w + 8u, 1);
         }
-        asm volatile("cp.async.commit_group;\n" ::: "memory");
-    };
-    if (t_begin + warp < t_end) stage(t_begin + warp);
+        mbar_init(tbar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && p.freq_bytes) {
+        mbar_expect(tbar, p.freq_bytes);
+        bulk_g2s(lut, p.freq, p.freq_bytes, tbar);
+    }
 
-    // ---- tables.  Every slot starts as an escape to token 255 with f = 2^11 and bias = slot
-    // (an identity step that decodes nothing: a damaged stream then fails its end checks);
-    // token info starts at zero.  Then the cumulative frequencies per context (warps take
-    // contexts round robin), then the slots of every token.
-    for (uint32_t i = threadIdx.x; i < kLutEntries; i += blockDim.x)
-        lut[i] = (kProbScale << 20) | kEsc | (255u << 11) | (i & (kProbScale - 1));
-    for (uint32_t i = threadIdx.x; i < kContexts * 256u; i += blockDim.x) tinfo[i] = 0;
+    // a tile's copy into buffer j of this warp; every lane computes whether it was issued
+    auto tile_ok = [&](uint32_t t, uint32_t &beg, uint32_t &bytes) -> bool {
+        beg = __ldg(p.dir + t);
+        uint32_t end = __ldg(p.dir + t + 1);
+        bytes = (end - beg) * 16u;
+        return end >= beg + uint32_t(kTileHead / 16) && uint64_t(end) <= p.tile_units;
+    };
+    auto issue = [&](uint32_t t, uint32_t j) -> bool {
+        uint32_t beg, bytes;
+        bool ok = tile_ok(t, beg, bytes) && nbuf && bytes + kSlack <= p.tile_buf;
+        if (ok && lane == 0) {
+            uint32_t bar = bars + 16u * warp + 8u * j;
+            fence_proxy_async();
+            mbar_expect(bar, bytes);
+            bulk_g2s(bufs + j * p.tile_buf, p.tiles + size_t(beg) * 16, bytes, bar);
+        }
+        return ok;
+    };
+    // per buffer: a copy in flight (bit 0 / 1) and the mbarrier phase to wait for (bit 2 / 3)
+    uint32_t pend = 0, phase = 0;
+    for (uint32_t j = 0; j < nbuf; ++j) {
+        uint32_t t = t_begin + warp + j * nwarps;
+        if (t < t_end && issue(t, j)) pend |= 1u << j;
+    }
+
+    // ---- slot tables: prefix sums per context (a warp per context), the first token of every
+    // 32-slot segment, then every slot's entry
+    bool tables_ok = p.freq_bytes == 0 || mbar_wait(tbar, 0);
+    if (!tables_ok && lane == 0 && p.status) atomicOr(p.status, EP_DEC_TIMEOUT);
     for (uint32_t c = warp; c < uint32_t(kContexts); c += nwarps) {
         uint32_t n = p.tab_off[c + 1] - p.tab_off[c], run = 0;
+        uint32_t crow = cum + c * kCumStride * 2u, srow = seg + c * kSegs * 2u;
+        for (uint32_t g = lane; g < kSegs; g += 32) sts16(srow + 2u * g, 0xffffu);
+        __syncwarp();
+        bool bad = false;
         for (uint32_t base = 0; base < n; base += 32) {
             uint32_t t = base + lane;
-            uint32_t f = t < n ? uint32_t(p.freq[p.tab_off[c] + t]) : 0u;
+            uint32_t f = t < n ? lds16(lut + 2u * (p.tab_off[c] + t)) : 0u;
+            bad |= f >= kProbScale;
+            f = min(f, kProbScale);
             uint32_t incl = f;
 #pragma unroll
             for (int d = 1; d < 32; d <<= 1) {
                 uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
                 if (lane >= uint32_t(d)) incl += y;
             }
-            if (t < n) cum[c * 257 + t] = run + incl - f;
-            run += __shfl_sync(0xffffffffu, incl, 31);
+            uint32_t lo = min(run + incl - f, kProbScale), hi = min(run + incl, kProbScale);
+            if (t < n) {
+                sts16(crow + 2u * t, lo);
+                for (uint32_t g = (lo + 31u) >> 5; g < ((hi + 31u) >> 5); ++g) sts16(srow + 2u * g, t);
+            }
+            run = min(run + __shfl_sync(0xffffffffu, incl, 31), 0xffffu);
         }
         if (lane == 0) {
-            cum[c * 257 + n] = run;
-            if (n && run != kProbScale && p.status) atomicOr(p.status, EP_DEC_BAD_TOKEN);
+            sts16(crow + 2u * n, min(run, kProbScale));
+            if (p.status && n && run != kProbScale) atomicOr(p.status, EP_DEC_BAD_TOKEN);
         }
+        if (__any_sync(0xffffffffu, bad) && lane == 0 && p.status) atomicOr(p.status, EP_DEC_BAD_TOKEN);
     }
     __syncthreads();
-    for (uint32_t i = warp; i < p.tab_off[kContexts]; i += nwarps) {
-        uint32_t c = 0;
-        while (c + 1 < uint32_t(kContexts) && p.tab_off[c + 1] <= i) ++c;
-        uint32_t t = i - p.tab_off[c];
-        uint32_t m = (p.splits >> (3 * c)) & 7u;
-        bool esc = t >= (1u << m);
-        // a direct token's value is unzigzag(token); an escape keeps the token index
-        uint32_t field = esc ? t : (uint32_t(unzigzag(t)) & 0xffu);
-        uint32_t lo = cum[c * 257 + t], f = cum[c * 257 + t + 1] - lo;
-        uint32_t fill = f < kProbScale ? f : kProbScale;
-        uint32_t head = (fill << 20) | (esc ? kEsc : 0u) | (field << 11);
-        for (uint32_t sl = lane; sl < fill; sl += 32)
-            if (lo + sl < kProbScale) lut[c * kProbScale + lo + sl] = head | sl;
-        if (lane == 0 && esc) {
-            // token -> value base and raw extra bits (h = min(m, 2))
-            uint32_t h = m < 2 ? m : 2;
-            uint32_t d = t - (1u << m), nn = m + (d >> h);
-            uint32_t nbits = nn - h;
-            uint32_t base = ((1u << h) | (d & ((1u << h) - 1u))) << (nbits & 31u);
-            tinfo[c * 256 + t] = nbits <= 21 ? (base << 5) | nbits : 0u;
+    // Each thread fills one 32-slot segment; lane l starts at slot l of its segment and wraps
+    // around, so the 32 lanes of a warp store to 32 different banks at every step.
+    for (uint32_t idx = threadIdx.x; idx < uint32_t(kContexts) * kSegs; idx += blockDim.x) {
+        uint32_t c = idx / kSegs, g = idx % kSegs;
+        uint32_t n = p.tab_off[c + 1] - p.tab_off[c];
+        uint32_t crow = cum + c * kCumStride * 2u, row = lut + c * kSlotBytes;
+        uint32_t t0 = lds16(seg + (c * kSegs + g) * 2u);
+        uint32_t m = split_of(p, c);
+        uint32_t l = idx & 31u;
+        if (n == 0 || t0 >= n) {
+            for (uint32_t j = 0; j < 32; ++j) sts32(row + 4u * (32u * g + ((l + j) & 31u)), 0u);
+            continue;
+        }
+        uint32_t t = t0, lo = lds16(crow + 2u * t), hi = lds16(crow + 2u * (t + 1));
+        uint32_t head = token_head(c, t, hi - lo, m);
+        for (uint32_t j = 0; j < 32; ++j) {
+            uint32_t s = 32u * g + ((l + j) & 31u);
+            if (l + j == 32u) {  // wrapped to the segment start
+                t = t0;
+                lo = lds16(crow + 2u * t);
+                hi = lds16(crow + 2u * (t + 1));
+                head = token_head(c, t, hi - lo, m);
+            }
+            while (s >= hi && t + 1 < n) {
+                ++t;
+                lo = hi;
+                hi = lds16(crow + 2u * (t + 1));
+                head = token_head(c, t, hi - lo, m);
+            }
+            sts32(row + 4u * s, head | ((s - lo) & (kProbScale - 1u)));
         }
     }
     __syncthreads();
 
-    // ---- tiles of this CTA: a contiguous range, warps round robin
-    for (uint32_t t = t_begin + warp; t < t_end; t += nwarps) {
-        if (t != t_begin + warp) {
-            __syncwarp();  // the previous tile's reads of the buffer are done
-            stage(t);
-        }
-        uint32_t beg = __ldg(p.dir + t), end = __ldg(p.dir + t + 1);
-        uint32_t err;
-        if (end < beg + uint32_t(kTileHead / 16) || uint64_t(end) > p.tile_units) {
+    // ---- tiles of this CTA: a contiguous range, warps round robin, nbuf copies in flight
+    uint32_t j = 0;
+    for (uint32_t t = t_begin + warp; t < t_end; t += nwarps, ++j) {
+        uint32_t b = nbuf ? j % nbuf : 0u;
+        uint32_t beg, bytes, err = 0;
+        bool valid = tile_ok(t, beg, bytes);
+        if (!valid) {
             err = EP_DEC_BAD_TILE;
-        } else {
-            const uint8_t *tp = p.tiles + size_t(beg) * 16;
-            uint32_t tile_bytes = (end - beg) * 16u;
-            if (tile_bytes <= p.tile_buf) {
-                asm volatile("cp.async.wait_all;\n" ::: "memory");
-                __syncwarp();
-                Words<true> W{buf_s + uint32_t(kTileHead)};
-                err = decode_tile<DT, true>(p, lut, tinfo, buf, W, tile_bytes, t, lane);
-            } else {
-                Words<false> W{reinterpret_cast<const uint16_t *>(tp + kTileHead)};
-                err = decode_tile<DT, false>(p, lut, tinfo, tp, W, tile_bytes, t, lane);
+        } else if (pend & (1u << b)) {
+            bool done = mbar_wait(bars + 16u * warp + 8u * b, (phase >> b) & 1u);
+            phase ^= 1u << b;
+            pend &= ~(1u << b);
+            if (!done) {  // a lost copy: report, let the other buffer's copy land, stop
+                if (lane == 0 && p.status) atomicOr(p.status, EP_DEC_TIMEOUT);
+                uint32_t o = b ^ 1u;
+                if (nbuf > 1 && (pend & (1u << o))) mbar_wait(bars + 16u * warp + 8u * o, (phase >> o) & 1u);
+                return;
             }
+            if (tables_ok) err = decode_tile<DT, true>(p, lut, bufs + b * p.tile_buf, bytes, t, lane);
+        } else if (tables_ok) {
+            err = decode_tile<DT, false>(p, lut, p.tiles + size_t(beg) * 16, bytes, t, lane);
         }
         if (err && p.status) atomicOr(p.status, err);
+        __syncwarp();
+        uint32_t tn = t + nbuf * nwarps;
+        if (nbuf && tn < t_end && issue(tn, b)) pend |= 1u << b;
     }
 }
 
@@ -437,7 +630,7 @@ struct DeviceCache {
 DeviceCache g_cache;
 
 template <int DT>
-cudaError_t launch(const Params &p, int device, cudaStream_t stream) {
+cudaError_t launch(Params &p, uint64_t max_tile, int device, cudaStream_t stream) {
     int sms;
     {
         std::lock_guard<std::mutex> g(g_cache.mu);
@@ -454,16 +647,32 @@ cudaError_t launch(const Params &p, int device, cudaStream_t stream) {
         }
         sms = g_cache.sms[device];
     }
-    // one CTA per SM, as many warps as tiles per SM, at most kMaxWarps and as many tile buffers
-    // as fit beside the tables
-    uint32_t cap = uint32_t((kSmemLimit - kFixedBytes) / p.tile_buf);
-    uint32_t warps = (p.T + uint32_t(sms) - 1) / uint32_t(sms);
-    warps = warps < 1 ? 1 : warps;
+    // one CTA per SM (at most one per tile); warps = tiles per CTA, within kMaxWarps and the
+    // tile buffers that fit beside the tables: two per warp when they fit, else one, else the
+    // tiles are read from global memory
+    uint32_t grid = p.T < uint32_t(sms) ? p.T : uint32_t(sms);
+    uint32_t warps = (p.T + grid - 1) / grid;
     warps = warps > uint32_t(kMaxWarps) ? uint32_t(kMaxWarps) : warps;
-    warps = warps > cap ? cap : warps;
-    uint32_t grid = (p.T + warps - 1) / warps;
-    if (grid > uint32_t(sms)) grid = uint32_t(sms);
-    decode_kernel<DT><<<grid, warps * 32, smem_bytes(warps, p.tile_buf), stream>>>(p);
+    const size_t avail = kSmemLimit - kFixedBytes;
+    p.tile_buf = uint32_t((max_tile + kSlack + 15) & ~uint64_t(15));
+    bool many = p.T > grid * warps;  // some warp decodes more than one tile
+    if (many && 2ull * warps * p.tile_buf <= avail) {
+        p.nbuf = 2;
+    } else if (uint64_t(warps) * p.tile_buf <= avail) {
+        p.nbuf = 1;
+    } else if (uint64_t(p.tile_buf) * 2 * 4 <= avail) {
+        warps = uint32_t(avail / (2ull * p.tile_buf));
+        p.nbuf = 2;
+    } else if (p.tile_buf <= avail) {
+        warps = uint32_t(avail / p.tile_buf);
+        p.nbuf = 1;
+    } else {
+        p.nbuf = 0;  // tiles beyond any buffer: read in place
+        p.tile_buf = 16;
+    }
+    if (warps < 1) warps = 1;
+    size_t smem = kFixedBytes + size_t(warps) * (p.nbuf ? p.nbuf : 1) * p.tile_buf;
+    decode_kernel<DT><<<grid, warps * 32, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -484,7 +693,7 @@ extern "C" int ep_decompress(const ep_info *info, const void *d_blob, void *d_ou
     p.dir = reinterpret_cast<const uint32_t *>(base + info->off_dir);
     p.tiles = base + info->off_tiles;
     p.rowf = reinterpret_cast<const float *>(base + info->off_rowf);
-    p.freq = reinterpret_cast<const uint16_t *>(base + info->off_freq);
+    p.freq = base + info->off_freq;
     p.out = d_out;
     p.status = d_status;
     p.tile_units = (info->storage_nbytes - info->off_tiles) / 16;
@@ -492,29 +701,28 @@ extern "C" int ep_decompress(const ep_info *info, const void *d_blob, void *d_ou
     p.cb = uint32_t(info->cols / 8);
     p.K = info->blocks_per_lane;
     p.T = info->n_tiles;
-    {
-        uint64_t need = (info->max_tile_nbytes + 15) & ~uint64_t(15);
-        // at least one 16-byte piece past the tile head, so a clamped word read stays inside
-        p.tile_buf = uint32_t(need < kTileHead + 16 ? kTileHead + 16 : (need > kTileBufMax ? kTileBufMax : need));
-    }
     p.splits = 0;
     p.tab_off[0] = 0;
     for (int c = 0; c < kContexts; ++c) {
-        if (info->split[c] > kMaxSplit || info->ntok[c] > 256) return EP_ERR_CORRUPT;
-        p.splits |= uint32_t(info->split[c]) << (3 * c);
+        if (!split_valid(info->split[c], c) || info->ntok[c] > split_alphabet(info->split[c], kCtxLow[c]))
+            return EP_ERR_CORRUPT;
+        p.splits |= uint32_t(info->split[c]) << (4 * c);
         p.tab_off[c + 1] = p.tab_off[c] + info->ntok[c];
     }
+    p.freq_bytes = uint32_t((uint64_t(p.tab_off[kContexts]) * 2 + 15) & ~uint64_t(15));
+    if (info->off_freq + p.freq_bytes > info->off_dir || p.freq_bytes > kLutBytes) return EP_ERR_CORRUPT;
     int device;
     cudaError_t e = cudaGetDevice(&device);
     if (e != cudaSuccess) return EP_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint64_t mt = info->max_tile_nbytes;
     switch (out_dtype) {
-    case EP_BF16: e = launch<EP_BF16>(p, device, s); break;
-    case EP_FP16: e = launch<EP_FP16>(p, device, s); break;
-    case EP_FP32: e = launch<EP_FP32>(p, device, s); break;
-    case EP_INT8: e = launch<EP_INT8>(p, device, s); break;
-    case EP_FP8_E4M3: e = launch<EP_FP8_E4M3>(p, device, s); break;
-    case EP_LATTICE_I32: e = launch<EP_LATTICE_I32>(p, device, s); break;
+    case EP_BF16: e = launch<EP_BF16>(p, mt, device, s); break;
+    case EP_FP16: e = launch<EP_FP16>(p, mt, device, s); break;
+    case EP_FP32: e = launch<EP_FP32>(p, mt, device, s); break;
+    case EP_INT8: e = launch<EP_INT8>(p, mt, device, s); break;
+    case EP_FP8_E4M3: e = launch<EP_FP8_E4M3>(p, mt, device, s); break;
+    case EP_LATTICE_I32: e = launch<EP_LATTICE_I32>(p, mt, device, s); break;
     default: return EP_ERR_INVALID_ARG;
     }
     return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;

@@ -1,4 +1,4 @@
-// Stream format v1 constants and small helpers shared by the library's host encoder, the
+// Stream format v3 constants and small helpers shared by the library's host encoder, the
 // stream parser and the decode kernel.  The byte layout is fixed by the library (the pages
 // give none): a 64-byte header, per-row factors, optional per-row code scales, per-context
 // frequency tables, a tile directory and the tiles.
@@ -9,16 +9,23 @@
 namespace ep {
 
 constexpr uint32_t kMagic = 0x31545045u;  // "EPT1"
-constexpr uint32_t kVersion = 2;
-constexpr uint32_t kProbBits = 11;         // frequency precision: tables sum to 2^11
+constexpr uint32_t kVersion = 3;
+constexpr uint32_t kProbBits = 11;         // frequency precision: tables sum to 2^11, each entry below it
 constexpr uint32_t kProbScale = 1u << kProbBits;
 constexpr uint32_t kStateLow = 1u << 16;   // rANS state interval [2^16, 2^32), 16-bit words
 constexpr int kLanes = 32;                 // interleaved states per tile = warp lanes
 constexpr int kContexts = 7;
-constexpr int kMaxSplit = 7;
-constexpr uint32_t kChunkBits = 11;        // extra bits travel in uniform chunks of <= 11 bits
+constexpr uint32_t kTopBits = 2;           // bits below the leading one carried by an escape token
+constexpr uint32_t kValueBits = 22;        // every coded value is below 2^22
+// low bits of the value kept in every token, and the largest split, per context: coordinate 0
+// keeps v0 mod 4 (coset, parity of y0), coordinates 1..6 the parity of y_i, coordinate 7 none.
+// At the largest splits every direct token decodes to a coordinate in [-256, 255].
+constexpr uint32_t kCtxLow[kContexts] = {2, 1, 1, 0, 0, 0, 0};
+constexpr uint32_t kCtxMaxSplit[kContexts] = {9, 8, 8, 7, 7, 7, 7};
+constexpr uint32_t kMaxAlphabet = 720;     // (1 << 9) + ((22 - 9) << 2 << 2): the largest context alphabet
 constexpr size_t kHeaderBytes = 64;
 constexpr size_t kTileHead = 192;            // per tile: 32 initial states (u32) + 32 word counts (u16)
+                                             // then the lanes' words, then the tile's raw extra bits
 constexpr double kTileBudget = 5952.0;       // expected payload bytes per tile (6 KB staging buffer)
 constexpr int kNumQ = 1280;                // resolution indices
 constexpr int64_t kSampleBlocks = 65536;   // blocks sampled by the storage estimate
@@ -27,10 +34,10 @@ constexpr double kTargetMargin = 0.995;
 
 inline size_t align16(size_t n) { return (n + 15) & ~size_t(15); }
 
-inline uint32_t split_h(uint32_t m) { return m < 2 ? m : 2; }
-
 // tokens a split can produce for values below 2^22
-inline uint32_t split_alphabet(uint32_t m) { return (1u << m) + ((22u - m) << split_h(m)); }
+inline uint32_t split_alphabet(uint32_t m, uint32_t low) { return (1u << m) + (((kValueBits - m) << kTopBits) << low); }
+
+inline bool split_valid(uint32_t m, int ctx) { return m >= kTopBits + kCtxLow[ctx] && m <= kCtxMaxSplit[ctx]; }
 
 inline int elt_bytes(int dt) { return dt == 3 ? 4 : (dt == 1 || dt == 2) ? 2 : 1; }
 

@@ -176,62 +176,78 @@ inline uint32_t zz(int32_t y) { return y < 0 ? uint32_t(-int64_t(y)) * 2u - 1u :
 
 inline int bitlen(uint32_t u) { return u ? 32 - __builtin_clz(u) : 0; }
 
-// contexts and values of one block: 0 for coordinate 0 (zz v0), 1 + c for coordinates 1..6
-// (zz y_i), 3 + 2c + p for coordinate 7 (zz of (y7 - p) / 2)
-inline void symbols_of(const int32_t *v, uint8_t *ctx, uint32_t *u) {
+// Contexts and coded values of one block, in coding order.  c = v0 mod 2, y_i = (v_i - c) / 2,
+// p = parity of y0 + ... + y6.  Coordinate 0: context 0, value 4 zz(a0) + r0 with v0 = 4 a0 + r0;
+// coordinates 1..6: context 1 + c, value 2 zz(a) + b with y = 2 a + b; coordinate 7: context
+// 3 + 2c + p, value zz((y7 - p) / 2).  Arithmetic shifts are floor divisions here.
+inline void symbols_of(const int32_t *v, uint8_t *ctx, uint32_t *s) {
     int32_t c = v[0] & 1;
-    int32_t par = 0;
+    int32_t par = ((v[0] - c) >> 1) & 1;
     ctx[0] = 0;
-    u[0] = zz(v[0]);
-    par ^= ((v[0] - c) >> 1) & 1;
+    s[0] = 4u * zz(v[0] >> 2) + uint32_t(v[0] & 3);
     for (int i = 1; i < 7; ++i) {
         int32_t y = (v[i] - c) >> 1;
         par ^= y & 1;
         ctx[i] = uint8_t(1 + c);
-        u[i] = zz(y);
+        s[i] = 2u * zz(y >> 1) + uint32_t(y & 1);
     }
     int32_t y7 = (v[7] - c) >> 1;
     ctx[7] = uint8_t(3 + 2 * c + par);
-    u[7] = zz((y7 - par) >> 1);
+    s[7] = zz((y7 - par) >> 1);
 }
 
 struct Token {
     uint32_t tok, nbits, extra;
 };
 
-inline Token token_of(uint32_t u, uint32_t m) {
-    if (u < (1u << m)) return {u, 0, 0};
-    uint32_t h = split_h(m);
-    uint32_t n = uint32_t(bitlen(u)) - 1;
-    uint32_t low = n - h;
-    return {(1u << m) + ((n - m) << h) + ((u >> low) & ((1u << h) - 1u)), low, u & ((1u << low) - 1u)};
+// hybrid-integer token of s with split m, keeping the `low` low bits of s in the token and two
+// bits below the leading one; the bits in between are raw extra bits
+inline Token token_of(uint32_t s, uint32_t m, uint32_t low) {
+    if (s < (1u << m)) return {s, 0, 0};
+    uint32_t n = uint32_t(bitlen(s)) - 1;
+    uint32_t nbits = n - kTopBits - low;
+    uint32_t top = (s >> (n - kTopBits)) & ((1u << kTopBits) - 1u);
+    uint32_t tok = (1u << m) + (((((n - m) << kTopBits) | top) << low) | (s & ((1u << low) - 1u)));
+    return {tok, nbits, (s >> low) & ((1u << nbits) - 1u)};
 }
 
-// smallest m in [0, 7] with >= 99.9% of the values below 2^m (bit length <= m)
-uint32_t pick_split(const uint64_t *by_len) {
+// smallest m allowed for the context with >= 99.9% of the values below 2^m (bit length <= m)
+uint32_t pick_split(const uint64_t *by_len, int ctx) {
+    uint32_t lo = kTopBits + kCtxLow[ctx], hi = kCtxMaxSplit[ctx];
     uint64_t n = 0;
     for (int i = 0; i <= 32; ++i) n += by_len[i];
-    if (!n) return 0;
+    if (!n) return lo;
     uint64_t acc = 0;
-    for (uint32_t m = 0; m <= uint32_t(kMaxSplit); ++m) {
+    for (uint32_t m = 0; m <= hi; ++m) {
         acc += by_len[m];
-        if (acc * 1000u >= n * 999u) return m;
+        if (m >= lo && acc * 1000u >= n * 999u) return m;
     }
-    return kMaxSplit;
+    return hi;
 }
 
 // largest remainders to a sum of 2^11, then every seen token raised to >= 1 from the
-// currently largest frequency (lowest index on ties)
+// currently largest frequency (lowest index on ties); a lone seen token keeps 2^11 - 1 and
+// gives one unit to a phantom token (token 1 if it is token 0, else token 0)
 uint32_t build_freqs(const std::vector<uint64_t> &cnt, std::vector<uint32_t> &f) {
     size_t n = cnt.size();
     f.assign(n, 0);
     uint64_t total = 0;
-    uint32_t len = 0;
+    uint32_t len = 0, seen = 0, only = 0;
     for (size_t i = 0; i < n; ++i) {
         total += cnt[i];
-        if (cnt[i]) len = uint32_t(i + 1);
+        if (cnt[i]) {
+            len = uint32_t(i + 1);
+            ++seen;
+            only = uint32_t(i);
+        }
     }
     if (!total) return 0;
+    if (seen == 1) {
+        uint32_t phantom = only == 0 ? 1u : 0u;
+        f[only] = kProbScale - 1;
+        f[phantom] = 1;
+        return std::max(len, phantom + 1);
+    }
     std::vector<std::pair<uint64_t, uint32_t>> rems;  // (remainder, index)
     uint32_t used = 0;
     for (size_t i = 0; i < n; ++i) {
@@ -341,12 +357,12 @@ struct Encoder {
         uint32_t m[kContexts];
         std::vector<uint64_t> cnt[kContexts];
         for (int c = 0; c < kContexts; ++c) {
-            m[c] = pick_split(by_len[c]);
-            cnt[c].assign(split_alphabet(m[c]), 0);
+            m[c] = pick_split(by_len[c], c);
+            cnt[c].assign(split_alphabet(m[c], kCtxLow[c]), 0);
         }
         uint64_t extra = 0;
         for (size_t i = 0; i < val.size(); ++i) {
-            Token t = token_of(val[i], m[ctx[i]]);
+            Token t = token_of(val[i], m[ctx[i]], kCtxLow[ctx[i]]);
             cnt[ctx[i]][t.tok]++;
             extra += t.nbits;
         }
@@ -372,39 +388,47 @@ struct Encoder {
         return 8.0 * bytes / double(rows * cols);
     }
 
-    // ---- one tile: 32 independent lanes, each its symbols in decode order encoded in reverse
+    // ---- one tile: 32 independent lanes.  A lane's region holds its rANS words in decode order
+    // followed by its raw extra bits, packed least significant bit first into 16-bit words that
+    // are stored back to front (the region's last word holds the first 16 raw bits).  Returns
+    // false when a region exceeds 65535 words.
     struct Event {
         uint16_t f, cum;
     };
 
-    static void encode_tile(const uint8_t *ctx, const uint32_t *val, int64_t nb, int64_t t, uint32_t K,
+    static bool encode_tile(const uint8_t *ctx, const uint32_t *val, int64_t nb, int64_t t, uint32_t K,
                             const uint32_t *m, const std::vector<uint32_t> *freq, const std::vector<uint32_t> *cum,
                             std::vector<Event> &ev, std::vector<uint16_t> &words, std::vector<uint8_t> &out) {
         int64_t first = t * int64_t(kLanes) * K;
         uint32_t state[kLanes];
         uint32_t count[kLanes];
+        bool fits = true;
         words.clear();
-        std::vector<size_t> lane_end(kLanes);
         for (int l = 0; l < kLanes; ++l) {
             ev.clear();
+            size_t before = words.size();
+            uint64_t acc = 0;
+            uint32_t nacc = 0;
+            std::vector<uint16_t> raw;
             for (uint32_t k = 0; k < K; ++k) {
                 int64_t b = first + int64_t(k) * kLanes + l;
                 if (b >= nb) break;
                 for (int i = 0; i < 8; ++i) {
                     size_t s = size_t(8 * b + i);
                     uint8_t c = ctx[s];
-                    Token tk = token_of(val[s], m[c]);
+                    Token tk = token_of(val[s], m[c], kCtxLow[c]);
                     ev.push_back({uint16_t(freq[c][tk.tok]), uint16_t(cum[c][tk.tok])});
-                    for (uint32_t j = 0; j * kChunkBits < tk.nbits; ++j) {
-                        uint32_t bits = std::min(kChunkBits, tk.nbits - j * kChunkBits);
-                        uint32_t chunk = (tk.extra >> (j * kChunkBits)) & ((1u << bits) - 1u);
-                        uint32_t f = 1u << (kProbBits - bits);
-                        ev.push_back({uint16_t(f), uint16_t(chunk * f)});
+                    acc |= uint64_t(tk.extra) << nacc;
+                    nacc += tk.nbits;
+                    while (nacc >= 16) {
+                        raw.push_back(uint16_t(acc));
+                        acc >>= 16;
+                        nacc -= 16;
                     }
                 }
             }
+            if (nacc) raw.push_back(uint16_t(acc));
             uint32_t x = kStateLow;
-            size_t before = words.size();
             for (size_t e = ev.size(); e-- > 0;) {
                 uint32_t f = ev[e].f;
                 if (uint64_t(x) >= (uint64_t(f) << (32 - kProbBits))) {  // keep the next state below 2^32
@@ -414,8 +438,11 @@ struct Encoder {
                 x = (x / f) * kProbScale + (x % f) + ev[e].cum;
             }
             std::reverse(words.begin() + long(before), words.end());  // decode order
+            words.insert(words.end(), raw.rbegin(), raw.rend());
             state[l] = x;
-            count[l] = uint32_t(words.size() - before);
+            size_t n = words.size() - before;
+            if (n > 0xffff) fits = false;
+            count[l] = uint32_t(n);
         }
         size_t base = out.size();
         size_t bytes = align16(kTileHead + 2 * words.size());
@@ -431,6 +458,7 @@ struct Encoder {
             p[2 * i] = uint8_t(words[i]);
             p[2 * i + 1] = uint8_t(words[i] >> 8);
         }
+        return fits;
     }
 
     // ---- full stream at resolution index k
@@ -459,24 +487,26 @@ struct Encoder {
             for (int c = 0; c < kContexts; ++c)
                 for (int i = 0; i < 33; ++i) by_len[c][i] += h[size_t(c * 33 + i)];
         uint32_t m[kContexts];
-        for (int c = 0; c < kContexts; ++c) m[c] = pick_split(by_len[c]);
+        for (int c = 0; c < kContexts; ++c) m[c] = pick_split(by_len[c], c);
         // token counts
         std::vector<std::vector<uint64_t>> part_cnt(static_cast<size_t>(nchunks));
         parallel_for(nchunks, nchunks, [&](int64_t c0, int64_t c1) {
             for (int64_t c = c0; c < c1; ++c) {
                 auto &cnt = part_cnt[size_t(c)];
-                cnt.assign(kContexts * 256, 0);
-                for (int64_t s = 8 * c * per; s < 8 * std::min(nb, (c + 1) * per); ++s)
-                    cnt[size_t(ctx[size_t(s)]) * 256 + token_of(val[size_t(s)], m[ctx[size_t(s)]]).tok]++;
+                cnt.assign(kContexts * kMaxAlphabet, 0);
+                for (int64_t s = 8 * c * per; s < 8 * std::min(nb, (c + 1) * per); ++s) {
+                    uint8_t cx = ctx[size_t(s)];
+                    cnt[size_t(cx) * kMaxAlphabet + token_of(val[size_t(s)], m[cx], kCtxLow[cx]).tok]++;
+                }
             }
         });
         std::vector<uint32_t> freq[kContexts], cum[kContexts];
         uint32_t ntok[kContexts];
         uint64_t tokens = 0;
         for (int c = 0; c < kContexts; ++c) {
-            std::vector<uint64_t> cnt(split_alphabet(m[c]), 0);
+            std::vector<uint64_t> cnt(split_alphabet(m[c], kCtxLow[c]), 0);
             for (auto &pc : part_cnt)
-                for (size_t t = 0; t < cnt.size(); ++t) cnt[t] += pc[size_t(c) * 256 + t];
+                for (size_t t = 0; t < cnt.size(); ++t) cnt[t] += pc[size_t(c) * kMaxAlphabet + t];
             ntok[c] = build_freqs(cnt, freq[c]);
             cum[c].assign(freq[c].size(), 0);
             for (size_t t = 1; t < freq[c].size(); ++t) cum[c][t] = cum[c][t - 1] + freq[c][t - 1];
@@ -488,16 +518,20 @@ struct Encoder {
         std::vector<std::vector<uint8_t>> part_tiles(static_cast<size_t>(tchunks));
         std::vector<std::vector<uint32_t>> part_sizes(static_cast<size_t>(tchunks));
         int64_t tper = (int64_t(T) + tchunks - 1) / tchunks;
+        std::vector<char> part_fits(static_cast<size_t>(tchunks), 1);
         parallel_for(tchunks, tchunks, [&](int64_t c0, int64_t c1) {
             std::vector<Event> ev;
             std::vector<uint16_t> words;
             for (int64_t c = c0; c < c1; ++c)
                 for (int64_t t = c * tper; t < std::min<int64_t>(T, (c + 1) * tper); ++t) {
                     size_t before = part_tiles[size_t(c)].size();
-                    encode_tile(ctx.data(), val.data(), nb, t, K, m, freq, cum, ev, words, part_tiles[size_t(c)]);
+                    if (!encode_tile(ctx.data(), val.data(), nb, t, K, m, freq, cum, ev, words, part_tiles[size_t(c)]))
+                        part_fits[size_t(c)] = 0;
                     part_sizes[size_t(c)].push_back(uint32_t((part_tiles[size_t(c)].size() - before) / 16));
                 }
         });
+        for (char f : part_fits)
+            if (!f) return {};
         Layout L = layout_for(rows, container, tokens, T);
         size_t tile_bytes = 0;
         for (auto &pt : part_tiles) tile_bytes += pt.size();
@@ -560,7 +594,7 @@ extern "C" size_t ep_compress_bound(int64_t rows, int64_t cols, const ep_config 
     uint32_t K = cfg->blocks_per_lane ? cfg->blocks_per_lane : ep::auto_blocks_per_lane(nb, cfg->target_bpp);
     uint64_t T = uint64_t((nb + 32 * int64_t(K) - 1) / (32 * int64_t(K)));
     return ep::layout_for(rows, ep::is_code_container(cfg->container_dtype) ? cfg->container_dtype : 0,
-                          7 * 256, T)
+                          7 * ep::kMaxAlphabet, T)
                .tiles +
            size_t(T) * (ep::kTileHead + 16) + size_t(5.0 * n);
 }
@@ -624,6 +658,7 @@ extern "C" int ep_compress_host(const void *src, int32_t src_dtype, int64_t rows
     std::vector<uint8_t> blob;
     for (;;) {
         blob = E.encode(k);
+        if (blob.empty()) return EP_ERR_UNSUPPORTED;  // a lane region beyond 65535 words (forced tile size)
         if (cfg->q_index >= 0 || 8.0 * double(blob.size()) <= target * double(rows * cols)) break;
         if (k == 0) {
             *out_nbytes = blob.size();

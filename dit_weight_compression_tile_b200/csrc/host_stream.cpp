@@ -47,7 +47,7 @@ extern "C" int ep_stream_info(const void *blob, size_t nbytes, ep_info *info) {
     for (int c = 0; c < kContexts; ++c) {
         I.split[c] = p[36 + c];
         I.ntok[c] = uint16_t(rd(p + 44 + 2 * c, 2));
-        if (I.split[c] > kMaxSplit || I.ntok[c] > split_alphabet(I.split[c])) return EP_ERR_CORRUPT;
+        if (!split_valid(I.split[c], c) || I.ntok[c] > split_alphabet(I.split[c], kCtxLow[c])) return EP_ERR_CORRUPT;
         tokens += I.ntok[c];
     }
     Layout L = layout_for(I.rows, I.container_dtype, tokens, I.n_tiles);
@@ -60,7 +60,11 @@ extern "C" int ep_stream_info(const void *blob, size_t nbytes, ep_info *info) {
     size_t q = L.freq;
     for (int c = 0; c < kContexts; ++c) {
         uint32_t sum = 0;
-        for (uint32_t t = 0; t < I.ntok[c]; ++t, q += 2) sum += uint32_t(rd(p + q, 2));
+        for (uint32_t t = 0; t < I.ntok[c]; ++t, q += 2) {
+            uint32_t f = uint32_t(rd(p + q, 2));
+            if (f >= kProbScale) return EP_ERR_CORRUPT;  // the decoder's table entry holds 11 bits
+            sum += f;
+        }
         if (I.ntok[c] && sum != kProbScale) return EP_ERR_CORRUPT;
     }
     const uint8_t *d = p + L.dir;
@@ -92,7 +96,7 @@ extern "C" const char *ep_status_string(int s) {
     case EP_ERR_BUFFER_TOO_SMALL: return "output buffer too small";
     case EP_ERR_CORRUPT: return "stream fails validation";
     case EP_ERR_CUDA: return "CUDA runtime error";
-    case EP_ERR_UNSUPPORTED: return "not supported by stream format v1";
+    case EP_ERR_UNSUPPORTED: return "not supported by the stream format";
     default: return "unknown status";
     }
 }

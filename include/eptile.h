@@ -57,7 +57,9 @@ enum ep_decode_flags {
                                  kernel reports such damage through the two flags below) */
     EP_DEC_BAD_END = 4u,      /* a lane's state did not return to 2^16 at the end of its tile */
     EP_DEC_WORD_COUNT = 8u,   /* the tile has unread words beyond its 16-byte padding */
-    EP_DEC_BAD_TILE = 16u     /* a tile directory entry points outside the tile section */
+    EP_DEC_BAD_TILE = 16u,    /* a tile directory entry points outside the tile section */
+    EP_DEC_TIMEOUT = 32u      /* a staging copy into shared memory did not complete within the
+                                 kernel's poll limit; the CTA's remaining tiles are skipped */
 };
 
 typedef struct {

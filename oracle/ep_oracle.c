@@ -29,24 +29,33 @@
 #include <string.h>
 
 /* ------------------------------------------------------------------------------------
- * Stream constants (format version 1).  These are the build's readings of what the
- * pages leave open: 11-bit frequency tables, 32-bit states with 16-bit renormalisation
- * words, 32 interleaved states per tile, seven coding contexts.
+ * Stream constants (format version 3).  These are the build's readings of what the
+ * pages leave open: 11-bit frequency tables (every frequency below 2^11), 32-bit states
+ * with 16-bit renormalisation words, 32 interleaved states per tile, seven coding
+ * contexts, hybrid-integer tokens with 2 bits below the leading one and a per-context
+ * number of low bits kept in the token, raw extra bits in a separate stream per tile.
  * ---------------------------------------------------------------------------------- */
 #define MAGIC 0x31545045u /* bytes 'E','P','T','1' */
-#define VERSION 2
+#define VERSION 3
 #define PROB_BITS 11
 #define PROB_M 2048u
 #define STATE_L 65536u
 #define LANES 32
 #define NCTX 7
-#define MAX_SPLIT 7
-#define CHUNK_BITS 11
+#define H_BITS 2             /* bits below the leading one carried by an escape token */
+#define VALUE_BITS 22        /* every symbol value is below 2^22 */
 #define HEADER_BYTES 64
 #define TILE_HEAD 192        /* 32 states (u32) + 32 word counts (u16) */
 #define TILE_BUDGET 5952.0   /* expected payload bytes a tile may hold (a 6 KB staging buffer) */
 #define NQ 1280
 #define SAMPLE_TARGET 65536
+
+/* low bits of the value kept inside every token, and the largest split, per context:
+ * coordinate 0 keeps v0 mod 4 (coset and the parity of y0), coordinates 1..6 keep the parity
+ * of y_i, coordinate 7 keeps nothing.  The largest splits keep every directly coded
+ * coordinate within |v| <= 256. */
+static const int32_t CTX_LOW[NCTX] = {2, 1, 1, 0, 0, 0, 0};
+static const int32_t CTX_MAX_SPLIT[NCTX] = {9, 8, 8, 7, 7, 7, 7};
 
 static size_t al16(size_t n) { return (n + 15) & ~(size_t)15; }
 
@@ -268,108 +277,149 @@ uint32_t or_zigzag(int32_t y) { return y >= 0 ? 2u * (uint32_t)y : 2u * (uint32_
 
 int32_t or_unzigzag(uint32_t u) { return (u & 1u) ? -(int32_t)((u + 1u) / 2u) : (int32_t)(u / 2u); }
 
-/* Conditional model (reading of [ABS] "conditional probability model of lattice
- * coordinates"): the coordinates of one block are coded in order 0..7.
- *   coordinate 0: context 0, symbol zigzag(v0); its parity is the coset c.
- *   coordinates 1..6: context 1 + c, symbol zigzag(y_i) with y_i = (v_i - c) / 2.
- *   coordinate 7: context 3 + 2c + p, p = (y_0 + ... + y_6) mod 2.  E8 forces
- *     y_7 = p (mod 2), so the symbol is zigzag((y_7 - p) / 2). */
-static void block_symbols(const int32_t *v, uint32_t *ctx, uint32_t *u)
+/* a mod b in [0, b) for b > 0 (C's % truncates toward zero) */
+static int32_t mod_floor(int32_t a, int32_t b)
 {
-    int32_t c = (v[0] % 2 != 0) ? 1 : 0;
+    int32_t r = a % b;
+    return r < 0 ? r + b : r;
+}
+
+/* Conditional model (reading of [ABS] "conditional probability model of lattice
+ * coordinates"): the coordinates of one block v = 2z are coded in order 0..7.  The coset is
+ * c = v0 mod 2 and y_i = (v_i - c) / 2; p = (y_0 + ... + y_6) mod 2.
+ *   coordinate 0: context 0, value 4 zigzag(a0) + r0 with v0 = 4 a0 + r0, r0 in [0, 4):
+ *     its two low bits are the coset and the parity of y_0.
+ *   coordinates 1..6: context 1 + c, value 2 zigzag(a) + b with y_i = 2 a + b, b in {0, 1}:
+ *     its low bit is the parity of y_i.
+ *   coordinate 7: context 3 + 2c + p.  E8 forces y_7 = p (mod 2), so the value is
+ *     zigzag((y_7 - p) / 2).
+ * The low bits named here are kept by every token (or_tokenize), so the contexts of a block
+ * follow from its tokens alone. */
+void or_block_symbols(const int32_t *v, uint32_t *ctx, uint32_t *s)
+{
+    int32_t c = mod_floor(v[0], 2);
     int32_t y[8], p = 0;
     for (int i = 0; i < 8; i++)
         y[i] = (v[i] - c) / 2; /* exact: v_i - c is even */
     for (int i = 0; i < 7; i++)
-        p ^= (y[i] % 2 != 0) ? 1 : 0;
+        p = mod_floor(p + y[i], 2);
+    int32_t r0 = mod_floor(v[0], 4);
     ctx[0] = 0;
-    u[0] = or_zigzag(v[0]);
+    s[0] = 4u * or_zigzag((v[0] - r0) / 4) + (uint32_t)r0;
     for (int i = 1; i < 7; i++) {
+        int32_t b = mod_floor(y[i], 2);
         ctx[i] = 1u + (uint32_t)c;
-        u[i] = or_zigzag(y[i]);
+        s[i] = 2u * or_zigzag((y[i] - b) / 2) + (uint32_t)b;
     }
     ctx[7] = 3u + 2u * (uint32_t)c + (uint32_t)p;
-    u[7] = or_zigzag((y[7] - p) / 2);
+    s[7] = or_zigzag((y[7] - p) / 2);
 }
 
-/* Token binarization ("hybrid integer"): with split m and h = min(m, 2), a value
- * u < 2^m is its own token; otherwise, with n = floor(log2 u), the token carries n and
- * the h bits below the leading one, and the remaining n - h low bits travel as raw
- * extra bits. */
-void or_tokenize(uint32_t u, int32_t m, uint32_t *tok, uint32_t *nbits, uint32_t *extra)
+/* Inverse of or_block_symbols for one block, coordinate by coordinate in coding order:
+ * returns v and the context of every coordinate. */
+void or_block_values(const uint32_t *s, int32_t *v, uint32_t *ctx)
 {
-    uint32_t h = (uint32_t)(m < 2 ? m : 2);
-    if (u < (1u << m)) {
-        *tok = u;
+    int32_t r0 = (int32_t)(s[0] % 4u);
+    v[0] = 4 * or_unzigzag(s[0] / 4u) + r0;
+    int32_t c = mod_floor(v[0], 2);
+    int32_t p = mod_floor((v[0] - c) / 2, 2);
+    ctx[0] = 0;
+    for (int i = 1; i < 7; i++) {
+        int32_t y = 2 * or_unzigzag(s[i] / 2u) + (int32_t)(s[i] % 2u);
+        v[i] = 2 * y + c;
+        p = mod_floor(p + y, 2);
+        ctx[i] = 1u + (uint32_t)c;
+    }
+    int32_t y7 = 2 * or_unzigzag(s[7]) + p;
+    v[7] = 2 * y7 + c;
+    ctx[7] = 3u + 2u * (uint32_t)c + (uint32_t)p;
+}
+
+static uint32_t floor_log2(uint32_t u)
+{
+    uint32_t n = 0;
+    while ((u >> (n + 1)) != 0)
+        n++;
+    return n;
+}
+
+/* Token binarization ("hybrid integer", with low bits kept): with split m, h = 2 and `low`
+ * kept bits (m >= h + low), a value s < 2^m is its own token.  Otherwise, with
+ * n = floor(log2 s), the token carries n, the h bits below the leading one and the `low`
+ * lowest bits of s; the n - h - low bits in between travel as raw extra bits. */
+void or_tokenize(uint32_t s, int32_t m, int32_t low, uint32_t *tok, uint32_t *nbits, uint32_t *extra)
+{
+    if (s < (1u << m)) {
+        *tok = s;
         *nbits = 0;
         *extra = 0;
         return;
     }
-    uint32_t n = 0;
-    while ((u >> (n + 1)) != 0)
-        n++;
-    uint32_t top = (u >> (n - h)) & ((1u << h) - 1u);
-    *tok = (1u << m) + ((n - (uint32_t)m) << h) + top;
-    *nbits = n - h;
-    *extra = u & ((1u << (n - h)) - 1u);
+    uint32_t n = floor_log2(s);
+    uint32_t top = (s >> (n - H_BITS)) & ((1u << H_BITS) - 1u);
+    uint32_t lo = s & ((1u << low) - 1u);
+    *nbits = n - H_BITS - (uint32_t)low;
+    *extra = (s >> low) & ((1u << *nbits) - 1u);
+    *tok = (1u << m) + (((((n - (uint32_t)m) << H_BITS) | top) << low) | lo);
 }
 
-uint32_t or_detokenize(uint32_t tok, int32_t m, uint32_t extra)
+/* raw extra bits that follow a token */
+static uint32_t token_extra_bits(uint32_t tok, int32_t m, int32_t low)
 {
-    uint32_t h = (uint32_t)(m < 2 ? m : 2);
+    if (tok < (1u << m))
+        return 0;
+    uint32_t n = (uint32_t)m + (((tok - (1u << m)) >> low) >> H_BITS);
+    return n - H_BITS - (uint32_t)low;
+}
+
+uint32_t or_detokenize(uint32_t tok, int32_t m, int32_t low, uint32_t extra)
+{
     if (tok < (1u << m))
         return tok;
     uint32_t d = tok - (1u << m);
-    uint32_t n = (uint32_t)m + (d >> h);
-    uint32_t top = (1u << h) | (d & ((1u << h) - 1u));
-    return (top << (n - h)) | extra;
+    uint32_t lo = d & ((1u << low) - 1u), q = d >> low;
+    uint32_t top = q & ((1u << H_BITS) - 1u);
+    uint32_t n = (uint32_t)m + (q >> H_BITS);
+    return (((1u << H_BITS) | top) << (n - H_BITS)) | (extra << low) | lo;
 }
 
-void or_detokenize_batch(const uint32_t *tok, int64_t n, int32_t m, const uint32_t *extra, uint32_t *u)
+void or_detokenize_batch(const uint32_t *tok, int64_t n, int32_t m, int32_t low, const uint32_t *extra,
+                         uint32_t *s)
 {
     for (int64_t i = 0; i < n; i++)
-        u[i] = or_detokenize(tok[i], m, extra[i]);
+        s[i] = or_detokenize(tok[i], m, low, extra[i]);
 }
 
-static void token_bits(uint32_t tok, int32_t m, uint32_t *nbits)
+/* number of tokens a split can produce for values below 2^VALUE_BITS */
+uint32_t or_alphabet_size(int32_t m, int32_t low)
 {
-    uint32_t h = (uint32_t)(m < 2 ? m : 2);
-    if (tok < (1u << m)) {
-        *nbits = 0;
-        return;
-    }
-    uint32_t n = (uint32_t)m + ((tok - (1u << m)) >> h);
-    *nbits = n - h;
+    return (1u << m) + ((((uint32_t)(VALUE_BITS - m)) << H_BITS) << low);
 }
 
-/* number of tokens a split can produce for values below 2^22 */
-static uint32_t max_tokens(int32_t m)
-{
-    uint32_t h = (uint32_t)(m < 2 ? m : 2);
-    return (1u << m) + ((22u - (uint32_t)m) << h);
-}
-
-void or_tokenize_batch(const uint32_t *u, int64_t n, int32_t m, uint32_t *tok, uint32_t *nbits, uint32_t *extra)
+void or_tokenize_batch(const uint32_t *s, int64_t n, int32_t m, int32_t low, uint32_t *tok, uint32_t *nbits,
+                       uint32_t *extra)
 {
     for (int64_t i = 0; i < n; i++)
-        or_tokenize(u[i], m, tok + i, nbits + i, extra + i);
+        or_tokenize(s[i], m, low, tok + i, nbits + i, extra + i);
 }
 
-/* split: smallest m in [0, 7] with at least 99.9% of the context's values below 2^m */
-static int32_t choose_split(const uint64_t *bitlen_hist /* [24]: count by bit length */)
+/* split of context c: the smallest m in [h + low, max split] with at least 99.9% of the
+ * context's values below 2^m, else the largest split */
+static int32_t choose_split(const uint64_t *bitlen_hist /* [VALUE_BITS + 1]: count by bit length */, int c)
 {
+    int32_t lo = H_BITS + CTX_LOW[c], hi = CTX_MAX_SPLIT[c];
     uint64_t n = 0;
-    for (int i = 0; i < 24; i++)
+    for (int i = 0; i <= VALUE_BITS; i++)
         n += bitlen_hist[i];
     if (n == 0)
-        return 0;
+        return lo;
     uint64_t below = 0;
-    for (int32_t m = 0; m <= MAX_SPLIT; m++) {
+    for (int32_t m = 0; m <= hi; m++) {
         below += bitlen_hist[m]; /* values with bit length m are below 2^m */
-        if (below * 1000u >= n * 999u)
+        if (m >= lo && below * 1000u >= n * 999u)
             return m;
     }
-    return MAX_SPLIT;
+    return hi;
 }
 
 static int bit_length(uint32_t u)
@@ -386,8 +436,10 @@ static int bit_length(uint32_t u)
 /* Counts -> frequencies summing to M = 2^11 by largest remainders: f_i = floor(c_i M / n);
  * the M - sum f_i leftover units go one each to the largest remainders (c_i M mod n),
  * lower index first on ties; then every seen token left at 0 is raised to 1 by taking a
- * unit from the currently largest frequency (lower index first on ties).  A context
- * with one token gets f = M.  Returns the table length (last seen token + 1). */
+ * unit from the currently largest frequency (lower index first on ties).  Every frequency
+ * stays below M: a context with one seen token t gives it M - 1 and one unit to a phantom
+ * token that never occurs (token 1 if t = 0, else token 0).  Returns the table length (last
+ * token with f > 0, plus 1), or -1 for a single-token alphabet. */
 int32_t or_normalize_freqs(const uint64_t *counts, int32_t n, uint32_t *f)
 {
     uint64_t total = 0;
@@ -432,6 +484,21 @@ int32_t or_normalize_freqs(const uint64_t *counts, int32_t n, uint32_t *f)
     }
     free(rem);
     free(given);
+    int32_t seen = 0, only = 0;
+    for (int32_t i = 0; i < n; i++)
+        if (counts[i]) {
+            seen++;
+            only = i;
+        }
+    if (seen == 1) {
+        if (n < 2)
+            return -1;
+        int32_t phantom = only == 0 ? 1 : 0;
+        f[only] = PROB_M - 1u;
+        f[phantom] = 1;
+        if (phantom + 1 > len)
+            len = phantom + 1;
+    }
     return len;
 }
 
@@ -596,7 +663,7 @@ static size_t meta_bytes(int64_t rows, int32_t container, uint64_t total_tokens,
  * plus its raw extra bits, scaled by nb / n_sample.  Exact metadata is added, the table
  * length taken from the sample, plus 168 bytes per tile: a final state holds about 24 bits
  * that carry no payload (32 lanes x 3 bytes), the 32 word counts take 64 bytes and a tile
- * pads to 16 bytes (8 on average). */
+ * pads to 16 bytes (8 on average; the raw bits' last word is counted in that padding). */
 static double estimate_bpp(const double *w, const float *s, int64_t rows, int64_t cols, int32_t container,
                            int32_t k, uint32_t K)
 {
@@ -607,26 +674,26 @@ static double estimate_bpp(const double *w, const float *s, int64_t rows, int64_
     int64_t ns = (nb + S - 1) / S;
     uint32_t *ctx = (uint32_t *)malloc((size_t)ns * 8 * sizeof(uint32_t));
     uint32_t *u = (uint32_t *)malloc((size_t)ns * 8 * sizeof(uint32_t));
-    uint64_t hist[NCTX][24];
+    uint64_t hist[NCTX][VALUE_BITS + 2];
     memset(hist, 0, sizeof hist);
     for (int64_t j = 0; j < ns; j++) {
         int64_t b = j * S;
         int32_t v[8];
         quantize_block(w + 8 * b, row_factor(s[b / cb], k), v);
-        block_symbols(v, ctx + 8 * j, u + 8 * j);
+        or_block_symbols(v, ctx + 8 * j, u + 8 * j);
         for (int i = 0; i < 8; i++)
             hist[ctx[8 * j + i]][bit_length(u[8 * j + i])]++;
     }
     int32_t m[NCTX];
     uint64_t *cnt[NCTX];
     for (int c = 0; c < NCTX; c++) {
-        m[c] = choose_split(hist[c]);
-        cnt[c] = (uint64_t *)calloc(max_tokens(m[c]), sizeof(uint64_t));
+        m[c] = choose_split(hist[c], c);
+        cnt[c] = (uint64_t *)calloc(or_alphabet_size(m[c], CTX_LOW[c]), sizeof(uint64_t));
     }
     double extra = 0.0;
     for (int64_t i = 0; i < ns * 8; i++) {
         uint32_t t, nbits, ex;
-        or_tokenize(u[i], m[ctx[i]], &t, &nbits, &ex);
+        or_tokenize(u[i], m[ctx[i]], CTX_LOW[ctx[i]], &t, &nbits, &ex);
         cnt[ctx[i]][t]++;
         extra += (double)nbits;
     }
@@ -635,7 +702,7 @@ static double estimate_bpp(const double *w, const float *s, int64_t rows, int64_
     for (int c = 0; c < NCTX; c++) {
         uint64_t n = 0;
         uint32_t len = 0;
-        for (uint32_t t = 0; t < max_tokens(m[c]); t++) {
+        for (uint32_t t = 0; t < or_alphabet_size(m[c], CTX_LOW[c]); t++) {
             n += cnt[c][t];
             if (cnt[c][t])
                 len = t + 1;
@@ -644,7 +711,7 @@ static double estimate_bpp(const double *w, const float *s, int64_t rows, int64_
         if (n == 0)
             continue;
         bits += (double)n * log2((double)n);
-        for (uint32_t t = 0; t < max_tokens(m[c]); t++)
+        for (uint32_t t = 0; t < or_alphabet_size(m[c], CTX_LOW[c]); t++)
             if (cnt[c][t])
                 bits -= (double)cnt[c][t] * log2((double)cnt[c][t]);
     }
@@ -698,7 +765,6 @@ static uint64_t get64(const uint8_t *p) { return (uint64_t)get32(p) | ((uint64_t
 
 /* ---------------------------------- tile encoder ------------------------------------- */
 typedef struct {
-    uint8_t lane;
     uint16_t f, cum;
 } event;
 
@@ -721,60 +787,70 @@ static void bytes_put(bytes *b, const void *src, size_t n)
 }
 
 /* Decode order inside a tile (the rule both sides follow): the 32 lanes are independent
- * rANS coders, each with its own word stream.  Lane l decodes its blocks t*32K + 32k + l in
- * order of k; per block the 8 coordinates in order; per coordinate its token, then the chunks
- * of its raw extra bits (at most 11 bits each, least significant first, each a uniform
- * symbol).  After every symbol the lane reads one 16-bit word from its own stream if its
- * state fell below L.  The encoder runs a lane's symbols in reverse, emitting words in
+ * rANS coders, each with its own region of 16-bit words.  Lane l decodes its blocks
+ * t*32K + 32k + l in order of k, and per block the tokens of coordinates 0..7 in order;
+ * after every token the lane reads the next word from the front of its region if its state
+ * fell below L.  After a block's 8 tokens the lane takes the raw extra bits of the block's
+ * escape tokens, coordinate by coordinate, from the back of its region: the region's last
+ * word holds the lane's first 16 raw bits (least significant bit first), the word before it
+ * the next 16, and so on.  The encoder runs a lane's tokens in reverse, emitting words in
  * reverse.  A tile stores the 32 final encoder states (= initial decoder states, u32), the
- * 32 word counts (u16), then the word streams of lanes 0..31 one after another, each in the
- * order the decoder reads it, zero padded to 16 bytes. */
-static void encode_tile(const uint32_t *ctx, const uint32_t *u, int64_t nb, int64_t t, uint32_t K,
-                        const int32_t *m, uint32_t *const *freq, uint32_t *const *cum, bytes *out)
+ * 32 region lengths in words (u16), then the regions of lanes 0..31 one after another, zero
+ * padded to 16 bytes. */
+static int encode_tile(const uint32_t *ctx, const uint32_t *s, int64_t nb, int64_t t, uint32_t K,
+                       const int32_t *m, uint32_t *const *freq, uint32_t *const *cum, bytes *out)
 {
     int64_t base = t * (int64_t)LANES * K;
-    size_t cap = (size_t)K * 8 * 3;
-    event *ev = (event *)malloc(cap * sizeof(event));
+    event *ev = (event *)malloc((size_t)K * 8 * sizeof(event));
+    uint8_t *raw = (uint8_t *)malloc((size_t)K * 8 * VALUE_BITS + 16);
     uint16_t *words[LANES];
     size_t nw[LANES];
     uint32_t x[LANES];
+    int rc = OR_OK;
     for (int l = 0; l < LANES; l++) {
-        size_t ne = 0;
+        size_t ne = 0, nraw = 0;
         for (uint32_t k = 0; k < K; k++) {
             int64_t b = base + (int64_t)k * LANES + l;
             if (b >= nb)
                 break;
             for (int i = 0; i < 8; i++) {
                 uint32_t c = ctx[8 * b + i], tok, nbits, extra;
-                or_tokenize(u[8 * b + i], m[c], &tok, &nbits, &extra);
-                ev[ne].lane = (uint8_t)l;
+                or_tokenize(s[8 * b + i], m[c], CTX_LOW[c], &tok, &nbits, &extra);
                 ev[ne].f = (uint16_t)freq[c][tok];
                 ev[ne].cum = (uint16_t)cum[c][tok];
                 ne++;
-                for (uint32_t j = 0; CHUNK_BITS * j < nbits; j++) {
-                    uint32_t left = nbits - CHUNK_BITS * j;
-                    uint32_t bits = left < CHUNK_BITS ? left : CHUNK_BITS;
-                    uint32_t val = (extra >> (CHUNK_BITS * j)) & ((1u << bits) - 1u);
-                    ev[ne].lane = (uint8_t)l;
-                    ev[ne].f = (uint16_t)(1u << (PROB_BITS - bits));
-                    ev[ne].cum = (uint16_t)(val << (PROB_BITS - bits));
-                    ne++;
-                }
+                for (uint32_t j = 0; j < nbits; j++)
+                    raw[nraw++] = (uint8_t)((extra >> j) & 1u);
             }
         }
-        words[l] = (uint16_t *)malloc((ne + 1) * sizeof(uint16_t));
+        size_t nrawords = (nraw + 15) / 16;
+        words[l] = (uint16_t *)malloc((ne + nrawords + 1) * sizeof(uint16_t));
         nw[l] = 0;
-        uint32_t s = STATE_L;
+        uint32_t st = STATE_L;
+        uint16_t *rw = (uint16_t *)malloc((nrawords + 1) * sizeof(uint16_t));
+        for (size_t j = 0; j < nrawords; j++) {
+            uint32_t wd = 0;
+            for (size_t q = 0; q < 16 && 16 * j + q < nraw; q++)
+                wd |= (uint32_t)raw[16 * j + q] << q;
+            rw[j] = (uint16_t)wd;
+        }
+        /* words[l] collects the region back to front: raw word 0 first, ..., then the rANS
+         * words in the order the encoder emits them (the reverse of decode order) */
+        for (size_t j = 0; j < nrawords; j++)
+            words[l][nw[l]++] = rw[j];
+        free(rw);
         for (size_t e = ne; e-- > 0;) {
             uint32_t f = ev[e].f;
             /* renormalise so that the encoded state stays below 2^32: x_max = (L >> 11) << 16 * f */
-            if ((uint64_t)s >= ((uint64_t)f << 21)) {
-                words[l][nw[l]++] = (uint16_t)(s & 0xffffu);
-                s >>= 16;
+            if ((uint64_t)st >= ((uint64_t)f << 21)) {
+                words[l][nw[l]++] = (uint16_t)(st & 0xffffu);
+                st >>= 16;
             }
-            s = ((s / f) << PROB_BITS) + (s % f) + ev[e].cum;
+            st = ((st / f) << PROB_BITS) + (st % f) + ev[e].cum;
         }
-        x[l] = s;
+        x[l] = st;
+        if (nw[l] > 0xffffu)
+            rc = OR_ERR_UNSUPPORTED;
     }
     uint8_t head[TILE_HEAD];
     for (int l = 0; l < LANES; l++) {
@@ -794,6 +870,8 @@ static void encode_tile(const uint32_t *ctx, const uint32_t *u, int64_t nb, int6
     size_t pad = al16(out->n) - out->n;
     bytes_put(out, zeros, pad);
     free(ev);
+    free(raw);
+    return rc;
 }
 
 /* ---------------------------------- full encode at one k ----------------------------- */
@@ -809,35 +887,36 @@ static int encode_at(const double *w, const float *s, const float *scales, int64
         return OR_ERR_INVALID_ARG;
     for (int64_t r = 0; r < rows; r++)
         f[r] = row_factor(s[r], k);
-    uint64_t hist[NCTX][24];
+    uint64_t hist[NCTX][VALUE_BITS + 2];
     memset(hist, 0, sizeof hist);
     for (int64_t b = 0; b < nb; b++) {
         int32_t v[8];
         quantize_block(w + 8 * b, f[b / cb], v);
-        block_symbols(v, ctx + 8 * b, u + 8 * b);
+        or_block_symbols(v, ctx + 8 * b, u + 8 * b);
         for (int i = 0; i < 8; i++)
             hist[ctx[8 * b + i]][bit_length(u[8 * b + i])]++;
     }
     int32_t m[NCTX];
     uint32_t *freq[NCTX], *cum[NCTX];
     uint64_t *cnt[NCTX];
-    uint32_t ntok[NCTX];
+    uint32_t ntok[NCTX], alpha[NCTX];
     uint64_t total_tokens = 0;
     for (int c = 0; c < NCTX; c++) {
-        m[c] = choose_split(hist[c]);
-        cnt[c] = (uint64_t *)calloc(max_tokens(m[c]), sizeof(uint64_t));
-        freq[c] = (uint32_t *)calloc(max_tokens(m[c]), sizeof(uint32_t));
-        cum[c] = (uint32_t *)calloc(max_tokens(m[c]), sizeof(uint32_t));
+        m[c] = choose_split(hist[c], c);
+        alpha[c] = or_alphabet_size(m[c], CTX_LOW[c]);
+        cnt[c] = (uint64_t *)calloc(alpha[c], sizeof(uint64_t));
+        freq[c] = (uint32_t *)calloc(alpha[c], sizeof(uint32_t));
+        cum[c] = (uint32_t *)calloc(alpha[c], sizeof(uint32_t));
     }
     for (int64_t i = 0; i < nb * 8; i++) {
         uint32_t t, nbits, ex;
-        or_tokenize(u[i], m[ctx[i]], &t, &nbits, &ex);
+        or_tokenize(u[i], m[ctx[i]], CTX_LOW[ctx[i]], &t, &nbits, &ex);
         cnt[ctx[i]][t]++;
     }
     for (int c = 0; c < NCTX; c++) {
-        ntok[c] = (uint32_t)or_normalize_freqs(cnt[c], (int32_t)max_tokens(m[c]), freq[c]);
+        ntok[c] = (uint32_t)or_normalize_freqs(cnt[c], (int32_t)alpha[c], freq[c]);
         uint32_t a = 0;
-        for (uint32_t t = 0; t < max_tokens(m[c]); t++) {
+        for (uint32_t t = 0; t < alpha[c]; t++) {
             cum[c][t] = a;
             a += freq[c][t];
         }
@@ -846,9 +925,11 @@ static int encode_at(const double *w, const float *s, const float *scales, int64
     uint32_t T = (uint32_t)((nb + (int64_t)LANES * K - 1) / ((int64_t)LANES * K));
     bytes tiles = {0, 0, 0};
     uint32_t *dir = (uint32_t *)malloc(((size_t)T + 1) * sizeof(uint32_t));
+    int trc = OR_OK;
     for (uint32_t t = 0; t < T; t++) {
         dir[t] = (uint32_t)(tiles.n / 16);
-        encode_tile(ctx, u, nb, t, K, m, freq, cum, &tiles);
+        if (encode_tile(ctx, u, nb, t, K, m, freq, cum, &tiles) != OR_OK)
+            trc = OR_ERR_UNSUPPORTED;
     }
     dir[T] = (uint32_t)(tiles.n / 16);
 
@@ -858,9 +939,11 @@ static int encode_at(const double *w, const float *s, const float *scales, int64
     size_t off_dir = off_freq + al16((size_t)total_tokens * 2);
     size_t off_tiles = off_dir + al16(((size_t)T + 1) * 4);
     size_t total = off_tiles + tiles.n;
-    int rc = OR_OK;
+    int rc = trc;
     *out_n = total;
-    if (total > cap || !out) {
+    if (rc != OR_OK) {
+        /* a lane region longer than 65535 words (only reachable with a forced tile size) */
+    } else if (total > cap || !out) {
         rc = OR_ERR_BUFFER_TOO_SMALL;
     } else {
         memset(out, 0, total);
@@ -959,6 +1042,8 @@ int or_compress(const void *src, int32_t sdt, int64_t rows, int64_t cols, double
     for (;;) {
         size_t n = 0;
         rc = encode_at(w, s, scales, rows, cols, sdt, container, k, K, NULL, 0, &n);
+        if (rc == OR_ERR_UNSUPPORTED)
+            break;
         if (q_override >= 0 || 8.0 * (double)n <= target * (double)(rows * cols)) {
             rc = encode_at(w, s, scales, rows, cols, sdt, container, k, K, out, cap, out_n);
             break;
@@ -1005,7 +1090,8 @@ int or_parse(const uint8_t *p, size_t n, or_info *info)
     for (int c = 0; c < NCTX; c++) {
         info->split[c] = p[36 + c];
         info->ntok[c] = (uint16_t)get16(p + 44 + 2 * c);
-        if (info->split[c] > MAX_SPLIT || info->ntok[c] > max_tokens(info->split[c]))
+        if (info->split[c] < H_BITS + CTX_LOW[c] || info->split[c] > CTX_MAX_SPLIT[c] ||
+            info->ntok[c] > or_alphabet_size(info->split[c], CTX_LOW[c]))
             return OR_ERR_CORRUPT;
         total_tokens += info->ntok[c];
     }
@@ -1016,12 +1102,15 @@ int or_parse(const uint8_t *p, size_t n, or_info *info)
     info->off_tiles = info->off_dir + al16(((size_t)T + 1) * 4);
     if (info->off_tiles > n)
         return OR_ERR_CORRUPT;
-    /* tables sum to M */
+    /* tables sum to M, every frequency below M */
     size_t q = info->off_freq;
     for (int c = 0; c < NCTX; c++) {
         uint32_t sum = 0;
-        for (uint32_t t = 0; t < info->ntok[c]; t++, q += 2)
+        for (uint32_t t = 0; t < info->ntok[c]; t++, q += 2) {
+            if (get16(p + q) >= PROB_M)
+                return OR_ERR_CORRUPT;
             sum += get16(p + q);
+        }
         if (info->ntok[c] && sum != PROB_M)
             return OR_ERR_CORRUPT;
     }
@@ -1121,8 +1210,32 @@ static void dec_renorm(uint32_t *x, const uint8_t *wp, uint64_t nwords, uint64_t
     *x = (*x << 16) | wd;
 }
 
-/* Decodes tile t lane by lane, each lane an independent coder over its own word stream
- * (the order written down at encode_tile). */
+/* a lane's raw extra bits: 16-bit words taken from the back of its region, each read least
+ * significant bit first */
+typedef struct {
+    const uint8_t *region; /* the lane's first word */
+    uint64_t len;          /* region length in words (as stored; may exceed the tile if damaged) */
+    uint64_t avail;        /* words of the region inside the tile */
+    uint64_t bit;          /* raw bits read so far */
+} raw_reader;
+
+static uint32_t raw_read(raw_reader *R, uint32_t nbits, uint32_t *status)
+{
+    uint32_t v = 0;
+    for (uint32_t j = 0; j < nbits; j++, R->bit++) {
+        uint64_t back = R->bit / 16; /* 0 = the region's last word */
+        uint32_t bitv = 0;
+        if (back < R->len && R->len - 1 - back < R->avail)
+            bitv = (get16(R->region + 2 * (R->len - 1 - back)) >> (R->bit % 16)) & 1u;
+        else
+            *status |= OR_DEC_WORD_OVERRUN;
+        v |= bitv << j;
+    }
+    return v;
+}
+
+/* Decodes tile t lane by lane in the order written down at encode_tile: each lane's tokens
+ * from the front of its region, its raw extra bits from the back. */
 static void decode_tile(dec_ctx *D, int64_t t, int32_t *vout, void *out, uint32_t *status, code_stats *cs)
 {
     const or_info *I = &D->in;
@@ -1136,56 +1249,53 @@ static void decode_tile(dec_ctx *D, int64_t t, int32_t *vout, void *out, uint32_
     int esz = elt_size(I->container_dtype);
     for (int l = 0; l < LANES; l++) {
         uint32_t x = get32(tp + 4 * l);
-        uint64_t nwords = get16(tp + 4 * LANES + 2 * l), pos = 0;
+        uint64_t len = get16(tp + 4 * LANES + 2 * l), pos = 0;
         const uint8_t *wp = tp + TILE_HEAD + 2 * start;
-        if (start + nwords > capacity) {
+        uint64_t avail = start < capacity ? capacity - start : 0;
+        if (avail > len)
+            avail = len;
+        if (start + len > capacity)
             *status |= OR_DEC_WORD_OVERRUN;
-            nwords = start < capacity ? capacity - start : 0;
-        }
-        start += get16(tp + 4 * LANES + 2 * l);
+        start += len;
+        raw_reader R = {wp, len, avail, 0};
         for (uint32_t k = 0; k < K; k++) {
             int64_t b = base + (int64_t)k * LANES + l;
             if (b >= nb)
                 break;
-            int32_t v[8], y[8], c = 0, p = 0;
+            uint32_t tok[8], ctx[8], sv[8];
+            int32_t c = 0, p = 0;
             for (int i = 0; i < 8; i++) {
-                uint32_t ctx = i == 0 ? 0u : i < 7 ? 1u + (uint32_t)c : 3u + 2u * (uint32_t)c + (uint32_t)p;
-                uint32_t tok = dec_token(D, ctx, &x, status, cs ? &cs->ideal : NULL), nbits, extra = 0;
-                dec_renorm(&x, wp, nwords, &pos, status);
-                token_bits(tok, I->split[ctx], &nbits);
+                ctx[i] = i == 0 ? 0u : i < 7 ? 1u + (uint32_t)c : 3u + 2u * (uint32_t)c + (uint32_t)p;
+                tok[i] = dec_token(D, ctx[i], &x, status, cs ? &cs->ideal : NULL);
+                dec_renorm(&x, wp, avail, &pos, status);
+                if (tok[i] >= I->ntok[ctx[i]])
+                    *status |= OR_DEC_BAD_TOKEN;
+                /* the value's low bits do not depend on the extra bits (they are in the token) */
+                uint32_t lowbits = or_detokenize(tok[i], I->split[ctx[i]], CTX_LOW[ctx[i]], 0);
+                if (i == 0) {
+                    c = (int32_t)(lowbits & 1u);
+                    p = (int32_t)((lowbits >> 1) & 1u);
+                } else if (i < 7) {
+                    p ^= (int32_t)(lowbits & 1u);
+                }
+            }
+            for (int i = 0; i < 8; i++) {
+                int32_t m = I->split[ctx[i]], low = CTX_LOW[ctx[i]];
+                uint32_t nbits = token_extra_bits(tok[i], m, low);
+                uint32_t extra = raw_read(&R, nbits, status);
+                sv[i] = or_detokenize(tok[i], m, low, extra);
                 if (cs) {
-                    cs->tokcount[ctx][tok]++;
+                    cs->tokcount[ctx[i]][tok[i] < I->ntok[ctx[i]] ? tok[i] : 0]++;
                     cs->extra += nbits;
                     cs->nsym++;
                 }
-                for (uint32_t j = 0; CHUNK_BITS * j < nbits; j++) {
-                    uint32_t left = nbits - CHUNK_BITS * j;
-                    uint32_t bits = left < CHUNK_BITS ? left : CHUNK_BITS;
-                    uint32_t f = 1u << (PROB_BITS - bits);
-                    uint32_t slot = x & (PROB_M - 1);
-                    uint32_t val = slot >> (PROB_BITS - bits);
-                    x = f * (x >> PROB_BITS) + slot - val * f;
-                    extra |= val << (CHUNK_BITS * j);
-                    dec_renorm(&x, wp, nwords, &pos, status);
-                }
-                /* inverse symbolization */
-                uint32_t uu = or_detokenize(tok, I->split[ctx], extra);
-                if (tok >= I->ntok[ctx])
-                    *status |= OR_DEC_BAD_TOKEN;
-                if (i == 0) {
-                    v[0] = or_unzigzag(uu);
-                    c = (v[0] % 2 != 0) ? 1 : 0;
-                    y[0] = (v[0] - c) / 2;
-                    p = (y[0] % 2 != 0) ? 1 : 0;
-                } else if (i < 7) {
-                    y[i] = or_unzigzag(uu);
-                    v[i] = 2 * y[i] + c;
-                    p ^= (y[i] % 2 != 0) ? 1 : 0;
-                } else {
-                    y[7] = 2 * or_unzigzag(uu) + p;
-                    v[7] = 2 * y[7] + c;
-                }
             }
+            int32_t v[8];
+            uint32_t ctx2[8];
+            or_block_values(sv, v, ctx2);
+            for (int i = 0; i < 8; i++)
+                if (ctx2[i] != ctx[i])
+                    *status |= OR_DEC_BAD_TOKEN;
             /* reconstruction: w = f_r * v in fp32, then the container conversion */
             int64_t r = b / cb;
             uint32_t fb = get32(D->rowf + 4 * r);
@@ -1202,8 +1312,10 @@ static void decode_tile(dec_ctx *D, int64_t t, int32_t *vout, void *out, uint32_
         }
         if (x != STATE_L)
             *status |= OR_DEC_BAD_END;
-        if (pos != nwords)
-            *status |= pos > nwords ? OR_DEC_WORD_OVERRUN : OR_DEC_WORD_COUNT;
+        /* the front reads and the back reads cover the region exactly */
+        uint64_t used = pos + (R.bit + 15) / 16;
+        if (used != len)
+            *status |= used > len ? OR_DEC_WORD_OVERRUN : OR_DEC_WORD_COUNT;
     }
     if (start > capacity || capacity - start >= 8)
         *status |= OR_DEC_WORD_COUNT;

@@ -48,7 +48,7 @@ enum {
 
 /* decode status bits (stream damage found while decoding a tile) */
 enum {
-    OR_DEC_WORD_OVERRUN = 1u,   /* a renormalisation read past the tile's words */
+    OR_DEC_WORD_OVERRUN = 1u,   /* a renormalisation or raw-bit read past the tile's words */
     OR_DEC_BAD_TOKEN = 2u,      /* a slot that maps to no token / token outside the table */
     OR_DEC_BAD_END = 4u,        /* a lane's final state differs from L */
     OR_DEC_WORD_COUNT = 8u      /* words left unread beyond the 16-byte padding */
@@ -74,10 +74,17 @@ void or_e8_nearest(const double *x, int32_t *v);
 void or_e8_nearest_batch(const double *x, int64_t nblocks, int32_t *v);
 uint32_t or_zigzag(int32_t y);
 int32_t or_unzigzag(uint32_t u);
-void or_tokenize(uint32_t u, int32_t m, uint32_t *tok, uint32_t *nbits, uint32_t *extra);
-uint32_t or_detokenize(uint32_t tok, int32_t m, uint32_t extra);
-void or_detokenize_batch(const uint32_t *tok, int64_t n, int32_t m, const uint32_t *extra, uint32_t *u);
-void or_tokenize_batch(const uint32_t *u, int64_t n, int32_t m, uint32_t *tok, uint32_t *nbits, uint32_t *extra);
+/* one block's contexts and values in coding order, and the inverse */
+void or_block_symbols(const int32_t *v, uint32_t *ctx, uint32_t *s);
+void or_block_values(const uint32_t *s, int32_t *v, uint32_t *ctx);
+/* hybrid-integer tokens with split m and `low` low bits kept in every token */
+void or_tokenize(uint32_t s, int32_t m, int32_t low, uint32_t *tok, uint32_t *nbits, uint32_t *extra);
+uint32_t or_detokenize(uint32_t tok, int32_t m, int32_t low, uint32_t extra);
+uint32_t or_alphabet_size(int32_t m, int32_t low);
+void or_detokenize_batch(const uint32_t *tok, int64_t n, int32_t m, int32_t low, const uint32_t *extra,
+                         uint32_t *s);
+void or_tokenize_batch(const uint32_t *s, int64_t n, int32_t m, int32_t low, uint32_t *tok, uint32_t *nbits,
+                       uint32_t *extra);
 int32_t or_normalize_freqs(const uint64_t *counts, int32_t n, uint32_t *freqs);
 uint32_t or_choose_blocks_per_lane(int64_t nblocks, double target_bpp);
 uint16_t or_bf16_from_float(float w);

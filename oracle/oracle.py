@@ -49,10 +49,14 @@ def lib():
         L.or_zigzag.argtypes = [C.c_int32]
         L.or_unzigzag.restype = C.c_int32
         L.or_unzigzag.argtypes = [C.c_uint32]
-        L.or_tokenize_batch.argtypes = [p, C.c_int64, C.c_int32, p, p, p]
+        L.or_tokenize_batch.argtypes = [p, C.c_int64, C.c_int32, C.c_int32, p, p, p]
         L.or_detokenize.restype = C.c_uint32
-        L.or_detokenize.argtypes = [C.c_uint32, C.c_int32, C.c_uint32]
-        L.or_detokenize_batch.argtypes = [p, C.c_int64, C.c_int32, p, p]
+        L.or_detokenize.argtypes = [C.c_uint32, C.c_int32, C.c_int32, C.c_uint32]
+        L.or_detokenize_batch.argtypes = [p, C.c_int64, C.c_int32, C.c_int32, p, p]
+        L.or_alphabet_size.restype = C.c_uint32
+        L.or_alphabet_size.argtypes = [C.c_int32, C.c_int32]
+        L.or_block_symbols.argtypes = [p, p, p]
+        L.or_block_values.argtypes = [p, p, p]
         L.or_normalize_freqs.restype = C.c_int32
         L.or_normalize_freqs.argtypes = [p, C.c_int32, p]
         L.or_choose_blocks_per_lane.restype = C.c_uint32
@@ -137,25 +141,51 @@ def unzigzag(u):
     return lib().or_unzigzag(int(u))
 
 
-def tokenize(u, m):
-    u = np.ascontiguousarray(u, dtype=np.uint32)
-    tok = np.zeros_like(u)
-    nb = np.zeros_like(u)
-    ex = np.zeros_like(u)
-    lib().or_tokenize_batch(_ptr(u), u.size, int(m), _ptr(tok), _ptr(nb), _ptr(ex))
+# low bits kept in every token, and the largest split, per context
+CTX_LOW = (2, 1, 1, 0, 0, 0, 0)
+CTX_MAX_SPLIT = (9, 8, 8, 7, 7, 7, 7)
+
+
+def tokenize(s, m, low):
+    s = np.ascontiguousarray(s, dtype=np.uint32)
+    tok = np.zeros_like(s)
+    nb = np.zeros_like(s)
+    ex = np.zeros_like(s)
+    lib().or_tokenize_batch(_ptr(s), s.size, int(m), int(low), _ptr(tok), _ptr(nb), _ptr(ex))
     return tok, nb, ex
 
 
-def detokenize(tok, m, extra):
-    return lib().or_detokenize(int(tok), int(m), int(extra))
+def detokenize(tok, m, low, extra):
+    return lib().or_detokenize(int(tok), int(m), int(low), int(extra))
 
 
-def detokenize_batch(tok, m, extra):
+def detokenize_batch(tok, m, low, extra):
     tok = np.ascontiguousarray(tok, dtype=np.uint32)
     extra = np.ascontiguousarray(extra, dtype=np.uint32)
-    u = np.zeros_like(tok)
-    lib().or_detokenize_batch(_ptr(tok), tok.size, int(m), _ptr(extra), _ptr(u))
-    return u
+    s = np.zeros_like(tok)
+    lib().or_detokenize_batch(_ptr(tok), tok.size, int(m), int(low), _ptr(extra), _ptr(s))
+    return s
+
+
+def alphabet_size(m, low):
+    return lib().or_alphabet_size(int(m), int(low))
+
+
+def block_symbols(v):
+    """contexts and coded values of one block of 8 lattice coordinates v = 2z"""
+    v = np.ascontiguousarray(v, dtype=np.int32)
+    ctx = np.zeros(8, np.uint32)
+    s = np.zeros(8, np.uint32)
+    lib().or_block_symbols(_ptr(v), _ptr(ctx), _ptr(s))
+    return ctx, s
+
+
+def block_values(s):
+    s = np.ascontiguousarray(s, dtype=np.uint32)
+    v = np.zeros(8, np.int32)
+    ctx = np.zeros(8, np.uint32)
+    lib().or_block_values(_ptr(s), _ptr(v), _ptr(ctx))
+    return v, ctx
 
 
 def normalize_freqs(counts):

@@ -64,8 +64,8 @@ def test_ragged_shapes_all_containers(oracle, container, shape, K):
 
 @pytest.mark.parametrize("target", [0.5, 1.0, 2.0, 3.5, 5.0, 8.0, 11.0])
 def test_rates(oracle, target):
-    """low rates (single-token contexts), mid rates, and high rates (most symbols carry raw
-    extra-bit chunks; outliers need two chunks)"""
+    """low rates (single-token contexts with a phantom token), mid rates, and high rates (many
+    escape tokens whose raw extra bits come from the back of the lane's region)"""
     w = synth.gaussian_outliers(256, 4096, seed=11)
     rc, blob = oracle.compress(w, target)
     assert rc == 0
@@ -152,13 +152,16 @@ def test_damaged_streams_flagged(oracle):
     assert int(status.item()) != 0
 
 
-@pytest.mark.parametrize("K,q", [(64, 900), (256, 760), (128, 1000)])
-def test_tiles_larger_than_staging_buffer(oracle, K, q):
-    """tiles above the kernel's 6 KB per-warp buffer are decoded in place from global memory"""
-    w = synth.gaussian_outliers(96, 4096, seed=K)
+@pytest.mark.parametrize("K,q", [(64, 900), (256, 760), (128, 1000), (1024, 900)])
+def test_large_tiles(oracle, K, q):
+    """tiles of tens of KB take fewer warps per CTA (their buffers fill shared memory); tiles
+    beyond every buffer (K = 1024 at ~8 bits, ~260 KB) are decoded in place from global memory"""
+    w = synth.gaussian_outliers(96, 4096, seed=K) if K < 1024 else synth.gaussian_outliers(128, 16384, seed=K)
     rc, blob = oracle.compress(w, 11.0, blocks_per_lane=K, q_override=q)
     assert rc == 0
     rc, info = oracle.parse(blob)
     sizes = np.diff(np.frombuffer(blob[info.off_dir: info.off_dir + 4 * (info.n_tiles + 1)].tobytes(), np.uint32))
     assert (16 * sizes > 6144).any()
+    if K == 1024:
+        assert (16 * sizes > 232448).any()
     check_parity(oracle, blob)

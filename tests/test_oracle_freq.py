@@ -1,6 +1,6 @@
 """Pins for the oracle's frequency tables: sums, support, the largest-remainder property
 (brute-forced as the least-squares apportionment on small alphabets), hand-worked golden
-examples."""
+examples, and the single-token rule (every frequency below M)."""
 import itertools
 import os
 
@@ -18,13 +18,13 @@ def test_golden(oracle):
         expect = [int(t) for t in b.split(":")[1].split()]
         f, n = oracle.normalize_freqs(counts)
         assert list(f) == expect
-        assert n == max(i + 1 for i, c in enumerate(counts) if c)
+        assert n == max(i + 1 for i, c in enumerate(expect) if c)
 
 
 def test_sum_and_support(oracle):
     rng = np.random.default_rng(0)
     for trial in range(300):
-        n = int(rng.integers(1, 200))
+        n = int(rng.integers(2, 200))
         kind = trial % 3
         if kind == 0:
             c = rng.integers(0, 1000, size=n)
@@ -36,9 +36,15 @@ def test_sum_and_support(oracle):
         if c.sum() == 0:
             c[0] = 1
         f, length = oracle.normalize_freqs(c)
-        assert f.sum() == M
-        assert np.array_equal(f > 0, c > 0)
-        assert length == np.flatnonzero(c).max() + 1
+        assert f.sum() == M and f.max() < M
+        if np.count_nonzero(c) == 1:  # the phantom token
+            only = int(np.flatnonzero(c)[0])
+            phantom = 1 if only == 0 else 0
+            assert f[only] == M - 1 and f[phantom] == 1 and np.count_nonzero(f) == 2
+            assert length == max(only, phantom) + 1
+        else:
+            assert np.array_equal(f > 0, c > 0)
+            assert length == np.flatnonzero(c).max() + 1
 
 
 def test_largest_remainder_is_least_squares(oracle):
@@ -59,3 +65,8 @@ def test_largest_remainder_is_least_squares(oracle):
                 best, arg = err, g
         assert abs(float(((f - q) ** 2).sum()) - best) < 1e-9, (c, f, arg)
         assert np.all(np.abs(f - q) < 1.0)
+
+
+def test_single_token_alphabet_rejected(oracle):
+    f, n = oracle.normalize_freqs([5])
+    assert n == -1
