@@ -205,16 +205,20 @@ def run_ours(a, rank, world, local_rank):
     outs = [torch.empty(info.shape, dtype=info.dtype, device=dev) for _ in range(ROTATE)]
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.Stream(dev)
+    # each device copy of the stream gets its slot tables once (ep_prepare), as when weights land
+    # on the device; every step then decodes with them
+    with torch.cuda.stream(stream):
+        works = [B.prepare(blobs[i], info, status=status, stream=stream) for i in range(ROTATE)]
     # first calls outside capture: sets the kernel attributes, checks the output
     with torch.cuda.stream(stream):
         for i in range(ROTATE):
-            B.decompress(blobs[i], info, out=outs[i], status=status, stream=stream)
+            B.decompress(blobs[i], info, workspace=works[i], out=outs[i], status=status, stream=stream)
     torch.cuda.synchronize(dev)
     assert int(status.item()) == 0, "decode reported stream damage"
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         for i in range(ROTATE):
-            B.decompress(blobs[i], info, out=outs[i], status=status, stream=stream)
+            B.decompress(blobs[i], info, workspace=works[i], out=outs[i], status=status, stream=stream)
     replays = max(1, -(-a.steps // ROTATE))
     steps = replays * ROTATE
     with torch.cuda.stream(stream):
@@ -248,25 +252,39 @@ def run_ours(a, rank, world, local_rank):
     achieved = (in_bytes + out_bytes) / kernel_s / 1e9
     traffic = traffic_for_kernel()
 
-    # end to end through the public API with host buffers: pinned H2D of the stream, decode,
-    # D2H of the container into pinned memory, every step
+    # the tables' preparation by itself (once per device copy of a stream)
+    prep_reps = 200
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        p0.record(stream)
+        for r in range(prep_reps):
+            B.prepare(blobs[r % ROTATE], info, workspace=works[r % ROTATE], stream=stream)
+        p1.record(stream)
+    torch.cuda.synchronize(dev)
+    prepare_us = p0.elapsed_time(p1) * 1e3 / prep_reps
+
+    # end to end through the public API with host buffers: pinned H2D of the stream, the tables,
+    # the decode, D2H of the container into pinned memory, every step
     host_blob = blob_cpu.pin_memory()
     host_out = torch.empty(info.shape, dtype=info.dtype).pin_memory()
     e2e_steps = max(8, min(200, a.steps // 200))
-    dblob, dout = blobs[0], outs[0]
+    dblob, dout, dwork = blobs[0], outs[0], works[0]
+
+    def e2e_step():
+        dblob.copy_(host_blob, non_blocking=True)
+        B.prepare(dblob, info, workspace=dwork, stream=stream)
+        B.decompress(dblob, info, workspace=dwork, out=dout, stream=stream)
+        host_out.copy_(dout, non_blocking=True)
+
     for _ in range(3):
         with torch.cuda.stream(stream):
-            dblob.copy_(host_blob, non_blocking=True)
-            B.decompress(dblob, info, out=dout, stream=stream)
-            host_out.copy_(dout, non_blocking=True)
+            e2e_step()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
         for _ in range(e2e_steps):
-            dblob.copy_(host_blob, non_blocking=True)
-            B.decompress(dblob, info, out=dout, stream=stream)
-            host_out.copy_(dout, non_blocking=True)
+            e2e_step()
         e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
@@ -294,6 +312,8 @@ def run_ours(a, rank, world, local_rank):
         "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": in_bytes,
                 "d2h_bytes_per_step": out_bytes},
         "gpu_launches": steps,
+        "tables": {"prepare_us": round(prepare_us, 3), "note": "slot tables built once per device copy of "
+                   "the stream (ep_prepare); each step stages them into shared memory and decodes"},
         "clocks": clk.summary(),
         "encode_s": round(t_enc, 3),
     }

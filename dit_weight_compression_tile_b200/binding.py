@@ -43,7 +43,7 @@ class StreamInfo(C.Structure):
         ("split", C.c_uint8 * 8), ("ntok", C.c_uint16 * 8),
         ("off_rowf", C.c_uint64), ("off_scales", C.c_uint64), ("off_freq", C.c_uint64),
         ("off_dir", C.c_uint64), ("off_tiles", C.c_uint64), ("out_nbytes", C.c_uint64),
-        ("max_tile_nbytes", C.c_uint64),
+        ("max_tile_nbytes", C.c_uint64), ("workspace_nbytes", C.c_uint64),
     ]
 
     @property
@@ -82,8 +82,10 @@ def lib():
                                        C.POINTER(C.c_size_t)]
         L.ep_stream_info.restype = C.c_int
         L.ep_stream_info.argtypes = [p, C.c_size_t, C.POINTER(StreamInfo)]
+        L.ep_prepare.restype = C.c_int
+        L.ep_prepare.argtypes = [C.POINTER(StreamInfo), p, p, p, p]
         L.ep_decompress.restype = C.c_int
-        L.ep_decompress.argtypes = [C.POINTER(StreamInfo), p, p, C.c_int32, p, p]
+        L.ep_decompress.argtypes = [C.POINTER(StreamInfo), p, p, p, C.c_int32, p, p]
         L.ep_status_string.restype = C.c_char_p
         L.ep_status_string.argtypes = [C.c_int]
         _lib = L
@@ -134,18 +136,43 @@ def stream_info(blob):
     return info
 
 
-def decompress(d_blob, info=None, out=None, status=None, stream=None, lattice=False):
+def prepare(d_blob, info=None, workspace=None, status=None, stream=None):
+    """The decoder's slot tables for one device copy of a stream (ep_prepare): run once when the
+    stream lands on the device.  Returns the workspace (CUDA uint8 tensor of
+    ``info.workspace_nbytes``), allocated here unless ``workspace`` is given."""
+    if not d_blob.is_cuda:
+        raise EpError(-1, "prepare needs the stream in device memory")
+    if info is None:
+        info = stream_info(d_blob.cpu())
+    if workspace is None:
+        workspace = torch.empty(info.workspace_nbytes, dtype=torch.uint8, device=d_blob.device)
+    if (not workspace.is_cuda or workspace.dtype != torch.uint8 or workspace.numel() < info.workspace_nbytes
+            or not workspace.is_contiguous()):
+        raise EpError(-1, "workspace does not match the stream")
+    st = status.data_ptr() if status is not None else None
+    s = (stream or torch.cuda.current_stream(d_blob.device)).cuda_stream
+    rc = lib().ep_prepare(C.byref(info), d_blob.data_ptr(), workspace.data_ptr(), st, s)
+    if rc != 0:
+        raise EpError(rc, "ep_prepare")
+    return workspace
+
+
+def decompress(d_blob, info=None, workspace=None, out=None, status=None, stream=None, lattice=False):
     """decompress(compressed): the fused GPU decode of a device-resident stream.
 
     ``d_blob``: CUDA uint8 tensor holding the whole stream.  ``info``: from ``stream_info``
-    (parsed from ``d_blob`` through a host copy when omitted).  ``out``: optional CUDA tensor
-    of ``info.shape`` / ``info.dtype``.  ``status``: optional CUDA int32 tensor of one element
-    into which damage flags are ORed.  Launches on ``stream`` (default: the current stream).
-    ``lattice=True`` returns the decoded lattice points v = 2z (int32) instead of weights."""
+    (parsed from ``d_blob`` through a host copy when omitted).  ``workspace``: from ``prepare``
+    on this ``d_blob`` (prepared here, on the same stream, when omitted).  ``out``: optional CUDA
+    tensor of ``info.shape`` / ``info.dtype``.  ``status``: optional CUDA int32 tensor of one
+    element into which damage flags are ORed.  Launches on ``stream`` (default: the current
+    stream).  ``lattice=True`` returns the decoded lattice points v = 2z (int32) instead of
+    weights."""
     if not d_blob.is_cuda:
         raise EpError(-1, "decompress needs the stream in device memory")
     if info is None:
         info = stream_info(d_blob.cpu())
+    if workspace is None:
+        workspace = prepare(d_blob, info, status=status, stream=stream)
     want = torch.int32 if lattice else info.dtype
     if out is None:
         out = torch.empty(info.shape, dtype=want, device=d_blob.device)
@@ -154,7 +181,7 @@ def decompress(d_blob, info=None, out=None, status=None, stream=None, lattice=Fa
     st = status.data_ptr() if status is not None else None
     s = (stream or torch.cuda.current_stream(d_blob.device)).cuda_stream
     dt = LATTICE_I32 if lattice else info.container_dtype
-    rc = lib().ep_decompress(C.byref(info), d_blob.data_ptr(), out.data_ptr(), dt, st, s)
+    rc = lib().ep_decompress(C.byref(info), d_blob.data_ptr(), workspace.data_ptr(), out.data_ptr(), dt, st, s)
     if rc != 0:
         raise EpError(rc, "ep_decompress")
     return out

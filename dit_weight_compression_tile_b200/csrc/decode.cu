@@ -38,13 +38,9 @@ namespace {
 
 constexpr int kMaxWarps = 32;
 constexpr uint32_t kSlotBytes = kProbScale * 4;                   // one context's slot table
-constexpr size_t kLutBytes = size_t(kContexts) * kSlotBytes;      // 56 KB
-constexpr uint32_t kCumStride = kMaxAlphabet + 8;                 // u16 per context (freqs, then their prefix sums)
-constexpr size_t kCumBytes = (size_t(kContexts) * kCumStride * 2 + 15) & ~size_t(15);
-constexpr uint32_t kSegs = kProbScale / 32;                       // 32-slot segments per context
-constexpr size_t kSegBytes = (size_t(kContexts) * kSegs * 2 + 15) & ~size_t(15);
+constexpr size_t kLutBytes = size_t(kContexts) * kSlotBytes;      // 56 KB: the prepared tables
 constexpr size_t kBarBytes = size_t(kMaxWarps) * 2 * 8 + 16;      // two mbarriers per warp + one for the tables
-constexpr size_t kFixedBytes = kLutBytes + kCumBytes + kSegBytes + kBarBytes;
+constexpr size_t kFixedBytes = kLutBytes + kBarBytes;
 constexpr uint32_t kSlack = 64;       // bytes past a tile that a lane's bounded over-read may touch
 constexpr size_t kSmemLimit = 232448; // shared memory one CTA may use on sm_100
 constexpr uint32_t kWaitLimit = 1u << 22;  // mbarrier polls before a copy is declared lost
@@ -63,7 +59,7 @@ struct Params {
     const uint32_t *dir;     // tile directory, 16-byte units (T + 1 entries)
     const uint8_t *tiles;    // tile section
     const float *rowf;       // per-row factors f_r
-    const uint8_t *freq;     // frequency tables (u16), contexts in order; 16-byte aligned
+    const uint32_t *tables;  // the stream's slot tables, prepared by ep_prepare (kLutBytes)
     void *out;               // container, row-major
     uint32_t *status;        // nullable
     uint64_t tile_units;     // size of the tile section in 16-byte units
@@ -73,12 +69,11 @@ struct Params {
     uint32_t T;              // tiles
     uint32_t tile_buf;       // bytes of each tile buffer (multiple of 16, includes kSlack)
     uint32_t nbuf;           // tile buffers per warp (1 or 2); 0: tiles are read from global memory
-    uint32_t freq_bytes;     // bytes of the frequency section to stage (multiple of 16)
     uint32_t splits;         // 4 bits per context
-    uint32_t tab_off[kContexts + 1];  // table start of each context (prefix sum of ntok)
 };
 
-__device__ __forceinline__ uint32_t split_of(const Params &p, uint32_t c) { return (p.splits >> (4 * c)) & 15u; }
+__device__ __forceinline__ uint32_t split_of_bits(uint32_t splits, uint32_t c) { return (splits >> (4 * c)) & 15u; }
+__device__ __forceinline__ uint32_t split_of(const Params &p, uint32_t c) { return split_of_bits(p.splits, c); }
 
 __device__ __forceinline__ int32_t unzigzag(uint32_t u) { return int32_t(u >> 1) ^ -int32_t(u & 1u); }
 
@@ -466,17 +461,82 @@ __device__ __forceinline__ uint32_t token_head(uint32_t c, uint32_t t, uint32_t 
     return (min(f, kProbScale - 1u) << 21) | field;
 }
 
-// ------------------------------------------------------------------ kernel
-// Shared memory: slot tables (the frequency section is first staged here), per-context
-// prefix sums, per-segment first tokens, mbarriers, then nbuf tile buffers per warp.
+// ------------------------------------------------------------------ ep_prepare: the slot tables
+// One CTA per (context, 256 slots): the context's frequencies and their prefix sums in shared
+// memory, then each thread finds the token of its slot by binary search.  Runs once per stream;
+// the decode kernel copies the 56 KB result into every CTA's shared memory.
+struct PrepParams {
+    const uint16_t *freq;    // frequency tables, contexts in order
+    uint32_t *tables;        // kContexts x 2048 entries
+    uint32_t *status;        // nullable
+    uint32_t splits;
+    uint32_t tab_off[kContexts + 1];
+};
+
+constexpr uint32_t kPrepThreads = 256;
+
+__global__ void __launch_bounds__(kPrepThreads) prepare_kernel(const __grid_constant__ PrepParams p) {
+    __shared__ uint32_t cum[kMaxAlphabet + 1];
+    __shared__ uint32_t part[kPrepThreads / 32];
+    const uint32_t c = blockIdx.x / (kProbScale / kPrepThreads);
+    const uint32_t slot = (blockIdx.x % (kProbScale / kPrepThreads)) * kPrepThreads + threadIdx.x;
+    const uint32_t n = min(p.tab_off[c + 1] - p.tab_off[c], kMaxAlphabet);
+    const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
+    // exclusive prefix sums of the (clamped) frequencies, 256 at a time
+    uint32_t run = 0;
+    bool bad = false;
+    for (uint32_t base = 0; base < n; base += kPrepThreads) {
+        uint32_t t = base + threadIdx.x;
+        uint32_t f = t < n ? uint32_t(p.freq[p.tab_off[c] + t]) : 0u;
+        bad |= f >= kProbScale;
+        f = min(f, kProbScale);
+        uint32_t incl = f;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= uint32_t(d)) incl += y;
+        }
+        if (lane == 31) part[warp] = incl;
+        __syncthreads();
+        uint32_t before = 0, all = 0;
+        for (uint32_t w = 0; w < kPrepThreads / 32; ++w) {
+            before += w < warp ? part[w] : 0u;
+            all += part[w];
+        }
+        if (t < n) cum[t] = min(run + before + incl - f, 0xffffu);
+        run = min(run + all, 0xffffu);
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) cum[n] = run;
+    __syncthreads();
+    if (p.status && blockIdx.x % (kProbScale / kPrepThreads) == 0 && threadIdx.x == 0 && n && run != kProbScale)
+        atomicOr(p.status, EP_DEC_BAD_TOKEN);
+    if (p.status && __syncthreads_or(bad) && threadIdx.x == 0) atomicOr(p.status, EP_DEC_BAD_TOKEN);
+    uint32_t e = 0;
+    if (n) {
+        // the last token t with cum[t] <= slot (tokens with f = 0 are skipped)
+        uint32_t lo = 0, hi = n;  // cum[lo] <= slot < cum[hi] (cum[n] may be short if damaged)
+        while (hi - lo > 1) {
+            uint32_t mid = (lo + hi) >> 1;
+            if (cum[mid] <= slot)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        uint32_t f = cum[lo + 1] - cum[lo];
+        e = token_head(c, lo, f, split_of_bits(p.splits, c)) | ((slot - cum[lo]) & (kProbScale - 1u));
+    }
+    p.tables[c * kProbScale + slot] = e;
+}
+
+// ------------------------------------------------------------------ decode kernel
+// Shared memory: the slot tables, mbarriers, then nbuf tile buffers per warp.
 template <int DT>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     const uint32_t lut = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-    const uint32_t cum = lut + uint32_t(kLutBytes);
-    const uint32_t seg = cum + uint32_t(kCumBytes);
-    const uint32_t bars = seg + uint32_t(kSegBytes);
+    const uint32_t bars = lut + uint32_t(kLutBytes);
     const uint32_t tbar = bars + uint32_t(kMaxWarps) * 16u;  // the tables' mbarrier
     const uint32_t nbuf = p.nbuf;
     const uint32_t bufs = bars + uint32_t(kBarBytes) + warp * (nbuf ? nbuf : 1u) * p.tile_buf;
@@ -491,12 +551,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_
         mbar_init(tbar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async();
+        mbar_expect(tbar, uint32_t(kLutBytes));
+        bulk_g2s(lut, p.tables, uint32_t(kLutBytes), tbar);
     }
     __syncthreads();
-    if (threadIdx.x == 0 && p.freq_bytes) {
-        mbar_expect(tbar, p.freq_bytes);
-        bulk_g2s(lut, p.freq, p.freq_bytes, tbar);
-    }
 
     // a tile's copy into buffer j of this warp; every lane computes whether it was issued
     auto tile_ok = [&](uint32_t t, uint32_t &beg, uint32_t &bytes) -> bool {
@@ -516,81 +574,14 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_
         }
         return ok;
     };
-    // per buffer: a copy in flight (bit 0 / 1) and the mbarrier phase to wait for (bit 2 / 3)
+    // per buffer: a copy in flight (bit 0 / 1) and the mbarrier phase to wait for (bit 0 / 1)
     uint32_t pend = 0, phase = 0;
     for (uint32_t j = 0; j < nbuf; ++j) {
         uint32_t t = t_begin + warp + j * nwarps;
         if (t < t_end && issue(t, j)) pend |= 1u << j;
     }
-
-    // ---- slot tables: prefix sums per context (a warp per context), the first token of every
-    // 32-slot segment, then every slot's entry
-    bool tables_ok = p.freq_bytes == 0 || mbar_wait(tbar, 0);
+    bool tables_ok = mbar_wait(tbar, 0);
     if (!tables_ok && lane == 0 && p.status) atomicOr(p.status, EP_DEC_TIMEOUT);
-    for (uint32_t c = warp; c < uint32_t(kContexts); c += nwarps) {
-        uint32_t n = p.tab_off[c + 1] - p.tab_off[c], run = 0;
-        uint32_t crow = cum + c * kCumStride * 2u, srow = seg + c * kSegs * 2u;
-        for (uint32_t g = lane; g < kSegs; g += 32) sts16(srow + 2u * g, 0xffffu);
-        __syncwarp();
-        bool bad = false;
-        for (uint32_t base = 0; base < n; base += 32) {
-            uint32_t t = base + lane;
-            uint32_t f = t < n ? lds16(lut + 2u * (p.tab_off[c] + t)) : 0u;
-            bad |= f >= kProbScale;
-            f = min(f, kProbScale);
-            uint32_t incl = f;
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
-                if (lane >= uint32_t(d)) incl += y;
-            }
-            uint32_t lo = min(run + incl - f, kProbScale), hi = min(run + incl, kProbScale);
-            if (t < n) {
-                sts16(crow + 2u * t, lo);
-                for (uint32_t g = (lo + 31u) >> 5; g < ((hi + 31u) >> 5); ++g) sts16(srow + 2u * g, t);
-            }
-            run = min(run + __shfl_sync(0xffffffffu, incl, 31), 0xffffu);
-        }
-        if (lane == 0) {
-            sts16(crow + 2u * n, min(run, kProbScale));
-            if (p.status && n && run != kProbScale) atomicOr(p.status, EP_DEC_BAD_TOKEN);
-        }
-        if (__any_sync(0xffffffffu, bad) && lane == 0 && p.status) atomicOr(p.status, EP_DEC_BAD_TOKEN);
-    }
-    __syncthreads();
-    // Each thread fills one 32-slot segment; lane l starts at slot l of its segment and wraps
-    // around, so the 32 lanes of a warp store to 32 different banks at every step.
-    for (uint32_t idx = threadIdx.x; idx < uint32_t(kContexts) * kSegs; idx += blockDim.x) {
-        uint32_t c = idx / kSegs, g = idx % kSegs;
-        uint32_t n = p.tab_off[c + 1] - p.tab_off[c];
-        uint32_t crow = cum + c * kCumStride * 2u, row = lut + c * kSlotBytes;
-        uint32_t t0 = lds16(seg + (c * kSegs + g) * 2u);
-        uint32_t m = split_of(p, c);
-        uint32_t l = idx & 31u;
-        if (n == 0 || t0 >= n) {
-            for (uint32_t j = 0; j < 32; ++j) sts32(row + 4u * (32u * g + ((l + j) & 31u)), 0u);
-            continue;
-        }
-        uint32_t t = t0, lo = lds16(crow + 2u * t), hi = lds16(crow + 2u * (t + 1));
-        uint32_t head = token_head(c, t, hi - lo, m);
-        for (uint32_t j = 0; j < 32; ++j) {
-            uint32_t s = 32u * g + ((l + j) & 31u);
-            if (l + j == 32u) {  // wrapped to the segment start
-                t = t0;
-                lo = lds16(crow + 2u * t);
-                hi = lds16(crow + 2u * (t + 1));
-                head = token_head(c, t, hi - lo, m);
-            }
-            while (s >= hi && t + 1 < n) {
-                ++t;
-                lo = hi;
-                hi = lds16(crow + 2u * (t + 1));
-                head = token_head(c, t, hi - lo, m);
-            }
-            sts32(row + 4u * s, head | ((s - lo) & (kProbScale - 1u)));
-        }
-    }
-    __syncthreads();
 
     // ---- tiles of this CTA: a contiguous range, warps round robin, nbuf copies in flight
     uint32_t j = 0;
@@ -648,8 +639,8 @@ cudaError_t launch(Params &p, uint64_t max_tile, int device, cudaStream_t stream
         sms = g_cache.sms[device];
     }
     // one CTA per SM (at most one per tile); warps = tiles per CTA, within kMaxWarps and the
-    // tile buffers that fit beside the tables: two per warp when they fit, else one, else the
-    // tiles are read from global memory
+    // tile buffers that fit beside the tables: two per warp when a warp has several tiles and
+    // they fit, else one, else the tiles are read from global memory
     uint32_t grid = p.T < uint32_t(sms) ? p.T : uint32_t(sms);
     uint32_t warps = (p.T + grid - 1) / grid;
     warps = warps > uint32_t(kMaxWarps) ? uint32_t(kMaxWarps) : warps;
@@ -676,41 +667,73 @@ cudaError_t launch(Params &p, uint64_t max_tile, int device, cudaStream_t stream
     return cudaGetLastError();
 }
 
-}  // namespace
-}  // namespace ep
-
-extern "C" int ep_decompress(const ep_info *info, const void *d_blob, void *d_out, int32_t out_dtype,
-                             uint32_t *d_status, ep_stream_t stream) {
-    using namespace ep;
-    if (!info || !d_blob || !d_out) return EP_ERR_INVALID_ARG;
-    if (out_dtype != info->container_dtype && out_dtype != EP_LATTICE_I32) return EP_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(d_blob) | reinterpret_cast<uintptr_t>(d_out)) & 15u) return EP_ERR_INVALID_ARG;
+int check_info(const ep_info *info) {
     if (info->rows <= 0 || info->cols <= 0 || info->cols % 8 || info->n_tiles == 0) return EP_ERR_INVALID_ARG;
     int64_t nb = info->rows * (info->cols / 8);
     if (nb >= (int64_t(1) << 31) || info->cols / 8 >= (int64_t(1) << 31)) return EP_ERR_UNSUPPORTED;
+    uint32_t total = 0;
+    for (int c = 0; c < kContexts; ++c) {
+        if (!split_valid(info->split[c], c) || info->ntok[c] > split_alphabet(info->split[c], kCtxLow[c]))
+            return EP_ERR_CORRUPT;
+        total += info->ntok[c];
+    }
+    if (info->off_freq + 2ull * total > info->off_dir) return EP_ERR_CORRUPT;
+    return EP_OK;
+}
+
+uint32_t pack_splits(const ep_info *info) {
+    uint32_t s = 0;
+    for (int c = 0; c < kContexts; ++c) s |= uint32_t(info->split[c]) << (4 * c);
+    return s;
+}
+
+}  // namespace
+}  // namespace ep
+
+extern "C" int ep_prepare(const ep_info *info, const void *d_blob, void *d_workspace, uint32_t *d_status,
+                          ep_stream_t stream) {
+    using namespace ep;
+    if (!info || !d_blob || !d_workspace) return EP_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(d_blob) | reinterpret_cast<uintptr_t>(d_workspace)) & 15u)
+        return EP_ERR_INVALID_ARG;
+    int rc = check_info(info);
+    if (rc != EP_OK) return rc;
+    PrepParams q;
+    q.freq = reinterpret_cast<const uint16_t *>(static_cast<const uint8_t *>(d_blob) + info->off_freq);
+    q.tables = static_cast<uint32_t *>(d_workspace);
+    q.status = d_status;
+    q.splits = pack_splits(info);
+    q.tab_off[0] = 0;
+    for (int c = 0; c < kContexts; ++c) q.tab_off[c + 1] = q.tab_off[c] + info->ntok[c];
+    prepare_kernel<<<kContexts * (kProbScale / kPrepThreads), kPrepThreads, 0,
+                     reinterpret_cast<cudaStream_t>(stream)>>>(q);
+    return cudaGetLastError() == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+extern "C" int ep_decompress(const ep_info *info, const void *d_blob, const void *d_workspace, void *d_out,
+                             int32_t out_dtype, uint32_t *d_status, ep_stream_t stream) {
+    using namespace ep;
+    if (!info || !d_blob || !d_workspace || !d_out) return EP_ERR_INVALID_ARG;
+    if (out_dtype != info->container_dtype && out_dtype != EP_LATTICE_I32) return EP_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(d_blob) | reinterpret_cast<uintptr_t>(d_out) |
+         reinterpret_cast<uintptr_t>(d_workspace)) & 15u)
+        return EP_ERR_INVALID_ARG;
+    int rc = check_info(info);
+    if (rc != EP_OK) return rc;
     Params p;
     const uint8_t *base = static_cast<const uint8_t *>(d_blob);
     p.dir = reinterpret_cast<const uint32_t *>(base + info->off_dir);
     p.tiles = base + info->off_tiles;
     p.rowf = reinterpret_cast<const float *>(base + info->off_rowf);
-    p.freq = base + info->off_freq;
+    p.tables = static_cast<const uint32_t *>(d_workspace);
     p.out = d_out;
     p.status = d_status;
     p.tile_units = (info->storage_nbytes - info->off_tiles) / 16;
-    p.nb = uint32_t(nb);
+    p.nb = uint32_t(info->rows * (info->cols / 8));
     p.cb = uint32_t(info->cols / 8);
     p.K = info->blocks_per_lane;
     p.T = info->n_tiles;
-    p.splits = 0;
-    p.tab_off[0] = 0;
-    for (int c = 0; c < kContexts; ++c) {
-        if (!split_valid(info->split[c], c) || info->ntok[c] > split_alphabet(info->split[c], kCtxLow[c]))
-            return EP_ERR_CORRUPT;
-        p.splits |= uint32_t(info->split[c]) << (4 * c);
-        p.tab_off[c + 1] = p.tab_off[c] + info->ntok[c];
-    }
-    p.freq_bytes = uint32_t((uint64_t(p.tab_off[kContexts]) * 2 + 15) & ~uint64_t(15));
-    if (info->off_freq + p.freq_bytes > info->off_dir || p.freq_bytes > kLutBytes) return EP_ERR_CORRUPT;
+    p.splits = pack_splits(info);
     int device;
     cudaError_t e = cudaGetDevice(&device);
     if (e != cudaSuccess) return EP_ERR_CUDA;

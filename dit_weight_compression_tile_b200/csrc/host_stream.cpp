@@ -2,7 +2,7 @@
 //
 // The CompressedTensor properties of the "EntroPack API reference" (shape, dtype,
 // actual_bpp = 8 * storage_nbytes / numel, storage_nbytes with and without the header)
-// read from a host copy of a format-v1 stream, which is validated before any decode.
+// read from a host copy of a format-v3 stream, which is validated before any decode.
 #include <cstring>
 
 #include "../../include/eptile.h"
@@ -82,6 +82,7 @@ extern "C" int ep_stream_info(const void *blob, size_t nbytes, ep_info *info) {
     I.header_nbytes = kHeaderBytes;
     I.actual_bpp = 8.0 * double(nbytes) / double(I.rows * I.cols);
     I.out_nbytes = uint64_t(I.rows * I.cols) * uint64_t(elt_bytes(I.container_dtype));
+    I.workspace_nbytes = uint64_t(kContexts) * kProbScale * 4;  // the decoder's slot tables
     *info = I;
     return EP_OK;
 }

@@ -18,8 +18,12 @@
  *   "Compressed Linear usage", Combine compression with FP8 or INT8 computation -- lossy
  *       compression of FP8 / INT8 weight codes, 0.001 <= target_bpp < 8, per-row scales
  *       counted in storage.
- * The byte layout of the stream (format version 1) is this library's own; it is written
+ * The byte layout of the stream (format version 3) is this library's own; it is written
  * out in the repository's design notes.
+ *
+ * Decoding a stream takes two calls: ep_prepare once per device copy of a stream (it turns
+ * the stream's frequency tables into the decoder's slot tables, in a caller-owned workspace
+ * of info.workspace_nbytes), then ep_decompress as often as the weights are needed.
  */
 #ifndef EPTILE_H
 #define EPTILE_H
@@ -47,14 +51,15 @@ enum ep_status {
     EP_ERR_BUFFER_TOO_SMALL = -5,   /* out_cap too small; *out_nbytes holds the size needed */
     EP_ERR_CORRUPT = -6,            /* the stream fails validation */
     EP_ERR_CUDA = -7,               /* a CUDA runtime call failed (launch, attribute) */
-    EP_ERR_UNSUPPORTED = -8         /* valid but outside format v1: cols % 8 != 0, > 2^32 blocks */
+    EP_ERR_UNSUPPORTED = -8         /* valid but outside the format: cols % 8 != 0, > 2^31 blocks,
+                                       a lane region beyond 65535 words with a forced tile size */
 };
 
 /* bits the decode kernel ORs into *d_status when a stream is damaged */
 enum ep_decode_flags {
     EP_DEC_WORD_OVERRUN = 1u, /* a renormalisation read ran past the tile's words */
-    EP_DEC_BAD_TOKEN = 2u,    /* a token outside its table (reported by the oracle; the
-                                 kernel reports such damage through the two flags below) */
+    EP_DEC_BAD_TOKEN = 2u,    /* frequency tables that do not sum to 2^11 or hold an entry of
+                                 2^11 or more (ep_prepare); a token outside its table (oracle) */
     EP_DEC_BAD_END = 4u,      /* a lane's state did not return to 2^16 at the end of its tile */
     EP_DEC_WORD_COUNT = 8u,   /* the tile has unread words beyond its 16-byte padding */
     EP_DEC_BAD_TILE = 16u,    /* a tile directory entry points outside the tile section */
@@ -85,6 +90,7 @@ typedef struct {
     uint64_t off_freq, off_dir, off_tiles;
     uint64_t out_nbytes;      /* rows * cols * container element size */
     uint64_t max_tile_nbytes; /* largest tile in the stream (sizes the decoder's staging buffers) */
+    uint64_t workspace_nbytes;/* device workspace ep_prepare fills and ep_decompress reads: 57344 */
 } ep_info;
 
 /* Upper bound of the stream size for ep_compress_host: with a searched resolution the
@@ -114,22 +120,40 @@ int ep_compress_host(const void *src, int32_t src_dtype, int64_t rows, int64_t c
  * the tile directory; returns EP_ERR_CORRUPT otherwise. */
 int ep_stream_info(const void *blob, size_t nbytes, ep_info *info);
 
+/* First half of decompress(compressed) (API reference): the decoder's tables for one device
+ * copy of a stream.  Run it once when the stream lands on the device; every ep_decompress of
+ * that copy then reuses the workspace.
+ *   info        from ep_stream_info on a host copy of the same stream.
+ *   d_blob      device pointer to the whole stream, 16-byte aligned.
+ *   d_workspace device buffer of info->workspace_nbytes bytes, 16-byte aligned, caller-owned;
+ *               overwritten with 7 slot tables of 2048 32-bit entries (one per context: the
+ *               token's frequency, the slot's offset in the token, the escape flag and the
+ *               decoded coordinate of a direct token).
+ *   d_status    nullable device uint32; EP_DEC_BAD_TOKEN is ORed in when the device copy's
+ *               frequency tables are damaged.
+ * One small kernel launch on `stream`; asynchronous. */
+int ep_prepare(const ep_info *info, const void *d_blob, void *d_workspace, uint32_t *d_status,
+               ep_stream_t stream);
+
 /* decompress(compressed) of the API reference: the fused decode on the GPU.
- *   info      from ep_stream_info on a host copy of the same stream.
- *   d_blob    device pointer to the whole stream (info->storage_nbytes bytes), 16-byte aligned.
- *   d_out     device pointer to rows * cols elements of out_dtype, row-major, 16-byte aligned.
- *   out_dtype info->container_dtype (the reconstructed weights or codes), or EP_LATTICE_I32 for
- *             the decoded lattice points v = 2z (int32) before scaling; no other conversion.
- *   d_status  nullable device pointer to one uint32; the kernel ORs EP_DEC_* bits into it
- *             when it meets a damaged tile (clear it before the call to read it per call).
- *   stream    CUDA stream of the launch.
- * One kernel launch (sm_100a): a persistent grid in which each warp decodes whole tiles with
- * its 32 lanes as interleaved rANS states, rebuilds the E8 coset in registers, scales by the
- * row factor in fp32 and stores the container with coalesced vector stores.  Asynchronous:
- * errors of the launch itself are returned; stream damage goes to d_status.  The library
- * allocates nothing and keeps a per-device cache of the SM count only. */
-int ep_decompress(const ep_info *info, const void *d_blob, void *d_out, int32_t out_dtype, uint32_t *d_status,
-                  ep_stream_t stream);
+ *   info        from ep_stream_info on a host copy of the same stream.
+ *   d_blob      device pointer to the whole stream (info->storage_nbytes bytes), 16-byte aligned.
+ *   d_workspace the workspace ep_prepare filled for this stream (read only here).
+ *   d_out       device pointer to rows * cols elements of out_dtype, row-major, 16-byte aligned.
+ *   out_dtype   info->container_dtype (the reconstructed weights or codes), or EP_LATTICE_I32 for
+ *               the decoded lattice points v = 2z (int32) before scaling; no other conversion.
+ *   d_status    nullable device pointer to one uint32; the kernel ORs EP_DEC_* bits into it
+ *               when it meets a damaged tile (clear it before the call to read it per call).
+ *   stream      CUDA stream of the launch.
+ * One kernel launch (sm_100a): a persistent grid, one CTA per SM, that bulk-copies the slot
+ * tables and each warp's tiles into shared memory (TMA, mbarrier completion); each warp decodes
+ * whole tiles with its 32 lanes as independent rANS coders, rebuilds the E8 coset in
+ * registers, scales by the row factor in fp32 and stores the container with coalesced vector
+ * stores.  Asynchronous: errors of the launch itself are returned; stream damage goes to
+ * d_status.  The library allocates nothing and keeps a per-device cache of the SM count
+ * only. */
+int ep_decompress(const ep_info *info, const void *d_blob, const void *d_workspace, void *d_out, int32_t out_dtype,
+                  uint32_t *d_status, ep_stream_t stream);
 
 /* static string for a status code */
 const char *ep_status_string(int status);

@@ -12,8 +12,8 @@ from dit_weight_compression_tile_b200 import synth
 
 def test_exports_every_declared_symbol():
     names = B.declared_functions()
-    assert set(names) == {"ep_compress_bound", "ep_compress_host", "ep_stream_info", "ep_decompress",
-                          "ep_status_string"}
+    assert set(names) == {"ep_compress_bound", "ep_compress_host", "ep_stream_info", "ep_prepare",
+                          "ep_decompress", "ep_status_string"}
     lib = B.lib()
     for n in names:
         assert hasattr(lib, n), n
@@ -38,6 +38,7 @@ def test_info_fields_and_storage():
     assert info.actual_bpp == 8.0 * blob.numel() / w.numel() <= 3.5  # "actual_bpp" of the API reference
     assert info.storage_nbytes_(include_header=False) == blob.numel() - 64
     assert info.out_nbytes == 2 * w.numel()
+    assert info.workspace_nbytes == 7 * 2048 * 4  # the decoder's slot tables
 
 
 def test_errors():
