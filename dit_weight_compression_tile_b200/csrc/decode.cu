@@ -41,7 +41,8 @@ constexpr uint32_t kSlotBytes = kProbScale * 4;                   // one context
 constexpr size_t kLutBytes = size_t(kContexts) * kSlotBytes;      // 56 KB: the prepared tables
 constexpr size_t kBarBytes = size_t(kMaxWarps) * 2 * 8 + 16;      // two mbarriers per warp + one for the tables
 constexpr size_t kFixedBytes = kLutBytes + kBarBytes;
-constexpr uint32_t kSlack = 64;       // bytes past a tile that a lane's bounded over-read may touch
+constexpr uint32_t kSlack = 160;      // bytes past a tile that a lane's bounded over-read may touch
+                                      // (8 blocks of 8 tokens between checks, one word each, + 1)
 constexpr size_t kSmemLimit = 232448; // shared memory one CTA may use on sm_100
 constexpr uint32_t kWaitLimit = 1u << 22;  // mbarrier polls before a copy is declared lost
 static_assert(kFixedBytes % 16 == 0, "tile buffers must start 16-byte aligned");
@@ -64,6 +65,7 @@ struct Params {
     uint32_t *status;        // nullable
     uint64_t tile_units;     // size of the tile section in 16-byte units
     uint32_t nb;             // E8 blocks (rows * cols / 8)
+    uint32_t rows;
     uint32_t cb;             // blocks per row
     uint32_t K;              // blocks per lane
     uint32_t T;              // tiles
@@ -274,7 +276,13 @@ __device__ __forceinline__ uint32_t step(Lane<SMEM> &L, bool act, uint32_t lut) 
     if (ACT && !act) return 0u;
     uint32_t e = lds32(lut + ((L.x & (kProbScale - 1u)) << 2));
     uint32_t xn = (e >> 21) * (L.x >> kProbBits) + (e & (kProbScale - 1u));
-    if (xn < kStateLow) {
+    if constexpr (SMEM) {
+        // predicated: x = (x << 16) | w, then the next word of the region is read ahead
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.lt.u32 p, %0, 65536;\n\t@p prmt.b32 %0, %2, %0, 0x5410;\n\t"
+            "@p add.u32 %1, %1, 2;\n\t@p ld.shared.u16 %2, [%1];\n\t}"
+            : "+r"(xn), "+r"(L.wp), "+r"(L.w));
+    } else if (xn < kStateLow) {
         xn = (xn << 16) | L.w;
         L.advance();
     }
@@ -339,45 +347,52 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
                                                   Lim wlim, uint32_t t, uint32_t lane) {
     uint32_t b = t * 32u * p.K + lane;
     uint32_t row = b / p.cb, col = b - row * p.cb;
-    float fr = (!ACT || b < p.nb) ? __ldg(p.rowf + row) : 0.0f;
+    // the factor of the current row and of the next one (read a row ahead)
+    float fr = row < p.rows ? __ldg(p.rowf + row) : 0.0f;
+    float frn = row + 1 < p.rows ? __ldg(p.rowf + row + 1) : 0.0f;
     uint32_t err = 0;
     for (uint32_t k = 0; k < p.K; ++k, b += 32u) {
         bool act = !ACT || b < p.nb;
         if (ACT && !__any_sync(0xffffffffu, act)) break;
-        // a damaged stream may drive a lane's reads ahead; stop before they leave the buffer
-        if (__any_sync(0xffffffffu, L.past(wlim))) {
+        // a damaged stream may drive a lane's reads ahead (at most one word per token); stop
+        // before they leave the buffer's slack
+        if ((k & 7u) == 0 && __any_sync(0xffffffffu, L.past(wlim))) {
             err |= EP_DEC_WORD_OVERRUN;
             break;
         }
-        uint32_t col_n = col + 32u, row_n = row;
-        while (col_n >= p.cb) {
-            col_n -= p.cb;
-            ++row_n;
-        }
-        float fr_n = (k + 1 < p.K && b + 32u < p.nb) ? __ldg(p.rowf + row_n) : 0.0f;
         uint32_t e[8];
-        // coordinate 0 (context 0) carries the coset c in bit 11 of its entry
+        // coordinate 0 (context 0); bit 11 of every entry of contexts 0..2 is the coset c
         e[0] = step<SMEM, ACT>(L, act, lut);
         uint32_t lutc = lut + kSlotBytes + ((e[0] & 0x800u) << 2);  // context 1 + c
 #pragma unroll
         for (int i = 1; i < 7; ++i) e[i] = step<SMEM, ACT>(L, act, lutc);
-        // bit 12 of an entry is the parity of y_i: coordinate 7 takes context 3 + 2c + p
+        // bits 11 and 12 of the XOR of entries 0..6 are c (seven copies) and the parity p of
+        // y0..y6; context 3 + 2c + p sits at table position 3 + c + 2p
         uint32_t X = e[0] ^ e[1] ^ e[2] ^ e[3] ^ e[4] ^ e[5] ^ e[6];
-        uint32_t lut7 = lut + 3u * kSlotBytes + ((e[0] & 0x800u) << 3) + ((X & 0x1000u) << 1);
+        uint32_t lut7 = lut + 3u * kSlotBytes + ((X & 0x1800u) << 2);
         e[7] = step<SMEM, ACT>(L, act, lut7);
         uint32_t F[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) F[i] = (e[i] & kFieldMask) | kMagic;
         uint32_t O = e[0] | e[1] | e[2] | e[3] | e[4] | e[5] | e[6] | e[7];
         if (__any_sync(0xffffffffu, O & kEscBit))
-            resolve_escapes<SMEM>(p, e, F, (e[0] >> 11) & 1u, (X >> 12) & 1u, L, rb);
+            resolve_escapes<SMEM>(p, e, F, (X >> 11) & 1u, (X >> 12) & 1u, L, rb);
         Packer<DT> pk;
 #pragma unroll
         for (int i = 0; i < 8; ++i) pk.put(i, __fmaf_rn(__uint_as_float(F[i]), kInvScale, -kBias), fr);
         if (act) pk.store(p.out, b);
-        col = col_n;
-        row = row_n;
-        fr = fr_n;
+        col += 32u;
+        if (col >= p.cb) {  // next row (all lanes at once when a row holds a multiple of 32 blocks)
+            col -= p.cb;
+            ++row;
+            fr = frn;
+            while (col >= p.cb) {
+                col -= p.cb;
+                ++row;
+                fr = row < p.rows ? __ldg(p.rowf + row) : 0.0f;
+            }
+            frn = row + 1 < p.rows ? __ldg(p.rowf + row + 1) : 0.0f;
+        }
     }
     return err;
 }
@@ -526,7 +541,10 @@ __global__ void __launch_bounds__(kPrepThreads) prepare_kernel(const __grid_cons
         uint32_t f = cum[lo + 1] - cum[lo];
         e = token_head(c, lo, f, split_of_bits(p.splits, c)) | ((slot - cum[lo]) & (kProbScale - 1u));
     }
-    p.tables[c * kProbScale + slot] = e;
+    // context 3 + 2c + p is stored at position 3 + c + 2p (the decoder forms that offset from
+    // the XOR of a block's first seven entries)
+    uint32_t pos = c < 3 ? c : 3u + ((c - 3u) >> 1) + 2u * ((c - 3u) & 1u);
+    p.tables[pos * kProbScale + slot] = e;
 }
 
 // ------------------------------------------------------------------ decode kernel
@@ -730,6 +748,7 @@ extern "C" int ep_decompress(const ep_info *info, const void *d_blob, const void
     p.status = d_status;
     p.tile_units = (info->storage_nbytes - info->off_tiles) / 16;
     p.nb = uint32_t(info->rows * (info->cols / 8));
+    p.rows = uint32_t(info->rows);
     p.cb = uint32_t(info->cols / 8);
     p.K = info->blocks_per_lane;
     p.T = info->n_tiles;
