@@ -274,12 +274,17 @@ struct Lane<false> {
 template <bool SMEM, bool ACT>
 __device__ __forceinline__ uint32_t step(Lane<SMEM> &L, bool act, uint32_t lut) {
     if (ACT && !act) return 0u;
-    uint32_t e = lds32(lut + ((L.x & (kProbScale - 1u)) << 2));
-    uint32_t xn = (e >> 21) * (L.x >> kProbBits) + (e & (kProbScale - 1u));
+    // slot address lut + 4 (x mod 2^11) as two multiply-adds (lut + 4x - 2^13 (x >> 11), exact
+    // modulo 2^32), which run on the FMA pipe beside the ALU work of the other lanes
+    uint32_t xs = L.x >> kProbBits, a, t;
+    asm("mad.lo.u32 %0, %1, 4, %2;" : "=r"(t) : "r"(L.x), "r"(lut));
+    asm("mad.lo.u32 %0, %1, -8192, %2;" : "=r"(a) : "r"(xs), "r"(t));
+    uint32_t e = lds32(a);
+    uint32_t xn = (e >> 21) * xs + (e & (kProbScale - 1u));
     if constexpr (SMEM) {
-        // predicated: x = (x << 16) | w, then the next word of the region is read ahead
+        // predicated: x = x * 2^16 + w, then the next word of the region is read ahead
         asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.lt.u32 p, %0, 65536;\n\t@p prmt.b32 %0, %2, %0, 0x5410;\n\t"
+            "{\n\t.reg .pred p;\n\tsetp.lt.u32 p, %0, 65536;\n\t@p mad.lo.u32 %0, %0, 65536, %2;\n\t"
             "@p add.u32 %1, %1, 2;\n\t@p ld.shared.u16 %2, [%1];\n\t}"
             : "+r"(xn), "+r"(L.wp), "+r"(L.w));
     } else if (xn < kStateLow) {
