@@ -86,6 +86,8 @@ def lib():
         L.ep_prepare.argtypes = [C.POINTER(StreamInfo), p, p, p, p]
         L.ep_decompress.restype = C.c_int
         L.ep_decompress.argtypes = [C.POINTER(StreamInfo), p, p, p, C.c_int32, p, p]
+        L.ep_decompress_noalloc.restype = C.c_int
+        L.ep_decompress_noalloc.argtypes = [C.POINTER(StreamInfo), p, p, C.c_int32, p, p]
         L.ep_status_string.restype = C.c_char_p
         L.ep_status_string.argtypes = [C.c_int]
         _lib = L

@@ -774,3 +774,52 @@ extern "C" int ep_decompress(const ep_info *info, const void *d_blob, const void
     }
     return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
+
+// ------------------------------------------------------------------ ep_decompress_noalloc
+// The same decode for callers that cannot allocate device memory: the slot tables live in one
+// file-scope device array instead of a caller workspace.  Every GPU that loads the library holds
+// this array (56 KB) until the process exits; all calls on a device share it.
+namespace ep {
+namespace {
+
+constexpr size_t kStaticTablesBytes = kLutBytes;  // the largest workspace a stream can need
+static __device__ __align__(256) uint32_t g_static_tables[kStaticTablesBytes / 4];
+
+struct StaticTables {
+    std::mutex mu;
+    void *ptr[64] = {};
+};
+StaticTables g_static;
+
+// device address of g_static_tables on the current device, looked up once per device (the host
+// name of the array is only a stand-in and must not reach a kernel)
+int static_tables(void **out) {
+    int device;
+    if (cudaGetDevice(&device) != cudaSuccess) return EP_ERR_CUDA;
+    if (device < 0 || device >= 64) return EP_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> g(g_static.mu);
+    if (!g_static.ptr[device]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_tables) != cudaSuccess || !p) return EP_ERR_CUDA;
+        g_static.ptr[device] = p;
+    }
+    *out = g_static.ptr[device];
+    return EP_OK;
+}
+
+}  // namespace
+}  // namespace ep
+
+extern "C" int ep_decompress_noalloc(const ep_info *info, const void *d_blob, void *d_out, int32_t out_dtype,
+                                     uint32_t *d_status, ep_stream_t stream) {
+    using namespace ep;
+    if (!info) return EP_ERR_INVALID_ARG;
+    if (info->workspace_nbytes > kStaticTablesBytes) return EP_ERR_UNSUPPORTED;
+    void *tables = nullptr;
+    int rc = static_tables(&tables);
+    if (rc != EP_OK) return rc;
+    // both launches go to the same stream, so the decode reads the tables this call prepared
+    rc = ep_prepare(info, d_blob, tables, d_status, stream);
+    if (rc != EP_OK) return rc;
+    return ep_decompress(info, d_blob, tables, d_out, out_dtype, d_status, stream);
+}

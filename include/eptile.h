@@ -155,6 +155,21 @@ int ep_prepare(const ep_info *info, const void *d_blob, void *d_workspace, uint3
 int ep_decompress(const ep_info *info, const void *d_blob, const void *d_workspace, void *d_out, int32_t out_dtype,
                   uint32_t *d_status, ep_stream_t stream);
 
+/* ep_prepare + ep_decompress for callers that cannot allocate device memory: a plugin inside an
+ * inference engine that owns all device memory and forbids allocation in its forward path, or code
+ * that must not trigger the device-wide synchronisation a cudaMalloc/cudaFree can cause.  No
+ * counterpart in the EntroPack pages; it exists for such callers only.
+ *   Arguments as ep_decompress, without a workspace: the slot tables go to one file-scope device
+ *   array of 57,344 bytes (info->workspace_nbytes of every stream), which each GPU that loads the
+ *   library keeps until the process exits.  A stream needing more returns EP_ERR_UNSUPPORTED.
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *   that device current; make that first call before any stream capture.
+ *   All calls on a device share the array and leave the last call's tables in it: calls that
+ *   overlap on the GPU (different streams without ordering) race and may decode with another
+ *   stream's tables.  Two launches (tables, decode) on `stream`; no allocation, no sync. */
+int ep_decompress_noalloc(const ep_info *info, const void *d_blob, void *d_out, int32_t out_dtype,
+                          uint32_t *d_status, ep_stream_t stream);
+
 /* static string for a status code */
 const char *ep_status_string(int status);
 

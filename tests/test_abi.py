@@ -13,7 +13,7 @@ from dit_weight_compression_tile_b200 import synth
 def test_exports_every_declared_symbol():
     names = B.declared_functions()
     assert set(names) == {"ep_compress_bound", "ep_compress_host", "ep_stream_info", "ep_prepare",
-                          "ep_decompress", "ep_status_string"}
+                          "ep_decompress", "ep_decompress_noalloc", "ep_status_string"}
     lib = B.lib()
     for n in names:
         assert hasattr(lib, n), n

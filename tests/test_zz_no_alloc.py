@@ -1,0 +1,62 @@
+"""ep_decompress_noalloc, the entry point for callers that cannot allocate device memory (for
+instance a plugin inside an inference engine that owns all device memory, or code that must
+avoid the synchronisation a cudaMalloc can cause): it keeps the decoder's tables in a static
+device array instead of a caller workspace.  Called through the C ABI, its output must equal
+the workspace path's (ep_prepare + ep_decompress) bit for bit, on two calls in a row with
+different streams, so the second call must replace the first call's tables.
+
+The file sorts last so that a run stopping at its first failure has already run every other
+test; it also passes alone in a fresh process."""
+import ctypes as C
+
+import numpy as np
+import pytest
+import torch
+
+from dit_weight_compression_tile_b200 import binding as B
+from dit_weight_compression_tile_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def noalloc_decode(d_blob, info, stream):
+    out = torch.empty(info.shape, dtype=info.dtype, device=d_blob.device)
+    status = torch.zeros(1, dtype=torch.int32, device=d_blob.device)
+    rc = B.lib().ep_decompress_noalloc(C.byref(info), d_blob.data_ptr(), out.data_ptr(), info.container_dtype,
+                                       status.data_ptr(), stream.cuda_stream)
+    assert rc == 0, B.lib().ep_status_string(rc)
+    return out, status
+
+
+def workspace_decode(d_blob, info, stream):
+    status = torch.zeros(1, dtype=torch.int32, device=d_blob.device)
+    work = B.prepare(d_blob, info, status=status, stream=stream)
+    out = B.decompress(d_blob, info, workspace=work, status=status, stream=stream)
+    return out, status
+
+
+def test_noalloc_matches_workspace_path_twice():
+    cases = [(synth.row_lognormal(512, 2048, 21), 4.0, 0), (synth.gaussian(256, 1024, 0.02, 22), 3.0, B.INT8)]
+    stream = torch.cuda.Stream()
+    for w, target, container in cases:  # two calls in a row, the second with other tables
+        blob = B.compress(w, target, container=container)
+        info = B.stream_info(blob)
+        d = blob.cuda()
+        with torch.cuda.stream(stream):
+            got, st_got = noalloc_decode(d, info, stream)
+            ref, st_ref = workspace_decode(d, info, stream)
+        stream.synchronize()
+        assert int(st_got.item()) == 0 and int(st_ref.item()) == 0
+        assert got.dtype == ref.dtype and got.shape == ref.shape
+        assert np.array_equal(got.view(torch.uint8).cpu().numpy(), ref.view(torch.uint8).cpu().numpy())
+
+
+def test_noalloc_rejects_oversized_workspace():
+    blob = B.compress(synth.gaussian(64, 256, 0.02, 23), 4.0)
+    info = B.stream_info(blob)
+    info.workspace_nbytes = 57344 + 16  # beyond the static array's stated maximum
+    d = blob.cuda()
+    out = torch.empty(info.shape, dtype=info.dtype, device="cuda")
+    rc = B.lib().ep_decompress_noalloc(C.byref(info), d.data_ptr(), out.data_ptr(), info.container_dtype, None,
+                                       torch.cuda.current_stream().cuda_stream)
+    assert rc == -8  # EP_ERR_UNSUPPORTED
