@@ -574,6 +574,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_
         mbar_init(tbar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async();
+    }
+    // launched with programmatic stream serialisation: the CTA may start while the previous kernel
+    // of the stream drains; nothing global is touched before that kernel's writes are visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (threadIdx.x == 0) {
         mbar_expect(tbar, uint32_t(kLutBytes));
         bulk_g2s(lut, p.tables, uint32_t(kLutBytes), tbar);
     }
@@ -686,8 +692,17 @@ cudaError_t launch(Params &p, uint64_t max_tile, int device, cudaStream_t stream
     }
     if (warps < 1) warps = 1;
     size_t smem = kFixedBytes + size_t(warps) * (p.nbuf ? p.nbuf : 1) * p.tile_buf;
-    decode_kernel<DT><<<grid, warps * 32, smem, stream>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(warps * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_kernel<DT>, p);
 }
 
 int check_info(const ep_info *info) {
