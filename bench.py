@@ -162,6 +162,21 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+# ------------------------------------------------------------------ ranks (replicas, no data exchange)
+def max_over_ranks(x, world, device):
+    """the slowest rank's time: every rank decodes its own replica, the job ends with the last"""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(per_rank_bytes, world, seconds):
+    """whole-job throughput: all ranks' bytes over the slowest rank's time"""
+    return world * per_rank_bytes / seconds
+
+
 # ------------------------------------------------------------------ CPU oracle leg
 def cpu_oracle_decode(blob_np, seconds):
     """the oracle decoder, as it stands, on one host core: consecutive tiles of one stream for a
@@ -309,15 +324,11 @@ def run_ours(a, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     per_replay = [ev[r].elapsed_time(ev[r + 1]) for r in range(replays)]
-    total_ms = ev[0].elapsed_time(ev[-1])
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), world, dev)
     assert int(status.item()) == 0
     kernel_s = statistics.mean(per_replay) / rot / 1e3  # decode launches of one step, back to back
     step_s = total_ms / steps / 1e3
-    value = world * out_bytes / step_s / 1e9
+    value = job_rate(out_bytes, world, step_s) / 1e9
     peak, peak_kind = measured_peaks()
     achieved = (in_bytes + out_bytes) / kernel_s / 1e9
     traffic = traffic_for_kernel(a.workload)
@@ -358,12 +369,8 @@ def run_ours(a, rank, world, local_rank):
             e2e_step()
         e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * out_bytes * e2e_steps / (e2e_ms / 1e3) / 1e9
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = job_rate(out_bytes * e2e_steps, world, e2e_ms / 1e3) / 1e9
 
     if rank != 0:
         return
@@ -379,7 +386,7 @@ def run_ours(a, rank, world, local_rank):
                        actual_bpp=round(8.0 * in_bytes / n_weights, 4), n_tensors=len(infos),
                        n_tiles=sum(i.n_tiles for i in infos), blocks_per_lane=i0.blocks_per_lane,
                        parallelism="replicas" if world > 1 else "single"),
-        "gweights_per_s": round(world * n_weights / step_s / 1e9, 3),
+        "gweights_per_s": round(job_rate(n_weights, world, step_s) / 1e9, 3),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": (in_bytes + out_bytes) // len(infos),

@@ -4,19 +4,20 @@
 // symbol decoding and numerical weight reconstruction on the GPU" ("EntroPack: Fast and
 // Accurate Entropy-Coded Weight Compression at Arbitrary Bitrates", Abstract).  One kernel, one
 // CTA per SM:
-//   * prologue: the frequency tables reach shared memory with one bulk (TMA) copy; the CTA turns
-//     them into seven 2048-slot tables.  A slot's 32-bit entry holds the token's frequency
-//     (11 bits), the slot's offset inside the token (11 bits), an escape flag and, for a
-//     direct token, the lattice coordinate v + 256 (9 bits);
+//   * ep_prepare (a small kernel, once per device copy of a stream) turns the frequency tables
+//     into seven 2048-slot tables in a workspace.  A slot's 32-bit entry holds the token's
+//     frequency (11 bits), the slot's offset inside the token (11 bits), an escape flag and, for
+//     a direct token, the lattice coordinate v + 256 (9 bits).  Each decode CTA stages the 56 KB
+//     with one bulk (TMA) copy;
 //   * each warp decodes whole tiles.  A tile (32 initial states, 32 word counts, the lanes'
 //     16-bit word streams, the raw extra bits) is brought into the warp's shared-memory buffer
-//     by one bulk copy completing on an mbarrier, two tiles in flight per warp.  Lane l runs the
+//     by one bulk copy completing on an mbarrier, up to two tiles in flight per warp.  Lane l runs the
 //     rANS coder of lane l over its own word stream, so a step is a table lookup, a
 //     multiply-add and a predicated word read, with no warp-wide exchange;
 //   * the coset c and the parity of y0..y6 that pick the contexts of coordinates 1..7 are bits
 //     of the table entries, so a block's 8 tokens decode without a branch; the rare escape
-//     tokens (at most a few per thousand) are resolved after the block from the tile's raw bit
-//     stream;
+//     tokens (a few per thousand) are resolved after the block from raw bits at the back of the
+//     lane's word region;
 //   * reconstruction stays in registers: the entry's value field becomes an exact float with
 //     one logic op and one fused multiply-add, w = fp32(f_r * v) is one multiply, and the
 //     container conversion rounds to nearest even; a warp stores 32 consecutive blocks with
@@ -90,8 +91,6 @@ __device__ __forceinline__ uint32_t lds16(uint32_t a) {
     asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a));
     return v;
 }
-__device__ __forceinline__ void sts32(uint32_t a, uint32_t v) { asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v)); }
-__device__ __forceinline__ void sts16(uint32_t a, uint32_t v) { asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "r"(v)); }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
