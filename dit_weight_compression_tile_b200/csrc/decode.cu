@@ -125,19 +125,29 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // ------------------------------------------------------------------ containers
-// put(i, v, fr): coordinate i of the block, v the exact lattice value as a float, fr the row
-// factor; the weight is fp32(fr * v), one correctly rounded multiply.
+// put(i, v, w): coordinate i of the block, v the exact lattice value as a float and w = fp32(f_r v)
+// the weight (one correctly rounded multiply), which the container rounds to nearest even.
 template <int DT>
 struct Packer;
 
-__device__ __forceinline__ float reconstruct(float v, float fr) { return __fmul_rn(fr, v); }
+// paired fp32 arithmetic of sm_100 (two independent IEEE operations, round to nearest each)
+__device__ __forceinline__ uint64_t fma_x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul_x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t pair(uint32_t lo, uint32_t hi) { return uint64_t(lo) | (uint64_t(hi) << 32); }
 
 template <>
 struct Packer<EP_BF16> {
     uint32_t o[4];
     float lo;
-    __device__ __forceinline__ void put(int i, float v, float fr) {
-        float w = reconstruct(v, fr);
+    __device__ __forceinline__ void put(int i, float, float w) {
         if (i & 1) {
             __nv_bfloat162 h = __floats2bfloat162_rn(lo, w);
             o[i >> 1] = *reinterpret_cast<uint32_t *>(&h);
@@ -154,8 +164,7 @@ template <>
 struct Packer<EP_FP16> {
     uint32_t o[4];
     float lo;
-    __device__ __forceinline__ void put(int i, float v, float fr) {
-        float w = reconstruct(v, fr);
+    __device__ __forceinline__ void put(int i, float, float w) {
         if (i & 1) {
             __half2 h = __floats2half2_rn(lo, w);
             o[i >> 1] = *reinterpret_cast<uint32_t *>(&h);
@@ -171,7 +180,7 @@ struct Packer<EP_FP16> {
 template <>
 struct Packer<EP_FP32> {
     float o[8];
-    __device__ __forceinline__ void put(int i, float v, float fr) { o[i] = reconstruct(v, fr); }
+    __device__ __forceinline__ void put(int i, float, float w) { o[i] = w; }
     __device__ __forceinline__ void store(void *out, uint32_t b) {
         float4 *p = reinterpret_cast<float4 *>(out) + 2 * size_t(b);
         p[0] = make_float4(o[0], o[1], o[2], o[3]);
@@ -182,8 +191,8 @@ struct Packer<EP_FP32> {
 template <>
 struct Packer<EP_INT8> {
     uint32_t o[2];
-    __device__ __forceinline__ void put(int i, float v, float fr) {
-        int q = min(127, max(-127, __float2int_rn(reconstruct(v, fr))));
+    __device__ __forceinline__ void put(int i, float, float w) {
+        int q = min(127, max(-127, __float2int_rn(w)));
         uint32_t byte = uint32_t(q) & 0xffu;
         if ((i & 3) == 0)
             o[i >> 2] = byte;
@@ -199,8 +208,7 @@ template <>
 struct Packer<EP_FP8_E4M3> {
     uint32_t o[2];
     float lo;
-    __device__ __forceinline__ void put(int i, float v, float fr) {
-        float w = reconstruct(v, fr);
+    __device__ __forceinline__ void put(int i, float, float w) {
         if (i & 1) {
             uint32_t pair = __nv_cvt_float2_to_fp8x2(make_float2(lo, w), __NV_SATFINITE, __NV_E4M3);
             if ((i & 3) == 1)
@@ -381,9 +389,18 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
         uint32_t O = e[0] | e[1] | e[2] | e[3] | e[4] | e[5] | e[6] | e[7];
         if (__any_sync(0xffffffffu, O & kEscBit))
             resolve_escapes<SMEM>(p, e, F, (X >> 11) & 1u, (X >> 12) & 1u, L, rb);
+        // v = F 2^-22 - (2^12 + 256) exactly, w = fp32(f_r v): two coordinates per instruction
+        const uint64_t scale2 = pair(__float_as_uint(kInvScale), __float_as_uint(kInvScale));
+        const uint64_t bias2 = pair(__float_as_uint(-kBias), __float_as_uint(-kBias));
+        const uint64_t fr2 = pair(__float_as_uint(fr), __float_as_uint(fr));
         Packer<DT> pk;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) pk.put(i, __fmaf_rn(__uint_as_float(F[i]), kInvScale, -kBias), fr);
+        for (int i = 0; i < 8; i += 2) {
+            uint64_t v2 = fma_x2(pair(F[i], F[i + 1]), scale2, bias2);
+            uint64_t w2 = mul_x2(v2, fr2);
+            pk.put(i, __uint_as_float(uint32_t(v2)), __uint_as_float(uint32_t(w2)));
+            pk.put(i + 1, __uint_as_float(uint32_t(v2 >> 32)), __uint_as_float(uint32_t(w2 >> 32)));
+        }
         if (act) pk.store(p.out, b);
         col += 32u;
         if (col >= p.cb) {  // next row (all lanes at once when a row holds a multiple of 32 blocks)
