@@ -303,34 +303,37 @@ __device__ __forceinline__ uint32_t step(Lane<SMEM> &L, bool act, uint32_t lut) 
 }
 
 // `nbits` raw bits at raw-bit position rb of the lane (the region's last word holds bits
-// 0..15), least significant first; nbits <= 24
+// 0..15), least significant first; nbits <= 19 and rb is clamped by the caller so that the three
+// words read lie inside the tile (shared memory: inside the buffer)
 template <bool SMEM>
 __device__ __forceinline__ uint32_t raw_bits(const Lane<SMEM> &L, uint32_t rb, uint32_t nbits) {
     int32_t j = int32_t(L.end) - 1 - int32_t(rb >> 4);
-    int32_t lo = SMEM ? -3 : -int32_t(kTileHead / 2);  // stays inside the buffer / the tile
-    uint32_t w0 = L.word(max(j, lo)), w1 = L.word(max(j - 1, lo)), w2 = L.word(max(j - 2, lo));
-    uint64_t win = uint64_t(w0) | (uint64_t(w1) << 16) | (uint64_t(w2) << 32);
-    return uint32_t(win >> (rb & 15u)) & ((1u << nbits) - 1u);
+    uint32_t lo = __byte_perm(L.word(j), L.word(j - 1), 0x5410);  // bits rb & ~15 .. + 31
+    uint32_t hi = L.word(j - 2);
+    return __funnelshift_r(lo, hi, rb & 15u) & ((1u << nbits) - 1u);
 }
 
 // Escape tokens of a block (the warp has at least one).  Token layout (split m, `low` kept
 // bits, 2 bits below the leading one): d = token - 2^m = ((n - m) << 2 | top) << low | lo; the
-// value is s = (4 | top) << (n - 2) | extra << low | lo with n - 2 - low raw extra bits.
+// value is s = (4 | top) << (n - 2) | extra << low | lo with n - 2 - low raw extra bits.  F[i]
+// holds the entry's value field (d, or 2d + c for coordinates 1..6) and its escape flag.
 template <bool SMEM>
-__device__ __forceinline__ void resolve_escapes(const Params &p, const uint32_t (&e)[8], uint32_t (&F)[8],
-                                                uint32_t c, uint32_t par, Lane<SMEM> &L, uint32_t &rb) {
+__device__ __forceinline__ void resolve_escapes(const Params &p, uint32_t (&F)[8], uint32_t c, uint32_t par,
+                                                Lane<SMEM> &L, uint32_t &rb) {
     uint32_t lm = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) lm |= ((e[i] >> 20) & 1u) << i;
+    for (int i = 0; i < 8; ++i) lm |= ((F[i] >> 20) & 1u) << i;
     uint32_t M = __reduce_or_sync(0xffffffffu, lm);
+    // a damaged region cannot move the raw reads below the tile's head
+    rb = min(rb, 16u * (L.end + 88u));
+    const uint32_t m0 = split_of(p, 0), m16 = split_of(p, 1u + c), m7 = split_of(p, 3u + 2u * c + par);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         if (M & (1u << i)) {
             if (lm & (1u << i)) {
-                uint32_t ctx = i == 0 ? 0u : (i < 7 ? 1u + c : 3u + 2u * c + par);
-                uint32_t low = i == 0 ? 2u : (i < 7 ? 1u : 0u);
-                uint32_t m = split_of(p, ctx);
-                uint32_t fld = (e[i] >> 11) & 0x1ffu;
+                const uint32_t low = i == 0 ? 2u : (i < 7 ? 1u : 0u);
+                uint32_t m = i == 0 ? m0 : (i < 7 ? m16 : m7);
+                uint32_t fld = (F[i] >> 11) & 0x1ffu;
                 uint32_t d = (i >= 1 && i <= 6) ? fld >> 1 : fld;
                 uint32_t q = d >> low;
                 uint32_t n = min(m + (q >> 2), kValueBits - 1u);
@@ -383,12 +386,14 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
         uint32_t X = e[0] ^ e[1] ^ e[2] ^ e[3] ^ e[4] ^ e[5] ^ e[6];
         uint32_t lut7 = lut + 3u * kSlotBytes + ((X & 0x1800u) << 2);
         e[7] = step<SMEM, ACT>(L, act, lut7);
+        // F keeps the value field and the escape flag of each entry (the flag only matters for
+        // escapes, whose F is rebuilt), so the entries themselves die here
         uint32_t F[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) F[i] = (e[i] & kFieldMask) | kMagic;
-        uint32_t O = e[0] | e[1] | e[2] | e[3] | e[4] | e[5] | e[6] | e[7];
+        for (int i = 0; i < 8; ++i) F[i] = (e[i] & (kFieldMask | kEscBit)) | kMagic;
+        uint32_t O = F[0] | F[1] | F[2] | F[3] | F[4] | F[5] | F[6] | F[7];
         if (__any_sync(0xffffffffu, O & kEscBit))
-            resolve_escapes<SMEM>(p, e, F, (X >> 11) & 1u, (X >> 12) & 1u, L, rb);
+            resolve_escapes<SMEM>(p, F, (X >> 11) & 1u, (X >> 12) & 1u, L, rb);
         // v = F 2^-22 - (2^12 + 256) exactly, w = fp32(f_r v): two coordinates per instruction
         const uint64_t scale2 = pair(__float_as_uint(kInvScale), __float_as_uint(kInvScale));
         const uint64_t bias2 = pair(__float_as_uint(-kBias), __float_as_uint(-kBias));
