@@ -190,17 +190,17 @@ struct Packer<EP_FP32> {
 
 template <>
 struct Packer<EP_INT8> {
-    uint32_t o[2];
+    // clamp to [-127, 127] in fp32, then adding 1.5 * 2^23 rounds to the nearest integer (ties to
+    // even) and leaves the code, two's complement, in the low byte of the sum's bits
+    uint32_t b[8];
     __device__ __forceinline__ void put(int i, float, float w) {
-        int q = min(127, max(-127, __float2int_rn(w)));
-        uint32_t byte = uint32_t(q) & 0xffu;
-        if ((i & 3) == 0)
-            o[i >> 2] = byte;
-        else
-            o[i >> 2] |= byte << (8 * (i & 3));
+        float r = __fadd_rn(fminf(fmaxf(w, -127.0f), 127.0f), 12582912.0f);
+        b[i] = __float_as_uint(r);
     }
-    __device__ __forceinline__ void store(void *out, uint32_t b) {
-        reinterpret_cast<uint2 *>(out)[b] = make_uint2(o[0], o[1]);
+    __device__ __forceinline__ void store(void *out, uint32_t blk) {
+        uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+        uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
+        reinterpret_cast<uint2 *>(out)[blk] = make_uint2(lo, hi);
     }
 };
 
