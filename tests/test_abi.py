@@ -99,3 +99,31 @@ def test_compress_bound_holds():
         assert blob.numel() <= bound
     cfg = B._config(4.0, q_index=900)
     assert B.compress(w, 4.0, q_index=900).numel() <= B.lib().ep_compress_bound(64, 256, C.byref(cfg))
+
+
+def test_decode_calls_reject_bad_arguments_before_any_launch():
+    """argument checks of ep_prepare / ep_decompress / ep_decompress_noalloc happen on the host and
+    need no device: null pointers, misaligned pointers, a container the stream does not hold, a
+    damaged plan"""
+    blob = B.compress(synth.gaussian(16, 64, 0.02, 5), 4.0)
+    info = B.stream_info(blob)
+    L = B.lib()
+    fake, odd = 1 << 20, (1 << 20) + 8  # never dereferenced: every call below fails its checks first
+    assert L.ep_prepare(None, fake, fake, None, None) == -1
+    assert L.ep_prepare(C.byref(info), None, fake, None, None) == -1
+    assert L.ep_prepare(C.byref(info), fake, None, None, None) == -1
+    assert L.ep_prepare(C.byref(info), odd, fake, None, None) == -1
+    assert L.ep_decompress(C.byref(info), fake, None, fake, info.container_dtype, None, None) == -1
+    assert L.ep_decompress(C.byref(info), fake, fake, None, info.container_dtype, None, None) == -1
+    assert L.ep_decompress(C.byref(info), fake, odd, fake, info.container_dtype, None, None) == -1
+    assert L.ep_decompress(C.byref(info), fake, fake, odd, info.container_dtype, None, None) == -1
+    assert L.ep_decompress(C.byref(info), fake, fake, fake, B.INT8, None, None) == -1  # a BF16 stream
+    assert L.ep_decompress(C.byref(info), fake, fake, fake, 99, None, None) == -1
+    assert L.ep_decompress_noalloc(None, fake, fake, info.container_dtype, None, None) == -1
+    bad = B.StreamInfo.from_buffer_copy(info)
+    bad.split[3] = 12  # beyond the largest split of its context
+    assert L.ep_decompress(C.byref(bad), fake, fake, fake, info.container_dtype, None, None) == -6
+    assert L.ep_prepare(C.byref(bad), fake, fake, None, None) == -6
+    bad = B.StreamInfo.from_buffer_copy(info)
+    bad.cols = 60  # not a multiple of 8
+    assert L.ep_decompress(C.byref(bad), fake, fake, fake, info.container_dtype, None, None) == -1

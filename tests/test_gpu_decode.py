@@ -165,3 +165,53 @@ def test_large_tiles(oracle, K, q):
     if K == 1024:
         assert (16 * sizes > 232448).any()
     check_parity(oracle, blob)
+
+
+def _expected_tables(oracle, blob_np):
+    """the decoder's slot tables as include/eptile.h documents them, from the oracle's parse of
+    the stream: per context 2048 entries f << 21 | escape << 20 | field << 11 | (slot - cum);
+    field = v + 256 for a direct token (v its lattice coordinate), the escape index d (2d + c for
+    coordinates 1..6) otherwise; context 3 + 2c + p stored at position 3 + c + 2p"""
+    rc, info = oracle.parse(blob_np)
+    assert rc == 0
+    b = blob_np.tobytes()
+    tab = np.zeros((7, 2048), np.uint32)
+    off = info.off_freq
+    for ctx in range(7):
+        n, m = info.ntok[ctx], info.split[ctx]
+        f = np.frombuffer(b, np.uint16, count=n, offset=off).astype(np.int64)
+        off += 2 * n
+        pos = ctx if ctx < 3 else 3 + ((ctx - 3) >> 1) + 2 * ((ctx - 3) & 1)
+        cum = 0
+        for t in range(n):
+            if t < (1 << m):
+                if ctx == 0:
+                    v = 4 * oracle.unzigzag(t >> 2) + (t & 3)
+                elif ctx < 3:
+                    v = 2 * (2 * oracle.unzigzag(t >> 1) + (t & 1)) + (ctx - 1)
+                else:
+                    v = 2 * (2 * oracle.unzigzag(t) + ((ctx - 3) & 1)) + ((ctx - 3) >> 1)
+                head = (int(f[t]) << 21) | (((v + 256) & 0x1FF) << 11)
+            else:
+                d = t - (1 << m)
+                fv = 2 * d + (ctx - 1) if ctx in (1, 2) else d
+                head = (int(f[t]) << 21) | (1 << 20) | ((fv & 0x1FF) << 11)
+            for s in range(cum, cum + int(f[t])):
+                tab[pos, s] = head | (s - cum)
+            cum += int(f[t])
+    return tab
+
+
+@pytest.mark.parametrize("target,container", [(4.0, 0), (0.5, 0), (8.0, 0), (3.0, B.INT8)])
+def test_prepared_tables_match_documented_layout(oracle, target, container):
+    w = synth.gaussian_outliers(128, 2048, seed=16)
+    rc, blob = oracle.compress(w, target, container=container)
+    assert rc == 0
+    d = torch.from_numpy(blob).cuda()
+    info = B.stream_info(torch.from_numpy(blob))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    work = B.prepare(d, info, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    got = work.cpu().numpy().view(np.uint32).reshape(7, 2048)
+    assert np.array_equal(got, _expected_tables(oracle, blob))
