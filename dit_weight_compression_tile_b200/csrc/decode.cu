@@ -356,8 +356,8 @@ __device__ __forceinline__ void resolve_escapes(const Params &p, uint32_t (&F)[8
 
 // ------------------------------------------------------------------ the blocks of one tile
 // Lane l decodes blocks t*32K + 32k + l, k = 0..K-1.  ACT: the last tile, where lanes run out
-// of blocks.  Returns EP_DEC_* bits.
-template <int DT, bool SMEM, bool ACT, typename Lim>
+// of blocks.  R32: 32 divides the blocks per row.  Returns EP_DEC_* bits.
+template <int DT, bool SMEM, bool ACT, bool R32, typename Lim>
 __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L, uint32_t &rb, uint32_t lut,
                                                   Lim wlim, uint32_t t, uint32_t lane) {
     uint32_t b = t * 32u * p.K + lane;
@@ -366,60 +366,79 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
     float fr = row < p.rows ? __ldg(p.rowf + row) : 0.0f;
     float frn = row + 1 < p.rows ? __ldg(p.rowf + row + 1) : 0.0f;
     uint32_t err = 0;
-    for (uint32_t k = 0; k < p.K; ++k, b += 32u) {
-        bool act = !ACT || b < p.nb;
-        if (ACT && !__any_sync(0xffffffffu, act)) break;
-        // a damaged stream may drive a lane's reads ahead (at most one word per token); stop
-        // before they leave the buffer's slack
-        if ((k & 7u) == 0 && __any_sync(0xffffffffu, L.past(wlim))) {
-            err |= EP_DEC_WORD_OVERRUN;
-            break;
+    uint32_t k = 0;
+    for (;;) {
+        // R32 (32 | blocks per row): the warp's 32 blocks of a step lie in one row, so all lanes
+        // change rows after the same number of steps and the step loop needs no row test
+        uint32_t kseg = p.K;
+        if constexpr (R32) {
+            uint32_t left = (p.cb - (col - lane)) >> 5;
+            kseg = k + left < p.K ? k + left : p.K;
         }
-        uint32_t e[8];
-        // coordinate 0 (context 0); bit 11 of every entry of contexts 0..2 is the coset c
-        e[0] = step<SMEM, ACT>(L, act, lut);
-        uint32_t lutc = lut + kSlotBytes + ((e[0] & 0x800u) << 2);  // context 1 + c
-#pragma unroll
-        for (int i = 1; i < 7; ++i) e[i] = step<SMEM, ACT>(L, act, lutc);
-        // bits 11 and 12 of the XOR of entries 0..6 are c (seven copies) and the parity p of
-        // y0..y6; context 3 + 2c + p sits at table position 3 + c + 2p
-        uint32_t X = e[0] ^ e[1] ^ e[2] ^ e[3] ^ e[4] ^ e[5] ^ e[6];
-        uint32_t lut7 = lut + 3u * kSlotBytes + ((X & 0x1800u) << 2);
-        e[7] = step<SMEM, ACT>(L, act, lut7);
-        // F keeps the value field and the escape flag of each entry (the flag only matters for
-        // escapes, whose F is rebuilt), so the entries themselves die here
-        uint32_t F[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) F[i] = (e[i] & (kFieldMask | kEscBit)) | kMagic;
-        uint32_t O = F[0] | F[1] | F[2] | F[3] | F[4] | F[5] | F[6] | F[7];
-        if (__any_sync(0xffffffffu, O & kEscBit))
-            resolve_escapes<SMEM>(p, F, (X >> 11) & 1u, (X >> 12) & 1u, L, rb);
-        // v = F 2^-22 - (2^12 + 256) exactly, w = fp32(f_r v): two coordinates per instruction
-        const uint64_t scale2 = pair(__float_as_uint(kInvScale), __float_as_uint(kInvScale));
-        const uint64_t bias2 = pair(__float_as_uint(-kBias), __float_as_uint(-kBias));
-        const uint64_t fr2 = pair(__float_as_uint(fr), __float_as_uint(fr));
-        Packer<DT> pk;
-#pragma unroll
-        for (int i = 0; i < 8; i += 2) {
-            uint64_t v2 = fma_x2(pair(F[i], F[i + 1]), scale2, bias2);
-            uint64_t w2 = mul_x2(v2, fr2);
-            pk.put(i, __uint_as_float(uint32_t(v2)), __uint_as_float(uint32_t(w2)));
-            pk.put(i + 1, __uint_as_float(uint32_t(v2 >> 32)), __uint_as_float(uint32_t(w2 >> 32)));
-        }
-        if (act) pk.store(p.out, b);
-        col += 32u;
-        if (col >= p.cb) {  // next row (all lanes at once when a row holds a multiple of 32 blocks)
-            col -= p.cb;
-            ++row;
-            fr = frn;
-            while (col >= p.cb) {
-                col -= p.cb;
-                ++row;
-                fr = row < p.rows ? __ldg(p.rowf + row) : 0.0f;
+        for (; k < kseg; ++k, b += 32u) {
+            bool act = !ACT || b < p.nb;
+            if (ACT && !__any_sync(0xffffffffu, act)) goto done;
+            // a damaged stream may drive a lane's reads ahead (at most one word per token); stop
+            // before they leave the buffer's slack
+            if ((k & 7u) == 0 && __any_sync(0xffffffffu, L.past(wlim))) {
+                err |= EP_DEC_WORD_OVERRUN;
+                goto done;
             }
-            frn = row + 1 < p.rows ? __ldg(p.rowf + row + 1) : 0.0f;
+            uint32_t e[8];
+            // coordinate 0 (context 0); bit 11 of every entry of contexts 0..2 is the coset c
+            e[0] = step<SMEM, ACT>(L, act, lut);
+            uint32_t lutc = lut + kSlotBytes + ((e[0] & 0x800u) << 2);  // context 1 + c
+#pragma unroll
+            for (int i = 1; i < 7; ++i) e[i] = step<SMEM, ACT>(L, act, lutc);
+            // bits 11 and 12 of the XOR of entries 0..6 are c (seven copies) and the parity p of
+            // y0..y6; context 3 + 2c + p sits at table position 3 + c + 2p
+            uint32_t X = e[0] ^ e[1] ^ e[2] ^ e[3] ^ e[4] ^ e[5] ^ e[6];
+            uint32_t lut7 = lut + 3u * kSlotBytes + ((X & 0x1800u) << 2);
+            e[7] = step<SMEM, ACT>(L, act, lut7);
+            // F keeps the value field and the escape flag of each entry (the flag only matters for
+            // escapes, whose F is rebuilt), so the entries themselves die here
+            uint32_t F[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) F[i] = (e[i] & (kFieldMask | kEscBit)) | kMagic;
+            uint32_t O = F[0] | F[1] | F[2] | F[3] | F[4] | F[5] | F[6] | F[7];
+            if (__any_sync(0xffffffffu, O & kEscBit))
+                resolve_escapes<SMEM>(p, F, (X >> 11) & 1u, (X >> 12) & 1u, L, rb);
+            // v = F 2^-22 - (2^12 + 256) exactly, w = fp32(f_r v): two coordinates per instruction
+            const uint64_t scale2 = pair(__float_as_uint(kInvScale), __float_as_uint(kInvScale));
+            const uint64_t bias2 = pair(__float_as_uint(-kBias), __float_as_uint(-kBias));
+            const uint64_t fr2 = pair(__float_as_uint(fr), __float_as_uint(fr));
+            Packer<DT> pk;
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+                uint64_t v2 = fma_x2(pair(F[i], F[i + 1]), scale2, bias2);
+                uint64_t w2 = mul_x2(v2, fr2);
+                pk.put(i, __uint_as_float(uint32_t(v2)), __uint_as_float(uint32_t(w2)));
+                pk.put(i + 1, __uint_as_float(uint32_t(v2 >> 32)), __uint_as_float(uint32_t(w2 >> 32)));
+            }
+            if (act) pk.store(p.out, b);
+            if constexpr (!R32) {
+                col += 32u;
+                if (col >= p.cb) {  // next row
+                    col -= p.cb;
+                    ++row;
+                    fr = frn;
+                    while (col >= p.cb) {
+                        col -= p.cb;
+                        ++row;
+                        fr = row < p.rows ? __ldg(p.rowf + row) : 0.0f;
+                    }
+                    frn = row + 1 < p.rows ? __ldg(p.rowf + row + 1) : 0.0f;
+                }
+            }
         }
+        if (!R32 || k >= p.K) break;
+        // the segment ended at the end of the row: the next step starts the next row at column lane
+        col = lane;
+        ++row;
+        fr = frn;
+        frn = row + 1 < p.rows ? __ldg(p.rowf + row + 1) : 0.0f;
     }
+done:
     return err;
 }
 
@@ -456,18 +475,22 @@ __device__ __forceinline__ uint32_t decode_tile(const Params &p, uint32_t lut, P
         L.w = lds16(L.wp);
         uint32_t wlim = L.area + 2u * capacity;
         if (uint64_t(t + 1) * 32u * p.K <= p.nb)
-            err = decode_blocks<DT, SMEM, false>(p, L, rb, lut, wlim, t, lane);
+            err = (p.cb & 31u) == 0 ? decode_blocks<DT, SMEM, false, true>(p, L, rb, lut, wlim, t, lane)
+                                : decode_blocks<DT, SMEM, false, false>(p, L, rb, lut, wlim, t, lane);
         else
-            err = decode_blocks<DT, SMEM, true>(p, L, rb, lut, wlim, t, lane);
+            err = (p.cb & 31u) == 0 ? decode_blocks<DT, SMEM, true, true>(p, L, rb, lut, wlim, t, lane)
+                                : decode_blocks<DT, SMEM, true, false>(p, L, rb, lut, wlim, t, lane);
     } else {
         L.area = reinterpret_cast<const uint16_t *>(head + kTileHead);
         L.wlim = L.area + (capacity ? capacity - 1u : 0u);
         L.wp = L.area + start < L.wlim ? L.area + start : L.wlim;
         L.w = __ldg(L.wp);
         if (uint64_t(t + 1) * 32u * p.K <= p.nb)
-            err = decode_blocks<DT, SMEM, false>(p, L, rb, lut, L.wlim, t, lane);
+            err = (p.cb & 31u) == 0 ? decode_blocks<DT, SMEM, false, true>(p, L, rb, lut, L.wlim, t, lane)
+                                : decode_blocks<DT, SMEM, false, false>(p, L, rb, lut, L.wlim, t, lane);
         else
-            err = decode_blocks<DT, SMEM, true>(p, L, rb, lut, L.wlim, t, lane);
+            err = (p.cb & 31u) == 0 ? decode_blocks<DT, SMEM, true, true>(p, L, rb, lut, L.wlim, t, lane)
+                                : decode_blocks<DT, SMEM, true, false>(p, L, rb, lut, L.wlim, t, lane);
     }
     if (L.x != kStateLow) err |= EP_DEC_BAD_END;
     // the front (rANS words) and the back (raw bits) cover the region exactly
