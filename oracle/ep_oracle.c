@@ -1136,6 +1136,7 @@ typedef struct {
     uint16_t *slot_tok[NCTX]; /* slot -> token (0xffff: slot outside the table) */
     uint32_t *freq[NCTX], *cum[NCTX];
     const uint8_t *rowf;
+    int32_t out_dtype; /* the container's dtype unless a float output dtype is asked for */
 } dec_ctx;
 
 static int dec_open(dec_ctx *D, const uint8_t *p, size_t n)
@@ -1145,6 +1146,7 @@ static int dec_open(dec_ctx *D, const uint8_t *p, size_t n)
         return rc;
     D->p = p;
     D->rowf = p + D->in.off_rowf;
+    D->out_dtype = D->in.container_dtype;
     size_t q = D->in.off_freq;
     for (int c = 0; c < NCTX; c++) {
         uint32_t nt = D->in.ntok[c];
@@ -1246,7 +1248,7 @@ static void decode_tile(dec_ctx *D, int64_t t, int32_t *vout, void *out, uint32_
     uint64_t tile_bytes = 16 * (uint64_t)(get32(dir + 4 * (t + 1)) - get32(dir + 4 * t));
     uint64_t capacity = (tile_bytes - TILE_HEAD) / 2, start = 0;
     int64_t base = t * (int64_t)LANES * K;
-    int esz = elt_size(I->container_dtype);
+    int esz = elt_size(D->out_dtype);
     for (int l = 0; l < LANES; l++) {
         uint32_t x = get32(tp + 4 * l);
         uint64_t len = get16(tp + 4 * LANES + 2 * l), pos = 0;
@@ -1307,7 +1309,7 @@ static void decode_tile(dec_ctx *D, int64_t t, int32_t *vout, void *out, uint32_
                 float wv[8];
                 for (int i = 0; i < 8; i++)
                     wv[i] = fr * (float)v[i];
-                or_convert_batch(wv, 8, I->container_dtype, (uint8_t *)out + (size_t)(8 * b) * (size_t)esz);
+                or_convert_batch(wv, 8, D->out_dtype, (uint8_t *)out + (size_t)(8 * b) * (size_t)esz);
             }
         }
         if (x != STATE_L)
@@ -1324,11 +1326,30 @@ static void decode_tile(dec_ctx *D, int64_t t, int32_t *vout, void *out, uint32_
 int or_decode(const uint8_t *blob, size_t n, uint32_t t0, uint32_t t1, int32_t *v, void *out,
               uint32_t *status)
 {
+    return or_decode_as(blob, n, t0, t1, v, out, 0, status);
+}
+
+/* [API] CompressedTensor.to(dtype=...): the output dtype changes without recompression.
+ * Reading: the fp32 weight f_r * v is rounded once into the requested dtype; a float
+ * container (BF16 / FP16 / FP32) may decode to any of the three, a code container only to
+ * its own dtype. */
+int or_decode_as(const uint8_t *blob, size_t n, uint32_t t0, uint32_t t1, int32_t *v, void *out,
+                 int32_t out_dtype, uint32_t *status)
+{
     dec_ctx D;
     uint32_t st = 0;
     int rc = dec_open(&D, blob, n);
     if (rc)
         return rc;
+    if (out_dtype) {
+        int fo = out_dtype >= ORD_BF16 && out_dtype <= ORD_FP32;
+        int fc = D.in.container_dtype >= ORD_BF16 && D.in.container_dtype <= ORD_FP32;
+        if (out_dtype != D.in.container_dtype && !(fo && fc)) {
+            dec_close(&D);
+            return OR_ERR_INVALID_ARG;
+        }
+        D.out_dtype = out_dtype;
+    }
     if (t1 > D.in.n_tiles)
         t1 = D.in.n_tiles;
     for (uint32_t t = t0; t < t1; t++)

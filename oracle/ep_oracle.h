@@ -118,6 +118,11 @@ int or_parse(const uint8_t *blob, size_t nbytes, or_info *info);
  * and ORs OR_DEC_* bits into *status */
 int or_decode(const uint8_t *blob, size_t nbytes, uint32_t t0, uint32_t t1, int32_t *v, void *out,
               uint32_t *status);
+/* or_decode with the output rounded into out_dtype (0: the container's dtype); a float
+ * container decodes to BF16, FP16 or FP32, a code container to its own dtype only
+ * (OR_ERR_INVALID_ARG otherwise) */
+int or_decode_as(const uint8_t *blob, size_t nbytes, uint32_t t0, uint32_t t1, int32_t *v, void *out,
+                 int32_t out_dtype, uint32_t *status);
 /* coding statistics over the whole stream, from a decode */
 int or_code_stats(const uint8_t *blob, size_t nbytes, double *ideal_bits, double *emp_entropy_bits,
                   double *extra_bits, uint64_t *n_symbols, uint64_t *payload_bytes);

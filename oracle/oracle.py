@@ -76,6 +76,8 @@ def lib():
         L.or_parse.argtypes = [p, C.c_size_t, C.POINTER(Info)]
         L.or_decode.restype = C.c_int
         L.or_decode.argtypes = [p, C.c_size_t, C.c_uint32, C.c_uint32, p, p, C.POINTER(C.c_uint32)]
+        L.or_decode_as.restype = C.c_int
+        L.or_decode_as.argtypes = [p, C.c_size_t, C.c_uint32, C.c_uint32, p, p, C.c_int32, C.POINTER(C.c_uint32)]
         L.or_code_stats.restype = C.c_int
         L.or_code_stats.argtypes = [p, C.c_size_t, C.POINTER(C.c_double), C.POINTER(C.c_double),
                                     C.POINTER(C.c_double), C.POINTER(C.c_uint64), C.POINTER(C.c_uint64)]
@@ -261,9 +263,11 @@ def parse(blob):
     return rc, info
 
 
-def decode(blob, t0=0, t1=None, want_v=True, want_out=True, out_buf=None):
+def decode(blob, t0=0, t1=None, want_v=True, want_out=True, out_buf=None, out_dtype=0):
     """Returns (rc, status, v (rows, cols) int32 or None, out (rows, cols) container array or None).
-    ``out_buf``: optional preallocated container array to decode into."""
+    ``out_buf``: optional preallocated container array to decode into.  ``out_dtype``: 0 (the
+    container's dtype) or, for a float container, BF16 / FP16 / FP32 (to(dtype=...) of the API
+    reference: the fp32 weight rounded once into that dtype)."""
     blob = np.ascontiguousarray(blob, dtype=np.uint8)
     rc, info = parse(blob)
     if rc != OK:
@@ -273,11 +277,11 @@ def decode(blob, t0=0, t1=None, want_v=True, want_out=True, out_buf=None):
     if out_buf is not None:
         out = out_buf
     else:
-        out = np.zeros((R, Cc), NP_DTYPE[info.container_dtype]) if want_out else None
+        out = np.zeros((R, Cc), NP_DTYPE[out_dtype or info.container_dtype]) if want_out else None
     st = C.c_uint32(0)
     t1 = info.n_tiles if t1 is None else t1
-    rc = lib().or_decode(_ptr(blob), blob.size, t0, t1, _ptr(v) if v is not None else None,
-                         _ptr(out) if out is not None else None, C.byref(st))
+    rc = lib().or_decode_as(_ptr(blob), blob.size, t0, t1, _ptr(v) if v is not None else None,
+                            _ptr(out) if out is not None else None, int(out_dtype), C.byref(st))
     return rc, st.value, v, out
 
 
