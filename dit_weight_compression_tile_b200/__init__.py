@@ -9,8 +9,14 @@ _BINDING_NAMES = ("BF16", "FP16", "FP32", "INT8", "FP8E4M3", "EpError", "compres
                   "stream_info", "lib", "StreamInfo")
 
 
+_COMPRESSED_NAMES = ("CompressedTensor", "LatticeRANSConfig")
+
+
 def __getattr__(name):
     if name in _BINDING_NAMES:
         from . import binding
         return getattr(binding, name)
+    if name in _COMPRESSED_NAMES:
+        from . import compressed
+        return getattr(compressed, name)
     raise AttributeError(name)

@@ -159,7 +159,19 @@ def prepare(d_blob, info=None, workspace=None, status=None, stream=None):
     return workspace
 
 
-def decompress(d_blob, info=None, workspace=None, out=None, status=None, stream=None, lattice=False):
+def dtype_code(d):
+    """EP_* dtype code of a torch dtype, a name ("bf16", ...) or a code"""
+    if isinstance(d, torch.dtype):
+        if d not in CODE_OF:
+            raise EpError(-1, f"no container dtype for {d}")
+        return CODE_OF[d]
+    if isinstance(d, str):
+        return NAMES[d]
+    return int(d)
+
+
+def decompress(d_blob, info=None, workspace=None, out=None, status=None, stream=None, lattice=False,
+               out_dtype=None):
     """decompress(compressed): the fused GPU decode of a device-resident stream.
 
     ``d_blob``: CUDA uint8 tensor holding the whole stream.  ``info``: from ``stream_info``
@@ -168,21 +180,24 @@ def decompress(d_blob, info=None, workspace=None, out=None, status=None, stream=
     tensor of ``info.shape`` / ``info.dtype``.  ``status``: optional CUDA int32 tensor of one
     element into which damage flags are ORed.  Launches on ``stream`` (default: the current
     stream).  ``lattice=True`` returns the decoded lattice points v = 2z (int32) instead of
-    weights."""
+    weights.  ``out_dtype``: for a BF16 / FP16 / FP32 container, any of the three (the fp32
+    weight rounded once into it); default the container's dtype."""
     if not d_blob.is_cuda:
         raise EpError(-1, "decompress needs the stream in device memory")
     if info is None:
         info = stream_info(d_blob.cpu())
     if workspace is None:
         workspace = prepare(d_blob, info, status=status, stream=stream)
-    want = torch.int32 if lattice else info.dtype
+    dt = LATTICE_I32 if lattice else (info.container_dtype if out_dtype is None else dtype_code(out_dtype))
+    want = torch.int32 if lattice else TORCH_DTYPE.get(dt)
+    if want is None:
+        raise EpError(-1, f"output dtype code {dt}")
     if out is None:
         out = torch.empty(info.shape, dtype=want, device=d_blob.device)
     if not out.is_cuda or out.dtype != want or tuple(out.shape) != info.shape or not out.is_contiguous():
         raise EpError(-1, "output tensor does not match the stream")
     st = status.data_ptr() if status is not None else None
     s = (stream or torch.cuda.current_stream(d_blob.device)).cuda_stream
-    dt = LATTICE_I32 if lattice else info.container_dtype
     rc = lib().ep_decompress(C.byref(info), d_blob.data_ptr(), workspace.data_ptr(), out.data_ptr(), dt, st, s)
     if rc != 0:
         raise EpError(rc, "ep_decompress")

@@ -763,6 +763,13 @@ int check_info(const ep_info *info) {
     return EP_OK;
 }
 
+// the container's dtype, another float dtype for a float container, or the lattice points
+bool out_dtype_ok(const ep_info *info, int32_t out_dtype) {
+    auto is_float = [](int32_t d) { return d == EP_BF16 || d == EP_FP16 || d == EP_FP32; };
+    return out_dtype == info->container_dtype || out_dtype == EP_LATTICE_I32 ||
+           (is_float(out_dtype) && is_float(info->container_dtype));
+}
+
 uint32_t pack_splits(const ep_info *info) {
     uint32_t s = 0;
     for (int c = 0; c < kContexts; ++c) s |= uint32_t(info->split[c]) << (4 * c);
@@ -796,7 +803,7 @@ extern "C" int ep_decompress(const ep_info *info, const void *d_blob, const void
                              int32_t out_dtype, uint32_t *d_status, ep_stream_t stream) {
     using namespace ep;
     if (!info || !d_blob || !d_workspace || !d_out) return EP_ERR_INVALID_ARG;
-    if (out_dtype != info->container_dtype && out_dtype != EP_LATTICE_I32) return EP_ERR_INVALID_ARG;
+    if (!out_dtype_ok(info, out_dtype)) return EP_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(d_blob) | reinterpret_cast<uintptr_t>(d_out) |
          reinterpret_cast<uintptr_t>(d_workspace)) & 15u)
         return EP_ERR_INVALID_ARG;
@@ -872,7 +879,7 @@ int static_tables(void **out) {
 extern "C" int ep_decompress_noalloc(const ep_info *info, const void *d_blob, void *d_out, int32_t out_dtype,
                                      uint32_t *d_status, ep_stream_t stream) {
     using namespace ep;
-    if (!info) return EP_ERR_INVALID_ARG;
+    if (!info || !d_blob || !d_out || !out_dtype_ok(info, out_dtype)) return EP_ERR_INVALID_ARG;
     if (info->workspace_nbytes > kStaticTablesBytes) return EP_ERR_UNSUPPORTED;
     void *tables = nullptr;
     int rc = static_tables(&tables);

@@ -140,8 +140,12 @@ int ep_prepare(const ep_info *info, const void *d_blob, void *d_workspace, uint3
  *   d_blob      device pointer to the whole stream (info->storage_nbytes bytes), 16-byte aligned.
  *   d_workspace the workspace ep_prepare filled for this stream (read only here).
  *   d_out       device pointer to rows * cols elements of out_dtype, row-major, 16-byte aligned.
- *   out_dtype   info->container_dtype (the reconstructed weights or codes), or EP_LATTICE_I32 for
- *               the decoded lattice points v = 2z (int32) before scaling; no other conversion.
+ *   out_dtype   info->container_dtype (the reconstructed weights or codes); for a BF16, FP16 or
+ *               FP32 container also either of the other two ("to(dtype=...)" of the API
+ *               reference: the output dtype changes without recompression; the fp32 weight
+ *               f_r * v is rounded once, to nearest even, into out_dtype); or EP_LATTICE_I32 for
+ *               the decoded lattice points v = 2z (int32) before scaling.  INT8 / FP8 code
+ *               containers decode to their own dtype only.  Anything else: EP_ERR_INVALID_ARG.
  *   d_status    nullable device pointer to one uint32; the kernel ORs EP_DEC_* bits into it
  *               when it meets a damaged tile (clear it before the call to read it per call).
  *   stream      CUDA stream of the launch.

@@ -120,6 +120,10 @@ def test_decode_calls_reject_bad_arguments_before_any_launch():
     assert L.ep_decompress(C.byref(info), fake, fake, fake, B.INT8, None, None) == -1  # a BF16 stream
     assert L.ep_decompress(C.byref(info), fake, fake, fake, 99, None, None) == -1
     assert L.ep_decompress_noalloc(None, fake, fake, info.container_dtype, None, None) == -1
+    assert L.ep_decompress_noalloc(C.byref(info), fake, fake, B.INT8, None, None) == -1
+    codes = B.stream_info(B.compress(synth.gaussian(64, 256, 0.02, 5), 6.0, container=B.INT8))
+    for dt in (B.BF16, B.FP16, B.FP32, B.FP8E4M3):  # code containers decode to their own dtype only
+        assert L.ep_decompress(C.byref(codes), fake, fake, fake, dt, None, None) == -1
     bad = B.StreamInfo.from_buffer_copy(info)
     bad.split[3] = 12  # beyond the largest split of its context
     assert L.ep_decompress(C.byref(bad), fake, fake, fake, info.container_dtype, None, None) == -6
