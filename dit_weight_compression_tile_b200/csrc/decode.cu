@@ -65,15 +65,22 @@ struct Params {
     void *out;               // container, row-major
     uint32_t *status;        // nullable
     uint64_t tile_units;     // size of the tile section in 16-byte units
-    uint32_t nb;             // E8 blocks (rows * cols / 8)
+    uint64_t cols;           // row length of the output in elements
+    uint32_t nb;             // E8 blocks (rows * cb)
     uint32_t rows;
-    uint32_t cb;             // blocks per row
+    uint32_t cb;             // blocks per row, ceil(cols / 8): a row is zero-padded to whole blocks
     uint32_t K;              // blocks per lane
     uint32_t T;              // tiles
     uint32_t tile_buf;       // bytes of each tile buffer (multiple of 16, includes kSlack)
     uint32_t nbuf;           // tile buffers per warp (1 or 2); 0: tiles are read from global memory
     uint32_t splits;         // 4 bits per context
 };
+
+// How a stream's blocks map onto rows, fixed per launch: kRowsAny (a lane's row is tested after
+// every block), kRows32 (32 divides the blocks per row: a warp's step never straddles rows, so the
+// loop runs row segment by row segment) and kRowsPadded (cols % 8 != 0: rows are zero-padded to
+// whole E8 blocks and stores go element by element).
+enum RowLayout { kRowsAny = 0, kRows32 = 1, kRowsPadded = 2 };
 
 __device__ __forceinline__ uint32_t split_of_bits(uint32_t splits, uint32_t c) { return (splits >> (4 * c)) & 15u; }
 __device__ __forceinline__ uint32_t split_of(const Params &p, uint32_t c) { return split_of_bits(p.splits, c); }
@@ -158,6 +165,11 @@ struct Packer<EP_BF16> {
     __device__ __forceinline__ void store(void *out, uint32_t b) {
         reinterpret_cast<uint4 *>(out)[b] = make_uint4(o[0], o[1], o[2], o[3]);
     }
+    // the first n values at element e (the last block of a padded row: no vector store)
+    __device__ __forceinline__ void store_n(void *out, uint64_t e, uint32_t n) {
+        for (uint32_t i = 0; i < n; ++i)
+            reinterpret_cast<uint16_t *>(out)[e + i] = uint16_t(o[i >> 1] >> (16 * (i & 1)));
+    }
 };
 
 template <>
@@ -175,6 +187,10 @@ struct Packer<EP_FP16> {
     __device__ __forceinline__ void store(void *out, uint32_t b) {
         reinterpret_cast<uint4 *>(out)[b] = make_uint4(o[0], o[1], o[2], o[3]);
     }
+    __device__ __forceinline__ void store_n(void *out, uint64_t e, uint32_t n) {
+        for (uint32_t i = 0; i < n; ++i)
+            reinterpret_cast<uint16_t *>(out)[e + i] = uint16_t(o[i >> 1] >> (16 * (i & 1)));
+    }
 };
 
 template <>
@@ -185,6 +201,9 @@ struct Packer<EP_FP32> {
         float4 *p = reinterpret_cast<float4 *>(out) + 2 * size_t(b);
         p[0] = make_float4(o[0], o[1], o[2], o[3]);
         p[1] = make_float4(o[4], o[5], o[6], o[7]);
+    }
+    __device__ __forceinline__ void store_n(void *out, uint64_t e, uint32_t n) {
+        for (uint32_t i = 0; i < n; ++i) reinterpret_cast<float *>(out)[e + i] = o[i];
     }
 };
 
@@ -201,6 +220,9 @@ struct Packer<EP_INT8> {
         uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
         uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
         reinterpret_cast<uint2 *>(out)[blk] = make_uint2(lo, hi);
+    }
+    __device__ __forceinline__ void store_n(void *out, uint64_t e, uint32_t n) {
+        for (uint32_t i = 0; i < n; ++i) reinterpret_cast<uint8_t *>(out)[e + i] = uint8_t(b[i]);
     }
 };
 
@@ -222,6 +244,9 @@ struct Packer<EP_FP8_E4M3> {
     __device__ __forceinline__ void store(void *out, uint32_t b) {
         reinterpret_cast<uint2 *>(out)[b] = make_uint2(o[0], o[1]);
     }
+    __device__ __forceinline__ void store_n(void *out, uint64_t e, uint32_t n) {
+        for (uint32_t i = 0; i < n; ++i) reinterpret_cast<uint8_t *>(out)[e + i] = uint8_t(o[i >> 2] >> (8 * (i & 3)));
+    }
 };
 
 // the lattice points themselves (v = 2z, int32), for consumers and bit-exact checks
@@ -233,6 +258,9 @@ struct Packer<EP_LATTICE_I32> {
         int4 *p = reinterpret_cast<int4 *>(out) + 2 * size_t(b);
         p[0] = make_int4(o[0], o[1], o[2], o[3]);
         p[1] = make_int4(o[4], o[5], o[6], o[7]);
+    }
+    __device__ __forceinline__ void store_n(void *out, uint64_t e, uint32_t n) {
+        for (uint32_t i = 0; i < n; ++i) reinterpret_cast<int32_t *>(out)[e + i] = o[i];
     }
 };
 
@@ -356,8 +384,8 @@ __device__ __forceinline__ void resolve_escapes(const Params &p, uint32_t (&F)[8
 
 // ------------------------------------------------------------------ the blocks of one tile
 // Lane l decodes blocks t*32K + 32k + l, k = 0..K-1.  ACT: the last tile, where lanes run out
-// of blocks.  R32: 32 divides the blocks per row.  Returns EP_DEC_* bits.
-template <int DT, bool SMEM, bool ACT, bool R32, typename Lim>
+// of blocks.  ROWS: the launch's RowLayout.  Returns EP_DEC_* bits.
+template <int DT, bool SMEM, bool ACT, int ROWS, typename Lim>
 __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L, uint32_t &rb, uint32_t lut,
                                                   Lim wlim, uint32_t t, uint32_t lane) {
     uint32_t b = t * 32u * p.K + lane;
@@ -365,6 +393,7 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
     // the factor of the current row and of the next one (read a row ahead)
     float fr = row < p.rows ? __ldg(p.rowf + row) : 0.0f;
     float frn = row + 1 < p.rows ? __ldg(p.rowf + row + 1) : 0.0f;
+    constexpr bool R32 = ROWS == kRows32, RAG = ROWS == kRowsPadded;
     uint32_t err = 0;
     uint32_t k = 0;
     for (;;) {
@@ -415,7 +444,13 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
                 pk.put(i, __uint_as_float(uint32_t(v2)), __uint_as_float(uint32_t(w2)));
                 pk.put(i + 1, __uint_as_float(uint32_t(v2 >> 32)), __uint_as_float(uint32_t(w2 >> 32)));
             }
-            if (act) pk.store(p.out, b);
+            if constexpr (RAG) {
+                // a padded row's last block keeps its first cols % 8 values
+                const uint64_t c0 = 8ull * col;
+                if (act) pk.store_n(p.out, uint64_t(row) * p.cols + c0, uint32_t(min(p.cols - c0, uint64_t(8))));
+            } else if (act) {
+                pk.store(p.out, b);
+            }
             if constexpr (!R32) {
                 col += 32u;
                 if (col >= p.cb) {  // next row
@@ -444,7 +479,7 @@ done:
 
 // Decodes tile t with one warp.  `head` points at the tile (states, region lengths, word area):
 // a shared address (SMEM) or a global pointer.  Returns the EP_DEC_* bits of this lane.
-template <int DT, bool SMEM, typename Ptr>
+template <int DT, int ROWS, bool SMEM, typename Ptr>
 __device__ __forceinline__ uint32_t decode_tile(const Params &p, uint32_t lut, Ptr head, uint32_t tile_bytes,
                                                 uint32_t t, uint32_t lane) {
     Lane<SMEM> L;
@@ -475,22 +510,18 @@ __device__ __forceinline__ uint32_t decode_tile(const Params &p, uint32_t lut, P
         L.w = lds16(L.wp);
         uint32_t wlim = L.area + 2u * capacity;
         if (uint64_t(t + 1) * 32u * p.K <= p.nb)
-            err = (p.cb & 31u) == 0 ? decode_blocks<DT, SMEM, false, true>(p, L, rb, lut, wlim, t, lane)
-                                : decode_blocks<DT, SMEM, false, false>(p, L, rb, lut, wlim, t, lane);
+            err = decode_blocks<DT, SMEM, false, ROWS>(p, L, rb, lut, wlim, t, lane);
         else
-            err = (p.cb & 31u) == 0 ? decode_blocks<DT, SMEM, true, true>(p, L, rb, lut, wlim, t, lane)
-                                : decode_blocks<DT, SMEM, true, false>(p, L, rb, lut, wlim, t, lane);
+            err = decode_blocks<DT, SMEM, true, ROWS>(p, L, rb, lut, wlim, t, lane);
     } else {
         L.area = reinterpret_cast<const uint16_t *>(head + kTileHead);
         L.wlim = L.area + (capacity ? capacity - 1u : 0u);
         L.wp = L.area + start < L.wlim ? L.area + start : L.wlim;
         L.w = __ldg(L.wp);
         if (uint64_t(t + 1) * 32u * p.K <= p.nb)
-            err = (p.cb & 31u) == 0 ? decode_blocks<DT, SMEM, false, true>(p, L, rb, lut, L.wlim, t, lane)
-                                : decode_blocks<DT, SMEM, false, false>(p, L, rb, lut, L.wlim, t, lane);
+            err = decode_blocks<DT, SMEM, false, ROWS>(p, L, rb, lut, L.wlim, t, lane);
         else
-            err = (p.cb & 31u) == 0 ? decode_blocks<DT, SMEM, true, true>(p, L, rb, lut, L.wlim, t, lane)
-                                : decode_blocks<DT, SMEM, true, false>(p, L, rb, lut, L.wlim, t, lane);
+            err = decode_blocks<DT, SMEM, true, ROWS>(p, L, rb, lut, L.wlim, t, lane);
     }
     if (L.x != kStateLow) err |= EP_DEC_BAD_END;
     // the front (rANS words) and the back (raw bits) cover the region exactly
@@ -598,7 +629,7 @@ __global__ void __launch_bounds__(kPrepThreads) prepare_kernel(const __grid_cons
 
 // ------------------------------------------------------------------ decode kernel
 // Shared memory: the slot tables, mbarriers, then nbuf tile buffers per warp.
-template <int DT>
+template <int DT, int ROWS>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
@@ -674,9 +705,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_
                 if (nbuf > 1 && (pend & (1u << o))) mbar_wait(bars + 16u * warp + 8u * o, (phase >> o) & 1u);
                 return;
             }
-            if (tables_ok) err = decode_tile<DT, true>(p, lut, bufs + b * p.tile_buf, bytes, t, lane);
+            if (tables_ok) err = decode_tile<DT, ROWS, true>(p, lut, bufs + b * p.tile_buf, bytes, t, lane);
         } else if (tables_ok) {
-            err = decode_tile<DT, false>(p, lut, p.tiles + size_t(beg) * 16, bytes, t, lane);
+            err = decode_tile<DT, ROWS, false>(p, lut, p.tiles + size_t(beg) * 16, bytes, t, lane);
         }
         if (err && p.status) atomicOr(p.status, err);
         __syncwarp();
@@ -704,8 +735,10 @@ cudaError_t launch(Params &p, uint64_t max_tile, int device, cudaStream_t stream
             if (e != cudaSuccess) return e;
         }
         if (!g_cache.attr[device][DT]) {
-            cudaError_t e = cudaFuncSetAttribute(decode_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 int(kSmemLimit));
+            cudaError_t e = cudaSuccess;
+            for (auto k : {decode_kernel<DT, kRowsAny>, decode_kernel<DT, kRows32>, decode_kernel<DT, kRowsPadded>})
+                if (e == cudaSuccess)
+                    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemLimit));
             if (e != cudaSuccess) return e;
             g_cache.attr[device][DT] = true;
         }
@@ -746,13 +779,16 @@ cudaError_t launch(Params &p, uint64_t max_tile, int device, cudaStream_t stream
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<DT>, p);
+    if (p.cols & 7u) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsPadded>, p);
+    if ((p.cb & 31u) == 0) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRows32>, p);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsAny>, p);
 }
 
 int check_info(const ep_info *info) {
-    if (info->rows <= 0 || info->cols <= 0 || info->cols % 8 || info->n_tiles == 0) return EP_ERR_INVALID_ARG;
-    int64_t nb = info->rows * (info->cols / 8);
-    if (nb >= (int64_t(1) << 31) || info->cols / 8 >= (int64_t(1) << 31)) return EP_ERR_UNSUPPORTED;
+    if (info->rows <= 0 || info->cols <= 0 || info->n_tiles == 0) return EP_ERR_INVALID_ARG;
+    const int64_t cb = (info->cols + 7) / 8;  // rows zero-padded to whole E8 blocks
+    if (info->rows >= (int64_t(1) << 31) || cb >= (int64_t(1) << 31) || info->rows * cb >= (int64_t(1) << 31))
+        return EP_ERR_UNSUPPORTED;
     uint32_t total = 0;
     for (int c = 0; c < kContexts; ++c) {
         if (!split_valid(info->split[c], c) || info->ntok[c] > split_alphabet(info->split[c], kCtxLow[c]))
@@ -818,9 +854,10 @@ extern "C" int ep_decompress(const ep_info *info, const void *d_blob, const void
     p.out = d_out;
     p.status = d_status;
     p.tile_units = (info->storage_nbytes - info->off_tiles) / 16;
-    p.nb = uint32_t(info->rows * (info->cols / 8));
+    p.cols = uint64_t(info->cols);
+    p.cb = uint32_t((info->cols + 7) / 8);
+    p.nb = uint32_t(info->rows) * p.cb;
     p.rows = uint32_t(info->rows);
-    p.cb = uint32_t(info->cols / 8);
     p.K = info->blocks_per_lane;
     p.T = info->n_tiles;
     p.splits = pack_splits(info);

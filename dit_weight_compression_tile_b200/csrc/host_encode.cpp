@@ -273,7 +273,7 @@ uint32_t build_freqs(const std::vector<uint64_t> &cnt, std::vector<uint32_t> &f)
 // ------------------------------------------------------------------ the encoder
 struct Encoder {
     Source src;
-    int64_t rows, cols, nb;
+    int64_t rows, cols, cb, nb;  // cb = ceil(cols / 8): a row is zero-padded to whole E8 blocks
     int container;
     int threads;
     uint32_t K;
@@ -288,13 +288,16 @@ struct Encoder {
             std::fill(v, v + 8, 0);
             return;
         }
+        // block b holds columns c0 .. c0 + 7 of row r; columns past the row's end are zeros
+        const int64_t r = b / cb, c0 = 8 * (b - r * cb), base = r * cols + c0;
+        const int n8 = int(std::min<int64_t>(8, cols - c0));
         double x[8], two_f = 2.0 * double(f);
-        for (int i = 0; i < 8; ++i) x[i] = value(8 * b + i) / two_f;
+        for (int i = 0; i < 8; ++i) x[i] = i < n8 ? value(base + i) / two_f : 0.0;
         quantize_e8(x, v);
     }
 
     void prepare() {
-        int64_t cb = cols / 8;
+        cb = (cols + 7) / 8;
         nb = rows * cb;
         if (is_code_container(container)) {
             codes.resize(size_t(rows * cols));
@@ -339,7 +342,6 @@ struct Encoder {
 
     // ---- sampled storage estimate (bits per weight at resolution index k)
     double estimate(int k) const {
-        int64_t cb = cols / 8;
         int64_t step = std::max<int64_t>(1, (nb + kSampleBlocks - 1) / kSampleBlocks);
         int64_t ns = (nb + step - 1) / step;
         std::vector<uint8_t> ctx(static_cast<size_t>(ns) * 8);
@@ -463,7 +465,6 @@ struct Encoder {
 
     // ---- full stream at resolution index k
     std::vector<uint8_t> encode(int k) const {
-        int64_t cb = cols / 8;
         std::vector<uint8_t> ctx(static_cast<size_t>(nb) * 8);
         std::vector<uint32_t> val(static_cast<size_t>(nb) * 8);
         std::vector<float> fac(static_cast<size_t>(rows));
@@ -590,7 +591,7 @@ extern "C" size_t ep_compress_bound(int64_t rows, int64_t cols, const ep_config 
     if (rows <= 0 || cols <= 0 || !cfg) return 0;
     double n = double(rows) * double(cols);
     if (cfg->q_index < 0) return size_t(std::floor(cfg->target_bpp * n / 8.0));
-    int64_t nb = rows * (cols / 8);
+    int64_t nb = rows * ((cols + 7) / 8);
     uint32_t K = cfg->blocks_per_lane ? cfg->blocks_per_lane : ep::auto_blocks_per_lane(nb, cfg->target_bpp);
     uint64_t T = uint64_t((nb + 32 * int64_t(K) - 1) / (32 * int64_t(K)));
     return ep::layout_for(rows, ep::is_code_container(cfg->container_dtype) ? cfg->container_dtype : 0,
@@ -608,9 +609,8 @@ extern "C" int ep_compress_host(const void *src, int32_t src_dtype, int64_t rows
     if (src_dtype != EP_BF16 && src_dtype != EP_FP16 && src_dtype != EP_FP32) return EP_ERR_UNSUPPORTED;
     int container = cfg->container_dtype ? cfg->container_dtype : src_dtype;
     if (container < EP_BF16 || container > EP_FP8_E4M3) return EP_ERR_INVALID_ARG;
-    if (cols % 8) return EP_ERR_UNSUPPORTED;
     if (cfg->blocks_per_lane > 4096) return EP_ERR_INVALID_ARG;
-    if ((rows * (cols / 8)) >> 32) return EP_ERR_UNSUPPORTED;
+    if ((rows * ((cols + 7) / 8)) >> 32) return EP_ERR_UNSUPPORTED;
 
     Encoder E;
     E.src = Source{src, src_dtype};

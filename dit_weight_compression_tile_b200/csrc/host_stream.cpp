@@ -37,10 +37,10 @@ extern "C" int ep_stream_info(const void *blob, size_t nbytes, ep_info *info) {
     if (I.src_dtype < EP_BF16 || I.src_dtype > EP_FP32 || I.container_dtype < EP_BF16 ||
         I.container_dtype > EP_FP8_E4M3)
         return EP_ERR_CORRUPT;
-    if (I.rows <= 0 || I.cols <= 0 || I.cols % 8 || I.rows >= (int64_t(1) << 40) || I.cols >= (int64_t(1) << 40) ||
+    if (I.rows <= 0 || I.cols <= 0 || I.rows >= (int64_t(1) << 40) || I.cols >= (int64_t(1) << 40) ||
         I.blocks_per_lane == 0 || I.blocks_per_lane > 4096 || I.q_index >= kNumQ)
         return EP_ERR_CORRUPT;
-    int64_t nb = I.rows * (I.cols / 8);
+    int64_t nb = I.rows * ((I.cols + 7) / 8);  // rows zero-padded to whole E8 blocks
     int64_t per_tile = int64_t(kLanes) * I.blocks_per_lane;
     if ((nb + per_tile - 1) / per_tile != int64_t(I.n_tiles)) return EP_ERR_CORRUPT;
     uint64_t tokens = 0;

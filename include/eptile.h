@@ -51,7 +51,7 @@ enum ep_status {
     EP_ERR_BUFFER_TOO_SMALL = -5,   /* out_cap too small; *out_nbytes holds the size needed */
     EP_ERR_CORRUPT = -6,            /* the stream fails validation */
     EP_ERR_CUDA = -7,               /* a CUDA runtime call failed (launch, attribute) */
-    EP_ERR_UNSUPPORTED = -8         /* valid but outside the format: cols % 8 != 0, > 2^31 blocks,
+    EP_ERR_UNSUPPORTED = -8         /* valid but outside the format: >= 2^31 blocks (rows x ceil(cols / 8)),
                                        a lane region beyond 65535 words with a forced tile size */
 };
 

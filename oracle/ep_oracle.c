@@ -598,6 +598,24 @@ static void row_rms(const double *w, int64_t rows, int64_t cols, float *s)
     }
 }
 
+/* Rows whose length is not a multiple of 8 are zero-padded to the next multiple before
+ * they are cut into E8 blocks (reading: the pages ask only for a non-empty 2-D tensor, so
+ * the last block of a row holds the row's last cols % 8 values and zeros).  The padding
+ * takes no part in the row statistics; its lattice coordinates are coded like any other
+ * and dropped by the decoder.  Returns w itself when no padding is needed. */
+static double *pad_rows(double *w, int64_t rows, int64_t cols)
+{
+    int64_t cp = (cols + 7) / 8 * 8;
+    if (cp == cols)
+        return w;
+    double *wp = (double *)calloc((size_t)(rows * cp), sizeof(double));
+    if (!wp)
+        return NULL;
+    for (int64_t r = 0; r < rows; r++)
+        memcpy(wp + r * cp, w + r * cols, (size_t)cols * sizeof(double));
+    return wp;
+}
+
 static float row_factor(float s, int32_t k)
 {
     if (s == 0.0f)
@@ -637,9 +655,17 @@ int or_quantize(const void *src, int32_t sdt, int64_t rows, int64_t cols, int32_
     double *w = lattice_input(src, sdt, rows, cols, container, NULL);
     float *s = (float *)malloc((size_t)rows * sizeof(float));
     row_rms(w, rows, cols, s);
-    int64_t cb = cols / 8;
-    for (int64_t b = 0; b < rows * cb; b++)
-        quantize_block(w + 8 * b, row_factor(s[b / cb], k), v + 8 * b);
+    double *wp = pad_rows(w, rows, cols);
+    int64_t cb = (cols + 7) / 8;
+    for (int64_t b = 0; b < rows * cb; b++) {
+        int32_t vb[8];
+        int64_t r = b / cb, c0 = 8 * (b % cb);
+        quantize_block(wp + 8 * b, row_factor(s[r], k), vb);
+        for (int i = 0; i < 8 && c0 + i < cols; i++)
+            v[r * cols + c0 + i] = vb[i];
+    }
+    if (wp != w)
+        free(wp);
     free(s);
     free(w);
     return OR_OK;
@@ -667,7 +693,8 @@ static size_t meta_bytes(int64_t rows, int32_t container, uint64_t total_tokens,
 static double estimate_bpp(const double *w, const float *s, int64_t rows, int64_t cols, int32_t container,
                            int32_t k, uint32_t K)
 {
-    int64_t cb = cols / 8, nb = rows * cb;
+    /* w: padded rows of 8 * ceil(cols / 8) values; the rate counts the cols true columns */
+    int64_t cb = (cols + 7) / 8, nb = rows * cb;
     int64_t S = (nb + SAMPLE_TARGET - 1) / SAMPLE_TARGET;
     if (S < 1)
         S = 1;
@@ -732,9 +759,12 @@ double or_estimate_bpp(const void *src, int32_t sdt, int64_t rows, int64_t cols,
     double *w = lattice_input(src, sdt, rows, cols, container, NULL);
     float *s = (float *)malloc((size_t)rows * sizeof(float));
     row_rms(w, rows, cols, s);
+    double *wp = pad_rows(w, rows, cols);
     if (K == 0)
-        K = or_choose_blocks_per_lane(rows * (cols / 8), 4.0);
-    double e = estimate_bpp(w, s, rows, cols, container, k, K);
+        K = or_choose_blocks_per_lane(rows * ((cols + 7) / 8), 4.0);
+    double e = estimate_bpp(wp, s, rows, cols, container, k, K);
+    if (wp != w)
+        free(wp);
     free(s);
     free(w);
     return e;
@@ -879,7 +909,8 @@ static int encode_at(const double *w, const float *s, const float *scales, int64
                      int32_t sdt, int32_t container, int32_t k, uint32_t K, uint8_t *out, size_t cap,
                      size_t *out_n)
 {
-    int64_t cb = cols / 8, nb = rows * cb;
+    /* w: padded rows of 8 * ceil(cols / 8) values; the header keeps the true cols */
+    int64_t cb = (cols + 7) / 8, nb = rows * cb;
     uint32_t *ctx = (uint32_t *)malloc((size_t)nb * 8 * sizeof(uint32_t));
     uint32_t *u = (uint32_t *)malloc((size_t)nb * 8 * sizeof(uint32_t));
     float *f = (float *)malloc((size_t)rows * sizeof(float));
@@ -1006,8 +1037,6 @@ int or_compress(const void *src, int32_t sdt, int64_t rows, int64_t cols, double
         container = sdt;
     if (container < ORD_BF16 || container > ORD_FP8E4M3)
         return OR_ERR_INVALID_ARG;
-    if (cols % 8 != 0)
-        return OR_ERR_UNSUPPORTED;
     if (K > 4096)
         return OR_ERR_INVALID_ARG;
     for (int64_t i = 0; i < rows * cols; i++)
@@ -1019,7 +1048,8 @@ int or_compress(const void *src, int32_t sdt, int64_t rows, int64_t cols, double
     double *w = lattice_input(src, sdt, rows, cols, container, scales);
     float *s = (float *)malloc((size_t)rows * sizeof(float));
     row_rms(w, rows, cols, s);
-    int64_t nb = rows * (cols / 8);
+    double *wp = pad_rows(w, rows, cols);
+    int64_t nb = rows * ((cols + 7) / 8);
     if (K == 0)
         K = or_choose_blocks_per_lane(nb, target);
     int32_t kmax = or_k_max(cols);
@@ -1031,7 +1061,7 @@ int or_compress(const void *src, int32_t sdt, int64_t rows, int64_t cols, double
         int32_t lo = 0, hi = kmax;
         while (lo < hi) {
             int32_t mid = lo + (hi - lo + 1) / 2;
-            if (estimate_bpp(w, s, rows, cols, container, mid, K) <= budget)
+            if (estimate_bpp(wp, s, rows, cols, container, mid, K) <= budget)
                 lo = mid;
             else
                 hi = mid - 1;
@@ -1041,11 +1071,11 @@ int or_compress(const void *src, int32_t sdt, int64_t rows, int64_t cols, double
     int rc;
     for (;;) {
         size_t n = 0;
-        rc = encode_at(w, s, scales, rows, cols, sdt, container, k, K, NULL, 0, &n);
+        rc = encode_at(wp, s, scales, rows, cols, sdt, container, k, K, NULL, 0, &n);
         if (rc == OR_ERR_UNSUPPORTED)
             break;
         if (q_override >= 0 || 8.0 * (double)n <= target * (double)(rows * cols)) {
-            rc = encode_at(w, s, scales, rows, cols, sdt, container, k, K, out, cap, out_n);
+            rc = encode_at(wp, s, scales, rows, cols, sdt, container, k, K, out, cap, out_n);
             break;
         }
         if (k == 0) {
@@ -1055,6 +1085,8 @@ int or_compress(const void *src, int32_t sdt, int64_t rows, int64_t cols, double
         }
         k--;
     }
+    if (wp != w)
+        free(wp);
     free(s);
     free(w);
     free(scales);
@@ -1079,10 +1111,10 @@ int or_parse(const uint8_t *p, size_t n, or_info *info)
     if (info->src_dtype < ORD_BF16 || info->src_dtype > ORD_FP32 || info->container_dtype < ORD_BF16 ||
         info->container_dtype > ORD_FP8E4M3)
         return OR_ERR_CORRUPT;
-    if (info->rows <= 0 || info->cols <= 0 || info->cols % 8 != 0 || info->rows > ((int64_t)1 << 40) ||
+    if (info->rows <= 0 || info->cols <= 0 || info->rows > ((int64_t)1 << 40) ||
         info->cols > ((int64_t)1 << 40) || info->blocks_per_lane == 0 || info->blocks_per_lane > 4096)
         return OR_ERR_CORRUPT;
-    int64_t nb = info->rows * (info->cols / 8);
+    int64_t nb = info->rows * ((info->cols + 7) / 8); /* rows padded to a multiple of 8 */
     int64_t T = (nb + (int64_t)LANES * info->blocks_per_lane - 1) / ((int64_t)LANES * info->blocks_per_lane);
     if (T != (int64_t)info->n_tiles)
         return OR_ERR_CORRUPT;
@@ -1241,7 +1273,7 @@ static uint32_t raw_read(raw_reader *R, uint32_t nbits, uint32_t *status)
 static void decode_tile(dec_ctx *D, int64_t t, int32_t *vout, void *out, uint32_t *status, code_stats *cs)
 {
     const or_info *I = &D->in;
-    int64_t cb = I->cols / 8, nb = I->rows * cb;
+    int64_t cb = (I->cols + 7) / 8, nb = I->rows * cb;
     uint32_t K = I->blocks_per_lane;
     const uint8_t *dir = D->p + I->off_dir;
     const uint8_t *tp = D->p + I->off_tiles + 16 * (uint64_t)get32(dir + 4 * t);
@@ -1298,18 +1330,20 @@ static void decode_tile(dec_ctx *D, int64_t t, int32_t *vout, void *out, uint32_
             for (int i = 0; i < 8; i++)
                 if (ctx2[i] != ctx[i])
                     *status |= OR_DEC_BAD_TOKEN;
-            /* reconstruction: w = f_r * v in fp32, then the container conversion */
-            int64_t r = b / cb;
+            /* reconstruction: w = f_r * v in fp32, then the container conversion; a padded
+             * row's last block keeps only its first cols % 8 values */
+            int64_t r = b / cb, c0 = 8 * (b % cb);
+            int n8 = I->cols - c0 < 8 ? (int)(I->cols - c0) : 8;
             uint32_t fb = get32(D->rowf + 4 * r);
             float fr;
             memcpy(&fr, &fb, 4);
             if (vout)
-                memcpy(vout + 8 * b, v, 8 * sizeof(int32_t));
+                memcpy(vout + r * I->cols + c0, v, (size_t)n8 * sizeof(int32_t));
             if (out) {
                 float wv[8];
                 for (int i = 0; i < 8; i++)
                     wv[i] = fr * (float)v[i];
-                or_convert_batch(wv, 8, D->out_dtype, (uint8_t *)out + (size_t)(8 * b) * (size_t)esz);
+                or_convert_batch(wv, n8, D->out_dtype, (uint8_t *)out + (size_t)(r * I->cols + c0) * (size_t)esz);
             }
         }
         if (x != STATE_L)

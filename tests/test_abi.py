@@ -57,9 +57,11 @@ def test_errors():
     with pytest.raises(B.EpError) as e:
         B.compress(w, 0.01)
     assert e.value.status == -4
+    # 8 x 12 at 4 bpp: the padded rows' metadata alone is over the target
     with pytest.raises(B.EpError) as e:
         B.compress(synth.gaussian(8, 12, 0.02, 1), 4.0)
-    assert e.value.status == -8
+    assert e.value.status == -4
+    assert B.stream_info(B.compress(synth.gaussian(64, 12, 0.02, 1), 11.0)).cols == 12
     with pytest.raises(B.EpError):
         B.compress(torch.zeros(0, 8), 4.0)
     with pytest.raises(B.EpError):
@@ -129,5 +131,5 @@ def test_decode_calls_reject_bad_arguments_before_any_launch():
     assert L.ep_decompress(C.byref(bad), fake, fake, fake, info.container_dtype, None, None) == -6
     assert L.ep_prepare(C.byref(bad), fake, fake, None, None) == -6
     bad = B.StreamInfo.from_buffer_copy(info)
-    bad.cols = 60  # not a multiple of 8
+    bad.cols = 0
     assert L.ep_decompress(C.byref(bad), fake, fake, fake, info.container_dtype, None, None) == -1

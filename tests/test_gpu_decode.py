@@ -53,7 +53,9 @@ def test_readme_example(oracle):
 
 @pytest.mark.parametrize("container", [B.BF16, B.FP16, B.FP32, B.INT8, B.FP8E4M3])
 @pytest.mark.parametrize("shape,K", [((1, 8), 0), ((3, 24), 1), ((5, 40), 3), ((17, 64), 7), ((33, 512), 0),
-                                     ((100, 808), 0), ((64, 1024), 16), ((300, 2048), 2)])
+                                     ((100, 808), 0), ((64, 1024), 16), ((300, 2048), 2),
+                                     # rows zero-padded to whole E8 blocks (cols % 8 != 0)
+                                     ((1, 1), 0), ((7, 13), 1), ((33, 255), 0), ((64, 1001), 2), ((5, 3), 0)])
 def test_ragged_shapes_all_containers(oracle, container, shape, K):
     src_dtype = torch.float16 if container == B.FP16 else (torch.float32 if container == B.FP32 else torch.bfloat16)
     w = synth.row_lognormal(*shape, seed=shape[0] + shape[1], dtype=src_dtype)

@@ -25,6 +25,10 @@ CASES = [
     ("K5", lambda: synth.gaussian(40, 256, 0.02, 5), 8.0, 0, 5),
     ("zero_rows", lambda: torch.cat([synth.gaussian(30, 512, 0.02, 6), torch.zeros(2, 512, dtype=torch.bfloat16)]),
      4.0, 0, 0),
+    # rows zero-padded to whole E8 blocks (cols % 8 != 0)
+    ("ragged_1001", lambda: synth.row_lognormal(96, 1001, 3), 4.0, 0, 0),
+    ("ragged_int8", lambda: synth.gaussian(64, 523, 0.02, 4), 3.0, B.INT8, 0),
+    ("ragged_K3", lambda: synth.row_lognormal(33, 13, 5, dtype=torch.float32), 9.0, 0, 3),
 ]
 
 
