@@ -178,24 +178,41 @@ def job_rate(per_rank_bytes, world, seconds):
 
 
 # ------------------------------------------------------------------ CPU oracle leg
-def cpu_oracle_decode(blob_np, seconds):
-    """the oracle decoder, as it stands, on one host core: consecutive tiles of one stream for a
-    bounded time; returns (weights decoded, seconds, tiles)"""
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_oracle_decode(blob_np, seconds, threads=1):
+    """the oracle decoder, as it stands, on `threads` host cores: each thread decodes runs of 16
+    consecutive tiles of one stream (threads start at different tiles; the oracle keeps no global
+    state and ctypes releases the GIL) until the time is up; returns (weights decoded, seconds,
+    tiles)"""
+    from concurrent.futures import ThreadPoolExecutor
     from oracle import oracle as O
     rc, info = O.parse(blob_np)
     per_tile = 32 * info.blocks_per_lane * 8
     n_w = info.rows * info.cols
-    done, t, tiles = 0, 0.0, 0
     t0 = time.perf_counter()
-    while t < seconds:
-        lo = tiles % info.n_tiles
-        hi = min(info.n_tiles, lo + 16)
-        rc, st, _, _ = O.decode(blob_np, lo, hi, want_v=False)
-        assert rc == 0 and st == 0
-        done += min(hi * per_tile, n_w) - lo * per_tile
-        tiles += hi - lo
-        t = time.perf_counter() - t0
-    return done, t, tiles
+
+    def worker(i):
+        done, tiles, lo = 0, 0, (i * info.n_tiles) // threads
+        while time.perf_counter() - t0 < seconds:
+            lo = lo % info.n_tiles
+            hi = min(info.n_tiles, lo + 16)
+            rc, st, _, _ = O.decode(blob_np, lo, hi, want_v=False)
+            assert rc == 0 and st == 0
+            done += min(hi * per_tile, n_w) - lo * per_tile
+            tiles += hi - lo
+            lo = hi
+        return done, tiles
+
+    with ThreadPoolExecutor(threads) as ex:
+        res = list(ex.map(worker, range(threads)))
+    t = time.perf_counter() - t0
+    return sum(r[0] for r in res), t, sum(r[1] for r in res)
 
 
 def traffic_for_kernel(workload):
@@ -223,20 +240,28 @@ def run_reference(a, rank, world):
     rc, info = O.parse(blob)
     T, per_tile_w = info.n_tiles, 32 * info.blocks_per_lane * 8
     esz = 2 if WORKLOADS[a.workload]["container"] in (0, "bf16") else 1
+    from concurrent.futures import ThreadPoolExecutor
+    ncores = host_cores()
     n_cal = min(16, T)
     t0 = time.perf_counter()
     O.decode(blob, 0, n_cal, want_v=False)
     sec_per_tile = (time.perf_counter() - t0) / n_cal
     budget = 60.0 / max(1, a.steps + a.warmup)
-    tiles = max(1, min(T - 1, int(budget / sec_per_tile))) if T > 1 else 1
+    tiles = max(1, min(T - 1, int(budget * ncores / sec_per_tile))) if T > 1 else 1
     start = 0
+    pool = ThreadPoolExecutor(ncores)
+
+    def one(r):
+        rc, st, _, _ = O.decode(blob, r[0], r[1], want_v=False)
+        assert rc == 0 and st == 0
 
     def step():
+        # a step: `tiles` consecutive tiles split into one range per host core
         nonlocal start
         if start + tiles > max(1, T - 1):
             start = 0
-        rc, st, _, _ = O.decode(blob, start, start + tiles, want_v=False)
-        assert rc == 0 and st == 0
+        cuts = [start + (tiles * i) // ncores for i in range(ncores + 1)]
+        list(pool.map(one, [(cuts[i], cuts[i + 1]) for i in range(ncores) if cuts[i + 1] > cuts[i]]))
         start += tiles
 
     for _ in range(a.warmup):
@@ -245,6 +270,7 @@ def run_reference(a, rank, world):
     for _ in range(a.steps):
         step()
     t = time.perf_counter() - t0
+    pool.shutdown()
     out_bytes = tiles * per_tile_w * esz * a.steps
     gbs = out_bytes / t / 1e9
     line = {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
@@ -252,9 +278,9 @@ def run_reference(a, rank, world):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32+f32",
             "data": "synthetic", "config": dict(workload_config(a), l2="n/a (host)"),
             "gweights_per_s": round(tiles * per_tile_w * a.steps / t / 1e9, 4),
-            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": ncores, "kind": "oracle",
                              "sample": f"{tiles} of {T} tiles ({tiles * per_tile_w} weights) of the first "
-                                       "stream per step, decoded by the C oracle"},
+                                       f"stream per step, decoded by the C oracle on {ncores} threads"},
             "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -400,12 +426,16 @@ def run_ours(a, rank, world, local_rank):
         "encode_s": round(t_enc, 3),
     }
     if world == 1 and not a.no_cpu_baseline:
-        done, el, tiles = cpu_oracle_decode(layers[0][1].numpy(), a.cpu_seconds)
         esz = i0.out_nbytes // (i0.rows * i0.cols)
-        line["cpu_baseline"] = {"value": round(done * esz / el / 1e9, 4), "unit": "GB/s", "cores": 1,
+        ncores = host_cores()
+        d1, e1, t1 = cpu_oracle_decode(layers[0][1].numpy(), a.cpu_seconds / 2, 1)
+        done, el, tiles = cpu_oracle_decode(layers[0][1].numpy(), a.cpu_seconds / 2, ncores)
+        line["cpu_baseline"] = {"value": round(done * esz / el / 1e9, 4), "unit": "GB/s", "cores": ncores,
                                 "kind": "oracle",
                                 "sample": f"{tiles} tiles ({done} weights) of the first stream, decoded by the "
-                                          f"C oracle in {el:.1f} s"}
+                                          f"C oracle on {ncores} threads in {el:.1f} s",
+                                "single_core": {"value": round(d1 * esz / e1 / 1e9, 4), "unit": "GB/s",
+                                                "sample": f"{t1} tiles in {e1:.1f} s on one thread"}}
     print(json.dumps(line), flush=True)
 
 
