@@ -13,7 +13,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libeptile.so")
 SOURCES = ["decode.cu", "host_encode.cpp", "host_stream.cpp"]
-HEADERS = [os.path.join(CSRC, "format.h"), os.path.join(ROOT, "include", "eptile.h")]
+HEADERS = [os.path.join(CSRC, h) for h in ("format.h", "encode_math.h", "encode_host.h")] + \
+    [os.path.join(ROOT, "include", "eptile.h")]
 
 
 def nvcc():

@@ -16,6 +16,8 @@
 #include <vector>
 
 #include "../../include/eptile.h"
+#include "encode_host.h"
+#include "encode_math.h"
 #include "format.h"
 
 namespace ep {
@@ -79,136 +81,14 @@ struct Source {
     }
 };
 
-// ------------------------------------------------------------------ FP8 E4M3 codes
-// The 127 non-negative finite E4M3 values in increasing order (code = index).
-const std::vector<double> &e4m3_values() {
-    static std::vector<double> vals = [] {
-        std::vector<double> v;
-        for (int code = 0; code <= 0x7e; ++code) {
-            int e = code >> 3, m = code & 7;
-            v.push_back(e == 0 ? m / 512.0 : std::ldexp(1.0 + m / 8.0, e - 7));
-        }
-        return v;
-    }();
-    return vals;
-}
+}  // namespace
 
-// round |t| to the E4M3 grid, nearest with ties to the even code, saturating at 448
-double e4m3_round(float t) {
-    const auto &vals = e4m3_values();
-    double a = std::fabs(double(t));
-    double r;
-    if (a >= vals.back()) {
-        r = vals.back();
-    } else {
-        size_t hi = size_t(std::upper_bound(vals.begin(), vals.end(), a) - vals.begin());  // vals[hi] > a
-        size_t lo = hi - 1;                                                                  // vals[lo] <= a
-        double dlo = a - vals[lo], dhi = vals[hi] - a;
-        if (dlo < dhi)
-            r = vals[lo];
-        else if (dhi < dlo)
-            r = vals[hi];
-        else
-            r = (lo % 2 == 0) ? vals[lo] : vals[hi];
-    }
-    return std::signbit(t) ? -r : r;
-}
-
-// ------------------------------------------------------------------ quantizer
-double q_value(int k) { return std::ldexp(double(64 + (k % 64)), k / 64 - 14); }
-
+// ------------------------------------------------------------------ decisions from histograms
 int max_q_index(int64_t cols) {
     double lim = std::ldexp(1.0, 20) / (std::sqrt(double(cols)) + 1.0);
     int k = kNumQ - 1;
     while (k > 0 && q_value(k) > lim) --k;
     return k;
-}
-
-float factor_of(float rms, int k) {
-    if (rms == 0.0f) return 0.0f;
-    float f = float(double(rms) / (2.0 * q_value(k)));
-    return std::isinf(f) ? FLT_MAX : f;
-}
-
-// nearest point of D8 (Conway & Sloane): round, then repair an odd coordinate sum at the
-// coordinate with the largest rounding error
-inline void nearest_d8(const double *y, double *r) {
-    long long s = 0;
-    for (int i = 0; i < 8; ++i) {
-        r[i] = std::nearbyint(y[i]);
-        s += static_cast<long long>(r[i]);
-    }
-    if (s & 1) {
-        int worst = 0;
-        double werr = std::fabs(y[0] - r[0]);
-        for (int i = 1; i < 8; ++i) {
-            double e = std::fabs(y[i] - r[i]);
-            if (e > werr) {
-                werr = e;
-                worst = i;
-            }
-        }
-        r[worst] += (y[worst] < r[worst]) ? -1.0 : 1.0;
-    }
-}
-
-// v = 2 * nearest point of E8 = D8 u (D8 + 1/2); ties keep the integer coset
-inline void quantize_e8(const double *x, int32_t *v) {
-    double a[8], b[8], ra[8], rb[8];
-    for (int i = 0; i < 8; ++i) {
-        a[i] = x[i];
-        b[i] = x[i] - 0.5;
-    }
-    nearest_d8(a, ra);
-    nearest_d8(b, rb);
-    double da = 0.0, db = 0.0;
-    for (int i = 0; i < 8; ++i) da += (a[i] - ra[i]) * (a[i] - ra[i]);
-    for (int i = 0; i < 8; ++i) db += (b[i] - rb[i]) * (b[i] - rb[i]);
-    if (db < da) {
-        for (int i = 0; i < 8; ++i) v[i] = int32_t(rb[i]) * 2 + 1;
-    } else {
-        for (int i = 0; i < 8; ++i) v[i] = int32_t(ra[i]) * 2;
-    }
-}
-
-// ------------------------------------------------------------------ symbols
-inline uint32_t zz(int32_t y) { return y < 0 ? uint32_t(-int64_t(y)) * 2u - 1u : uint32_t(y) * 2u; }
-
-inline int bitlen(uint32_t u) { return u ? 32 - __builtin_clz(u) : 0; }
-
-// Contexts and coded values of one block, in coding order.  c = v0 mod 2, y_i = (v_i - c) / 2,
-// p = parity of y0 + ... + y6.  Coordinate 0: context 0, value 4 zz(a0) + r0 with v0 = 4 a0 + r0;
-// coordinates 1..6: context 1 + c, value 2 zz(a) + b with y = 2 a + b; coordinate 7: context
-// 3 + 2c + p, value zz((y7 - p) / 2).  Arithmetic shifts are floor divisions here.
-inline void symbols_of(const int32_t *v, uint8_t *ctx, uint32_t *s) {
-    int32_t c = v[0] & 1;
-    int32_t par = ((v[0] - c) >> 1) & 1;
-    ctx[0] = 0;
-    s[0] = 4u * zz(v[0] >> 2) + uint32_t(v[0] & 3);
-    for (int i = 1; i < 7; ++i) {
-        int32_t y = (v[i] - c) >> 1;
-        par ^= y & 1;
-        ctx[i] = uint8_t(1 + c);
-        s[i] = 2u * zz(y >> 1) + uint32_t(y & 1);
-    }
-    int32_t y7 = (v[7] - c) >> 1;
-    ctx[7] = uint8_t(3 + 2 * c + par);
-    s[7] = zz((y7 - par) >> 1);
-}
-
-struct Token {
-    uint32_t tok, nbits, extra;
-};
-
-// hybrid-integer token of s with split m, keeping the `low` low bits of s in the token and two
-// bits below the leading one; the bits in between are raw extra bits
-inline Token token_of(uint32_t s, uint32_t m, uint32_t low) {
-    if (s < (1u << m)) return {s, 0, 0};
-    uint32_t n = uint32_t(bitlen(s)) - 1;
-    uint32_t nbits = n - kTopBits - low;
-    uint32_t top = (s >> (n - kTopBits)) & ((1u << kTopBits) - 1u);
-    uint32_t tok = (1u << m) + (((((n - m) << kTopBits) | top) << low) | (s & ((1u << low) - 1u)));
-    return {tok, nbits, (s >> low) & ((1u << nbits) - 1u)};
 }
 
 // smallest m allowed for the context with >= 99.9% of the values below 2^m (bit length <= m)
@@ -269,6 +149,66 @@ uint32_t build_freqs(const std::vector<uint64_t> &cnt, std::vector<uint32_t> &f)
     }
     return len;
 }
+
+double estimate_from_counts(const std::vector<uint64_t> *cnt, uint64_t extra_bits, int64_t nb, int64_t ns,
+                            int64_t rows, int64_t cols, int container, uint32_t T) {
+    double bits = 0.0;
+    uint64_t tokens = 0;
+    for (int c = 0; c < kContexts; ++c) {
+        uint64_t n = 0;
+        uint32_t len = 0;
+        for (size_t t = 0; t < cnt[c].size(); ++t) {
+            n += cnt[c][t];
+            if (cnt[c][t]) len = uint32_t(t + 1);
+        }
+        tokens += len;
+        if (!n) continue;
+        bits += double(n) * std::log2(double(n));
+        for (size_t t = 0; t < cnt[c].size(); ++t)
+            if (cnt[c][t]) bits -= double(cnt[c][t]) * std::log2(double(cnt[c][t]));
+    }
+    bits += double(extra_bits);
+    Layout L = layout_for(rows, container, tokens, T);
+    double bytes = double(L.tiles) + kTileOverheadBytes * double(T) + bits * (double(nb) / double(ns)) / 8.0;
+    return 8.0 * bytes / double(rows * cols);
+}
+
+void write_front(uint8_t *h, const Layout &L, int src_dt, int container, int64_t rows, int64_t cols, uint32_t T,
+                 uint32_t K, int k, const uint32_t *m, const uint32_t *ntok, const std::vector<uint32_t> *freq,
+                 const float *fac, const float *scales) {
+    auto put = [](uint8_t *p, uint64_t v, int n) {
+        for (int i = 0; i < n; ++i) p[i] = uint8_t(v >> (8 * i));
+    };
+    put(h, kMagic, 4);
+    put(h + 4, kVersion, 2);
+    h[6] = uint8_t(src_dt);
+    h[7] = uint8_t(container);
+    put(h + 8, uint64_t(rows), 8);
+    put(h + 16, uint64_t(cols), 8);
+    put(h + 24, T, 4);
+    put(h + 28, K, 4);
+    put(h + 32, uint32_t(k), 2);
+    h[34] = uint8_t(kProbBits);
+    h[35] = uint8_t(kContexts);
+    for (int c = 0; c < kContexts; ++c) {
+        h[36 + c] = uint8_t(m[c]);
+        put(h + 44 + 2 * c, ntok[c], 2);
+    }
+    std::memcpy(h + L.rowf, fac, size_t(rows) * 4);
+    if (is_code_container(container)) std::memcpy(h + L.scales, scales, size_t(rows) * 4);
+    size_t q = L.freq;
+    for (int c = 0; c < kContexts; ++c)
+        for (uint32_t t = 0; t < ntok[c]; ++t, q += 2) put(h + q, freq[c][t], 2);
+}
+
+bool little_endian_host() {
+    uint32_t one = 1;
+    uint8_t b;
+    std::memcpy(&b, &one, 1);
+    return b == 1;
+}
+
+namespace {
 
 // ------------------------------------------------------------------ the encoder
 struct Encoder {
@@ -368,26 +308,7 @@ struct Encoder {
             cnt[ctx[i]][t.tok]++;
             extra += t.nbits;
         }
-        double bits = 0.0;
-        uint64_t tokens = 0;
-        for (int c = 0; c < kContexts; ++c) {
-            uint64_t n = 0;
-            uint32_t len = 0;
-            for (size_t t = 0; t < cnt[c].size(); ++t) {
-                n += cnt[c][t];
-                if (cnt[c][t]) len = uint32_t(t + 1);
-            }
-            tokens += len;
-            if (!n) continue;
-            bits += double(n) * std::log2(double(n));
-            for (size_t t = 0; t < cnt[c].size(); ++t)
-                if (cnt[c][t]) bits -= double(cnt[c][t]) * std::log2(double(cnt[c][t]));
-        }
-        bits += double(extra);
-        uint32_t T = tile_count();
-        Layout L = layout_for(rows, container, tokens, T);
-        double bytes = double(L.tiles) + kTileOverheadBytes * double(T) + bits * (double(nb) / double(ns)) / 8.0;
-        return 8.0 * bytes / double(rows * cols);
+        return estimate_from_counts(cnt, extra, nb, ns, rows, cols, container, tile_count());
     }
 
     // ---- one tile: 32 independent lanes.  A lane's region holds its rANS words in decode order
@@ -541,26 +462,7 @@ struct Encoder {
         auto put = [](uint8_t *p, uint64_t v, int n) {
             for (int i = 0; i < n; ++i) p[i] = uint8_t(v >> (8 * i));
         };
-        put(h, kMagic, 4);
-        put(h + 4, kVersion, 2);
-        h[6] = uint8_t(src.dt);
-        h[7] = uint8_t(container);
-        put(h + 8, uint64_t(rows), 8);
-        put(h + 16, uint64_t(cols), 8);
-        put(h + 24, T, 4);
-        put(h + 28, K, 4);
-        put(h + 32, uint32_t(k), 2);
-        h[34] = uint8_t(kProbBits);
-        h[35] = uint8_t(kContexts);
-        for (int c = 0; c < kContexts; ++c) {
-            h[36 + c] = uint8_t(m[c]);
-            put(h + 44 + 2 * c, ntok[c], 2);
-        }
-        std::memcpy(h + L.rowf, fac.data(), size_t(rows) * 4);
-        if (is_code_container(container)) std::memcpy(h + L.scales, scales.data(), size_t(rows) * 4);
-        size_t q = L.freq;
-        for (int c = 0; c < kContexts; ++c)
-            for (uint32_t t = 0; t < ntok[c]; ++t, q += 2) put(h + q, freq[c][t], 2);
+        write_front(h, L, src.dt, container, rows, cols, T, K, k, m, ntok, freq, fac.data(), scales.data());
         uint32_t at = 0;
         size_t d = L.dir, o = L.tiles;
         for (int c = 0; c < tchunks; ++c) {
@@ -576,13 +478,6 @@ struct Encoder {
         return out;
     }
 };
-
-bool little_endian_host() {
-    uint32_t one = 1;
-    uint8_t b;
-    std::memcpy(&b, &one, 1);
-    return b == 1;
-}
 
 }  // namespace
 }  // namespace ep
