@@ -88,16 +88,20 @@ def workload_config(a):
 
 
 def compress_layers(a):
-    """the workload's streams (host), encoded once, untimed; returns [(name, blob)] and seconds"""
+    """the workload's streams, encoded once on the GPU (ep_compress_device: the host compressor's
+    bytes), untimed for the metric; returns [(name, host copy of the blob)] and the encode seconds"""
     from dit_weight_compression_tile_b200 import binding as B
     wl = WORKLOADS[a.workload]
     out, t = [], 0.0
     for name, make in wl["layers"]():
-        w = make()
+        w = make().cuda()
+        torch.cuda.synchronize()
         t0 = time.perf_counter()
-        out.append((name, B.compress(w, a.target, container=wl["container"])))
+        blob = B.compress_device(w, a.target, container=wl["container"])
+        torch.cuda.synchronize()
         t += time.perf_counter() - t0
-        del w
+        out.append((name, blob.cpu()))
+        del w, blob
     return out, t
 
 

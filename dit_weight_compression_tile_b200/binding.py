@@ -77,6 +77,11 @@ def lib():
         p = C.c_void_p
         L.ep_compress_bound.restype = C.c_size_t
         L.ep_compress_bound.argtypes = [C.c_int64, C.c_int64, C.POINTER(Config)]
+        L.ep_compress_device_scratch.restype = C.c_size_t
+        L.ep_compress_device_scratch.argtypes = [C.c_int64, C.c_int64, C.POINTER(Config)]
+        L.ep_compress_device.restype = C.c_int
+        L.ep_compress_device.argtypes = [p, C.c_int32, C.c_int64, C.c_int64, C.POINTER(Config), p, C.c_size_t,
+                                         C.POINTER(C.c_size_t), p, C.c_size_t, p]
         L.ep_compress_host.restype = C.c_int
         L.ep_compress_host.argtypes = [p, C.c_int32, C.c_int64, C.c_int64, C.POINTER(Config), p, C.c_size_t,
                                        C.POINTER(C.c_size_t)]
@@ -125,6 +130,32 @@ def compress(tensor, target_bpp, container=0, blocks_per_lane=0, q_index=-1, n_t
                                 out.data_ptr(), out.numel(), C.byref(n))
     if rc != 0:
         raise EpError(rc, "ep_compress_host")
+    return out[: n.value].clone()
+
+
+def compress_device(tensor, target_bpp, container=0, blocks_per_lane=0, q_index=-1, stream=None):
+    """compress(tensor, config) for a CUDA tensor (ep_compress_device): the same stream as
+    ``compress`` byte for byte, built on the GPU.  Returns a CUDA uint8 tensor."""
+    if tensor.dim() != 2 or tensor.numel() == 0:
+        raise EpError(-1, "compress needs a non-empty 2-D tensor")
+    if not tensor.is_cuda:
+        raise EpError(-1, "compress_device needs a CUDA tensor")
+    src = tensor.detach().contiguous()
+    if src.dtype not in (torch.bfloat16, torch.float16, torch.float32):
+        raise EpError(-8, f"source dtype {src.dtype}")
+    cfg = _config(target_bpp, container, blocks_per_lane, q_index, 0)
+    L = lib()
+    R, Cc = src.shape
+    scratch = torch.empty(max(1, L.ep_compress_device_scratch(R, Cc, C.byref(cfg))), dtype=torch.uint8,
+                          device=src.device)
+    cap = L.ep_compress_bound(R, Cc, C.byref(cfg))
+    out = torch.empty(max(cap, 64), dtype=torch.uint8, device=src.device)
+    n = C.c_size_t(0)
+    s = (stream or torch.cuda.current_stream(src.device)).cuda_stream
+    rc = L.ep_compress_device(src.data_ptr(), CODE_OF[src.dtype], R, Cc, C.byref(cfg), out.data_ptr(), out.numel(),
+                              C.byref(n), scratch.data_ptr(), scratch.numel(), s)
+    if rc != 0:
+        raise EpError(rc, "ep_compress_device")
     return out[: n.value].clone()
 
 

@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libeptile.so")
-SOURCES = ["decode.cu", "host_encode.cpp", "host_stream.cpp"]
+SOURCES = ["decode.cu", "device_encode.cu", "host_encode.cpp", "host_stream.cpp"]
 HEADERS = [os.path.join(CSRC, h) for h in ("format.h", "encode_math.h", "encode_host.h")] + \
     [os.path.join(ROOT, "include", "eptile.h")]
 

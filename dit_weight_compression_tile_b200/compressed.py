@@ -1,7 +1,7 @@
 """compress(tensor, config) -> CompressedTensor and decompress(compressed, config) -> tensor, the calls
 of the API reference ("EntroPack API reference", Tensor encoding and decoding; CompressedTensor),
-over the C ABI: ep_compress_host builds the stream on the host, ep_prepare and the fused
-ep_decompress kernel decode it on the GPU.  This module only keeps the pieces together (stream,
+over the C ABI: ep_compress_device (a CUDA tensor) or ep_compress_host (a host tensor) builds the
+stream, the same bytes either way; ep_prepare and the fused ep_decompress kernel decode it.  This module only keeps the pieces together (stream,
 parsed plan, prepared tables, output dtype); it computes nothing itself.
 
 Differences from the pages, by design: CompressedTensor is a plain object, not a torch.Tensor
@@ -166,15 +166,19 @@ def compress(tensor, config):
         raise B.EpError(-1, "config must be a LatticeRANSConfig")
     container = 0 if config.container is None else config.container
     try:
-        blob = B.compress(tensor, config.target_bpp, container=container,
-                          blocks_per_lane=config.blocks_per_lane, n_threads=config.n_threads)
+        if tensor.is_cuda:  # the GPU compressor writes the host compressor's bytes
+            blob = B.compress_device(tensor, config.target_bpp, container=container,
+                                     blocks_per_lane=config.blocks_per_lane)
+        else:
+            blob = B.compress(tensor, config.target_bpp, container=container,
+                              blocks_per_lane=config.blocks_per_lane, n_threads=config.n_threads)
     except B.EpError as e:
         if e.status != -4:  # EP_ERR_TARGET_UNREACHABLE
             raise
         warnings.warn(f"target_bpp {config.target_bpp} is below what the stream's metadata alone needs for "
                       f"shape {tuple(tensor.shape)}; the tensor is stored uncompressed (compress_method='raw')")
         return CompressedTensor(raw=tensor.detach().clone(), out_dtype=tensor.dtype)
-    info = B.stream_info(blob)
+    info = B.stream_info(blob.cpu() if blob.is_cuda else blob)
     # by default the output has the input's dtype; code containers decode to their codes
     out_dtype = tensor.dtype if B.CODE_OF.get(tensor.dtype) in _allowed_out(info.container_dtype) else info.dtype
     return CompressedTensor(blob.to(tensor.device), info, out_dtype)

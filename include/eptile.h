@@ -112,6 +112,31 @@ size_t ep_compress_bound(int64_t rows, int64_t cols, const ep_config *cfg);
 int ep_compress_host(const void *src, int32_t src_dtype, int64_t rows, int64_t cols, const ep_config *cfg,
                      void *out, size_t out_cap, size_t *out_nbytes);
 
+/* Scratch bytes ep_compress_device needs for this shape and config (0 for invalid arguments):
+ * about 9 bytes per weight (context and value of every coordinate, the INT8 / FP8 code matrix)
+ * plus small tables; it does not depend on the container or the data. */
+size_t ep_compress_device_scratch(int64_t rows, int64_t cols, const ep_config *cfg);
+
+/* compress(tensor, config) of the API reference with the tensor in DEVICE memory: the same stream
+ * as ep_compress_host, byte for byte (same steps, same decisions), with the work over elements,
+ * blocks and lanes on the GPU (row statistics, E8 quantization, token histograms, one rANS coder
+ * per lane) and the decisions taken from integer histograms on the host (splits, frequency tables,
+ * the sampled estimate and its bisection over the resolution, tile offsets).
+ *   d_src       device pointer, row-major rows x cols elements of src_dtype (BF16/FP16/FP32).
+ *   cfg         as for ep_compress_host (n_threads unused).
+ *   d_out       device buffer of out_cap bytes (16-byte aligned) that receives the stream;
+ *               ep_compress_bound gives a sufficient capacity.
+ *   out_nbytes  receives the stream size (also on EP_ERR_BUFFER_TOO_SMALL / UNREACHABLE).
+ *   d_scratch   device buffer of at least ep_compress_device_scratch bytes, 256-byte aligned,
+ *               caller-owned; its contents are not needed afterwards.
+ *   stream      CUDA stream of every launch and copy.
+ * Errors as ep_compress_host.  Synchronous: the call waits on `stream` at each decision (a few
+ * dozen times during the resolution search) and returns when the stream is written.  The
+ * library allocates nothing. */
+int ep_compress_device(const void *d_src, int32_t src_dtype, int64_t rows, int64_t cols, const ep_config *cfg,
+                       void *d_out, size_t out_cap, size_t *out_nbytes, void *d_scratch, size_t scratch_nbytes,
+                       ep_stream_t stream);
+
 /* CompressedTensor's properties (API reference) from a HOST copy of the stream.
  *   blob   host pointer to the first nbytes of the stream; nbytes must be the whole stream
  *          (the tile directory is checked against the stream end).

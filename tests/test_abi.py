@@ -12,8 +12,9 @@ from dit_weight_compression_tile_b200 import synth
 
 def test_exports_every_declared_symbol():
     names = B.declared_functions()
-    assert set(names) == {"ep_compress_bound", "ep_compress_host", "ep_stream_info", "ep_prepare",
-                          "ep_decompress", "ep_decompress_noalloc", "ep_status_string"}
+    assert set(names) == {"ep_compress_bound", "ep_compress_host", "ep_compress_device_scratch",
+                          "ep_compress_device", "ep_stream_info", "ep_prepare", "ep_decompress",
+                          "ep_decompress_noalloc", "ep_status_string"}
     lib = B.lib()
     for n in names:
         assert hasattr(lib, n), n
@@ -21,6 +22,23 @@ def test_exports_every_declared_symbol():
     raw = C.CDLL(B.LIB_PATH)
     for n in names:
         assert C.cast(getattr(raw, n), C.c_void_p).value
+
+
+def test_device_compress_rejects_bad_arguments_before_any_launch():
+    cfg = B._config(4.0)
+    L = B.lib()
+    fake = 1 << 20
+    n = C.c_size_t(0)
+    need = L.ep_compress_device_scratch(64, 256, C.byref(cfg))
+    assert need >= 64 * 256 * 9  # symbols (5 bytes per weight) and the code matrix (4)
+    assert L.ep_compress_device_scratch(0, 256, C.byref(cfg)) == 0
+    assert L.ep_compress_device(None, B.BF16, 64, 256, C.byref(cfg), fake, 1 << 20, C.byref(n), fake, need, None) == -1
+    assert L.ep_compress_device(fake, B.BF16, 64, 256, C.byref(cfg), fake, 1 << 20, C.byref(n), None, need, None) == -1
+    assert L.ep_compress_device(fake, B.INT8, 64, 256, C.byref(cfg), fake, 1 << 20, C.byref(n), fake, need, None) == -8
+    assert L.ep_compress_device(fake, B.BF16, 64, 256, C.byref(cfg), fake, 1 << 20, C.byref(n), fake + 16, need,
+                                None) == -1  # scratch not 256-byte aligned
+    assert L.ep_compress_device(fake, B.BF16, 64, 256, C.byref(cfg), fake, 1 << 20, C.byref(n), fake, need - 1,
+                                None) == -1  # scratch too small
 
 
 def test_status_strings():
