@@ -10,6 +10,7 @@ _BINDING_NAMES = ("BF16", "FP16", "FP32", "INT8", "FP8E4M3", "EpError", "compres
 
 
 _COMPRESSED_NAMES = ("CompressedTensor", "LatticeRANSConfig")
+_LINEAR_NAMES = ("CompressedLinear", "CompressedFP8Linear", "CompressedINT8Linear")
 
 
 def __getattr__(name):
@@ -19,4 +20,7 @@ def __getattr__(name):
     if name in _COMPRESSED_NAMES:
         from . import compressed
         return getattr(compressed, name)
+    if name in _LINEAR_NAMES:
+        from . import linear
+        return getattr(linear, name)
     raise AttributeError(name)
