@@ -5,8 +5,8 @@ the stream parser and the sm_100a decode kernel; ``binding`` marshals torch tens
 it.  Importing the package loads nothing; the first use of a binding name imports
 ``binding``, whose ``lib()`` fails loudly when the built library is missing.
 """
-_BINDING_NAMES = ("BF16", "FP16", "FP32", "INT8", "FP8E4M3", "EpError", "compress", "prepare", "decompress",
-                  "stream_info", "lib", "StreamInfo")
+_BINDING_NAMES = ("BF16", "FP16", "FP32", "INT8", "FP8E4M3", "EpError", "compress", "compress_device", "prepare",
+                  "decompress", "stream_info", "lib", "StreamInfo")
 
 
 _COMPRESSED_NAMES = ("CompressedTensor", "LatticeRANSConfig")
