@@ -375,29 +375,50 @@ def run_ours(a, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     prepare_us = p0.elapsed_time(p1) * 1e3 / (prep_reps * len(infos))
 
-    # end to end through the public API with host buffers: pinned H2D of every stream, the
-    # tables, the decode, D2H of every container into pinned memory, every step
+    # end to end through the public API with host buffers: every step, pinned H2D of every
+    # stream, the tables, the decode and D2H of every container into pinned memory.  Consecutive
+    # (step, tensor) units alternate between two CUDA streams with their own device buffers, so
+    # that one unit's device-to-host read overlaps the next unit's host-to-device copy
     host_blobs = [blob.pin_memory() for _, blob in layers]
     biggest = max(range(len(infos)), key=lambda i: infos[i].out_nbytes)
-    host_out = torch.empty(infos[biggest].shape, dtype=infos[biggest].dtype).pin_memory()
+    host_outs = [torch.empty(infos[biggest].shape, dtype=infos[biggest].dtype).pin_memory() for _ in range(2)]
+    streams = [stream, torch.cuda.Stream(dev)]
+    n = len(infos)
+    sets = []  # per stream: (device blob, workspace, device output) of every tensor
+    for j in range(2):
+        if rot >= 2:
+            sets.append([(blobs[j * n + i], works[j * n + i], outs[j * n + i]) for i in range(n)])
+        elif j == 0:
+            sets.append([(blobs[i], works[i], outs[i]) for i in range(n)])
+        else:
+            sets.append([(torch.empty_like(blobs[i]), torch.empty_like(works[i]), torch.empty_like(outs[i]))
+                         for i in range(n)])
+    unit = [0]
 
     def e2e_step():
         for i, info in enumerate(infos):
-            blobs[i].copy_(host_blobs[i], non_blocking=True)
-            B.prepare(blobs[i], info, workspace=works[i], stream=stream)
-            B.decompress(blobs[i], info, workspace=works[i], out=outs[i], stream=stream)
-            host_out.view(-1)[: outs[i].numel()].copy_(outs[i].view(-1), non_blocking=True)
+            j = unit[0] % 2
+            unit[0] += 1
+            d, w_, o = sets[j][i]
+            s_ = streams[j]
+            with torch.cuda.stream(s_):
+                d.copy_(host_blobs[i], non_blocking=True)
+                B.prepare(d, info, workspace=w_, stream=s_)
+                B.decompress(d, info, workspace=w_, out=o, stream=s_)
+                host_outs[j].view(-1)[: o.numel()].copy_(o.view(-1), non_blocking=True)
 
     e2e_steps = max(2, min(200, int(0.5 / max(1e-9, (in_bytes + out_bytes) / 40e9))))
-    with torch.cuda.stream(stream):
-        e2e_step()
+    e2e_step()
     torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record(stream)
+    e0, e1, ej = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+                  torch.cuda.Event())
+    e0.record(streams[0])
+    streams[1].wait_event(e0)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ej.record(streams[1])
+    streams[0].wait_event(ej)
+    e1.record(streams[0])
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = job_rate(out_bytes * e2e_steps, world, e2e_ms / 1e3) / 1e9
