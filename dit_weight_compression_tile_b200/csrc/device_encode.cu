@@ -5,8 +5,9 @@
 // lattice quantization, a conditional model of the coordinates, a resolution picked by sampled
 // storage estimates, tiles of interleaved rANS), with the work over elements, blocks and lanes on
 // the GPU:
-//   * rows_kernel      one thread per row: finite check, INT8 / FP8 codes and scales, the row RMS
-//                      summed left to right in double (the order is part of the result);
+//   * rows_kernel      one lane per row over 32x32 shared-memory tiles: finite check, INT8 / FP8
+//                      codes and scales, the row RMS summed left to right in double (the order is
+//                      part of the result);
 //   * quant_kernel     per block: x = w / (2 f_r), E8 nearest point, symbols and contexts, and a
 //                      histogram of the values' bit lengths per context;
 //   * token_kernel     per coordinate: its token at the chosen splits, token counts per context
@@ -57,43 +58,75 @@ struct Splits {
 };
 
 // ------------------------------------------------------------------ rows
-__global__ void rows_kernel(DevSrc src, int64_t rows, int64_t cols, int container, float *codes, float *scales,
-                            float *rms, uint32_t *bad) {
-    const int64_t r = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (r >= rows) return;
-    const int64_t base = r * cols;
+// A warp owns 32 rows, lane l row row0 + l.  Columns go through shared memory 32 at a time: the
+// warp loads a 32x32 tile row by row (coalesced), then every lane walks its own row's 32 values in
+// column order, so the RMS is still summed left to right in double.  Tile rows are padded to 33
+// words (conflict-free column walks).
+constexpr int kRowWarps = 8;
+
+__global__ void __launch_bounds__(kRowWarps * 32) rows_kernel(DevSrc src, int64_t rows, int64_t cols,
+                                                                int container, float *codes, float *scales,
+                                                                float *rms, uint32_t *bad) {
+    __shared__ float tile[kRowWarps][32][33];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t row0 = (int64_t(blockIdx.x) * kRowWarps + wid) * 32;
+    if (row0 >= rows) return;  // the whole warp
+    float(*t)[33] = tile[wid];
+    const int64_t r = row0 + lane;
+    const bool live = r < rows;
+    const int nr = int(rows - row0 < 32 ? rows - row0 : 32);
+    auto load = [&](int64_t c0, int nc) {  // t[rr][j] = source element (row0 + rr, c0 + j)
+        for (int rr = 0; rr < nr; ++rr)
+            if (lane < nc) t[rr][lane] = src_at(src, (row0 + rr) * cols + c0 + lane);
+        __syncwarp();
+    };
     bool nonfinite = false;
+    double amax = 0.0, acc = 0.0;
+    float s = 1.0f;
     if (codes) {
         // per-row absmax codes: symmetric INT8 [-127, 127] or E4M3 with saturation at 448
-        double amax = 0.0;
-        for (int64_t j = 0; j < cols; ++j) {
-            float w = src_at(src, base + j);
-            nonfinite |= !isfinite(w);
-            amax = fmax(amax, fabs(double(w)));
+        for (int64_t c0 = 0; c0 < cols; c0 += 32) {
+            const int nc = int(cols - c0 < 32 ? cols - c0 : 32);
+            load(c0, nc);
+            if (live)
+                for (int j = 0; j < nc; ++j) {
+                    const float w = t[lane][j];
+                    nonfinite |= !isfinite(w);
+                    amax = fmax(amax, fabs(double(w)));
+                }
+            __syncwarp();
         }
         const double bound = container == EP_INT8 ? 127.0 : 448.0;
-        float s = amax > 0.0 ? float(ddiv(amax, bound)) : 1.0f;
+        s = amax > 0.0 ? float(ddiv(amax, bound)) : 1.0f;
         if (s == 0.0f) s = FLT_MIN;
-        scales[r] = s;
-        for (int64_t j = 0; j < cols; ++j) {
-            double w = src_at(src, base + j), c;
-            if (amax == 0.0)
-                c = 0.0;
-            else if (container == EP_INT8)
-                c = fmin(127.0, fmax(-127.0, dround(ddiv(w, double(s)))));
-            else
-                c = e4m3_round(float(ddiv(w, double(s))));
-            codes[base + j] = float(c);
-        }
-    } else {
-        for (int64_t j = 0; j < cols; ++j) nonfinite |= !isfinite(src_at(src, base + j));
+        if (live) scales[r] = s;
     }
-    double acc = 0.0;
-    for (int64_t j = 0; j < cols; ++j) {
-        double a = value_at(src, codes, base + j);
-        acc = dadd(acc, dmul(a, a));
+    for (int64_t c0 = 0; c0 < cols; c0 += 32) {
+        const int nc = int(cols - c0 < 32 ? cols - c0 : 32);
+        load(c0, nc);
+        if (live)
+            for (int j = 0; j < nc; ++j) {
+                double a = t[lane][j];
+                if (codes) {
+                    if (amax == 0.0)
+                        a = 0.0;
+                    else if (container == EP_INT8)
+                        a = fmin(127.0, fmax(-127.0, dround(ddiv(a, double(s)))));
+                    else
+                        a = e4m3_round(float(ddiv(a, double(s))));
+                    t[lane][j] = float(a);
+                } else {
+                    nonfinite |= !isfinite(float(a));
+                }
+                acc = dadd(acc, dmul(a, a));
+            }
+        __syncwarp();
+        if (codes)  // write the tile's codes back, row by row (coalesced)
+            for (int rr = 0; rr < nr; ++rr)
+                if (lane < nc) codes[(row0 + rr) * cols + c0 + lane] = t[rr][lane];
+        __syncwarp();
     }
-    rms[r] = float(__dsqrt_rn(ddiv(acc, double(cols))));
+    if (live) rms[r] = float(__dsqrt_rn(ddiv(acc, double(cols))));
     if (nonfinite) atomicOr(bad, 1u);
 }
 
@@ -430,8 +463,8 @@ extern "C" int ep_compress_device(const void *d_src, int32_t src_dtype, int64_t 
 
     // rows: finite check, codes, scales, RMS
     R.check(cudaMemsetAsync(R.S.bad, 0, 4, R.st));
-    rows_kernel<<<int((rows + 127) / 128), 128, 0, R.st>>>(R.src, rows, cols, container, R.S.codes, R.S.scales,
-                                                          R.S.rms, R.S.bad);
+    rows_kernel<<<int((rows + 32 * kRowWarps - 1) / (32 * kRowWarps)), 32 * kRowWarps, 0, R.st>>>(
+        R.src, rows, cols, container, R.S.codes, R.S.scales, R.S.rms, R.S.bad);
     R.check(cudaGetLastError());
     uint32_t bad = 0;
     R.d2h(&bad, R.S.bad, 1);
