@@ -20,7 +20,7 @@ def as_bytes(t):
 
 
 @pytest.mark.parametrize("container", [B.BF16, B.FP16, B.FP32])
-@pytest.mark.parametrize("shape,K", [((100, 808), 0), ((512, 2048), 0), ((64, 1024), 4)])
+@pytest.mark.parametrize("shape,K", [((100, 808), 0), ((512, 2048), 0), ((64, 1024), 4), ((33, 1001), 2)])
 def test_float_containers_to_every_float_dtype(oracle, container, shape, K):
     w = synth.row_lognormal(*shape, seed=shape[0] + container, dtype=SRC[container])
     rc, blob = oracle.compress(w, 4.5, blocks_per_lane=K)

@@ -3,6 +3,8 @@ oracle's stream byte for byte (the oracle's encoder is the reference; the librar
 compressor is pinned to the same bytes elsewhere), for every container, ragged rows, forced tile
 sizes and resolutions, zero rows, escapes at high rates; and fail like the host compressor on
 invalid input.  The streams it writes also decode on the GPU to the oracle's weights."""
+import ctypes as C
+
 import numpy as np
 import pytest
 import torch
@@ -71,3 +73,21 @@ def test_device_errors_match_host():
         with pytest.raises(B.EpError) as e:
             B.compress(tensor, target, container=container)
         assert e.value.status == status
+
+
+def test_device_buffer_too_small_reports_the_size(oracle):
+    w = synth.row_lognormal(128, 512, 4).cuda()
+    rc, ref = oracle.compress(w.cpu(), 4.0)
+    cfg = B._config(4.0)
+    L = B.lib()
+    scratch = torch.empty(L.ep_compress_device_scratch(128, 512, C.byref(cfg)), dtype=torch.uint8, device="cuda")
+    small = torch.empty(256, dtype=torch.uint8, device="cuda")
+    n = C.c_size_t(0)
+    s = torch.cuda.current_stream().cuda_stream
+    rc = L.ep_compress_device(w.data_ptr(), B.BF16, 128, 512, C.byref(cfg), small.data_ptr(), small.numel(),
+                              C.byref(n), scratch.data_ptr(), scratch.numel(), s)
+    assert rc == -5 and n.value == ref.size
+    big = torch.empty(n.value, dtype=torch.uint8, device="cuda")
+    rc = L.ep_compress_device(w.data_ptr(), B.BF16, 128, 512, C.byref(cfg), big.data_ptr(), big.numel(),
+                              C.byref(n), scratch.data_ptr(), scratch.numel(), s)
+    assert rc == 0 and np.array_equal(big.cpu().numpy(), ref)
