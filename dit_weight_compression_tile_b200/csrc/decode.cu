@@ -1,9 +1,8 @@
 // Fused tile decode for sm_100a: ep_decompress.
 //
-// The pages' pipeline ends in entropy coding "in independently decodable tiles" with "fused
-// symbol decoding and numerical weight reconstruction on the GPU" ("EntroPack: Fast and
-// Accurate Entropy-Coded Weight Compression at Arbitrary Bitrates", Abstract).  One kernel, one
-// CTA per SM:
+// The method's last stage ("EntroPack: Fast and Accurate Entropy-Coded Weight Compression at
+// Arbitrary Bitrates", Abstract) is entropy coding in tiles that decode on their own, decoded on
+// the GPU in the same pass that rebuilds the weights.  One kernel, one CTA per SM:
 //   * ep_prepare (a small kernel, once per device copy of a stream) turns the frequency tables
 //     into seven 2048-slot tables in a workspace.  A slot's 32-bit entry holds the token's
 //     frequency (11 bits), the slot's offset inside the token (11 bits), an escape flag and, for

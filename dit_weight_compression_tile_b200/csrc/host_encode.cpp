@@ -4,7 +4,7 @@
 // "EntroPack: Fast and Accurate Entropy-Coded Weight Compression at Arbitrary Bitrates"
 // Abstract: row-normalized E8 lattice quantization, a conditional model of the lattice
 // coordinates, a resolution picked by sampled storage estimates (no repeated full-stream
-// encoding in the normal case), and entropy coding in independently decodable tiles.
+// encoding in the normal case), and entropy coding in tiles that decode on their own.
 // Multithreaded over rows, blocks and tiles; the output bytes do not depend on the thread
 // count (every floating-point reduction keeps a fixed order).
 #include <algorithm>

@@ -17,13 +17,10 @@ import torch.nn.functional as F
 from . import binding as B
 from .compressed import CompressedTensor, LatticeRANSConfig, compress, decompress
 
-_CODE = {torch.float8_e4m3fn: B.FP8E4M3, torch.int8: B.INT8}
-
-
 class CompressedLinear(nn.Module):
     """y = x W^T + b with W held compressed (lossy lattice-rANS, `config`) and decoded per call.
-    Constructing the layer directly leaves it without weight data: call compress_weight or load a
-    checkpoint before running it."""
+    A layer built by the constructor holds no weight until compress_weight runs or a checkpoint
+    is loaded."""
 
     code_dtype = None  # the FP8 / INT8 layers store codes of this dtype
 

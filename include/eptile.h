@@ -12,7 +12,7 @@
  *   "EntroPack: Fast and Accurate Entropy-Coded Weight Compression at Arbitrary Bitrates",
  *       Abstract -- row-normalized E8 lattice quantization, a conditional model of the
  *       lattice coordinates, resolution chosen by sampled storage estimates, entropy coding
- *       in independently decodable tiles, fused GPU symbol decode and reconstruction,
+ *       in tiles that decode on their own, fused GPU symbol decode and reconstruction,
  *       BF16 / FP16 / FP8 / INT8 containers.
  *   "EntroPack README", Configuration -- 0.001 <= target_bpp <= 11.
  *   "Compressed Linear usage", Combine compression with FP8 or INT8 computation -- lossy

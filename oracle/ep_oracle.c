@@ -6,7 +6,7 @@
  *   [ABS]  "EntroPack: Fast and Accurate Entropy-Coded Weight Compression at Arbitrary
  *          Bitrates", Abstract -- row-normalized E8 lattice quantization, conditional
  *          model of lattice coordinates, sampled storage estimates pick the resolution,
- *          entropy coding in independently decodable tiles, fused decode + reconstruction,
+ *          entropy coding in tiles that decode on their own, fused decode + reconstruction,
  *          BF16 / FP16 / FP8 / INT8 containers.
  *   [API]  "EntroPack API reference", compress / CompressedTensor -- non-empty 2-D finite
  *          input, actual_bpp = 8 * storage_nbytes / numel including metadata.
@@ -503,7 +503,7 @@ int32_t or_normalize_freqs(const uint64_t *counts, int32_t n, uint32_t *f)
 }
 
 /* ---------------------------------- tiles -------------------------------------------- */
-/* Reading of "independently decodable tiles" ([ABS]): a tile is 32 lanes x K blocks;
+/* Reading of the tiles ([ABS]: each decodes without the others): a tile is 32 lanes x K blocks;
  * lane l of tile t owns blocks t*32K + 32k + l, k = 0..K-1.  K comes from the block count and
  * the target rate: the power of two at or below nb / 2^16 (at least 16, at most 256), which
  * keeps mid-sized matrices near 2048 tiles, then halved (down to 1) while the tile's expected
@@ -522,7 +522,7 @@ uint32_t or_choose_blocks_per_lane(int64_t nb, double target)
 /* ---------------------------------- value preparation -------------------------------- */
 static int is_code_container(int32_t c) { return c == ORD_INT8 || c == ORD_FP8E4M3; }
 
-/* Per-row absmax INT8 / FP8 codes ([LIN], "lossy compression to the quantized weights";
+/* Per-row absmax INT8 / FP8 codes ([LIN]: the lossy coding applies to the codes themselves;
  * readings: INT8 uses the symmetric range [-127, 127]; an all-zero row gets scale 1). */
 int or_prequant(const void *src, int32_t sdt, int64_t rows, int64_t cols, int32_t container, double *codes,
                 float *scales)
@@ -682,8 +682,8 @@ static size_t meta_bytes(int64_t rows, int32_t container, uint64_t total_tokens,
     return m;
 }
 
-/* Sampled storage estimate ([ABS]: "sampled storage estimates select the quantization
- * resolution without repeated full-stream encoding").  Every S-th block (S = ceil(nb /
+/* Sampled storage estimate ([ABS]: the resolution comes from storage estimated on a sample,
+ * so the full stream is not encoded again and again).  Every S-th block (S = ceil(nb /
  * 65536)) is quantized at k; its symbols are tokenized with splits chosen on the sample,
  * and the payload is estimated as the sample's empirical conditional entropy of tokens
  * plus its raw extra bits, scaled by nb / n_sample.  Exact metadata is added, the table
