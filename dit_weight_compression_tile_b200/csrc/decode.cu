@@ -344,7 +344,7 @@ __device__ __forceinline__ uint32_t raw_bits(const Lane<SMEM> &L, uint32_t rb, u
 // bits, 2 bits below the leading one): d = token - 2^m = ((n - m) << 2 | top) << low | lo; the
 // value is s = (4 | top) << (n - 2) | extra << low | lo with n - 2 - low raw extra bits.  F[i]
 // holds the entry's value field (d, or 2d + c for coordinates 1..6) and its escape flag.
-template <bool SMEM>
+template <bool SMEM, bool WIDE>
 __device__ __forceinline__ void resolve_escapes(const Params &p, uint32_t (&F)[8], uint32_t c, uint32_t par,
                                                 Lane<SMEM> &L, uint32_t &rb) {
     uint32_t lm = 0;
@@ -361,7 +361,7 @@ __device__ __forceinline__ void resolve_escapes(const Params &p, uint32_t (&F)[8
                 const uint32_t low = i == 0 ? 2u : (i < 7 ? 1u : 0u);
                 uint32_t m = i == 0 ? m0 : (i < 7 ? m16 : m7);
                 uint32_t fld = (F[i] >> 11) & 0x1ffu;
-                uint32_t d = (i >= 1 && i <= 6) ? fld >> 1 : fld;
+                uint32_t d = (!WIDE && i >= 1 && i <= 6) ? fld >> 1 : fld;
                 uint32_t q = d >> low;
                 uint32_t n = min(m + (q >> 2), kValueBits - 1u);
                 uint32_t nbits = n - 2u - low;
@@ -375,7 +375,10 @@ __device__ __forceinline__ void resolve_escapes(const Params &p, uint32_t (&F)[8
                     v = 2 * (2 * unzigzag(s >> 1) + int32_t(s & 1u)) + int32_t(c);
                 else
                     v = 2 * (2 * unzigzag(s) + int32_t(par)) + int32_t(c);
-                F[i] = __float_as_uint(__int2float_rn(v + 4352) * 4194304.0f);
+                // the word the reconstruction expects: v (coordinate 0, narrow tables) or
+                // y = (v - c) / 2 (coordinates 1..7 of wide tables), plus 4352, times 2^22
+                const int32_t u = (WIDE && i > 0) ? (v - int32_t(c)) >> 1 : v;
+                F[i] = __float_as_uint(__int2float_rn(u + 4352) * 4194304.0f);
             }
         }
     }
@@ -384,7 +387,7 @@ __device__ __forceinline__ void resolve_escapes(const Params &p, uint32_t (&F)[8
 // ------------------------------------------------------------------ the blocks of one tile
 // Lane l decodes blocks t*32K + 32k + l, k = 0..K-1.  ACT: the last tile, where lanes run out
 // of blocks.  ROWS: the launch's RowLayout.  Returns EP_DEC_* bits.
-template <int DT, bool SMEM, bool ACT, int ROWS, typename Lim>
+template <int DT, bool SMEM, bool ACT, int ROWS, bool WIDE, typename Lim>
 __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L, uint32_t &rb, uint32_t lut,
                                                   Lim wlim, uint32_t t, uint32_t lane) {
     uint32_t b = t * 32u * p.K + lane;
@@ -418,10 +421,19 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
             uint32_t lutc = lut + kSlotBytes + ((e[0] & 0x800u) << 2);  // context 1 + c
 #pragma unroll
             for (int i = 1; i < 7; ++i) e[i] = step<SMEM, ACT>(L, act, lutc);
-            // bits 11 and 12 of the XOR of entries 0..6 are c (seven copies) and the parity p of
-            // y0..y6; context 3 + 2c + p sits at table position 3 + c + 2p
-            uint32_t X = e[0] ^ e[1] ^ e[2] ^ e[3] ^ e[4] ^ e[5] ^ e[6];
-            uint32_t lut7 = lut + 3u * kSlotBytes + ((X & 0x1800u) << 2);
+            // narrow tables: bits 11 and 12 of the XOR of entries 0..6 are c (seven copies) and
+            // the parity p of y0..y6.  Wide tables: bit 11 of entries 1..6 is the parity of y_i,
+            // so c is bit 11 of entry 0 and p is bit 12 of entry 0 xor bit 11 of the others' XOR.
+            // Context 3 + 2c + p sits at table position 3 + c + 2p
+            uint32_t Y;
+            if constexpr (WIDE) {
+                const uint32_t X1 = e[1] ^ e[2] ^ e[3] ^ e[4] ^ e[5] ^ e[6];
+                Y = (e[0] & 0x800u) | ((e[0] ^ (X1 << 1)) & 0x1000u);
+            } else {
+                Y = (e[0] ^ e[1] ^ e[2] ^ e[3] ^ e[4] ^ e[5] ^ e[6]) & 0x1800u;
+            }
+            const uint32_t cbit = (Y >> 11) & 1u, pbit = (Y >> 12) & 1u;
+            uint32_t lut7 = lut + 3u * kSlotBytes + (Y << 2);
             e[7] = step<SMEM, ACT>(L, act, lut7);
             // F keeps the value field and the escape flag of each entry (the flag only matters for
             // escapes, whose F is rebuilt), so the entries themselves die here
@@ -430,15 +442,22 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
             for (int i = 0; i < 8; ++i) F[i] = (e[i] & (kFieldMask | kEscBit)) | kMagic;
             uint32_t O = F[0] | F[1] | F[2] | F[3] | F[4] | F[5] | F[6] | F[7];
             if (__any_sync(0xffffffffu, O & kEscBit))
-                resolve_escapes<SMEM>(p, F, (X >> 11) & 1u, (X >> 12) & 1u, L, rb);
+                resolve_escapes<SMEM, WIDE>(p, F, cbit, pbit, L, rb);
             // v = F 2^-22 - (2^12 + 256) exactly, w = fp32(f_r v): two coordinates per instruction
-            const uint64_t scale2 = pair(__float_as_uint(kInvScale), __float_as_uint(kInvScale));
-            const uint64_t bias2 = pair(__float_as_uint(-kBias), __float_as_uint(-kBias));
+            // narrow: v = F 2^-22 - 4352 for every coordinate; wide: coordinates 1..7 hold y, and
+            // v = 2 y + c = F 2^-21 - 8704 + c (exact: integers below 2^24)
+            const uint64_t scale2 = WIDE ? pair(__float_as_uint(2.0f * kInvScale), __float_as_uint(2.0f * kInvScale))
+                                         : pair(__float_as_uint(kInvScale), __float_as_uint(kInvScale));
+            const float bw = cbit ? -2.0f * kBias + 1.0f : -2.0f * kBias;
+            const uint64_t bias2 = WIDE ? pair(__float_as_uint(bw), __float_as_uint(bw))
+                                        : pair(__float_as_uint(-kBias), __float_as_uint(-kBias));
+            const uint64_t scale01 = WIDE ? pair(__float_as_uint(kInvScale), __float_as_uint(2.0f * kInvScale)) : scale2;
+            const uint64_t bias01 = WIDE ? pair(__float_as_uint(-kBias), __float_as_uint(bw)) : bias2;
             const uint64_t fr2 = pair(__float_as_uint(fr), __float_as_uint(fr));
             Packer<DT> pk;
 #pragma unroll
             for (int i = 0; i < 8; i += 2) {
-                uint64_t v2 = fma_x2(pair(F[i], F[i + 1]), scale2, bias2);
+                uint64_t v2 = fma_x2(pair(F[i], F[i + 1]), i == 0 ? scale01 : scale2, i == 0 ? bias01 : bias2);
                 uint64_t w2 = mul_x2(v2, fr2);
                 pk.put(i, __uint_as_float(uint32_t(v2)), __uint_as_float(uint32_t(w2)));
                 pk.put(i + 1, __uint_as_float(uint32_t(v2 >> 32)), __uint_as_float(uint32_t(w2 >> 32)));
@@ -478,7 +497,7 @@ done:
 
 // Decodes tile t with one warp.  `head` points at the tile (states, region lengths, word area):
 // a shared address (SMEM) or a global pointer.  Returns the EP_DEC_* bits of this lane.
-template <int DT, int ROWS, bool SMEM, typename Ptr>
+template <int DT, int ROWS, bool WIDE, bool SMEM, typename Ptr>
 __device__ __forceinline__ uint32_t decode_tile(const Params &p, uint32_t lut, Ptr head, uint32_t tile_bytes,
                                                 uint32_t t, uint32_t lane) {
     Lane<SMEM> L;
@@ -509,18 +528,18 @@ __device__ __forceinline__ uint32_t decode_tile(const Params &p, uint32_t lut, P
         L.w = lds16(L.wp);
         uint32_t wlim = L.area + 2u * capacity;
         if (uint64_t(t + 1) * 32u * p.K <= p.nb)
-            err = decode_blocks<DT, SMEM, false, ROWS>(p, L, rb, lut, wlim, t, lane);
+            err = decode_blocks<DT, SMEM, false, ROWS, WIDE>(p, L, rb, lut, wlim, t, lane);
         else
-            err = decode_blocks<DT, SMEM, true, ROWS>(p, L, rb, lut, wlim, t, lane);
+            err = decode_blocks<DT, SMEM, true, ROWS, WIDE>(p, L, rb, lut, wlim, t, lane);
     } else {
         L.area = reinterpret_cast<const uint16_t *>(head + kTileHead);
         L.wlim = L.area + (capacity ? capacity - 1u : 0u);
         L.wp = L.area + start < L.wlim ? L.area + start : L.wlim;
         L.w = __ldg(L.wp);
         if (uint64_t(t + 1) * 32u * p.K <= p.nb)
-            err = decode_blocks<DT, SMEM, false, ROWS>(p, L, rb, lut, L.wlim, t, lane);
+            err = decode_blocks<DT, SMEM, false, ROWS, WIDE>(p, L, rb, lut, L.wlim, t, lane);
         else
-            err = decode_blocks<DT, SMEM, true, ROWS>(p, L, rb, lut, L.wlim, t, lane);
+            err = decode_blocks<DT, SMEM, true, ROWS, WIDE>(p, L, rb, lut, L.wlim, t, lane);
     }
     if (L.x != kStateLow) err |= EP_DEC_BAD_END;
     // the front (rANS words) and the back (raw bits) cover the region exactly
@@ -536,20 +555,22 @@ __device__ __forceinline__ uint32_t decode_tile(const Params &p, uint32_t lut, P
 // the coordinate it stands for; an escape token stores its index past 2^m (for coordinates
 // 1..6 as 2 d + c, so that bits 0 and 1 of the field are the coset and the parity of y in
 // every entry of contexts 0..2).
-__device__ __forceinline__ uint32_t token_head(uint32_t c, uint32_t t, uint32_t f, uint32_t m) {
+__device__ __forceinline__ uint32_t token_head(uint32_t c, uint32_t t, uint32_t f, uint32_t m, bool wide) {
     uint32_t field;
     if (t < (1u << m)) {
-        int32_t v;
+        int32_t v;  // narrow tables: the coordinate v; wide tables: y = (v - c) / 2 for coordinates 1..7
         if (c == 0)
             v = 4 * unzigzag(t >> 2) + int32_t(t & 3u);
         else if (c < 3)
-            v = 2 * (2 * unzigzag(t >> 1) + int32_t(t & 1u)) + int32_t(c - 1);
+            v = wide ? 2 * unzigzag(t >> 1) + int32_t(t & 1u)
+                     : 2 * (2 * unzigzag(t >> 1) + int32_t(t & 1u)) + int32_t(c - 1);
         else
-            v = 2 * (2 * unzigzag(t) + int32_t((c - 3) & 1u)) + int32_t((c - 3) >> 1);
+            v = wide ? 2 * unzigzag(t) + int32_t((c - 3) & 1u)
+                     : 2 * (2 * unzigzag(t) + int32_t((c - 3) & 1u)) + int32_t((c - 3) >> 1);
         field = (uint32_t(v + 256) & 0x1ffu) << 11;
     } else {
         uint32_t d = t - (1u << m);
-        uint32_t fv = (c == 1 || c == 2) ? 2u * d + (c - 1) : d;
+        uint32_t fv = (!wide && (c == 1 || c == 2)) ? 2u * d + (c - 1) : d;
         field = kEscBit | ((fv & 0x1ffu) << 11);
     }
     return (min(f, kProbScale - 1u) << 21) | field;
@@ -564,6 +585,7 @@ struct PrepParams {
     uint32_t *tables;        // kContexts x 2048 entries
     uint32_t *status;        // nullable
     uint32_t splits;
+    uint32_t wide;  // value fields hold y for coordinates 1..7
     uint32_t tab_off[kContexts + 1];
 };
 
@@ -618,7 +640,7 @@ __global__ void __launch_bounds__(kPrepThreads) prepare_kernel(const __grid_cons
                 hi = mid;
         }
         uint32_t f = cum[lo + 1] - cum[lo];
-        e = token_head(c, lo, f, split_of_bits(p.splits, c)) | ((slot - cum[lo]) & (kProbScale - 1u));
+        e = token_head(c, lo, f, split_of_bits(p.splits, c), p.wide != 0) | ((slot - cum[lo]) & (kProbScale - 1u));
     }
     // context 3 + 2c + p is stored at position 3 + c + 2p (the decoder forms that offset from
     // the XOR of a block's first seven entries)
@@ -628,7 +650,7 @@ __global__ void __launch_bounds__(kPrepThreads) prepare_kernel(const __grid_cons
 
 // ------------------------------------------------------------------ decode kernel
 // Shared memory: the slot tables, mbarriers, then nbuf tile buffers per warp.
-template <int DT, int ROWS>
+template <int DT, int ROWS, bool WIDE>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
@@ -704,9 +726,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_
                 if (nbuf > 1 && (pend & (1u << o))) mbar_wait(bars + 16u * warp + 8u * o, (phase >> o) & 1u);
                 return;
             }
-            if (tables_ok) err = decode_tile<DT, ROWS, true>(p, lut, bufs + b * p.tile_buf, bytes, t, lane);
+            if (tables_ok) err = decode_tile<DT, ROWS, WIDE, true>(p, lut, bufs + b * p.tile_buf, bytes, t, lane);
         } else if (tables_ok) {
-            err = decode_tile<DT, ROWS, false>(p, lut, p.tiles + size_t(beg) * 16, bytes, t, lane);
+            err = decode_tile<DT, ROWS, WIDE, false>(p, lut, p.tiles + size_t(beg) * 16, bytes, t, lane);
         }
         if (err && p.status) atomicOr(p.status, err);
         __syncwarp();
@@ -724,7 +746,7 @@ struct DeviceCache {
 DeviceCache g_cache;
 
 template <int DT>
-cudaError_t launch(Params &p, uint64_t max_tile, int device, cudaStream_t stream) {
+cudaError_t launch(Params &p, uint64_t max_tile, bool wide, int device, cudaStream_t stream) {
     int sms;
     {
         std::lock_guard<std::mutex> g(g_cache.mu);
@@ -735,7 +757,9 @@ cudaError_t launch(Params &p, uint64_t max_tile, int device, cudaStream_t stream
         }
         if (!g_cache.attr[device][DT]) {
             cudaError_t e = cudaSuccess;
-            for (auto k : {decode_kernel<DT, kRowsAny>, decode_kernel<DT, kRows32>, decode_kernel<DT, kRowsPadded>})
+            for (auto k : {decode_kernel<DT, kRowsAny, false>, decode_kernel<DT, kRows32, false>,
+                           decode_kernel<DT, kRowsPadded, false>, decode_kernel<DT, kRowsAny, true>,
+                           decode_kernel<DT, kRows32, true>, decode_kernel<DT, kRowsPadded, true>})
                 if (e == cudaSuccess)
                     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemLimit));
             if (e != cudaSuccess) return e;
@@ -778,9 +802,14 @@ cudaError_t launch(Params &p, uint64_t max_tile, int device, cudaStream_t stream
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (p.cols & 7u) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsPadded>, p);
-    if ((p.cb & 31u) == 0) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRows32>, p);
-    return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsAny>, p);
+    if (wide) {
+        if (p.cols & 7u) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsPadded, true>, p);
+        if ((p.cb & 31u) == 0) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRows32, true>, p);
+        return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsAny, true>, p);
+    }
+    if (p.cols & 7u) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsPadded, false>, p);
+    if ((p.cb & 31u) == 0) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRows32, false>, p);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsAny, false>, p);
 }
 
 int check_info(const ep_info *info) {
@@ -805,6 +834,14 @@ bool out_dtype_ok(const ep_info *info, int32_t out_dtype) {
            (is_float(out_dtype) && is_float(info->container_dtype));
 }
 
+// tables hold y = (v - c) / 2 instead of v for coordinates 1..7 when a split is beyond the
+// narrow range (v itself would not fit the 9-bit value field)
+bool wide_fields(const ep_info *info) {
+    for (int c = 0; c < kContexts; ++c)
+        if (info->split[c] > kCtxNarrowSplit[c]) return true;
+    return false;
+}
+
 uint32_t pack_splits(const ep_info *info) {
     uint32_t s = 0;
     for (int c = 0; c < kContexts; ++c) s |= uint32_t(info->split[c]) << (4 * c);
@@ -827,6 +864,7 @@ extern "C" int ep_prepare(const ep_info *info, const void *d_blob, void *d_works
     q.tables = static_cast<uint32_t *>(d_workspace);
     q.status = d_status;
     q.splits = pack_splits(info);
+    q.wide = wide_fields(info) ? 1u : 0u;
     q.tab_off[0] = 0;
     for (int c = 0; c < kContexts; ++c) q.tab_off[c + 1] = q.tab_off[c] + info->ntok[c];
     prepare_kernel<<<kContexts * (kProbScale / kPrepThreads), kPrepThreads, 0,
@@ -865,13 +903,14 @@ extern "C" int ep_decompress(const ep_info *info, const void *d_blob, const void
     if (e != cudaSuccess) return EP_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint64_t mt = info->max_tile_nbytes;
+    const bool wide = wide_fields(info);
     switch (out_dtype) {
-    case EP_BF16: e = launch<EP_BF16>(p, mt, device, s); break;
-    case EP_FP16: e = launch<EP_FP16>(p, mt, device, s); break;
-    case EP_FP32: e = launch<EP_FP32>(p, mt, device, s); break;
-    case EP_INT8: e = launch<EP_INT8>(p, mt, device, s); break;
-    case EP_FP8_E4M3: e = launch<EP_FP8_E4M3>(p, mt, device, s); break;
-    case EP_LATTICE_I32: e = launch<EP_LATTICE_I32>(p, mt, device, s); break;
+    case EP_BF16: e = launch<EP_BF16>(p, mt, wide, device, s); break;
+    case EP_FP16: e = launch<EP_FP16>(p, mt, wide, device, s); break;
+    case EP_FP32: e = launch<EP_FP32>(p, mt, wide, device, s); break;
+    case EP_INT8: e = launch<EP_INT8>(p, mt, wide, device, s); break;
+    case EP_FP8_E4M3: e = launch<EP_FP8_E4M3>(p, mt, wide, device, s); break;
+    case EP_LATTICE_I32: e = launch<EP_LATTICE_I32>(p, mt, wide, device, s); break;
     default: return EP_ERR_INVALID_ARG;
     }
     return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;

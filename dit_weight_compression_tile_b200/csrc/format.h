@@ -19,9 +19,12 @@ constexpr uint32_t kTopBits = 2;           // bits below the leading one carried
 constexpr uint32_t kValueBits = 22;        // every coded value is below 2^22
 // low bits of the value kept in every token, and the largest split, per context: coordinate 0
 // keeps v0 mod 4 (coset, parity of y0), coordinates 1..6 the parity of y_i, coordinate 7 none.
-// At the largest splits every direct token decodes to a coordinate in [-256, 255].
+// At the largest splits a direct token decodes to v0 in [-256, 255] (coordinate 0) or to
+// y = (v - c) / 2 in [-256, 255] (coordinates 1..7); up to the narrow splits below, v itself
+// stays in [-256, 255].
 constexpr uint32_t kCtxLow[kContexts] = {2, 1, 1, 0, 0, 0, 0};
-constexpr uint32_t kCtxMaxSplit[kContexts] = {9, 8, 8, 7, 7, 7, 7};
+constexpr uint32_t kCtxMaxSplit[kContexts] = {9, 9, 9, 8, 8, 8, 8};
+constexpr uint32_t kCtxNarrowSplit[kContexts] = {9, 8, 8, 7, 7, 7, 7};
 constexpr uint32_t kMaxAlphabet = 720;     // (1 << 9) + ((22 - 9) << 2 << 2): the largest context alphabet
 constexpr size_t kHeaderBytes = 64;
 constexpr size_t kTileHead = 192;            // per tile: 32 initial states (u32) + 32 word counts (u16)

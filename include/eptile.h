@@ -153,7 +153,9 @@ int ep_stream_info(const void *blob, size_t nbytes, ep_info *info);
  *   d_workspace device buffer of info->workspace_nbytes bytes, 16-byte aligned, caller-owned;
  *               overwritten with 7 slot tables of 2048 32-bit entries (one per context: the
  *               token's frequency, the slot's offset in the token, the escape flag and the
- *               decoded coordinate of a direct token).
+ *               decoded value of a direct token: the coordinate v, or, when a split of the
+ *               stream is beyond the narrow range (8 for coordinates 1..6, 7 for coordinate 7),
+ *               y = (v - c) / 2 for coordinates 1..7).
  *   d_status    nullable device uint32; EP_DEC_BAD_TOKEN is ORed in when the device copy's
  *               frequency tables are damaged.
  * One small kernel launch on `stream`; asynchronous. */

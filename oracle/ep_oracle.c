@@ -52,10 +52,11 @@
 
 /* low bits of the value kept inside every token, and the largest split, per context:
  * coordinate 0 keeps v0 mod 4 (coset and the parity of y0), coordinates 1..6 keep the parity
- * of y_i, coordinate 7 keeps nothing.  The largest splits keep every directly coded
- * coordinate within |v| <= 256. */
+ * of y_i, coordinate 7 keeps nothing.  The largest splits keep every directly coded coordinate
+ * 0 within -256 <= v0 <= 255 and every directly coded y_i = (v_i - c) / 2 of coordinates 1..7
+ * within -256 <= y_i <= 255. */
 static const int32_t CTX_LOW[NCTX] = {2, 1, 1, 0, 0, 0, 0};
-static const int32_t CTX_MAX_SPLIT[NCTX] = {9, 8, 8, 7, 7, 7, 7};
+static const int32_t CTX_MAX_SPLIT[NCTX] = {9, 9, 9, 8, 8, 8, 8};
 
 static size_t al16(size_t n) { return (n + 15) & ~(size_t)15; }
 

@@ -145,7 +145,7 @@ def unzigzag(u):
 
 # low bits kept in every token, and the largest split, per context
 CTX_LOW = (2, 1, 1, 0, 0, 0, 0)
-CTX_MAX_SPLIT = (9, 8, 8, 7, 7, 7, 7)
+CTX_MAX_SPLIT = (9, 9, 9, 8, 8, 8, 8)
 
 
 def tokenize(s, m, low):

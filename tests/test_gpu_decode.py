@@ -173,9 +173,12 @@ def _expected_tables(oracle, blob_np):
     """the decoder's slot tables as include/eptile.h documents them, from the oracle's parse of
     the stream: per context 2048 entries f << 21 | escape << 20 | field << 11 | (slot - cum);
     field = v + 256 for a direct token (v its lattice coordinate), the escape index d (2d + c for
-    coordinates 1..6) otherwise; context 3 + 2c + p stored at position 3 + c + 2p"""
+    coordinates 1..6) otherwise; context 3 + 2c + p stored at position 3 + c + 2p.  When a split
+    is beyond the narrow range (8 for contexts 1, 2, 7 for contexts 3..6) the tables are wide:
+    coordinates 1..7 store y = (v - c) / 2 + 256 and escape index d"""
     rc, info = oracle.parse(blob_np)
     assert rc == 0
+    wide = any(info.split[c] > m for c, m in enumerate((9, 8, 8, 7, 7, 7, 7)))
     b = blob_np.tobytes()
     tab = np.zeros((7, 2048), np.uint32)
     off = info.off_freq
@@ -190,13 +193,15 @@ def _expected_tables(oracle, blob_np):
                 if ctx == 0:
                     v = 4 * oracle.unzigzag(t >> 2) + (t & 3)
                 elif ctx < 3:
-                    v = 2 * (2 * oracle.unzigzag(t >> 1) + (t & 1)) + (ctx - 1)
+                    y = 2 * oracle.unzigzag(t >> 1) + (t & 1)
+                    v = y if wide else 2 * y + (ctx - 1)
                 else:
-                    v = 2 * (2 * oracle.unzigzag(t) + ((ctx - 3) & 1)) + ((ctx - 3) >> 1)
+                    y = 2 * oracle.unzigzag(t) + ((ctx - 3) & 1)
+                    v = y if wide else 2 * y + ((ctx - 3) >> 1)
                 head = (int(f[t]) << 21) | (((v + 256) & 0x1FF) << 11)
             else:
                 d = t - (1 << m)
-                fv = 2 * d + (ctx - 1) if ctx in (1, 2) else d
+                fv = 2 * d + (ctx - 1) if ctx in (1, 2) and not wide else d
                 head = (int(f[t]) << 21) | (1 << 20) | ((fv & 0x1FF) << 11)
             for s in range(cum, cum + int(f[t])):
                 tab[pos, s] = head | (s - cum)
@@ -204,11 +209,14 @@ def _expected_tables(oracle, blob_np):
     return tab
 
 
-@pytest.mark.parametrize("target,container", [(4.0, 0), (0.5, 0), (8.0, 0), (3.0, B.INT8)])
+@pytest.mark.parametrize("target,container", [(4.0, 0), (0.5, 0), (8.0, 0), (11.0, 0), (3.0, B.INT8)])
 def test_prepared_tables_match_documented_layout(oracle, target, container):
     w = synth.gaussian_outliers(128, 2048, seed=16)
     rc, blob = oracle.compress(w, target, container=container)
     assert rc == 0
+    if target == 11.0:  # the wide layout is exercised
+        rc, info = oracle.parse(blob)
+        assert any(info.split[c] > m for c, m in enumerate((9, 8, 8, 7, 7, 7, 7)))
     d = torch.from_numpy(blob).cuda()
     info = B.stream_info(torch.from_numpy(blob))
     status = torch.zeros(1, dtype=torch.int32, device="cuda")

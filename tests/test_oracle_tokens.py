@@ -74,22 +74,32 @@ def test_block_symbols_roundtrip(oracle):
 
 
 def test_direct_tokens_fit_decoder_field(oracle):
-    """at the largest split of each context every direct token names a coordinate with
-    -256 <= v <= 255 (the decoder's 9-bit value field)"""
-    for ctx_kind, (low, mmax) in enumerate([(2, 9), (1, 8), (0, 7)]):
+    """at the largest split of each context every direct token names a coordinate 0 with
+    -256 <= v0 <= 255, and for coordinates 1..7 a y = (v - c) / 2 with -256 <= y <= 255 (the
+    decoder's 9-bit value field); with the splits of the narrow range (8 for coordinates 1..6,
+    7 for coordinate 7) the coordinates themselves stay within -256 <= v <= 255"""
+    for ctx_kind, (low, mmax) in enumerate([(2, 9), (1, 9), (0, 8)]):
         vals = []
         for s in range(1 << mmax):
             if ctx_kind == 0:
                 vals.append(4 * oracle.unzigzag(s >> 2) + (s & 3))
             elif ctx_kind == 1:
-                for c in (0, 1):
-                    vals.append(2 * (2 * oracle.unzigzag(s >> 1) + (s & 1)) + c)
+                vals.append(2 * oracle.unzigzag(s >> 1) + (s & 1))
             else:
-                for c in (0, 1):
+                for p in (0, 1):
+                    vals.append(2 * oracle.unzigzag(s) + p)
+        assert min(vals) >= -256 and max(vals) <= 255
+    for ctx_kind, mmax in ((1, 8), (2, 7)):
+        vals = []
+        for s in range(1 << mmax):
+            for c in (0, 1):
+                if ctx_kind == 1:
+                    vals.append(2 * (2 * oracle.unzigzag(s >> 1) + (s & 1)) + c)
+                else:
                     for p in (0, 1):
                         vals.append(2 * (2 * oracle.unzigzag(s) + p) + c)
         assert min(vals) >= -256 and max(vals) <= 255
-    assert oracle.CTX_LOW == (2, 1, 1, 0, 0, 0, 0) and oracle.CTX_MAX_SPLIT == (9, 8, 8, 7, 7, 7, 7)
+    assert oracle.CTX_LOW == (2, 1, 1, 0, 0, 0, 0) and oracle.CTX_MAX_SPLIT == (9, 9, 9, 8, 8, 8, 8)
 
 
 def test_resolution_grid(oracle):
