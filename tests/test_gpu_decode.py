@@ -115,10 +115,12 @@ def test_repeat_and_streams(oracle):
         assert np.array_equal(as_bytes(o2), r2.view(np.uint8).reshape(-1))
 
 
-def test_damaged_streams_flagged(oracle):
-    """damage found on the device goes to the status word; the decode stays in bounds"""
+@pytest.mark.parametrize("target", [4.0, 8.0])
+def test_damaged_streams_flagged(oracle, target):
+    """damage found on the device goes to the status word; the decode stays in bounds (narrow
+    value fields at 4 bpp, wide ones at 8 bpp)"""
     w = synth.gaussian(256, 1024, 0.02, 15)
-    rc, blob = oracle.compress(w, 4.0)
+    rc, blob = oracle.compress(w, target)
     rc, info = oracle.parse(blob)
     host_info = B.stream_info(torch.from_numpy(blob))
     rng = np.random.default_rng(1)
