@@ -147,6 +147,11 @@ __device__ __forceinline__ uint64_t mul_x2(uint64_t a, uint64_t b) {
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
+__device__ __forceinline__ uint64_t add_x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
 __device__ __forceinline__ uint64_t pair(uint32_t lo, uint32_t hi) { return uint64_t(lo) | (uint64_t(hi) << 32); }
 
 template <>
@@ -214,6 +219,15 @@ struct Packer<EP_INT8> {
     __device__ __forceinline__ void put(int i, float, float w) {
         float r = __fadd_rn(fminf(fmaxf(w, -127.0f), 127.0f), 12582912.0f);
         b[i] = __float_as_uint(r);
+    }
+    // coordinates i and i + 1 at once: the two clamps, then one paired add
+    __device__ __forceinline__ void put2(int i, uint64_t w2) {
+        const float c0 = fminf(fmaxf(__uint_as_float(uint32_t(w2)), -127.0f), 127.0f);
+        const float c1 = fminf(fmaxf(__uint_as_float(uint32_t(w2 >> 32)), -127.0f), 127.0f);
+        const uint64_t r = add_x2(pair(__float_as_uint(c0), __float_as_uint(c1)),
+                                  pair(__float_as_uint(12582912.0f), __float_as_uint(12582912.0f)));
+        b[i] = uint32_t(r);
+        b[i + 1] = uint32_t(r >> 32);
     }
     __device__ __forceinline__ void store(void *out, uint32_t blk) {
         uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
@@ -459,8 +473,12 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
             for (int i = 0; i < 8; i += 2) {
                 uint64_t v2 = fma_x2(pair(F[i], F[i + 1]), i == 0 ? scale01 : scale2, i == 0 ? bias01 : bias2);
                 uint64_t w2 = mul_x2(v2, fr2);
-                pk.put(i, __uint_as_float(uint32_t(v2)), __uint_as_float(uint32_t(w2)));
-                pk.put(i + 1, __uint_as_float(uint32_t(v2 >> 32)), __uint_as_float(uint32_t(w2 >> 32)));
+                if constexpr (DT == EP_INT8) {
+                    pk.put2(i, w2);
+                } else {
+                    pk.put(i, __uint_as_float(uint32_t(v2)), __uint_as_float(uint32_t(w2)));
+                    pk.put(i + 1, __uint_as_float(uint32_t(v2 >> 32)), __uint_as_float(uint32_t(w2 >> 32)));
+                }
             }
             if constexpr (RAG) {
                 // a padded row's last block keeps its first cols % 8 values
