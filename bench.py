@@ -375,37 +375,25 @@ def run_ours(a, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     prepare_us = p0.elapsed_time(p1) * 1e3 / (prep_reps * len(infos))
 
-    # end to end through the public API with host buffers: every step, pinned H2D of every
-    # stream, the tables, the decode and D2H of every container into pinned memory.  Consecutive
-    # (step, tensor) units alternate between two CUDA streams with their own device buffers, so
-    # that one unit's device-to-host read overlaps the next unit's host-to-device copy
+    # end to end through the C ABI with host buffers (ep_decompress_host): every step, for every
+    # tensor, the pinned stream copied in, the tables, the decode and the container copied back
+    # into pinned memory.  Consecutive (step, tensor) units alternate between two CUDA streams with
+    # their own device scratch, so that one unit's device-to-host read overlaps the next unit's
+    # host-to-device copy
     host_blobs = [blob.pin_memory() for _, blob in layers]
     biggest = max(range(len(infos)), key=lambda i: infos[i].out_nbytes)
     host_outs = [torch.empty(infos[biggest].shape, dtype=infos[biggest].dtype).pin_memory() for _ in range(2)]
     streams = [stream, torch.cuda.Stream(dev)]
-    n = len(infos)
-    sets = []  # per stream: (device blob, workspace, device output) of every tensor
-    for j in range(2):
-        if rot >= 2:
-            sets.append([(blobs[j * n + i], works[j * n + i], outs[j * n + i]) for i in range(n)])
-        elif j == 0:
-            sets.append([(blobs[i], works[i], outs[i]) for i in range(n)])
-        else:
-            sets.append([(torch.empty_like(blobs[i]), torch.empty_like(works[i]), torch.empty_like(outs[i]))
-                         for i in range(n)])
+    scratch_nbytes = max(B.decompress_host_scratch(info) for info in infos)
+    scratches = [torch.empty(scratch_nbytes, dtype=torch.uint8, device=dev) for _ in range(2)]
     unit = [0]
 
     def e2e_step():
         for i, info in enumerate(infos):
             j = unit[0] % 2
             unit[0] += 1
-            d, w_, o = sets[j][i]
-            s_ = streams[j]
-            with torch.cuda.stream(s_):
-                d.copy_(host_blobs[i], non_blocking=True)
-                B.prepare(d, info, workspace=w_, stream=s_)
-                B.decompress(d, info, workspace=w_, out=o, stream=s_)
-                host_outs[j].view(-1)[: o.numel()].copy_(o.view(-1), non_blocking=True)
+            o = host_outs[j].view(-1)[: info.rows * info.cols].view(info.shape)
+            B.decompress_host(host_blobs[i], info, out=o, scratch=scratches[j], stream=streams[j], sync=False)
 
     e2e_steps = max(2, min(200, int(0.5 / max(1e-9, (in_bytes + out_bytes) / 40e9))))
     e2e_step()

@@ -6,7 +6,7 @@ it.  Importing the package loads nothing; the first use of a binding name import
 ``binding``, whose ``lib()`` fails loudly when the built library is missing.
 """
 _BINDING_NAMES = ("BF16", "FP16", "FP32", "INT8", "FP8E4M3", "EpError", "compress", "compress_device", "prepare",
-                  "decompress", "stream_info", "lib", "StreamInfo")
+                  "decompress", "decompress_host", "stream_info", "lib", "StreamInfo")
 
 
 _COMPRESSED_NAMES = ("CompressedTensor", "LatticeRANSConfig")

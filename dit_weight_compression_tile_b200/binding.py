@@ -93,6 +93,10 @@ def lib():
         L.ep_decompress.argtypes = [C.POINTER(StreamInfo), p, p, p, C.c_int32, p, p]
         L.ep_decompress_noalloc.restype = C.c_int
         L.ep_decompress_noalloc.argtypes = [C.POINTER(StreamInfo), p, p, C.c_int32, p, p]
+        L.ep_decompress_host_scratch.restype = C.c_size_t
+        L.ep_decompress_host_scratch.argtypes = [C.POINTER(StreamInfo), C.c_int32]
+        L.ep_decompress_host.restype = C.c_int
+        L.ep_decompress_host.argtypes = [C.POINTER(StreamInfo), p, p, C.c_int32, p, C.c_size_t, p, p]
         L.ep_status_string.restype = C.c_char_p
         L.ep_status_string.argtypes = [C.c_int]
         _lib = L
@@ -232,4 +236,51 @@ def decompress(d_blob, info=None, workspace=None, out=None, status=None, stream=
     rc = lib().ep_decompress(C.byref(info), d_blob.data_ptr(), workspace.data_ptr(), out.data_ptr(), dt, st, s)
     if rc != 0:
         raise EpError(rc, "ep_decompress")
+    return out
+
+
+def decompress_host_scratch(info, out_dtype=None):
+    """bytes of device scratch that ``decompress_host`` needs (ep_decompress_host_scratch)"""
+    dt = info.container_dtype if out_dtype is None else dtype_code(out_dtype)
+    return int(lib().ep_decompress_host_scratch(C.byref(info), dt))
+
+
+def decompress_host(h_blob, info=None, out=None, out_dtype=None, scratch=None, status=None, stream=None,
+                    device=None, sync=True):
+    """decompress(compressed) for a stream in host memory (ep_decompress_host): the stream is
+    copied to the GPU, decoded by the fused kernel there and the weights copied back into a host
+    tensor, all on one CUDA stream.  ``h_blob``: CPU uint8 tensor (pinned memory lets the copies
+    run without staging).  ``out``: optional CPU tensor of ``info.shape`` and the output dtype.
+    ``scratch``: optional CUDA uint8 tensor of ``decompress_host_scratch`` bytes, allocated on
+    ``device`` (default: the current CUDA device) when omitted.  With ``sync`` the call waits for
+    the stream before returning; otherwise ``out`` is valid once ``stream`` has been synchronised."""
+    if h_blob.is_cuda or h_blob.dtype != torch.uint8 or not h_blob.is_contiguous():
+        raise EpError(-1, "decompress_host takes the stream as a contiguous CPU uint8 tensor")
+    if not torch.cuda.is_available():
+        raise EpError(-1, "decompress_host decodes on a CUDA device and none is available")
+    if info is None:
+        info = stream_info(h_blob)
+    dt = info.container_dtype if out_dtype is None else dtype_code(out_dtype)
+    want = TORCH_DTYPE.get(dt)
+    if want is None:
+        raise EpError(-1, f"output dtype code {dt}")
+    if out is None:
+        out = torch.empty(info.shape, dtype=want, pin_memory=True)
+    if out.is_cuda or out.dtype != want or tuple(out.shape) != info.shape or not out.is_contiguous():
+        raise EpError(-1, "output tensor does not match the stream")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    need = decompress_host_scratch(info, dt)
+    if scratch is None:
+        scratch = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    if not scratch.is_cuda or scratch.dtype != torch.uint8 or scratch.numel() < need:
+        raise EpError(-1, "scratch does not match the stream")
+    st = status.data_ptr() if status is not None else None
+    cs = stream or torch.cuda.current_stream(scratch.device)
+    with torch.cuda.device(scratch.device):
+        rc = lib().ep_decompress_host(C.byref(info), h_blob.data_ptr(), out.data_ptr(), dt, scratch.data_ptr(),
+                                      scratch.numel(), st, cs.cuda_stream)
+    if rc != 0:
+        raise EpError(rc, "ep_decompress_host")
+    if sync:
+        cs.synchronize()
     return out

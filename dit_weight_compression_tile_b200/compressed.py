@@ -198,13 +198,18 @@ def _tables(ct, stream):
 
 def decompress(compressed, config=None, stream=None, out=None, status=None):
     """decompress(compressed, config) -> tensor of compressed.shape and compressed.dtype on
-    compressed.device (which must be a CUDA device for a lattice stream).  ``config`` carries
-    only encoding settings here, so it is accepted and not used."""
+    compressed.device.  A lattice stream is always decoded by the GPU kernel: a stream held in
+    host memory is copied to the current CUDA device, decoded there and the weights copied back
+    (ep_decompress_host); without a CUDA device that raises.  ``config`` carries only encoding
+    settings here, so it is accepted and not used."""
     ct = compressed
     if ct._raw is not None:
         return ct._raw.to(dtype=ct.dtype, copy=True)
     if not ct._blob.is_cuda:
-        raise B.EpError(-1, "decompress needs the stream on a CUDA device: use .to('cuda') first")
+        if out is not None and out.is_cuda:
+            raise B.EpError(-1, "the output of a host-resident stream is a host tensor")
+        return B.decompress_host(ct._blob.contiguous(), ct._info, out=out, out_dtype=ct.dtype, status=status,
+                                 stream=stream)
     s = stream or torch.cuda.current_stream(ct._blob.device)
     work = _tables(ct, s)
     return B.decompress(ct._blob, ct._info, workspace=work, out=out, status=status, stream=s, out_dtype=ct.dtype)

@@ -982,3 +982,45 @@ extern "C" int ep_decompress_noalloc(const ep_info *info, const void *d_blob, vo
     if (rc != EP_OK) return rc;
     return ep_decompress(info, d_blob, tables, d_out, out_dtype, d_status, stream);
 }
+
+// ------------------------------------------------------------------ ep_decompress_host
+// The same decode for a stream and an output in host memory: one copy in, ep_prepare,
+// ep_decompress, one copy out, all on the caller's stream; the device buffers are carved from
+// caller scratch (stream, tables, output, each 256-byte aligned).
+namespace ep {
+namespace {
+
+size_t out_elt_bytes(int32_t dt) { return dt == EP_FP32 || dt == EP_LATTICE_I32 ? 4 : (dt == EP_BF16 || dt == EP_FP16) ? 2 : 1; }
+size_t al256(size_t n) { return (n + 255) & ~size_t(255); }
+
+}  // namespace
+}  // namespace ep
+
+extern "C" size_t ep_decompress_host_scratch(const ep_info *info, int32_t out_dtype) {
+    using namespace ep;
+    if (!info || info->rows <= 0 || info->cols <= 0 || !out_dtype_ok(info, out_dtype)) return 0;
+    return al256(info->storage_nbytes) + al256(info->workspace_nbytes) +
+           al256(size_t(info->rows) * size_t(info->cols) * out_elt_bytes(out_dtype));
+}
+
+extern "C" int ep_decompress_host(const ep_info *info, const void *h_blob, void *h_out, int32_t out_dtype,
+                                  void *d_scratch, size_t scratch_nbytes, uint32_t *d_status, ep_stream_t stream) {
+    using namespace ep;
+    if (!info || !h_blob || !h_out || !d_scratch || !out_dtype_ok(info, out_dtype)) return EP_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(d_scratch) & 255u) return EP_ERR_INVALID_ARG;
+    int rc = check_info(info);
+    if (rc != EP_OK) return rc;
+    if (scratch_nbytes < ep_decompress_host_scratch(info, out_dtype)) return EP_ERR_INVALID_ARG;
+    uint8_t *d_blob = static_cast<uint8_t *>(d_scratch);
+    uint8_t *d_work = d_blob + al256(info->storage_nbytes);
+    uint8_t *d_out = d_work + al256(info->workspace_nbytes);
+    const size_t out_bytes = size_t(info->rows) * size_t(info->cols) * out_elt_bytes(out_dtype);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(d_blob, h_blob, info->storage_nbytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return EP_ERR_CUDA;
+    rc = ep_prepare(info, d_blob, d_work, d_status, stream);
+    if (rc != EP_OK) return rc;
+    rc = ep_decompress(info, d_blob, d_work, d_out, out_dtype, d_status, stream);
+    if (rc != EP_OK) return rc;
+    return cudaMemcpyAsync(h_out, d_out, out_bytes, cudaMemcpyDeviceToHost, s) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}

@@ -201,6 +201,25 @@ int ep_decompress(const ep_info *info, const void *d_blob, const void *d_workspa
 int ep_decompress_noalloc(const ep_info *info, const void *d_blob, void *d_out, int32_t out_dtype,
                           uint32_t *d_status, ep_stream_t stream);
 
+/* Device scratch that ep_decompress_host needs for this stream and output dtype: the device copy
+ * of the stream, the slot tables and the output, each rounded up to 256 bytes.  0 for invalid
+ * arguments (an output dtype the stream cannot decode to included). */
+size_t ep_decompress_host_scratch(const ep_info *info, int32_t out_dtype);
+
+/* decompress(compressed) for a stream and an output in HOST memory (the API reference returns the
+ * tensor on the compressed tensor's device): one copy of the stream to the device, ep_prepare,
+ * ep_decompress, one copy of the output back, all on `stream`.  Asynchronous: synchronise the
+ * stream before reading h_out; pinned host buffers let the copies run without staging.
+ *   info        from ep_stream_info on the same stream.
+ *   h_blob      host pointer to the whole stream (info->storage_nbytes bytes).
+ *   h_out       host pointer to rows * cols elements of out_dtype (as for ep_decompress).
+ *   d_scratch   device buffer of at least ep_decompress_host_scratch bytes, 256-byte aligned,
+ *               caller-owned.
+ *   d_status    nullable device uint32 (as for ep_decompress).
+ * Errors as ep_decompress; the library allocates nothing. */
+int ep_decompress_host(const ep_info *info, const void *h_blob, void *h_out, int32_t out_dtype, void *d_scratch,
+                       size_t scratch_nbytes, uint32_t *d_status, ep_stream_t stream);
+
 /* static string for a status code */
 const char *ep_status_string(int status);
 

@@ -14,7 +14,8 @@ def test_exports_every_declared_symbol():
     names = B.declared_functions()
     assert set(names) == {"ep_compress_bound", "ep_compress_host", "ep_compress_device_scratch",
                           "ep_compress_device", "ep_stream_info", "ep_prepare", "ep_decompress",
-                          "ep_decompress_noalloc", "ep_status_string"}
+                          "ep_decompress_noalloc", "ep_decompress_host_scratch", "ep_decompress_host",
+                          "ep_status_string"}
     lib = B.lib()
     for n in names:
         assert hasattr(lib, n), n
@@ -151,3 +152,33 @@ def test_decode_calls_reject_bad_arguments_before_any_launch():
     bad = B.StreamInfo.from_buffer_copy(info)
     bad.cols = 0
     assert L.ep_decompress(C.byref(bad), fake, fake, fake, info.container_dtype, None, None) == -1
+
+
+def test_host_buffer_decode_checks_arguments_before_any_copy():
+    """ep_decompress_host_scratch sums the 256-byte rounded stream, tables and output; the call
+    rejects null pointers, misaligned or short scratch and an output dtype the stream cannot
+    decode to, on the host"""
+    blob = B.compress(synth.gaussian(40, 100, 0.02, 6), 4.0)
+    info = B.stream_info(blob)
+    L = B.lib()
+    r = lambda n: (n + 255) // 256 * 256
+    assert L.ep_decompress_host_scratch(C.byref(info), B.BF16) == \
+        r(info.storage_nbytes) + r(info.workspace_nbytes) + r(40 * 100 * 2)
+    assert L.ep_decompress_host_scratch(C.byref(info), B.FP32) == \
+        r(info.storage_nbytes) + r(info.workspace_nbytes) + r(40 * 100 * 4)
+    assert L.ep_decompress_host_scratch(C.byref(info), B.INT8) == 0
+    assert L.ep_decompress_host_scratch(None, B.BF16) == 0
+    need = L.ep_decompress_host_scratch(C.byref(info), info.container_dtype)
+    fake = 1 << 20  # never dereferenced: every call below fails its checks first
+    h = blob.data_ptr()
+    dt = info.container_dtype
+    assert L.ep_decompress_host(None, h, fake, dt, fake, need, None, None) == -1
+    assert L.ep_decompress_host(C.byref(info), None, fake, dt, fake, need, None, None) == -1
+    assert L.ep_decompress_host(C.byref(info), h, None, dt, fake, need, None, None) == -1
+    assert L.ep_decompress_host(C.byref(info), h, fake, dt, None, need, None, None) == -1
+    assert L.ep_decompress_host(C.byref(info), h, fake, dt, fake + 16, need, None, None) == -1
+    assert L.ep_decompress_host(C.byref(info), h, fake, dt, fake, need - 1, None, None) == -1
+    assert L.ep_decompress_host(C.byref(info), h, fake, B.INT8, fake, need, None, None) == -1
+    bad = B.StreamInfo.from_buffer_copy(info)
+    bad.split[3] = 12
+    assert L.ep_decompress_host(C.byref(bad), h, fake, dt, fake, need, None, None) == -6

@@ -74,10 +74,12 @@ def test_unreachable_target_keeps_the_tensor_raw():
     assert back.compress_method == "raw" and torch.equal(back.to(dtype=torch.float32).decompress(), w.float())
 
 
-def test_decode_without_a_gpu_copy_fails_loudly():
+def test_decode_without_a_cuda_device_fails_loudly(monkeypatch):
+    """a host-resident lattice stream is decoded by the GPU kernel or not at all"""
     ct = compress(synth.gaussian(32, 256, 0.02, 2), LatticeRANSConfig(target_bpp=4.0))
     assert ct.device.type == "cpu"
-    with pytest.raises(B.EpError):
+    monkeypatch.setattr(torch.cuda, "is_available", lambda: False)
+    with pytest.raises(B.EpError, match="CUDA device"):
         decompress(ct)
 
 

@@ -77,3 +77,36 @@ def test_cpu_copy_moves_to_the_gpu(oracle):
     out = g.decompress()
     assert out.dtype == torch.float8_e4m3fn
     assert np.array_equal(as_bytes(out), ref.view(np.uint8).reshape(-1))
+
+
+@pytest.mark.parametrize("container,out_dt,shape", [(B.BF16, None, (300, 1000)), (B.FP16, B.FP32, (64, 2048)),
+                                                    (B.FP32, B.BF16, (17, 37)), (B.INT8, None, (128, 512)),
+                                                    (B.FP8E4M3, None, (96, 808))])
+def test_host_buffer_decode(oracle, container, out_dt, shape):
+    """ep_decompress_host: the stream in host memory, the weights back in host memory, equal byte
+    for byte to the oracle's decode; also through CompressedTensor.decompress on a CPU copy"""
+    src = {B.INT8: torch.bfloat16, B.FP8E4M3: torch.bfloat16}.get(container, SRC.get(container))
+    w = synth.row_lognormal(*shape, seed=shape[1], dtype=src)
+    target = 6.0 if container in (B.INT8, B.FP8E4M3) else 5.0
+    rc, blob = oracle.compress(w, target, container=container)
+    assert rc == 0
+    h = torch.from_numpy(blob).pin_memory()
+    info = B.stream_info(h)
+    rc, st, _, ref = oracle.decode(blob, out_dtype=out_dt or 0)
+    assert rc == 0 and st == 0
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = B.decompress_host(h, info, out_dtype=out_dt, status=status)
+    assert not got.is_cuda and int(status.item()) == 0
+    assert np.array_equal(as_bytes(got), ref.view(np.uint8).reshape(-1))
+    # caller-owned scratch and output, asynchronous on a side stream
+    s = torch.cuda.Stream()
+    scratch = torch.empty(B.decompress_host_scratch(info, out_dt), dtype=torch.uint8, device="cuda")
+    out = torch.empty(info.shape, dtype=got.dtype).pin_memory()
+    B.decompress_host(h, info, out=out, out_dtype=out_dt, scratch=scratch, stream=s, sync=False)
+    s.synchronize()
+    assert np.array_equal(as_bytes(out), ref.view(np.uint8).reshape(-1))
+    if out_dt is None:
+        ct = CompressedTensor(torch.from_numpy(blob), info)
+        via_ct = ct.decompress()
+        assert via_ct.device.type == "cpu"
+        assert np.array_equal(as_bytes(via_ct), ref.view(np.uint8).reshape(-1))
