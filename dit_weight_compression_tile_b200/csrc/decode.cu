@@ -39,8 +39,21 @@ namespace {
 constexpr int kMaxWarps = 32;
 constexpr uint32_t kSlotBytes = kProbScale * 4;                   // one context's slot table
 constexpr size_t kLutBytes = size_t(kContexts) * kSlotBytes;      // 56 KB: the prepared tables
+// A paired stream's tables: contexts 0 and 3..6 (slot tables, context 3 + 2c + p at position
+// 1 + c + 2p), the pair tables of cosets 0 and 1 (4096 slots of 8 bytes), then 2 x 256 token
+// fields for escaped pairs.
+constexpr uint32_t kPairTabOff = 5 * kSlotBytes;
+constexpr uint32_t kPairTabBytes = kPairScale * 8;
+constexpr uint32_t kTokFieldOff = kPairTabOff + 2 * kPairTabBytes;
+static_assert(kTokFieldOff + 2 * kPairTokFields * 4 == kPairedTableBytes, "paired table layout");
 constexpr size_t kBarBytes = size_t(kMaxWarps) * 2 * 8 + 16;      // two mbarriers per warp + one for the tables
 constexpr size_t kFixedBytes = kLutBytes + kBarBytes;
+constexpr size_t kPairedFixedBytes = kPairedTableBytes + kBarBytes;
+static_assert(kPairedFixedBytes % 16 == 0, "tile buffers must start 16-byte aligned");
+
+// How a block's coordinates are coded, fixed per launch: one token each with value fields
+// holding v (narrow) or y (wide), or coordinates 1..6 as three pair symbols (paired, narrow fields)
+enum Coding { kNarrow = 0, kWide = 1, kPaired = 2 };
 constexpr uint32_t kSlack = 160;      // bytes past a tile that a lane's bounded over-read may touch
                                       // (8 blocks of 8 tokens between checks, one word each, + 1)
 constexpr size_t kSmemLimit = 232448; // shared memory one CTA may use on sm_100
@@ -73,6 +86,8 @@ struct Params {
     uint32_t tile_buf;       // bytes of each tile buffer (multiple of 16, includes kSlack)
     uint32_t nbuf;           // tile buffers per warp (1 or 2); 0: tiles are read from global memory
     uint32_t splits;         // 4 bits per context
+    uint32_t pair_A[2];      // paired: token alphabet length of contexts 1 and 2
+    uint32_t pair_rawb[2];   // paired: raw bits of one token of an escaped pair (<= 6)
 };
 
 // How a stream's blocks map onto rows, fixed per launch: kRowsAny (a lane's row is tested after
@@ -96,6 +111,9 @@ __device__ __forceinline__ uint32_t lds16(uint32_t a) {
     uint32_t v;
     asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a));
     return v;
+}
+__device__ __forceinline__ void lds64(uint32_t a, uint32_t &lo, uint32_t &hi) {
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo), "=r"(hi) : "r"(a));
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -317,6 +335,22 @@ struct Lane<false> {
     __device__ __forceinline__ uint32_t consumed(uint32_t start) const { return uint32_t(wp - area) - start; }
 };
 
+// Below 2^16 the state takes the next word of the lane's region; the new state is stored.
+template <bool SMEM>
+__device__ __forceinline__ void renorm(Lane<SMEM> &L, uint32_t xn) {
+    if constexpr (SMEM) {
+        // predicated: x = x * 2^16 + w, then the next word of the region is read ahead
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.lt.u32 p, %0, 65536;\n\t@p mad.lo.u32 %0, %0, 65536, %2;\n\t"
+            "@p add.u32 %1, %1, 2;\n\t@p ld.shared.u16 %2, [%1];\n\t}"
+            : "+r"(xn), "+r"(L.wp), "+r"(L.w));
+    } else if (xn < kStateLow) {
+        xn = (xn << 16) | L.w;
+        L.advance();
+    }
+    L.x = xn;
+}
+
 // One token of one lane: a lookup in the context's slot table and the rANS update
 // x' = f (x >> 11) + (slot - cum); below 2^16 the state takes the next word of the region.
 template <bool SMEM, bool ACT>
@@ -329,18 +363,25 @@ __device__ __forceinline__ uint32_t step(Lane<SMEM> &L, bool act, uint32_t lut) 
     asm("mad.lo.u32 %0, %1, -8192, %2;" : "=r"(a) : "r"(xs), "r"(t));
     uint32_t e = lds32(a);
     uint32_t xn = (e >> 21) * xs + (e & (kProbScale - 1u));
-    if constexpr (SMEM) {
-        // predicated: x = x * 2^16 + w, then the next word of the region is read ahead
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.lt.u32 p, %0, 65536;\n\t@p mad.lo.u32 %0, %0, 65536, %2;\n\t"
-            "@p add.u32 %1, %1, 2;\n\t@p ld.shared.u16 %2, [%1];\n\t}"
-            : "+r"(xn), "+r"(L.wp), "+r"(L.w));
-    } else if (xn < kStateLow) {
-        xn = (xn << 16) | L.w;
-        L.advance();
-    }
-    L.x = xn;
+    renorm(L, xn);
     return e;
+}
+
+// One pair symbol: a lookup in the coset's 4096-slot pair table of 8-byte entries (frequency
+// [20,32) and slot offset [0,12), then the two coordinates' value fields at bits 11..20 and
+// 21..30, or bit 31 for an escaped pair) and the update x' = f (x >> 12) + (slot - cum).
+// Returns the entry's second word.
+template <bool SMEM, bool ACT>
+__device__ __forceinline__ uint32_t step2(Lane<SMEM> &L, bool act, uint32_t lutp) {
+    if (ACT && !act) return 0u;
+    // slot address lutp + 8 (x mod 2^12) = lutp + 8x - 2^15 (x >> 12), exact modulo 2^32
+    uint32_t xs = L.x >> kPairBits, a, t, lo, hi;
+    asm("mad.lo.u32 %0, %1, 8, %2;" : "=r"(t) : "r"(L.x), "r"(lutp));
+    asm("mad.lo.u32 %0, %1, -32768, %2;" : "=r"(a) : "r"(xs), "r"(t));
+    lds64(a, lo, hi);
+    uint32_t xn = (lo >> 20) * xs + (lo & (kPairScale - 1u));
+    renorm(L, xn);
+    return hi;
 }
 
 // `nbits` raw bits at raw-bit position rb of the lane (the region's last word holds bits
@@ -398,12 +439,30 @@ __device__ __forceinline__ void resolve_escapes(const Params &p, uint32_t (&F)[8
     }
 }
 
+// Escaped pairs of a block (the warp has at least one): their two tokens are the first raw bits of
+// the block, pair by pair, each in p.pair_rawb[c] bits; the value fields come from the coset's
+// token-field table.  A token beyond the alphabet is reported (the index stays inside the table).
+template <bool SMEM>
+__device__ __forceinline__ uint32_t resolve_pair(const Params &p, uint32_t h, uint32_t c, uint32_t tf,
+                                                 const Lane<SMEM> &L, uint32_t &rb, uint32_t &err) {
+    if (!(h >> 31)) return h;
+    // a damaged region cannot move the raw reads below the tile's head
+    rb = min(rb, 16u * (L.end + 88u));
+    const uint32_t nb = p.pair_rawb[c];
+    const uint32_t bits = raw_bits(L, rb, 2u * nb);
+    rb += 2u * nb;
+    const uint32_t ta = bits & ((1u << nb) - 1u), tb = bits >> nb;
+    if (ta >= p.pair_A[c] || tb >= p.pair_A[c]) err |= EP_DEC_BAD_TOKEN;
+    return lds32(tf + 4u * (ta & (kPairTokFields - 1u))) | (lds32(tf + 4u * (tb & (kPairTokFields - 1u))) << 10);
+}
+
 // ------------------------------------------------------------------ the blocks of one tile
 // Lane l decodes blocks t*32K + 32k + l, k = 0..K-1.  ACT: the last tile, where lanes run out
 // of blocks.  ROWS: the launch's RowLayout.  Returns EP_DEC_* bits.
-template <int DT, bool SMEM, bool ACT, int ROWS, bool WIDE, typename Lim>
+template <int DT, bool SMEM, bool ACT, int ROWS, int MODE, typename Lim>
 __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L, uint32_t &rb, uint32_t lut,
                                                   Lim wlim, uint32_t t, uint32_t lane) {
+    constexpr bool WIDE = MODE == kWide;
     uint32_t b = t * 32u * p.K + lane;
     uint32_t row = b / p.cb, col = b - row * p.cb;
     // the factor of the current row and of the next one (read a row ahead)
@@ -429,31 +488,59 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
                 err |= EP_DEC_WORD_OVERRUN;
                 goto done;
             }
-            uint32_t e[8];
-            // coordinate 0 (context 0); bit 11 of every entry of contexts 0..2 is the coset c
-            e[0] = step<SMEM, ACT>(L, act, lut);
-            uint32_t lutc = lut + kSlotBytes + ((e[0] & 0x800u) << 2);  // context 1 + c
-#pragma unroll
-            for (int i = 1; i < 7; ++i) e[i] = step<SMEM, ACT>(L, act, lutc);
-            // narrow tables: bits 11 and 12 of the XOR of entries 0..6 are c (seven copies) and
-            // the parity p of y0..y6.  Wide tables: bit 11 of entries 1..6 is the parity of y_i,
-            // so c is bit 11 of entry 0 and p is bit 12 of entry 0 xor bit 11 of the others' XOR.
-            // Context 3 + 2c + p sits at table position 3 + c + 2p
-            uint32_t Y;
-            if constexpr (WIDE) {
-                const uint32_t X1 = e[1] ^ e[2] ^ e[3] ^ e[4] ^ e[5] ^ e[6];
-                Y = (e[0] & 0x800u) | ((e[0] ^ (X1 << 1)) & 0x1000u);
+            // F keeps the value field and the escape flag of each coordinate (the flag only matters
+            // for escapes, whose F is rebuilt), so the entries themselves die early
+            uint32_t F[8], Y;
+            if constexpr (MODE == kPaired) {
+                // token 0, the pairs (1,2), (3,4), (5,6) from the coset's pair table, token 7.
+                // The pair entries carry the same value fields as token entries, so bits 11 and
+                // 12 of the XOR of all seven fields are again c and the parity p of y0..y6
+                const uint32_t e0 = step<SMEM, ACT>(L, act, lut);
+                const uint32_t lutp = lut + kPairTabOff + ((e0 & 0x800u) << 4);  // pair table of c
+                uint32_t h0 = step2<SMEM, ACT>(L, act, lutp);
+                uint32_t h1 = step2<SMEM, ACT>(L, act, lutp);
+                uint32_t h2 = step2<SMEM, ACT>(L, act, lutp);
+                if (__any_sync(0xffffffffu, (h0 | h1 | h2) >> 31)) {
+                    const uint32_t c = (e0 >> 11) & 1u, tf = lut + kTokFieldOff + 4u * kPairTokFields * c;
+                    h0 = resolve_pair(p, h0, c, tf, L, rb, err);
+                    h1 = resolve_pair(p, h1, c, tf, L, rb, err);
+                    h2 = resolve_pair(p, h2, c, tf, L, rb, err);
+                }
+                const uint32_t H = h0 ^ h1 ^ h2;
+                Y = (e0 ^ H ^ (H >> 10)) & 0x1800u;
+                // context 3 + 2c + p sits at table position 1 + c + 2p
+                const uint32_t e7 = step<SMEM, ACT>(L, act, lut + kSlotBytes + (Y << 2));
+                F[0] = (e0 & (kFieldMask | kEscBit)) | kMagic;
+                F[1] = (h0 & (kFieldMask | kEscBit)) | kMagic;
+                F[2] = ((h0 >> 10) & (kFieldMask | kEscBit)) | kMagic;
+                F[3] = (h1 & (kFieldMask | kEscBit)) | kMagic;
+                F[4] = ((h1 >> 10) & (kFieldMask | kEscBit)) | kMagic;
+                F[5] = (h2 & (kFieldMask | kEscBit)) | kMagic;
+                F[6] = ((h2 >> 10) & (kFieldMask | kEscBit)) | kMagic;
+                F[7] = (e7 & (kFieldMask | kEscBit)) | kMagic;
             } else {
-                Y = (e[0] ^ e[1] ^ e[2] ^ e[3] ^ e[4] ^ e[5] ^ e[6]) & 0x1800u;
+                uint32_t e[8];
+                // coordinate 0 (context 0); bit 11 of every entry of contexts 0..2 is the coset c
+                e[0] = step<SMEM, ACT>(L, act, lut);
+                uint32_t lutc = lut + kSlotBytes + ((e[0] & 0x800u) << 2);  // context 1 + c
+#pragma unroll
+                for (int i = 1; i < 7; ++i) e[i] = step<SMEM, ACT>(L, act, lutc);
+                // narrow tables: bits 11 and 12 of the XOR of entries 0..6 are c (seven copies) and
+                // the parity p of y0..y6.  Wide tables: bit 11 of entries 1..6 is the parity of y_i,
+                // so c is bit 11 of entry 0 and p is bit 12 of entry 0 xor bit 11 of the others' XOR.
+                // Context 3 + 2c + p sits at table position 3 + c + 2p
+                if constexpr (WIDE) {
+                    const uint32_t X1 = e[1] ^ e[2] ^ e[3] ^ e[4] ^ e[5] ^ e[6];
+                    Y = (e[0] & 0x800u) | ((e[0] ^ (X1 << 1)) & 0x1000u);
+                } else {
+                    Y = (e[0] ^ e[1] ^ e[2] ^ e[3] ^ e[4] ^ e[5] ^ e[6]) & 0x1800u;
+                }
+                uint32_t lut7 = lut + 3u * kSlotBytes + (Y << 2);
+                e[7] = step<SMEM, ACT>(L, act, lut7);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) F[i] = (e[i] & (kFieldMask | kEscBit)) | kMagic;
             }
             const uint32_t cbit = (Y >> 11) & 1u, pbit = (Y >> 12) & 1u;
-            uint32_t lut7 = lut + 3u * kSlotBytes + (Y << 2);
-            e[7] = step<SMEM, ACT>(L, act, lut7);
-            // F keeps the value field and the escape flag of each entry (the flag only matters for
-            // escapes, whose F is rebuilt), so the entries themselves die here
-            uint32_t F[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) F[i] = (e[i] & (kFieldMask | kEscBit)) | kMagic;
             uint32_t O = F[0] | F[1] | F[2] | F[3] | F[4] | F[5] | F[6] | F[7];
             if (__any_sync(0xffffffffu, O & kEscBit))
                 resolve_escapes<SMEM, WIDE>(p, F, cbit, pbit, L, rb);
@@ -515,7 +602,7 @@ done:
 
 // Decodes tile t with one warp.  `head` points at the tile (states, region lengths, word area):
 // a shared address (SMEM) or a global pointer.  Returns the EP_DEC_* bits of this lane.
-template <int DT, int ROWS, bool WIDE, bool SMEM, typename Ptr>
+template <int DT, int ROWS, int MODE, bool SMEM, typename Ptr>
 __device__ __forceinline__ uint32_t decode_tile(const Params &p, uint32_t lut, Ptr head, uint32_t tile_bytes,
                                                 uint32_t t, uint32_t lane) {
     Lane<SMEM> L;
@@ -546,18 +633,18 @@ __device__ __forceinline__ uint32_t decode_tile(const Params &p, uint32_t lut, P
         L.w = lds16(L.wp);
         uint32_t wlim = L.area + 2u * capacity;
         if (uint64_t(t + 1) * 32u * p.K <= p.nb)
-            err = decode_blocks<DT, SMEM, false, ROWS, WIDE>(p, L, rb, lut, wlim, t, lane);
+            err = decode_blocks<DT, SMEM, false, ROWS, MODE>(p, L, rb, lut, wlim, t, lane);
         else
-            err = decode_blocks<DT, SMEM, true, ROWS, WIDE>(p, L, rb, lut, wlim, t, lane);
+            err = decode_blocks<DT, SMEM, true, ROWS, MODE>(p, L, rb, lut, wlim, t, lane);
     } else {
         L.area = reinterpret_cast<const uint16_t *>(head + kTileHead);
         L.wlim = L.area + (capacity ? capacity - 1u : 0u);
         L.wp = L.area + start < L.wlim ? L.area + start : L.wlim;
         L.w = __ldg(L.wp);
         if (uint64_t(t + 1) * 32u * p.K <= p.nb)
-            err = decode_blocks<DT, SMEM, false, ROWS, WIDE>(p, L, rb, lut, L.wlim, t, lane);
+            err = decode_blocks<DT, SMEM, false, ROWS, MODE>(p, L, rb, lut, L.wlim, t, lane);
         else
-            err = decode_blocks<DT, SMEM, true, ROWS, WIDE>(p, L, rb, lut, L.wlim, t, lane);
+            err = decode_blocks<DT, SMEM, true, ROWS, MODE>(p, L, rb, lut, L.wlim, t, lane);
     }
     if (L.x != kStateLow) err |= EP_DEC_BAD_END;
     // the front (rANS words) and the back (raw bits) cover the region exactly
@@ -596,25 +683,51 @@ __device__ __forceinline__ uint32_t token_head(uint32_t c, uint32_t t, uint32_t 
 
 // ------------------------------------------------------------------ ep_prepare: the slot tables
 // One CTA per (context, 256 slots): the context's frequencies and their prefix sums in shared
-// memory, then each thread finds the token of its slot by binary search.  Runs once per stream;
-// the decode kernel copies the 56 KB result into every CTA's shared memory.
+// memory, then each thread finds the symbol of its slot by binary search.  Runs once per stream;
+// the decode kernel copies the result (56 KB; a paired stream's 106 KB) into every CTA's
+// shared memory.  Grid: 7 contexts x 8 CTAs; paired streams: contexts 0, 3..6 x 8 CTAs, then
+// the pair tables of contexts 1, 2 x 16 CTAs (4096 slots each).
 struct PrepParams {
     const uint16_t *freq;    // frequency tables, contexts in order
-    uint32_t *tables;        // kContexts x 2048 entries
+    uint32_t *tables;        // the decoder's tables (kLutBytes, or kPairedTableBytes when paired)
     uint32_t *status;        // nullable
     uint32_t splits;
-    uint32_t wide;  // value fields hold y for coordinates 1..7
+    uint32_t wide;           // value fields hold y for coordinates 1..7
+    uint32_t paired;
+    uint32_t ntok[kContexts];
     uint32_t tab_off[kContexts + 1];
 };
 
 constexpr uint32_t kPrepThreads = 256;
+constexpr uint32_t kPrepSingleCtas = kProbScale / kPrepThreads;  // 8 per token table
+constexpr uint32_t kPrepPairCtas = kPairScale / kPrepThreads;    // 16 per pair table
+
+// value field and escape flag (bits 11..20) of token t of context c
+__device__ __forceinline__ uint32_t token_field(uint32_t c, uint32_t t, uint32_t m, bool wide) {
+    return token_head(c, t, 0u, m, wide) & (kFieldMask | kEscBit);
+}
 
 __global__ void __launch_bounds__(kPrepThreads) prepare_kernel(const __grid_constant__ PrepParams p) {
-    __shared__ uint32_t cum[kMaxAlphabet + 1];
+    __shared__ uint32_t cum[kPairMaxTable + 1];
     __shared__ uint32_t part[kPrepThreads / 32];
-    const uint32_t c = blockIdx.x / (kProbScale / kPrepThreads);
-    const uint32_t slot = (blockIdx.x % (kProbScale / kPrepThreads)) * kPrepThreads + threadIdx.x;
-    const uint32_t n = min(p.tab_off[c + 1] - p.tab_off[c], kMaxAlphabet);
+    uint32_t c, slot0;
+    bool pair = false;
+    if (!p.paired) {
+        c = blockIdx.x / kPrepSingleCtas;
+        slot0 = (blockIdx.x % kPrepSingleCtas) * kPrepThreads;
+    } else if (blockIdx.x < 5 * kPrepSingleCtas) {
+        const uint32_t i = blockIdx.x / kPrepSingleCtas;
+        c = i == 0 ? 0u : i + 2u;
+        slot0 = (blockIdx.x % kPrepSingleCtas) * kPrepThreads;
+    } else {
+        const uint32_t j = blockIdx.x - 5 * kPrepSingleCtas;
+        c = 1u + j / kPrepPairCtas;
+        slot0 = (j % kPrepPairCtas) * kPrepThreads;
+        pair = true;
+    }
+    const uint32_t M = pair ? kPairScale : kProbScale;
+    const uint32_t slot = slot0 + threadIdx.x;
+    const uint32_t n = min(p.tab_off[c + 1] - p.tab_off[c], pair ? kPairMaxTable : kMaxAlphabet);
     const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
     // exclusive prefix sums of the (clamped) frequencies, 256 at a time
     uint32_t run = 0;
@@ -622,8 +735,8 @@ __global__ void __launch_bounds__(kPrepThreads) prepare_kernel(const __grid_cons
     for (uint32_t base = 0; base < n; base += kPrepThreads) {
         uint32_t t = base + threadIdx.x;
         uint32_t f = t < n ? uint32_t(p.freq[p.tab_off[c] + t]) : 0u;
-        bad |= f >= kProbScale;
-        f = min(f, kProbScale);
+        bad |= f >= M;
+        f = min(f, M);
         uint32_t incl = f;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
@@ -643,12 +756,11 @@ __global__ void __launch_bounds__(kPrepThreads) prepare_kernel(const __grid_cons
     }
     if (threadIdx.x == 0) cum[n] = run;
     __syncthreads();
-    if (p.status && blockIdx.x % (kProbScale / kPrepThreads) == 0 && threadIdx.x == 0 && n && run != kProbScale)
-        atomicOr(p.status, EP_DEC_BAD_TOKEN);
+    if (p.status && slot0 == 0 && threadIdx.x == 0 && n && run != M) atomicOr(p.status, EP_DEC_BAD_TOKEN);
     if (p.status && __syncthreads_or(bad) && threadIdx.x == 0) atomicOr(p.status, EP_DEC_BAD_TOKEN);
-    uint32_t e = 0;
+    // the last symbol s with cum[s] <= slot (symbols with f = 0 are skipped)
+    uint32_t sym = 0, f = 0;
     if (n) {
-        // the last token t with cum[t] <= slot (tokens with f = 0 are skipped)
         uint32_t lo = 0, hi = n;  // cum[lo] <= slot < cum[hi] (cum[n] may be short if damaged)
         while (hi - lo > 1) {
             uint32_t mid = (lo + hi) >> 1;
@@ -657,23 +769,44 @@ __global__ void __launch_bounds__(kPrepThreads) prepare_kernel(const __grid_cons
             else
                 hi = mid;
         }
-        uint32_t f = cum[lo + 1] - cum[lo];
-        e = token_head(c, lo, f, split_of_bits(p.splits, c), p.wide != 0) | ((slot - cum[lo]) & (kProbScale - 1u));
+        sym = lo;
+        f = cum[lo + 1] - cum[lo];
     }
-    // context 3 + 2c + p is stored at position 3 + c + 2p (the decoder forms that offset from
-    // the XOR of a block's first seven entries)
-    uint32_t pos = c < 3 ? c : 3u + ((c - 3u) >> 1) + 2u * ((c - 3u) & 1u);
-    p.tables[pos * kProbScale + slot] = e;
+    const uint32_t m = split_of_bits(p.splits, c);
+    if (!pair) {
+        uint32_t e = n ? token_head(c, sym, f, m, p.wide != 0) | ((slot - cum[sym]) & (kProbScale - 1u)) : 0u;
+        // context 3 + 2c + p is stored at position 3 + c + 2p (1 + c + 2p in a paired stream's
+        // tables); the decoder forms that offset from the XOR of a block's first seven fields
+        const uint32_t first = p.paired ? 1u : 3u;
+        uint32_t pos = c < 3 ? c : first + ((c - 3u) >> 1) + 2u * ((c - 3u) & 1u);
+        p.tables[pos * kProbScale + slot] = e;
+    } else {
+        // pair entry: frequency and slot offset, then the fields of tokens (t_a, t_b) = (s / B, s % B)
+        // or bit 31 for the escape symbol s = B * B (B = min(A, 40))
+        const uint32_t A = p.ntok[c], B = min(A, kPairBaseMax);
+        uint32_t lo = 0, hi = 0;
+        if (n) {
+            lo = (min(f, kPairScale - 1u) << 20) | ((slot - cum[sym]) & (kPairScale - 1u));
+            hi = sym >= B * B ? (1u << 31)
+                              : token_field(c, sym / B, m, false) | (token_field(c, sym % B, m, false) << 10);
+        }
+        uint32_t *dst = p.tables + (kPairTabOff + (c - 1u) * kPairTabBytes) / 4u + 2u * slot;
+        dst[0] = lo;
+        dst[1] = hi;
+        if (slot < kPairTokFields)
+            p.tables[kTokFieldOff / 4u + (c - 1u) * kPairTokFields + slot] = slot < A ? token_field(c, slot, m, false) : 0u;
+    }
 }
 
 // ------------------------------------------------------------------ decode kernel
 // Shared memory: the slot tables, mbarriers, then nbuf tile buffers per warp.
-template <int DT, int ROWS, bool WIDE>
+template <int DT, int ROWS, int MODE>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(128) uint8_t smem[];
+    constexpr uint32_t kTables = uint32_t(MODE == kPaired ? kPairedTableBytes : kLutBytes);
     const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     const uint32_t lut = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-    const uint32_t bars = lut + uint32_t(kLutBytes);
+    const uint32_t bars = lut + kTables;
     const uint32_t tbar = bars + uint32_t(kMaxWarps) * 16u;  // the tables' mbarrier
     const uint32_t nbuf = p.nbuf;
     const uint32_t bufs = bars + uint32_t(kBarBytes) + warp * (nbuf ? nbuf : 1u) * p.tile_buf;
@@ -694,8 +827,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
-        mbar_expect(tbar, uint32_t(kLutBytes));
-        bulk_g2s(lut, p.tables, uint32_t(kLutBytes), tbar);
+        mbar_expect(tbar, kTables);
+        bulk_g2s(lut, p.tables, kTables, tbar);
     }
     __syncthreads();
 
@@ -744,9 +877,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_
                 if (nbuf > 1 && (pend & (1u << o))) mbar_wait(bars + 16u * warp + 8u * o, (phase >> o) & 1u);
                 return;
             }
-            if (tables_ok) err = decode_tile<DT, ROWS, WIDE, true>(p, lut, bufs + b * p.tile_buf, bytes, t, lane);
+            if (tables_ok) err = decode_tile<DT, ROWS, MODE, true>(p, lut, bufs + b * p.tile_buf, bytes, t, lane);
         } else if (tables_ok) {
-            err = decode_tile<DT, ROWS, WIDE, false>(p, lut, p.tiles + size_t(beg) * 16, bytes, t, lane);
+            err = decode_tile<DT, ROWS, MODE, false>(p, lut, p.tiles + size_t(beg) * 16, bytes, t, lane);
         }
         if (err && p.status) atomicOr(p.status, err);
         __syncwarp();
@@ -764,7 +897,7 @@ struct DeviceCache {
 DeviceCache g_cache;
 
 template <int DT>
-cudaError_t launch(Params &p, uint64_t max_tile, bool wide, int device, cudaStream_t stream) {
+cudaError_t launch(Params &p, uint64_t max_tile, int mode, int device, cudaStream_t stream) {
     int sms;
     {
         std::lock_guard<std::mutex> g(g_cache.mu);
@@ -775,9 +908,11 @@ cudaError_t launch(Params &p, uint64_t max_tile, bool wide, int device, cudaStre
         }
         if (!g_cache.attr[device][DT]) {
             cudaError_t e = cudaSuccess;
-            for (auto k : {decode_kernel<DT, kRowsAny, false>, decode_kernel<DT, kRows32, false>,
-                           decode_kernel<DT, kRowsPadded, false>, decode_kernel<DT, kRowsAny, true>,
-                           decode_kernel<DT, kRows32, true>, decode_kernel<DT, kRowsPadded, true>})
+            for (auto k : {decode_kernel<DT, kRowsAny, kNarrow>, decode_kernel<DT, kRows32, kNarrow>,
+                           decode_kernel<DT, kRowsPadded, kNarrow>, decode_kernel<DT, kRowsAny, kWide>,
+                           decode_kernel<DT, kRows32, kWide>, decode_kernel<DT, kRowsPadded, kWide>,
+                           decode_kernel<DT, kRowsAny, kPaired>, decode_kernel<DT, kRows32, kPaired>,
+                           decode_kernel<DT, kRowsPadded, kPaired>})
                 if (e == cudaSuccess)
                     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemLimit));
             if (e != cudaSuccess) return e;
@@ -791,7 +926,8 @@ cudaError_t launch(Params &p, uint64_t max_tile, bool wide, int device, cudaStre
     uint32_t grid = p.T < uint32_t(sms) ? p.T : uint32_t(sms);
     uint32_t warps = (p.T + grid - 1) / grid;
     warps = warps > uint32_t(kMaxWarps) ? uint32_t(kMaxWarps) : warps;
-    const size_t avail = kSmemLimit - kFixedBytes;
+    const size_t fixed = mode == kPaired ? kPairedFixedBytes : kFixedBytes;
+    const size_t avail = kSmemLimit - fixed;
     p.tile_buf = uint32_t((max_tile + kSlack + 15) & ~uint64_t(15));
     bool many = p.T > grid * warps;  // some warp decodes more than one tile
     if (many && 2ull * warps * p.tile_buf <= avail) {
@@ -809,7 +945,7 @@ cudaError_t launch(Params &p, uint64_t max_tile, bool wide, int device, cudaStre
         p.tile_buf = 16;
     }
     if (warps < 1) warps = 1;
-    size_t smem = kFixedBytes + size_t(warps) * (p.nbuf ? p.nbuf : 1) * p.tile_buf;
+    size_t smem = fixed + size_t(warps) * (p.nbuf ? p.nbuf : 1) * p.tile_buf;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(warps * 32);
@@ -820,14 +956,19 @@ cudaError_t launch(Params &p, uint64_t max_tile, bool wide, int device, cudaStre
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (wide) {
-        if (p.cols & 7u) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsPadded, true>, p);
-        if ((p.cb & 31u) == 0) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRows32, true>, p);
-        return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsAny, true>, p);
+    if (mode == kPaired) {
+        if (p.cols & 7u) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsPadded, kPaired>, p);
+        if ((p.cb & 31u) == 0) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRows32, kPaired>, p);
+        return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsAny, kPaired>, p);
     }
-    if (p.cols & 7u) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsPadded, false>, p);
-    if ((p.cb & 31u) == 0) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRows32, false>, p);
-    return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsAny, false>, p);
+    if (mode == kWide) {
+        if (p.cols & 7u) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsPadded, kWide>, p);
+        if ((p.cb & 31u) == 0) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRows32, kWide>, p);
+        return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsAny, kWide>, p);
+    }
+    if (p.cols & 7u) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsPadded, kNarrow>, p);
+    if ((p.cb & 31u) == 0) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRows32, kNarrow>, p);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsAny, kNarrow>, p);
 }
 
 int check_info(const ep_info *info) {
@@ -835,11 +976,18 @@ int check_info(const ep_info *info) {
     const int64_t cb = (info->cols + 7) / 8;  // rows zero-padded to whole E8 blocks
     if (info->rows >= (int64_t(1) << 31) || cb >= (int64_t(1) << 31) || info->rows * cb >= (int64_t(1) << 31))
         return EP_ERR_UNSUPPORTED;
+    if (info->paired > 1) return EP_ERR_CORRUPT;
     uint32_t total = 0;
     for (int c = 0; c < kContexts; ++c) {
         if (!split_valid(info->split[c], c) || info->ntok[c] > split_alphabet(info->split[c], kCtxLow[c]))
             return EP_ERR_CORRUPT;
-        total += info->ntok[c];
+        if (info->paired && info->split[c] > kCtxNarrowSplit[c]) return EP_ERR_CORRUPT;
+        if (info->paired && (c == 1 || c == 2)) {
+            if (info->split[c] > kPairMaxSplit) return EP_ERR_CORRUPT;
+            total += pair_table_len(info->ntok[c]);
+        } else {
+            total += info->ntok[c];
+        }
     }
     if (info->off_freq + 2ull * total > info->off_dir) return EP_ERR_CORRUPT;
     return EP_OK;
@@ -859,6 +1007,8 @@ bool wide_fields(const ep_info *info) {
         if (info->split[c] > kCtxNarrowSplit[c]) return true;
     return false;
 }
+
+int coding_of(const ep_info *info) { return info->paired ? kPaired : wide_fields(info) ? kWide : kNarrow; }
 
 uint32_t pack_splits(const ep_info *info) {
     uint32_t s = 0;
@@ -883,10 +1033,15 @@ extern "C" int ep_prepare(const ep_info *info, const void *d_blob, void *d_works
     q.status = d_status;
     q.splits = pack_splits(info);
     q.wide = wide_fields(info) ? 1u : 0u;
+    q.paired = info->paired ? 1u : 0u;
     q.tab_off[0] = 0;
-    for (int c = 0; c < kContexts; ++c) q.tab_off[c + 1] = q.tab_off[c] + info->ntok[c];
-    prepare_kernel<<<kContexts * (kProbScale / kPrepThreads), kPrepThreads, 0,
-                     reinterpret_cast<cudaStream_t>(stream)>>>(q);
+    for (int c = 0; c < kContexts; ++c) {
+        q.ntok[c] = info->ntok[c];
+        const bool pair = info->paired && (c == 1 || c == 2);
+        q.tab_off[c + 1] = q.tab_off[c] + (pair ? pair_table_len(info->ntok[c]) : info->ntok[c]);
+    }
+    const uint32_t grid = info->paired ? 5 * kPrepSingleCtas + 2 * kPrepPairCtas : kContexts * kPrepSingleCtas;
+    prepare_kernel<<<grid, kPrepThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(q);
     return cudaGetLastError() == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 
@@ -916,19 +1071,23 @@ extern "C" int ep_decompress(const ep_info *info, const void *d_blob, const void
     p.K = info->blocks_per_lane;
     p.T = info->n_tiles;
     p.splits = pack_splits(info);
+    for (int c = 0; c < 2; ++c) {
+        p.pair_A[c] = info->paired ? info->ntok[1 + c] : 0u;
+        p.pair_rawb[c] = pair_raw_bits(p.pair_A[c]);
+    }
     int device;
     cudaError_t e = cudaGetDevice(&device);
     if (e != cudaSuccess) return EP_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint64_t mt = info->max_tile_nbytes;
-    const bool wide = wide_fields(info);
+    const int mode = coding_of(info);
     switch (out_dtype) {
-    case EP_BF16: e = launch<EP_BF16>(p, mt, wide, device, s); break;
-    case EP_FP16: e = launch<EP_FP16>(p, mt, wide, device, s); break;
-    case EP_FP32: e = launch<EP_FP32>(p, mt, wide, device, s); break;
-    case EP_INT8: e = launch<EP_INT8>(p, mt, wide, device, s); break;
-    case EP_FP8_E4M3: e = launch<EP_FP8_E4M3>(p, mt, wide, device, s); break;
-    case EP_LATTICE_I32: e = launch<EP_LATTICE_I32>(p, mt, wide, device, s); break;
+    case EP_BF16: e = launch<EP_BF16>(p, mt, mode, device, s); break;
+    case EP_FP16: e = launch<EP_FP16>(p, mt, mode, device, s); break;
+    case EP_FP32: e = launch<EP_FP32>(p, mt, mode, device, s); break;
+    case EP_INT8: e = launch<EP_INT8>(p, mt, mode, device, s); break;
+    case EP_FP8_E4M3: e = launch<EP_FP8_E4M3>(p, mt, mode, device, s); break;
+    case EP_LATTICE_I32: e = launch<EP_LATTICE_I32>(p, mt, mode, device, s); break;
     default: return EP_ERR_INVALID_ARG;
     }
     return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
@@ -937,11 +1096,11 @@ extern "C" int ep_decompress(const ep_info *info, const void *d_blob, const void
 // ------------------------------------------------------------------ ep_decompress_noalloc
 // The same decode for callers that cannot allocate device memory: the slot tables live in one
 // file-scope device array instead of a caller workspace.  Every GPU that loads the library holds
-// this array (56 KB) until the process exits; all calls on a device share it.
+// this array (106 KB) until the process exits; all calls on a device share it.
 namespace ep {
 namespace {
 
-constexpr size_t kStaticTablesBytes = kLutBytes;  // the largest workspace a stream can need
+constexpr size_t kStaticTablesBytes = kPairedTableBytes;  // the largest workspace a stream can need
 static __device__ __align__(256) uint32_t g_static_tables[kStaticTablesBytes / 4];
 
 struct StaticTables {

@@ -12,6 +12,8 @@
 //                      histogram of the values' bit lengths per context;
 //   * token_kernel     per coordinate: its token at the chosen splits, token counts per context
 //                      and the raw extra bits;
+//   * pair_kernel      per block of a paired stream: counts of the token pairs of coordinates
+//                      (1,2), (3,4), (5,6);
 //   * lane_kernel      one thread per (tile, lane), twice: the lane's rANS encode (tokens in
 //                      reverse) and raw bits, first counting words, then writing them in decode
 //                      order into the lane's region of the tile.
@@ -34,6 +36,9 @@ namespace ep {
 namespace {
 
 constexpr int kLenBins = 33;  // bit lengths 0..32
+// frequency tables as the lane kernel holds them: one row per context, long enough for a pair table
+constexpr uint32_t kTableStride = kPairMaxTable > kMaxAlphabet ? kPairMaxTable : kMaxAlphabet;
+constexpr uint32_t kPairBins = kPairBaseMax * kPairBaseMax;
 
 struct DevSrc {
     const void *p;
@@ -185,6 +190,27 @@ __global__ void token_kernel(const uint8_t *ctx, const uint32_t *val, int64_t n,
         if (h[i]) atomicAdd(&cnt[i], (unsigned long long)h[i]);
 }
 
+// counts of the token pairs inside the bases of contexts 1 and 2 (B1 x B1 and B2 x B2 bins at
+// offsets 0 and kPairBins)
+__global__ void pair_kernel(const uint8_t *ctx, const uint32_t *val, int64_t nb, Splits sp, uint32_t B1, uint32_t B2,
+                            unsigned long long *pc) {
+    __shared__ unsigned int h[2 * kPairBins];
+    for (int i = threadIdx.x; i < int(2 * kPairBins); i += blockDim.x) h[i] = 0;
+    __syncthreads();
+    for (int64_t b = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; b < nb; b += int64_t(gridDim.x) * blockDim.x) {
+        const uint32_t c = ctx[8 * b + 1];  // 1 or 2
+        const uint32_t B = c == 1 ? B1 : B2;
+        for (int j = 0; j < 3; ++j) {
+            const uint32_t ta = token_of(val[8 * b + 1 + 2 * j], sp.m[c], 1).tok;
+            const uint32_t tb = token_of(val[8 * b + 2 + 2 * j], sp.m[c], 1).tok;
+            if (ta < B && tb < B) atomicAdd(&h[(c - 1) * kPairBins + ta * B + tb], 1u);
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < int(2 * kPairBins); i += blockDim.x)
+        if (h[i]) atomicAdd(&pc[i], (unsigned long long)h[i]);
+}
+
 // ------------------------------------------------------------------ lanes
 // One thread per (tile, lane); a warp is a tile.  Lane l of tile t codes blocks t 32 K + 32 k + l.
 // Its region holds the rANS words in decode order, then its raw extra bits packed least
@@ -193,8 +219,8 @@ __global__ void token_kernel(const uint8_t *ctx, const uint32_t *val, int64_t n,
 struct LaneArgs {
     const uint8_t *ctx;
     const uint32_t *val;
-    const uint16_t *freq;   // kContexts x kMaxAlphabet
-    const uint16_t *cum;    // kContexts x kMaxAlphabet
+    const uint16_t *freq;   // kContexts x kTableStride (paired contexts 1, 2: the pair tables)
+    const uint16_t *cum;    // kContexts x kTableStride
     uint32_t *count;        // T x 32: words of each lane's region
     uint32_t *rwords;       // T x 32: of which rANS words
     uint32_t *state;        // T x 32: final encoder state (the decoder's initial state)
@@ -204,12 +230,53 @@ struct LaneArgs {
     int64_t nb;
     uint32_t K, T;
     Splits sp;
+    uint32_t paired;
+    uint32_t B[kContexts];     // paired contexts 1, 2: pair base min(A, 40)
+    uint32_t rawb[kContexts];  // paired contexts 1, 2: raw bits of one token of an escaped pair
 };
+
+// A block's rANS symbols in decode order (context row, symbol, table bits) and, through `push`,
+// its raw bits: single coding, the 8 tokens; paired coding, token 0, the three pair symbols
+// (a pair with a token outside the base B, or whose table entry is 0, is the escape B * B) and
+// token 7, the escaped pairs' tokens leading the raw bits.  Returns the symbol count.
+struct Sym {
+    uint32_t c, s, bits;
+};
+template <typename Push>
+__device__ __forceinline__ int block_syms(const LaneArgs &a, const uint16_t *sf, int64_t b, Sym *sym, Push push) {
+    Token tk[8];
+    uint32_t cx[8];
+    for (int i = 0; i < 8; ++i) {
+        cx[i] = a.ctx[8 * b + i];
+        tk[i] = token_of(a.val[8 * b + i], a.sp.m[cx[i]], low_of(cx[i]));
+    }
+    int n = 0;
+    if (!a.paired) {
+        for (int i = 0; i < 8; ++i) sym[n++] = {cx[i], tk[i].tok, kProbBits};
+    } else {
+        const uint32_t pc = cx[1], B = a.B[pc];
+        bool esc[3];
+        sym[n++] = {cx[0], tk[0].tok, kProbBits};
+        for (int j = 0; j < 3; ++j) {
+            const uint32_t ta = tk[1 + 2 * j].tok, tb = tk[2 + 2 * j].tok;
+            esc[j] = ta >= B || tb >= B || sf[pc * kTableStride + ta * B + tb] == 0;
+            sym[n++] = {pc, esc[j] ? B * B : ta * B + tb, kPairBits};
+        }
+        sym[n++] = {cx[7], tk[7].tok, kProbBits};
+        for (int j = 0; j < 3; ++j)
+            if (esc[j]) {
+                push(tk[1 + 2 * j].tok, a.rawb[pc]);
+                push(tk[2 + 2 * j].tok, a.rawb[pc]);
+            }
+    }
+    for (int i = 0; i < 8; ++i) push(tk[i].extra, tk[i].nbits);
+    return n;
+}
 
 template <bool WRITE>
 __global__ void lane_kernel(LaneArgs a) {
-    __shared__ uint16_t sf[kContexts * kMaxAlphabet], sc[kContexts * kMaxAlphabet];
-    for (int i = threadIdx.x; i < kContexts * int(kMaxAlphabet); i += blockDim.x) {
+    __shared__ uint16_t sf[kContexts * kTableStride], sc[kContexts * kTableStride];
+    for (int i = threadIdx.x; i < kContexts * int(kTableStride); i += blockDim.x) {
         sf[i] = a.freq[i];
         sc[i] = a.cum[i];
     }
@@ -240,42 +307,39 @@ __global__ void lane_kernel(LaneArgs a) {
         tile[4 * 32 + 2 * lane + 1] = uint8_t(n >> 8);
         area = reinterpret_cast<uint16_t *>(tile + kTileHead);
     }
-    // raw extra bits, forward
+    // raw bits, forward
     uint64_t acc = 0;
     uint32_t nacc = 0, raw = 0;
-    for (uint32_t k = 0; k < nk; ++k) {
-        const int64_t b = first + int64_t(k) * 32 + lane;
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t c = a.ctx[8 * b + i];
-            const Token tk = token_of(a.val[8 * b + i], a.sp.m[c], low_of(c));
-            acc |= uint64_t(tk.extra) << nacc;
-            nacc += tk.nbits;
-            while (nacc >= 16) {
-                if (WRITE) area[start + n - 1 - raw] = uint16_t(acc);
-                ++raw;
-                acc >>= 16;
-                nacc -= 16;
-            }
+    auto push = [&](uint32_t v, uint32_t nbits) {
+        acc |= uint64_t(v) << nacc;
+        nacc += nbits;
+        while (nacc >= 16) {
+            if (WRITE) area[start + n - 1 - raw] = uint16_t(acc);
+            ++raw;
+            acc >>= 16;
+            nacc -= 16;
         }
-    }
+    };
+    auto skip = [](uint32_t, uint32_t) {};
+    Sym sym[8];
+    for (uint32_t k = 0; k < nk; ++k) block_syms(a, sf, first + int64_t(k) * 32 + lane, sym, push);
     if (nacc) {
         if (WRITE) area[start + n - 1 - raw] = uint16_t(acc);
         ++raw;
     }
-    // rANS, tokens in reverse; the i-th word emitted is word nr - 1 - i in decode order
+    // rANS, symbols in reverse; the i-th word emitted is word nr - 1 - i in decode order
     uint32_t x = kStateLow, emitted = 0;
     for (uint32_t k = nk; k-- > 0;) {
-        const int64_t b = first + int64_t(k) * 32 + lane;
-        for (int i = 7; i >= 0; --i) {
-            const uint32_t c = a.ctx[8 * b + i];
-            const Token tk = token_of(a.val[8 * b + i], a.sp.m[c], low_of(c));
-            const uint32_t f = sf[c * kMaxAlphabet + tk.tok], cu = sc[c * kMaxAlphabet + tk.tok];
-            if (uint64_t(x) >= (uint64_t(f) << (32 - kProbBits))) {  // keep the next state below 2^32
+        const int ns = block_syms(a, sf, first + int64_t(k) * 32 + lane, sym, skip);
+        for (int i = ns - 1; i >= 0; --i) {
+            const uint32_t at = sym[i].c * kTableStride + sym[i].s, nbits = sym[i].bits;
+            const uint32_t f = sf[at], cu = sc[at];
+            if (uint64_t(x) >= (uint64_t(f) << (32 - nbits))) {  // keep the next state below 2^32
                 if (WRITE) area[start + nr - 1 - emitted] = uint16_t(x);
                 ++emitted;
                 x >>= 16;
             }
-            x = (x / f) * kProbScale + (x % f) + cu;
+            x = (x / f) * (1u << nbits) + (x % f) + cu;
         }
     }
     if (!WRITE) {
@@ -300,7 +364,7 @@ struct Scratch {
     float *codes, *scales, *rms;
     uint8_t *ctx;
     uint32_t *val;
-    unsigned long long *by_len, *cnt, *extra;
+    unsigned long long *by_len, *cnt, *extra, *pairs;
     uint32_t *bad, *too_long;
     uint16_t *freq, *cum;
     uint32_t *count, *rwords, *state, *dir;
@@ -323,10 +387,11 @@ Scratch carve(uint8_t *base, int64_t rows, int64_t cols, int container, int64_t 
     S.by_len = reinterpret_cast<unsigned long long *>(take(kContexts * kLenBins * 8));
     S.cnt = reinterpret_cast<unsigned long long *>(take(kContexts * kMaxAlphabet * 8));
     S.extra = reinterpret_cast<unsigned long long *>(take(8));
+    S.pairs = reinterpret_cast<unsigned long long *>(take(2 * kPairBins * 8));
     S.bad = reinterpret_cast<uint32_t *>(take(4));
     S.too_long = reinterpret_cast<uint32_t *>(take(4));
-    S.freq = reinterpret_cast<uint16_t *>(take(kContexts * kMaxAlphabet * 2));
-    S.cum = reinterpret_cast<uint16_t *>(take(kContexts * kMaxAlphabet * 2));
+    S.freq = reinterpret_cast<uint16_t *>(take(kContexts * kTableStride * 2));
+    S.cum = reinterpret_cast<uint16_t *>(take(kContexts * kTableStride * 2));
     S.count = reinterpret_cast<uint32_t *>(take(size_t(T) * 32 * 4));
     S.rwords = reinterpret_cast<uint32_t *>(take(size_t(T) * 32 * 4));
     S.state = reinterpret_cast<uint32_t *>(take(size_t(T) * 32 * 4));
@@ -338,7 +403,7 @@ Scratch carve(uint8_t *base, int64_t rows, int64_t cols, int container, int64_t 
 
 struct Plan {
     int64_t rows, cols, cb, nb;
-    int src_dt, container;
+    int src_dt, container, coding;
     uint32_t K, T;
     bool ok;
 };
@@ -351,6 +416,7 @@ Plan plan_of(int64_t rows, int64_t cols, int32_t src_dtype, const ep_config *cfg
     P.nb = rows * P.cb;
     P.src_dt = src_dtype;
     P.container = cfg->container_dtype ? cfg->container_dtype : src_dtype;
+    P.coding = cfg->coding;
     P.K = cfg->blocks_per_lane ? cfg->blocks_per_lane : auto_blocks_per_lane(P.nb, cfg->target_bpp);
     P.T = P.K ? uint32_t((P.nb + 32 * int64_t(P.K) - 1) / (32 * int64_t(P.K))) : 0;
     P.ok = P.K > 0;
@@ -422,7 +488,7 @@ struct Run {
         Splits sp = quantize(k, step, ns);
         std::vector<uint64_t> cnt[kContexts];
         uint64_t extra = tokens(sp, ns, cnt);
-        return estimate_from_counts(cnt, extra, P.nb, ns, P.rows, P.cols, P.container, P.T);
+        return estimate_from_counts(cnt, sp.m, P.coding, extra, P.nb, ns, P.rows, P.cols, P.container, P.T);
     }
 };
 
@@ -449,6 +515,7 @@ extern "C" int ep_compress_device(const void *d_src, int32_t src_dtype, int64_t 
     int container = cfg->container_dtype ? cfg->container_dtype : src_dtype;
     if (container < EP_BF16 || container > EP_FP8_E4M3) return EP_ERR_INVALID_ARG;
     if (cfg->blocks_per_lane > 4096) return EP_ERR_INVALID_ARG;
+    if (cfg->coding < EP_CODING_AUTO || cfg->coding > EP_CODING_PAIRED) return EP_ERR_INVALID_ARG;
     if ((rows * ((cols + 7) / 8)) >> 32) return EP_ERR_UNSUPPORTED;
     if (reinterpret_cast<uintptr_t>(d_scratch) & 255u || reinterpret_cast<uintptr_t>(d_out) & 15u)
         return EP_ERR_INVALID_ARG;
@@ -506,16 +573,40 @@ extern "C" int ep_compress_device(const void *d_src, int32_t src_dtype, int64_t 
         std::vector<uint64_t> cnt[kContexts];
         R.tokens(sp, P.nb, cnt);
         std::vector<uint32_t> freq[kContexts];
-        uint32_t ntok[kContexts];
+        std::vector<uint8_t> rare;
+        uint32_t ntok[kContexts], tablen[kContexts], A[kContexts] = {};
         uint64_t tokens = 0;
-        std::vector<uint16_t> hf(kContexts * kMaxAlphabet, 0), hc(kContexts * kMaxAlphabet, 0);
+        const bool paired = pair_eligible(P.coding, P.nb, sp.m);
+        std::vector<unsigned long long> pc;
+        if (paired) {
+            A[1] = seen_len(cnt[1]);
+            A[2] = seen_len(cnt[2]);
+            R.check(cudaMemsetAsync(R.S.pairs, 0, 2 * kPairBins * 8, R.st));
+            pair_kernel<<<R.blocks_for(P.nb, 256), 256, 0, R.st>>>(R.S.ctx, R.S.val, P.nb, sp, pair_base(A[1]),
+                                                                   pair_base(A[2]), R.S.pairs);
+            R.check(cudaGetLastError());
+            pc.resize(2 * kPairBins);
+            R.d2h(pc.data(), R.S.pairs, pc.size());
+        }
+        std::vector<uint16_t> hf(kContexts * kTableStride, 0), hc(kContexts * kTableStride, 0);
         for (int c = 0; c < kContexts; ++c) {
-            ntok[c] = build_freqs(cnt[c], freq[c]);
-            tokens += ntok[c];
+            if (paired && (c == 1 || c == 2)) {
+                std::vector<uint64_t> pair_cnt(size_t(pair_base(A[c])) * pair_base(A[c]));
+                for (size_t q = 0; q < pair_cnt.size(); ++q) pair_cnt[q] = pc[size_t(c - 1) * kPairBins + q];
+                uint64_t N = 0;  // every token of the context belongs to one of its pairs
+                for (uint64_t x : cnt[c]) N += x;
+                build_pair_table(pair_cnt, A[c], N / 2, freq[c], rare);
+                ntok[c] = A[c];
+                tablen[c] = pair_table_len(A[c]);
+            } else {
+                ntok[c] = build_freqs(cnt[c], freq[c]);
+                tablen[c] = ntok[c];
+            }
+            tokens += tablen[c];
             uint32_t a = 0;
-            for (size_t t = 0; t < freq[c].size(); ++t) {
-                hf[size_t(c) * kMaxAlphabet + t] = uint16_t(freq[c][t]);
-                hc[size_t(c) * kMaxAlphabet + t] = uint16_t(a);
+            for (size_t t = 0; t < tablen[c]; ++t) {
+                hf[size_t(c) * kTableStride + t] = uint16_t(freq[c][t]);
+                hc[size_t(c) * kTableStride + t] = uint16_t(a);
                 a += freq[c][t];
             }
         }
@@ -523,7 +614,11 @@ extern "C" int ep_compress_device(const void *d_src, int32_t src_dtype, int64_t 
         R.h2d(R.S.cum, hc.data(), hc.size());
         R.check(cudaMemsetAsync(R.S.too_long, 0, 4, R.st));
         LaneArgs la{R.S.ctx, R.S.val, R.S.freq, R.S.cum, R.S.count, R.S.rwords, R.S.state, R.S.too_long,
-                    R.S.dir, nullptr, P.nb, P.K, P.T, sp};
+                    R.S.dir, nullptr, P.nb, P.K, P.T, sp, paired ? 1u : 0u, {}, {}};
+        for (int c = 0; c < kContexts; ++c) {
+            la.B[c] = pair_base(A[c]);
+            la.rawb[c] = pair_raw_bits(A[c]);
+        }
         const int lane_blocks = int((uint64_t(P.T) * 32 + 255) / 256);
         lane_kernel<false><<<lane_blocks, 256, 0, R.st>>>(la);
         R.check(cudaGetLastError());
@@ -558,8 +653,8 @@ extern "C" int ep_compress_device(const void *d_src, int32_t src_dtype, int64_t 
         for (int64_t r = 0; r < rows; ++r) fac[size_t(r)] = factor_of(rms[size_t(r)], k);
         uint32_t mm[kContexts];
         for (int c = 0; c < kContexts; ++c) mm[c] = sp.m[c];
-        write_front(front.data(), L, src_dtype, container, rows, cols, P.T, P.K, k, mm, ntok, freq, fac.data(),
-                    scales.data());
+        write_front(front.data(), L, src_dtype, container, rows, cols, P.T, P.K, k, mm, ntok, tablen, paired, freq,
+                    fac.data(), scales.data());
         for (uint32_t t = 0; t <= P.T; ++t)
             for (int b = 0; b < 4; ++b) front[L.dir + 4 * t + b] = uint8_t(dir[t] >> (8 * b));
         uint8_t *out = static_cast<uint8_t *>(d_out);

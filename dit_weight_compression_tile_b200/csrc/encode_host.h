@@ -17,19 +17,33 @@ int max_q_index(int64_t cols);
 // of the values' bit lengths (by_len[0..32])
 uint32_t pick_split(const uint64_t *by_len, int ctx);
 
-// frequency table (sum 2^11, every entry below 2^11) from token counts; returns the table length
-uint32_t build_freqs(const std::vector<uint64_t> &cnt, std::vector<uint32_t> &f);
+// frequency table (sum `scale`, every entry below it) from counts; returns the table length
+uint32_t build_freqs(const std::vector<uint64_t> &cnt, std::vector<uint32_t> &f, uint32_t scale = kProbScale);
+
+// last token seen, plus one
+uint32_t seen_len(const std::vector<uint64_t> &cnt);
+
+// whether a stream pairs coordinates 1..6 (coding: EP_CODING_*; m: the splits)
+bool pair_eligible(int coding, int64_t nb, const uint32_t *m);
+
+// pair table of a context with alphabet length A from the counts of its token pairs inside the
+// base (B * B of them, B = pair_base(A)) and of all its pairs (N): pairs outside the base and rare
+// pairs go to the escape symbol B * B, then the table is normalised to 2^12; `rare` flags the
+// escaped pair indices inside the base
+void build_pair_table(std::vector<uint64_t> pair_cnt, uint32_t A, uint64_t N, std::vector<uint32_t> &f,
+                      std::vector<uint8_t> &rare);
 
 // bits per weight estimated from a sample of ns of the nb blocks: the sample's token counts per
-// context (at the splits picked on the sample) and its raw extra bits
-double estimate_from_counts(const std::vector<uint64_t> *cnt, uint64_t extra_bits, int64_t nb, int64_t ns,
-                            int64_t rows, int64_t cols, int container, uint32_t T);
+// context (at the splits m picked on the sample) and its raw extra bits
+double estimate_from_counts(const std::vector<uint64_t> *cnt, const uint32_t *m, int coding, uint64_t extra_bits,
+                            int64_t nb, int64_t ns, int64_t rows, int64_t cols, int container, uint32_t T);
 
 // header, row factors, code scales and frequency tables (everything before the directory);
-// `h` holds at least L.dir bytes, zeroed
+// `h` holds at least L.dir bytes, zeroed.  ntok: the header's per-context lengths; tablen: the
+// entries of freq[c] written (the pair tables' A * A + 1 for a paired stream's contexts 1, 2)
 void write_front(uint8_t *h, const Layout &L, int src_dt, int container, int64_t rows, int64_t cols, uint32_t T,
-                 uint32_t K, int k, const uint32_t *m, const uint32_t *ntok, const std::vector<uint32_t> *freq,
-                 const float *fac, const float *scales);
+                 uint32_t K, int k, const uint32_t *m, const uint32_t *ntok, const uint32_t *tablen, bool paired,
+                 const std::vector<uint32_t> *freq, const float *fac, const float *scales);
 
 bool little_endian_host();
 

@@ -1,4 +1,4 @@
-// Stream format v3 constants and small helpers shared by the library's host encoder, the
+// Stream format v4 constants and small helpers shared by the library's host encoder, the
 // stream parser and the decode kernel.  The byte layout is fixed by the library (the pages
 // give none): a 64-byte header, per-row factors, optional per-row code scales, per-context
 // frequency tables, a tile directory and the tiles.
@@ -9,7 +9,7 @@
 namespace ep {
 
 constexpr uint32_t kMagic = 0x31545045u;  // "EPT1"
-constexpr uint32_t kVersion = 3;
+constexpr uint32_t kVersion = 4;
 constexpr uint32_t kProbBits = 11;         // frequency precision: tables sum to 2^11, each entry below it
 constexpr uint32_t kProbScale = 1u << kProbBits;
 constexpr uint32_t kStateLow = 1u << 16;   // rANS state interval [2^16, 2^32), 16-bit words
@@ -26,6 +26,23 @@ constexpr uint32_t kCtxLow[kContexts] = {2, 1, 1, 0, 0, 0, 0};
 constexpr uint32_t kCtxMaxSplit[kContexts] = {9, 9, 9, 8, 8, 8, 8};
 constexpr uint32_t kCtxNarrowSplit[kContexts] = {9, 8, 8, 7, 7, 7, 7};
 constexpr uint32_t kMaxAlphabet = 720;     // (1 << 9) + ((22 - 9) << 2 << 2): the largest context alphabet
+// Paired coding: coordinates (1,2), (3,4), (5,6) of a block as one symbol each.  With A the
+// context's token alphabet length and B = min(A, 40), a pair of tokens both below B is index
+// t_a B + t_b of a table of B^2 + 1 symbols summing to 2^12; the last symbol is an escape, taken
+// by pairs with a token at or above B and by pairs seen fewer than N / 2^16 times (N: the
+// context's pair count), whose tokens follow in the raw bits.  Contexts 1 and 2 are paired up to
+// split 5.  Header byte 43 holds 1 for a paired stream.
+constexpr uint32_t kPairBits = 12;
+constexpr uint32_t kPairScale = 1u << kPairBits;
+constexpr uint32_t kPairBaseMax = 40;
+constexpr uint32_t kPairMaxSplit = 5;
+constexpr uint32_t kPairMaxTable = kPairBaseMax * kPairBaseMax + 1;
+constexpr uint32_t kPairTokFields = 256;  // token fields per coset in the decoder's tables (A <= 168)
+constexpr int64_t kPairMinBlocks = int64_t(1) << 17;  // automatic coding pairs from this many blocks on
+constexpr uint64_t kPairRareScale = 65536;            // a pair seen c times is escaped when c 2^16 < N
+// the decoder's tables for a paired stream: token tables of contexts 0, 3..6 (2048 4-byte slots
+// each), pair tables of contexts 1, 2 (4096 8-byte slots each), and 2 x 256 token fields
+constexpr uint64_t kPairedTableBytes = 5ull * 2048 * 4 + 2ull * 4096 * 8 + 2ull * kPairTokFields * 4;
 constexpr size_t kHeaderBytes = 64;
 constexpr size_t kTileHead = 192;            // per tile: 32 initial states (u32) + 32 word counts (u16)
                                              // then the lanes' words, then the tile's raw extra bits
@@ -41,6 +58,19 @@ inline size_t align16(size_t n) { return (n + 15) & ~size_t(15); }
 inline uint32_t split_alphabet(uint32_t m, uint32_t low) { return (1u << m) + (((kValueBits - m) << kTopBits) << low); }
 
 inline bool split_valid(uint32_t m, int ctx) { return m >= kTopBits + kCtxLow[ctx] && m <= kCtxMaxSplit[ctx]; }
+
+inline uint32_t pair_base(uint32_t A) { return A < kPairBaseMax ? A : kPairBaseMax; }
+inline uint32_t pair_table_len(uint32_t A) { return A ? pair_base(A) * pair_base(A) + 1u : 0u; }
+
+// raw bits of one token of an escaped pair: the bit length of A - 1
+inline uint32_t pair_raw_bits(uint32_t A) {
+    uint32_t v = A > 1 ? A - 1 : 0, n = 0;
+    while (v) {
+        ++n;
+        v >>= 1;
+    }
+    return n;
+}
 
 inline int elt_bytes(int dt) { return dt == 3 ? 4 : (dt == 1 || dt == 2) ? 2 : 1; }
 

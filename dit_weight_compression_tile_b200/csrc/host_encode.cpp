@@ -105,10 +105,10 @@ uint32_t pick_split(const uint64_t *by_len, int ctx) {
     return hi;
 }
 
-// largest remainders to a sum of 2^11, then every seen token raised to >= 1 from the
-// currently largest frequency (lowest index on ties); a lone seen token keeps 2^11 - 1 and
-// gives one unit to a phantom token (token 1 if it is token 0, else token 0)
-uint32_t build_freqs(const std::vector<uint64_t> &cnt, std::vector<uint32_t> &f) {
+// largest remainders to a sum of `scale` (2^11 for token tables, 2^12 for pair tables), then
+// every seen symbol raised to >= 1 from the currently largest frequency (lowest index on ties);
+// a lone seen symbol keeps scale - 1 and gives one unit to a phantom symbol (1 if it is 0, else 0)
+uint32_t build_freqs(const std::vector<uint64_t> &cnt, std::vector<uint32_t> &f, uint32_t scale) {
     size_t n = cnt.size();
     f.assign(n, 0);
     uint64_t total = 0;
@@ -124,7 +124,7 @@ uint32_t build_freqs(const std::vector<uint64_t> &cnt, std::vector<uint32_t> &f)
     if (!total) return 0;
     if (seen == 1) {
         uint32_t phantom = only == 0 ? 1u : 0u;
-        f[only] = kProbScale - 1;
+        f[only] = scale - 1;
         f[phantom] = 1;
         return std::max(len, phantom + 1);
     }
@@ -132,14 +132,14 @@ uint32_t build_freqs(const std::vector<uint64_t> &cnt, std::vector<uint32_t> &f)
     uint32_t used = 0;
     for (size_t i = 0; i < n; ++i) {
         if (!cnt[i]) continue;
-        uint64_t scaled = cnt[i] * kProbScale;
+        uint64_t scaled = cnt[i] * scale;
         f[i] = uint32_t(scaled / total);
         used += f[i];
         rems.emplace_back(scaled % total, uint32_t(i));
     }
     std::stable_sort(rems.begin(), rems.end(),
                      [](const auto &a, const auto &b) { return a.first > b.first; });
-    for (uint32_t r = 0; r < kProbScale - used; ++r) f[rems[r].second] += 1;
+    for (uint32_t r = 0; r < scale - used; ++r) f[rems[r].second] += 1;
     for (size_t i = 0; i < n; ++i) {
         if (cnt[i] && !f[i]) {
             size_t big = size_t(std::max_element(f.begin(), f.end()) - f.begin());
@@ -150,18 +150,54 @@ uint32_t build_freqs(const std::vector<uint64_t> &cnt, std::vector<uint32_t> &f)
     return len;
 }
 
-double estimate_from_counts(const std::vector<uint64_t> *cnt, uint64_t extra_bits, int64_t nb, int64_t ns,
-                            int64_t rows, int64_t cols, int container, uint32_t T) {
+uint32_t seen_len(const std::vector<uint64_t> &cnt) {
+    uint32_t len = 0;
+    for (size_t t = 0; t < cnt.size(); ++t)
+        if (cnt[t]) len = uint32_t(t + 1);
+    return len;
+}
+
+// pairs when asked to (EP_CODING_PAIRED) or, automatically, from 2^17 blocks on; in both cases
+// only with splits of contexts 1 and 2 up to 5 and splits that keep every coordinate in [-256, 255]
+bool pair_eligible(int coding, int64_t nb, const uint32_t *m) {
+    if (coding == EP_CODING_SINGLE) return false;
+    for (int c = 0; c < kContexts; ++c)
+        if (m[c] > kCtxNarrowSplit[c]) return false;
+    if (m[1] > kPairMaxSplit || m[2] > kPairMaxSplit) return false;
+    return coding == EP_CODING_PAIRED || nb >= kPairMinBlocks;
+}
+
+void build_pair_table(std::vector<uint64_t> pair_cnt, uint32_t A, uint64_t N, std::vector<uint32_t> &f,
+                      std::vector<uint8_t> &rare) {
+    const uint32_t n = pair_table_len(A);
+    pair_cnt.resize(n, 0);
+    rare.assign(n, 0);
+    f.assign(n, 0);
+    if (!n) return;
+    uint64_t inside = 0;
+    for (uint32_t q = 0; q + 1 < n; ++q) inside += pair_cnt[q];
+    pair_cnt[n - 1] = N - inside;  // pairs with a token outside the base
+    for (uint32_t q = 0; q + 1 < n; ++q)
+        if (pair_cnt[q] && pair_cnt[q] * kPairRareScale < N) {
+            rare[q] = 1;
+            pair_cnt[n - 1] += pair_cnt[q];
+            pair_cnt[q] = 0;
+        }
+    build_freqs(pair_cnt, f, kPairScale);
+}
+
+double estimate_from_counts(const std::vector<uint64_t> *cnt, const uint32_t *m, int coding, uint64_t extra_bits,
+                            int64_t nb, int64_t ns, int64_t rows, int64_t cols, int container, uint32_t T) {
     double bits = 0.0;
     uint64_t tokens = 0;
+    // a paired stream stores pair tables for contexts 1 and 2; its payload is estimated by the
+    // same token entropy
+    const bool paired = pair_eligible(coding, nb, m);
     for (int c = 0; c < kContexts; ++c) {
         uint64_t n = 0;
-        uint32_t len = 0;
-        for (size_t t = 0; t < cnt[c].size(); ++t) {
-            n += cnt[c][t];
-            if (cnt[c][t]) len = uint32_t(t + 1);
-        }
-        tokens += len;
+        for (size_t t = 0; t < cnt[c].size(); ++t) n += cnt[c][t];
+        const uint32_t len = seen_len(cnt[c]);
+        tokens += paired && (c == 1 || c == 2) ? pair_table_len(len) : len;
         if (!n) continue;
         bits += double(n) * std::log2(double(n));
         for (size_t t = 0; t < cnt[c].size(); ++t)
@@ -174,8 +210,8 @@ double estimate_from_counts(const std::vector<uint64_t> *cnt, uint64_t extra_bit
 }
 
 void write_front(uint8_t *h, const Layout &L, int src_dt, int container, int64_t rows, int64_t cols, uint32_t T,
-                 uint32_t K, int k, const uint32_t *m, const uint32_t *ntok, const std::vector<uint32_t> *freq,
-                 const float *fac, const float *scales) {
+                 uint32_t K, int k, const uint32_t *m, const uint32_t *ntok, const uint32_t *tablen, bool paired,
+                 const std::vector<uint32_t> *freq, const float *fac, const float *scales) {
     auto put = [](uint8_t *p, uint64_t v, int n) {
         for (int i = 0; i < n; ++i) p[i] = uint8_t(v >> (8 * i));
     };
@@ -190,6 +226,7 @@ void write_front(uint8_t *h, const Layout &L, int src_dt, int container, int64_t
     put(h + 32, uint32_t(k), 2);
     h[34] = uint8_t(kProbBits);
     h[35] = uint8_t(kContexts);
+    h[43] = paired ? 1 : 0;
     for (int c = 0; c < kContexts; ++c) {
         h[36 + c] = uint8_t(m[c]);
         put(h + 44 + 2 * c, ntok[c], 2);
@@ -198,7 +235,7 @@ void write_front(uint8_t *h, const Layout &L, int src_dt, int container, int64_t
     if (is_code_container(container)) std::memcpy(h + L.scales, scales, size_t(rows) * 4);
     size_t q = L.freq;
     for (int c = 0; c < kContexts; ++c)
-        for (uint32_t t = 0; t < ntok[c]; ++t, q += 2) put(h + q, freq[c][t], 2);
+        for (uint32_t t = 0; t < tablen[c]; ++t, q += 2) put(h + q, freq[c][t], 2);
 }
 
 bool little_endian_host() {
@@ -216,6 +253,7 @@ struct Encoder {
     int64_t rows, cols, cb, nb;  // cb = ceil(cols / 8): a row is zero-padded to whole E8 blocks
     int container;
     int threads;
+    int coding;  // EP_CODING_*
     uint32_t K;
     std::vector<float> codes;   // INT8/FP8 code matrix (exact in fp32), empty otherwise
     std::vector<float> scales;  // INT8/FP8 per-row scales
@@ -308,20 +346,31 @@ struct Encoder {
             cnt[ctx[i]][t.tok]++;
             extra += t.nbits;
         }
-        return estimate_from_counts(cnt, extra, nb, ns, rows, cols, container, tile_count());
+        return estimate_from_counts(cnt, m, coding, extra, nb, ns, rows, cols, container, tile_count());
     }
 
     // ---- one tile: 32 independent lanes.  A lane's region holds its rANS words in decode order
-    // followed by its raw extra bits, packed least significant bit first into 16-bit words that
-    // are stored back to front (the region's last word holds the first 16 raw bits).  Returns
-    // false when a region exceeds 65535 words.
+    // followed by its raw bits, packed least significant bit first into 16-bit words that are
+    // stored back to front (the region's last word holds the first 16 raw bits).  Per block the
+    // symbols are the 8 tokens (single coding) or token 0, the pair symbols of coordinates (1,2),
+    // (3,4), (5,6) and token 7 (paired coding); the raw bits are the tokens of the escaped pairs
+    // (paired coding), then the extra bits of coordinates 0..7.  Returns false when a region
+    // exceeds 65535 words.
     struct Event {
         uint16_t f, cum;
+        uint8_t bits;  // the symbol's table sums to 2^bits
+    };
+    struct Model {
+        const uint32_t *m;
+        const std::vector<uint32_t> *freq, *cum;  // paired contexts 1, 2: the pair tables
+        bool paired;
+        const uint32_t *A;                         // paired contexts 1, 2: token alphabet length
+        const std::vector<uint8_t> *rare;          // paired contexts 1, 2: escaped pair indices
     };
 
     static bool encode_tile(const uint8_t *ctx, const uint32_t *val, int64_t nb, int64_t t, uint32_t K,
-                            const uint32_t *m, const std::vector<uint32_t> *freq, const std::vector<uint32_t> *cum,
-                            std::vector<Event> &ev, std::vector<uint16_t> &words, std::vector<uint8_t> &out) {
+                            const Model &M, std::vector<Event> &ev, std::vector<uint16_t> &words,
+                            std::vector<uint8_t> &out) {
         int64_t first = t * int64_t(kLanes) * K;
         uint32_t state[kLanes];
         uint32_t count[kLanes];
@@ -333,32 +382,53 @@ struct Encoder {
             uint64_t acc = 0;
             uint32_t nacc = 0;
             std::vector<uint16_t> raw;
+            auto add = [&](uint32_t c, uint32_t sym, uint32_t bits) {
+                ev.push_back({uint16_t(M.freq[c][sym]), uint16_t(M.cum[c][sym]), uint8_t(bits)});
+            };
+            auto push = [&](uint32_t v, uint32_t nbits) {
+                acc |= uint64_t(v) << nacc;
+                nacc += nbits;
+                while (nacc >= 16) {
+                    raw.push_back(uint16_t(acc));
+                    acc >>= 16;
+                    nacc -= 16;
+                }
+            };
             for (uint32_t k = 0; k < K; ++k) {
                 int64_t b = first + int64_t(k) * kLanes + l;
                 if (b >= nb) break;
-                for (int i = 0; i < 8; ++i) {
-                    size_t s = size_t(8 * b + i);
-                    uint8_t c = ctx[s];
-                    Token tk = token_of(val[s], m[c], kCtxLow[c]);
-                    ev.push_back({uint16_t(freq[c][tk.tok]), uint16_t(cum[c][tk.tok])});
-                    acc |= uint64_t(tk.extra) << nacc;
-                    nacc += tk.nbits;
-                    while (nacc >= 16) {
-                        raw.push_back(uint16_t(acc));
-                        acc >>= 16;
-                        nacc -= 16;
+                const size_t s0 = size_t(8 * b);
+                Token tk[8];
+                for (int i = 0; i < 8; ++i) tk[i] = token_of(val[s0 + i], M.m[ctx[s0 + i]], kCtxLow[ctx[s0 + i]]);
+                if (!M.paired) {
+                    for (int i = 0; i < 8; ++i) add(ctx[s0 + i], tk[i].tok, kProbBits);
+                } else {
+                    const uint32_t pc = ctx[s0 + 1], A = M.A[pc], B = pair_base(A);
+                    bool esc[3];
+                    add(ctx[s0], tk[0].tok, kProbBits);
+                    for (int j = 0; j < 3; ++j) {
+                        const uint32_t ta = tk[1 + 2 * j].tok, tb = tk[2 + 2 * j].tok;
+                        esc[j] = ta >= B || tb >= B || M.rare[pc][ta * B + tb] != 0;
+                        add(pc, esc[j] ? B * B : ta * B + tb, kPairBits);
                     }
+                    add(ctx[s0 + 7], tk[7].tok, kProbBits);
+                    for (int j = 0; j < 3; ++j)
+                        if (esc[j]) {
+                            push(tk[1 + 2 * j].tok, pair_raw_bits(A));
+                            push(tk[2 + 2 * j].tok, pair_raw_bits(A));
+                        }
                 }
+                for (int i = 0; i < 8; ++i) push(tk[i].extra, tk[i].nbits);
             }
             if (nacc) raw.push_back(uint16_t(acc));
             uint32_t x = kStateLow;
             for (size_t e = ev.size(); e-- > 0;) {
-                uint32_t f = ev[e].f;
-                if (uint64_t(x) >= (uint64_t(f) << (32 - kProbBits))) {  // keep the next state below 2^32
+                const uint32_t f = ev[e].f, n = ev[e].bits;
+                if (uint64_t(x) >= (uint64_t(f) << (32 - n))) {  // keep the next state below 2^32
                     words.push_back(uint16_t(x));
                     x >>= 16;
                 }
-                x = (x / f) * kProbScale + (x % f) + ev[e].cum;
+                x = (x / f) * (1u << n) + (x % f) + ev[e].cum;
             }
             std::reverse(words.begin() + long(before), words.end());  // decode order
             words.insert(words.end(), raw.rbegin(), raw.rend());
@@ -423,17 +493,53 @@ struct Encoder {
             }
         });
         std::vector<uint32_t> freq[kContexts], cum[kContexts];
-        uint32_t ntok[kContexts];
+        std::vector<uint8_t> rare[kContexts];
+        uint32_t ntok[kContexts], tablen[kContexts], A[kContexts] = {};
         uint64_t tokens = 0;
+        std::vector<uint64_t> cnt[kContexts];
         for (int c = 0; c < kContexts; ++c) {
-            std::vector<uint64_t> cnt(split_alphabet(m[c], kCtxLow[c]), 0);
+            cnt[c].assign(split_alphabet(m[c], kCtxLow[c]), 0);
             for (auto &pc : part_cnt)
-                for (size_t t = 0; t < cnt.size(); ++t) cnt[t] += pc[size_t(c) * kMaxAlphabet + t];
-            ntok[c] = build_freqs(cnt, freq[c]);
+                for (size_t t = 0; t < cnt[c].size(); ++t) cnt[c][t] += pc[size_t(c) * kMaxAlphabet + t];
+        }
+        const bool paired = pair_eligible(coding, nb, m);
+        for (int c = 0; c < kContexts; ++c) {
+            if (paired && (c == 1 || c == 2)) {
+                // counts of the token pairs of coordinates (1,2), (3,4), (5,6) inside the base
+                A[c] = seen_len(cnt[c]);
+                const uint32_t B = pair_base(A[c]), a2 = B * B;
+                std::vector<std::vector<uint64_t>> part_pair(static_cast<size_t>(nchunks));
+                parallel_for(nchunks, nchunks, [&](int64_t c0, int64_t c1) {
+                    for (int64_t q = c0; q < c1; ++q) {
+                        auto &pp = part_pair[size_t(q)];
+                        pp.assign(a2, 0);
+                        for (int64_t b = q * per; b < std::min(nb, (q + 1) * per); ++b) {
+                            if (ctx[size_t(8 * b + 1)] != c) continue;
+                            for (int j = 0; j < 3; ++j) {
+                                uint32_t ta = token_of(val[size_t(8 * b + 1 + 2 * j)], m[c], kCtxLow[c]).tok;
+                                uint32_t tb = token_of(val[size_t(8 * b + 2 + 2 * j)], m[c], kCtxLow[c]).tok;
+                                if (ta < B && tb < B) pp[ta * B + tb]++;
+                            }
+                        }
+                    }
+                });
+                std::vector<uint64_t> pair_cnt(a2, 0);
+                for (auto &pp : part_pair)
+                    for (uint32_t q = 0; q < a2; ++q) pair_cnt[q] += pp[q];
+                uint64_t N = 0;  // every token of the context belongs to one of its pairs
+                for (uint64_t x : cnt[c]) N += x;
+                build_pair_table(pair_cnt, A[c], N / 2, freq[c], rare[c]);
+                ntok[c] = A[c];
+                tablen[c] = pair_table_len(A[c]);
+            } else {
+                ntok[c] = build_freqs(cnt[c], freq[c]);
+                tablen[c] = ntok[c];
+            }
             cum[c].assign(freq[c].size(), 0);
             for (size_t t = 1; t < freq[c].size(); ++t) cum[c][t] = cum[c][t - 1] + freq[c][t - 1];
-            tokens += ntok[c];
+            tokens += tablen[c];
         }
+        const Model model{m, freq, cum, paired, A, rare};
         // tiles, encoded in parallel into per-range buffers
         uint32_t T = tile_count();
         int tchunks = int(std::max<int64_t>(1, std::min<int64_t>(threads, T)));
@@ -447,7 +553,7 @@ struct Encoder {
             for (int64_t c = c0; c < c1; ++c)
                 for (int64_t t = c * tper; t < std::min<int64_t>(T, (c + 1) * tper); ++t) {
                     size_t before = part_tiles[size_t(c)].size();
-                    if (!encode_tile(ctx.data(), val.data(), nb, t, K, m, freq, cum, ev, words, part_tiles[size_t(c)]))
+                    if (!encode_tile(ctx.data(), val.data(), nb, t, K, model, ev, words, part_tiles[size_t(c)]))
                         part_fits[size_t(c)] = 0;
                     part_sizes[size_t(c)].push_back(uint32_t((part_tiles[size_t(c)].size() - before) / 16));
                 }
@@ -462,7 +568,8 @@ struct Encoder {
         auto put = [](uint8_t *p, uint64_t v, int n) {
             for (int i = 0; i < n; ++i) p[i] = uint8_t(v >> (8 * i));
         };
-        write_front(h, L, src.dt, container, rows, cols, T, K, k, m, ntok, freq, fac.data(), scales.data());
+        write_front(h, L, src.dt, container, rows, cols, T, K, k, m, ntok, tablen, paired, freq, fac.data(),
+                    scales.data());
         uint32_t at = 0;
         size_t d = L.dir, o = L.tiles;
         for (int c = 0; c < tchunks; ++c) {
@@ -490,7 +597,7 @@ extern "C" size_t ep_compress_bound(int64_t rows, int64_t cols, const ep_config 
     uint32_t K = cfg->blocks_per_lane ? cfg->blocks_per_lane : ep::auto_blocks_per_lane(nb, cfg->target_bpp);
     uint64_t T = uint64_t((nb + 32 * int64_t(K) - 1) / (32 * int64_t(K)));
     return ep::layout_for(rows, ep::is_code_container(cfg->container_dtype) ? cfg->container_dtype : 0,
-                          7 * ep::kMaxAlphabet, T)
+                          7 * ep::kPairMaxTable, T)
                .tiles +
            size_t(T) * (ep::kTileHead + 16) + size_t(5.0 * n);
 }
@@ -505,6 +612,7 @@ extern "C" int ep_compress_host(const void *src, int32_t src_dtype, int64_t rows
     int container = cfg->container_dtype ? cfg->container_dtype : src_dtype;
     if (container < EP_BF16 || container > EP_FP8_E4M3) return EP_ERR_INVALID_ARG;
     if (cfg->blocks_per_lane > 4096) return EP_ERR_INVALID_ARG;
+    if (cfg->coding < EP_CODING_AUTO || cfg->coding > EP_CODING_PAIRED) return EP_ERR_INVALID_ARG;
     if ((rows * ((cols + 7) / 8)) >> 32) return EP_ERR_UNSUPPORTED;
 
     Encoder E;
@@ -512,6 +620,7 @@ extern "C" int ep_compress_host(const void *src, int32_t src_dtype, int64_t rows
     E.rows = rows;
     E.cols = cols;
     E.container = container;
+    E.coding = cfg->coding;
     E.threads = cfg->n_threads > 0 ? cfg->n_threads : int(std::max(1u, std::thread::hardware_concurrency()));
     // finite check
     {

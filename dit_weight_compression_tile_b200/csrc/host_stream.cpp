@@ -2,7 +2,7 @@
 //
 // The CompressedTensor properties of the "EntroPack API reference" (shape, dtype,
 // actual_bpp = 8 * storage_nbytes / numel, storage_nbytes with and without the header)
-// read from a host copy of a format-v3 stream, which is validated before any decode.
+// read from a host copy of a format-v4 stream, which is validated before any decode.
 #include <cstring>
 
 #include "../../include/eptile.h"
@@ -43,12 +43,20 @@ extern "C" int ep_stream_info(const void *blob, size_t nbytes, ep_info *info) {
     int64_t nb = I.rows * ((I.cols + 7) / 8);  // rows zero-padded to whole E8 blocks
     int64_t per_tile = int64_t(kLanes) * I.blocks_per_lane;
     if ((nb + per_tile - 1) / per_tile != int64_t(I.n_tiles)) return EP_ERR_CORRUPT;
+    if (p[43] > 1) return EP_ERR_CORRUPT;
+    I.paired = p[43];
     uint64_t tokens = 0;
+    uint32_t tablen[kContexts];
     for (int c = 0; c < kContexts; ++c) {
         I.split[c] = p[36 + c];
         I.ntok[c] = uint16_t(rd(p + 44 + 2 * c, 2));
         if (!split_valid(I.split[c], c) || I.ntok[c] > split_alphabet(I.split[c], kCtxLow[c])) return EP_ERR_CORRUPT;
-        tokens += I.ntok[c];
+        // a paired stream keeps every split in the narrow range and pairs splits up to 5
+        if (I.paired && I.split[c] > kCtxNarrowSplit[c]) return EP_ERR_CORRUPT;
+        const bool pair = I.paired && (c == 1 || c == 2);
+        if (pair && I.split[c] > kPairMaxSplit) return EP_ERR_CORRUPT;
+        tablen[c] = pair ? pair_table_len(I.ntok[c]) : I.ntok[c];
+        tokens += tablen[c];
     }
     Layout L = layout_for(I.rows, I.container_dtype, tokens, I.n_tiles);
     if (L.tiles > nbytes) return EP_ERR_CORRUPT;
@@ -59,13 +67,14 @@ extern "C" int ep_stream_info(const void *blob, size_t nbytes, ep_info *info) {
     I.off_tiles = L.tiles;
     size_t q = L.freq;
     for (int c = 0; c < kContexts; ++c) {
+        const uint32_t M = I.paired && (c == 1 || c == 2) ? kPairScale : kProbScale;
         uint32_t sum = 0;
-        for (uint32_t t = 0; t < I.ntok[c]; ++t, q += 2) {
+        for (uint32_t t = 0; t < tablen[c]; ++t, q += 2) {
             uint32_t f = uint32_t(rd(p + q, 2));
-            if (f >= kProbScale) return EP_ERR_CORRUPT;  // the decoder's table entry holds 11 bits
+            if (f >= M) return EP_ERR_CORRUPT;  // the decoder's table entry holds 11 (pairs: 12) bits
             sum += f;
         }
-        if (I.ntok[c] && sum != kProbScale) return EP_ERR_CORRUPT;
+        if (tablen[c] && sum != M) return EP_ERR_CORRUPT;
     }
     const uint8_t *d = p + L.dir;
     uint64_t prev = rd(d, 4), largest = 0;
@@ -82,7 +91,9 @@ extern "C" int ep_stream_info(const void *blob, size_t nbytes, ep_info *info) {
     I.header_nbytes = kHeaderBytes;
     I.actual_bpp = 8.0 * double(nbytes) / double(I.rows * I.cols);
     I.out_nbytes = uint64_t(I.rows * I.cols) * uint64_t(elt_bytes(I.container_dtype));
-    I.workspace_nbytes = uint64_t(kContexts) * kProbScale * 4;  // the decoder's slot tables
+    // the decoder's slot tables: 7 token tables, or 5 token tables, two pair tables of 8-byte
+    // entries and the token fields of the escaped pairs
+    I.workspace_nbytes = I.paired ? kPairedTableBytes : uint64_t(kContexts) * kProbScale * 4;
     *info = I;
     return EP_OK;
 }

@@ -36,7 +36,7 @@
  * number of low bits kept in the token, raw extra bits in a separate stream per tile.
  * ---------------------------------------------------------------------------------- */
 #define MAGIC 0x31545045u /* bytes 'E','P','T','1' */
-#define VERSION 3
+#define VERSION 4
 #define PROB_BITS 11
 #define PROB_M 2048u
 #define STATE_L 65536u
@@ -57,6 +57,21 @@
  * within -256 <= y_i <= 255. */
 static const int32_t CTX_LOW[NCTX] = {2, 1, 1, 0, 0, 0, 0};
 static const int32_t CTX_MAX_SPLIT[NCTX] = {9, 9, 9, 8, 8, 8, 8};
+/* splits up to which every directly coded coordinate v itself lies in [-256, 255] */
+static const int32_t CTX_NARROW_SPLIT[NCTX] = {9, 8, 8, 7, 7, 7, 7};
+
+/* Paired coding (a reading of the pages' conditional model, which they leave open): with small
+ * splits, coordinates (1,2), (3,4) and (5,6) of a block are coded as one symbol each.  With A the
+ * context's token alphabet length and B = min(A, 40), a pair of tokens both below B is symbol
+ * t_a B + t_b of a table of B^2 + 1 symbols summing to 2^12; the last symbol is an escape, taken
+ * by pairs with a token at or above B and by pairs seen fewer than N / 2^16 times (N: the
+ * context's pair count).  An escaped pair's two tokens follow in the raw bits. */
+#define PAIR_BITS 12
+#define PAIR_M 4096u
+#define PAIR_BASE_MAX 40u           /* largest pair base B */
+#define PAIR_MAX_SPLIT 5            /* contexts 1 and 2 are paired up to this split */
+#define PAIR_MIN_BLOCKS (1 << 17)   /* automatic coding pairs tensors of at least this many blocks */
+#define PAIR_RARE_SCALE 65536u      /* a pair seen c times is escaped when c * 2^16 < N */
 
 static size_t al16(size_t n) { return (n + 15) & ~(size_t)15; }
 
@@ -434,14 +449,15 @@ static int bit_length(uint32_t u)
 }
 
 /* ---------------------------------- frequency tables --------------------------------- */
-/* Counts -> frequencies summing to M = 2^11 by largest remainders: f_i = floor(c_i M / n);
+/* Counts -> frequencies summing to M (2^11 for token tables, 2^12 for pair tables) by largest
+ * remainders: f_i = floor(c_i M / n);
  * the M - sum f_i leftover units go one each to the largest remainders (c_i M mod n),
  * lower index first on ties; then every seen token left at 0 is raised to 1 by taking a
  * unit from the currently largest frequency (lower index first on ties).  Every frequency
  * stays below M: a context with one seen token t gives it M - 1 and one unit to a phantom
  * token that never occurs (token 1 if t = 0, else token 0).  Returns the table length (last
  * token with f > 0, plus 1), or -1 for a single-token alphabet. */
-int32_t or_normalize_freqs(const uint64_t *counts, int32_t n, uint32_t *f)
+static int32_t normalize_to(const uint64_t *counts, int32_t n, uint32_t M, uint32_t *f)
 {
     uint64_t total = 0;
     int32_t len = 0;
@@ -458,12 +474,12 @@ int32_t or_normalize_freqs(const uint64_t *counts, int32_t n, uint32_t *f)
     for (int32_t i = 0; i < n; i++) {
         if (!counts[i])
             continue;
-        /* c * M < 2^64 for any realistic count (c < 2^53) */
-        f[i] = (uint32_t)((counts[i] * PROB_M) / total);
-        rem[i] = (counts[i] * PROB_M) % total;
+        /* c * M < 2^64 for any realistic count (c < 2^51) */
+        f[i] = (uint32_t)((counts[i] * M) / total);
+        rem[i] = (counts[i] * M) % total;
         sum += f[i];
     }
-    uint32_t left = PROB_M - sum;
+    uint32_t left = M - sum;
     unsigned char *given = (unsigned char *)calloc((size_t)n, 1);
     for (uint32_t r = 0; r < left; r++) {
         int32_t best = -1;
@@ -495,12 +511,56 @@ int32_t or_normalize_freqs(const uint64_t *counts, int32_t n, uint32_t *f)
         if (n < 2)
             return -1;
         int32_t phantom = only == 0 ? 1 : 0;
-        f[only] = PROB_M - 1u;
+        f[only] = M - 1u;
         f[phantom] = 1;
         if (phantom + 1 > len)
             len = phantom + 1;
     }
     return len;
+}
+
+int32_t or_normalize_freqs(const uint64_t *counts, int32_t n, uint32_t *f)
+{
+    return normalize_to(counts, n, PROB_M, f);
+}
+
+int32_t or_normalize_freqs_to(const uint64_t *counts, int32_t n, int32_t bits, uint32_t *f)
+{
+    return normalize_to(counts, n, 1u << bits, f);
+}
+
+/* ---------------------------------- paired coding ----------------------------------- */
+/* pair base B of a context with token alphabet length A, and its table length (0: no table) */
+static uint32_t pair_base(uint32_t A) { return A < PAIR_BASE_MAX ? A : PAIR_BASE_MAX; }
+static uint32_t pair_table_len(uint32_t A) { return A ? pair_base(A) * pair_base(A) + 1u : 0u; }
+
+/* raw bits of one token of an escaped pair: enough for A - 1 */
+static uint32_t pair_raw_bits(uint32_t A) { return (uint32_t)bit_length(A > 1 ? A - 1 : 0); }
+
+/* last token seen, plus one */
+static uint32_t seen_len(const uint64_t *cnt, uint32_t n)
+{
+    uint32_t len = 0;
+    for (uint32_t t = 0; t < n; t++)
+        if (cnt[t])
+            len = t + 1;
+    return len;
+}
+
+/* The stream pairs coordinates 1..6 when it is asked to (OR_CODING_PAIRED) or, under automatic
+ * coding, when it holds at least 2^17 blocks (the pair tables then cost under 1 % of a 4-bit
+ * stream); in both cases only when the splits of contexts 1 and 2 are at most 5 (their direct
+ * tokens fit the pair base) and every split keeps the coordinates' values in [-256, 255]. */
+static int pair_eligible(int32_t coding, int64_t nb, const int32_t *m)
+{
+    if (coding == OR_CODING_SINGLE)
+        return 0;
+    for (int c = 0; c < NCTX; c++)
+        if (m[c] > CTX_NARROW_SPLIT[c])
+            return 0;
+    if (m[1] > PAIR_MAX_SPLIT || m[2] > PAIR_MAX_SPLIT)
+        return 0;
+    return coding == OR_CODING_PAIRED || nb >= PAIR_MIN_BLOCKS;
 }
 
 /* ---------------------------------- tiles -------------------------------------------- */
@@ -692,7 +752,7 @@ static size_t meta_bytes(int64_t rows, int32_t container, uint64_t total_tokens,
  * that carry no payload (32 lanes x 3 bytes), the 32 word counts take 64 bytes and a tile
  * pads to 16 bytes (8 on average; the raw bits' last word is counted in that padding). */
 static double estimate_bpp(const double *w, const float *s, int64_t rows, int64_t cols, int32_t container,
-                           int32_t k, uint32_t K)
+                           int32_t k, uint32_t K, int32_t coding)
 {
     /* w: padded rows of 8 * ceil(cols / 8) values; the rate counts the cols true columns */
     int64_t cb = (cols + 7) / 8, nb = rows * cb;
@@ -727,15 +787,17 @@ static double estimate_bpp(const double *w, const float *s, int64_t rows, int64_
     }
     double bits = 0.0;
     uint64_t total_tokens = 0;
+    uint32_t lens[NCTX];
+    for (int c = 0; c < NCTX; c++)
+        lens[c] = seen_len(cnt[c], or_alphabet_size(m[c], CTX_LOW[c]));
+    /* a paired stream stores pair tables for contexts 1 and 2; its payload is estimated by
+     * the same token entropy */
+    int paired = pair_eligible(coding, nb, m);
     for (int c = 0; c < NCTX; c++) {
         uint64_t n = 0;
-        uint32_t len = 0;
-        for (uint32_t t = 0; t < or_alphabet_size(m[c], CTX_LOW[c]); t++) {
+        for (uint32_t t = 0; t < or_alphabet_size(m[c], CTX_LOW[c]); t++)
             n += cnt[c][t];
-            if (cnt[c][t])
-                len = t + 1;
-        }
-        total_tokens += len;
+        total_tokens += paired && (c == 1 || c == 2) ? pair_table_len(lens[c]) : lens[c];
         if (n == 0)
             continue;
         bits += (double)n * log2((double)n);
@@ -755,7 +817,7 @@ static double estimate_bpp(const double *w, const float *s, int64_t rows, int64_
 }
 
 double or_estimate_bpp(const void *src, int32_t sdt, int64_t rows, int64_t cols, int32_t container, int32_t k,
-                       uint32_t K)
+                       uint32_t K, int32_t coding)
 {
     double *w = lattice_input(src, sdt, rows, cols, container, NULL);
     float *s = (float *)malloc((size_t)rows * sizeof(float));
@@ -763,7 +825,7 @@ double or_estimate_bpp(const void *src, int32_t sdt, int64_t rows, int64_t cols,
     double *wp = pad_rows(w, rows, cols);
     if (K == 0)
         K = or_choose_blocks_per_lane(rows * ((cols + 7) / 8), 4.0);
-    double e = estimate_bpp(wp, s, rows, cols, container, k, K);
+    double e = estimate_bpp(wp, s, rows, cols, container, k, K, coding);
     if (wp != w)
         free(wp);
     free(s);
@@ -797,7 +859,73 @@ static uint64_t get64(const uint8_t *p) { return (uint64_t)get32(p) | ((uint64_t
 /* ---------------------------------- tile encoder ------------------------------------- */
 typedef struct {
     uint16_t f, cum;
+    uint8_t bits; /* the symbol's table sums to 2^bits */
 } event;
+
+/* what the tile encoder needs of the stream's model */
+typedef struct {
+    int32_t m[NCTX];
+    uint32_t *freq[NCTX], *cum[NCTX]; /* contexts 1 and 2 of a paired stream: the pair tables */
+    int paired;
+    uint32_t A[NCTX];   /* contexts 1 and 2 of a paired stream: token alphabet length */
+    uint8_t *rare[NCTX]; /* contexts 1 and 2 of a paired stream: pair index -> coded as an escape */
+} coder;
+
+/* a token pair's symbol in a pair table of base B: its index, or the escape B * B */
+static uint32_t pair_symbol(const coder *C, uint32_t c, uint32_t ta, uint32_t tb)
+{
+    uint32_t B = pair_base(C->A[c]);
+    if (ta >= B || tb >= B || C->rare[c][ta * B + tb])
+        return B * B;
+    return ta * B + tb;
+}
+
+static void add_event(event *ev, size_t *ne, const coder *C, uint32_t c, uint32_t sym, uint32_t bits)
+{
+    ev[*ne].f = (uint16_t)C->freq[c][sym];
+    ev[*ne].cum = (uint16_t)C->cum[c][sym];
+    ev[*ne].bits = (uint8_t)bits;
+    (*ne)++;
+}
+
+static void push_bits(uint8_t *raw, size_t *nraw, uint32_t v, uint32_t nbits)
+{
+    for (uint32_t j = 0; j < nbits; j++)
+        raw[(*nraw)++] = (uint8_t)((v >> j) & 1u);
+}
+
+/* One block's rANS symbols (in decode order) and raw bits.  Single coding: the 8 tokens.
+ * Paired coding: token 0, the pair symbols of coordinates (1,2), (3,4), (5,6), token 7; the raw
+ * bits start with the two tokens of every escaped pair (first then second, each in
+ * pair_raw_bits(A) bits).  Then, in both codings, the extra bits of coordinates 0..7. */
+static void block_events(const coder *C, const uint32_t *ctx, const uint32_t *s, event *ev, size_t *ne,
+                         uint8_t *raw, size_t *nraw)
+{
+    uint32_t tok[8], nbits[8], extra[8];
+    for (int i = 0; i < 8; i++)
+        or_tokenize(s[i], C->m[ctx[i]], CTX_LOW[ctx[i]], &tok[i], &nbits[i], &extra[i]);
+    if (!C->paired) {
+        for (int i = 0; i < 8; i++)
+            add_event(ev, ne, C, ctx[i], tok[i], PROB_BITS);
+    } else {
+        uint32_t pc = ctx[1], A = C->A[pc], B = pair_base(A);
+        int esc[3];
+        add_event(ev, ne, C, ctx[0], tok[0], PROB_BITS);
+        for (int j = 0; j < 3; j++) {
+            uint32_t sym = pair_symbol(C, pc, tok[1 + 2 * j], tok[2 + 2 * j]);
+            esc[j] = sym == B * B;
+            add_event(ev, ne, C, pc, sym, PAIR_BITS);
+        }
+        add_event(ev, ne, C, ctx[7], tok[7], PROB_BITS);
+        for (int j = 0; j < 3; j++)
+            if (esc[j]) {
+                push_bits(raw, nraw, tok[1 + 2 * j], pair_raw_bits(A));
+                push_bits(raw, nraw, tok[2 + 2 * j], pair_raw_bits(A));
+            }
+    }
+    for (int i = 0; i < 8; i++)
+        push_bits(raw, nraw, extra[i], nbits[i]);
+}
 
 typedef struct {
     uint8_t *p;
@@ -819,21 +947,20 @@ static void bytes_put(bytes *b, const void *src, size_t n)
 
 /* Decode order inside a tile (the rule both sides follow): the 32 lanes are independent
  * rANS coders, each with its own region of 16-bit words.  Lane l decodes its blocks
- * t*32K + 32k + l in order of k, and per block the tokens of coordinates 0..7 in order;
- * after every token the lane reads the next word from the front of its region if its state
- * fell below L.  After a block's 8 tokens the lane takes the raw extra bits of the block's
- * escape tokens, coordinate by coordinate, from the back of its region: the region's last
- * word holds the lane's first 16 raw bits (least significant bit first), the word before it
- * the next 16, and so on.  The encoder runs a lane's tokens in reverse, emitting words in
- * reverse.  A tile stores the 32 final encoder states (= initial decoder states, u32), the
- * 32 region lengths in words (u16), then the regions of lanes 0..31 one after another, zero
- * padded to 16 bytes. */
+ * t*32K + 32k + l in order of k, and per block its rANS symbols in the order block_events
+ * lists them; after every symbol the lane reads the next word from the front of its region if
+ * its state fell below L.  After a block's symbols the lane takes the block's raw bits (in
+ * block_events' order) from the back of its region: the region's last word holds the lane's
+ * first 16 raw bits (least significant bit first), the word before it the next 16, and so on.
+ * The encoder runs a lane's symbols in reverse, emitting words in reverse.  A tile stores the
+ * 32 final encoder states (= initial decoder states, u32), the 32 region lengths in words
+ * (u16), then the regions of lanes 0..31 one after another, zero padded to 16 bytes. */
 static int encode_tile(const uint32_t *ctx, const uint32_t *s, int64_t nb, int64_t t, uint32_t K,
-                       const int32_t *m, uint32_t *const *freq, uint32_t *const *cum, bytes *out)
+                       const coder *C, bytes *out)
 {
     int64_t base = t * (int64_t)LANES * K;
     event *ev = (event *)malloc((size_t)K * 8 * sizeof(event));
-    uint8_t *raw = (uint8_t *)malloc((size_t)K * 8 * VALUE_BITS + 16);
+    uint8_t *raw = (uint8_t *)malloc((size_t)K * (8 * VALUE_BITS + 48) + 16);
     uint16_t *words[LANES];
     size_t nw[LANES];
     uint32_t x[LANES];
@@ -844,15 +971,7 @@ static int encode_tile(const uint32_t *ctx, const uint32_t *s, int64_t nb, int64
             int64_t b = base + (int64_t)k * LANES + l;
             if (b >= nb)
                 break;
-            for (int i = 0; i < 8; i++) {
-                uint32_t c = ctx[8 * b + i], tok, nbits, extra;
-                or_tokenize(s[8 * b + i], m[c], CTX_LOW[c], &tok, &nbits, &extra);
-                ev[ne].f = (uint16_t)freq[c][tok];
-                ev[ne].cum = (uint16_t)cum[c][tok];
-                ne++;
-                for (uint32_t j = 0; j < nbits; j++)
-                    raw[nraw++] = (uint8_t)((extra >> j) & 1u);
-            }
+            block_events(C, ctx + 8 * b, s + 8 * b, ev, &ne, raw, &nraw);
         }
         size_t nrawords = (nraw + 15) / 16;
         words[l] = (uint16_t *)malloc((ne + nrawords + 1) * sizeof(uint16_t));
@@ -871,13 +990,13 @@ static int encode_tile(const uint32_t *ctx, const uint32_t *s, int64_t nb, int64
             words[l][nw[l]++] = rw[j];
         free(rw);
         for (size_t e = ne; e-- > 0;) {
-            uint32_t f = ev[e].f;
-            /* renormalise so that the encoded state stays below 2^32: x_max = (L >> 11) << 16 * f */
-            if ((uint64_t)st >= ((uint64_t)f << 21)) {
+            uint32_t f = ev[e].f, n = ev[e].bits;
+            /* renormalise so that the encoded state stays below 2^32: x_max = (L >> n) << 16 * f */
+            if ((uint64_t)st >= ((uint64_t)f << (32 - n))) {
                 words[l][nw[l]++] = (uint16_t)(st & 0xffffu);
                 st >>= 16;
             }
-            st = ((st / f) << PROB_BITS) + (st % f) + ev[e].cum;
+            st = ((st / f) << n) + (st % f) + ev[e].cum;
         }
         x[l] = st;
         if (nw[l] > 0xffffu)
@@ -907,8 +1026,8 @@ static int encode_tile(const uint32_t *ctx, const uint32_t *s, int64_t nb, int64
 
 /* ---------------------------------- full encode at one k ----------------------------- */
 static int encode_at(const double *w, const float *s, const float *scales, int64_t rows, int64_t cols,
-                     int32_t sdt, int32_t container, int32_t k, uint32_t K, uint8_t *out, size_t cap,
-                     size_t *out_n)
+                     int32_t sdt, int32_t container, int32_t k, uint32_t K, int32_t coding, uint8_t *out,
+                     size_t cap, size_t *out_n)
 {
     /* w: padded rows of 8 * ceil(cols / 8) values; the header keeps the true cols */
     int64_t cb = (cols + 7) / 8, nb = rows * cb;
@@ -945,14 +1064,60 @@ static int encode_at(const double *w, const float *s, const float *scales, int64
         or_tokenize(u[i], m[ctx[i]], CTX_LOW[ctx[i]], &t, &nbits, &ex);
         cnt[ctx[i]][t]++;
     }
+    coder C;
+    memset(&C, 0, sizeof C);
+    uint32_t tablen[NCTX];
+    C.paired = pair_eligible(coding, nb, m);
     for (int c = 0; c < NCTX; c++) {
-        ntok[c] = (uint32_t)or_normalize_freqs(cnt[c], (int32_t)alpha[c], freq[c]);
+        C.m[c] = m[c];
+        if (C.paired && (c == 1 || c == 2)) {
+            /* pair table: counts of (t_a, t_b) over the whole tensor; pairs outside the base and
+             * rare pairs escaped */
+            uint32_t A = seen_len(cnt[c], alpha[c]), B = pair_base(A), n = pair_table_len(A);
+            ntok[c] = A;
+            tablen[c] = n;
+            C.A[c] = A;
+            C.rare[c] = (uint8_t *)calloc(n + 1, 1);
+            free(freq[c]);
+            free(cum[c]);
+            freq[c] = (uint32_t *)calloc(n + 1, sizeof(uint32_t));
+            cum[c] = (uint32_t *)calloc(n + 1, sizeof(uint32_t));
+            uint64_t *pc = (uint64_t *)calloc(n + 1, sizeof(uint64_t));
+            uint64_t N = 0;
+            for (int64_t b = 0; b < nb; b++)
+                if (ctx[8 * b + 1] == (uint32_t)c)
+                    for (int j = 0; j < 3; j++) {
+                        uint32_t ta, tb, nbits, ex;
+                        or_tokenize(u[8 * b + 1 + 2 * j], m[c], CTX_LOW[c], &ta, &nbits, &ex);
+                        or_tokenize(u[8 * b + 2 + 2 * j], m[c], CTX_LOW[c], &tb, &nbits, &ex);
+                        if (ta < B && tb < B)
+                            pc[ta * B + tb]++;
+                        else
+                            pc[n - 1]++;
+                        N++;
+                    }
+            if (n) {
+                for (uint32_t q = 0; q + 1 < n; q++)
+                    if (pc[q] && pc[q] * PAIR_RARE_SCALE < N) {
+                        C.rare[c][q] = 1;
+                        pc[n - 1] += pc[q];
+                        pc[q] = 0;
+                    }
+                normalize_to(pc, (int32_t)n, PAIR_M, freq[c]);
+            }
+            free(pc);
+        } else {
+            ntok[c] = (uint32_t)or_normalize_freqs(cnt[c], (int32_t)alpha[c], freq[c]);
+            tablen[c] = ntok[c];
+        }
         uint32_t a = 0;
-        for (uint32_t t = 0; t < alpha[c]; t++) {
+        for (uint32_t t = 0; t < tablen[c]; t++) {
             cum[c][t] = a;
             a += freq[c][t];
         }
-        total_tokens += ntok[c];
+        C.freq[c] = freq[c];
+        C.cum[c] = cum[c];
+        total_tokens += tablen[c];
     }
     uint32_t T = (uint32_t)((nb + (int64_t)LANES * K - 1) / ((int64_t)LANES * K));
     bytes tiles = {0, 0, 0};
@@ -960,7 +1125,7 @@ static int encode_at(const double *w, const float *s, const float *scales, int64
     int trc = OR_OK;
     for (uint32_t t = 0; t < T; t++) {
         dir[t] = (uint32_t)(tiles.n / 16);
-        if (encode_tile(ctx, u, nb, t, K, m, freq, cum, &tiles) != OR_OK)
+        if (encode_tile(ctx, u, nb, t, K, &C, &tiles) != OR_OK)
             trc = OR_ERR_UNSUPPORTED;
     }
     dir[T] = (uint32_t)(tiles.n / 16);
@@ -990,6 +1155,7 @@ static int encode_at(const double *w, const float *s, const float *scales, int64
         put16(out + 32, (uint32_t)k);
         out[34] = PROB_BITS;
         out[35] = NCTX;
+        out[43] = (uint8_t)C.paired;
         for (int c = 0; c < NCTX; c++) {
             out[36 + c] = (uint8_t)m[c];
             put16(out + 44 + 2 * c, ntok[c]);
@@ -1007,7 +1173,7 @@ static int encode_at(const double *w, const float *s, const float *scales, int64
             }
         size_t p = off_freq;
         for (int c = 0; c < NCTX; c++)
-            for (uint32_t t = 0; t < ntok[c]; t++, p += 2)
+            for (uint32_t t = 0; t < tablen[c]; t++, p += 2)
                 put16(out + p, freq[c][t]);
         for (uint32_t t = 0; t <= T; t++)
             put32(out + off_dir + 4 * t, dir[t]);
@@ -1017,6 +1183,7 @@ static int encode_at(const double *w, const float *s, const float *scales, int64
         free(cnt[c]);
         free(freq[c]);
         free(cum[c]);
+        free(C.rare[c]);
     }
     free(tiles.p);
     free(dir);
@@ -1028,7 +1195,7 @@ static int encode_at(const double *w, const float *s, const float *scales, int64
 
 /* ---------------------------------- compress ----------------------------------------- */
 int or_compress(const void *src, int32_t sdt, int64_t rows, int64_t cols, double target, int32_t container,
-                uint32_t K, int32_t q_override, uint8_t *out, size_t cap, size_t *out_n)
+                uint32_t K, int32_t q_override, int32_t coding, uint8_t *out, size_t cap, size_t *out_n)
 {
     if (!src || !out_n || rows <= 0 || cols <= 0)
         return OR_ERR_INVALID_ARG;
@@ -1038,7 +1205,7 @@ int or_compress(const void *src, int32_t sdt, int64_t rows, int64_t cols, double
         container = sdt;
     if (container < ORD_BF16 || container > ORD_FP8E4M3)
         return OR_ERR_INVALID_ARG;
-    if (K > 4096)
+    if (K > 4096 || coding < OR_CODING_AUTO || coding > OR_CODING_PAIRED)
         return OR_ERR_INVALID_ARG;
     for (int64_t i = 0; i < rows * cols; i++)
         if (!isfinite(src_value(src, sdt, i)))
@@ -1062,7 +1229,7 @@ int or_compress(const void *src, int32_t sdt, int64_t rows, int64_t cols, double
         int32_t lo = 0, hi = kmax;
         while (lo < hi) {
             int32_t mid = lo + (hi - lo + 1) / 2;
-            if (estimate_bpp(wp, s, rows, cols, container, mid, K) <= budget)
+            if (estimate_bpp(wp, s, rows, cols, container, mid, K, coding) <= budget)
                 lo = mid;
             else
                 hi = mid - 1;
@@ -1072,11 +1239,11 @@ int or_compress(const void *src, int32_t sdt, int64_t rows, int64_t cols, double
     int rc;
     for (;;) {
         size_t n = 0;
-        rc = encode_at(wp, s, scales, rows, cols, sdt, container, k, K, NULL, 0, &n);
+        rc = encode_at(wp, s, scales, rows, cols, sdt, container, k, K, coding, NULL, 0, &n);
         if (rc == OR_ERR_UNSUPPORTED)
             break;
         if (q_override >= 0 || 8.0 * (double)n <= target * (double)(rows * cols)) {
-            rc = encode_at(wp, s, scales, rows, cols, sdt, container, k, K, out, cap, out_n);
+            rc = encode_at(wp, s, scales, rows, cols, sdt, container, k, K, coding, out, cap, out_n);
             break;
         }
         if (k == 0) {
@@ -1119,6 +1286,9 @@ int or_parse(const uint8_t *p, size_t n, or_info *info)
     int64_t T = (nb + (int64_t)LANES * info->blocks_per_lane - 1) / ((int64_t)LANES * info->blocks_per_lane);
     if (T != (int64_t)info->n_tiles)
         return OR_ERR_CORRUPT;
+    if (p[43] > 1)
+        return OR_ERR_CORRUPT;
+    info->paired = p[43];
     uint64_t total_tokens = 0;
     for (int c = 0; c < NCTX; c++) {
         info->split[c] = p[36 + c];
@@ -1126,7 +1296,15 @@ int or_parse(const uint8_t *p, size_t n, or_info *info)
         if (info->split[c] < H_BITS + CTX_LOW[c] || info->split[c] > CTX_MAX_SPLIT[c] ||
             info->ntok[c] > or_alphabet_size(info->split[c], CTX_LOW[c]))
             return OR_ERR_CORRUPT;
-        total_tokens += info->ntok[c];
+        if (info->paired && info->split[c] > CTX_NARROW_SPLIT[c])
+            return OR_ERR_CORRUPT;
+        if (info->paired && (c == 1 || c == 2)) {
+            if (info->split[c] > PAIR_MAX_SPLIT)
+                return OR_ERR_CORRUPT;
+            total_tokens += pair_table_len(info->ntok[c]);
+        } else {
+            total_tokens += info->ntok[c];
+        }
     }
     info->off_rowf = HEADER_BYTES;
     info->off_scales = info->off_rowf + al16((size_t)info->rows * 4);
@@ -1135,16 +1313,18 @@ int or_parse(const uint8_t *p, size_t n, or_info *info)
     info->off_tiles = info->off_dir + al16(((size_t)T + 1) * 4);
     if (info->off_tiles > n)
         return OR_ERR_CORRUPT;
-    /* tables sum to M, every frequency below M */
+    /* tables sum to M, every frequency below M (2^12 for pair tables) */
     size_t q = info->off_freq;
     for (int c = 0; c < NCTX; c++) {
+        int pair = info->paired && (c == 1 || c == 2);
+        uint32_t len = pair ? pair_table_len(info->ntok[c]) : info->ntok[c], M = pair ? PAIR_M : PROB_M;
         uint32_t sum = 0;
-        for (uint32_t t = 0; t < info->ntok[c]; t++, q += 2) {
-            if (get16(p + q) >= PROB_M)
+        for (uint32_t t = 0; t < len; t++, q += 2) {
+            if (get16(p + q) >= M)
                 return OR_ERR_CORRUPT;
             sum += get16(p + q);
         }
-        if (info->ntok[c] && sum != PROB_M)
+        if (len && sum != M)
             return OR_ERR_CORRUPT;
     }
     /* directory: starts at 0, each tile holds at least its states, ends at the blob end */
@@ -1166,8 +1346,9 @@ int or_parse(const uint8_t *p, size_t n, or_info *info)
 typedef struct {
     or_info in;
     const uint8_t *p;
-    uint16_t *slot_tok[NCTX]; /* slot -> token (0xffff: slot outside the table) */
+    uint16_t *slot_tok[NCTX]; /* slot -> symbol (0xffff: slot outside the table) */
     uint32_t *freq[NCTX], *cum[NCTX];
+    uint32_t len[NCTX], bits[NCTX]; /* table length; the table sums to 2^bits */
     const uint8_t *rowf;
     int32_t out_dtype; /* the container's dtype unless a float output dtype is asked for */
 } dec_ctx;
@@ -1182,11 +1363,15 @@ static int dec_open(dec_ctx *D, const uint8_t *p, size_t n)
     D->out_dtype = D->in.container_dtype;
     size_t q = D->in.off_freq;
     for (int c = 0; c < NCTX; c++) {
-        uint32_t nt = D->in.ntok[c];
-        D->slot_tok[c] = (uint16_t *)malloc(PROB_M * sizeof(uint16_t));
+        int pair = D->in.paired && (c == 1 || c == 2);
+        uint32_t nt = pair ? pair_table_len(D->in.ntok[c]) : D->in.ntok[c];
+        uint32_t M = pair ? PAIR_M : PROB_M;
+        D->len[c] = nt;
+        D->bits[c] = pair ? PAIR_BITS : PROB_BITS;
+        D->slot_tok[c] = (uint16_t *)malloc(M * sizeof(uint16_t));
         D->freq[c] = (uint32_t *)calloc(nt + 1, sizeof(uint32_t));
         D->cum[c] = (uint32_t *)calloc(nt + 1, sizeof(uint32_t));
-        for (uint32_t s = 0; s < PROB_M; s++)
+        for (uint32_t s = 0; s < M; s++)
             D->slot_tok[c][s] = 0xffff;
         uint32_t a = 0;
         for (uint32_t t = 0; t < nt; t++, q += 2) {
@@ -1209,19 +1394,20 @@ static void dec_close(dec_ctx *D)
     }
 }
 
-/* one lane's rANS step for a table symbol; returns the token */
+/* one lane's rANS step for a table symbol; returns the symbol */
 static uint32_t dec_token(dec_ctx *D, uint32_t c, uint32_t *x, uint32_t *status, double *ideal)
 {
-    uint32_t slot = *x & (PROB_M - 1);
+    uint32_t n = D->bits[c];
+    uint32_t slot = *x & ((1u << n) - 1u);
     uint32_t t = D->slot_tok[c][slot];
     if (t == 0xffff) {
         *status |= OR_DEC_BAD_TOKEN;
         return 0;
     }
     uint32_t f = D->freq[c][t];
-    *x = f * (*x >> PROB_BITS) + slot - D->cum[c][t];
+    *x = f * (*x >> n) + slot - D->cum[c][t];
     if (ideal)
-        *ideal += -log2((double)f / (double)PROB_M);
+        *ideal += -log2((double)f / (double)(1u << n));
     return t;
 }
 
@@ -1299,19 +1485,77 @@ static void decode_tile(dec_ctx *D, int64_t t, int32_t *vout, void *out, uint32_
                 break;
             uint32_t tok[8], ctx[8], sv[8];
             int32_t c = 0, p = 0;
-            for (int i = 0; i < 8; i++) {
-                ctx[i] = i == 0 ? 0u : i < 7 ? 1u + (uint32_t)c : 3u + 2u * (uint32_t)c + (uint32_t)p;
-                tok[i] = dec_token(D, ctx[i], &x, status, cs ? &cs->ideal : NULL);
+            if (!I->paired) {
+                for (int i = 0; i < 8; i++) {
+                    ctx[i] = i == 0 ? 0u : i < 7 ? 1u + (uint32_t)c : 3u + 2u * (uint32_t)c + (uint32_t)p;
+                    tok[i] = dec_token(D, ctx[i], &x, status, cs ? &cs->ideal : NULL);
+                    dec_renorm(&x, wp, avail, &pos, status);
+                    if (tok[i] >= I->ntok[ctx[i]])
+                        *status |= OR_DEC_BAD_TOKEN;
+                    if (cs) {
+                        cs->tokcount[ctx[i]][tok[i] < D->len[ctx[i]] ? tok[i] : 0]++;
+                        cs->nsym++;
+                    }
+                    /* the value's low bits do not depend on the extra bits (they are in the token) */
+                    uint32_t lowbits = or_detokenize(tok[i], I->split[ctx[i]], CTX_LOW[ctx[i]], 0);
+                    if (i == 0) {
+                        c = (int32_t)(lowbits & 1u);
+                        p = (int32_t)((lowbits >> 1) & 1u);
+                    } else if (i < 7) {
+                        p ^= (int32_t)(lowbits & 1u);
+                    }
+                }
+            } else {
+                /* paired: token 0, three pair symbols, the escaped pairs' tokens from the raw
+                 * bits, token 7 */
+                ctx[0] = 0;
+                tok[0] = dec_token(D, 0, &x, status, cs ? &cs->ideal : NULL);
                 dec_renorm(&x, wp, avail, &pos, status);
-                if (tok[i] >= I->ntok[ctx[i]])
+                if (tok[0] >= I->ntok[0])
                     *status |= OR_DEC_BAD_TOKEN;
-                /* the value's low bits do not depend on the extra bits (they are in the token) */
-                uint32_t lowbits = or_detokenize(tok[i], I->split[ctx[i]], CTX_LOW[ctx[i]], 0);
-                if (i == 0) {
-                    c = (int32_t)(lowbits & 1u);
-                    p = (int32_t)((lowbits >> 1) & 1u);
-                } else if (i < 7) {
-                    p ^= (int32_t)(lowbits & 1u);
+                uint32_t low0 = or_detokenize(tok[0], I->split[0], CTX_LOW[0], 0);
+                c = (int32_t)(low0 & 1u);
+                p = (int32_t)((low0 >> 1) & 1u);
+                uint32_t pc = 1u + (uint32_t)c, A = I->ntok[pc], B = pair_base(A), sym[3];
+                for (int j = 0; j < 3; j++) {
+                    sym[j] = dec_token(D, pc, &x, status, cs ? &cs->ideal : NULL);
+                    dec_renorm(&x, wp, avail, &pos, status);
+                    if (sym[j] >= D->len[pc])
+                        *status |= OR_DEC_BAD_TOKEN;
+                    if (cs) {
+                        cs->tokcount[pc][sym[j] < D->len[pc] ? sym[j] : 0]++;
+                        cs->nsym++;
+                    }
+                }
+                for (int j = 0; j < 3; j++) {
+                    uint32_t ta = 0, tb = 0;
+                    if (A && sym[j] == B * B) {
+                        ta = raw_read(&R, pair_raw_bits(A), status);
+                        tb = raw_read(&R, pair_raw_bits(A), status);
+                        if (ta >= A || tb >= A)
+                            *status |= OR_DEC_BAD_TOKEN;
+                        if (cs)
+                            cs->extra += 2.0 * pair_raw_bits(A);
+                    } else if (A) {
+                        ta = sym[j] / B;
+                        tb = sym[j] % B;
+                    }
+                    tok[1 + 2 * j] = ta;
+                    tok[2 + 2 * j] = tb;
+                }
+                for (int i = 1; i < 7; i++) {
+                    ctx[i] = pc;
+                    p ^= (int32_t)(or_detokenize(tok[i], I->split[pc], CTX_LOW[pc], 0) & 1u);
+                }
+                ctx[7] = 3u + 2u * (uint32_t)c + (uint32_t)p;
+                tok[7] = dec_token(D, ctx[7], &x, status, cs ? &cs->ideal : NULL);
+                dec_renorm(&x, wp, avail, &pos, status);
+                if (tok[7] >= I->ntok[ctx[7]])
+                    *status |= OR_DEC_BAD_TOKEN;
+                if (cs) {
+                    cs->tokcount[0][tok[0] < D->len[0] ? tok[0] : 0]++;
+                    cs->tokcount[ctx[7]][tok[7] < D->len[ctx[7]] ? tok[7] : 0]++;
+                    cs->nsym += 2;
                 }
             }
             for (int i = 0; i < 8; i++) {
@@ -1319,11 +1563,8 @@ static void decode_tile(dec_ctx *D, int64_t t, int32_t *vout, void *out, uint32_
                 uint32_t nbits = token_extra_bits(tok[i], m, low);
                 uint32_t extra = raw_read(&R, nbits, status);
                 sv[i] = or_detokenize(tok[i], m, low, extra);
-                if (cs) {
-                    cs->tokcount[ctx[i]][tok[i] < I->ntok[ctx[i]] ? tok[i] : 0]++;
+                if (cs)
                     cs->extra += nbits;
-                    cs->nsym++;
-                }
             }
             int32_t v[8];
             uint32_t ctx2[8];
@@ -1406,15 +1647,15 @@ int or_code_stats(const uint8_t *blob, size_t n, double *ideal_bits, double *emp
     code_stats cs;
     memset(&cs, 0, sizeof cs);
     for (int c = 0; c < NCTX; c++)
-        cs.tokcount[c] = (uint64_t *)calloc(D.in.ntok[c] + 1, sizeof(uint64_t));
+        cs.tokcount[c] = (uint64_t *)calloc(D.len[c] + 1, sizeof(uint64_t));
     for (uint32_t t = 0; t < D.in.n_tiles; t++)
         decode_tile(&D, t, NULL, NULL, &st, &cs);
     double H = 0.0;
     for (int c = 0; c < NCTX; c++) {
         uint64_t tot = 0;
-        for (uint32_t t = 0; t < D.in.ntok[c]; t++)
+        for (uint32_t t = 0; t < D.len[c]; t++)
             tot += cs.tokcount[c][t];
-        for (uint32_t t = 0; t < D.in.ntok[c]; t++)
+        for (uint32_t t = 0; t < D.len[c]; t++)
             if (cs.tokcount[c][t])
                 H += (double)cs.tokcount[c][t] * log2((double)tot / (double)cs.tokcount[c][t]);
         free(cs.tokcount[c]);

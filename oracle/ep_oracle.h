@@ -46,6 +46,10 @@ enum {
     OR_ERR_UNSUPPORTED = -8
 };
 
+/* coding of coordinates 1..6 asked of the compressor: automatic, one token per coordinate,
+ * or paired whenever the token alphabets allow it (any tensor size) */
+enum { OR_CODING_AUTO = 0, OR_CODING_SINGLE = 1, OR_CODING_PAIRED = 2 };
+
 /* decode status bits (stream damage found while decoding a tile) */
 enum {
     OR_DEC_WORD_OVERRUN = 1u,   /* a renormalisation or raw-bit read past the tile's words */
@@ -64,6 +68,7 @@ typedef struct {
     uint8_t split[7];
     uint16_t ntok[7];
     uint64_t off_rowf, off_scales, off_freq, off_dir, off_tiles;
+    uint32_t paired; /* 1: coordinates 1..6 coded as three pairs */
 } or_info;
 
 /* ---- scalar pieces, exposed so that tests can pin them one by one ---- */
@@ -86,6 +91,8 @@ void or_detokenize_batch(const uint32_t *tok, int64_t n, int32_t m, int32_t low,
 void or_tokenize_batch(const uint32_t *s, int64_t n, int32_t m, int32_t low, uint32_t *tok, uint32_t *nbits,
                        uint32_t *extra);
 int32_t or_normalize_freqs(const uint64_t *counts, int32_t n, uint32_t *freqs);
+/* the same rule for tables summing to 2^bits */
+int32_t or_normalize_freqs_to(const uint64_t *counts, int32_t n, int32_t bits, uint32_t *freqs);
 uint32_t or_choose_blocks_per_lane(int64_t nblocks, double target_bpp);
 uint16_t or_bf16_from_float(float w);
 uint16_t or_fp16_from_float(float w);
@@ -105,12 +112,13 @@ int or_quantize(const void *src, int32_t src_dtype, int64_t rows, int64_t cols, 
 /* sampled storage estimate (bits per weight) at resolution index k; blocks_per_lane 0 takes
  * the automatic tile size for a 4 bpp target */
 double or_estimate_bpp(const void *src, int32_t src_dtype, int64_t rows, int64_t cols, int32_t container,
-                       int32_t k, uint32_t blocks_per_lane);
+                       int32_t k, uint32_t blocks_per_lane, int32_t coding);
 
 /* ---- the stream ---- */
-/* q_override >= 0 skips the search and encodes at that index; blocks_per_lane 0 = automatic */
+/* q_override >= 0 skips the search and encodes at that index; blocks_per_lane 0 = automatic;
+ * coding: OR_CODING_* */
 int or_compress(const void *src, int32_t src_dtype, int64_t rows, int64_t cols, double target_bpp,
-                int32_t container, uint32_t blocks_per_lane, int32_t q_override,
+                int32_t container, uint32_t blocks_per_lane, int32_t q_override, int32_t coding,
                 uint8_t *out, size_t cap, size_t *out_nbytes);
 int or_parse(const uint8_t *blob, size_t nbytes, or_info *info);
 /* decodes tiles [t0, t1): lattice points into v (indexed by weight, rows*cols, nullable) and

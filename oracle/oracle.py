@@ -13,6 +13,7 @@ from . import build as _build
 BF16, FP16, FP32, INT8, FP8E4M3 = 1, 2, 3, 4, 5
 OK, ERR_INVALID_ARG, ERR_NONFINITE, ERR_TARGET_RANGE, ERR_TARGET_UNREACHABLE = 0, -1, -2, -3, -4
 ERR_BUFFER_TOO_SMALL, ERR_CORRUPT, ERR_UNSUPPORTED = -5, -6, -8
+CODING_AUTO, CODING_SINGLE, CODING_PAIRED = 0, 1, 2
 ELT = {BF16: 2, FP16: 2, FP32: 4, INT8: 1, FP8E4M3: 1}
 NP_DTYPE = {BF16: np.uint16, FP16: np.uint16, FP32: np.float32, INT8: np.int8, FP8E4M3: np.uint8}
 
@@ -26,7 +27,7 @@ class Info(C.Structure):
         ("n_tiles", C.c_uint32), ("blocks_per_lane", C.c_uint32),
         ("split", C.c_uint8 * 7), ("ntok", C.c_uint16 * 7),
         ("off_rowf", C.c_uint64), ("off_scales", C.c_uint64), ("off_freq", C.c_uint64),
-        ("off_dir", C.c_uint64), ("off_tiles", C.c_uint64),
+        ("off_dir", C.c_uint64), ("off_tiles", C.c_uint64), ("paired", C.c_uint32),
     ]
 
 
@@ -59,6 +60,8 @@ def lib():
         L.or_block_values.argtypes = [p, p, p]
         L.or_normalize_freqs.restype = C.c_int32
         L.or_normalize_freqs.argtypes = [p, C.c_int32, p]
+        L.or_normalize_freqs_to.restype = C.c_int32
+        L.or_normalize_freqs_to.argtypes = [p, C.c_int32, C.c_int32, p]
         L.or_choose_blocks_per_lane.restype = C.c_uint32
         L.or_choose_blocks_per_lane.argtypes = [C.c_int64, C.c_double]
         L.or_convert_batch.argtypes = [p, C.c_int64, C.c_int32, p]
@@ -68,10 +71,11 @@ def lib():
         L.or_quantize.restype = C.c_int
         L.or_quantize.argtypes = [p, C.c_int32, C.c_int64, C.c_int64, C.c_int32, C.c_int32, p]
         L.or_estimate_bpp.restype = C.c_double
-        L.or_estimate_bpp.argtypes = [p, C.c_int32, C.c_int64, C.c_int64, C.c_int32, C.c_int32, C.c_uint32]
+        L.or_estimate_bpp.argtypes = [p, C.c_int32, C.c_int64, C.c_int64, C.c_int32, C.c_int32, C.c_uint32,
+                                      C.c_int32]
         L.or_compress.restype = C.c_int
         L.or_compress.argtypes = [p, C.c_int32, C.c_int64, C.c_int64, C.c_double, C.c_int32, C.c_uint32,
-                                  C.c_int32, p, C.c_size_t, C.POINTER(C.c_size_t)]
+                                  C.c_int32, C.c_int32, p, C.c_size_t, C.POINTER(C.c_size_t)]
         L.or_parse.restype = C.c_int
         L.or_parse.argtypes = [p, C.c_size_t, C.POINTER(Info)]
         L.or_decode.restype = C.c_int
@@ -190,10 +194,10 @@ def block_values(s):
     return v, ctx
 
 
-def normalize_freqs(counts):
+def normalize_freqs(counts, bits=11):
     c = np.ascontiguousarray(counts, dtype=np.uint64)
     f = np.zeros(c.size, np.uint32)
-    n = lib().or_normalize_freqs(_ptr(c), c.size, _ptr(f))
+    n = lib().or_normalize_freqs_to(_ptr(c), c.size, int(bits), _ptr(f))
     return f, n
 
 
@@ -234,25 +238,26 @@ def quantize(src, k, container=0):
     return v
 
 
-def estimate_bpp(src, k, container=0, blocks_per_lane=0):
+def estimate_bpp(src, k, container=0, blocks_per_lane=0, coding=CODING_AUTO):
     a, dt = _src(src)
     R, Cc = a.shape
-    return lib().or_estimate_bpp(_ptr(a), dt, R, Cc, container or dt, int(k), blocks_per_lane)
+    return lib().or_estimate_bpp(_ptr(a), dt, R, Cc, container or dt, int(k), blocks_per_lane, int(coding))
 
 
 # ---- the stream ----
-def compress(src, target_bpp, container=0, blocks_per_lane=0, q_override=-1):
-    """Returns (rc, blob as a uint8 numpy array)."""
+def compress(src, target_bpp, container=0, blocks_per_lane=0, q_override=-1, coding=CODING_AUTO):
+    """Returns (rc, blob as a uint8 numpy array).  ``coding``: CODING_AUTO, CODING_SINGLE or
+    CODING_PAIRED (coordinates 1..6 paired whenever the alphabets allow, at any size)."""
     a, dt = _src(src)
     R, Cc = a.shape
     n = C.c_size_t(0)
     rc = lib().or_compress(_ptr(a), dt, R, Cc, float(target_bpp), container, blocks_per_lane, q_override,
-                           None, 0, C.byref(n))
+                           int(coding), None, 0, C.byref(n))
     if rc not in (OK, ERR_BUFFER_TOO_SMALL):
         return rc, None
     out = np.zeros(n.value, np.uint8)
     rc = lib().or_compress(_ptr(a), dt, R, Cc, float(target_bpp), container, blocks_per_lane, q_override,
-                           _ptr(out), out.size, C.byref(n))
+                           int(coding), _ptr(out), out.size, C.byref(n))
     return rc, (out[: n.value] if rc == OK else None)
 
 

@@ -1,5 +1,5 @@
 """Seeded random sweep of GPU parity: shapes (ragged rows included), rates, containers, forced tile
-sizes and output dtypes drawn from a fixed generator; every case is encoded by the ORACLE and the
+sizes, output dtypes and (every third case) paired coding drawn from a fixed generator; every case is encoded by the ORACLE and the
 GPU decode must equal the oracle's decode byte for byte (lattice points and container bytes), and
 the GPU compressor must write the oracle's stream for the same tensor."""
 import numpy as np
@@ -26,23 +26,23 @@ def cases(n=40, seed=2024):
         hi = 7.9 if container in (B.INT8, B.FP8E4M3) else 11.0
         target = float(np.round(rng.uniform(0.3, hi), 2))
         K = int(rng.choice([0, 0, 1, 2, 3, 8, 16, 64]))
-        out.append((i, rows, cols, container, target, K))
+        out.append((i, rows, cols, container, target, K, 2 if i % 3 == 1 else 0))
     return out
 
 
-@pytest.mark.parametrize("i,rows,cols,container,target,K", cases(), ids=lambda v: str(v))
-def test_random_case(oracle, i, rows, cols, container, target, K):
+@pytest.mark.parametrize("i,rows,cols,container,target,K,coding", cases(), ids=lambda v: str(v))
+def test_random_case(oracle, i, rows, cols, container, target, K, coding):
     w = synth.row_lognormal(rows, cols, seed=1000 + i, dtype=SRC[container])
     if i % 3 == 0:
         w = synth.gaussian_outliers(rows, cols, seed=1000 + i, dtype=SRC[container])
-    rc, blob = oracle.compress(w, target, container=container, blocks_per_lane=K)
+    rc, blob = oracle.compress(w, target, container=container, blocks_per_lane=K, coding=coding)
     if rc == oracle.ERR_TARGET_UNREACHABLE:
         with pytest.raises(B.EpError):
-            B.compress_device(w.cuda(), target, container=container, blocks_per_lane=K)
+            B.compress_device(w.cuda(), target, container=container, blocks_per_lane=K, coding=coding)
         return
     assert rc == 0
     # the GPU compressor writes the same stream
-    got = B.compress_device(w.cuda(), target, container=container, blocks_per_lane=K).cpu().numpy()
+    got = B.compress_device(w.cuda(), target, container=container, blocks_per_lane=K, coding=coding).cpu().numpy()
     assert np.array_equal(got, blob)
     # the GPU decode equals the oracle's, for the container and the lattice points
     d = torch.from_numpy(blob).cuda()

@@ -32,6 +32,28 @@ CASES = [
 ]
 
 
+PAIRED_CASES = [
+    ("paired_lognormal", lambda: synth.row_lognormal(300, 1000, 7), 3.0, 0, 0),
+    ("paired_outliers", lambda: synth.gaussian_outliers(96, 2048, 2), 3.5, 0, 0),
+    ("paired_outliers_low", lambda: synth.gaussian_outliers(96, 2048, 4), 2.0, 0, 0),
+    ("paired_ragged_K3", lambda: synth.row_lognormal(137, 455, 5), 3.5, 0, 3),
+    ("paired_int8", lambda: synth.gaussian(96, 808, 0.02, 3), 4.0, B.INT8, 0),
+    ("paired_fp8", lambda: synth.gaussian(256, 512, 0.02, 2), 3.0, B.FP8E4M3, 0),
+]
+
+
+@pytest.mark.parametrize("name,make,target,container,K", PAIRED_CASES, ids=[c[0] for c in PAIRED_CASES])
+def test_paired_bytes_identical_to_oracle(oracle, name, make, target, container, K):
+    """paired coding asked for at sizes below the automatic threshold"""
+    w = make()
+    rc, ref = oracle.compress(w, target, container=container, blocks_per_lane=K, coding=oracle.CODING_PAIRED)
+    assert rc == 0
+    assert oracle.parse(ref)[1].paired == 1
+    blob = B.compress(w, target, container=container, blocks_per_lane=K, coding=B.CODING_PAIRED).numpy()
+    assert np.array_equal(blob, ref)
+    assert B.stream_info(torch.from_numpy(blob)).paired == 1
+
+
 @pytest.mark.parametrize("name,make,target,container,K", CASES, ids=[c[0] for c in CASES])
 def test_bytes_identical_to_oracle(oracle, name, make, target, container, K):
     w = make()
