@@ -922,7 +922,9 @@ cudaError_t launch(Params &p, uint64_t max_tile, int mode, int device, cudaStrea
     }
     // one CTA per SM (at most one per tile); warps = tiles per CTA, within kMaxWarps and the
     // tile buffers that fit beside the tables: two per warp when a warp has several tiles and
-    // they fit, else one, else the tiles are read from global memory
+    // they fit, else one; when even one per warp does not fit, fewer warps with one buffer each
+    // (the decode is bound by latency, so warps matter more than overlapping the next copy),
+    // else the tiles are read from global memory
     uint32_t grid = p.T < uint32_t(sms) ? p.T : uint32_t(sms);
     uint32_t warps = (p.T + grid - 1) / grid;
     warps = warps > uint32_t(kMaxWarps) ? uint32_t(kMaxWarps) : warps;
@@ -934,9 +936,6 @@ cudaError_t launch(Params &p, uint64_t max_tile, int mode, int device, cudaStrea
         p.nbuf = 2;
     } else if (uint64_t(warps) * p.tile_buf <= avail) {
         p.nbuf = 1;
-    } else if (uint64_t(p.tile_buf) * 2 * 4 <= avail) {
-        warps = uint32_t(avail / (2ull * p.tile_buf));
-        p.nbuf = 2;
     } else if (p.tile_buf <= avail) {
         warps = uint32_t(avail / p.tile_buf);
         p.nbuf = 1;
@@ -983,7 +982,7 @@ int check_info(const ep_info *info) {
             return EP_ERR_CORRUPT;
         if (info->paired && info->split[c] > kCtxNarrowSplit[c]) return EP_ERR_CORRUPT;
         if (info->paired && (c == 1 || c == 2)) {
-            if (info->split[c] > kPairMaxSplit) return EP_ERR_CORRUPT;
+            if (info->ntok[c] > kPairMaxAlphabet) return EP_ERR_CORRUPT;
             total += pair_table_len(info->ntok[c]);
         } else {
             total += info->ntok[c];

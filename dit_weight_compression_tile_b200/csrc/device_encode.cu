@@ -576,7 +576,7 @@ extern "C" int ep_compress_device(const void *d_src, int32_t src_dtype, int64_t 
         std::vector<uint8_t> rare;
         uint32_t ntok[kContexts], tablen[kContexts], A[kContexts] = {};
         uint64_t tokens = 0;
-        const bool paired = pair_eligible(P.coding, P.nb, sp.m);
+        const bool paired = pair_eligible(P.coding, P.nb, sp.m, cnt[1], cnt[2]);
         std::vector<unsigned long long> pc;
         if (paired) {
             A[1] = seen_len(cnt[1]);

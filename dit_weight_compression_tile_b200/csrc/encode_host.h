@@ -23,8 +23,10 @@ uint32_t build_freqs(const std::vector<uint64_t> &cnt, std::vector<uint32_t> &f,
 // last token seen, plus one
 uint32_t seen_len(const std::vector<uint64_t> &cnt);
 
-// whether a stream pairs coordinates 1..6 (coding: EP_CODING_*; m: the splits)
-bool pair_eligible(int coding, int64_t nb, const uint32_t *m);
+// whether a stream pairs coordinates 1..6 (coding: EP_CODING_*; m: the splits; cnt1, cnt2: the
+// token counts of contexts 1 and 2)
+bool pair_eligible(int coding, int64_t nb, const uint32_t *m, const std::vector<uint64_t> &cnt1,
+                   const std::vector<uint64_t> &cnt2);
 
 // pair table of a context with alphabet length A from the counts of its token pairs inside the
 // base (B * B of them, B = pair_base(A)) and of all its pairs (N): pairs outside the base and rare

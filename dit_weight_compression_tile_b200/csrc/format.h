@@ -30,14 +30,16 @@ constexpr uint32_t kMaxAlphabet = 720;     // (1 << 9) + ((22 - 9) << 2 << 2): t
 // context's token alphabet length and B = min(A, 40), a pair of tokens both below B is index
 // t_a B + t_b of a table of B^2 + 1 symbols summing to 2^12; the last symbol is an escape, taken
 // by pairs with a token at or above B and by pairs seen fewer than N / 2^16 times (N: the
-// context's pair count), whose tokens follow in the raw bits.  Contexts 1 and 2 are paired up to
-// split 5.  Header byte 43 holds 1 for a paired stream.
+// context's pair count), whose tokens follow in the raw bits.  Contexts 1 and 2 are paired while
+// their alphabets have at most 256 tokens and at most 1 / 2^12 of their tokens lie at or beyond
+// the base 40.  Header byte 43 holds 1 for a paired stream.
 constexpr uint32_t kPairBits = 12;
 constexpr uint32_t kPairScale = 1u << kPairBits;
 constexpr uint32_t kPairBaseMax = 40;
-constexpr uint32_t kPairMaxSplit = 5;
+constexpr uint32_t kPairMaxAlphabet = 256;
+constexpr uint64_t kPairOutsideScale = 4096;
 constexpr uint32_t kPairMaxTable = kPairBaseMax * kPairBaseMax + 1;
-constexpr uint32_t kPairTokFields = 256;  // token fields per coset in the decoder's tables (A <= 168)
+constexpr uint32_t kPairTokFields = kPairMaxAlphabet;  // token fields per coset in the decoder's tables
 constexpr int64_t kPairMinBlocks = int64_t(1) << 17;  // automatic coding pairs from this many blocks on
 constexpr uint64_t kPairRareScale = 65536;            // a pair seen c times is escaped when c 2^16 < N
 // the decoder's tables for a paired stream: token tables of contexts 0, 3..6 (2048 4-byte slots

@@ -158,12 +158,21 @@ uint32_t seen_len(const std::vector<uint64_t> &cnt) {
 }
 
 // pairs when asked to (EP_CODING_PAIRED) or, automatically, from 2^17 blocks on; in both cases
-// only with splits of contexts 1 and 2 up to 5 and splits that keep every coordinate in [-256, 255]
-bool pair_eligible(int coding, int64_t nb, const uint32_t *m) {
+// only with splits that keep every coordinate in [-256, 255], alphabets of contexts 1 and 2 of at
+// most 256 tokens and at most 1 / 2^12 of their tokens at or beyond the base
+bool pair_eligible(int coding, int64_t nb, const uint32_t *m, const std::vector<uint64_t> &cnt1,
+                   const std::vector<uint64_t> &cnt2) {
     if (coding == EP_CODING_SINGLE) return false;
     for (int c = 0; c < kContexts; ++c)
         if (m[c] > kCtxNarrowSplit[c]) return false;
-    if (m[1] > kPairMaxSplit || m[2] > kPairMaxSplit) return false;
+    for (const std::vector<uint64_t> *cnt : {&cnt1, &cnt2}) {
+        uint64_t all = 0, outside = 0;
+        for (size_t t = 0; t < cnt->size(); ++t) {
+            all += (*cnt)[t];
+            if (t >= kPairBaseMax) outside += (*cnt)[t];
+        }
+        if (seen_len(*cnt) > kPairMaxAlphabet || outside * kPairOutsideScale > all) return false;
+    }
     return coding == EP_CODING_PAIRED || nb >= kPairMinBlocks;
 }
 
@@ -192,7 +201,7 @@ double estimate_from_counts(const std::vector<uint64_t> *cnt, const uint32_t *m,
     uint64_t tokens = 0;
     // a paired stream stores pair tables for contexts 1 and 2; its payload is estimated by the
     // same token entropy
-    const bool paired = pair_eligible(coding, nb, m);
+    const bool paired = pair_eligible(coding, nb, m, cnt[1], cnt[2]);
     for (int c = 0; c < kContexts; ++c) {
         uint64_t n = 0;
         for (size_t t = 0; t < cnt[c].size(); ++t) n += cnt[c][t];
@@ -502,7 +511,7 @@ struct Encoder {
             for (auto &pc : part_cnt)
                 for (size_t t = 0; t < cnt[c].size(); ++t) cnt[c][t] += pc[size_t(c) * kMaxAlphabet + t];
         }
-        const bool paired = pair_eligible(coding, nb, m);
+        const bool paired = pair_eligible(coding, nb, m, cnt[1], cnt[2]);
         for (int c = 0; c < kContexts; ++c) {
             if (paired && (c == 1 || c == 2)) {
                 // counts of the token pairs of coordinates (1,2), (3,4), (5,6) inside the base

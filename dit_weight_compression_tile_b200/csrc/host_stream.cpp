@@ -51,10 +51,10 @@ extern "C" int ep_stream_info(const void *blob, size_t nbytes, ep_info *info) {
         I.split[c] = p[36 + c];
         I.ntok[c] = uint16_t(rd(p + 44 + 2 * c, 2));
         if (!split_valid(I.split[c], c) || I.ntok[c] > split_alphabet(I.split[c], kCtxLow[c])) return EP_ERR_CORRUPT;
-        // a paired stream keeps every split in the narrow range and pairs splits up to 5
+        // a paired stream keeps every split in the narrow range and pairs alphabets of <= 256 tokens
         if (I.paired && I.split[c] > kCtxNarrowSplit[c]) return EP_ERR_CORRUPT;
         const bool pair = I.paired && (c == 1 || c == 2);
-        if (pair && I.split[c] > kPairMaxSplit) return EP_ERR_CORRUPT;
+        if (pair && I.ntok[c] > kPairMaxAlphabet) return EP_ERR_CORRUPT;
         tablen[c] = pair ? pair_table_len(I.ntok[c]) : I.ntok[c];
         tokens += tablen[c];
     }

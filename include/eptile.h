@@ -77,10 +77,10 @@ typedef struct {
 } ep_config;
 
 /* EP_CODING_AUTO pairs coordinates (1,2), (3,4), (5,6) of every block into one symbol each
- * when the stream holds at least 2^17 blocks and the token splits of their contexts are at most
- * 5 (about 4.5 bpp and below): 5 table lookups per block instead of 8 in the decoder, for well
- * under 1 % more bits at 4 bpp; EP_CODING_SINGLE never pairs; EP_CODING_PAIRED pairs whenever the
- * splits allow, at any size. */
+ * when the stream holds at least 2^17 blocks and the tokens of their contexts concentrate below
+ * 40 (at most 1 / 2^12 of them beyond, alphabets of at most 256 tokens; about 4.5 bpp and below):
+ * 5 table lookups per block instead of 8 in the decoder, for well under 1 % more bits at 4 bpp;
+ * EP_CODING_SINGLE never pairs; EP_CODING_PAIRED pairs whenever the tokens allow, at any size. */
 enum ep_coding { EP_CODING_AUTO = 0, EP_CODING_SINGLE = 1, EP_CODING_PAIRED = 2 };
 
 typedef struct {

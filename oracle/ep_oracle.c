@@ -60,8 +60,9 @@ static const int32_t CTX_MAX_SPLIT[NCTX] = {9, 9, 9, 8, 8, 8, 8};
 /* splits up to which every directly coded coordinate v itself lies in [-256, 255] */
 static const int32_t CTX_NARROW_SPLIT[NCTX] = {9, 8, 8, 7, 7, 7, 7};
 
-/* Paired coding (a reading of the pages' conditional model, which they leave open): with small
- * splits, coordinates (1,2), (3,4) and (5,6) of a block are coded as one symbol each.  With A the
+/* Paired coding (a reading of the pages' conditional model, which they leave open): when the
+ * tokens of contexts 1 and 2 concentrate below 40, coordinates (1,2), (3,4) and (5,6) of a block
+ * are coded as one symbol each.  With A the
  * context's token alphabet length and B = min(A, 40), a pair of tokens both below B is symbol
  * t_a B + t_b of a table of B^2 + 1 symbols summing to 2^12; the last symbol is an escape, taken
  * by pairs with a token at or above B and by pairs seen fewer than N / 2^16 times (N: the
@@ -69,7 +70,8 @@ static const int32_t CTX_NARROW_SPLIT[NCTX] = {9, 8, 8, 7, 7, 7, 7};
 #define PAIR_BITS 12
 #define PAIR_M 4096u
 #define PAIR_BASE_MAX 40u           /* largest pair base B */
-#define PAIR_MAX_SPLIT 5            /* contexts 1 and 2 are paired up to this split */
+#define PAIR_MAX_ALPHABET 256u      /* contexts 1 and 2 are paired up to this alphabet length */
+#define PAIR_OUTSIDE_SCALE 4096u    /* ... and while at most 1 / 2^12 of their tokens lie beyond the base */
 #define PAIR_MIN_BLOCKS (1 << 17)   /* automatic coding pairs tensors of at least this many blocks */
 #define PAIR_RARE_SCALE 65536u      /* a pair seen c times is escaped when c * 2^16 < N */
 
@@ -549,17 +551,29 @@ static uint32_t seen_len(const uint64_t *cnt, uint32_t n)
 
 /* The stream pairs coordinates 1..6 when it is asked to (OR_CODING_PAIRED) or, under automatic
  * coding, when it holds at least 2^17 blocks (the pair tables then cost under 1 % of a 4-bit
- * stream); in both cases only when the splits of contexts 1 and 2 are at most 5 (their direct
- * tokens fit the pair base) and every split keeps the coordinates' values in [-256, 255]. */
-static int pair_eligible(int32_t coding, int64_t nb, const int32_t *m)
+ * stream); in both cases only when every split keeps the coordinates' values in [-256, 255],
+ * the alphabets of contexts 1 and 2 have at most 256 tokens and at most 1 / 2^12 of their tokens
+ * (counted in cnt[1], cnt[2], of lengths n1, n2) lie at or beyond the base 40. */
+static int pair_eligible(int32_t coding, int64_t nb, const int32_t *m, const uint64_t *cnt1, uint32_t n1,
+                         const uint64_t *cnt2, uint32_t n2)
 {
     if (coding == OR_CODING_SINGLE)
         return 0;
     for (int c = 0; c < NCTX; c++)
         if (m[c] > CTX_NARROW_SPLIT[c])
             return 0;
-    if (m[1] > PAIR_MAX_SPLIT || m[2] > PAIR_MAX_SPLIT)
-        return 0;
+    const uint64_t *cnt[2] = {cnt1, cnt2};
+    uint32_t n[2] = {n1, n2};
+    for (int c = 0; c < 2; c++) {
+        uint64_t all = 0, outside = 0;
+        for (uint32_t t = 0; t < n[c]; t++) {
+            all += cnt[c][t];
+            if (t >= PAIR_BASE_MAX)
+                outside += cnt[c][t];
+        }
+        if (seen_len(cnt[c], n[c]) > PAIR_MAX_ALPHABET || outside * PAIR_OUTSIDE_SCALE > all)
+            return 0;
+    }
     return coding == OR_CODING_PAIRED || nb >= PAIR_MIN_BLOCKS;
 }
 
@@ -792,7 +806,8 @@ static double estimate_bpp(const double *w, const float *s, int64_t rows, int64_
         lens[c] = seen_len(cnt[c], or_alphabet_size(m[c], CTX_LOW[c]));
     /* a paired stream stores pair tables for contexts 1 and 2; its payload is estimated by
      * the same token entropy */
-    int paired = pair_eligible(coding, nb, m);
+    int paired = pair_eligible(coding, nb, m, cnt[1], or_alphabet_size(m[1], CTX_LOW[1]), cnt[2],
+                               or_alphabet_size(m[2], CTX_LOW[2]));
     for (int c = 0; c < NCTX; c++) {
         uint64_t n = 0;
         for (uint32_t t = 0; t < or_alphabet_size(m[c], CTX_LOW[c]); t++)
@@ -1067,7 +1082,7 @@ static int encode_at(const double *w, const float *s, const float *scales, int64
     coder C;
     memset(&C, 0, sizeof C);
     uint32_t tablen[NCTX];
-    C.paired = pair_eligible(coding, nb, m);
+    C.paired = pair_eligible(coding, nb, m, cnt[1], alpha[1], cnt[2], alpha[2]);
     for (int c = 0; c < NCTX; c++) {
         C.m[c] = m[c];
         if (C.paired && (c == 1 || c == 2)) {
@@ -1299,7 +1314,7 @@ int or_parse(const uint8_t *p, size_t n, or_info *info)
         if (info->paired && info->split[c] > CTX_NARROW_SPLIT[c])
             return OR_ERR_CORRUPT;
         if (info->paired && (c == 1 || c == 2)) {
-            if (info->split[c] > PAIR_MAX_SPLIT)
+            if (info->ntok[c] > PAIR_MAX_ALPHABET)
                 return OR_ERR_CORRUPT;
             total_tokens += pair_table_len(info->ntok[c]);
         } else {

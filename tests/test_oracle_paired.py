@@ -57,15 +57,15 @@ def test_paired_and_single_give_the_same_points(oracle):
 
 
 def test_automatic_choice(oracle):
-    """automatic coding pairs from 2^17 blocks on, with splits of contexts 1 and 2 up to 5"""
+    """automatic coding pairs from 2^17 blocks on, when the tokens of contexts 1 and 2 concentrate
+    below the base 40"""
     big = synth.row_lognormal(1024, 1024, seed=1)        # 131072 blocks
     small = synth.row_lognormal(1024, 1016, seed=1)      # 130048 blocks
     b1, i1 = compress(oracle, big, 4.0, oracle.CODING_AUTO)
     b2, i2 = compress(oracle, small, 4.0, oracle.CODING_AUTO)
     assert i1.paired == 1 and i2.paired == 0
-    assert i1.split[1] <= 5 and i1.split[2] <= 5
-    b3, i3 = compress(oracle, big, 8.0, oracle.CODING_AUTO)   # splits far above 5
-    assert i3.paired == 0 and i3.split[1] > 5
+    b3, i3 = compress(oracle, big, 8.0, oracle.CODING_AUTO)   # most tokens far beyond 40
+    assert i3.paired == 0 and i3.ntok[1] > 40
     b4, i4 = compress(oracle, big, 8.0, oracle.CODING_PAIRED)  # asked for, but not possible
     assert i4.paired == 0
     for blob, info in ((b1, i1), (b3, i3)):
