@@ -202,7 +202,7 @@ int ep_decompress(const ep_info *info, const void *d_blob, const void *d_workspa
  * that must not trigger the device-wide synchronisation a cudaMalloc/cudaFree can cause.  No
  * counterpart in the EntroPack pages; it exists for such callers only.
  *   Arguments as ep_decompress, without a workspace: the slot tables go to one file-scope device
- *   array of 57,344 bytes (info->workspace_nbytes of every stream), which each GPU that loads the
+ *   array of 108,544 bytes (info->workspace_nbytes of every stream), which each GPU that loads the
  *   library keeps until the process exits.  A stream needing more returns EP_ERR_UNSUPPORTED.
  *   The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
  *   that device current; make that first call before any stream capture.
