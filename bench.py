@@ -81,6 +81,12 @@ def args_():
     return a
 
 
+def coding_label(infos):
+    """how the workload's streams code coordinates 1..6: paired, single or mixed"""
+    paired = sum(1 for i in infos if i.paired)
+    return "paired" if paired == len(infos) else ("single" if paired == 0 else "mixed")
+
+
 def workload_config(a):
     wl = WORKLOADS[a.workload]
     return {"workload": a.workload, "shape": wl["shape"], "target_bpp": a.target,
@@ -422,7 +428,8 @@ def run_ours(a, rank, world, local_rank):
                        l2=(f"inputs larger than L2: {rot} rotating stream+output copies "
                            f"({rot * (in_bytes + out_bytes) / 1e6:.0f} MB)") if rot > 1 else
                           f"inputs larger than L2: {(in_bytes + out_bytes) / 1e6:.0f} MB per step",
-                       actual_bpp=round(8.0 * in_bytes / n_weights, 4), n_tensors=len(infos),
+                       actual_bpp=round(8.0 * in_bytes / n_weights, 4), coding=coding_label(infos),
+                       n_tensors=len(infos),
                        n_tiles=sum(i.n_tiles for i in infos), blocks_per_lane=i0.blocks_per_lane,
                        parallelism="replicas" if world > 1 else "single"),
         "gweights_per_s": round(job_rate(n_weights, world, step_s) / 1e9, 3),
