@@ -26,11 +26,14 @@ class LatticeRANSConfig:
     """target_bpp: stored bits per element including metadata, in [0.001, 11] ([0.001, 8) for
     code containers).  container: None (the source dtype) or torch.int8 / torch.float8_e4m3fn
     (per-row absmax codes; the rate then counts the row scales).  blocks_per_lane: 0 picks it
-    from the shape.  n_threads: host encoder threads (0: all cores)."""
+    from the shape.  n_threads: host encoder threads (0: all cores).  coding: 0 automatic, 1 one
+    token per coordinate, 2 coordinates 1..6 in pairs whenever their tokens allow (the decoder
+    then does 5 table lookups per E8 block instead of 8)."""
     target_bpp: float = 4.0
     container: object = None
     blocks_per_lane: int = 0
     n_threads: int = 0
+    coding: int = 0
 
 
 class CompressedTensor:
@@ -168,10 +171,11 @@ def compress(tensor, config):
     try:
         if tensor.is_cuda:  # the GPU compressor writes the host compressor's bytes
             blob = B.compress_device(tensor, config.target_bpp, container=container,
-                                     blocks_per_lane=config.blocks_per_lane)
+                                     blocks_per_lane=config.blocks_per_lane, coding=config.coding)
         else:
             blob = B.compress(tensor, config.target_bpp, container=container,
-                              blocks_per_lane=config.blocks_per_lane, n_threads=config.n_threads)
+                              blocks_per_lane=config.blocks_per_lane, n_threads=config.n_threads,
+                              coding=config.coding)
     except B.EpError as e:
         if e.status != -4:  # EP_ERR_TARGET_UNREACHABLE
             raise

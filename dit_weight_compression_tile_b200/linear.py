@@ -10,6 +10,8 @@ The FP8 / INT8 layers hold per-row absmax codes (the stream's code container) an
 activations per row of x the same way (E4M3 with scale amax / 448, INT8 with amax / 127, RNE);
 the GEMM multiplies codes and applies both scales to the fp32 / int32 products.
 """
+import dataclasses
+
 import torch
 import torch.nn as nn
 import torch.nn.functional as F
@@ -29,7 +31,7 @@ class CompressedLinear(nn.Module):
         self.in_features, self.out_features = in_features, out_features
         self.config = config if config is not None else LatticeRANSConfig()
         if self.code_dtype is not None:
-            self.config = LatticeRANSConfig(self.config.target_bpp, self.code_dtype, self.config.blocks_per_lane)
+            self.config = dataclasses.replace(self.config, container=self.code_dtype)
         self.init_dtype = dtype
         self.bias = nn.Parameter(torch.zeros(out_features, device=device, dtype=dtype), requires_grad=False) \
             if bias else None

@@ -6,6 +6,7 @@ import io
 import math
 import warnings
 
+import numpy as np
 import pytest
 import torch
 
@@ -93,3 +94,13 @@ def test_invalid_inputs_raise():
     with pytest.raises(B.EpError):
         compress(bad, 4.0)
     assert math.isfinite(compress(synth.gaussian(16, 64, 0.02, 1), LatticeRANSConfig(target_bpp=8.0)).actual_bpp)
+
+
+def test_config_coding_reaches_the_stream(oracle):
+    """LatticeRANSConfig.coding selects paired or single coding of coordinates 1..6"""
+    w = synth.row_lognormal(128, 1024, 3)
+    paired = compress(w, LatticeRANSConfig(target_bpp=4.0, coding=2))
+    single = compress(w, LatticeRANSConfig(target_bpp=4.0, coding=1))
+    assert paired._info.paired == 1 and single._info.paired == 0
+    rc, ref = oracle.compress(w, 4.0, coding=oracle.CODING_PAIRED)
+    assert np.array_equal(paired.blob.numpy(), ref)
