@@ -58,8 +58,9 @@ enum ep_status {
 /* bits the decode kernel ORs into *d_status when a stream is damaged */
 enum ep_decode_flags {
     EP_DEC_WORD_OVERRUN = 1u, /* a renormalisation read ran past the tile's words */
-    EP_DEC_BAD_TOKEN = 2u,    /* frequency tables that do not sum to 2^11 or hold an entry of
-                                 2^11 or more (ep_prepare); a token outside its table (oracle) */
+    EP_DEC_BAD_TOKEN = 2u,    /* frequency tables that do not sum to 2^11 (pair tables: 2^12) or
+                                 hold an entry of that much or more (ep_prepare); an escaped pair's
+                                 token beyond its alphabet; a token outside its table (oracle) */
     EP_DEC_BAD_END = 4u,      /* a lane's state did not return to 2^16 at the end of its tile */
     EP_DEC_WORD_COUNT = 8u,   /* the tile has unread words beyond its 16-byte padding */
     EP_DEC_BAD_TILE = 16u,    /* a tile directory entry points outside the tile section */
@@ -152,8 +153,9 @@ int ep_compress_device(const void *d_src, int32_t src_dtype, int64_t rows, int64
  *   blob   host pointer to the first nbytes of the stream; nbytes must be the whole stream
  *          (the tile directory is checked against the stream end).
  *   info   filled on success.
- * Validates magic, version, shape, dtypes, table sums (each used context sums to 2048) and
- * the tile directory; returns EP_ERR_CORRUPT otherwise. */
+ * Validates magic, version, shape, dtypes, the coding byte, table sums (each used context sums
+ * to 2048; a paired stream's pair tables to 4096) and the tile directory; returns EP_ERR_CORRUPT
+ * otherwise. */
 int ep_stream_info(const void *blob, size_t nbytes, ep_info *info);
 
 /* First half of decompress(compressed) (API reference): the decoder's tables for one device
@@ -166,7 +168,10 @@ int ep_stream_info(const void *blob, size_t nbytes, ep_info *info);
  *               token's frequency, the slot's offset in the token, the escape flag and the
  *               decoded value of a direct token: the coordinate v, or, when a split of the
  *               stream is beyond the narrow range (8 for coordinates 1..6, 7 for coordinate 7),
- *               y = (v - c) / 2 for coordinates 1..7).
+ *               y = (v - c) / 2 for coordinates 1..7).  A paired stream's workspace holds the
+ *               slot tables of contexts 0 and 3..6, one 4096-slot table of 64-bit entries per
+ *               coset (frequency, slot offset and the two coordinates' values, or an escape
+ *               mark) and 2 x 256 token values for escaped pairs.
  *   d_status    nullable device uint32; EP_DEC_BAD_TOKEN is ORed in when the device copy's
  *               frequency tables are damaged.
  * One small kernel launch on `stream`; asynchronous. */
