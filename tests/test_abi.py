@@ -87,6 +87,18 @@ def test_errors():
         B.stream_info(torch.zeros(10, dtype=torch.uint8))
 
 
+def test_coding_option_checked():
+    w = synth.gaussian(64, 256, 0.02, 7)
+    for bad in (-1, 3):
+        with pytest.raises(B.EpError) as e:
+            B.compress(w, 4.0, coding=bad)
+        assert e.value.status == -1
+    # the three codings decode to the same plan shape; paired streams need more table memory
+    infos = [B.stream_info(B.compress(w, 4.0, coding=c)) for c in (0, 1, 2)]
+    assert [i.paired for i in infos] == [0, 0, 1]
+    assert infos[1].workspace_nbytes == 57344 and infos[2].workspace_nbytes == 108544
+
+
 def test_corrupt_streams_rejected():
     w = synth.gaussian(64, 512, 0.02, 2)
     blob = B.compress(w, 4.0)
