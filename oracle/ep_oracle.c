@@ -532,6 +532,32 @@ int32_t or_normalize_freqs_to(const uint64_t *counts, int32_t n, int32_t bits, u
 }
 
 /* ---------------------------------- paired coding ----------------------------------- */
+/* Pair table of a context with alphabet length A from the counts of its token pairs inside the
+ * base (B * B of them, B = min(A, 40); index t_a B + t_b) and the count N of all its pairs: a pair
+ * seen c > 0 times with c 2^16 < N, and every pair with a token outside the base, go to the
+ * escape symbol B * B; the B * B + 1 counts are then normalised to 2^12.  rare[] (B * B) flags the
+ * escaped pairs inside the base. */
+void or_pair_table(const uint64_t *inside, uint32_t A, uint64_t N, uint32_t *freq, uint8_t *rare)
+{
+    uint32_t B = A < PAIR_BASE_MAX ? A : PAIR_BASE_MAX, n = B * B + 1;
+    uint64_t *pc = (uint64_t *)calloc(n, sizeof(uint64_t));
+    uint64_t in = 0;
+    for (uint32_t q = 0; q + 1 < n; q++) {
+        pc[q] = inside[q];
+        in += inside[q];
+        rare[q] = 0;
+    }
+    pc[n - 1] = N - in;
+    for (uint32_t q = 0; q + 1 < n; q++)
+        if (pc[q] && pc[q] * PAIR_RARE_SCALE < N) {
+            rare[q] = 1;
+            pc[n - 1] += pc[q];
+            pc[q] = 0;
+        }
+    normalize_to(pc, (int32_t)n, PAIR_M, freq);
+    free(pc);
+}
+
 /* pair base B of a context with token alphabet length A, and its table length (0: no table) */
 static uint32_t pair_base(uint32_t A) { return A < PAIR_BASE_MAX ? A : PAIR_BASE_MAX; }
 static uint32_t pair_table_len(uint32_t A) { return A ? pair_base(A) * pair_base(A) + 1u : 0u; }
@@ -1107,19 +1133,10 @@ static int encode_at(const double *w, const float *s, const float *scales, int64
                         or_tokenize(u[8 * b + 2 + 2 * j], m[c], CTX_LOW[c], &tb, &nbits, &ex);
                         if (ta < B && tb < B)
                             pc[ta * B + tb]++;
-                        else
-                            pc[n - 1]++;
                         N++;
                     }
-            if (n) {
-                for (uint32_t q = 0; q + 1 < n; q++)
-                    if (pc[q] && pc[q] * PAIR_RARE_SCALE < N) {
-                        C.rare[c][q] = 1;
-                        pc[n - 1] += pc[q];
-                        pc[q] = 0;
-                    }
-                normalize_to(pc, (int32_t)n, PAIR_M, freq[c]);
-            }
+            if (n)
+                or_pair_table(pc, A, N, freq[c], C.rare[c]);
             free(pc);
         } else {
             ntok[c] = (uint32_t)or_normalize_freqs(cnt[c], (int32_t)alpha[c], freq[c]);

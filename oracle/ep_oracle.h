@@ -93,6 +93,10 @@ void or_tokenize_batch(const uint32_t *s, int64_t n, int32_t m, int32_t low, uin
 int32_t or_normalize_freqs(const uint64_t *counts, int32_t n, uint32_t *freqs);
 /* the same rule for tables summing to 2^bits */
 int32_t or_normalize_freqs_to(const uint64_t *counts, int32_t n, int32_t bits, uint32_t *freqs);
+/* paired coding: the pair table (B * B + 1 frequencies summing to 2^12, B = min(A, 40)) of a
+ * context with alphabet length A from its pair counts inside the base (B * B) and its pair count
+ * N; rare (B * B) flags the pairs coded as the escape */
+void or_pair_table(const uint64_t *inside, uint32_t A, uint64_t N, uint32_t *freq, uint8_t *rare);
 uint32_t or_choose_blocks_per_lane(int64_t nblocks, double target_bpp);
 uint16_t or_bf16_from_float(float w);
 uint16_t or_fp16_from_float(float w);

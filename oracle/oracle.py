@@ -62,6 +62,7 @@ def lib():
         L.or_normalize_freqs.argtypes = [p, C.c_int32, p]
         L.or_normalize_freqs_to.restype = C.c_int32
         L.or_normalize_freqs_to.argtypes = [p, C.c_int32, C.c_int32, p]
+        L.or_pair_table.argtypes = [p, C.c_uint32, C.c_uint64, p, p]
         L.or_choose_blocks_per_lane.restype = C.c_uint32
         L.or_choose_blocks_per_lane.argtypes = [C.c_int64, C.c_double]
         L.or_convert_batch.argtypes = [p, C.c_int64, C.c_int32, p]
@@ -236,6 +237,17 @@ def quantize(src, k, container=0):
     v = np.zeros((R, Cc), np.int32)
     lib().or_quantize(_ptr(a), dt, R, Cc, container or dt, int(k), _ptr(v))
     return v
+
+
+def pair_table(inside, A, N):
+    """(frequencies, rare flags) of a pair table: ``inside`` the B * B pair counts inside the base"""
+    B = min(int(A), 40)
+    c = np.ascontiguousarray(inside, dtype=np.uint64)
+    assert c.size == B * B
+    f = np.zeros(B * B + 1, np.uint32)
+    r = np.zeros(max(B * B, 1), np.uint8)
+    lib().or_pair_table(_ptr(c), int(A), int(N), _ptr(f), _ptr(r))
+    return f, r[: B * B]
 
 
 def estimate_bpp(src, k, container=0, blocks_per_lane=0, coding=CODING_AUTO):
