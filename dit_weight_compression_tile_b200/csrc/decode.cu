@@ -87,7 +87,7 @@ struct Params {
     uint32_t nbuf;           // tile buffers per warp (1 or 2); 0: tiles are read from global memory
     uint32_t splits;         // 4 bits per context
     uint32_t pair_A[2];      // paired: token alphabet length of contexts 1 and 2
-    uint32_t pair_rawb[2];   // paired: raw bits of one token of an escaped pair (<= 6)
+    uint32_t pair_rawb[2];   // paired: raw bits of one token of an escaped pair (<= 8)
 };
 
 // How a stream's blocks map onto rows, fixed per launch: kRowsAny (a lane's row is tested after
