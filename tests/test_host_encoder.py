@@ -79,11 +79,12 @@ def test_thread_count_independent():
 
 def test_parse_matches_oracle(oracle):
     w = synth.gaussian(256, 512, 0.02, 9)
-    for container in (0, B.INT8):
-        blob = B.compress(w, 3.0, container=container)
+    for container, coding in ((0, 0), (B.INT8, 0), (0, B.CODING_PAIRED), (B.INT8, B.CODING_PAIRED)):
+        blob = B.compress(w, 3.0, container=container, coding=coding)
         info = B.stream_info(blob)
         rc, oi = oracle.parse(blob.numpy())
         assert rc == 0
+        assert info.paired == oi.paired == (1 if coding else 0)
         for f in ("rows", "cols", "src_dtype", "container_dtype", "storage_nbytes", "header_nbytes",
                   "actual_bpp", "q_index", "n_tiles", "blocks_per_lane", "off_rowf", "off_scales",
                   "off_freq", "off_dir", "off_tiles"):
