@@ -99,6 +99,22 @@ def test_coding_option_checked():
     assert infos[1].workspace_nbytes == 57344 and infos[2].workspace_nbytes == 108544
 
 
+def test_malformed_paired_streams_rejected(oracle):
+    """the library parser refuses what the oracle's parser refuses in a paired stream"""
+    w = synth.row_lognormal(64, 512, 9)
+    blob = B.compress(w, 4.0, coding=B.CODING_PAIRED)
+    info = B.stream_info(blob)
+    assert info.paired == 1
+    q = info.off_freq + 2 * info.ntok[0]
+    for off, val in ((43, 2), (39, 8), (43, 0), (q, None)):
+        bad = blob.clone()
+        bad[off] = (int(bad[off]) ^ 1) if val is None else val
+        with pytest.raises(B.EpError) as e:
+            B.stream_info(bad)
+        assert e.value.status == -6, off
+        assert oracle.parse(bad.numpy())[0] == oracle.ERR_CORRUPT
+
+
 def test_corrupt_streams_rejected():
     w = synth.gaussian(64, 512, 0.02, 2)
     blob = B.compress(w, 4.0)
