@@ -180,6 +180,17 @@ def test_decode_calls_reject_bad_arguments_before_any_launch():
     bad = B.StreamInfo.from_buffer_copy(info)
     bad.cols = 0
     assert L.ep_decompress(C.byref(bad), fake, fake, fake, info.container_dtype, None, None) == -1
+    # a paired plan: alphabets above 256 tokens, splits beyond the narrow range, an unknown coding
+    paired = B.stream_info(B.compress(synth.row_lognormal(64, 512, 5), 4.0, coding=B.CODING_PAIRED))
+    assert paired.paired == 1
+    for field, idx, val in (("ntok", 1, 300), ("split", 4, 8), ("paired", None, 2)):
+        bad = B.StreamInfo.from_buffer_copy(paired)
+        if idx is None:
+            setattr(bad, field, val)
+        else:
+            getattr(bad, field)[idx] = val
+        assert L.ep_decompress(C.byref(bad), fake, fake, fake, bad.container_dtype, None, None) == -6, field
+        assert L.ep_prepare(C.byref(bad), fake, fake, None, None) == -6, field
 
 
 def test_host_buffer_decode_checks_arguments_before_any_copy():
