@@ -18,7 +18,7 @@
  *   "Compressed Linear usage", Combine compression with FP8 or INT8 computation -- lossy
  *       compression of FP8 / INT8 weight codes, 0.001 <= target_bpp < 8, per-row scales
  *       counted in storage.
- * The byte layout of the stream (format version 3) is this library's own; it is written
+ * The byte layout of the stream (format version 4) is this library's own; it is written
  * out in the repository's design notes.
  *
  * Decoding a stream takes two calls: ep_prepare once per device copy of a stream (it turns

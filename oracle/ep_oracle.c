@@ -29,11 +29,12 @@
 #include <string.h>
 
 /* ------------------------------------------------------------------------------------
- * Stream constants (format version 3).  These are the build's readings of what the
+ * Stream constants (format version 4).  These are the build's readings of what the
  * pages leave open: 11-bit frequency tables (every frequency below 2^11), 32-bit states
  * with 16-bit renormalisation words, 32 interleaved states per tile, seven coding
  * contexts, hybrid-integer tokens with 2 bits below the leading one and a per-context
- * number of low bits kept in the token, raw extra bits in a separate stream per tile.
+ * number of low bits kept in the token, raw extra bits in a separate stream per tile,
+ * and, when the tokens allow it, coordinates 1..6 coded in pairs (12-bit pair tables).
  * ---------------------------------------------------------------------------------- */
 #define MAGIC 0x31545045u /* bytes 'E','P','T','1' */
 #define VERSION 4
