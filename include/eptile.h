@@ -18,8 +18,9 @@
  *   "Compressed Linear usage", Combine compression with FP8 or INT8 computation -- lossy
  *       compression of FP8 / INT8 weight codes, 0.001 <= target_bpp < 8, per-row scales
  *       counted in storage.
- * The byte layout of the stream (format version 4) is this library's own; it is written
- * out in the repository's design notes.
+ * The byte layout of the stream (format version 4) is this library's own: a 64-byte header,
+ * per-row factors, per-row code scales (INT8 / FP8), frequency tables, a tile directory and the
+ * tiles (32 lane states, 32 region lengths, the lanes' words and raw bits).
  *
  * Decoding a stream takes two calls: ep_prepare once per device copy of a stream (it turns
  * the stream's frequency tables into the decoder's slot tables, in a caller-owned workspace

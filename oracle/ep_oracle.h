@@ -9,7 +9,7 @@
  * coding in independently decodable tiles, and decode with numerical
  * reconstruction into a weight container.  Where the pages leave a step open
  * (stream layout, model, tile size, rANS parameters) this file follows the
- * readings fixed in the repository's design notes; each function says which.
+ * readings stated beside each function.
  *
  * Only the test-suite, the smoke check and the CPU-baseline leg of the
  * benchmark may load this library.  It shares no source with the product
