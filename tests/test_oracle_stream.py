@@ -158,8 +158,10 @@ def test_code_containers(oracle, container, target):
     rel = np.linalg.norm(dec - codes) / np.linalg.norm(codes)
     assert rel < 0.25
     if target > 7:
-        # near 8 bits (6.5 payload bits per code on this small matrix) about two codes in
-        # three come back exactly and the rest move by one grid step
+        # near 8 bits about two codes in three come back exactly and the rest move by one grid
+        # step.  Measured on this 64 x 512 matrix: 7.46 bpp stored, of which 6.44 bits per code
+        # are payload (the header, tables and eight tile heads take the rest), and 69.4 % of the
+        # codes exact; the bound sits below that with room for the rounding of the resolution
         assert rel < 0.02 and np.mean(dec == codes) > 0.65
 
 
