@@ -13,7 +13,9 @@ gate the GPU.
 
 N > 1 runs N independent replicas (the decode has no exchange step, so there is no collective):
 one process per GPU under torchrun, timed on the device, max over ranks.  The reference arm
-(--impl reference) is the CPU oracle decoder, timed on one host core.
+(--impl reference) is the CPU oracle: it encodes the workload's first tensor with the oracle's
+compressor and times the oracle's decoder on every host core the process may use.  Both arms
+print the same ``config`` (the workload and how the timed region defeats the L2).
 """
 import argparse
 import hashlib
@@ -41,20 +43,24 @@ L2_BYTES = 126 * 2 ** 20
 WORKLOADS = {
     "lognormal_rows_4096x4096_bf16": dict(
         layers=lambda: [("w", lambda: _synth().row_lognormal(4096, 4096, 1))], target=4.0, container=0,
-        distribution="N(0, s_r^2), s_r = 0.02 exp(0.3 g), seed 1", shape="4096x4096"),
+        dims=[(4096, 4096)], distribution="N(0, s_r^2), s_r = 0.02 exp(0.3 g), seed 1", shape="4096x4096"),
     "dit_28blocks_hidden3072_bf16": dict(
         layers=lambda: [(f"block{b}.{n}", (lambda b=b, l=l: _synth().dit_layer(b, l)))
                         for b in range(28) for l, n in enumerate(("qkv", "out", "mlp_up", "mlp_down"))],
         target=4.0, container=0, shape="28 x {3072x9216, 3072x3072, 3072x12288, 12288x3072}",
+        dims=[(3072, 9216), (3072, 3072), (3072, 12288), (12288, 3072)] * 28,
         distribution="Student-t(5) / sqrt(5/3) * 0.02 * per-row exp(0.3 g), seed 100 + 4 block + layer"),
     "int8_codes_8192x8192": dict(
         layers=lambda: [("w", lambda: _synth().gaussian(8192, 8192, 0.02, 2))], target=3.0, container="int8",
+        dims=[(8192, 8192)],
         distribution="N(0, 0.02^2), seed 2, per-row absmax INT8 codes", shape="8192x8192"),
     "fp8_codes_8192x8192": dict(
         layers=lambda: [("w", lambda: _synth().gaussian(8192, 8192, 0.02, 2))], target=3.0, container="fp8_e4m3",
+        dims=[(8192, 8192)],
         distribution="N(0, 0.02^2), seed 2, per-row absmax FP8 E4M3 codes", shape="8192x8192"),
     "outliers_8192x28672_bf16": dict(
         layers=lambda: [("w", lambda: _synth().gaussian_outliers(8192, 28672, 3))], target=4.0, container=0,
+        dims=[(8192, 28672)],
         distribution="N(0, 0.02^2), seed 3, 0.1% of entries set to +-8 sigma", shape="8192x28672"),
 }
 DEFAULT_WORKLOAD = "lognormal_rows_4096x4096_bf16"
@@ -93,12 +99,35 @@ def workload_config(a):
             "distribution": wl["distribution"], "container": wl["container"] or "bf16"}
 
 
+def l2_policy(a):
+    """(device copies to rotate over, the sentence that says how the timed region defeats the
+    L2), from the workload's nominal bytes (target rate in, container out) so that both arms
+    state the same policy: workloads smaller than twice the L2 rotate over copies whose streams
+    and outputs together exceed twice the L2"""
+    wl = WORKLOADS[a.workload]
+    esz = 1 if wl["container"] in ("int8", "fp8_e4m3") else 2
+    nominal = sum(r * c for r, c in wl["dims"]) * (a.target / 8.0 + esz)
+    if nominal >= 2 * L2_BYTES:
+        return 1, f"inputs larger than L2: {nominal / 1e6:.0f} MB per step"
+    rot = min(8, -(-2 * L2_BYTES // int(nominal)))
+    return rot, f"inputs larger than L2: {rot} rotating stream+output copies ({rot * nominal / 1e6:.0f} MB)"
+
+
+def bench_config(a, world):
+    """the ``config`` both arms print: the workload and the L2 policy of the timed region"""
+    return dict(workload_config(a), l2=l2_policy(a)[1], parallelism="replicas" if world > 1 else "single")
+
+
 def compress_layers(a):
     """the workload's streams, encoded once on the GPU (ep_compress_device: the host compressor's
-    bytes), untimed for the metric; returns [(name, host copy of the blob)] and the encode seconds"""
+    bytes), untimed for the metric; returns [(name, host copy of the blob)], the encode seconds
+    and the relative L2 error of the decoded weights against the source tensors,
+    sqrt(sum (W - What)^2 / sum W^2) over the whole workload (INT8 / FP8 codes dequantized with
+    the stream's row scales)"""
     from dit_weight_compression_tile_b200 import binding as B
     wl = WORKLOADS[a.workload]
     out, t = [], 0.0
+    err2 = ref2 = 0.0
     for name, make in wl["layers"]():
         w = make().cuda()
         torch.cuda.synchronize()
@@ -106,9 +135,18 @@ def compress_layers(a):
         blob = B.compress_device(w, a.target, container=wl["container"])
         torch.cuda.synchronize()
         t += time.perf_counter() - t0
-        out.append((name, blob.cpu()))
-        del w, blob
-    return out, t
+        host = blob.cpu()
+        info = B.stream_info(host)
+        dec = B.decompress(blob, info).double()
+        if info.container_dtype in (B.INT8, B.FP8E4M3):
+            scales = blob[info.off_scales: info.off_scales + 4 * info.rows].view(torch.float32).double()
+            dec = dec * scales[:, None]
+        w64 = w.double()
+        err2 += float(((w64 - dec) ** 2).sum())
+        ref2 += float((w64 ** 2).sum())
+        out.append((name, host))
+        del w, w64, blob, dec
+    return out, t, (err2 / ref2) ** 0.5 if ref2 > 0 else 0.0
 
 
 def measured_peaks():
@@ -144,14 +182,19 @@ class ClockSampler:
         except Exception:  # no NVML: clocks are reported as unknown
             self.nv = None
 
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            pass
+
     def _run(self):
+        # every 5 ms while the timed region runs, plus one sample as it ends (a short region
+        # still gets two)
         while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-            except Exception:
-                pass
-            time.sleep(0.02)
+            self._sample()
+            time.sleep(0.005)
 
     def __enter__(self):
         if self.nv:
@@ -163,6 +206,7 @@ class ClockSampler:
         self._stop.set()
         if self.nv:
             self.t.join()
+            self._sample()
 
     def summary(self):
         if not self.samples:
@@ -245,8 +289,7 @@ def run_reference(a, rank, world):
     if rank != 0:
         return
     from oracle import oracle as O
-    layers, _ = compress_layers_first(a)
-    blob = layers[0][1].numpy()
+    blob = oracle_first_stream(a)
     rc, info = O.parse(blob)
     T, per_tile_w = info.n_tiles, 32 * info.blocks_per_lane * 8
     esz = 2 if WORKLOADS[a.workload]["container"] in (0, "bf16") else 1
@@ -286,7 +329,10 @@ def run_reference(a, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
             "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(1e3 * t / a.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32+f32",
-            "data": "synthetic", "config": dict(workload_config(a), l2="n/a (host)"),
+            "data": "synthetic", "config": bench_config(a, world),
+            "stream": {"actual_bpp": round(info.actual_bpp, 4), "coding": "paired" if info.paired else "single",
+                       "n_tiles": info.n_tiles, "blocks_per_lane": info.blocks_per_lane,
+                       "encoder": "the oracle's compressor (first tensor of the workload)"},
             "gweights_per_s": round(tiles * per_tile_w * a.steps / t / 1e9, 4),
             "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": ncores, "kind": "oracle",
                              "sample": f"{tiles} of {T} tiles ({tiles * per_tile_w} weights) of the first "
@@ -295,12 +341,16 @@ def run_reference(a, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def compress_layers_first(a):
-    """only the first stream of the workload (the reference arm decodes a sample of it)"""
-    from dit_weight_compression_tile_b200 import binding as B
+def oracle_first_stream(a):
+    """the workload's first tensor encoded by the oracle's own compressor (the reference arm decodes
+    a sample of it; the oracle's bytes equal the library's, and this arm loads no library code)"""
+    from oracle import oracle as O
     wl = WORKLOADS[a.workload]
     name, make = wl["layers"]()[0]
-    return [(name, B.compress(make(), a.target, container=wl["container"]))], 0.0
+    container = {0: 0, "bf16": O.BF16, "int8": O.INT8, "fp8_e4m3": O.FP8E4M3}[wl["container"]]
+    rc, blob = O.compress(make(), a.target, container=container)
+    assert rc == O.OK, rc
+    return blob
 
 
 # ------------------------------------------------------------------ our arm
@@ -308,13 +358,13 @@ def run_ours(a, rank, world, local_rank):
     from dit_weight_compression_tile_b200 import binding as B
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    layers, t_enc = compress_layers(a)
+    layers, t_enc, rel_l2 = compress_layers(a)
     infos = [B.stream_info(blob) for _, blob in layers]
     n_weights = sum(i.rows * i.cols for i in infos)
     in_bytes = sum(i.storage_nbytes for i in infos)
     out_bytes = sum(i.out_nbytes for i in infos)
     # rotate device copies so that every step reads and writes more than the L2 holds
-    rot = 1 if in_bytes + out_bytes >= 2 * L2_BYTES else min(8, -(-2 * L2_BYTES // (in_bytes + out_bytes)))
+    rot = l2_policy(a)[0]
     stream = torch.cuda.Stream(dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     blobs, works, outs = [], [], []
@@ -328,27 +378,39 @@ def run_ours(a, rank, world, local_rank):
                 outs.append(torch.empty(info.shape, dtype=info.dtype, device=dev))
     per = [infos[i % len(infos)] for i in range(len(blobs))]
 
-    def decode_all():
-        for d, w_, o, info in zip(blobs, works, outs, per):
-            B.decompress(d, info, workspace=w_, out=o, status=status, stream=stream)
+    ntens = len(infos)
+
+    def decode_steps(first, count):
+        # `count` steps from copy `first` on: each step decodes every tensor of one copy
+        for j in range(count):
+            r = (first + j) % rot
+            for i in range(ntens):
+                k = r * ntens + i
+                B.decompress(blobs[k], per[k], workspace=works[k], out=outs[k], status=status, stream=stream)
 
     # first calls outside capture: sets the kernel attributes, checks the output
     with torch.cuda.stream(stream):
-        decode_all()
+        decode_steps(0, rot)
     torch.cuda.synchronize(dev)
     assert int(status.item()) == 0, "decode reported stream damage"
+    # exactly a.steps timed steps: whole replays of a graph of `rot` steps, then a graph of the rest
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
-        decode_all()
-    replays = max(1, -(-a.steps // rot))
-    steps = replays * rot
+        decode_steps(0, rot)
+    replays, rest = divmod(a.steps, rot)
+    tail = None
+    if rest:
+        tail = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(tail, stream=stream):
+            decode_steps(0, rest)
+    steps = a.steps
     with torch.cuda.stream(stream):
         for _ in range(max(1, -(-a.warmup // rot))):
             graph.replay()
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(replays + 1)]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(replays + 2)]
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
         with torch.cuda.stream(stream):
@@ -356,14 +418,20 @@ def run_ours(a, rank, world, local_rank):
             for r in range(replays):
                 graph.replay()
                 ev[r + 1].record(stream)
+            if tail is not None:
+                tail.replay()
+            ev[-1].record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
     per_replay = [ev[r].elapsed_time(ev[r + 1]) for r in range(replays)]
     total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), world, dev)
     assert int(status.item()) == 0
-    kernel_s = statistics.mean(per_replay) / rot / 1e3  # decode launches of one step, back to back
     step_s = total_ms / steps / 1e3
+    # the decode launches of one step run back to back on one stream: the mean launch time is
+    # the timed region over its launches; median and minimum come from whole replays
+    kernel_s = ev[0].elapsed_time(ev[-1]) / steps / 1e3
+    per_launch_us = sorted(1e3 * x / (rot * ntens) for x in per_replay)
     value = job_rate(out_bytes, world, step_s) / 1e9
     peak, peak_kind = measured_peaks()
     achieved = (in_bytes + out_bytes) / kernel_s / 1e9
@@ -424,19 +492,18 @@ def run_ours(a, rank, world, local_rank):
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": steps,
         "warmup": a.warmup, "ms_per_step": round(step_s * 1e3, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u32+f32", "data": "synthetic",
-        "config": dict(workload_config(a),
-                       l2=(f"inputs larger than L2: {rot} rotating stream+output copies "
-                           f"({rot * (in_bytes + out_bytes) / 1e6:.0f} MB)") if rot > 1 else
-                          f"inputs larger than L2: {(in_bytes + out_bytes) / 1e6:.0f} MB per step",
-                       actual_bpp=round(8.0 * in_bytes / n_weights, 4), coding=coding_label(infos),
-                       n_tensors=len(infos),
-                       n_tiles=sum(i.n_tiles for i in infos), blocks_per_lane=i0.blocks_per_lane,
-                       parallelism="replicas" if world > 1 else "single"),
+        "config": bench_config(a, world),
+        "stream": {"actual_bpp": round(8.0 * in_bytes / n_weights, 4), "coding": coding_label(infos),
+                   "n_tensors": len(infos), "n_tiles": sum(i.n_tiles for i in infos),
+                   "blocks_per_lane": i0.blocks_per_lane, "rel_l2": round(rel_l2, 5),
+                   "rel_l2_note": "||W - What|| / ||W|| against the source weights over the whole workload"},
         "gweights_per_s": round(job_rate(n_weights, world, step_s) / 1e9, 3),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": (in_bytes + out_bytes) // len(infos),
-                     "kernel_us": round(kernel_s * 1e6 / len(infos), 3)},
+                     "kernel_us": round(kernel_s * 1e6 / len(infos), 3),
+                     "kernel_us_median": round(statistics.median(per_launch_us), 3) if per_launch_us else None,
+                     "kernel_us_min": round(per_launch_us[0], 3) if per_launch_us else None},
         "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": in_bytes,
                 "d2h_bytes_per_step": out_bytes},
         "gpu_launches": steps * len(infos),

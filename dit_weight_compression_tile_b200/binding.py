@@ -217,7 +217,10 @@ def decompress(d_blob, info=None, workspace=None, out=None, status=None, stream=
 
     ``d_blob``: CUDA uint8 tensor holding the whole stream.  ``info``: from ``stream_info``
     (parsed from ``d_blob`` through a host copy when omitted).  ``workspace``: from ``prepare``
-    on this ``d_blob`` (prepared here, on the same stream, when omitted).  ``out``: optional CUDA
+    on this ``d_blob``.  When omitted, every call allocates a workspace and runs ``prepare``
+    again on the same stream (a few microseconds of table building per call); callers that
+    decode one stream repeatedly should prepare once and pass the workspace, as
+    ``CompressedTensor`` does.  ``out``: optional CUDA
     tensor of ``info.shape`` / ``info.dtype``.  ``status``: optional CUDA int32 tensor of one
     element into which damage flags are ORed.  Launches on ``stream`` (default: the current
     stream).  ``lattice=True`` returns the decoded lattice points v = 2z (int32) instead of

@@ -40,7 +40,13 @@ extern "C" int ep_stream_info(const void *blob, size_t nbytes, ep_info *info) {
     if (I.rows <= 0 || I.cols <= 0 || I.rows >= (int64_t(1) << 40) || I.cols >= (int64_t(1) << 40) ||
         I.blocks_per_lane == 0 || I.blocks_per_lane > 4096 || I.q_index >= kNumQ)
         return EP_ERR_CORRUPT;
-    int64_t nb = I.rows * ((I.cols + 7) / 8);  // rows zero-padded to whole E8 blocks
+    // every product below is formed only once it is known to fit (rows and cols may each come
+    // close to 2^40 in a damaged header)
+    int64_t nb, elems, out_bytes;
+    if (__builtin_mul_overflow(I.rows, (I.cols + 7) / 8, &nb) || __builtin_mul_overflow(I.rows, I.cols, &elems) ||
+        __builtin_mul_overflow(elems, int64_t(elt_bytes(I.container_dtype)), &out_bytes))
+        return EP_ERR_CORRUPT;
+    // nb: rows zero-padded to whole E8 blocks
     int64_t per_tile = int64_t(kLanes) * I.blocks_per_lane;
     if ((nb + per_tile - 1) / per_tile != int64_t(I.n_tiles)) return EP_ERR_CORRUPT;
     if (p[43] > 1) return EP_ERR_CORRUPT;
@@ -89,8 +95,8 @@ extern "C" int ep_stream_info(const void *blob, size_t nbytes, ep_info *info) {
     if (L.tiles + 16 * prev != nbytes) return EP_ERR_CORRUPT;
     I.storage_nbytes = nbytes;
     I.header_nbytes = kHeaderBytes;
-    I.actual_bpp = 8.0 * double(nbytes) / double(I.rows * I.cols);
-    I.out_nbytes = uint64_t(I.rows * I.cols) * uint64_t(elt_bytes(I.container_dtype));
+    I.actual_bpp = 8.0 * double(nbytes) / double(elems);
+    I.out_nbytes = uint64_t(out_bytes);
     // the decoder's slot tables: 7 token tables, or 5 token tables, two pair tables of 8-byte
     // entries and the token fields of the escaped pairs
     I.workspace_nbytes = I.paired ? kPairedTableBytes : uint64_t(kContexts) * kProbScale * 4;

@@ -211,7 +211,10 @@ int ep_decompress(const ep_info *info, const void *d_blob, const void *d_workspa
  *   array of 108,544 bytes (info->workspace_nbytes of every stream), which each GPU that loads the
  *   library keeps until the process exits.  A stream needing more returns EP_ERR_UNSUPPORTED.
  *   The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
- *   that device current; make that first call before any stream capture.
+ *   that device current and keeps it for the life of the process; make that first call before
+ *   any stream capture.  A device reset (cudaDeviceReset, or the primary context torn down and
+ *   created again) reloads the module and invalidates the kept address: do not call this entry
+ *   point again in a process after resetting a device it was called on.
  *   All calls on a device share the array and leave the last call's tables in it: calls that
  *   overlap on the GPU (different streams without ordering) race and may decode with another
  *   stream's tables.  Two launches (tables, decode) on `stream`; no allocation, no sync. */

@@ -221,3 +221,16 @@ def test_host_buffer_decode_checks_arguments_before_any_copy():
     bad = B.StreamInfo.from_buffer_copy(info)
     bad.split[3] = 12
     assert L.ep_decompress_host(C.byref(bad), h, fake, dt, fake, need, None, None) == -6
+
+
+def test_huge_header_shapes_rejected_without_overflow():
+    """rows and cols near the parser's 2^40 bound make rows * cols overflow 64 bits: the parser
+    refuses such headers as corrupt before it forms any product"""
+    import struct
+    blob = B.compress(synth.gaussian(64, 512, 0.02, 2), 4.0)
+    for rows, cols in [((1 << 40) - 1, (1 << 40) - 1), ((1 << 39), (1 << 30)), ((1 << 35), (1 << 36))]:
+        bad = bytearray(blob.numpy().tobytes())
+        struct.pack_into("<qq", bad, 8, rows, cols)
+        with pytest.raises(B.EpError) as e:
+            B.stream_info(torch.frombuffer(bad, dtype=torch.uint8))
+        assert e.value.status == -6, (rows, cols)

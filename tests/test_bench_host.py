@@ -14,3 +14,35 @@ def test_coding_label():
     assert bench.coding_label([paired, paired]) == "paired"
     assert bench.coding_label([single]) == "single"
     assert bench.coding_label([paired, single]) == "mixed"
+
+
+def _args(workload, target=None):
+    import argparse
+    wl = bench.WORKLOADS[workload]
+    return argparse.Namespace(workload=workload, target=wl["target"] if target is None else target)
+
+
+def test_both_arms_state_the_same_config():
+    """the GPU arm and the reference arm print one config: the workload and the L2 policy, with
+    nothing taken from either arm's own streams"""
+    for name in bench.WORKLOADS:
+        a = _args(name)
+        c1, c2 = bench.bench_config(a, 1), bench.bench_config(a, 1)
+        assert c1 == c2 and c1["workload"] == name and c1["parallelism"] == "single"
+        assert bench.bench_config(a, 4)["parallelism"] == "replicas"
+        assert set(c1) == {"workload", "shape", "target_bpp", "distribution", "container", "l2", "parallelism"}
+
+
+def test_l2_policy():
+    """workloads below twice the L2 rotate over enough copies to exceed it; the others need none"""
+    rot, text = bench.l2_policy(_args("lognormal_rows_4096x4096_bf16"))
+    nominal = 4096 * 4096 * (4.0 / 8 + 2)
+    assert rot == 7 and rot * nominal >= 2 * bench.L2_BYTES and (rot - 1) * nominal < 2 * bench.L2_BYTES
+    assert "7 rotating" in text
+    for name in ("dit_28blocks_hidden3072_bf16", "outliers_8192x28672_bf16"):
+        assert bench.l2_policy(_args(name))[0] == 1
+    rot, _ = bench.l2_policy(_args("int8_codes_8192x8192"))
+    assert rot * 8192 * 8192 * (3.0 / 8 + 1) >= 2 * bench.L2_BYTES
+    # the DiT set lists 112 tensors of the four block shapes
+    dims = bench.WORKLOADS["dit_28blocks_hidden3072_bf16"]["dims"]
+    assert len(dims) == 112 and sum(r * c for r, c in dims) == 28 * 3072 * (9216 + 3072 + 12288 + 12288)

@@ -2,8 +2,9 @@
 instance a plugin inside an inference engine that owns all device memory, or code that must
 avoid the synchronisation a cudaMalloc can cause): it keeps the decoder's tables in a static
 device array instead of a caller workspace.  Called through the C ABI, its output must equal
-the workspace path's (ep_prepare + ep_decompress) bit for bit, on two calls in a row with
-different streams, so the second call must replace the first call's tables.
+the workspace path's (ep_prepare + ep_decompress) bit for bit, on calls in a row with
+different streams and table layouts (paired, single-coded, paired), so each call must replace
+the previous call's tables.
 
 The file sorts last so that a run stopping at its first failure has already run every other
 test; it also passes alone in a fresh process."""
@@ -36,11 +37,17 @@ def workspace_decode(d_blob, info, stream):
 
 
 def test_noalloc_matches_workspace_path_twice():
-    cases = [(synth.row_lognormal(512, 2048, 21), 4.0, 0), (synth.gaussian(256, 1024, 0.02, 22), 3.0, B.INT8)]
+    # a paired stream (108,544 bytes of tables) then a single-coded one (57,344 bytes) and a paired
+    # one again: each call must leave its own tables in the shared array, whatever the one before
+    cases = [(synth.row_lognormal(512, 2048, 21), 4.0, 0, B.CODING_PAIRED),
+             (synth.gaussian(256, 1024, 0.02, 22), 3.0, B.INT8, B.CODING_SINGLE),
+             (synth.gaussian(256, 1024, 0.02, 23), 3.0, B.FP8E4M3, B.CODING_PAIRED)]
     stream = torch.cuda.Stream()
-    for w, target, container in cases:  # two calls in a row, the second with other tables
-        blob = B.compress(w, target, container=container)
+    layouts = []
+    for w, target, container, coding in cases:  # calls in a row, each with other tables
+        blob = B.compress(w, target, container=container, coding=coding)
         info = B.stream_info(blob)
+        layouts.append((info.paired, info.workspace_nbytes))
         d = blob.cuda()
         with torch.cuda.stream(stream):
             got, st_got = noalloc_decode(d, info, stream)
@@ -49,6 +56,7 @@ def test_noalloc_matches_workspace_path_twice():
         assert int(st_got.item()) == 0 and int(st_ref.item()) == 0
         assert got.dtype == ref.dtype and got.shape == ref.shape
         assert np.array_equal(got.view(torch.uint8).cpu().numpy(), ref.view(torch.uint8).cpu().numpy())
+    assert layouts == [(1, 108544), (0, 57344), (1, 108544)]
 
 
 def test_noalloc_rejects_oversized_workspace():
