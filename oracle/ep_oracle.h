@@ -139,6 +139,25 @@ int or_decode_as(const uint8_t *blob, size_t nbytes, uint32_t t0, uint32_t t1, i
 int or_code_stats(const uint8_t *blob, size_t nbytes, double *ideal_bits, double *emp_entropy_bits,
                   double *extra_bits, uint64_t *n_symbols, uint64_t *payload_bytes);
 
+/* ---- the Tile-ANS lossless stream (ep_tile_ans.c) ---- */
+typedef struct {
+    int64_t n;               /* elements */
+    int32_t dtype, ndim;
+    int64_t shape[8];
+    uint32_t n_tiles, blocks_per_lane;
+    uint64_t off_freq, off_dir, off_raw, off_tiles, storage_nbytes;
+} ota_info;
+
+/* the tile size (chunks of 8 elements per lane) chosen for a tensor of n_chunks chunks */
+uint32_t ota_blocks_per_lane(int64_t n_chunks);
+/* compresses n elements of dtype (shape of ndim <= 8 dims, product n); blocks_per_lane 0 =
+ * automatic; OR_ERR_BUFFER_TOO_SMALL with *out_nbytes = the size needed when cap is short */
+int ota_compress(const void *src, int32_t dtype, int64_t n, int32_t ndim, const int64_t *shape,
+                 uint32_t blocks_per_lane, uint8_t *out, size_t cap, size_t *out_nbytes);
+int ota_parse(const uint8_t *blob, size_t nbytes, ota_info *info);
+/* decodes tiles [t0, t1) into out (the tensor's bytes); ORs OR_DEC_* bits into *status */
+int ota_decode(const uint8_t *blob, size_t nbytes, uint32_t t0, uint32_t t1, void *out, uint32_t *status);
+
 #ifdef __cplusplus
 }
 #endif

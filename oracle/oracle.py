@@ -31,6 +31,15 @@ class Info(C.Structure):
     ]
 
 
+class TAInfo(C.Structure):
+    _fields_ = [
+        ("n", C.c_int64), ("dtype", C.c_int32), ("ndim", C.c_int32), ("shape", C.c_int64 * 8),
+        ("n_tiles", C.c_uint32), ("blocks_per_lane", C.c_uint32),
+        ("off_freq", C.c_uint64), ("off_dir", C.c_uint64), ("off_raw", C.c_uint64), ("off_tiles", C.c_uint64),
+        ("storage_nbytes", C.c_uint64),
+    ]
+
+
 _lib = None
 
 
@@ -86,6 +95,12 @@ def lib():
         L.or_code_stats.restype = C.c_int
         L.or_code_stats.argtypes = [p, C.c_size_t, C.POINTER(C.c_double), C.POINTER(C.c_double),
                                     C.POINTER(C.c_double), C.POINTER(C.c_uint64), C.POINTER(C.c_uint64)]
+        L.ota_blocks_per_lane.restype = C.c_uint32
+        L.ota_blocks_per_lane.argtypes = [C.c_int64]
+        L.ota_compress.argtypes = [p, C.c_int32, C.c_int64, C.c_int32, p, C.c_uint32, p, C.c_size_t,
+                                   C.POINTER(C.c_size_t)]
+        L.ota_parse.argtypes = [p, C.c_size_t, C.POINTER(TAInfo)]
+        L.ota_decode.argtypes = [p, C.c_size_t, C.c_uint32, C.c_uint32, p, C.POINTER(C.c_uint32)]
         _lib = L
     return _lib
 
@@ -302,6 +317,44 @@ def decode(blob, t0=0, t1=None, want_v=True, want_out=True, out_buf=None, out_dt
     return rc, st.value, v, out
 
 
+def decode_parallel(blob, threads=None, want_v=True, out_dtype=0):
+    """``decode`` of the whole stream with the oracle's tile decoder on several host threads:
+    the tiles are independent, so each thread decodes its own contiguous range of them into the
+    shared output arrays (ctypes releases the GIL during the C call).  Same results as
+    ``decode``; returns (rc, status, v or None, out)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    blob = np.ascontiguousarray(blob, dtype=np.uint8)
+    rc, info = parse(blob)
+    if rc != OK:
+        return rc, 0, None, None
+    R, Cc = info.rows, info.cols
+    v = np.zeros((R, Cc), np.int32) if want_v else None
+    out = np.zeros((R, Cc), NP_DTYPE[out_dtype or info.container_dtype])
+    if threads is None:
+        try:
+            threads = len(os.sched_getaffinity(0))
+        except AttributeError:
+            threads = os.cpu_count() or 1
+    T = info.n_tiles
+    n = max(1, min(int(threads), T))
+    cuts = [(T * i) // n for i in range(n + 1)]
+
+    def one(i):
+        st = C.c_uint32(0)
+        r = lib().or_decode_as(_ptr(blob), blob.size, cuts[i], cuts[i + 1], _ptr(v) if v is not None else None,
+                               _ptr(out), int(out_dtype), C.byref(st))
+        return r, st.value
+
+    with ThreadPoolExecutor(n) as ex:
+        res = list(ex.map(one, range(n)))
+    rc = next((r for r, _ in res if r != OK), OK)
+    st = 0
+    for _, s_ in res:
+        st |= s_
+    return rc, st, v, out
+
+
 def code_stats(blob):
     blob = np.ascontiguousarray(blob, dtype=np.uint8)
     ideal, H, extra = C.c_double(), C.c_double(), C.c_double()
@@ -310,3 +363,43 @@ def code_stats(blob):
                              C.byref(ns), C.byref(pb))
     return rc, dict(ideal_bits=ideal.value, entropy_bits=H.value, extra_bits=extra.value,
                     n_symbols=ns.value, payload_bytes=pb.value)
+
+
+# ---- the Tile-ANS lossless stream ----
+TA_NP = {BF16: np.uint16, FP16: np.uint16, FP32: np.uint32, INT8: np.uint8, FP8E4M3: np.uint8}
+
+
+def ta_compress(bits, dtype, shape=None, blocks_per_lane=0):
+    """Tile-ANS stream of the elements ``bits`` (a numpy array of the dtype's raw bit patterns:
+    uint16 for BF16 / FP16, uint32 for FP32, uint8 for INT8 / FP8).  Returns (rc, blob)."""
+    a = np.ascontiguousarray(bits)
+    shape = tuple(a.shape) if shape is None else tuple(shape)
+    dims = (C.c_int64 * 8)(*shape)
+    n = C.c_size_t(0)
+    rc = lib().ota_compress(_ptr(a), dtype, a.size, len(shape), dims, blocks_per_lane, None, 0, C.byref(n))
+    if rc not in (OK, ERR_BUFFER_TOO_SMALL):
+        return rc, None
+    out = np.zeros(n.value, np.uint8)
+    rc = lib().ota_compress(_ptr(a), dtype, a.size, len(shape), dims, blocks_per_lane, _ptr(out), out.size,
+                            C.byref(n))
+    return rc, (out if rc == OK else None)
+
+
+def ta_parse(blob):
+    blob = np.ascontiguousarray(blob, dtype=np.uint8)
+    info = TAInfo()
+    rc = lib().ota_parse(_ptr(blob), blob.size, C.byref(info))
+    return rc, info
+
+
+def ta_decode(blob, t0=0, t1=None):
+    """(rc, status, elements as a numpy array of the dtype's bit patterns in the stream's shape)"""
+    blob = np.ascontiguousarray(blob, dtype=np.uint8)
+    rc, info = ta_parse(blob)
+    if rc != OK:
+        return rc, 0, None
+    out = np.zeros(info.n, TA_NP[info.dtype])
+    st = C.c_uint32(0)
+    t1 = info.n_tiles if t1 is None else t1
+    rc = lib().ota_decode(_ptr(blob), blob.size, t0, t1, _ptr(out), C.byref(st))
+    return rc, st.value, out.reshape(tuple(info.shape[: info.ndim]))

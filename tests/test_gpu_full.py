@@ -1,9 +1,14 @@
-"""GPU parity at the workloads' full sizes, in the launch configuration the benchmark times
-(the library's own host encoder writes the streams; it is byte-identical to the oracle on
-the 4096x4096 workload, checked here at full size).  Where a full oracle decode would take
-minutes, the oracle decodes sampled tiles (first, last and seeded random ones) and the GPU
-output must match them bit for bit; the rest is held to properties that hold at any size
-(zero status, stored rate at most the target)."""
+"""GPU parity at the workloads' full sizes, in the launch configuration the benchmark times.
+Every weight and every lattice point of every workload is compared with the oracle's decode of
+the same stream (the oracle's tile decoder on every host core, tiles split among threads):
+
+* 4096x4096 log-normal rows at 4 bpp, and 8192x8192 INT8 / FP8 codes at 3 bpp;
+* the 8192x28672 outlier matrix at 0.5, 1, 2, 3.5, 5 and 8 bpp;
+* all 112 tensors of the DiT weight set (28 blocks of hidden 3072) at 2.5 and 4 bpp.
+
+The streams the GPU decodes come from the GPU compressor, as in the benchmark; its bytes equal the
+host compressor's on every tensor checked here, and the host compressor's equal the oracle's on
+the 4096x4096 matrix, on one DiT tensor of each shape and on the outlier matrix at 3.5 bpp."""
 import numpy as np
 import pytest
 import torch
@@ -18,35 +23,23 @@ def as_bytes(t):
     return t.contiguous().view(torch.uint8).cpu().numpy().reshape(-1)
 
 
-def decode_gpu(blob, lattice=False):
-    info = B.stream_info(blob)
-    d = blob.cuda()
+def decode_gpu(d_blob, info):
+    """container and lattice points of a device stream, with the decode's status checked"""
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    out = B.decompress(d, info, status=status, lattice=lattice)
+    work = B.prepare(d_blob, info, status=status)
+    out = B.decompress(d_blob, info, workspace=work, status=status)
+    v = B.decompress(d_blob, info, workspace=work, status=status, lattice=True)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    return info, out
+    return out, v
 
 
-def sampled_tiles(T, n=24, seed=0):
-    rng = np.random.default_rng(seed)
-    picks = set(range(min(4, T))) | set(range(max(0, T - 4), T))
-    picks |= set(int(t) for t in rng.integers(0, T, size=n))
-    return sorted(picks)
-
-
-def compare_tiles(oracle, blob, info, out, v, tiles):
-    nb = info.rows * info.cols // 8
-    per = 32 * info.blocks_per_lane
-    ob = as_bytes(out)
-    esz = out.element_size()
-    vv = v.cpu().numpy().reshape(-1)
-    for t in tiles:
-        rc, st, v_ref, out_ref = oracle.decode(blob.numpy(), t, t + 1)
-        assert rc == 0 and st == 0
-        lo, hi = 8 * t * per, 8 * min((t + 1) * per, nb)
-        assert np.array_equal(vv[lo:hi], v_ref.reshape(-1)[lo:hi]), t
-        assert np.array_equal(ob[lo * esz:hi * esz], out_ref.view(np.uint8).reshape(-1)[lo * esz:hi * esz]), t
+def check_all(oracle, host_blob, out, v, what):
+    """every container byte and every lattice point equal the oracle's decode of the stream"""
+    rc, st, v_ref, out_ref = oracle.decode_parallel(host_blob.numpy())
+    assert rc == 0 and st == 0, what
+    assert np.array_equal(as_bytes(out), out_ref.view(np.uint8).reshape(-1)), what
+    assert np.array_equal(v.cpu().numpy(), v_ref), what
 
 
 def test_lognormal_4096_full(oracle):
@@ -56,12 +49,12 @@ def test_lognormal_4096_full(oracle):
     blob = B.compress(w, 4.0)
     rc, ref = oracle.compress(w, 4.0)
     assert rc == 0 and np.array_equal(blob.numpy(), ref)
-    info, out = decode_gpu(blob)
+    d = B.compress_device(w.cuda(), 4.0)
+    assert np.array_equal(d.cpu().numpy(), ref)
+    info = B.stream_info(blob)
     assert info.actual_bpp <= 4.0
-    rc, st, v_ref, out_ref = oracle.decode(ref)
-    assert st == 0 and np.array_equal(as_bytes(out), out_ref.view(np.uint8).reshape(-1))
-    _, v = decode_gpu(blob, lattice=True)
-    assert np.array_equal(v.cpu().numpy(), v_ref)
+    out, v = decode_gpu(d, info)
+    check_all(oracle, blob, out, v, "4096x4096")
 
 
 @pytest.mark.parametrize("container", [B.INT8, B.FP8E4M3])
@@ -69,34 +62,51 @@ def test_codes_8192_full(oracle, container):
     """8192x8192 N(0, 0.02^2) as per-row absmax INT8 / FP8 codes at 3 bpp, all weights"""
     w = synth.gaussian(8192, 8192, 0.02, 2)
     blob = B.compress(w, 3.0, container=container)
-    info, out = decode_gpu(blob)
+    d = B.compress_device(w.cuda(), 3.0, container=container)
+    assert np.array_equal(d.cpu().numpy(), blob.numpy())
+    info = B.stream_info(blob)
     assert info.actual_bpp <= 3.0 and info.container_dtype == container
-    rc, st, v_ref, out_ref = oracle.decode(blob.numpy())
-    assert st == 0 and np.array_equal(as_bytes(out), out_ref.view(np.uint8).reshape(-1))
+    out, v = decode_gpu(d, info)
+    check_all(oracle, blob, out, v, container)
+
+
+@pytest.fixture(scope="module")
+def outlier_matrix():
+    return synth.gaussian_outliers(8192, 28672, 3)
 
 
 @pytest.mark.parametrize("target", [0.5, 1.0, 2.0, 3.5, 5.0, 8.0])
-def test_outlier_sweep_full(oracle, target):
-    """8192x28672 with 0.1% 8-sigma outliers across the bitrate sweep: sampled tiles"""
-    if not hasattr(test_outlier_sweep_full, "w"):
-        test_outlier_sweep_full.w = synth.gaussian_outliers(8192, 28672, 3)
-    w = test_outlier_sweep_full.w
-    blob = B.compress(w, target)
-    info, out = decode_gpu(blob)
-    _, v = decode_gpu(blob, lattice=True)
+def test_outlier_sweep_full(oracle, outlier_matrix, target):
+    """8192x28672 with 0.1 % 8-sigma outliers across the bitrate sweep: every weight"""
+    w = outlier_matrix
+    d = B.compress_device(w.cuda(), target)
+    host = d.cpu()
+    assert np.array_equal(B.compress(w, target).numpy(), host.numpy())
+    if target == 3.5:
+        rc, ref = oracle.compress(w, target)
+        assert rc == 0 and np.array_equal(ref, host.numpy())
+    info = B.stream_info(host)
     assert info.actual_bpp <= target
-    compare_tiles(oracle, blob, info, out, v, sampled_tiles(info.n_tiles, seed=int(target * 10)))
+    out, v = decode_gpu(d, info)
+    check_all(oracle, host, out, v, target)
 
 
-@pytest.mark.parametrize("block", [0, 27])
-@pytest.mark.parametrize("layer", [0, 1, 2, 3])
-def test_dit_layers(oracle, block, layer):
-    """DiT weight set (28 blocks, hidden 3072): the four layer shapes of the first and last
-    block at 2.5 and 4 bpp, sampled tiles"""
-    w = synth.dit_layer(block, layer)
-    for target in (2.5, 4.0):
-        blob = B.compress(w, target)
-        info, out = decode_gpu(blob)
-        _, v = decode_gpu(blob, lattice=True)
-        assert info.actual_bpp <= target
-        compare_tiles(oracle, blob, info, out, v, sampled_tiles(info.n_tiles, n=8, seed=block * 4 + layer))
+@pytest.mark.parametrize("target", [2.5, 4.0])
+def test_dit_weight_set_full(oracle, target):
+    """the DiT weight set (28 blocks x qkv 3072x9216, out 3072x3072, MLP 3072x12288 and
+    12288x3072, Student-t entries with per-row log-normal scale): all 112 tensors, every weight"""
+    for block in range(28):
+        for layer in range(4):
+            w = synth.dit_layer(block, layer)
+            d = B.compress_device(w.cuda(), target)
+            host = d.cpu()
+            if block == 0:
+                # one tensor of each shape: GPU compressor = host compressor = oracle
+                assert np.array_equal(B.compress(w, target).numpy(), host.numpy()), layer
+                if target == 4.0:
+                    rc, ref = oracle.compress(w, target)
+                    assert rc == 0 and np.array_equal(ref, host.numpy()), layer
+            info = B.stream_info(host)
+            assert info.actual_bpp <= target
+            out, v = decode_gpu(d, info)
+            check_all(oracle, host, out, v, (block, layer, target))
