@@ -58,12 +58,21 @@ WORKLOADS = {
         layers=lambda: [("w", lambda: _synth().gaussian(8192, 8192, 0.02, 2))], target=3.0, container="fp8_e4m3",
         dims=[(8192, 8192)],
         distribution="N(0, 0.02^2), seed 2, per-row absmax FP8 E4M3 codes", shape="8192x8192"),
+    "tile_ans_lognormal_4096x4096_bf16": dict(
+        layers=lambda: [("w", lambda: _synth().row_lognormal(4096, 4096, 1))], target=16.0, container=0,
+        dims=[(4096, 4096)], scheme="tile_ans", shape="4096x4096",
+        distribution="N(0, s_r^2), s_r = 0.02 exp(0.3 g), seed 1; lossless Tile-ANS (every bit kept)"),
     "outliers_8192x28672_bf16": dict(
         layers=lambda: [("w", lambda: _synth().gaussian_outliers(8192, 28672, 3))], target=4.0, container=0,
         dims=[(8192, 28672)],
         distribution="N(0, 0.02^2), seed 3, 0.1% of entries set to +-8 sigma", shape="8192x28672"),
 }
 DEFAULT_WORKLOAD = "lognormal_rows_4096x4096_bf16"
+TILE_ANS_METRIC = "lossless Tile-ANS decode GB/s (tensor out) & Gelements/s; % of HBM roofline"
+
+
+def is_tile_ans(a):
+    return WORKLOADS[a.workload].get("scheme") == "tile_ans"
 
 
 def _synth():
@@ -95,7 +104,8 @@ def coding_label(infos):
 
 def workload_config(a):
     wl = WORKLOADS[a.workload]
-    return {"workload": a.workload, "shape": wl["shape"], "target_bpp": a.target,
+    return {"workload": a.workload, "shape": wl["shape"],
+            "target_bpp": "lossless" if wl.get("scheme") == "tile_ans" else a.target,
             "distribution": wl["distribution"], "container": wl["container"] or "bf16"}
 
 
@@ -526,20 +536,204 @@ def run_ours(a, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ the lossless Tile-ANS workload
+def _bits(t):
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16) if t.element_size() == 2 else \
+        t.contiguous().view(torch.uint8).numpy()
+
+
+def run_ours_tile_ans(a, rank, world, local_rank):
+    """the lossless scheme's decode (ep_ans_decompress) of the workload's tensor, timed as the
+    lattice decode is: streams, tables and outputs resident, rotating copies past the L2, CUDA-graph
+    replays of exactly --steps decodes; e2e copies the stream in and the tensor out every step"""
+    from dit_weight_compression_tile_b200 import binding as B
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    name, make = WORKLOADS[a.workload]["layers"]()[0]
+    w = make()
+    t0 = time.perf_counter()
+    blob = B.ans_compress(w)
+    t_enc = time.perf_counter() - t0
+    info = B.ans_stream_info(blob)
+    in_bytes, out_bytes, n = info.storage_nbytes, info.out_nbytes, info.n_elems
+    rot = l2_policy(a)[0]
+    stream = torch.cuda.Stream(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    with torch.cuda.stream(stream):
+        blobs = [blob.to(dev) for _ in range(rot)]
+        works = [B.ans_prepare(d, info, status=status, stream=stream) for d in blobs]
+        outs = [torch.empty(info.shape, dtype=info.torch_dtype, device=dev) for _ in range(rot)]
+
+    def steps_(first, count):
+        for j in range(count):
+            r = (first + j) % rot
+            B.ans_decompress(blobs[r], info, workspace=works[r], out=outs[r], status=status, stream=stream)
+
+    with torch.cuda.stream(stream):
+        steps_(0, rot)
+    torch.cuda.synchronize(dev)
+    assert int(status.item()) == 0 and torch.equal(outs[0].cpu().view(torch.int16), w.view(torch.int16)), \
+        "lossless decode differs from the input"
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        steps_(0, rot)
+    replays, rest = divmod(a.steps, rot)
+    tail = None
+    if rest:
+        tail = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(tail, stream=stream):
+            steps_(0, rest)
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, -(-a.warmup // rot))):
+            graph.replay()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(replays + 2)]
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        with torch.cuda.stream(stream):
+            ev[0].record(stream)
+            for r in range(replays):
+                graph.replay()
+                ev[r + 1].record(stream)
+            if tail is not None:
+                tail.replay()
+            ev[-1].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    per_launch_us = sorted(1e3 * ev[r].elapsed_time(ev[r + 1]) / rot for r in range(replays))
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), world, dev)
+    assert int(status.item()) == 0
+    step_s = total_ms / a.steps / 1e3
+    kernel_s = ev[0].elapsed_time(ev[-1]) / a.steps / 1e3
+    peak, peak_kind = measured_peaks()
+    achieved = (in_bytes + out_bytes) / kernel_s / 1e9
+
+    # end to end through the public API's host-resident path: the pinned stream copied in, the
+    # decode, the tensor copied back into pinned memory, on two CUDA streams so that one step's
+    # copy-out overlaps the next step's copy-in
+    host_blob = blob.pin_memory()
+    host_outs = [torch.empty(info.shape, dtype=info.torch_dtype).pin_memory() for _ in range(2)]
+    streams = [stream, torch.cuda.Stream(dev)]
+    dblobs = [torch.empty_like(blobs[0]) for _ in range(2)]
+    douts = [torch.empty_like(outs[0]) for _ in range(2)]
+    dworks = [torch.empty_like(works[0]) for _ in range(2)]
+    e2e_steps = max(2, min(200, int(0.5 / max(1e-9, (in_bytes + out_bytes) / 40e9))))
+
+    def e2e_step(j):
+        s_ = streams[j % 2]
+        with torch.cuda.stream(s_):
+            dblobs[j % 2].copy_(host_blob, non_blocking=True)
+            B.ans_prepare(dblobs[j % 2], info, workspace=dworks[j % 2], stream=s_)
+            B.ans_decompress(dblobs[j % 2], info, workspace=dworks[j % 2], out=douts[j % 2], stream=s_)
+            host_outs[j % 2].copy_(douts[j % 2], non_blocking=True)
+
+    e2e_step(0)
+    torch.cuda.synchronize(dev)
+    e0, e1, ej = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True), torch.cuda.Event())
+    e0.record(streams[0])
+    streams[1].wait_event(e0)
+    for j in range(e2e_steps):
+        e2e_step(j)
+    ej.record(streams[1])
+    streams[0].wait_event(ej)
+    e1.record(streams[0])
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    if rank != 0:
+        return
+    line = {
+        "metric": TILE_ANS_METRIC, "value": round(job_rate(out_bytes, world, step_s) / 1e9, 2), "unit": "GB/s",
+        "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(step_s * 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32+u8", "data": "synthetic",
+        "config": bench_config(a, world),
+        "stream": {"ratio": round(info.ratio, 5), "bits_per_element": round(8.0 * in_bytes / n, 4),
+                   "n_tiles": info.n_tiles, "blocks_per_lane": info.blocks_per_lane, "lossless": True},
+        "gelements_per_s": round(job_rate(n, world, step_s) / 1e9, 3),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": in_bytes + out_bytes, "kernel_us": round(kernel_s * 1e6, 3),
+                     "kernel_us_median": round(statistics.median(per_launch_us), 3) if per_launch_us else None,
+                     "kernel_us_min": round(per_launch_us[0], 3) if per_launch_us else None},
+        "e2e": {"value": round(job_rate(out_bytes * e2e_steps, world, e2e_ms / 1e3) / 1e9, 3), "unit": "GB/s",
+                "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes},
+        "gpu_launches": a.steps,
+        "clocks": clk.summary(),
+        "encode_s": round(t_enc, 3),
+    }
+    if world == 1 and not a.no_cpu_baseline:
+        from concurrent.futures import ThreadPoolExecutor
+        from oracle import oracle as O
+        ncores = host_cores()
+        b_np = blob.numpy()
+        t0 = time.perf_counter()
+        done = 0
+        with ThreadPoolExecutor(ncores) as ex:
+            while time.perf_counter() - t0 < a.cpu_seconds:
+                cuts = [(info.n_tiles * i) // ncores for i in range(ncores + 1)]
+                list(ex.map(lambda i: O.ta_decode(b_np, cuts[i], cuts[i + 1]), range(ncores)))
+                done += 1
+        el = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": round(done * out_bytes / el / 1e9, 4), "unit": "GB/s", "cores": ncores,
+                                "kind": "oracle", "sample": f"{done} whole-stream decodes by the C oracle on "
+                                                            f"{ncores} threads in {el:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_tile_ans(a, rank, world):
+    """the oracle's Tile-ANS decoder on every host core, on the oracle's own stream of the workload"""
+    if rank != 0:
+        return
+    from concurrent.futures import ThreadPoolExecutor
+    from oracle import oracle as O
+    name, make = WORKLOADS[a.workload]["layers"]()[0]
+    w = make()
+    rc, blob = O.ta_compress(_bits(w), O.BF16, shape=tuple(w.shape))
+    assert rc == O.OK
+    rc, info = O.ta_parse(blob)
+    ncores = host_cores()
+    out_bytes = info.n * 2
+    pool = ThreadPoolExecutor(ncores)
+    cuts = [(info.n_tiles * i) // ncores for i in range(ncores + 1)]
+
+    def step():
+        list(pool.map(lambda i: O.ta_decode(blob, cuts[i], cuts[i + 1]), range(ncores)))
+
+    for _ in range(a.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        step()
+    t = time.perf_counter() - t0
+    pool.shutdown()
+    gbs = out_bytes * a.steps / t / 1e9
+    line = {"impl": "reference", "metric": TILE_ANS_METRIC, "value": round(gbs, 4), "unit": "GB/s",
+            "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(1e3 * t / a.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32+u8",
+            "data": "synthetic", "config": bench_config(a, world),
+            "gelements_per_s": round(info.n * a.steps / t / 1e9, 4),
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": ncores, "kind": "oracle",
+                             "sample": f"the whole stream ({info.n_tiles} tiles) per step, decoded by the C oracle "
+                                       f"on {ncores} threads"},
+            "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     a = args_()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if a.impl == "reference":
-        run_reference(a, rank, world)
+        (run_reference_tile_ans if is_tile_ans(a) else run_reference)(a, rank, world)
         return
     if world > 1:
         import datetime
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        run_ours(a, rank, world, local_rank)
+        (run_ours_tile_ans if is_tile_ans(a) else run_ours)(a, rank, world, local_rank)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -9,7 +9,7 @@ _BINDING_NAMES = ("BF16", "FP16", "FP32", "INT8", "FP8E4M3", "EpError", "compres
                   "decompress", "decompress_host", "stream_info", "lib", "StreamInfo")
 
 
-_COMPRESSED_NAMES = ("CompressedTensor", "LatticeRANSConfig")
+_COMPRESSED_NAMES = ("CompressedTensor", "LatticeRANSConfig", "TileANSConfig")
 _LINEAR_NAMES = ("CompressedLinear", "CompressedFP8Linear", "CompressedINT8Linear")
 
 

@@ -58,6 +58,29 @@ class StreamInfo(C.Structure):
         return self.storage_nbytes - (0 if include_header else self.header_nbytes)
 
 
+class AnsConfig(C.Structure):
+    _fields_ = [("dtype", C.c_int32), ("blocks_per_lane", C.c_uint32), ("n_threads", C.c_int32),
+                ("reserved", C.c_int32)]
+
+
+class AnsInfo(C.Structure):
+    _fields_ = [
+        ("n_elems", C.c_int64), ("dtype", C.c_int32), ("ndim", C.c_int32), ("shape_", C.c_int64 * 8),
+        ("storage_nbytes", C.c_uint64), ("ratio", C.c_double), ("n_tiles", C.c_uint32),
+        ("blocks_per_lane", C.c_uint32), ("off_freq", C.c_uint64), ("off_dir", C.c_uint64),
+        ("off_raw", C.c_uint64), ("off_tiles", C.c_uint64), ("out_nbytes", C.c_uint64),
+        ("max_tile_nbytes", C.c_uint64), ("workspace_nbytes", C.c_uint64),
+    ]
+
+    @property
+    def shape(self):
+        return tuple(self.shape_[: self.ndim])
+
+    @property
+    def torch_dtype(self):
+        return TORCH_DTYPE[self.dtype]
+
+
 _lib = None
 
 
@@ -97,6 +120,17 @@ def lib():
         L.ep_decompress_host_scratch.argtypes = [C.POINTER(StreamInfo), C.c_int32]
         L.ep_decompress_host.restype = C.c_int
         L.ep_decompress_host.argtypes = [C.POINTER(StreamInfo), p, p, C.c_int32, p, C.c_size_t, p, p]
+        L.ep_ans_compress_bound.restype = C.c_size_t
+        L.ep_ans_compress_bound.argtypes = [C.c_int64, C.c_int32]
+        L.ep_ans_compress_host.restype = C.c_int
+        L.ep_ans_compress_host.argtypes = [p, C.c_int64, C.c_int32, p, C.POINTER(AnsConfig), p, C.c_size_t,
+                                           C.POINTER(C.c_size_t)]
+        L.ep_ans_stream_info.restype = C.c_int
+        L.ep_ans_stream_info.argtypes = [p, C.c_size_t, C.POINTER(AnsInfo)]
+        L.ep_ans_prepare.restype = C.c_int
+        L.ep_ans_prepare.argtypes = [C.POINTER(AnsInfo), p, p, p, p]
+        L.ep_ans_decompress.restype = C.c_int
+        L.ep_ans_decompress.argtypes = [C.POINTER(AnsInfo), p, p, p, p, p]
         L.ep_status_string.restype = C.c_char_p
         L.ep_status_string.argtypes = [C.c_int]
         _lib = L
@@ -292,4 +326,76 @@ def decompress_host(h_blob, info=None, out=None, out_dtype=None, scratch=None, s
         raise EpError(rc, "ep_decompress_host")
     if sync:
         cs.synchronize()
+    return out
+
+
+# ---------------------------------------------------------------- the Tile-ANS lossless scheme
+def ans_compress(tensor, blocks_per_lane=0, n_threads=0):
+    """compress(tensor, TileANSConfig()) on the host (ep_ans_compress_host): every bit of a BF16,
+    FP16, FP32, INT8 or FP8 E4M3 tensor of any shape (1 to 8 dims).  Returns the stream as a CPU
+    uint8 tensor."""
+    if tensor.dtype not in CODE_OF:
+        raise EpError(-1, f"Tile-ANS takes BF16, FP16, FP32, INT8 or FP8 E4M3, not {tensor.dtype}")
+    if tensor.numel() == 0 or tensor.dim() < 1 or tensor.dim() > 8:
+        raise EpError(-1, "Tile-ANS needs a non-empty tensor of 1 to 8 dims")
+    src = tensor.detach().to("cpu").contiguous()
+    cfg = AnsConfig(CODE_OF[src.dtype], int(blocks_per_lane), int(n_threads), 0)
+    dims = (C.c_int64 * 8)(*src.shape)
+    L = lib()
+    cap = L.ep_ans_compress_bound(src.numel(), cfg.dtype)
+    out = torch.empty(max(cap, 1024), dtype=torch.uint8)
+    n = C.c_size_t(0)
+    rc = L.ep_ans_compress_host(src.data_ptr(), src.numel(), src.dim(), dims, C.byref(cfg), out.data_ptr(),
+                                out.numel(), C.byref(n))
+    if rc == -5:
+        out = torch.empty(n.value, dtype=torch.uint8)
+        rc = L.ep_ans_compress_host(src.data_ptr(), src.numel(), src.dim(), dims, C.byref(cfg), out.data_ptr(),
+                                    out.numel(), C.byref(n))
+    if rc != 0:
+        raise EpError(rc, "ep_ans_compress_host")
+    return out[: n.value].clone()
+
+
+def ans_stream_info(blob):
+    b = blob.detach().to("cpu").contiguous()
+    info = AnsInfo()
+    rc = lib().ep_ans_stream_info(b.data_ptr(), b.numel(), C.byref(info))
+    if rc != 0:
+        raise EpError(rc, "ep_ans_stream_info")
+    return info
+
+
+def ans_prepare(d_blob, info, workspace=None, status=None, stream=None):
+    """the decoder's slot table for one device copy of a Tile-ANS stream (ep_ans_prepare)"""
+    if not d_blob.is_cuda:
+        raise EpError(-1, "ans_prepare needs the stream in device memory")
+    if workspace is None:
+        workspace = torch.empty(info.workspace_nbytes, dtype=torch.uint8, device=d_blob.device)
+    if not workspace.is_cuda or workspace.numel() < info.workspace_nbytes:
+        raise EpError(-1, "workspace does not match the stream")
+    st = status.data_ptr() if status is not None else None
+    s = (stream or torch.cuda.current_stream(d_blob.device)).cuda_stream
+    rc = lib().ep_ans_prepare(C.byref(info), d_blob.data_ptr(), workspace.data_ptr(), st, s)
+    if rc != 0:
+        raise EpError(rc, "ep_ans_prepare")
+    return workspace
+
+
+def ans_decompress(d_blob, info, workspace=None, out=None, status=None, stream=None):
+    """decompress of a device-resident Tile-ANS stream (ep_ans_decompress): the tensor, bit for bit.
+    Without ``workspace`` the table is prepared here on every call."""
+    if not d_blob.is_cuda:
+        raise EpError(-1, "ans_decompress needs the stream in device memory")
+    if workspace is None:
+        workspace = ans_prepare(d_blob, info, status=status, stream=stream)
+    want = TORCH_DTYPE[info.dtype]
+    if out is None:
+        out = torch.empty(info.shape, dtype=want, device=d_blob.device)
+    if not out.is_cuda or out.dtype != want or tuple(out.shape) != info.shape or not out.is_contiguous():
+        raise EpError(-1, "output tensor does not match the stream")
+    st = status.data_ptr() if status is not None else None
+    s = (stream or torch.cuda.current_stream(d_blob.device)).cuda_stream
+    rc = lib().ep_ans_decompress(C.byref(info), d_blob.data_ptr(), workspace.data_ptr(), out.data_ptr(), st, s)
+    if rc != 0:
+        raise EpError(rc, "ep_ans_decompress")
     return out

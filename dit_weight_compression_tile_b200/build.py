@@ -12,8 +12,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libeptile.so")
-SOURCES = ["decode.cu", "device_encode.cu", "host_encode.cpp", "host_stream.cpp"]
-HEADERS = [os.path.join(CSRC, h) for h in ("format.h", "encode_math.h", "encode_host.h")] + \
+SOURCES = ["decode.cu", "device_encode.cu", "host_encode.cpp", "host_stream.cpp", "tile_ans.cu", "tile_ans_host.cpp"]
+HEADERS = [os.path.join(CSRC, h) for h in ("format.h", "encode_math.h", "encode_host.h", "device_util.cuh",
+                                           "tile_ans.h")] + \
     [os.path.join(ROOT, "include", "eptile.h")]
 
 

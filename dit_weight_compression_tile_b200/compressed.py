@@ -4,9 +4,13 @@ over the C ABI: ep_compress_device (a CUDA tensor) or ep_compress_host (a host t
 stream, the same bytes either way; ep_prepare and the fused ep_decompress kernel decode it.  This module only keeps the pieces together (stream,
 parsed plan, prepared tables, output dtype); it computes nothing itself.
 
+Two schemes: the lossy lattice-rANS tile stream (LatticeRANSConfig) and the lossless Tile-ANS
+stream (TileANSConfig: each element's top byte rANS-coded in the same lane tiles, the other bytes
+kept as they are; ep_ans_compress_host, ep_ans_prepare, ep_ans_decompress).
+
 Differences from the pages, by design: CompressedTensor is a plain object, not a torch.Tensor
-subclass; decoding needs the stream on a CUDA device (no CPU decoder); the only scheme is the
-lattice-rANS tile stream (plus the "raw" container that the pages return when encoding fails).
+subclass; decoding needs a CUDA device (no CPU decoder); DFloat11Config is not offered (Tile-ANS
+covers BF16 losslessly); the "raw" container that the pages return when encoding fails is kept.
 """
 import math
 import warnings
@@ -17,7 +21,7 @@ import torch
 from . import binding as B
 
 STATE_VERSION = 1
-_LATTICE, _RAW = 0, 1
+_LATTICE, _RAW, _TILE_ANS = 0, 1, 2
 _ELT = {torch.bfloat16: 2, torch.float16: 2, torch.float32: 4, torch.int8: 1, torch.float8_e4m3fn: 1}
 
 
@@ -36,23 +40,34 @@ class LatticeRANSConfig:
     coding: int = 0
 
 
-class CompressedTensor:
-    """One compressed 2-D tensor: the stream (a uint8 tensor on some device) and its parsed plan,
-    or, for compress_method == "raw", the tensor itself."""
+@dataclass
+class TileANSConfig:
+    """The lossless scheme: every bit of a BF16, FP16, FP32, INT8 or FP8 E4M3 tensor of any shape.
+    blocks_per_lane: chunks of 8 elements per lane, 0 picks it from the size.  n_threads: host
+    encoder threads (0: all cores)."""
+    blocks_per_lane: int = 0
+    n_threads: int = 0
 
-    def __init__(self, blob=None, info=None, out_dtype=None, raw=None):
-        self._blob, self._info, self._raw = blob, info, raw
-        self._dtype = out_dtype if out_dtype is not None else (raw.dtype if raw is not None else info.dtype)
+
+class CompressedTensor:
+    """One compressed tensor: the stream (a uint8 tensor on some device) and its parsed plan, or,
+    for compress_method == "raw", the tensor itself.  ``ans`` marks a Tile-ANS stream."""
+
+    def __init__(self, blob=None, info=None, out_dtype=None, raw=None, ans=False):
+        self._blob, self._info, self._raw, self._ans = blob, info, raw, ans
+        if out_dtype is None:
+            out_dtype = raw.dtype if raw is not None else (info.torch_dtype if ans else info.dtype)
+        self._dtype = out_dtype
         self._work = None  # (workspace, event) of the slot tables prepared for this device copy
 
     # ---- properties of the API reference
     @property
     def compress_method(self):
-        return "raw" if self._raw is not None else "lattice_rans"
+        return "raw" if self._raw is not None else ("tile_ans" if self._ans else "lattice_rans")
 
     @property
     def lossless(self):
-        return self._raw is not None
+        return self._raw is not None or self._ans
 
     @property
     def shape(self):
@@ -65,7 +80,9 @@ class CompressedTensor:
 
     @property
     def encoded_dtype(self):
-        return self._raw.dtype if self._raw is not None else self._info.dtype
+        if self._raw is not None:
+            return self._raw.dtype
+        return self._info.torch_dtype if self._ans else self._info.dtype
 
     @property
     def device(self):
@@ -82,7 +99,8 @@ class CompressedTensor:
     def storage_nbytes(self, include_header=True):
         if self._raw is not None:
             return self._raw.numel() * _ELT[self._raw.dtype]
-        return self._info.storage_nbytes - (0 if include_header else self._info.header_nbytes)
+        header = 64 if self._ans else self._info.header_nbytes
+        return self._info.storage_nbytes - (0 if include_header else header)
 
     @property
     def actual_bpp(self):
@@ -96,7 +114,9 @@ class CompressedTensor:
         if isinstance(device, torch.dtype):
             device, dtype = None, device
         dtype = self._dtype if dtype is None else dtype
-        if self._raw is None and dtype != self._dtype:
+        if self._ans and dtype != self._dtype:
+            raise B.EpError(-1, "a lossless Tile-ANS stream decodes to its own dtype only")
+        if self._raw is None and not self._ans and dtype != self._dtype:
             if B.dtype_code(dtype) not in _allowed_out(self._info.container_dtype):
                 raise B.EpError(-1, f"a {self._info.dtype} container does not decode to {dtype}")
         dev = self.device if device is None else torch.device(device)
@@ -104,15 +124,15 @@ class CompressedTensor:
             raw = self._raw.to(dev, copy=copy)
             return CompressedTensor(raw=raw, out_dtype=dtype)
         blob = self._blob.to(dev, copy=copy)
-        ct = CompressedTensor(blob, self._info, dtype)
+        ct = CompressedTensor(blob, self._info, dtype, ans=self._ans)
         if blob.data_ptr() == self._blob.data_ptr():
             ct._work = self._work  # same device copy: the prepared tables stay valid
         return ct
 
     def state_dict(self, prefix=""):
         """tensors only, so that torch.load(..., weights_only=True) restores it"""
-        meta = torch.tensor([STATE_VERSION, _RAW if self._raw is not None else _LATTICE,
-                             _dtype_tag(self._dtype)], dtype=torch.int64)
+        method = _RAW if self._raw is not None else (_TILE_ANS if self._ans else _LATTICE)
+        meta = torch.tensor([STATE_VERSION, method, _dtype_tag(self._dtype)], dtype=torch.int64)
         if self._raw is not None:
             return {prefix + "ep_meta": meta, prefix + "ep_raw": self._raw}
         return {prefix + "ep_meta": meta, prefix + "ep_stream": self._blob}
@@ -128,6 +148,13 @@ class CompressedTensor:
         blob = state[prefix + "ep_stream"]
         if blob.dtype != torch.uint8 or blob.dim() != 1:
             raise B.EpError(-6, "stream tensor")
+        if meta[1] == _TILE_ANS:
+            info = B.ans_stream_info(_host_view(blob))
+            if blob.numel() != info.storage_nbytes:
+                raise B.EpError(-6, "stream length")
+            return cls(blob, info, out_dtype, ans=True)
+        if meta[1] != _LATTICE:
+            raise B.EpError(-6, f"method tag {meta[1]}")
         info = B.stream_info(_host_view(blob))
         if blob.numel() != info.storage_nbytes:
             raise B.EpError(-6, "stream length")
@@ -162,11 +189,17 @@ def _host_view(blob):
 
 
 def compress(tensor, config):
-    """compress(tensor, config) -> CompressedTensor on the tensor's device.  Input: non-empty,
-    2-D, finite BF16 / FP16 / FP32.  If even the coarsest resolution exceeds the target, a
-    warning says so and the tensor is kept uncompressed (compress_method == "raw")."""
+    """compress(tensor, config) -> CompressedTensor on the tensor's device.
+    LatticeRANSConfig: a non-empty, 2-D, finite BF16 / FP16 / FP32 tensor; if even the coarsest
+    resolution exceeds the target, a warning says so and the tensor is kept uncompressed
+    (compress_method == "raw").  TileANSConfig: any non-empty BF16 / FP16 / FP32 / INT8 / FP8 E4M3
+    tensor of 1 to 8 dims, every bit kept (the host compressor encodes a copy of a CUDA tensor)."""
+    if isinstance(config, TileANSConfig):
+        blob = B.ans_compress(tensor, blocks_per_lane=config.blocks_per_lane, n_threads=config.n_threads)
+        info = B.ans_stream_info(blob)
+        return CompressedTensor(blob.to(tensor.device), info, tensor.dtype, ans=True)
     if not isinstance(config, LatticeRANSConfig):
-        raise B.EpError(-1, "config must be a LatticeRANSConfig")
+        raise B.EpError(-1, "config must be a LatticeRANSConfig or a TileANSConfig")
     container = 0 if config.container is None else config.container
     try:
         if tensor.is_cuda:  # the GPU compressor writes the host compressor's bytes
@@ -191,7 +224,7 @@ def compress(tensor, config):
 def _tables(ct, stream):
     """slot tables for this device copy, prepared once; later decodes on other streams wait for them"""
     if ct._work is None:
-        work = B.prepare(ct._blob, ct._info, stream=stream)
+        work = (B.ans_prepare if ct._ans else B.prepare)(ct._blob, ct._info, stream=stream)
         ev = torch.cuda.Event()
         ev.record(stream)
         ct._work = (work, ev)
@@ -209,6 +242,22 @@ def decompress(compressed, config=None, stream=None, out=None, status=None):
     ct = compressed
     if ct._raw is not None:
         return ct._raw.to(dtype=ct.dtype, copy=True)
+    if ct._ans:
+        if not ct._blob.is_cuda:
+            # the GPU decodes a host-resident stream: copy in, decode, copy back
+            if not torch.cuda.is_available():
+                raise B.EpError(-1, "decompress decodes on a CUDA device and none is available")
+            dev = torch.device("cuda", torch.cuda.current_device())
+            s = stream or torch.cuda.current_stream(dev)
+            with torch.cuda.stream(s):
+                d = ct._blob.to(dev, non_blocking=False)
+                res = B.ans_decompress(d, ct._info, status=status, stream=s)
+                host = res.to("cpu") if out is None else out.copy_(res)
+            s.synchronize()
+            return host
+        s = stream or torch.cuda.current_stream(ct._blob.device)
+        work = _tables(ct, s)
+        return B.ans_decompress(ct._blob, ct._info, workspace=work, out=out, status=status, stream=s)
     if not ct._blob.is_cuda:
         if out is not None and out.is_cuda:
             raise B.EpError(-1, "the output of a host-resident stream is a host tensor")

@@ -31,6 +31,7 @@
 #include <mutex>
 
 #include "../../include/eptile.h"
+#include "device_util.cuh"
 #include "format.h"
 
 namespace ep {
@@ -57,7 +58,6 @@ enum Coding { kNarrow = 0, kWide = 1, kPaired = 2 };
 constexpr uint32_t kSlack = 160;      // bytes past a tile that a lane's bounded over-read may touch
                                       // (8 blocks of 8 tokens between checks, one word each, + 1)
 constexpr size_t kSmemLimit = 232448; // shared memory one CTA may use on sm_100
-constexpr uint32_t kWaitLimit = 1u << 22;  // mbarrier polls before a copy is declared lost
 static_assert(kFixedBytes % 16 == 0, "tile buffers must start 16-byte aligned");
 
 // slot entry: bias [0,11) | value field [11,20) | escape [20] | frequency [21,32)
@@ -100,53 +100,6 @@ __device__ __forceinline__ uint32_t split_of_bits(uint32_t splits, uint32_t c) {
 __device__ __forceinline__ uint32_t split_of(const Params &p, uint32_t c) { return split_of_bits(p.splits, c); }
 
 __device__ __forceinline__ int32_t unzigzag(uint32_t u) { return int32_t(u >> 1) ^ -int32_t(u & 1u); }
-
-// ------------------------------------------------------------------ shared memory, mbarriers, bulk copies
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-    uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ uint32_t lds16(uint32_t a) {
-    uint32_t v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ void lds64(uint32_t a, uint32_t &lo, uint32_t &hi) {
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo), "=r"(hi) : "r"(a));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-// the issuing thread's arrival, announcing the bytes the copy will deliver
-__device__ __forceinline__ void mbar_expect(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// bounded wait for a phase; false when the limit ran out
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i)
-        if (mbar_try(bar, parity)) return true;
-    return false;
-}
-// one bulk copy global -> this CTA's shared memory, completing on an mbarrier (TMA, no tensor map)
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
-        "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
-}
-// orders this thread's earlier generic-proxy accesses of shared memory before later async-proxy ones
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // ------------------------------------------------------------------ containers
 // put(i, v, w): coordinate i of the block, v the exact lattice value as a float and w = fp32(f_r v)

@@ -240,6 +240,74 @@ size_t ep_decompress_host_scratch(const ep_info *info, int32_t out_dtype);
 int ep_decompress_host(const ep_info *info, const void *h_blob, void *h_out, int32_t out_dtype, void *d_scratch,
                        size_t scratch_nbytes, uint32_t *d_status, ep_stream_t stream);
 
+/* ---------------------------------------------------------------- the Tile-ANS lossless scheme
+ * "EntroPack README", Configuration (TileANSConfig: lossless compression for BF16, FP16, FP32,
+ * FP8 and INT8 tensors, the ratio depending on the data) and "EntroPack API reference",
+ * decompress (lossless schemes restore every input bit).  The pages give no format; this
+ * library's (format version 1): each element's most significant byte (the sign and top exponent
+ * bits of a float, the whole byte of an 8-bit type) is rANS-coded with one static 256-symbol
+ * table of 12-bit frequencies, in the lattice stream's lane tiles (chunks of 8 elements, 32 or 16
+ * chunks per lane); the element's other bytes are kept as they are in a raw plane. */
+
+typedef struct {
+    int32_t dtype;            /* EP_BF16, EP_FP16, EP_FP32, EP_INT8 or EP_FP8_E4M3 */
+    uint32_t blocks_per_lane; /* chunks of 8 elements per lane; 0 = 32, or 16 below 1024 tiles */
+    int32_t n_threads;        /* host encoder threads; 0 = all hardware threads */
+    int32_t reserved;         /* 0 */
+} ep_ans_config;
+
+typedef struct {
+    int64_t n_elems;
+    int32_t dtype, ndim;
+    int64_t shape[8];         /* ndim dims, product n_elems */
+    uint64_t storage_nbytes;  /* total stream bytes */
+    double ratio;             /* storage_nbytes / (n_elems * element size) */
+    uint32_t n_tiles, blocks_per_lane;
+    uint64_t off_freq, off_dir, off_raw, off_tiles;
+    uint64_t out_nbytes;      /* n_elems * element size */
+    uint64_t max_tile_nbytes; /* largest tile (sizes the decoder's staging buffers) */
+    uint64_t workspace_nbytes;/* 16384: the decoder's 4096-slot table */
+} ep_ans_info;
+
+/* Size of the Tile-ANS stream of n elements of `dtype` is at most this (0 for invalid
+ * arguments): the raw bytes, one byte per element for the coded symbols plus their
+ * worst-case growth, tables and tile heads. */
+size_t ep_ans_compress_bound(int64_t n_elems, int32_t dtype);
+
+/* compress(tensor, TileANSConfig()) on the host.
+ *   src        host pointer to n_elems elements of cfg->dtype (any bit patterns: NaN payloads,
+ *              infinities, signed zeros and subnormals are kept), read only.
+ *   ndim/shape the tensor's shape (1..8 dims, product n_elems), stored for decompress.
+ *   out        host buffer of out_cap bytes, caller-owned; out_nbytes receives the size (also on
+ *              EP_ERR_BUFFER_TOO_SMALL: the size needed).
+ * Byte-identical to the oracle's compressor.  Errors: EP_ERR_INVALID_ARG (null, empty, bad
+ * dtype or shape), EP_ERR_BUFFER_TOO_SMALL, EP_ERR_UNSUPPORTED (a lane region beyond 65535
+ * words with a forced tile size). */
+int ep_ans_compress_host(const void *src, int64_t n_elems, int32_t ndim, const int64_t *shape,
+                         const ep_ans_config *cfg, void *out, size_t out_cap, size_t *out_nbytes);
+
+/* Parses and validates a host copy of a Tile-ANS stream (header, tables, directory and total
+ * length).  EP_ERR_CORRUPT when it fails. */
+int ep_ans_stream_info(const void *blob, size_t nbytes, ep_ans_info *info);
+
+/* The decoder's slot table (4096 x u32: frequency, symbol, slot offset) from the stream's
+ * frequencies, into a caller-owned device workspace of info->workspace_nbytes, 16-byte aligned;
+ * once per device copy of a stream.  Tables that do not sum to 2^12 set EP_DEC_BAD_TOKEN in
+ * d_status (nullable).  One small launch on `stream`; asynchronous. */
+int ep_ans_prepare(const ep_ans_info *info, const void *d_blob, void *d_workspace, uint32_t *d_status,
+                   ep_stream_t stream);
+
+/* decompress(compressed) of a Tile-ANS stream in device memory: every element bit for bit.
+ *   d_blob      device copy of the whole stream (16-byte aligned), caller-owned.
+ *   d_workspace the table ep_ans_prepare filled from this copy.
+ *   d_out       device buffer of info->out_nbytes (16-byte aligned): the tensor, row-major.
+ *   d_status    nullable device uint32: EP_DEC_* bits of stream damage.
+ * One persistent launch (one CTA per SM): the table and each warp's tiles staged in shared
+ * memory by bulk copies, 32 rANS lanes per tile, each lane merging its decoded top bytes with
+ * the raw plane and storing whole chunks.  Asynchronous; allocates nothing. */
+int ep_ans_decompress(const ep_ans_info *info, const void *d_blob, const void *d_workspace, void *d_out,
+                      uint32_t *d_status, ep_stream_t stream);
+
 /* static string for a status code */
 const char *ep_status_string(int status);
 

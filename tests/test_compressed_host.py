@@ -104,3 +104,25 @@ def test_config_coding_reaches_the_stream(oracle):
     assert paired._info.paired == 1 and single._info.paired == 0
     rc, ref = oracle.compress(w, 4.0, coding=oracle.CODING_PAIRED)
     assert np.array_equal(paired.blob.numpy(), ref)
+
+
+def test_tile_ans_container_host():
+    """compress(tensor, TileANSConfig()): a lossless container of any shape and dtype; its
+    properties, its state_dict round trip and the refusal to change dtype"""
+    from dit_weight_compression_tile_b200.compressed import TileANSConfig
+    for t in (synth.row_lognormal(64, 256, seed=30), synth.gaussian(4, 8, 0.02, seed=31).float().reshape(2, 2, 8),
+              torch.clamp(torch.round(torch.randn(1000) * 20), -127, 127).to(torch.int8)):
+        ct = compress(t, TileANSConfig())
+        assert ct.compress_method == "tile_ans" and ct.lossless
+        assert ct.shape == t.shape and ct.dtype == t.dtype and ct.encoded_dtype == t.dtype
+        assert ct.storage_nbytes() == ct.blob.numel() and ct.storage_nbytes(include_header=False) == ct.blob.numel() - 64
+        assert ct.actual_bpp == pytest.approx(8.0 * ct.blob.numel() / t.numel())
+        with pytest.raises(B.EpError):
+            ct.to(dtype=torch.float16 if t.dtype != torch.float16 else torch.float32)
+        buf = io.BytesIO()
+        torch.save(ct.state_dict("w."), buf)
+        buf.seek(0)
+        back = CompressedTensor.from_state_dict(torch.load(buf, weights_only=True), "w.")
+        assert back.compress_method == "tile_ans" and torch.equal(back.blob, ct.blob) and back.shape == t.shape
+    bf16 = compress(synth.row_lognormal(512, 512, seed=32), TileANSConfig())
+    assert 0.66 * 16 < bf16.actual_bpp < 0.72 * 16

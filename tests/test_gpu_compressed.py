@@ -110,3 +110,21 @@ def test_host_buffer_decode(oracle, container, out_dt, shape):
         via_ct = ct.decompress()
         assert via_ct.device.type == "cpu"
         assert np.array_equal(as_bytes(via_ct), ref.view(np.uint8).reshape(-1))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16, torch.float32, torch.int8, torch.float8_e4m3fn])
+def test_tile_ans_round_trip(dtype):
+    """compress(tensor, TileANSConfig()) and decompress on the GPU, from a CUDA tensor and from a
+    host-resident stream: every bit of the input, in its shape and dtype"""
+    from dit_weight_compression_tile_b200.compressed import TileANSConfig
+    g = torch.Generator().manual_seed(40)
+    t = (torch.randn(3, 257, 129, generator=g) * (20 if dtype in (torch.int8, torch.float8_e4m3fn) else 0.02)).to(dtype)
+    view = torch.int16 if t.element_size() == 2 else (torch.int32 if t.element_size() == 4 else torch.uint8)
+    for src in (t, t.cuda()):
+        ct = compress(src, TileANSConfig())
+        assert ct.device == src.device and ct.lossless
+        out = decompress(ct)
+        assert out.device == src.device and out.dtype == dtype and out.shape == t.shape
+        assert torch.equal(out.cpu().view(view), t.view(view))
+        # a second decode reuses the prepared table
+        assert torch.equal(ct.decompress().cpu().view(view), t.view(view))
