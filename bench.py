@@ -90,9 +90,22 @@ def args_():
     p.add_argument("--target", type=float, default=None, help="bits per weight (default: the workload's)")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--shape", default=None,
+                   help="RxC: the workload's first R rows and C columns instead of the whole tensor "
+                        "(single-tensor workloads; a smaller case of the same kernel for profiler captures)")
     a = p.parse_args()
     wl = WORKLOADS[a.workload]
     a.target = wl["target"] if a.target is None else a.target
+    if a.shape:
+        if len(wl["dims"]) != 1:
+            raise SystemExit("--shape applies to single-tensor workloads")
+        R, Cc = (int(v) for v in a.shape.lower().split("x"))
+        full = wl["layers"]()[0][1]
+        sub = dict(wl)
+        sub["layers"] = lambda: [("w", lambda: full()[:R, :Cc].contiguous())]
+        sub["dims"] = [(R, Cc)]
+        sub["shape"] = f"{R}x{Cc} (top-left part of {wl['shape']})"
+        WORKLOADS[a.workload] = sub
     return a
 
 
