@@ -34,7 +34,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "fused decode GB/s (container out) & Gweights/s at 4 bpp; % of HBM roofline"
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
-KERNEL_SRC = os.path.join(ROOT, "dit_weight_compression_tile_b200", "csrc", "decode.cu")
+KERNEL_SRCS = {"decode_kernel": ("decode.cu", "device_util.cuh", "format.h"),
+               "ans_decode_kernel": ("tile_ans.cu", "device_util.cuh", "tile_ans.h")}
 L2_BYTES = 126 * 2 ** 20
 
 # The workloads (synthetic, seeded; shapes and distributions as stated).  The default is the
@@ -292,17 +293,39 @@ def cpu_oracle_decode(blob_np, seconds, threads=1):
     return sum(r[0] for r in res), t, sum(r[1] for r in res)
 
 
-def traffic_for_kernel(workload):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on this kernel source"""
+def kernel_source_hash(kernel):
+    """sha256 (16 hex digits) of the sources that make up a kernel"""
+    h = hashlib.sha256()
+    for name in KERNEL_SRCS[kernel]:
+        with open(os.path.join(ROOT, "dit_weight_compression_tile_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for_kernel(kernel, key):
+    """DRAM bytes per launch (read + write) from the committed ncu record for this workload key,
+    if it was captured on the kernel's current sources; None otherwise"""
     if not os.path.exists(PROFILE_TRAFFIC):
         return None
     with open(PROFILE_TRAFFIC) as f:
         d = json.load(f)
-    with open(KERNEL_SRC, "rb") as f:
-        h = hashlib.sha256(f.read()).hexdigest()[:16]
-    if d.get("kernel_sha256_16") != h or d.get("workload") != workload:
+    rec = d.get(kernel, {})
+    if rec.get("sources_sha256_16") != kernel_source_hash(kernel):
         return None
-    return d.get("dram_bytes_per_launch")
+    w = rec.get("workloads", {}).get(key)
+    return None if w is None else w.get("dram_bytes_per_launch")
+
+
+def traffic_key(a):
+    """the record's key for a workload: its name, plus the rate and shape when they differ from the
+    workload's own"""
+    wl = WORKLOADS[a.workload]
+    key = a.workload
+    if a.target != wl["target"]:
+        key += f"@{a.target:g}"
+    if getattr(a, "shape", None):
+        key += f"[{a.shape}]"
+    return key
 
 
 # ------------------------------------------------------------------ the reference arm
@@ -458,7 +481,7 @@ def run_ours(a, rank, world, local_rank):
     value = job_rate(out_bytes, world, step_s) / 1e9
     peak, peak_kind = measured_peaks()
     achieved = (in_bytes + out_bytes) / kernel_s / 1e9
-    traffic = traffic_for_kernel(a.workload)
+    traffic = traffic_for_kernel("decode_kernel", traffic_key(a))
 
     # the tables' preparation by itself (once per device copy of a stream)
     prep_reps = max(1, 200 // len(infos))
@@ -665,7 +688,8 @@ def run_ours_tile_ans(a, rank, world, local_rank):
                    "n_tiles": info.n_tiles, "blocks_per_lane": info.blocks_per_lane, "lossless": True},
         "gelements_per_s": round(job_rate(n, world, step_s) / 1e9, 3),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                     "frac": round(achieved / peak, 4), "traffic": traffic_for_kernel("ans_decode_kernel", traffic_key(a)),
+                     "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": in_bytes + out_bytes, "kernel_us": round(kernel_s * 1e6, 3),
                      "kernel_us_median": round(statistics.median(per_launch_us), 3) if per_launch_us else None,
                      "kernel_us_min": round(per_launch_us[0], 3) if per_launch_us else None},

@@ -79,30 +79,48 @@ __device__ __forceinline__ void store_element(const Params &p, uint64_t i, uint3
     o[ESZ - 1] = uint8_t(s);
 }
 
+// the raw bytes of whole chunk c (8 for 16-bit types, 24 for FP32; none for 8-bit types), loaded
+// before the chunk's symbols are decoded so that the load's latency hides behind the rANS chain
+template <int ESZ>
+struct RawChunk {
+    uint2 r[ESZ == 1 ? 1 : ESZ - 1];
+};
+
+template <int ESZ>
+__device__ __forceinline__ RawChunk<ESZ> load_raw(const Params &p, uint64_t c, bool whole) {
+    RawChunk<ESZ> R{};
+    if constexpr (ESZ > 1) {
+        const uint2 *rp = reinterpret_cast<const uint2 *>(p.raw + (ESZ - 1) * 8 * c);
+#pragma unroll
+        for (int q = 0; q < ESZ - 1; ++q) R.r[q] = whole ? __ldg(rp + q) : make_uint2(0u, 0u);
+    }
+    return R;
+}
+
 // chunk c: merge and store (whole chunks as vectors; the tensor's last, partial chunk element by
 // element)
 template <int ESZ>
-__device__ __forceinline__ void store_chunk(const Params &p, uint64_t c, const uint32_t (&e)[8]) {
+__device__ __forceinline__ void store_chunk(const Params &p, uint64_t c, const uint32_t (&e)[8], const RawChunk<ESZ> &R) {
     uint32_t lo, hi;
     pack_symbols(e, lo, hi);
     if (8 * c + 8 > p.n) {
         const uint32_t k = uint32_t(p.n - 8 * c);
-        for (uint32_t j = 0; j < k; ++j) store_element<ESZ>(p, 8 * c + j, (e[j] >> 12) & 0xffu);
+#pragma unroll
+        for (uint32_t j = 0; j < 8; ++j)  // constant indices keep e[] in registers
+            if (j < k) store_element<ESZ>(p, 8 * c + j, (e[j] >> 12) & 0xffu);
         return;
     }
     if constexpr (ESZ == 1) {
         reinterpret_cast<uint2 *>(p.out)[c] = make_uint2(lo, hi);
     } else if constexpr (ESZ == 2) {
         // bytes r0..r7 of the raw plane, then [r0 s0 r1 s1] [r2 s2 r3 s3] ...
-        const uint2 r = __ldg(reinterpret_cast<const uint2 *>(p.raw) + c);
+        const uint2 r = R.r[0];
         reinterpret_cast<uint4 *>(p.out)[c] =
             make_uint4(__byte_perm(r.x, lo, 0x5140), __byte_perm(r.x, lo, 0x7362), __byte_perm(r.y, hi, 0x5140),
                        __byte_perm(r.y, hi, 0x7362));
     } else {
         // 24 raw bytes: element j's low three bytes start at byte 3j
-        const uint2 *rp = reinterpret_cast<const uint2 *>(p.raw + 24 * c);
-        const uint2 r0 = __ldg(rp), r1 = __ldg(rp + 1), r2 = __ldg(rp + 2);
-        const uint32_t W[7] = {r0.x, r0.y, r1.x, r1.y, r2.x, r2.y, 0u};
+        const uint32_t W[7] = {R.r[0].x, R.r[0].y, R.r[1].x, R.r[1].y, R.r[2].x, R.r[2].y, 0u};
         uint32_t o[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -147,10 +165,11 @@ __device__ __forceinline__ uint32_t decode_tile(const Params &p, uint32_t lut, u
             break;
         }
         if (act) {
+            const RawChunk<ESZ> R = load_raw<ESZ>(p, c, 8 * c + 8 <= p.n);
             uint32_t e[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) e[j] = ans_step(x, wp, w, lut);
-            store_chunk<ESZ>(p, c, e);
+            store_chunk<ESZ>(p, c, e, R);
         }
     }
     if (err) return err;
