@@ -305,7 +305,7 @@ def kernel_source_hash(kernel):
 def traffic_for_kernel(kernel, key):
     """DRAM bytes per launch (read + write) from the committed ncu record for this workload key,
     if it was captured on the kernel's current sources; None otherwise"""
-    if not os.path.exists(PROFILE_TRAFFIC):
+    if not os.path.exists(PROFILE_TRAFFIC) or kernel not in KERNEL_SRCS:
         return None
     with open(PROFILE_TRAFFIC) as f:
         d = json.load(f)

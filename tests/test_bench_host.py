@@ -46,3 +46,15 @@ def test_l2_policy():
     # the DiT set lists 112 tensors of the four block shapes
     dims = bench.WORKLOADS["dit_28blocks_hidden3072_bf16"]["dims"]
     assert len(dims) == 112 and sum(r * c for r, c in dims) == 28 * 3072 * (9216 + 3072 + 12288 + 12288)
+
+
+def test_traffic_record_keys():
+    """the committed traffic record is looked up by kernel sources and by workload, rate and shape"""
+    import argparse
+    a = argparse.Namespace(workload="outliers_8192x28672_bf16", target=3.5, shape="8192x8192")
+    assert bench.traffic_key(a) == "outliers_8192x28672_bf16@3.5[8192x8192]"
+    a = argparse.Namespace(workload="lognormal_rows_4096x4096_bf16", target=4.0, shape=None)
+    assert bench.traffic_key(a) == "lognormal_rows_4096x4096_bf16"
+    assert len(bench.kernel_source_hash("decode_kernel")) == 16
+    # a record taken on other sources is not reported
+    assert bench.traffic_for_kernel("no_such_kernel", "lognormal_rows_4096x4096_bf16") is None
