@@ -987,6 +987,24 @@ static void bytes_put(bytes *b, const void *src, size_t n)
     b->n += n;
 }
 
+/* Which block (row-major index row * cb + column block) lane l of tile t takes as its k-th.
+ * Layout 0 (reading R15): tile t holds the 32K consecutive blocks from t * 32K, lane l the blocks
+ * t*32K + 32k + l.  Layout 1 (reading R32, the block order of a consumer GEMM: one tile is one
+ * operand tile of 128 output rows by 64 input columns; K = 32, rows a multiple of 128, columns a
+ * multiple of 64): with KT = cb / 8 tiles across a row band, tile t covers rows
+ * 128 (t / KT) .. +127 and column blocks 8 (t mod KT) .. +7, and lane l takes row 32 (k mod 4) + l
+ * of the tile at column block k / 4, so that one step of the 32 lanes fills 32 consecutive rows of
+ * one 8-column slice. */
+static int64_t lane_block(int32_t layout, int64_t cb, int64_t t, int l, uint32_t K, uint32_t k)
+{
+    if (layout == 0)
+        return t * (int64_t)LANES * K + (int64_t)k * LANES + l;
+    int64_t kt = cb / 8;
+    int64_t row = 128 * (t / kt) + 32 * (int64_t)(k % 4) + l;
+    int64_t colb = 8 * (t % kt) + (int64_t)(k / 4);
+    return row * cb + colb;
+}
+
 /* Decode order inside a tile (the rule both sides follow): the 32 lanes are independent
  * rANS coders, each with its own region of 16-bit words.  Lane l decodes its blocks
  * t*32K + 32k + l in order of k, and per block its rANS symbols in the order block_events
@@ -997,10 +1015,9 @@ static void bytes_put(bytes *b, const void *src, size_t n)
  * The encoder runs a lane's symbols in reverse, emitting words in reverse.  A tile stores the
  * 32 final encoder states (= initial decoder states, u32), the 32 region lengths in words
  * (u16), then the regions of lanes 0..31 one after another, zero padded to 16 bytes. */
-static int encode_tile(const uint32_t *ctx, const uint32_t *s, int64_t nb, int64_t t, uint32_t K,
-                       const coder *C, bytes *out)
+static int encode_tile(const uint32_t *ctx, const uint32_t *s, int64_t nb, int64_t cb, int32_t layout, int64_t t,
+                       uint32_t K, const coder *C, bytes *out)
 {
-    int64_t base = t * (int64_t)LANES * K;
     event *ev = (event *)malloc((size_t)K * 8 * sizeof(event));
     uint8_t *raw = (uint8_t *)malloc((size_t)K * (8 * VALUE_BITS + 48) + 16);
     uint16_t *words[LANES];
@@ -1010,7 +1027,7 @@ static int encode_tile(const uint32_t *ctx, const uint32_t *s, int64_t nb, int64
     for (int l = 0; l < LANES; l++) {
         size_t ne = 0, nraw = 0;
         for (uint32_t k = 0; k < K; k++) {
-            int64_t b = base + (int64_t)k * LANES + l;
+            int64_t b = lane_block(layout, cb, t, l, K, k);
             if (b >= nb)
                 break;
             block_events(C, ctx + 8 * b, s + 8 * b, ev, &ne, raw, &nraw);
@@ -1068,7 +1085,7 @@ static int encode_tile(const uint32_t *ctx, const uint32_t *s, int64_t nb, int64
 
 /* ---------------------------------- full encode at one k ----------------------------- */
 static int encode_at(const double *w, const float *s, const float *scales, int64_t rows, int64_t cols,
-                     int32_t sdt, int32_t container, int32_t k, uint32_t K, int32_t coding, uint8_t *out,
+                     int32_t sdt, int32_t container, int32_t k, uint32_t K, int32_t coding, int32_t layout, uint8_t *out,
                      size_t cap, size_t *out_n)
 {
     /* w: padded rows of 8 * ceil(cols / 8) values; the header keeps the true cols */
@@ -1158,7 +1175,7 @@ static int encode_at(const double *w, const float *s, const float *scales, int64
     int trc = OR_OK;
     for (uint32_t t = 0; t < T; t++) {
         dir[t] = (uint32_t)(tiles.n / 16);
-        if (encode_tile(ctx, u, nb, t, K, &C, &tiles) != OR_OK)
+        if (encode_tile(ctx, u, nb, cb, layout, t, K, &C, &tiles) != OR_OK)
             trc = OR_ERR_UNSUPPORTED;
     }
     dir[T] = (uint32_t)(tiles.n / 16);
@@ -1189,6 +1206,7 @@ static int encode_at(const double *w, const float *s, const float *scales, int64
         out[34] = PROB_BITS;
         out[35] = NCTX;
         out[43] = (uint8_t)C.paired;
+        out[58] = (uint8_t)layout;
         for (int c = 0; c < NCTX; c++) {
             out[36 + c] = (uint8_t)m[c];
             put16(out + 44 + 2 * c, ntok[c]);
@@ -1230,8 +1248,23 @@ static int encode_at(const double *w, const float *s, const float *scales, int64
 int or_compress(const void *src, int32_t sdt, int64_t rows, int64_t cols, double target, int32_t container,
                 uint32_t K, int32_t q_override, int32_t coding, uint8_t *out, size_t cap, size_t *out_n)
 {
+    return or_compress_layout(src, sdt, rows, cols, target, container, K, q_override, coding, 0, out, cap, out_n);
+}
+
+int or_compress_layout(const void *src, int32_t sdt, int64_t rows, int64_t cols, double target, int32_t container,
+                       uint32_t K, int32_t q_override, int32_t coding, int32_t layout, uint8_t *out, size_t cap,
+                       size_t *out_n)
+{
     if (!src || !out_n || rows <= 0 || cols <= 0)
         return OR_ERR_INVALID_ARG;
+    /* layout 1 (R32): GEMM operand tiles of 128 rows x 64 columns, 32 blocks per lane */
+    if (layout < 0 || layout > 1)
+        return OR_ERR_INVALID_ARG;
+    if (layout == 1) {
+        if (rows % 128 != 0 || cols % 64 != 0 || (K != 0 && K != 32))
+            return OR_ERR_INVALID_ARG;
+        K = 32;
+    }
     if (sdt != ORD_BF16 && sdt != ORD_FP16 && sdt != ORD_FP32)
         return OR_ERR_UNSUPPORTED;
     if (container == 0)
@@ -1272,11 +1305,11 @@ int or_compress(const void *src, int32_t sdt, int64_t rows, int64_t cols, double
     int rc;
     for (;;) {
         size_t n = 0;
-        rc = encode_at(wp, s, scales, rows, cols, sdt, container, k, K, coding, NULL, 0, &n);
+        rc = encode_at(wp, s, scales, rows, cols, sdt, container, k, K, coding, layout, NULL, 0, &n);
         if (rc == OR_ERR_UNSUPPORTED)
             break;
         if (q_override >= 0 || 8.0 * (double)n <= target * (double)(rows * cols)) {
-            rc = encode_at(wp, s, scales, rows, cols, sdt, container, k, K, coding, out, cap, out_n);
+            rc = encode_at(wp, s, scales, rows, cols, sdt, container, k, K, coding, layout, out, cap, out_n);
             break;
         }
         if (k == 0) {
@@ -1322,6 +1355,12 @@ int or_parse(const uint8_t *p, size_t n, or_info *info)
     if (p[43] > 1)
         return OR_ERR_CORRUPT;
     info->paired = p[43];
+    /* byte 58: the block order of the tiles (0 row-major lanes, 1 GEMM operand tiles) */
+    if (p[58] > 1)
+        return OR_ERR_CORRUPT;
+    info->layout = p[58];
+    if (info->layout == 1 && (info->rows % 128 != 0 || info->cols % 64 != 0 || info->blocks_per_lane != 32))
+        return OR_ERR_CORRUPT;
     uint64_t total_tokens = 0;
     for (int c = 0; c < NCTX; c++) {
         info->split[c] = p[36 + c];
@@ -1499,7 +1538,6 @@ static void decode_tile(dec_ctx *D, int64_t t, int32_t *vout, void *out, uint32_
     const uint8_t *tp = D->p + I->off_tiles + 16 * (uint64_t)get32(dir + 4 * t);
     uint64_t tile_bytes = 16 * (uint64_t)(get32(dir + 4 * (t + 1)) - get32(dir + 4 * t));
     uint64_t capacity = (tile_bytes - TILE_HEAD) / 2, start = 0;
-    int64_t base = t * (int64_t)LANES * K;
     int esz = elt_size(D->out_dtype);
     for (int l = 0; l < LANES; l++) {
         uint32_t x = get32(tp + 4 * l);
@@ -1513,7 +1551,7 @@ static void decode_tile(dec_ctx *D, int64_t t, int32_t *vout, void *out, uint32_
         start += len;
         raw_reader R = {wp, len, avail, 0};
         for (uint32_t k = 0; k < K; k++) {
-            int64_t b = base + (int64_t)k * LANES + l;
+            int64_t b = lane_block(I->layout, cb, t, l, K, k);
             if (b >= nb)
                 break;
             uint32_t tok[8], ctx[8], sv[8];

@@ -69,6 +69,7 @@ typedef struct {
     uint16_t ntok[7];
     uint64_t off_rowf, off_scales, off_freq, off_dir, off_tiles;
     uint32_t paired; /* 1: coordinates 1..6 coded as three pairs */
+    uint32_t layout; /* block order of the tiles: 0 lanes along rows, 1 GEMM operand tiles (128 x 64) */
 } or_info;
 
 /* ---- scalar pieces, exposed so that tests can pin them one by one ---- */
@@ -124,6 +125,12 @@ double or_estimate_bpp(const void *src, int32_t src_dtype, int64_t rows, int64_t
 int or_compress(const void *src, int32_t src_dtype, int64_t rows, int64_t cols, double target_bpp,
                 int32_t container, uint32_t blocks_per_lane, int32_t q_override, int32_t coding,
                 uint8_t *out, size_t cap, size_t *out_nbytes);
+/* or_compress with the tiles' block order: layout 0 (lane l of tile t takes blocks t*32K + 32k + l)
+ * or layout 1 (each tile one 128-row x 64-column operand tile of a consumer GEMM; K = 32, rows a
+ * multiple of 128, columns a multiple of 64) */
+int or_compress_layout(const void *src, int32_t src_dtype, int64_t rows, int64_t cols, double target_bpp,
+                       int32_t container, uint32_t blocks_per_lane, int32_t q_override, int32_t coding,
+                       int32_t layout, uint8_t *out, size_t cap, size_t *out_nbytes);
 int or_parse(const uint8_t *blob, size_t nbytes, or_info *info);
 /* decodes tiles [t0, t1): lattice points into v (indexed by weight, rows*cols, nullable) and
  * container bytes into out (rows*cols elements, nullable); returns OR_OK or a negative error,

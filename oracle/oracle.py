@@ -27,7 +27,7 @@ class Info(C.Structure):
         ("n_tiles", C.c_uint32), ("blocks_per_lane", C.c_uint32),
         ("split", C.c_uint8 * 7), ("ntok", C.c_uint16 * 7),
         ("off_rowf", C.c_uint64), ("off_scales", C.c_uint64), ("off_freq", C.c_uint64),
-        ("off_dir", C.c_uint64), ("off_tiles", C.c_uint64), ("paired", C.c_uint32),
+        ("off_dir", C.c_uint64), ("off_tiles", C.c_uint64), ("paired", C.c_uint32), ("layout", C.c_uint32),
     ]
 
 
@@ -95,6 +95,8 @@ def lib():
         L.or_code_stats.restype = C.c_int
         L.or_code_stats.argtypes = [p, C.c_size_t, C.POINTER(C.c_double), C.POINTER(C.c_double),
                                     C.POINTER(C.c_double), C.POINTER(C.c_uint64), C.POINTER(C.c_uint64)]
+        L.or_compress_layout.argtypes = [p, C.c_int32, C.c_int64, C.c_int64, C.c_double, C.c_int32, C.c_uint32,
+                                         C.c_int32, C.c_int32, C.c_int32, p, C.c_size_t, C.POINTER(C.c_size_t)]
         L.ota_blocks_per_lane.restype = C.c_uint32
         L.ota_blocks_per_lane.argtypes = [C.c_int64]
         L.ota_compress.argtypes = [p, C.c_int32, C.c_int64, C.c_int32, p, C.c_uint32, p, C.c_size_t,
@@ -272,19 +274,20 @@ def estimate_bpp(src, k, container=0, blocks_per_lane=0, coding=CODING_AUTO):
 
 
 # ---- the stream ----
-def compress(src, target_bpp, container=0, blocks_per_lane=0, q_override=-1, coding=CODING_AUTO):
+def compress(src, target_bpp, container=0, blocks_per_lane=0, q_override=-1, coding=CODING_AUTO, layout=0):
     """Returns (rc, blob as a uint8 numpy array).  ``coding``: CODING_AUTO, CODING_SINGLE or
-    CODING_PAIRED (coordinates 1..6 paired whenever the alphabets allow, at any size)."""
+    CODING_PAIRED (coordinates 1..6 paired whenever the alphabets allow, at any size).  ``layout``:
+    0 (lanes along rows) or 1 (tiles of 128 rows x 64 columns, the block order of a consumer GEMM)."""
     a, dt = _src(src)
     R, Cc = a.shape
     n = C.c_size_t(0)
-    rc = lib().or_compress(_ptr(a), dt, R, Cc, float(target_bpp), container, blocks_per_lane, q_override,
-                           int(coding), None, 0, C.byref(n))
+    rc = lib().or_compress_layout(_ptr(a), dt, R, Cc, float(target_bpp), container, blocks_per_lane, q_override,
+                                  int(coding), int(layout), None, 0, C.byref(n))
     if rc not in (OK, ERR_BUFFER_TOO_SMALL):
         return rc, None
     out = np.zeros(n.value, np.uint8)
-    rc = lib().or_compress(_ptr(a), dt, R, Cc, float(target_bpp), container, blocks_per_lane, q_override,
-                           int(coding), _ptr(out), out.size, C.byref(n))
+    rc = lib().or_compress_layout(_ptr(a), dt, R, Cc, float(target_bpp), container, blocks_per_lane, q_override,
+                                  int(coding), int(layout), _ptr(out), out.size, C.byref(n))
     return rc, (out[: n.value] if rc == OK else None)
 
 
