@@ -30,7 +30,7 @@ class EpError(RuntimeError):
 
 class Config(C.Structure):
     _fields_ = [("target_bpp", C.c_double), ("container_dtype", C.c_int32), ("blocks_per_lane", C.c_uint32),
-                ("q_index", C.c_int32), ("n_threads", C.c_int32), ("coding", C.c_int32)]
+                ("q_index", C.c_int32), ("n_threads", C.c_int32), ("coding", C.c_int32), ("layout", C.c_int32)]
 
 
 class StreamInfo(C.Structure):
@@ -44,6 +44,7 @@ class StreamInfo(C.Structure):
         ("off_rowf", C.c_uint64), ("off_scales", C.c_uint64), ("off_freq", C.c_uint64),
         ("off_dir", C.c_uint64), ("off_tiles", C.c_uint64), ("out_nbytes", C.c_uint64),
         ("max_tile_nbytes", C.c_uint64), ("workspace_nbytes", C.c_uint64), ("paired", C.c_uint32),
+        ("layout", C.c_uint32),
     ]
 
     @property
@@ -138,29 +139,33 @@ def lib():
 
 
 CODING_AUTO, CODING_SINGLE, CODING_PAIRED = 0, 1, 2
+LAYOUT_ROWS, LAYOUT_GEMM = 0, 1
 
 
-def _config(target_bpp, container=0, blocks_per_lane=0, q_index=-1, n_threads=0, coding=CODING_AUTO):
+def _config(target_bpp, container=0, blocks_per_lane=0, q_index=-1, n_threads=0, coding=CODING_AUTO,
+            layout=LAYOUT_ROWS):
     if isinstance(container, str):
         container = NAMES[container]
     if isinstance(container, torch.dtype):
         container = CODE_OF[container]
     return Config(float(target_bpp), int(container or 0), int(blocks_per_lane), int(q_index), int(n_threads),
-                  int(coding))
+                  int(coding), int(layout))
 
 
-def compress(tensor, target_bpp, container=0, blocks_per_lane=0, q_index=-1, n_threads=0, coding=CODING_AUTO):
+def compress(tensor, target_bpp, container=0, blocks_per_lane=0, q_index=-1, n_threads=0, coding=CODING_AUTO,
+             layout=LAYOUT_ROWS):
     """compress(tensor, config) on the host: returns the stream as a CPU uint8 tensor.
 
     ``tensor``: 2-D BF16/FP16/FP32 (moved to the CPU if needed).  ``container``: 0 (same as
     the source), a dtype code / name / torch dtype; INT8 and FP8 store per-row absmax codes.
-    ``coding``: CODING_AUTO, CODING_SINGLE or CODING_PAIRED (ep_config.coding)."""
+    ``coding``: CODING_AUTO, CODING_SINGLE or CODING_PAIRED (ep_config.coding).  ``layout``:
+    LAYOUT_ROWS, or LAYOUT_GEMM for tiles that are a consumer GEMM's 128 x 64 operand tiles."""
     if tensor.dim() != 2 or tensor.numel() == 0:
         raise EpError(-1, "compress needs a non-empty 2-D tensor")
     src = tensor.detach().to("cpu").contiguous()
     if src.dtype not in (torch.bfloat16, torch.float16, torch.float32):
         raise EpError(-8, f"source dtype {src.dtype}")
-    cfg = _config(target_bpp, container, blocks_per_lane, q_index, n_threads, coding)
+    cfg = _config(target_bpp, container, blocks_per_lane, q_index, n_threads, coding, layout)
     L = lib()
     cap = L.ep_compress_bound(src.shape[0], src.shape[1], C.byref(cfg))
     out = torch.empty(max(cap, 64), dtype=torch.uint8)
@@ -177,7 +182,7 @@ def compress(tensor, target_bpp, container=0, blocks_per_lane=0, q_index=-1, n_t
 
 
 def compress_device(tensor, target_bpp, container=0, blocks_per_lane=0, q_index=-1, stream=None,
-                    coding=CODING_AUTO):
+                    coding=CODING_AUTO, layout=LAYOUT_ROWS):
     """compress(tensor, config) for a CUDA tensor (ep_compress_device): the same stream as
     ``compress`` byte for byte, built on the GPU.  Returns a CUDA uint8 tensor."""
     if tensor.dim() != 2 or tensor.numel() == 0:
@@ -187,7 +192,7 @@ def compress_device(tensor, target_bpp, container=0, blocks_per_lane=0, q_index=
     src = tensor.detach().contiguous()
     if src.dtype not in (torch.bfloat16, torch.float16, torch.float32):
         raise EpError(-8, f"source dtype {src.dtype}")
-    cfg = _config(target_bpp, container, blocks_per_lane, q_index, 0, coding)
+    cfg = _config(target_bpp, container, blocks_per_lane, q_index, 0, coding, layout)
     L = lib()
     R, Cc = src.shape
     scratch = torch.empty(max(1, L.ep_compress_device_scratch(R, Cc, C.byref(cfg))), dtype=torch.uint8,

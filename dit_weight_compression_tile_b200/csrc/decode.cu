@@ -93,8 +93,10 @@ struct Params {
 // How a stream's blocks map onto rows, fixed per launch: kRowsAny (a lane's row is tested after
 // every block), kRows32 (32 divides the blocks per row: a warp's step never straddles rows, so the
 // loop runs row segment by row segment) and kRowsPadded (cols % 8 != 0: rows are zero-padded to
-// whole E8 blocks and stores go element by element).
-enum RowLayout { kRowsAny = 0, kRows32 = 1, kRowsPadded = 2 };
+// whole E8 blocks and stores go element by element); kRowsGemm: the tiles are 128 x 64 operand
+// tiles of a consumer GEMM (format.h lane_block), lane l taking row 32 (k mod 4) + l of its tile
+// at column block k / 4, so each lane works on four rows whose factors it loads once per tile.
+enum RowLayout { kRowsAny = 0, kRows32 = 1, kRowsPadded = 2, kRowsGemm = 3 };
 
 __device__ __forceinline__ uint32_t split_of_bits(uint32_t splits, uint32_t c) { return (splits >> (4 * c)) & 15u; }
 __device__ __forceinline__ uint32_t split_of(const Params &p, uint32_t c) { return split_of_bits(p.splits, c); }
@@ -416,12 +418,26 @@ template <int DT, bool SMEM, bool ACT, int ROWS, int MODE, typename Lim>
 __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L, uint32_t &rb, uint32_t lut,
                                                   Lim wlim, uint32_t t, uint32_t lane) {
     constexpr bool WIDE = MODE == kWide;
+    constexpr bool R32 = ROWS == kRows32, RAG = ROWS == kRowsPadded, GEMM = ROWS == kRowsGemm;
     uint32_t b = t * 32u * p.K + lane;
     uint32_t row = b / p.cb, col = b - row * p.cb;
     // the factor of the current row and of the next one (read a row ahead)
-    float fr = row < p.rows ? __ldg(p.rowf + row) : 0.0f;
-    float frn = row + 1 < p.rows ? __ldg(p.rowf + row + 1) : 0.0f;
-    constexpr bool R32 = ROWS == kRows32, RAG = ROWS == kRowsPadded;
+    float fr = 0.0f, frn = 0.0f;
+    // GEMM tiles: the lane's four rows r0 + 32 j and their factors; block k sits at
+    // (r0 + 32 (k mod 4)) cb + c0 + k / 4
+    float fg0 = 0.0f, fg1 = 0.0f, fg2 = 0.0f, fg3 = 0.0f;
+    uint32_t gbase = 0;
+    if constexpr (GEMM) {
+        const uint32_t kt = p.cb >> 3, r0 = 128u * (t / kt) + lane;
+        gbase = r0 * p.cb + 8u * (t % kt);
+        fg0 = __ldg(p.rowf + r0);
+        fg1 = __ldg(p.rowf + r0 + 32);
+        fg2 = __ldg(p.rowf + r0 + 64);
+        fg3 = __ldg(p.rowf + r0 + 96);
+    } else {
+        fr = row < p.rows ? __ldg(p.rowf + row) : 0.0f;
+        frn = row + 1 < p.rows ? __ldg(p.rowf + row + 1) : 0.0f;
+    }
     uint32_t err = 0;
     uint32_t k = 0;
     for (;;) {
@@ -433,6 +449,10 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
             kseg = k + left < p.K ? k + left : p.K;
         }
         for (; k < kseg; ++k, b += 32u) {
+            if constexpr (GEMM) {
+                b = gbase + (k & 3u) * 32u * p.cb + (k >> 2);
+                fr = (k & 2u) ? ((k & 1u) ? fg3 : fg2) : ((k & 1u) ? fg1 : fg0);
+            }
             bool act = !ACT || b < p.nb;
             if (ACT && !__any_sync(0xffffffffu, act)) goto done;
             // a damaged stream may drive a lane's reads ahead (at most one word per token); stop
@@ -527,7 +547,7 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
             } else if (act) {
                 pk.store(p.out, b);
             }
-            if constexpr (!R32) {
+            if constexpr (!R32 && !GEMM) {
                 col += 32u;
                 if (col >= p.cb) {  // next row
                     col -= p.cb;
@@ -850,7 +870,7 @@ struct DeviceCache {
 DeviceCache g_cache;
 
 template <int DT>
-cudaError_t launch(Params &p, uint64_t max_tile, int mode, int device, cudaStream_t stream) {
+cudaError_t launch(Params &p, uint64_t max_tile, int mode, bool gemm, int device, cudaStream_t stream) {
     int sms;
     {
         std::lock_guard<std::mutex> g(g_cache.mu);
@@ -862,10 +882,11 @@ cudaError_t launch(Params &p, uint64_t max_tile, int mode, int device, cudaStrea
         if (!g_cache.attr[device][DT]) {
             cudaError_t e = cudaSuccess;
             for (auto k : {decode_kernel<DT, kRowsAny, kNarrow>, decode_kernel<DT, kRows32, kNarrow>,
-                           decode_kernel<DT, kRowsPadded, kNarrow>, decode_kernel<DT, kRowsAny, kWide>,
-                           decode_kernel<DT, kRows32, kWide>, decode_kernel<DT, kRowsPadded, kWide>,
+                           decode_kernel<DT, kRowsPadded, kNarrow>, decode_kernel<DT, kRowsGemm, kNarrow>,
+                           decode_kernel<DT, kRowsAny, kWide>, decode_kernel<DT, kRows32, kWide>,
+                           decode_kernel<DT, kRowsPadded, kWide>, decode_kernel<DT, kRowsGemm, kWide>,
                            decode_kernel<DT, kRowsAny, kPaired>, decode_kernel<DT, kRows32, kPaired>,
-                           decode_kernel<DT, kRowsPadded, kPaired>})
+                           decode_kernel<DT, kRowsPadded, kPaired>, decode_kernel<DT, kRowsGemm, kPaired>})
                 if (e == cudaSuccess)
                     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemLimit));
             if (e != cudaSuccess) return e;
@@ -908,6 +929,11 @@ cudaError_t launch(Params &p, uint64_t max_tile, int mode, int device, cudaStrea
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (gemm) {
+        if (mode == kPaired) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsGemm, kPaired>, p);
+        if (mode == kWide) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsGemm, kWide>, p);
+        return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsGemm, kNarrow>, p);
+    }
     if (mode == kPaired) {
         if (p.cols & 7u) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRowsPadded, kPaired>, p);
         if ((p.cb & 31u) == 0) return cudaLaunchKernelEx(&cfg, decode_kernel<DT, kRows32, kPaired>, p);
@@ -929,6 +955,8 @@ int check_info(const ep_info *info) {
     if (info->rows >= (int64_t(1) << 31) || cb >= (int64_t(1) << 31) || info->rows * cb >= (int64_t(1) << 31))
         return EP_ERR_UNSUPPORTED;
     if (info->paired > 1) return EP_ERR_CORRUPT;
+    if (info->layout > 1 || !layout_fits(int(info->layout), info->rows, info->cols, info->blocks_per_lane))
+        return EP_ERR_CORRUPT;
     uint32_t total = 0;
     for (int c = 0; c < kContexts; ++c) {
         if (!split_valid(info->split[c], c) || info->ntok[c] > split_alphabet(info->split[c], kCtxLow[c]))
@@ -1034,12 +1062,12 @@ extern "C" int ep_decompress(const ep_info *info, const void *d_blob, const void
     uint64_t mt = info->max_tile_nbytes;
     const int mode = coding_of(info);
     switch (out_dtype) {
-    case EP_BF16: e = launch<EP_BF16>(p, mt, mode, device, s); break;
-    case EP_FP16: e = launch<EP_FP16>(p, mt, mode, device, s); break;
-    case EP_FP32: e = launch<EP_FP32>(p, mt, mode, device, s); break;
-    case EP_INT8: e = launch<EP_INT8>(p, mt, mode, device, s); break;
-    case EP_FP8_E4M3: e = launch<EP_FP8_E4M3>(p, mt, mode, device, s); break;
-    case EP_LATTICE_I32: e = launch<EP_LATTICE_I32>(p, mt, mode, device, s); break;
+    case EP_BF16: e = launch<EP_BF16>(p, mt, mode, info->layout == 1, device, s); break;
+    case EP_FP16: e = launch<EP_FP16>(p, mt, mode, info->layout == 1, device, s); break;
+    case EP_FP32: e = launch<EP_FP32>(p, mt, mode, info->layout == 1, device, s); break;
+    case EP_INT8: e = launch<EP_INT8>(p, mt, mode, info->layout == 1, device, s); break;
+    case EP_FP8_E4M3: e = launch<EP_FP8_E4M3>(p, mt, mode, info->layout == 1, device, s); break;
+    case EP_LATTICE_I32: e = launch<EP_LATTICE_I32>(p, mt, mode, info->layout == 1, device, s); break;
     default: return EP_ERR_INVALID_ARG;
     }
     return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;

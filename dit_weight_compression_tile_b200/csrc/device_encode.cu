@@ -229,6 +229,8 @@ struct LaneArgs {
     uint8_t *tiles;         // tile section of the output (WRITE)
     int64_t nb;
     uint32_t K, T;
+    int64_t cb;             // blocks per row
+    int layout;             // block order of the tiles (format.h lane_block)
     Splits sp;
     uint32_t paired;
     uint32_t B[kContexts];     // paired contexts 1, 2: pair base min(A, 40)
@@ -284,10 +286,10 @@ __global__ void lane_kernel(LaneArgs a) {
     const uint32_t lane = threadIdx.x & 31u;
     const uint64_t t = (uint64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     if (t >= a.T) return;  // whole warps leave together
-    const int64_t first = int64_t(t) * 32 * a.K;
-    // blocks of this lane
+    // blocks of this lane, in the layout's order
+    auto blk = [&](uint32_t k) { return lane_block(a.layout, a.cb, int64_t(t), int(lane), a.K, k); };
     uint32_t nk = 0;
-    while (nk < a.K && first + int64_t(nk) * 32 + lane < a.nb) ++nk;
+    while (nk < a.K && blk(nk) < a.nb) ++nk;
 
     uint32_t n = 0, nr = 0, start = 0;
     uint16_t *area = nullptr;
@@ -322,7 +324,7 @@ __global__ void lane_kernel(LaneArgs a) {
     };
     auto skip = [](uint32_t, uint32_t) {};
     Sym sym[8];
-    for (uint32_t k = 0; k < nk; ++k) block_syms(a, sf, first + int64_t(k) * 32 + lane, sym, push);
+    for (uint32_t k = 0; k < nk; ++k) block_syms(a, sf, blk(k), sym, push);
     if (nacc) {
         if (WRITE) area[start + n - 1 - raw] = uint16_t(acc);
         ++raw;
@@ -330,7 +332,7 @@ __global__ void lane_kernel(LaneArgs a) {
     // rANS, symbols in reverse; the i-th word emitted is word nr - 1 - i in decode order
     uint32_t x = kStateLow, emitted = 0;
     for (uint32_t k = nk; k-- > 0;) {
-        const int ns = block_syms(a, sf, first + int64_t(k) * 32 + lane, sym, skip);
+        const int ns = block_syms(a, sf, blk(k), sym, skip);
         for (int i = ns - 1; i >= 0; --i) {
             const uint32_t at = sym[i].c * kTableStride + sym[i].s, nbits = sym[i].bits;
             const uint32_t f = sf[at], cu = sc[at];
@@ -403,7 +405,7 @@ Scratch carve(uint8_t *base, int64_t rows, int64_t cols, int container, int64_t 
 
 struct Plan {
     int64_t rows, cols, cb, nb;
-    int src_dt, container, coding;
+    int src_dt, container, coding, layout;
     uint32_t K, T;
     bool ok;
 };
@@ -417,9 +419,11 @@ Plan plan_of(int64_t rows, int64_t cols, int32_t src_dtype, const ep_config *cfg
     P.src_dt = src_dtype;
     P.container = cfg->container_dtype ? cfg->container_dtype : src_dtype;
     P.coding = cfg->coding;
-    P.K = cfg->blocks_per_lane ? cfg->blocks_per_lane : auto_blocks_per_lane(P.nb, cfg->target_bpp);
+    P.layout = cfg->layout;
+    P.K = cfg->blocks_per_lane ? cfg->blocks_per_lane
+                               : (P.layout == kLayoutGemm ? 32u : auto_blocks_per_lane(P.nb, cfg->target_bpp));
     P.T = P.K ? uint32_t((P.nb + 32 * int64_t(P.K) - 1) / (32 * int64_t(P.K))) : 0;
-    P.ok = P.K > 0;
+    P.ok = P.K > 0 && (P.layout == kLayoutRows || P.layout == kLayoutGemm) && layout_fits(P.layout, rows, cols, P.K);
     return P;
 }
 
@@ -520,6 +524,7 @@ extern "C" int ep_compress_device(const void *d_src, int32_t src_dtype, int64_t 
     if (reinterpret_cast<uintptr_t>(d_scratch) & 255u || reinterpret_cast<uintptr_t>(d_out) & 15u)
         return EP_ERR_INVALID_ARG;
     Plan P = plan_of(rows, cols, src_dtype, cfg);
+    // P.ok is false for an unknown layout and for a shape or tile size the GEMM block order cannot take
     if (!P.ok || scratch_nbytes < ep_compress_device_scratch(rows, cols, cfg)) return EP_ERR_INVALID_ARG;
     int device = 0, sms = 0;
     if (cudaGetDevice(&device) != cudaSuccess ||
@@ -614,7 +619,7 @@ extern "C" int ep_compress_device(const void *d_src, int32_t src_dtype, int64_t 
         R.h2d(R.S.cum, hc.data(), hc.size());
         R.check(cudaMemsetAsync(R.S.too_long, 0, 4, R.st));
         LaneArgs la{R.S.ctx, R.S.val, R.S.freq, R.S.cum, R.S.count, R.S.rwords, R.S.state, R.S.too_long,
-                    R.S.dir, nullptr, P.nb, P.K, P.T, sp, paired ? 1u : 0u, {}, {}};
+                    R.S.dir, nullptr, P.nb, P.K, P.T, P.cb, P.layout, sp, paired ? 1u : 0u, {}, {}};
         for (int c = 0; c < kContexts; ++c) {
             la.B[c] = pair_base(A[c]);
             la.rawb[c] = pair_raw_bits(A[c]);
@@ -654,7 +659,7 @@ extern "C" int ep_compress_device(const void *d_src, int32_t src_dtype, int64_t 
         uint32_t mm[kContexts];
         for (int c = 0; c < kContexts; ++c) mm[c] = sp.m[c];
         write_front(front.data(), L, src_dtype, container, rows, cols, P.T, P.K, k, mm, ntok, tablen, paired, freq,
-                    fac.data(), scales.data());
+                    fac.data(), scales.data(), P.layout);
         for (uint32_t t = 0; t <= P.T; ++t)
             for (int b = 0; b < 4; ++b) front[L.dir + 4 * t + b] = uint8_t(dir[t] >> (8 * b));
         uint8_t *out = static_cast<uint8_t *>(d_out);

@@ -45,7 +45,7 @@ double estimate_from_counts(const std::vector<uint64_t> *cnt, const uint32_t *m,
 // entries of freq[c] written (the pair tables' A * A + 1 for a paired stream's contexts 1, 2)
 void write_front(uint8_t *h, const Layout &L, int src_dt, int container, int64_t rows, int64_t cols, uint32_t T,
                  uint32_t K, int k, const uint32_t *m, const uint32_t *ntok, const uint32_t *tablen, bool paired,
-                 const std::vector<uint32_t> *freq, const float *fac, const float *scales);
+                 const std::vector<uint32_t> *freq, const float *fac, const float *scales, int layout);
 
 bool little_endian_host();
 

@@ -56,6 +56,36 @@ constexpr double kTargetMargin = 0.995;
 
 inline size_t align16(size_t n) { return (n + 15) & ~size_t(15); }
 
+#ifdef __CUDACC__
+#define EP_HD __host__ __device__
+#else
+#define EP_HD
+#endif
+
+// Block order of the tiles (header byte 58).  kLayoutRows: lane l of tile t codes blocks
+// t*32K + 32k + l.  kLayoutGemm: every tile is one operand tile of a consumer GEMM, 128 rows by 64
+// columns (K = 32, rows a multiple of 128, columns a multiple of 64); with KT = cb / 8 tiles
+// across a row band, tile t covers rows 128 (t / KT) .. +127 and column blocks 8 (t mod KT) .. +7,
+// and lane l codes row 32 (k mod 4) + l of it at column block k / 4, so one step of the 32 lanes
+// covers 32 consecutive rows of one 8-column slice.
+constexpr int kLayoutRows = 0;
+constexpr int kLayoutGemm = 1;
+constexpr int64_t kGemmTileRows = 128;
+constexpr int64_t kGemmTileCols = 64;
+
+// row-major index (row * cb + column block) of lane l's k-th block in tile t
+EP_HD inline int64_t lane_block(int layout, int64_t cb, int64_t t, int l, uint32_t K, uint32_t k) {
+    if (layout == kLayoutRows) return t * int64_t(kLanes) * K + int64_t(k) * kLanes + l;
+    const int64_t kt = cb / 8;
+    return (kGemmTileRows * (t / kt) + 32 * int64_t(k % 4) + l) * cb + 8 * (t % kt) + int64_t(k / 4);
+}
+
+// whether a shape and tile size can take a layout
+inline bool layout_fits(int layout, int64_t rows, int64_t cols, uint32_t K) {
+    if (layout == kLayoutRows) return true;
+    return layout == kLayoutGemm && rows % kGemmTileRows == 0 && cols % kGemmTileCols == 0 && K == 32;
+}
+
 // tokens a split can produce for values below 2^22
 inline uint32_t split_alphabet(uint32_t m, uint32_t low) { return (1u << m) + (((kValueBits - m) << kTopBits) << low); }
 

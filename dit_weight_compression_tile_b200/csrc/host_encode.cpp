@@ -220,7 +220,7 @@ double estimate_from_counts(const std::vector<uint64_t> *cnt, const uint32_t *m,
 
 void write_front(uint8_t *h, const Layout &L, int src_dt, int container, int64_t rows, int64_t cols, uint32_t T,
                  uint32_t K, int k, const uint32_t *m, const uint32_t *ntok, const uint32_t *tablen, bool paired,
-                 const std::vector<uint32_t> *freq, const float *fac, const float *scales) {
+                 const std::vector<uint32_t> *freq, const float *fac, const float *scales, int layout) {
     auto put = [](uint8_t *p, uint64_t v, int n) {
         for (int i = 0; i < n; ++i) p[i] = uint8_t(v >> (8 * i));
     };
@@ -236,6 +236,7 @@ void write_front(uint8_t *h, const Layout &L, int src_dt, int container, int64_t
     h[34] = uint8_t(kProbBits);
     h[35] = uint8_t(kContexts);
     h[43] = paired ? 1 : 0;
+    h[58] = uint8_t(layout);
     for (int c = 0; c < kContexts; ++c) {
         h[36 + c] = uint8_t(m[c]);
         put(h + 44 + 2 * c, ntok[c], 2);
@@ -263,6 +264,7 @@ struct Encoder {
     int container;
     int threads;
     int coding;  // EP_CODING_*
+    int layout;  // EP_LAYOUT_*: the block order of the tiles
     uint32_t K;
     std::vector<float> codes;   // INT8/FP8 code matrix (exact in fp32), empty otherwise
     std::vector<float> scales;  // INT8/FP8 per-row scales
@@ -377,10 +379,9 @@ struct Encoder {
         const std::vector<uint8_t> *rare;          // paired contexts 1, 2: escaped pair indices
     };
 
-    static bool encode_tile(const uint8_t *ctx, const uint32_t *val, int64_t nb, int64_t t, uint32_t K,
-                            const Model &M, std::vector<Event> &ev, std::vector<uint16_t> &words,
+    static bool encode_tile(const uint8_t *ctx, const uint32_t *val, int64_t nb, int64_t cb, int layout, int64_t t,
+                            uint32_t K, const Model &M, std::vector<Event> &ev, std::vector<uint16_t> &words,
                             std::vector<uint8_t> &out) {
-        int64_t first = t * int64_t(kLanes) * K;
         uint32_t state[kLanes];
         uint32_t count[kLanes];
         bool fits = true;
@@ -404,7 +405,7 @@ struct Encoder {
                 }
             };
             for (uint32_t k = 0; k < K; ++k) {
-                int64_t b = first + int64_t(k) * kLanes + l;
+                int64_t b = lane_block(layout, cb, t, l, K, k);
                 if (b >= nb) break;
                 const size_t s0 = size_t(8 * b);
                 Token tk[8];
@@ -562,7 +563,8 @@ struct Encoder {
             for (int64_t c = c0; c < c1; ++c)
                 for (int64_t t = c * tper; t < std::min<int64_t>(T, (c + 1) * tper); ++t) {
                     size_t before = part_tiles[size_t(c)].size();
-                    if (!encode_tile(ctx.data(), val.data(), nb, t, K, model, ev, words, part_tiles[size_t(c)]))
+                    if (!encode_tile(ctx.data(), val.data(), nb, cb, layout, t, K, model, ev, words,
+                                     part_tiles[size_t(c)]))
                         part_fits[size_t(c)] = 0;
                     part_sizes[size_t(c)].push_back(uint32_t((part_tiles[size_t(c)].size() - before) / 16));
                 }
@@ -578,7 +580,7 @@ struct Encoder {
             for (int i = 0; i < n; ++i) p[i] = uint8_t(v >> (8 * i));
         };
         write_front(h, L, src.dt, container, rows, cols, T, K, k, m, ntok, tablen, paired, freq, fac.data(),
-                    scales.data());
+                    scales.data(), layout);
         uint32_t at = 0;
         size_t d = L.dir, o = L.tiles;
         for (int c = 0; c < tchunks; ++c) {
@@ -603,7 +605,9 @@ extern "C" size_t ep_compress_bound(int64_t rows, int64_t cols, const ep_config 
     double n = double(rows) * double(cols);
     if (cfg->q_index < 0) return size_t(std::floor(cfg->target_bpp * n / 8.0));
     int64_t nb = rows * ((cols + 7) / 8);
-    uint32_t K = cfg->blocks_per_lane ? cfg->blocks_per_lane : ep::auto_blocks_per_lane(nb, cfg->target_bpp);
+    uint32_t K = cfg->blocks_per_lane ? cfg->blocks_per_lane
+                                      : (cfg->layout == ep::kLayoutGemm ? 32u
+                                                                         : ep::auto_blocks_per_lane(nb, cfg->target_bpp));
     uint64_t T = uint64_t((nb + 32 * int64_t(K) - 1) / (32 * int64_t(K)));
     return ep::layout_for(rows, ep::is_code_container(cfg->container_dtype) ? cfg->container_dtype : 0,
                           7 * ep::kPairMaxTable, T)
@@ -623,6 +627,10 @@ extern "C" int ep_compress_host(const void *src, int32_t src_dtype, int64_t rows
     if (cfg->blocks_per_lane > 4096) return EP_ERR_INVALID_ARG;
     if (cfg->coding < EP_CODING_AUTO || cfg->coding > EP_CODING_PAIRED) return EP_ERR_INVALID_ARG;
     if ((rows * ((cols + 7) / 8)) >> 32) return EP_ERR_UNSUPPORTED;
+    // the GEMM block order takes whole 128 x 64 operand tiles and 32 blocks per lane
+    if (cfg->layout != kLayoutRows && cfg->layout != kLayoutGemm) return EP_ERR_INVALID_ARG;
+    if (cfg->layout == kLayoutGemm && !layout_fits(kLayoutGemm, rows, cols, cfg->blocks_per_lane ? cfg->blocks_per_lane : 32u))
+        return EP_ERR_INVALID_ARG;
 
     Encoder E;
     E.src = Source{src, src_dtype};
@@ -630,6 +638,7 @@ extern "C" int ep_compress_host(const void *src, int32_t src_dtype, int64_t rows
     E.cols = cols;
     E.container = container;
     E.coding = cfg->coding;
+    E.layout = cfg->layout;
     E.threads = cfg->n_threads > 0 ? cfg->n_threads : int(std::max(1u, std::thread::hardware_concurrency()));
     // finite check
     {
@@ -651,7 +660,8 @@ extern "C" int ep_compress_host(const void *src, int32_t src_dtype, int64_t rows
     if (!(target >= 0.001) || !(target <= 11.0) || (is_code_container(container) && !(target < 8.0)))
         return EP_ERR_TARGET_RANGE;
     E.prepare();
-    E.K = cfg->blocks_per_lane ? cfg->blocks_per_lane : auto_blocks_per_lane(E.nb, target);
+    E.K = cfg->blocks_per_lane ? cfg->blocks_per_lane
+                               : (E.layout == kLayoutGemm ? 32u : auto_blocks_per_lane(E.nb, target));
     int kmax = max_q_index(cols);
     int k;
     if (cfg->q_index >= 0) {

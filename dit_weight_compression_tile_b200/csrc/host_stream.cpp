@@ -51,6 +51,10 @@ extern "C" int ep_stream_info(const void *blob, size_t nbytes, ep_info *info) {
     if ((nb + per_tile - 1) / per_tile != int64_t(I.n_tiles)) return EP_ERR_CORRUPT;
     if (p[43] > 1) return EP_ERR_CORRUPT;
     I.paired = p[43];
+    // byte 58: the block order of the tiles (EP_LAYOUT_ROWS or EP_LAYOUT_GEMM)
+    if (p[58] > 1) return EP_ERR_CORRUPT;
+    I.layout = p[58];
+    if (!layout_fits(int(I.layout), I.rows, I.cols, I.blocks_per_lane)) return EP_ERR_CORRUPT;
     uint64_t tokens = 0;
     uint32_t tablen[kContexts];
     for (int c = 0; c < kContexts; ++c) {

@@ -76,7 +76,15 @@ typedef struct {
     int32_t q_index;          /* -1 = search the resolution; >= 0 = encode at this resolution index */
     int32_t n_threads;        /* host encoder threads; 0 = all hardware threads */
     int32_t coding;           /* EP_CODING_*: how coordinates 1..6 of a block are coded */
+    int32_t layout;           /* EP_LAYOUT_*: the block order of the tiles */
 } ep_config;
+
+/* EP_LAYOUT_ROWS: lane l of tile t codes blocks t*32K + 32k + l (the tiles follow the rows).
+ * EP_LAYOUT_GEMM: every tile is one operand tile of a consumer GEMM, 128 rows by 64 columns (32
+ * blocks per lane; rows a multiple of 128, columns a multiple of 64): tile t covers rows
+ * 128 (t / KT) .. +127 and columns 64 (t mod KT) .. +63 with KT = cols / 64, and lane l codes row
+ * 32 (k mod 4) + l of it at columns 8 (k / 4) .. +7. */
+enum ep_layout { EP_LAYOUT_ROWS = 0, EP_LAYOUT_GEMM = 1 };
 
 /* EP_CODING_AUTO pairs coordinates (1,2), (3,4), (5,6) of every block into one symbol each
  * when the stream holds at least 2^17 blocks and the tokens of their contexts concentrate below
@@ -104,6 +112,7 @@ typedef struct {
     uint64_t workspace_nbytes;/* device workspace ep_prepare fills and ep_decompress reads: 57344,
                                  108544 for a paired stream */
     uint32_t paired;          /* 1: coordinates 1..6 are coded as three pairs per block */
+    uint32_t layout;          /* EP_LAYOUT_*: the block order of the tiles */
 } ep_info;
 
 /* Upper bound of the stream size for ep_compress_host: with a searched resolution the
