@@ -121,6 +121,10 @@ def lib():
         L.ep_decompress_host_scratch.argtypes = [C.POINTER(StreamInfo), C.c_int32]
         L.ep_decompress_host.restype = C.c_int
         L.ep_decompress_host.argtypes = [C.POINTER(StreamInfo), p, p, C.c_int32, p, C.c_size_t, p, p]
+        L.ep_linear_fused_workspace.restype = C.c_size_t
+        L.ep_linear_fused_workspace.argtypes = [C.POINTER(StreamInfo), C.c_int64]
+        L.ep_linear_fused.restype = C.c_int
+        L.ep_linear_fused.argtypes = [C.POINTER(StreamInfo), p, p, p, C.c_int64, p, p, p, C.c_size_t, p, p]
         L.ep_ans_compress_bound.restype = C.c_size_t
         L.ep_ans_compress_bound.argtypes = [C.c_int64, C.c_int32]
         L.ep_ans_compress_host.restype = C.c_int
@@ -403,4 +407,47 @@ def ans_decompress(d_blob, info, workspace=None, out=None, status=None, stream=N
     rc = lib().ep_ans_decompress(C.byref(info), d_blob.data_ptr(), workspace.data_ptr(), out.data_ptr(), st, s)
     if rc != 0:
         raise EpError(rc, "ep_ans_decompress")
+    return out
+
+
+# ---------------------------------------------------------------- the decode fused into a GEMM
+def linear_fused_workspace(info, m):
+    """bytes of the fp32 partial sums ep_linear_fused needs for m tokens (0: the stream or m is not
+    one it takes)"""
+    return int(lib().ep_linear_fused_workspace(C.byref(info), m))
+
+
+def linear_fused(x, d_blob, info, tables, bias=None, out=None, work=None, status=None, stream=None):
+    """Y = X W^T (+ bias) with W decoded inside the tcgen05 GEMM (ep_linear_fused).  ``x``: CUDA
+    BF16 (m, K) with 1 <= m <= 128; ``d_blob``: a GEMM-ordered (LAYOUT_GEMM) BF16 stream on the
+    device; ``tables``: from ``prepare``.  Returns the BF16 (m, N) output."""
+    if not (x.is_cuda and d_blob.is_cuda and tables.is_cuda):
+        raise EpError(-1, "linear_fused works on CUDA tensors")
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != info.cols:
+        raise EpError(-1, "x must be a BF16 (m, in_features) tensor")
+    x = x.contiguous()
+    m = x.shape[0]
+    L = lib()
+    need = linear_fused_workspace(info, m)
+    if need == 0:
+        raise EpError(-1, "ep_linear_fused takes a GEMM-ordered BF16 stream and 1 <= m <= 128")
+    if work is None or work.numel() * work.element_size() < need:
+        work = torch.empty(need, dtype=torch.uint8, device=x.device)
+    elif not (work.is_cuda and work.is_contiguous()):
+        raise EpError(-1, "work must be a contiguous CUDA tensor")
+    if out is None:
+        out = torch.empty((m, info.rows), dtype=torch.bfloat16, device=x.device)
+    elif not (out.is_cuda and out.dtype == torch.bfloat16 and out.is_contiguous() and out.numel() == m * info.rows):
+        raise EpError(-1, "out must be a contiguous CUDA BF16 tensor of m x out_features elements")
+    if bias is not None:
+        bias = bias.contiguous()
+        if not bias.is_cuda or bias.dtype != torch.bfloat16 or bias.numel() != info.rows:
+            raise EpError(-1, "bias must be a CUDA BF16 tensor with out_features elements")
+    st = status.data_ptr() if status is not None else None
+    s = (stream or torch.cuda.current_stream(x.device)).cuda_stream
+    rc = L.ep_linear_fused(C.byref(info), d_blob.data_ptr(), tables.data_ptr(), x.data_ptr(), m,
+                           bias.data_ptr() if bias is not None else None, out.data_ptr(), work.data_ptr(),
+                           work.numel() * work.element_size(), st, s)
+    if rc != 0:
+        raise EpError(rc, "ep_linear_fused")
     return out

@@ -32,12 +32,15 @@ class LatticeRANSConfig:
     (per-row absmax codes; the rate then counts the row scales).  blocks_per_lane: 0 picks it
     from the shape.  n_threads: host encoder threads (0: all cores).  coding: 0 automatic, 1 one
     token per coordinate, 2 coordinates 1..6 in pairs whenever their tokens allow (the decoder
-    then does 5 table lookups per E8 block instead of 8)."""
+    then does 5 table lookups per E8 block instead of 8).  layout: "rows" (the tiles follow the
+    rows) or "gemm" (every tile one 128 x 64 operand tile of a consumer GEMM; rows a multiple of
+    128, columns of 64; what CompressedLinear's fused forward reads)."""
     target_bpp: float = 4.0
     container: object = None
     blocks_per_lane: int = 0
     n_threads: int = 0
     coding: int = 0
+    layout: str = "rows"
 
 
 @dataclass
@@ -201,14 +204,18 @@ def compress(tensor, config):
     if not isinstance(config, LatticeRANSConfig):
         raise B.EpError(-1, "config must be a LatticeRANSConfig or a TileANSConfig")
     container = 0 if config.container is None else config.container
+    layouts = {"rows": B.LAYOUT_ROWS, "gemm": B.LAYOUT_GEMM}
+    if config.layout not in layouts:
+        raise B.EpError(-1, f"layout must be 'rows' or 'gemm', not {config.layout!r}")
+    layout = layouts[config.layout]
     try:
         if tensor.is_cuda:  # the GPU compressor writes the host compressor's bytes
             blob = B.compress_device(tensor, config.target_bpp, container=container,
-                                     blocks_per_lane=config.blocks_per_lane, coding=config.coding)
+                                     blocks_per_lane=config.blocks_per_lane, coding=config.coding, layout=layout)
         else:
             blob = B.compress(tensor, config.target_bpp, container=container,
                               blocks_per_lane=config.blocks_per_lane, n_threads=config.n_threads,
-                              coding=config.coding)
+                              coding=config.coding, layout=layout)
     except B.EpError as e:
         if e.status != -4:  # EP_ERR_TARGET_UNREACHABLE
             raise

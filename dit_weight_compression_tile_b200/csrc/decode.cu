@@ -28,6 +28,7 @@
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "../../include/eptile.h"
@@ -141,6 +142,11 @@ struct Packer<EP_BF16> {
     }
     __device__ __forceinline__ void store(void *out, uint32_t b) {
         reinterpret_cast<uint4 *>(out)[b] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    // the 8 values as 16 bytes at a shared-memory address (an operand tile of the fused GEMM)
+    __device__ __forceinline__ void store_shared(uint32_t a) {
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
+                     : "memory");
     }
     // the first n values at element e (the last block of a padded row: no vector store)
     __device__ __forceinline__ void store_n(void *out, uint64_t e, uint32_t n) {
@@ -414,9 +420,12 @@ __device__ __forceinline__ uint32_t resolve_pair(const Params &p, uint32_t h, ui
 // ------------------------------------------------------------------ the blocks of one tile
 // Lane l decodes blocks t*32K + 32k + l, k = 0..K-1.  ACT: the last tile, where lanes run out
 // of blocks.  ROWS: the launch's RowLayout.  Returns EP_DEC_* bits.
-template <int DT, bool SMEM, bool ACT, int ROWS, int MODE, typename Lim>
+// TO_SMEM (BF16 GEMM-ordered tiles only): the blocks go to the 128 x 64 BF16 operand tile at the
+// shared address `btile` in the 128-byte-swizzled K-major layout the tensor cores read (row r's
+// 16-byte chunk j at (r / 8) 1024 + (r mod 8) 128 + 16 (j xor r mod 8)), not to global memory.
+template <int DT, bool SMEM, bool ACT, int ROWS, int MODE, typename Lim, bool TO_SMEM = false>
 __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L, uint32_t &rb, uint32_t lut,
-                                                  Lim wlim, uint32_t t, uint32_t lane) {
+                                                  Lim wlim, uint32_t t, uint32_t lane, uint32_t btile = 0) {
     constexpr bool WIDE = MODE == kWide;
     constexpr bool R32 = ROWS == kRows32, RAG = ROWS == kRowsPadded, GEMM = ROWS == kRowsGemm;
     uint32_t b = t * 32u * p.K + lane;
@@ -544,6 +553,10 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
                 // a padded row's last block keeps its first cols % 8 values
                 const uint64_t c0 = 8ull * col;
                 if (act) pk.store_n(p.out, uint64_t(row) * p.cols + c0, uint32_t(min(p.cols - c0, uint64_t(8))));
+            } else if constexpr (TO_SMEM) {
+                static_assert(DT == EP_BF16 && ROWS == kRowsGemm, "operand tiles are BF16 GEMM tiles");
+                const uint32_t r = 32u * (k & 3u) + lane, ch = k >> 2;
+                pk.store_shared(btile + (r >> 3) * 1024u + (r & 7u) * 128u + ((ch ^ (r & 7u)) << 4));
             } else if (act) {
                 pk.store(p.out, b);
             }
@@ -575,9 +588,9 @@ done:
 
 // Decodes tile t with one warp.  `head` points at the tile (states, region lengths, word area):
 // a shared address (SMEM) or a global pointer.  Returns the EP_DEC_* bits of this lane.
-template <int DT, int ROWS, int MODE, bool SMEM, typename Ptr>
+template <int DT, int ROWS, int MODE, bool SMEM, typename Ptr, bool TO_SMEM = false>
 __device__ __forceinline__ uint32_t decode_tile(const Params &p, uint32_t lut, Ptr head, uint32_t tile_bytes,
-                                                uint32_t t, uint32_t lane) {
+                                                uint32_t t, uint32_t lane, uint32_t btile = 0) {
     Lane<SMEM> L;
     uint32_t len;
     if constexpr (SMEM) {
@@ -605,8 +618,8 @@ __device__ __forceinline__ uint32_t decode_tile(const Params &p, uint32_t lut, P
         L.wp = L.area + 2u * start;
         L.w = lds16(L.wp);
         uint32_t wlim = L.area + 2u * capacity;
-        if (uint64_t(t + 1) * 32u * p.K <= p.nb)
-            err = decode_blocks<DT, SMEM, false, ROWS, MODE>(p, L, rb, lut, wlim, t, lane);
+        if (TO_SMEM || uint64_t(t + 1) * 32u * p.K <= p.nb)
+            err = decode_blocks<DT, SMEM, false, ROWS, MODE, uint32_t, TO_SMEM>(p, L, rb, lut, wlim, t, lane, btile);
         else
             err = decode_blocks<DT, SMEM, true, ROWS, MODE>(p, L, rb, lut, wlim, t, lane);
     } else {
@@ -861,6 +874,222 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_
     }
 }
 
+// ------------------------------------------------------------------ the decode fused into a GEMM
+// Y = X W^T for a weight W (N x K) held as a GEMM-ordered stream (EP_LAYOUT_GEMM): each stream tile
+// is one 128 x 64 operand tile of W.  One CTA per (band of 128 output features, range of K tiles);
+// warps 0 .. S-1 each own a pipeline stage: they bulk-copy a stream tile into shared memory, decode
+// its 1024 blocks straight into the stage's B tile (BF16, 128-byte swizzled, K-major), copy the
+// matching 128 x 64 slice of X into the stage's A tile and arrive on the stage's `full` barrier;
+// warp S allocates the tensor memory, waits for each stage in K order, issues four
+// tcgen05.mma (M = 128 tokens, N = 128 features, K = 16 each) accumulating in TMEM and commits them
+// to the stage's `empty` barrier; after the last stage warps 0..3 read the 128 x 128 fp32
+// accumulator out of TMEM (tcgen05.ld) into the CTA's slice of the fp32 partial sums.
+constexpr int kLinMaxStages = 4;
+constexpr uint32_t kLinOpBytes = 128u * 64u * 2u;  // one 128 x 64 BF16 operand tile
+constexpr uint32_t kLinTmemCols = 128;             // the 128 x 128 fp32 accumulator
+
+struct LinParams {
+    Params dp;                 // the stream (tiles, tables, row factors, status)
+    const uint16_t *x;         // activations, BF16, M x cols row-major
+    float *part;               // fp32 partial sums, splits x M x N
+    uint32_t M, N;             // tokens, output features (rows of W)
+    uint32_t KT;               // K tiles per band (cols / 64)
+    uint32_t kt_per_split;
+    uint32_t stages;           // decoding warps = pipeline stages (<= kLinMaxStages)
+    uint32_t tile_buf;         // bytes of a stream-tile staging buffer
+    uint32_t off_bars, off_tile, off_ab;  // shared-memory layout (offsets from the dynamic base)
+};
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// UMMA shared-memory descriptor of a K-major, 128-byte-swizzled operand at shared address a: start
+// address and stride between 8-row groups (1024 bytes) in 16-byte units, descriptor version 1,
+// layout type 2 (128-byte swizzle); the leading offset is unused by swizzled K-major layouts (1)
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t a) {
+    return uint64_t((a >> 4) & 0x3fffu) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) | (uint64_t(1) << 46) |
+           (uint64_t(2) << 61);
+}
+
+// instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator, BF16 A and B, both K-major,
+// N = 128 (bits 17..22: N / 8), M = 128 (bits 24..28: M / 16)
+constexpr uint32_t kLinIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+
+template <int MODE>
+__global__ void __launch_bounds__((kLinMaxStages + 1) * 32, 1) linear_kernel(const __grid_constant__ LinParams P) {
+    extern __shared__ __align__(128) uint8_t smem[];  // operand tiles are aligned to 1024 bytes below
+    const Params &p = P.dp;
+    constexpr uint32_t kTables = uint32_t(MODE == kPaired ? kPairedTableBytes : kLutBytes);
+    const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5, S = P.stages;
+    const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    const uint32_t lut = base;
+    const uint32_t bars = base + P.off_bars;  // full[4], empty[4], copy[4], tables, done; then the TMEM slot
+    auto full = [&](uint32_t s) { return bars + 8u * s; };
+    auto empty = [&](uint32_t s) { return bars + 32u + 8u * s; };
+    auto copyb = [&](uint32_t s) { return bars + 64u + 8u * s; };
+    const uint32_t tbar = bars + 96u, done = bars + 104u, tmem_slot = bars + 112u;
+    // operand tiles: 1024-byte aligned in the shared window
+    const uint32_t ab = (base + P.off_ab + 1023u) & ~1023u;
+    auto atile = [&](uint32_t s) { return ab + 2u * kLinOpBytes * s; };
+    auto btile = [&](uint32_t s) { return ab + 2u * kLinOpBytes * s + kLinOpBytes; };
+    auto tbuf = [&](uint32_t s) { return base + P.off_tile + P.tile_buf * s; };
+    const uint32_t band = blockIdx.x;
+    const uint32_t kt0 = blockIdx.y * P.kt_per_split;
+    const uint32_t nkt = min(P.KT, kt0 + P.kt_per_split) - kt0;
+
+    if (threadIdx.x == 0) {
+        for (uint32_t s = 0; s < S; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+            mbar_init(copyb(s), 1);
+        }
+        mbar_init(tbar, 1);
+        mbar_init(done, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async();
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (warp == S) {  // the tensor memory of the accumulator (the whole warp allocates)
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tmem_slot),
+                     "r"(kLinTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (threadIdx.x == 0) {
+        mbar_expect(tbar, kTables);
+        bulk_g2s(lut, p.tables, kTables, tbar);
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = lds32(tmem_slot);
+    bool ok = mbar_wait(tbar, 0);
+    uint32_t err = ok ? 0u : uint32_t(EP_DEC_TIMEOUT);
+
+    if (warp < S) {
+        // ---- producers: stream tile -> B stage (decoded), X slice -> A stage
+        uint32_t use = 0;
+        for (uint32_t j = warp; j < nkt && ok; j += S, ++use) {
+            const uint32_t kt = kt0 + j, t = band * P.KT + kt;
+            if (use > 0 && !mbar_wait(empty(warp), (use - 1) & 1u)) {  // the MMAs of the stage's last use
+                err |= EP_DEC_TIMEOUT;
+                break;
+            }
+            const uint32_t beg = __ldg(p.dir + t), end = __ldg(p.dir + t + 1), bytes = (end - beg) * 16u;
+            if (end < beg + uint32_t(kTileHead / 16) || uint64_t(end) > p.tile_units || bytes + kSlack > P.tile_buf) {
+                err |= EP_DEC_BAD_TILE;
+                break;
+            }
+            if (lane == 0) {
+                fence_proxy_async();
+                mbar_expect(copyb(warp), bytes);
+                bulk_g2s(tbuf(warp), p.tiles + size_t(beg) * 16, bytes, copyb(warp));
+            }
+            // X rows m < M, columns 64 kt .. +63: 8 lanes per row, 16 bytes each; rows >= M zero
+            const uint32_t a = atile(warp), c = lane & 7u;
+            for (uint32_t m = lane >> 3; m < 128u; m += 4u) {
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (m < P.M) v = __ldg(reinterpret_cast<const uint4 *>(P.x + size_t(m) * p.cols + 64u * kt) + c);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a + (m >> 3) * 1024u + (m & 7u) * 128u +
+                                                                              ((c ^ (m & 7u)) << 4)),
+                             "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                             : "memory");
+            }
+            if (!mbar_wait(copyb(warp), use & 1u)) {
+                err |= EP_DEC_TIMEOUT;
+                break;
+            }
+            err |= decode_tile<EP_BF16, kRowsGemm, MODE, true, uint32_t, true>(p, lut, tbuf(warp), bytes, t, lane,
+                                                                              btile(warp));
+            // the operand tiles, written through the generic proxy, become visible to the tensor cores
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(full(warp));
+        }
+    } else if (warp == S) {
+        // ---- the MMA issuer: stages in K order, four K = 16 steps each
+        for (uint32_t j = 0; j < nkt; ++j) {
+            const uint32_t s = j % S;
+            if (!mbar_wait(full(s), (j / S) & 1u)) {
+                err |= EP_DEC_TIMEOUT;
+                break;
+            }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            if (lane == 0) {
+#pragma unroll
+                for (uint32_t ks = 0; ks < 4; ++ks) {
+                    const uint64_t da = umma_desc_sw128(atile(s) + 32u * ks), db = umma_desc_sw128(btile(s) + 32u * ks);
+                    const uint32_t acc = (j | ks) ? 1u : 0u;
+                    asm volatile(
+                        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+                        "l"(da), "l"(db), "r"(kLinIdesc), "r"(acc)
+                        : "memory");
+                }
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                                 empty(s))
+                             : "memory");
+            }
+            __syncwarp();
+        }
+        if (lane == 0)
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(done)
+                         : "memory");
+        __syncwarp();
+    }
+    // ---- epilogue: warps 0..3 read TMEM lanes 32 w .. 32 w + 31 (tokens), 128 fp32 columns each
+    if (warp < 4) {
+        if (!mbar_wait(done, 0)) err |= EP_DEC_TIMEOUT;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t m = 32u * warp + lane;
+        float *dst = P.part + (size_t(blockIdx.y) * P.M + m) * P.N + 128u * band;
+#pragma unroll
+        for (uint32_t c0 = 0; c0 < 128u; c0 += 32u) {
+            uint32_t r[32];
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+                "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                  "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                  "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+                  "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+                  "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                : "r"(tmem + ((32u * warp) << 16) + c0));
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            if (m < P.M) {
+#pragma unroll
+                for (uint32_t q = 0; q < 32u; q += 4u)
+                    *reinterpret_cast<float4 *>(dst + c0 + q) =
+                        make_float4(__uint_as_float(r[q]), __uint_as_float(r[q + 1]), __uint_as_float(r[q + 2]),
+                                    __uint_as_float(r[q + 3]));
+            }
+        }
+    }
+    if (err && p.status && lane == 0) atomicOr(p.status, err);
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == S) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kLinTmemCols)
+                     : "memory");
+    }
+}
+
+// Y (BF16, M x N) = the sum of the splits' fp32 partial sums, plus the bias (BF16, nullable), rounded
+// once to nearest even
+__global__ void linear_reduce_kernel(const float *part, uint32_t splits, uint32_t M, uint32_t N, const uint16_t *bias,
+                                     uint16_t *y) {
+    const size_t n = size_t(M) * N;
+    for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += size_t(gridDim.x) * blockDim.x) {
+        float acc = 0.0f;
+        for (uint32_t s = 0; s < splits; ++s) acc += part[s * n + i];
+        if (bias) acc += __uint_as_float(uint32_t(bias[i % N]) << 16);
+        const __nv_bfloat16 h = __float2bfloat16_rn(acc);
+        y[i] = *reinterpret_cast<const uint16_t *>(&h);
+    }
+}
+
 // ------------------------------------------------------------------ host side
 struct DeviceCache {
     std::mutex mu;
@@ -996,6 +1225,59 @@ uint32_t pack_splits(const ep_info *info) {
     return s;
 }
 
+// the decode kernels' view of a device stream and its prepared tables
+Params params_of(const ep_info *info, const void *d_blob, const void *d_tables, void *d_out, uint32_t *d_status) {
+    Params p;
+    const uint8_t *base = static_cast<const uint8_t *>(d_blob);
+    p.dir = reinterpret_cast<const uint32_t *>(base + info->off_dir);
+    p.tiles = base + info->off_tiles;
+    p.rowf = reinterpret_cast<const float *>(base + info->off_rowf);
+    p.tables = static_cast<const uint32_t *>(d_tables);
+    p.out = d_out;
+    p.status = d_status;
+    p.tile_units = (info->storage_nbytes - info->off_tiles) / 16;
+    p.cols = uint64_t(info->cols);
+    p.cb = uint32_t((info->cols + 7) / 8);
+    p.nb = uint32_t(info->rows) * p.cb;
+    p.rows = uint32_t(info->rows);
+    p.K = info->blocks_per_lane;
+    p.T = info->n_tiles;
+    p.splits = pack_splits(info);
+    for (int c = 0; c < 2; ++c) {
+        p.pair_A[c] = info->paired ? info->ntok[1 + c] : 0u;
+        p.pair_rawb[c] = pair_raw_bits(p.pair_A[c]);
+    }
+    p.tile_buf = 0;
+    p.nbuf = 0;
+    return p;
+}
+
+// ---- the fused GEMM's launch plan: bands of 128 output features, K tiles split across CTAs so that
+// about one CTA runs per SM; shared memory = tables, barriers, the stages' stream-tile buffers and
+// their A and B operand tiles
+struct LinPlan {
+    uint32_t nbands, KT, splits, kt_per_split, stages, tile_buf, off_bars, off_tile, off_ab;
+    size_t smem;
+};
+
+LinPlan lin_plan(const ep_info *info, int sms) {
+    LinPlan L{};
+    const bool paired = info->paired != 0;
+    L.nbands = uint32_t(info->rows / 128);
+    L.KT = uint32_t(info->cols / 64);
+    uint32_t want = L.nbands ? (uint32_t(sms) + L.nbands - 1) / L.nbands : 1u;
+    want = want < 1 ? 1u : (want > L.KT ? L.KT : want);
+    L.kt_per_split = (L.KT + want - 1) / want;
+    L.splits = (L.KT + L.kt_per_split - 1) / L.kt_per_split;
+    L.stages = paired ? 3u : 4u;
+    L.tile_buf = uint32_t((info->max_tile_nbytes + kSlack + 15) & ~uint64_t(15));
+    L.off_bars = uint32_t(paired ? kPairedTableBytes : kLutBytes);
+    L.off_tile = L.off_bars + 128u;
+    L.off_ab = L.off_tile + L.stages * L.tile_buf;
+    L.smem = size_t(L.off_ab) + 1024u + size_t(L.stages) * 2u * kLinOpBytes;
+    return L;
+}
+
 }  // namespace
 }  // namespace ep
 
@@ -1035,26 +1317,7 @@ extern "C" int ep_decompress(const ep_info *info, const void *d_blob, const void
         return EP_ERR_INVALID_ARG;
     int rc = check_info(info);
     if (rc != EP_OK) return rc;
-    Params p;
-    const uint8_t *base = static_cast<const uint8_t *>(d_blob);
-    p.dir = reinterpret_cast<const uint32_t *>(base + info->off_dir);
-    p.tiles = base + info->off_tiles;
-    p.rowf = reinterpret_cast<const float *>(base + info->off_rowf);
-    p.tables = static_cast<const uint32_t *>(d_workspace);
-    p.out = d_out;
-    p.status = d_status;
-    p.tile_units = (info->storage_nbytes - info->off_tiles) / 16;
-    p.cols = uint64_t(info->cols);
-    p.cb = uint32_t((info->cols + 7) / 8);
-    p.nb = uint32_t(info->rows) * p.cb;
-    p.rows = uint32_t(info->rows);
-    p.K = info->blocks_per_lane;
-    p.T = info->n_tiles;
-    p.splits = pack_splits(info);
-    for (int c = 0; c < 2; ++c) {
-        p.pair_A[c] = info->paired ? info->ntok[1 + c] : 0u;
-        p.pair_rawb[c] = pair_raw_bits(p.pair_A[c]);
-    }
+    Params p = params_of(info, d_blob, d_workspace, d_out, d_status);
     int device;
     cudaError_t e = cudaGetDevice(&device);
     if (e != cudaSuccess) return EP_ERR_CUDA;
@@ -1071,6 +1334,104 @@ extern "C" int ep_decompress(const ep_info *info, const void *d_blob, const void
     default: return EP_ERR_INVALID_ARG;
     }
     return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ ep_linear_fused
+namespace ep {
+namespace {
+
+int device_sms(int *device, int *sms) {
+    if (cudaGetDevice(device) != cudaSuccess || *device < 0 || *device >= 64) return EP_ERR_CUDA;
+    std::lock_guard<std::mutex> g(g_cache.mu);
+    if (!g_cache.sms[*device] &&
+        cudaDeviceGetAttribute(&g_cache.sms[*device], cudaDevAttrMultiProcessorCount, *device) != cudaSuccess)
+        return EP_ERR_CUDA;
+    *sms = g_cache.sms[*device];
+    return EP_OK;
+}
+
+bool linear_ok(const ep_info *info, int64_t m) {
+    return info && info->layout == 1 && info->container_dtype == EP_BF16 && m >= 1 && m <= 128 &&
+           check_info(info) == EP_OK;
+}
+
+struct LinCache {
+    std::mutex mu;
+    size_t smem_set[64][2] = {};
+};
+LinCache g_lin;
+
+}  // namespace
+}  // namespace ep
+
+extern "C" size_t ep_linear_fused_workspace(const ep_info *info, int64_t m) {
+    using namespace ep;
+    if (!linear_ok(info, m)) return 0;
+    int device, sms;
+    if (device_sms(&device, &sms) != EP_OK) return 0;
+    const LinPlan L = lin_plan(info, sms);
+    return size_t(L.splits) * size_t(m) * size_t(info->rows) * sizeof(float);
+}
+
+extern "C" int ep_linear_fused(const ep_info *info, const void *d_blob, const void *d_tables, const void *d_x,
+                               int64_t m, const void *d_bias, void *d_y, void *d_work, size_t work_nbytes,
+                               uint32_t *d_status, ep_stream_t stream) {
+    using namespace ep;
+    if (!d_blob || !d_tables || !d_x || !d_y || !d_work || !linear_ok(info, m)) return EP_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(d_blob) | reinterpret_cast<uintptr_t>(d_tables) |
+         reinterpret_cast<uintptr_t>(d_x) | reinterpret_cast<uintptr_t>(d_work)) & 15u)
+        return EP_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(d_y) & 1u || reinterpret_cast<uintptr_t>(d_bias) & 1u) return EP_ERR_INVALID_ARG;
+    int device, sms;
+    if (device_sms(&device, &sms) != EP_OK) return EP_ERR_CUDA;
+    const LinPlan L = lin_plan(info, sms);
+    if (work_nbytes < size_t(L.splits) * size_t(m) * size_t(info->rows) * sizeof(float)) return EP_ERR_INVALID_ARG;
+    if (L.smem > kSmemLimit) return EP_ERR_UNSUPPORTED;  // tiles too large for the stages beside the tables
+    LinParams P;
+    P.dp = params_of(info, d_blob, d_tables, nullptr, d_status);
+    P.x = static_cast<const uint16_t *>(d_x);
+    P.part = static_cast<float *>(d_work);
+    P.M = uint32_t(m);
+    P.N = uint32_t(info->rows);
+    P.KT = L.KT;
+    P.kt_per_split = L.kt_per_split;
+    P.stages = L.stages;
+    P.tile_buf = L.tile_buf;
+    P.off_bars = L.off_bars;
+    P.off_tile = L.off_tile;
+    P.off_ab = L.off_ab;
+    const bool paired = info->paired != 0;
+    auto kern = paired ? linear_kernel<kPaired> : (wide_fields(info) ? linear_kernel<kWide> : linear_kernel<kNarrow>);
+    {
+        std::lock_guard<std::mutex> g(g_lin.mu);
+        size_t &set = g_lin.smem_set[device][paired ? 1 : 0];
+        if (set < L.smem) {
+            // one attribute for the coding modes of a table size
+            decltype(kern) ks[2] = {linear_kernel<kNarrow>, linear_kernel<kWide>};
+            if (paired) ks[0] = ks[1] = linear_kernel<kPaired>;
+            for (auto k : ks)
+                if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(L.smem)) != cudaSuccess)
+                    return EP_ERR_CUDA;
+            set = L.smem;
+        }
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(L.nbands, L.splits);
+    cfg.blockDim = dim3((L.stages + 1) * 32);
+    cfg.dynamicSmemBytes = L.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, P) != cudaSuccess) return EP_ERR_CUDA;
+    const size_t n = size_t(m) * info->rows;
+    const unsigned rgrid = unsigned(std::min<size_t>((n + 255) / 256, size_t(sms) * 8));
+    linear_reduce_kernel<<<rgrid, 256, 0, s>>>(P.part, L.splits, P.M, P.N, static_cast<const uint16_t *>(d_bias),
+                                               static_cast<uint16_t *>(d_y));
+    return cudaGetLastError() == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------ ep_decompress_noalloc

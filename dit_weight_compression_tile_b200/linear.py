@@ -3,8 +3,9 @@
 linear layers whose weight is held as a lattice-rANS stream and reconstructed for every forward
 call.  The reconstruction is the fused decode kernel (ep_decompress) into a buffer the layer
 keeps; the product is the library GEMM (cuBLAS through torch: F.linear, torch._scaled_mm for
-FP8, torch._int_mm for INT8).  Decoding into the GEMM's operand tiles, without the weight's round
-trip through memory, is not done here.
+FP8, torch._int_mm for INT8).  A BF16 layer whose stream is GEMM-ordered (LatticeRANSConfig(layout=
+"gemm")) instead decodes inside its own tcgen05 GEMM (ep_linear_fused) when the call has at most
+128 tokens: the weight then never passes through memory in BF16.
 
 The FP8 / INT8 layers hold per-row absmax codes (the stream's code container) and quantize the
 activations per row of x the same way (E4M3 with scale amax / 448, INT8 with amax / 127, RNE);
@@ -17,7 +18,7 @@ import torch.nn as nn
 import torch.nn.functional as F
 
 from . import binding as B
-from .compressed import CompressedTensor, LatticeRANSConfig, compress, decompress
+from .compressed import CompressedTensor, LatticeRANSConfig, _tables, compress, decompress
 
 class CompressedLinear(nn.Module):
     """y = x W^T + b with W held compressed (lossy lattice-rANS, `config`) and decoded per call.
@@ -37,6 +38,7 @@ class CompressedLinear(nn.Module):
             if bias else None
         self._weight = None
         self._buf = None  # decoded weight (or codes), reused across calls
+        self._work = None  # fp32 partial sums of the fused GEMM, reused across calls
 
     # ---- construction
     @classmethod
@@ -95,7 +97,28 @@ class CompressedLinear(nn.Module):
         out = decompress(w).to(self.init_dtype)
         return out if device is None else out.to(device)
 
+    def fused_for(self, x):
+        """whether forward(x) decodes inside the fused GEMM (ep_linear_fused): a GEMM-ordered BF16
+        stream on x's CUDA device, x BF16 with 1..128 tokens"""
+        w = self._weight
+        if w is None or w.compress_method != "lattice_rans" or not x.is_cuda or x.dtype != torch.bfloat16:
+            return False
+        info = w.info
+        tokens = x.numel() // self.in_features if x.dim() else 0
+        return (info.layout == B.LAYOUT_GEMM and info.container_dtype == B.BF16 and w.device == x.device
+                and 1 <= tokens <= 128)
+
     def forward(self, x):
+        if self.fused_for(x):
+            w = self._weight
+            s = torch.cuda.current_stream(x.device)
+            tables = _tables(w, s)
+            bias = None if self.bias is None else self.bias.to(torch.bfloat16)
+            if self._work is None or self._work.device != x.device:
+                self._work = torch.empty(B.linear_fused_workspace(w.info, 128), dtype=torch.uint8, device=x.device)
+            y = B.linear_fused(x.reshape(-1, self.in_features), w.blob, w.info, tables, bias=bias, work=self._work,
+                               stream=s)
+            return y.reshape(*x.shape[:-1], self.out_features)
         w = self._decoded()
         return F.linear(x, w.to(x.dtype) if w.dtype != x.dtype else w, self.bias)
 
@@ -106,7 +129,7 @@ class CompressedLinear(nn.Module):
             probe = fn(torch.empty(0, device=self._weight.device))
             if probe.device != self._weight.device:  # .to(device) moves the stream; dtypes stay as encoded
                 self._weight = self._weight.to(probe.device)
-                self._buf = None
+                self._buf = self._work = None
         return self
 
     def _save_to_state_dict(self, destination, prefix, keep_vars):
@@ -126,7 +149,7 @@ class CompressedLinear(nn.Module):
             else:
                 dev = self.bias.device if self.bias is not None else w.device
                 self._weight = w.to(dev)
-                self._buf = None
+                self._buf = self._work = None
         elif strict:
             missing_keys.append(prefix + "weight.ep_meta")
         rest = {k: v for k, v in state_dict.items() if not k.startswith(prefix + "weight.")}

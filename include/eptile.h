@@ -212,6 +212,30 @@ int ep_prepare(const ep_info *info, const void *d_blob, void *d_workspace, uint3
 int ep_decompress(const ep_info *info, const void *d_blob, const void *d_workspace, void *d_out, int32_t out_dtype,
                   uint32_t *d_status, ep_stream_t stream);
 
+/* A linear layer's forward with the weight decoded inside the GEMM ("EntroPack API reference",
+ * CompressedLinear: the weight is reconstructed for every forward call; here it never reaches
+ * global memory): Y = X W^T (+ bias) for a stream written with EP_LAYOUT_GEMM and a BF16 container.
+ *   info        from ep_stream_info; W is info->rows (N, output features) x info->cols (K).
+ *   d_blob      the stream in device memory (16-byte aligned); d_tables the slot tables
+ *               ep_prepare built from it.
+ *   d_x         BF16 activations, m x K row-major (16-byte aligned), 1 <= m <= 128.
+ *   d_bias      nullable BF16 bias of N elements.
+ *   d_y         BF16 output, m x N row-major: the fp32 sum rounded once to nearest even.
+ *   d_work      caller-owned device scratch of ep_linear_fused_workspace(info, m) bytes (fp32
+ *               partial sums of the K splits), 16-byte aligned.
+ *   d_status    nullable device uint32: EP_DEC_* bits of stream damage.
+ * One launch of the fused kernel (a CTA per band of 128 output features and range of K tiles:
+ * warps bulk-copy stream tiles into shared memory and decode them straight into 128-byte-swizzled
+ * BF16 operand tiles beside the matching slices of X; one warp issues tcgen05.mma into a
+ * 128 x 128 fp32 accumulator in tensor memory; the accumulator leaves through tcgen05.ld) and
+ * one small launch that adds the splits and the bias.  Asynchronous; allocates nothing.
+ * EP_ERR_INVALID_ARG for another layout, container or m out of range, EP_ERR_UNSUPPORTED when a
+ * tile is too large for the pipeline's shared memory. */
+size_t ep_linear_fused_workspace(const ep_info *info, int64_t m);
+int ep_linear_fused(const ep_info *info, const void *d_blob, const void *d_tables, const void *d_x, int64_t m,
+                    const void *d_bias, void *d_y, void *d_work, size_t work_nbytes, uint32_t *d_status,
+                    ep_stream_t stream);
+
 /* ep_prepare + ep_decompress for callers that cannot allocate device memory: a plugin inside an
  * inference engine that owns all device memory and forbids allocation in its forward path, or code
  * that must not trigger the device-wide synchronisation a cudaMalloc/cudaFree can cause.  No

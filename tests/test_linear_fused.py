@@ -1,0 +1,117 @@
+"""The decode fused into a tcgen05 GEMM (ep_linear_fused; "EntroPack API reference",
+CompressedLinear: the weight is reconstructed on every forward call).
+
+Host side: the entry point refuses what it cannot take before any launch (a row-ordered stream, a
+non-BF16 container, m outside [1, 128], null or misaligned pointers).  GPU side (marked gpu): the
+output equals the library GEMM applied to the oracle's decoded weight, within the tolerance of two
+fp32 sums of the same BF16 products taken in different orders and rounded once to BF16 (the bound
+below), for single and paired streams, with and without bias, several m and K splits."""
+import ctypes as C
+
+import numpy as np
+import pytest
+import torch
+
+from dit_weight_compression_tile_b200 import binding as B
+from dit_weight_compression_tile_b200 import synth
+
+
+def gemm_stream(shape, target=4.0, coding=B.CODING_AUTO, container=0, seed=1):
+    w = synth.row_lognormal(*shape, seed=seed)
+    blob = B.compress(w, target, coding=coding, container=container, layout=B.LAYOUT_GEMM)
+    return w, blob, B.stream_info(blob)
+
+
+def test_refused_before_any_launch():
+    L = B.lib()
+    _, blob, info = gemm_stream((128, 128))
+    fake = C.c_void_p(1 << 20)  # never dereferenced: every call below returns before a launch
+    assert L.ep_linear_fused_workspace(C.byref(info), 0) == 0
+    assert L.ep_linear_fused_workspace(C.byref(info), 129) == 0
+    assert L.ep_linear_fused(C.byref(info), fake, fake, fake, 0, None, fake, fake, 1 << 20, None, None) == -1
+    assert L.ep_linear_fused(C.byref(info), None, fake, fake, 4, None, fake, fake, 1 << 20, None, None) == -1
+    assert L.ep_linear_fused(C.byref(info), C.c_void_p((1 << 20) + 4), fake, fake, 4, None, fake, fake, 1 << 20,
+                             None, None) == -1
+    rows = B.stream_info(B.compress(synth.gaussian(128, 128, 0.02, seed=2), 4.0))
+    assert rows.layout == 0
+    assert L.ep_linear_fused_workspace(C.byref(rows), 4) == 0
+    assert L.ep_linear_fused(C.byref(rows), fake, fake, fake, 4, None, fake, fake, 1 << 20, None, None) == -1
+    int8 = B.stream_info(B.compress(synth.gaussian(128, 128, 0.02, seed=3), 3.0, container=B.INT8,
+                                    layout=B.LAYOUT_GEMM))
+    assert L.ep_linear_fused(C.byref(int8), fake, fake, fake, 4, None, fake, fake, 1 << 20, None, None) == -1
+
+
+def reference(oracle, blob, x, bias):
+    """the library GEMM (fp32) on the oracle's decoded weight, and the bound on the fused result:
+    both sum the same exact BF16 x BF16 products in fp32, in different orders; the difference is at
+    most K u sum |x_k w_k| (u = 2^-24, a standard bound for two recursive sums), and one BF16
+    rounding (half an ulp, 2^-9 relative) of each"""
+    rc, st, _, wd = oracle.decode(blob.numpy())
+    assert rc == 0 and st == 0
+    wf = torch.from_numpy(wd.view(np.int16)).view(torch.bfloat16).float()
+    xf = x.float().cpu()
+    y = xf @ wf.T + (bias.float().cpu() if bias is not None else 0.0)
+    mag = xf.abs() @ wf.abs().T + (bias.float().cpu().abs() if bias is not None else 0.0)
+    K = xf.shape[1]
+    tol = K * 2.0 ** -24 * mag + 2.0 ** -8 * y.abs() + 1e-30
+    return y, tol
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("shape,m,coding,with_bias", [((128, 128), 1, B.CODING_SINGLE, False),
+                                                      ((256, 512), 16, B.CODING_SINGLE, True),
+                                                      ((384, 1024), 64, B.CODING_PAIRED, True),
+                                                      ((128, 3072), 128, B.CODING_AUTO, False),
+                                                      ((1024, 3072), 7, B.CODING_PAIRED, True)])
+def test_fused_equals_gemm_on_decoded_weight(oracle, shape, m, coding, with_bias):
+    w, blob, info = gemm_stream(shape, coding=coding, seed=shape[1] + m)
+    g = torch.Generator().manual_seed(m)
+    x = (torch.randn(m, shape[1], generator=g) * 0.5).to(torch.bfloat16)
+    bias = (torch.randn(shape[0], generator=g) * 0.1).to(torch.bfloat16) if with_bias else None
+    d = blob.cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tables = B.prepare(d, info, status=status)
+    y = B.linear_fused(x.cuda(), d, info, tables, bias=bias.cuda() if bias is not None else None, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref, tol = reference(oracle, blob, x, bias)
+    got = y.float().cpu()
+    assert got.shape == ref.shape
+    bad = (got - ref).abs() > tol
+    assert not bad.any(), (float((got - ref).abs().max()), int(bad.sum()))
+    # a second call on the same tables gives the same bits
+    y2 = B.linear_fused(x.cuda(), d, info, tables, bias=bias.cuda() if bias is not None else None)
+    assert torch.equal(y2, y)
+
+
+def test_layer_takes_the_fused_path_only_where_it_applies():
+    from dit_weight_compression_tile_b200 import CompressedLinear, LatticeRANSConfig
+    lin = torch.nn.Linear(128, 256, dtype=torch.bfloat16)
+    gemm = CompressedLinear.from_linear(lin, config=LatticeRANSConfig(4.0, layout="gemm"))
+    rows = CompressedLinear.from_linear(lin, config=LatticeRANSConfig(4.0))
+    assert gemm.weight.info.layout == B.LAYOUT_GEMM and rows.weight.info.layout == B.LAYOUT_ROWS
+    x = torch.zeros(3, 128, dtype=torch.bfloat16)
+    assert not gemm.fused_for(x)  # a host tensor
+    with pytest.raises(B.EpError):
+        CompressedLinear.from_linear(lin, config=LatticeRANSConfig(4.0, layout="columns"))
+    with pytest.raises(B.EpError):  # 100 output features are not whole 128-row bands
+        CompressedLinear.from_linear(torch.nn.Linear(128, 100), config=LatticeRANSConfig(4.0, layout="gemm"))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("tokens", [(1,), (4, 7), (128,), (3, 50)])
+def test_layer_forward(oracle, tokens):
+    from dit_weight_compression_tile_b200 import CompressedLinear, LatticeRANSConfig
+    torch.manual_seed(3)
+    lin = torch.nn.Linear(1024, 384, dtype=torch.bfloat16)
+    layer = CompressedLinear.from_linear(lin, config=LatticeRANSConfig(4.0, layout="gemm")).cuda()
+    x = (torch.randn(*tokens, 1024) * 0.5).to(torch.bfloat16)
+    y = layer(x.cuda())
+    m = x.numel() // 1024
+    assert layer.fused_for(x.cuda()) == (m <= 128)
+    blob = layer.weight.blob.cpu()
+    ref, tol = reference(oracle, blob, x.reshape(-1, 1024), layer.bias.detach().cpu())
+    got = y.float().cpu().reshape(-1, 384)
+    assert y.shape == (*tokens, 384)
+    # above 128 tokens the layer decodes and calls the library GEMM: summed in another order, same bound
+    assert torch.all((got - ref).abs() <= tol), float((got - ref).abs().max())
