@@ -35,6 +35,7 @@ sys.path.insert(0, ROOT)
 METRIC = "fused decode GB/s (container out) & Gweights/s at 4 bpp; % of HBM roofline"
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
 KERNEL_SRCS = {"decode_kernel": ("decode.cu", "device_util.cuh", "format.h"),
+               "linear_kernel": ("decode.cu", "device_util.cuh", "format.h"),
                "ans_decode_kernel": ("tile_ans.cu", "device_util.cuh", "tile_ans.h")}
 L2_BYTES = 126 * 2 ** 20
 
@@ -63,6 +64,14 @@ WORKLOADS = {
         layers=lambda: [("w", lambda: _synth().row_lognormal(4096, 4096, 1))], target=16.0, container=0,
         dims=[(4096, 4096)], scheme="tile_ans", shape="4096x4096",
         distribution="N(0, s_r^2), s_r = 0.02 exp(0.3 g), seed 1; lossless Tile-ANS (every bit kept)"),
+    "linear_fused_dit_block_16tok_bf16": dict(
+        layers=lambda: [(f"block0.{n}", (lambda l=l: _synth().dit_layer(0, l)))
+                        for l, n in enumerate(("qkv", "out", "mlp_up", "mlp_down"))],
+        target=4.0, container=0, scheme="linear_fused", tokens=16,
+        dims=[(3072, 9216), (3072, 3072), (3072, 12288), (12288, 3072)],
+        shape="block 0 linears {3072x9216, 3072x3072, 3072x12288, 12288x3072} (out x in), 16 tokens",
+        distribution="DiT block 0 weights (as dit_28blocks_hidden3072_bf16), GEMM block order; "
+                     "x = 0.5 N(0, 1) BF16, seed 5"),
     "outliers_8192x28672_bf16": dict(
         layers=lambda: [("w", lambda: _synth().gaussian_outliers(8192, 28672, 3))], target=4.0, container=0,
         dims=[(8192, 28672)],
@@ -74,6 +83,10 @@ TILE_ANS_METRIC = "lossless Tile-ANS decode GB/s (tensor out) & Gelements/s; % o
 
 def is_tile_ans(a):
     return WORKLOADS[a.workload].get("scheme") == "tile_ans"
+
+
+def is_linear(a):
+    return WORKLOADS[a.workload].get("scheme") == "linear_fused"
 
 
 def _synth():
@@ -118,9 +131,12 @@ def coding_label(infos):
 
 def workload_config(a):
     wl = WORKLOADS[a.workload]
-    return {"workload": a.workload, "shape": wl["shape"],
-            "target_bpp": "lossless" if wl.get("scheme") == "tile_ans" else a.target,
-            "distribution": wl["distribution"], "container": wl["container"] or "bf16"}
+    cfg = {"workload": a.workload, "shape": wl["shape"],
+           "target_bpp": "lossless" if wl.get("scheme") == "tile_ans" else a.target,
+           "distribution": wl["distribution"], "container": wl["container"] or "bf16"}
+    if wl.get("scheme") == "linear_fused":
+        cfg["tokens"] = wl["tokens"]
+    return cfg
 
 
 def l2_policy(a):
@@ -129,12 +145,15 @@ def l2_policy(a):
     state the same policy: workloads smaller than twice the L2 rotate over copies whose streams
     and outputs together exceed twice the L2"""
     wl = WORKLOADS[a.workload]
-    esz = 1 if wl["container"] in ("int8", "fp8_e4m3") else 2
+    # bytes per weight a step moves besides the stream: the container written (none for the fused
+    # GEMM, whose weight stays on chip)
+    esz = 0 if wl.get("scheme") == "linear_fused" else (1 if wl["container"] in ("int8", "fp8_e4m3") else 2)
     nominal = sum(r * c for r, c in wl["dims"]) * (a.target / 8.0 + esz)
     if nominal >= 2 * L2_BYTES:
         return 1, f"inputs larger than L2: {nominal / 1e6:.0f} MB per step"
     rot = min(8, -(-2 * L2_BYTES // int(nominal)))
-    return rot, f"inputs larger than L2: {rot} rotating stream+output copies ({rot * nominal / 1e6:.0f} MB)"
+    what = "stream" if esz == 0 else "stream+output"
+    return rot, f"inputs larger than L2: {rot} rotating {what} copies ({rot * nominal / 1e6:.0f} MB)"
 
 
 def bench_config(a, world):
@@ -756,6 +775,239 @@ def run_reference_tile_ans(a, rank, world):
             "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
+LINEAR_METRIC = "fused decode + tcgen05 GEMM Gweights/s (DiT block linears, 16 tokens); % of HBM roofline"
+
+
+def run_ours_linear(a, rank, world, local_rank):
+    """the decode fused into the tcgen05 GEMM (ep_linear_fused) on one DiT block's four linear
+    layers at a small token count: one step = the four products Y = X W^T, W from GEMM-ordered
+    streams, streams rotating past the L2 as in the other workloads.  Beside it, timed the same way
+    for context: the decode into a buffer followed by the library GEMM, and the library GEMM on
+    the BF16 weights (nn.Linear).  The decode-then-GEMM leg reads the same weights' row-ordered
+    streams at the same rate"""
+    import torch.nn.functional as F
+    from dit_weight_compression_tile_b200 import binding as B
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[a.workload]
+    m = wl["tokens"]
+    rot = l2_policy(a)[0]
+    stream = torch.cuda.Stream(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    g = torch.Generator().manual_seed(5)
+    layers, t_enc = [], 0.0
+    for name, make in wl["layers"]():
+        w = make().to(dev)
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        blob = B.compress_device(w, a.target, layout=B.LAYOUT_GEMM)
+        torch.cuda.synchronize(dev)
+        t_enc += time.perf_counter() - t0
+        info = B.stream_info(blob.cpu())
+        # the same weights in the row order, for the decode-then-GEMM comparison (its decode stores
+        # whole rows, the faster order for a decode into memory)
+        rblob = B.compress_device(w, a.target)
+        rinfo = B.stream_info(rblob.cpu())
+        x = (torch.randn(m, info.cols, generator=g) * 0.5).to(torch.bfloat16)
+        with torch.cuda.stream(stream):
+            blobs = [blob.clone() for _ in range(rot)]
+            tables = B.prepare(blobs[0], info, status=status, stream=stream)  # the copies hold the same stream
+            rblobs = [rblob.clone() for _ in range(rot)]
+            rtables = B.prepare(rblobs[0], rinfo, status=status, stream=stream)
+        layers.append(dict(name=name, w=w, info=info, blobs=blobs, tables=tables, rinfo=rinfo, rblobs=rblobs,
+                           rtables=rtables, x_host=x, x=x.to(dev),
+                           y=torch.empty(m, info.rows, dtype=torch.bfloat16, device=dev),
+                           work=torch.empty(B.linear_fused_workspace(info, m), dtype=torch.uint8, device=dev),
+                           wbuf=torch.empty(info.rows, info.cols, dtype=torch.bfloat16, device=dev)))
+    torch.cuda.synchronize(dev)
+
+    def fused(r, s_=stream):
+        for L in layers:
+            B.linear_fused(L["x"], L["blobs"][r], L["info"], L["tables"], out=L["y"], work=L["work"],
+                           status=status, stream=s_)
+
+    def unfused(r):
+        for L in layers:
+            F.linear(L["x"], B.decompress(L["rblobs"][r], L["rinfo"], workspace=L["rtables"], out=L["wbuf"],
+                                          stream=stream))
+
+    def dense(r):
+        for L in layers:
+            F.linear(L["x"], L["w"])
+
+    # the fused result against the library GEMM on the decoded weight: the same BF16 products summed
+    # in fp32 in another order (bound K 2^-24 sum |x w| + one BF16 rounding each)
+    with torch.cuda.stream(stream):
+        fused(0)
+    torch.cuda.synchronize(dev)
+    assert int(status.item()) == 0, "fused GEMM status"
+    for L in layers:
+        wd = B.decompress(L["blobs"][0], L["info"], workspace=L["tables"]).float()
+        ref = L["x"].float() @ wd.T
+        mag = L["x"].float().abs() @ wd.abs().T
+        tol = L["info"].cols * 2.0 ** -24 * mag + 2.0 ** -8 * ref.abs()
+        assert bool(((L["y"].float() - ref).abs() <= tol + 2.0 ** -8 * L["y"].float().abs()).all()), L["name"]
+
+    def timed(body, steps):
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for r in range(rot):
+                body(r)
+        replays, rest = divmod(steps, rot)
+        tail = None
+        if rest:
+            tail = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(tail, stream=stream):
+                for r in range(rest):
+                    body(r)
+        with torch.cuda.stream(stream):
+            for _ in range(max(1, -(-a.warmup // rot))):
+                graph.replay()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(replays + 2)]
+        with torch.cuda.stream(stream):
+            ev[0].record(stream)
+            for r in range(replays):
+                graph.replay()
+                ev[r + 1].record(stream)
+            if tail is not None:
+                tail.replay()
+            ev[-1].record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        per_step = sorted(1e3 * ev[r].elapsed_time(ev[r + 1]) / rot for r in range(replays))
+        return ev[0].elapsed_time(ev[-1]), per_step
+
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        fused_ms, per_step = timed(fused, a.steps)
+    total_ms = max_over_ranks(fused_ms, world, dev)
+    assert int(status.item()) == 0
+    unfused_ms, _ = timed(unfused, a.steps)
+    dense_ms, _ = timed(dense, a.steps)
+    nweights = sum(L["info"].rows * L["info"].cols for L in layers)
+    stream_bytes = sum(L["info"].storage_nbytes for L in layers)
+    act_bytes = sum(2 * m * (L["info"].cols + L["info"].rows) for L in layers)
+    step_s = total_ms / a.steps / 1e3
+    kernel_s = fused_ms / a.steps / 1e3
+    peak, peak_kind = measured_peaks()
+    achieved = (stream_bytes + act_bytes) / kernel_s / 1e9
+
+    # end to end through the public API: x copied in from pinned memory, the four fused products,
+    # y copied back into pinned memory, every step
+    xs_host = [L["x_host"].pin_memory() for L in layers]
+    ys_host = [torch.empty(m, L["info"].rows, dtype=torch.bfloat16).pin_memory() for L in layers]
+    e2e_steps = max(4, min(400, a.steps))
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for j in range(e2e_steps):
+            for L, xh, yh in zip(layers, xs_host, ys_host):
+                L["x"].copy_(xh, non_blocking=True)
+                B.linear_fused(L["x"], L["blobs"][j % rot], L["info"], L["tables"], out=L["y"], work=L["work"],
+                               stream=stream)
+                yh.copy_(L["y"], non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    if rank != 0:
+        return
+    line = {
+        "metric": LINEAR_METRIC, "value": round(job_rate(nweights, world, step_s) / 1e9, 2), "unit": "Gweights/s",
+        "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(step_s * 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": bench_config(a, world),
+        "stream": {"bpp": [round(L["info"].actual_bpp, 4) for L in layers], "paired": [L["info"].paired for L in layers],
+                   "layout": "gemm"},
+        "step_us": {"fused": round(1e3 * fused_ms / a.steps, 2),
+                    "decode_row_stream_then_library_gemm": round(1e3 * unfused_ms / a.steps, 2),
+                    "library_gemm_bf16_weights": round(1e3 * dense_ms / a.steps, 2)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic_for_kernel("linear_kernel", traffic_key(a)),
+                     "peak_kind": peak_kind, "algorithmic_bytes_per_step": stream_bytes + act_bytes,
+                     "note": "four linear_kernel + four partial-sum reduce launches per step; the fused kernel "
+                             "is bound by its decoding warps, not by HBM",
+                     "step_us_median": round(statistics.median(per_step), 3) if per_step else None,
+                     "step_us_min": round(per_step[0], 3) if per_step else None},
+        "e2e": {"value": round(job_rate(nweights * e2e_steps, world, e2e_ms / 1e3) / 1e9, 3), "unit": "Gweights/s",
+                "h2d_bytes_per_step": sum(2 * m * L["info"].cols for L in layers),
+                "d2h_bytes_per_step": sum(2 * m * L["info"].rows for L in layers)},
+        "gpu_launches": 2 * len(layers) * a.steps,
+        "clocks": clk.summary(),
+        "encode_s": round(t_enc, 3),
+    }
+    if world == 1 and not a.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_linear_baseline(a, layers, m)
+    print(json.dumps(line), flush=True)
+
+
+def cpu_linear_baseline(a, layers, m):
+    """the oracle (tile-parallel decode on every host core) plus a numpy fp32 GEMM, on a bounded
+    sample: the 3072x3072 layer's stream, whole, repeated for about --cpu-seconds"""
+    from oracle import oracle as O
+    L = min(layers, key=lambda L: L["info"].rows * L["info"].cols)
+    blob_np = L["blobs"][0].cpu().numpy()
+    rc, oinfo = O.parse(blob_np)
+    assert rc == 0
+    x_np = L["x_host"].float().numpy()
+    ncores = host_cores()
+    done = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < a.cpu_seconds:
+        rc, st, _, wd = O.decode_parallel(blob_np, threads=ncores, want_v=False)
+        assert rc == 0 and st == 0
+        _ = x_np @ (wd.view(np.uint16).astype(np.uint32) << 16).view(np.float32).T
+        done += 1
+    el = time.perf_counter() - t0
+    n = oinfo.rows * oinfo.cols
+    return {"value": round(done * n / el / 1e9, 4), "unit": "Gweights/s", "cores": ncores, "kind": "oracle",
+            "sample": f"{done} decodes of the {oinfo.rows}x{oinfo.cols} layer's stream by the C oracle on {ncores} "
+                      f"threads, each followed by x W^T in numpy fp32 ({m} tokens), in {el:.1f} s"}
+
+
+def run_reference_linear(a, rank, world):
+    """the oracle as the reference arm of the fused GEMM: the oracle's own GEMM-ordered stream of the
+    block's 3072x3072 layer, decoded on every host core and multiplied in numpy fp32, each step"""
+    if rank != 0:
+        return
+    from oracle import oracle as O
+    wl = WORKLOADS[a.workload]
+    m = wl["tokens"]
+    name, make = [(n, f) for n, f in wl["layers"]() if n.endswith(".out")][0]
+    w = make()
+    rc, blob = O.compress(w, a.target, layout=1)
+    assert rc == 0
+    rc, oinfo = O.parse(blob)
+    g = torch.Generator().manual_seed(5)
+    x_np = (torch.randn(m, oinfo.cols, generator=g) * 0.5).to(torch.bfloat16).float().numpy()
+    ncores = host_cores()
+
+    def step():
+        rc_, st_, _, wd = O.decode_parallel(blob, threads=ncores, want_v=False)
+        assert rc_ == 0 and st_ == 0
+        return x_np @ (wd.view(np.uint16).astype(np.uint32) << 16).view(np.float32).T
+
+    for _ in range(a.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        step()
+    t = time.perf_counter() - t0
+    n = oinfo.rows * oinfo.cols
+    rate = n * a.steps / t / 1e9
+    line = {"impl": "reference", "metric": LINEAR_METRIC, "value": round(rate, 4), "unit": "Gweights/s",
+            "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(1e3 * t / a.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": bench_config(a, world),
+            "cpu_baseline": {"value": round(rate, 4), "unit": "Gweights/s", "cores": ncores, "kind": "oracle",
+                             "sample": f"the {oinfo.rows}x{oinfo.cols} layer's stream per step, decoded by the C oracle "
+                                       f"on {ncores} threads, then x W^T in numpy fp32 ({m} tokens)"},
+            "e2e": {"value": round(rate, 4), "unit": "Gweights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
 
 def main():
     a = args_()
@@ -763,14 +1015,16 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if a.impl == "reference":
-        (run_reference_tile_ans if is_tile_ans(a) else run_reference)(a, rank, world)
+        (run_reference_tile_ans if is_tile_ans(a) else run_reference_linear if is_linear(a) else run_reference)(
+            a, rank, world)
         return
     if world > 1:
         import datetime
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        (run_ours_tile_ans if is_tile_ans(a) else run_ours)(a, rank, world, local_rank)
+        (run_ours_tile_ans if is_tile_ans(a) else run_ours_linear if is_linear(a) else run_ours)(
+            a, rank, world, local_rank)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -29,6 +29,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <type_traits>
 #include <mutex>
 
 #include "../../include/eptile.h"
@@ -420,12 +421,16 @@ __device__ __forceinline__ uint32_t resolve_pair(const Params &p, uint32_t h, ui
 // ------------------------------------------------------------------ the blocks of one tile
 // Lane l decodes blocks t*32K + 32k + l, k = 0..K-1.  ACT: the last tile, where lanes run out
 // of blocks.  ROWS: the launch's RowLayout.  Returns EP_DEC_* bits.
-// TO_SMEM (BF16 GEMM-ordered tiles only): the blocks go to the 128 x 64 BF16 operand tile at the
-// shared address `btile` in the 128-byte-swizzled K-major layout the tensor cores read (row r's
-// 16-byte chunk j at (r / 8) 1024 + (r mod 8) 128 + 16 (j xor r mod 8)), not to global memory.
-template <int DT, bool SMEM, bool ACT, int ROWS, int MODE, typename Lim, bool TO_SMEM = false>
+// Sink (BF16 GEMM-ordered tiles only; NoSink otherwise): the blocks go to shared-memory operand
+// tiles of the fused GEMM instead of global memory.  sink.begin(k) runs before step k (it may
+// wait for a buffer; false gives up), sink.put(k, lane, pk) stores the step's 8 weights and
+// sink.end(k, lane) runs after the store.
+struct NoSink {};
+
+template <int DT, bool SMEM, bool ACT, int ROWS, int MODE, typename Lim, typename Sink = NoSink>
 __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L, uint32_t &rb, uint32_t lut,
-                                                  Lim wlim, uint32_t t, uint32_t lane, uint32_t btile = 0) {
+                                                  Lim wlim, uint32_t t, uint32_t lane, Sink *sink = nullptr) {
+    constexpr bool TO_SMEM = !std::is_same<Sink, NoSink>::value;
     constexpr bool WIDE = MODE == kWide;
     constexpr bool R32 = ROWS == kRows32, RAG = ROWS == kRowsPadded, GEMM = ROWS == kRowsGemm;
     uint32_t b = t * 32u * p.K + lane;
@@ -464,6 +469,12 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
             }
             bool act = !ACT || b < p.nb;
             if (ACT && !__any_sync(0xffffffffu, act)) goto done;
+            if constexpr (TO_SMEM) {
+                if (!sink->begin(k)) {
+                    err |= EP_DEC_TIMEOUT;
+                    goto done;
+                }
+            }
             // a damaged stream may drive a lane's reads ahead (at most one word per token); stop
             // before they leave the buffer's slack
             if ((k & 7u) == 0 && __any_sync(0xffffffffu, L.past(wlim))) {
@@ -555,8 +566,8 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
                 if (act) pk.store_n(p.out, uint64_t(row) * p.cols + c0, uint32_t(min(p.cols - c0, uint64_t(8))));
             } else if constexpr (TO_SMEM) {
                 static_assert(DT == EP_BF16 && ROWS == kRowsGemm, "operand tiles are BF16 GEMM tiles");
-                const uint32_t r = 32u * (k & 3u) + lane, ch = k >> 2;
-                pk.store_shared(btile + (r >> 3) * 1024u + (r & 7u) * 128u + ((ch ^ (r & 7u)) << 4));
+                sink->put(k, lane, pk);
+                sink->end(k, lane);
             } else if (act) {
                 pk.store(p.out, b);
             }
@@ -588,9 +599,10 @@ done:
 
 // Decodes tile t with one warp.  `head` points at the tile (states, region lengths, word area):
 // a shared address (SMEM) or a global pointer.  Returns the EP_DEC_* bits of this lane.
-template <int DT, int ROWS, int MODE, bool SMEM, typename Ptr, bool TO_SMEM = false>
+template <int DT, int ROWS, int MODE, bool SMEM, typename Ptr, typename Sink = NoSink>
 __device__ __forceinline__ uint32_t decode_tile(const Params &p, uint32_t lut, Ptr head, uint32_t tile_bytes,
-                                                uint32_t t, uint32_t lane, uint32_t btile = 0) {
+                                                uint32_t t, uint32_t lane, Sink *sink = nullptr) {
+    constexpr bool TO_SMEM = !std::is_same<Sink, NoSink>::value;
     Lane<SMEM> L;
     uint32_t len;
     if constexpr (SMEM) {
@@ -619,7 +631,7 @@ __device__ __forceinline__ uint32_t decode_tile(const Params &p, uint32_t lut, P
         L.w = lds16(L.wp);
         uint32_t wlim = L.area + 2u * capacity;
         if (TO_SMEM || uint64_t(t + 1) * 32u * p.K <= p.nb)
-            err = decode_blocks<DT, SMEM, false, ROWS, MODE, uint32_t, TO_SMEM>(p, L, rb, lut, wlim, t, lane, btile);
+            err = decode_blocks<DT, SMEM, false, ROWS, MODE, uint32_t, Sink>(p, L, rb, lut, wlim, t, lane, sink);
         else
             err = decode_blocks<DT, SMEM, true, ROWS, MODE>(p, L, rb, lut, wlim, t, lane);
     } else {
@@ -875,84 +887,104 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_
 }
 
 // ------------------------------------------------------------------ the decode fused into a GEMM
-// Y = X W^T for a weight W (N x K) held as a GEMM-ordered stream (EP_LAYOUT_GEMM): each stream tile
-// is one 128 x 64 operand tile of W.  One CTA per (band of 128 output features, range of K tiles);
-// warps 0 .. S-1 each own a pipeline stage: they bulk-copy a stream tile into shared memory, decode
-// its 1024 blocks straight into the stage's B tile (BF16, 128-byte swizzled, K-major), copy the
-// matching 128 x 64 slice of X into the stage's A tile and arrive on the stage's `full` barrier;
-// warp S allocates the tensor memory, waits for each stage in K order, issues four
-// tcgen05.mma (M = 128 tokens, N = 128 features, K = 16 each) accumulating in TMEM and commits them
-// to the stage's `empty` barrier; after the last stage warps 0..3 read the 128 x 128 fp32
-// accumulator out of TMEM (tcgen05.ld) into the CTA's slice of the fp32 partial sums.
-constexpr int kLinMaxStages = 4;
-constexpr uint32_t kLinOpBytes = 128u * 64u * 2u;  // one 128 x 64 BF16 operand tile
-constexpr uint32_t kLinTmemCols = 128;             // the 128 x 128 fp32 accumulator
+// Y^T = W X^T for a weight W (N x K) held as a GEMM-ordered stream (EP_LAYOUT_GEMM): each stream tile
+// is one 128 x 64 tile of W.  One CTA per (band of 128 output features, range of K tiles); warps
+// 0 .. S-1 decode, one tile at a time each: a bulk copy of the stream tile into the warp's buffer,
+// the matching slice of X (tokens padded to a multiple of 16) into the warp's X buffer, then the
+// tile's 32 steps.  Every 8 steps complete a 128 x 16 K-slice of the tile, which goes to one of the
+// warp's two 4 KB slice buffers (a ring) and is announced on that buffer's `full` barrier.  Warp S
+// issues the tensor-core work: for each round of tiles, slice by slice, warp by warp (a fixed
+// order, so the fp32 sums are the same on every call), one tcgen05.mma (M = 128 features,
+// N = tokens, K = 16, A = the W slice, B = the X slice, both K-major) accumulating in tensor
+// memory, committed to the slice buffer's `empty` barrier.  After the last MMA, warps 0..3 read
+// the 128 x N fp32 accumulator out of tensor memory into the CTA's slice of the partial sums.
+constexpr uint32_t kLinMaxWarps = 15;       // decoding warps per CTA
+constexpr uint32_t kLinSlice = 128u * 16u * 2u;  // one 128 x 16 BF16 K-slice of a W tile
+constexpr uint32_t kLinBarBytes = 40;       // per decoding warp: full[2], empty[2], copy
 
 struct LinParams {
     Params dp;                 // the stream (tiles, tables, row factors, status)
     const uint16_t *x;         // activations, BF16, M x cols row-major
     float *part;               // fp32 partial sums, splits x M x N
     uint32_t M, N;             // tokens, output features (rows of W)
+    uint32_t npad;             // tokens padded to a multiple of 16 (the MMA's N)
+    uint32_t idesc;            // the MMA's instruction descriptor
+    uint32_t tmem_cols;        // tensor-memory columns of the accumulator (a power of 2, >= 32)
     uint32_t KT;               // K tiles per band (cols / 64)
     uint32_t kt_per_split;
-    uint32_t stages;           // decoding warps = pipeline stages (<= kLinMaxStages)
-    uint32_t tile_buf;         // bytes of a stream-tile staging buffer
-    uint32_t off_bars, off_tile, off_ab;  // shared-memory layout (offsets from the dynamic base)
+    uint32_t S;                // decoding warps
+    uint32_t tile_buf;         // bytes of a stream-tile buffer
+    uint32_t off_bars, off_tile, off_w, off_x;  // shared-memory layout (offsets from the dynamic base)
 };
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-// UMMA shared-memory descriptor of a K-major, 128-byte-swizzled operand at shared address a: start
-// address and stride between 8-row groups (1024 bytes) in 16-byte units, descriptor version 1,
-// layout type 2 (128-byte swizzle); the leading offset is unused by swizzled K-major layouts (1)
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t a) {
-    return uint64_t((a >> 4) & 0x3fffu) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) | (uint64_t(1) << 46) |
-           (uint64_t(2) << 61);
+// UMMA shared-memory descriptor of a K-major operand without swizzle at shared address a: 8 x 16-byte
+// core matrices, `lbo` bytes apart along K and `sbo` bytes apart along M / N (both in 16-byte
+// units), descriptor version 1, layout type 0
+__device__ __forceinline__ uint64_t umma_desc_plain(uint32_t a, uint32_t lbo, uint32_t sbo) {
+    return uint64_t((a >> 4) & 0x3fffu) | (uint64_t((lbo >> 4) & 0x3fffu) << 16) |
+           (uint64_t((sbo >> 4) & 0x3fffu) << 32) | (uint64_t(1) << 46);
 }
 
-// instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator, BF16 A and B, both K-major,
-// N = 128 (bits 17..22: N / 8), M = 128 (bits 24..28: M / 16)
-constexpr uint32_t kLinIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+// where a decoding warp's steps go: step k writes rows 32 (k mod 4) + lane, columns 8 (k / 4) .. + 7
+// of the tile, i.e. K-slice k / 8, which lives in ring buffer (k / 8) mod 2; inside a slice, row r's
+// 16-byte chunk c (columns 8c .. 8c + 7 of the slice) sits at (r / 8) 256 + 128 c + 16 (r mod 8)
+struct SliceSink {
+    uint32_t ring;   // shared address of the warp's two slice buffers
+    uint32_t full;   // full[0]; full[1] = full + 8, empty[j] = full + 16 + 8 j
+    uint32_t round;  // the warp's tile number: slice j of this tile is the warp's use 4 round + j
+    __device__ __forceinline__ bool begin(uint32_t k) const {
+        // slices 2 and 3 reuse the buffers of slices 0 and 1: wait for their MMAs (use u - 2); the
+        // buffers of slices 0 and 1 were freed before the tile started
+        if ((k & 7u) != 0 || k < 16u) return true;
+        const uint32_t u = 4u * round + (k >> 3);
+        return mbar_wait(full + 16u + 8u * (u & 1u), ((u - 2u) >> 1) & 1u);
+    }
+    __device__ __forceinline__ void put(uint32_t k, uint32_t lane, Packer<EP_BF16> &pk) const {
+        const uint32_t r = 32u * (k & 3u) + lane, c = (k >> 2) & 1u;
+        pk.store_shared(ring + ((k >> 3) & 1u) * kLinSlice + (r >> 3) * 256u + c * 128u + (r & 7u) * 16u);
+    }
+    __device__ __forceinline__ void end(uint32_t k, uint32_t lane) const {
+        if ((k & 7u) != 7u) return;
+        // the slice, written through the generic proxy, becomes visible to the tensor cores
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(full + 8u * ((k >> 3) & 1u));
+    }
+};
 
 template <int MODE>
-__global__ void __launch_bounds__((kLinMaxStages + 1) * 32, 1) linear_kernel(const __grid_constant__ LinParams P) {
-    extern __shared__ __align__(128) uint8_t smem[];  // operand tiles are aligned to 1024 bytes below
+__global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(const __grid_constant__ LinParams P) {
+    extern __shared__ __align__(128) uint8_t smem[];
     const Params &p = P.dp;
     constexpr uint32_t kTables = uint32_t(MODE == kPaired ? kPairedTableBytes : kLutBytes);
-    const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5, S = P.stages;
+    const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5, S = P.S;
     const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
     const uint32_t lut = base;
-    const uint32_t bars = base + P.off_bars;  // full[4], empty[4], copy[4], tables, done; then the TMEM slot
-    auto full = [&](uint32_t s) { return bars + 8u * s; };
-    auto empty = [&](uint32_t s) { return bars + 32u + 8u * s; };
-    auto copyb = [&](uint32_t s) { return bars + 64u + 8u * s; };
-    const uint32_t tbar = bars + 96u, done = bars + 104u, tmem_slot = bars + 112u;
-    // operand tiles: 1024-byte aligned in the shared window
-    const uint32_t ab = (base + P.off_ab + 1023u) & ~1023u;
-    auto atile = [&](uint32_t s) { return ab + 2u * kLinOpBytes * s; };
-    auto btile = [&](uint32_t s) { return ab + 2u * kLinOpBytes * s + kLinOpBytes; };
-    auto tbuf = [&](uint32_t s) { return base + P.off_tile + P.tile_buf * s; };
+    auto wbar = [&](uint32_t w) { return base + P.off_bars + kLinBarBytes * w; };  // full[2], empty[2], copy
+    const uint32_t tbar = base + P.off_bars + kLinBarBytes * S, done = tbar + 8u, tmem_slot = tbar + 16u;
+    auto ring = [&](uint32_t w) { return base + P.off_w + 2u * kLinSlice * w; };
+    auto xbuf = [&](uint32_t w) { return base + P.off_x + P.npad * 128u * w; };
+    auto tbuf = [&](uint32_t w) { return base + P.off_tile + P.tile_buf * w; };
     const uint32_t band = blockIdx.x;
     const uint32_t kt0 = blockIdx.y * P.kt_per_split;
-    const uint32_t nkt = min(P.KT, kt0 + P.kt_per_split) - kt0;
+    const uint32_t nkt = min(P.KT, kt0 + P.kt_per_split) - kt0;  // >= 1: the plan leaves no split empty
 
     if (threadIdx.x == 0) {
-        for (uint32_t s = 0; s < S; ++s) {
-            mbar_init(full(s), 1);
-            mbar_init(empty(s), 1);
-            mbar_init(copyb(s), 1);
-        }
+        for (uint32_t w = 0; w < S; ++w)
+            for (uint32_t i = 0; i < 5; ++i) mbar_init(wbar(w) + 8u * i, 1);
         mbar_init(tbar, 1);
         mbar_init(done, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async();
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (warp == S) {  // the tensor memory of the accumulator (the whole warp allocates)
+    if (warp == S) {  // the accumulator's tensor memory (the whole warp allocates)
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tmem_slot),
-                     "r"(kLinTmemCols) : "memory");
+                     "r"(P.tmem_cols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (threadIdx.x == 0) {
@@ -967,11 +999,14 @@ __global__ void __launch_bounds__((kLinMaxStages + 1) * 32, 1) linear_kernel(con
     uint32_t err = ok ? 0u : uint32_t(EP_DEC_TIMEOUT);
 
     if (warp < S) {
-        // ---- producers: stream tile -> B stage (decoded), X slice -> A stage
-        uint32_t use = 0;
-        for (uint32_t j = warp; j < nkt && ok; j += S, ++use) {
+        // ---- decoding warps: tiles j = warp, warp + S, ... of the CTA's K range
+        SliceSink sink{ring(warp), wbar(warp), 0u};
+        const uint32_t copyb = wbar(warp) + 32u;
+        for (uint32_t j = warp; j < nkt && ok; j += S, ++sink.round) {
             const uint32_t kt = kt0 + j, t = band * P.KT + kt;
-            if (use > 0 && !mbar_wait(empty(warp), (use - 1) & 1u)) {  // the MMAs of the stage's last use
+            // the MMAs of the previous tile (its last slice, use 4 round - 1, and so all before it)
+            // are done: the X buffer and both slice buffers are free
+            if (sink.round > 0 && !mbar_wait(wbar(warp) + 24u, 1u)) {
                 err |= EP_DEC_TIMEOUT;
                 break;
             }
@@ -982,87 +1017,84 @@ __global__ void __launch_bounds__((kLinMaxStages + 1) * 32, 1) linear_kernel(con
             }
             if (lane == 0) {
                 fence_proxy_async();
-                mbar_expect(copyb(warp), bytes);
-                bulk_g2s(tbuf(warp), p.tiles + size_t(beg) * 16, bytes, copyb(warp));
+                mbar_expect(copyb, bytes);
+                bulk_g2s(tbuf(warp), p.tiles + size_t(beg) * 16, bytes, copyb);
             }
-            // X rows m < M, columns 64 kt .. +63: 8 lanes per row, 16 bytes each; rows >= M zero
-            const uint32_t a = atile(warp), c = lane & 7u;
-            for (uint32_t m = lane >> 3; m < 128u; m += 4u) {
+            // X rows n < npad, columns 64 kt .. + 63 (zero for n >= M): 8 lanes per row, 16 bytes
+            // each; row n's chunk c at (n / 8) 1024 + 128 c + 16 (n mod 8)
+            const uint32_t xb = xbuf(warp), c = lane & 7u;
+            for (uint32_t n = lane >> 3; n < P.npad; n += 4u) {
                 uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (m < P.M) v = __ldg(reinterpret_cast<const uint4 *>(P.x + size_t(m) * p.cols + 64u * kt) + c);
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a + (m >> 3) * 1024u + (m & 7u) * 128u +
-                                                                              ((c ^ (m & 7u)) << 4)),
+                if (n < P.M) v = __ldg(reinterpret_cast<const uint4 *>(P.x + size_t(n) * p.cols + 64u * kt) + c);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(xb + (n >> 3) * 1024u + c * 128u +
+                                                                              (n & 7u) * 16u),
                              "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                              : "memory");
             }
-            if (!mbar_wait(copyb(warp), use & 1u)) {
+            if (!mbar_wait(copyb, sink.round & 1u)) {
                 err |= EP_DEC_TIMEOUT;
                 break;
             }
-            err |= decode_tile<EP_BF16, kRowsGemm, MODE, true, uint32_t, true>(p, lut, tbuf(warp), bytes, t, lane,
-                                                                              btile(warp));
-            // the operand tiles, written through the generic proxy, become visible to the tensor cores
-            fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(full(warp));
+            const uint32_t e = decode_tile<EP_BF16, kRowsGemm, MODE, true, uint32_t, SliceSink>(
+                p, lut, tbuf(warp), bytes, t, lane, &sink);
+            err |= e;
+            if (__any_sync(0xffffffffu, e != 0)) break;  // the tile's slices may be missing: stop here
         }
     } else if (warp == S) {
-        // ---- the MMA issuer: stages in K order, four K = 16 steps each
-        for (uint32_t j = 0; j < nkt; ++j) {
-            const uint32_t s = j % S;
-            if (!mbar_wait(full(s), (j / S) & 1u)) {
-                err |= EP_DEC_TIMEOUT;
-                break;
-            }
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            if (lane == 0) {
-#pragma unroll
-                for (uint32_t ks = 0; ks < 4; ++ks) {
-                    const uint64_t da = umma_desc_sw128(atile(s) + 32u * ks), db = umma_desc_sw128(btile(s) + 32u * ks);
-                    const uint32_t acc = (j | ks) ? 1u : 0u;
-                    asm volatile(
-                        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
-                        "l"(da), "l"(db), "r"(kLinIdesc), "r"(acc)
-                        : "memory");
+        // ---- the MMA issuer: round by round, slice by slice, warp by warp
+        const uint32_t rounds = (nkt + S - 1) / S;
+        bool first = true;
+        for (uint32_t r = 0; r < rounds && ok; ++r)
+            for (uint32_t sl = 0; sl < 4u && ok; ++sl)
+                for (uint32_t w = 0; w < S && r * S + w < nkt; ++w) {
+                    const uint32_t u = 4u * r + sl, fb = wbar(w) + 8u * (u & 1u);
+                    if (!mbar_wait(fb, (u >> 1) & 1u)) {
+                        err |= EP_DEC_TIMEOUT;
+                        ok = false;
+                        break;
+                    }
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    if (lane == 0) {
+                        const uint64_t da = umma_desc_plain(ring(w) + (u & 1u) * kLinSlice, 128u, 256u);
+                        const uint64_t db = umma_desc_plain(xbuf(w) + 256u * sl, 128u, 1024u);
+                        const uint32_t acc = first ? 0u : 1u;
+                        asm volatile(
+                            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+                            "l"(da), "l"(db), "r"(P.idesc), "r"(acc)
+                            : "memory");
+                        asm volatile(
+                            "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                                fb + 16u)
+                            : "memory");
+                    }
+                    first = false;
+                    __syncwarp();
                 }
-                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                                 empty(s))
-                             : "memory");
-            }
-            __syncwarp();
-        }
         if (lane == 0)
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(done)
                          : "memory");
         __syncwarp();
     }
-    // ---- epilogue: warps 0..3 read TMEM lanes 32 w .. 32 w + 31 (tokens), 128 fp32 columns each
+    // ---- epilogue: warp q < 4 reads tensor-memory lanes 32 q .. 32 q + 31 (features), one column per
+    // token, and writes each token's 32 features (128 contiguous bytes) of the partial sums
     if (warp < 4) {
         if (!mbar_wait(done, 0)) err |= EP_DEC_TIMEOUT;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t m = 32u * warp + lane;
-        float *dst = P.part + (size_t(blockIdx.y) * P.M + m) * P.N + 128u * band;
-#pragma unroll
-        for (uint32_t c0 = 0; c0 < 128u; c0 += 32u) {
-            uint32_t r[32];
+        float *dst = P.part + size_t(blockIdx.y) * P.M * P.N + 128u * band + 32u * warp + lane;
+        for (uint32_t c0 = 0; c0 < P.npad; c0 += 16u) {
+            uint32_t r[16];
             asm volatile(
-                "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-                "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+                "%14, %15}, [%16];"
                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-                  "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-                  "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-                  "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                  "=r"(r[15])
                 : "r"(tmem + ((32u * warp) << 16) + c0));
             asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-            if (m < P.M) {
 #pragma unroll
-                for (uint32_t q = 0; q < 32u; q += 4u)
-                    *reinterpret_cast<float4 *>(dst + c0 + q) =
-                        make_float4(__uint_as_float(r[q]), __uint_as_float(r[q + 1]), __uint_as_float(r[q + 2]),
-                                    __uint_as_float(r[q + 3]));
-            }
+            for (uint32_t i = 0; i < 16u; ++i)
+                if (c0 + i < P.M) dst[size_t(c0 + i) * P.N] = __uint_as_float(r[i]);
         }
     }
     if (err && p.status && lane == 0) atomicOr(p.status, err);
@@ -1071,7 +1103,7 @@ __global__ void __launch_bounds__((kLinMaxStages + 1) * 32, 1) linear_kernel(con
     __syncthreads();
     if (warp == S) {
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kLinTmemCols)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(P.tmem_cols)
                      : "memory");
     }
 }
@@ -1253,28 +1285,42 @@ Params params_of(const ep_info *info, const void *d_blob, const void *d_tables, 
 }
 
 // ---- the fused GEMM's launch plan: bands of 128 output features, K tiles split across CTAs so that
-// about one CTA runs per SM; shared memory = tables, barriers, the stages' stream-tile buffers and
-// their A and B operand tiles
+// all CTAs run in one wave (one per SM); shared memory = tables, barriers, then per decoding warp a
+// stream-tile buffer, two W slice buffers and an X buffer.  Decoding warps: as many as fit, then as
+// few as give the same number of rounds of tiles.
 struct LinPlan {
-    uint32_t nbands, KT, splits, kt_per_split, stages, tile_buf, off_bars, off_tile, off_ab;
+    uint32_t nbands, KT, splits, kt_per_split, S, npad, tmem_cols, tile_buf, off_bars, off_tile, off_w, off_x;
     size_t smem;
 };
 
-LinPlan lin_plan(const ep_info *info, int sms) {
+LinPlan lin_plan(const ep_info *info, int sms, int64_t m) {
     LinPlan L{};
-    const bool paired = info->paired != 0;
     L.nbands = uint32_t(info->rows / 128);
     L.KT = uint32_t(info->cols / 64);
-    uint32_t want = L.nbands ? (uint32_t(sms) + L.nbands - 1) / L.nbands : 1u;
-    want = want < 1 ? 1u : (want > L.KT ? L.KT : want);
-    L.kt_per_split = (L.KT + want - 1) / want;
+    uint32_t splits_max = L.nbands < uint32_t(sms) ? uint32_t(sms) / L.nbands : 1u;
+    splits_max = std::max(1u, std::min(splits_max, L.KT));
+    L.kt_per_split = (L.KT + splits_max - 1) / splits_max;
     L.splits = (L.KT + L.kt_per_split - 1) / L.kt_per_split;
-    L.stages = paired ? 3u : 4u;
+    L.npad = uint32_t((m + 15) / 16 * 16);
     L.tile_buf = uint32_t((info->max_tile_nbytes + kSlack + 15) & ~uint64_t(15));
-    L.off_bars = uint32_t(paired ? kPairedTableBytes : kLutBytes);
-    L.off_tile = L.off_bars + 128u;
-    L.off_ab = L.off_tile + L.stages * L.tile_buf;
-    L.smem = size_t(L.off_ab) + 1024u + size_t(L.stages) * 2u * kLinOpBytes;
+    const uint32_t tables = uint32_t(info->paired ? kPairedTableBytes : kLutBytes);
+    auto layout = [&](uint32_t S) {
+        L.S = S;
+        L.off_bars = tables;
+        L.off_tile = (L.off_bars + kLinBarBytes * S + 24u + 15u) & ~15u;
+        L.off_w = (L.off_tile + S * L.tile_buf + 127u) & ~127u;
+        L.off_x = L.off_w + S * 2u * kLinSlice;
+        L.smem = size_t(L.off_x) + size_t(S) * L.npad * 128u;
+    };
+    uint32_t S = std::min(kLinMaxWarps, L.kt_per_split);
+    for (layout(S); S > 1 && L.smem > kSmemLimit; layout(--S)) {
+    }
+    const uint32_t rounds = (L.kt_per_split + S - 1) / S;
+    layout((L.kt_per_split + rounds - 1) / rounds);
+    L.tmem_cols = 32;
+    while (L.tmem_cols < L.npad) L.tmem_cols *= 2;
+    // more than half an SM's shared memory: one CTA per SM, so no CTA waits for another's tensor memory
+    L.smem = std::max(L.smem, kSmemLimit / 2 + 1024);
     return L;
 }
 
@@ -1369,7 +1415,7 @@ extern "C" size_t ep_linear_fused_workspace(const ep_info *info, int64_t m) {
     if (!linear_ok(info, m)) return 0;
     int device, sms;
     if (device_sms(&device, &sms) != EP_OK) return 0;
-    const LinPlan L = lin_plan(info, sms);
+    const LinPlan L = lin_plan(info, sms, m);
     return size_t(L.splits) * size_t(m) * size_t(info->rows) * sizeof(float);
 }
 
@@ -1384,22 +1430,28 @@ extern "C" int ep_linear_fused(const ep_info *info, const void *d_blob, const vo
     if (reinterpret_cast<uintptr_t>(d_y) & 1u || reinterpret_cast<uintptr_t>(d_bias) & 1u) return EP_ERR_INVALID_ARG;
     int device, sms;
     if (device_sms(&device, &sms) != EP_OK) return EP_ERR_CUDA;
-    const LinPlan L = lin_plan(info, sms);
+    const LinPlan L = lin_plan(info, sms, m);
     if (work_nbytes < size_t(L.splits) * size_t(m) * size_t(info->rows) * sizeof(float)) return EP_ERR_INVALID_ARG;
-    if (L.smem > kSmemLimit) return EP_ERR_UNSUPPORTED;  // tiles too large for the stages beside the tables
+    if (L.smem > kSmemLimit) return EP_ERR_UNSUPPORTED;  // tiles too large for one warp's buffers beside the tables
     LinParams P;
     P.dp = params_of(info, d_blob, d_tables, nullptr, d_status);
     P.x = static_cast<const uint16_t *>(d_x);
     P.part = static_cast<float *>(d_work);
     P.M = uint32_t(m);
     P.N = uint32_t(info->rows);
+    P.npad = L.npad;
+    // the MMA: fp32 accumulator, BF16 A and B, both K-major, N = npad (bits 17..22: N / 8),
+    // M = 128 (bits 24..28: M / 16)
+    P.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((L.npad >> 3) << 17) | ((128u >> 4) << 24);
+    P.tmem_cols = L.tmem_cols;
     P.KT = L.KT;
     P.kt_per_split = L.kt_per_split;
-    P.stages = L.stages;
+    P.S = L.S;
     P.tile_buf = L.tile_buf;
     P.off_bars = L.off_bars;
     P.off_tile = L.off_tile;
-    P.off_ab = L.off_ab;
+    P.off_w = L.off_w;
+    P.off_x = L.off_x;
     const bool paired = info->paired != 0;
     auto kern = paired ? linear_kernel<kPaired> : (wide_fields(info) ? linear_kernel<kWide> : linear_kernel<kNarrow>);
     {
@@ -1418,7 +1470,7 @@ extern "C" int ep_linear_fused(const ep_info *info, const void *d_blob, const vo
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(L.nbands, L.splits);
-    cfg.blockDim = dim3((L.stages + 1) * 32);
+    cfg.blockDim = dim3(std::max(L.S + 1, 4u) * 32);  // the epilogue needs warps 0..3
     cfg.dynamicSmemBytes = L.smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];

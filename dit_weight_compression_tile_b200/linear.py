@@ -5,7 +5,9 @@ call.  The reconstruction is the fused decode kernel (ep_decompress) into a buff
 keeps; the product is the library GEMM (cuBLAS through torch: F.linear, torch._scaled_mm for
 FP8, torch._int_mm for INT8).  A BF16 layer whose stream is GEMM-ordered (LatticeRANSConfig(layout=
 "gemm")) instead decodes inside its own tcgen05 GEMM (ep_linear_fused) when the call has at most
-128 tokens: the weight then never passes through memory in BF16.
+FUSED_MAX_TOKENS tokens: the weight then never passes through memory in BF16.  Above that the decode
+into a buffer plus the library GEMM is faster (the fused kernel's decoding warps share each SM with
+the operand buffers and go no faster with more tokens, while its X slices grow).
 
 The FP8 / INT8 layers hold per-row absmax codes (the stream's code container) and quantize the
 activations per row of x the same way (E4M3 with scale amax / 448, INT8 with amax / 127, RNE);
@@ -19,6 +21,9 @@ import torch.nn.functional as F
 
 from . import binding as B
 from .compressed import CompressedTensor, LatticeRANSConfig, _tables, compress, decompress
+
+FUSED_MAX_TOKENS = 16
+
 
 class CompressedLinear(nn.Module):
     """y = x W^T + b with W held compressed (lossy lattice-rANS, `config`) and decoded per call.
@@ -99,14 +104,14 @@ class CompressedLinear(nn.Module):
 
     def fused_for(self, x):
         """whether forward(x) decodes inside the fused GEMM (ep_linear_fused): a GEMM-ordered BF16
-        stream on x's CUDA device, x BF16 with 1..128 tokens"""
+        stream on x's CUDA device, x BF16 with 1..FUSED_MAX_TOKENS tokens"""
         w = self._weight
         if w is None or w.compress_method != "lattice_rans" or not x.is_cuda or x.dtype != torch.bfloat16:
             return False
         info = w.info
         tokens = x.numel() // self.in_features if x.dim() else 0
         return (info.layout == B.LAYOUT_GEMM and info.container_dtype == B.BF16 and w.device == x.device
-                and 1 <= tokens <= 128)
+                and 1 <= tokens <= FUSED_MAX_TOKENS)
 
     def forward(self, x):
         if self.fused_for(x):
@@ -115,7 +120,8 @@ class CompressedLinear(nn.Module):
             tables = _tables(w, s)
             bias = None if self.bias is None else self.bias.to(torch.bfloat16)
             if self._work is None or self._work.device != x.device:
-                self._work = torch.empty(B.linear_fused_workspace(w.info, 128), dtype=torch.uint8, device=x.device)
+                self._work = torch.empty(B.linear_fused_workspace(w.info, FUSED_MAX_TOKENS), dtype=torch.uint8,
+                                         device=x.device)
             y = B.linear_fused(x.reshape(-1, self.in_features), w.blob, w.info, tables, bias=bias, work=self._work,
                                stream=s)
             return y.reshape(*x.shape[:-1], self.out_features)

@@ -30,7 +30,8 @@ def test_both_arms_state_the_same_config():
         c1, c2 = bench.bench_config(a, 1), bench.bench_config(a, 1)
         assert c1 == c2 and c1["workload"] == name and c1["parallelism"] == "single"
         assert bench.bench_config(a, 4)["parallelism"] == "replicas"
-        assert set(c1) == {"workload", "shape", "target_bpp", "distribution", "container", "l2", "parallelism"}
+        keys = {"workload", "shape", "target_bpp", "distribution", "container", "l2", "parallelism"}
+        assert set(c1) == (keys | {"tokens"} if bench.WORKLOADS[name].get("scheme") == "linear_fused" else keys)
 
 
 def test_l2_policy():
@@ -43,6 +44,12 @@ def test_l2_policy():
         assert bench.l2_policy(_args(name))[0] == 1
     rot, _ = bench.l2_policy(_args("int8_codes_8192x8192"))
     assert rot * 8192 * 8192 * (3.0 / 8 + 1) >= 2 * bench.L2_BYTES
+    # the fused GEMM writes no weight: its copies hold the streams alone (4 bpp of the block's 113 M
+    # weights), five of them to exceed twice the L2
+    rot, text = bench.l2_policy(_args("linear_fused_dit_block_16tok_bf16"))
+    nominal = 3072 * (9216 + 3072 + 12288 + 12288) * 0.5
+    assert rot * nominal >= 2 * bench.L2_BYTES and (rot - 1) * nominal < 2 * bench.L2_BYTES
+    assert "rotating stream copies" in text
     # the DiT set lists 112 tensors of the four block shapes
     dims = bench.WORKLOADS["dit_28blocks_hidden3072_bf16"]["dims"]
     assert len(dims) == 112 and sum(r * c for r, c in dims) == 28 * 3072 * (9216 + 3072 + 12288 + 12288)

@@ -62,7 +62,12 @@ def reference(oracle, blob, x, bias):
                                                       ((256, 512), 16, B.CODING_SINGLE, True),
                                                       ((384, 1024), 64, B.CODING_PAIRED, True),
                                                       ((128, 3072), 128, B.CODING_AUTO, False),
-                                                      ((1024, 3072), 7, B.CODING_PAIRED, True)])
+                                                      ((1024, 3072), 7, B.CODING_PAIRED, True),
+                                                      # DiT shapes: 8 and 10 decoding warps per CTA, 3 and 5
+                                                      # rounds of tiles; the largest token count paired
+                                                      ((3072, 9216), 16, B.CODING_AUTO, True),
+                                                      ((12288, 3072), 3, B.CODING_SINGLE, False),
+                                                      ((3072, 3072), 128, B.CODING_PAIRED, True)])
 def test_fused_equals_gemm_on_decoded_weight(oracle, shape, m, coding, with_bias):
     w, blob, info = gemm_stream(shape, coding=coding, seed=shape[1] + m)
     g = torch.Generator().manual_seed(m)
@@ -99,19 +104,20 @@ def test_layer_takes_the_fused_path_only_where_it_applies():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("tokens", [(1,), (4, 7), (128,), (3, 50)])
+@pytest.mark.parametrize("tokens", [(1,), (2, 8), (4, 7), (3, 50)])
 def test_layer_forward(oracle, tokens):
     from dit_weight_compression_tile_b200 import CompressedLinear, LatticeRANSConfig
+    from dit_weight_compression_tile_b200.linear import FUSED_MAX_TOKENS
     torch.manual_seed(3)
     lin = torch.nn.Linear(1024, 384, dtype=torch.bfloat16)
     layer = CompressedLinear.from_linear(lin, config=LatticeRANSConfig(4.0, layout="gemm")).cuda()
     x = (torch.randn(*tokens, 1024) * 0.5).to(torch.bfloat16)
     y = layer(x.cuda())
     m = x.numel() // 1024
-    assert layer.fused_for(x.cuda()) == (m <= 128)
+    assert layer.fused_for(x.cuda()) == (m <= FUSED_MAX_TOKENS)
     blob = layer.weight.blob.cpu()
     ref, tol = reference(oracle, blob, x.reshape(-1, 1024), layer.bias.detach().cpu())
     got = y.float().cpu().reshape(-1, 384)
     assert y.shape == (*tokens, 384)
-    # above 128 tokens the layer decodes and calls the library GEMM: summed in another order, same bound
+    # above FUSED_MAX_TOKENS the layer decodes and calls the library GEMM: summed in another order, same bound
     assert torch.all((got - ref).abs() <= tol), float((got - ref).abs().max())
