@@ -420,7 +420,9 @@ def linear_fused_workspace(info, m):
 def linear_fused(x, d_blob, info, tables, bias=None, out=None, work=None, status=None, stream=None):
     """Y = X W^T (+ bias) with W decoded inside the tcgen05 GEMM (ep_linear_fused).  ``x``: CUDA
     BF16 (m, K) with 1 <= m <= 128; ``d_blob``: a GEMM-ordered (LAYOUT_GEMM) BF16 stream on the
-    device; ``tables``: from ``prepare``.  Returns the BF16 (m, N) output."""
+    device; ``tables``: from ``prepare``; ``work``: scratch of linear_fused_workspace bytes,
+    zero-filled before its first use (the call leaves it reusable; a new one is zero-allocated
+    when absent or too small).  Returns the BF16 (m, N) output."""
     if not (x.is_cuda and d_blob.is_cuda and tables.is_cuda):
         raise EpError(-1, "linear_fused works on CUDA tensors")
     if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != info.cols:
@@ -432,7 +434,7 @@ def linear_fused(x, d_blob, info, tables, bias=None, out=None, work=None, status
     if need == 0:
         raise EpError(-1, "ep_linear_fused takes a GEMM-ordered BF16 stream and 1 <= m <= 128")
     if work is None or work.numel() * work.element_size() < need:
-        work = torch.empty(need, dtype=torch.uint8, device=x.device)
+        work = torch.zeros(need, dtype=torch.uint8, device=x.device)
     elif not (work.is_cuda and work.is_contiguous()):
         raise EpError(-1, "work must be a contiguous CUDA tensor")
     if out is None:

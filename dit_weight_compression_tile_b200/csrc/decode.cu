@@ -897,7 +897,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) decode_kernel(const __grid_
 // order, so the fp32 sums are the same on every call), one tcgen05.mma (M = 128 features,
 // N = tokens, K = 16, A = the W slice, B = the X slice, both K-major) accumulating in tensor
 // memory, committed to the slice buffer's `empty` barrier.  After the last MMA, warps 0..3 read
-// the 128 x N fp32 accumulator out of tensor memory into the CTA's slice of the partial sums.
+// the 128 x N fp32 accumulator out of tensor memory into the CTA's slice of the partial sums; the
+// band's last CTA to finish adds the splits' partial sums in split order (the same sums on every
+// call), adds the bias, rounds once to BF16 and writes Y.
 constexpr uint32_t kLinMaxWarps = 15;       // decoding warps per CTA
 constexpr uint32_t kLinSlice = 128u * 16u * 2u;  // one 128 x 16 BF16 K-slice of a W tile
 constexpr uint32_t kLinBarBytes = 40;       // per decoding warp: full[2], empty[2], copy
@@ -906,6 +908,10 @@ struct LinParams {
     Params dp;                 // the stream (tiles, tables, row factors, status)
     const uint16_t *x;         // activations, BF16, M x cols row-major
     float *part;               // fp32 partial sums, splits x M x N
+    uint32_t *count;           // per band: CTAs done (zero between calls)
+    const uint16_t *bias;      // nullable, BF16, N
+    uint16_t *y;               // BF16, M x N
+    uint32_t splits;
     uint32_t M, N;             // tokens, output features (rows of W)
     uint32_t npad;             // tokens padded to a multiple of 16 (the MMA's N)
     uint32_t idesc;            // the MMA's instruction descriptor
@@ -1099,6 +1105,8 @@ __global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(cons
     }
     if (err && p.status && lane == 0) atomicOr(p.status, err);
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // the partial sums are visible device-wide before this CTA counts itself done
+    __threadfence();
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     if (warp == S) {
@@ -1106,20 +1114,50 @@ __global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(cons
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(P.tmem_cols)
                      : "memory");
     }
-}
-
-// Y (BF16, M x N) = the sum of the splits' fp32 partial sums, plus the bias (BF16, nullable), rounded
-// once to nearest even
-__global__ void linear_reduce_kernel(const float *part, uint32_t splits, uint32_t M, uint32_t N, const uint16_t *bias,
-                                     uint16_t *y) {
-    const size_t n = size_t(M) * N;
-    for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += size_t(gridDim.x) * blockDim.x) {
-        float acc = 0.0f;
-        for (uint32_t s = 0; s < splits; ++s) acc += part[s * n + i];
-        if (bias) acc += __uint_as_float(uint32_t(bias[i % N]) << 16);
-        const __nv_bfloat16 h = __float2bfloat16_rn(acc);
-        y[i] = *reinterpret_cast<const uint16_t *>(&h);
+    // ---- the band's last CTA: Y = the splits' partial sums in split order, plus the bias
+    if (threadIdx.x == 0) {
+        const uint32_t ticket = atomicAdd(P.count + band, 1u);
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(tmem_slot), "r"(ticket == P.splits - 1u ? 1u : 0u) : "memory");
     }
+    __syncthreads();
+    if (lds32(tmem_slot) == 0u) return;
+    __threadfence();
+    // four features per thread and step; the loads of up to eight splits are issued before their
+    // additions, which stay in split order
+    const size_t MN4 = size_t(P.M) * P.N / 4u;
+    for (uint32_t i = threadIdx.x; i < P.M * 32u; i += blockDim.x) {
+        const uint32_t m = i >> 5, n = 128u * band + 4u * (i & 31u);
+        const float4 *src = reinterpret_cast<const float4 *>(P.part + size_t(m) * P.N + n);
+        float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+        for (uint32_t s0 = 0; s0 < P.splits; s0 += 8u) {
+            float4 v[8];
+#pragma unroll
+            for (uint32_t j = 0; j < 8u; ++j)
+                if (s0 + j < P.splits) v[j] = __ldcg(src + (s0 + j) * MN4);
+#pragma unroll
+            for (uint32_t j = 0; j < 8u; ++j)
+                if (s0 + j < P.splits) {
+                    a0 += v[j].x;
+                    a1 += v[j].y;
+                    a2 += v[j].z;
+                    a3 += v[j].w;
+                }
+        }
+        if (P.bias) {
+            a0 += __uint_as_float(uint32_t(P.bias[n]) << 16);
+            a1 += __uint_as_float(uint32_t(P.bias[n + 1]) << 16);
+            a2 += __uint_as_float(uint32_t(P.bias[n + 2]) << 16);
+            a3 += __uint_as_float(uint32_t(P.bias[n + 3]) << 16);
+        }
+        uint16_t *dst = P.y + size_t(m) * P.N + n;
+        const float a[4] = {a0, a1, a2, a3};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __nv_bfloat16 h = __float2bfloat16_rn(a[j]);
+            dst[j] = *reinterpret_cast<const uint16_t *>(&h);
+        }
+    }
+    if (threadIdx.x == 0) P.count[band] = 0u;  // ready for the next call
 }
 
 // ------------------------------------------------------------------ host side
@@ -1324,6 +1362,12 @@ LinPlan lin_plan(const ep_info *info, int sms, int64_t m) {
     return L;
 }
 
+// the caller's scratch: the fp32 partial sums (splits x m x N), then one counter per band
+size_t lin_count_offset(const LinPlan &L, int64_t m) {
+    return (size_t(L.splits) * size_t(m) * size_t(L.nbands) * 128u * sizeof(float) + 15u) & ~size_t(15);
+}
+size_t lin_work_bytes(const LinPlan &L, int64_t m) { return lin_count_offset(L, m) + size_t(L.nbands) * 4u; }
+
 }  // namespace
 }  // namespace ep
 
@@ -1416,7 +1460,7 @@ extern "C" size_t ep_linear_fused_workspace(const ep_info *info, int64_t m) {
     int device, sms;
     if (device_sms(&device, &sms) != EP_OK) return 0;
     const LinPlan L = lin_plan(info, sms, m);
-    return size_t(L.splits) * size_t(m) * size_t(info->rows) * sizeof(float);
+    return lin_work_bytes(L, m);
 }
 
 extern "C" int ep_linear_fused(const ep_info *info, const void *d_blob, const void *d_tables, const void *d_x,
@@ -1431,12 +1475,16 @@ extern "C" int ep_linear_fused(const ep_info *info, const void *d_blob, const vo
     int device, sms;
     if (device_sms(&device, &sms) != EP_OK) return EP_ERR_CUDA;
     const LinPlan L = lin_plan(info, sms, m);
-    if (work_nbytes < size_t(L.splits) * size_t(m) * size_t(info->rows) * sizeof(float)) return EP_ERR_INVALID_ARG;
+    if (work_nbytes < lin_work_bytes(L, m)) return EP_ERR_INVALID_ARG;
     if (L.smem > kSmemLimit) return EP_ERR_UNSUPPORTED;  // tiles too large for one warp's buffers beside the tables
     LinParams P;
     P.dp = params_of(info, d_blob, d_tables, nullptr, d_status);
     P.x = static_cast<const uint16_t *>(d_x);
     P.part = static_cast<float *>(d_work);
+    P.count = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(d_work) + lin_count_offset(L, m));
+    P.bias = static_cast<const uint16_t *>(d_bias);
+    P.y = static_cast<uint16_t *>(d_y);
+    P.splits = L.splits;
     P.M = uint32_t(m);
     P.N = uint32_t(info->rows);
     P.npad = L.npad;
@@ -1478,12 +1526,7 @@ extern "C" int ep_linear_fused(const ep_info *info, const void *d_blob, const vo
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, P) != cudaSuccess) return EP_ERR_CUDA;
-    const size_t n = size_t(m) * info->rows;
-    const unsigned rgrid = unsigned(std::min<size_t>((n + 255) / 256, size_t(sms) * 8));
-    linear_reduce_kernel<<<rgrid, 256, 0, s>>>(P.part, L.splits, P.M, P.N, static_cast<const uint16_t *>(d_bias),
-                                               static_cast<uint16_t *>(d_y));
-    return cudaGetLastError() == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, kern, P) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------ ep_decompress_noalloc

@@ -120,7 +120,7 @@ class CompressedLinear(nn.Module):
             tables = _tables(w, s)
             bias = None if self.bias is None else self.bias.to(torch.bfloat16)
             if self._work is None or self._work.device != x.device:
-                self._work = torch.empty(B.linear_fused_workspace(w.info, FUSED_MAX_TOKENS), dtype=torch.uint8,
+                self._work = torch.zeros(B.linear_fused_workspace(w.info, FUSED_MAX_TOKENS), dtype=torch.uint8,
                                          device=x.device)
             y = B.linear_fused(x.reshape(-1, self.in_features), w.blob, w.info, tables, bias=bias, work=self._work,
                                stream=s)

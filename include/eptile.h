@@ -221,16 +221,18 @@ int ep_decompress(const ep_info *info, const void *d_blob, const void *d_workspa
  *   d_x         BF16 activations, m x K row-major (16-byte aligned), 1 <= m <= 128.
  *   d_bias      nullable BF16 bias of N elements.
  *   d_y         BF16 output, m x N row-major: the fp32 sum rounded once to nearest even.
- *   d_work      caller-owned device scratch of ep_linear_fused_workspace(info, m) bytes (fp32
- *               partial sums of the K splits), 16-byte aligned.
+ *   d_work      caller-owned device scratch of ep_linear_fused_workspace(info, m) bytes, 16-byte
+ *               aligned: the fp32 partial sums of the K splits and one counter per band of 128
+ *               output features.  It must be zero-filled before its first use; every call leaves
+ *               the counters at zero again.  One call at a time per scratch buffer.
  *   d_status    nullable device uint32: EP_DEC_* bits of stream damage.
- * One launch of the fused kernel (a CTA per band of 128 output features and range of K tiles:
- * warps bulk-copy stream tiles into shared memory and decode them straight into 128-byte-swizzled
- * BF16 operand tiles beside the matching slices of X; one warp issues tcgen05.mma into a
- * 128 x 128 fp32 accumulator in tensor memory; the accumulator leaves through tcgen05.ld) and
- * one small launch that adds the splits and the bias.  Asynchronous; allocates nothing.
- * EP_ERR_INVALID_ARG for another layout, container or m out of range, EP_ERR_UNSUPPORTED when a
- * tile is too large for the pipeline's shared memory. */
+ * One launch: a CTA per band of 128 output features and range of K tiles.  Its warps bulk-copy
+ * stream tiles into shared memory and decode them straight into BF16 operand slices (128 features
+ * x 16 inputs) beside the matching slices of X; one warp issues tcgen05.mma (M = 128 features,
+ * N = m padded to 16) into an fp32 accumulator in tensor memory, read out with tcgen05.ld into the
+ * partial sums; the band's last CTA adds the splits in order and the bias.  Asynchronous;
+ * allocates nothing.  EP_ERR_INVALID_ARG for another layout, container or m out of range,
+ * EP_ERR_UNSUPPORTED when a tile is too large for the shared memory of one decoding warp. */
 size_t ep_linear_fused_workspace(const ep_info *info, int64_t m);
 int ep_linear_fused(const ep_info *info, const void *d_blob, const void *d_tables, const void *d_x, int64_t m,
                     const void *d_bias, void *d_y, void *d_work, size_t work_nbytes, uint32_t *d_status,

@@ -76,7 +76,9 @@ def test_fused_equals_gemm_on_decoded_weight(oracle, shape, m, coding, with_bias
     d = blob.cuda()
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     tables = B.prepare(d, info, status=status)
-    y = B.linear_fused(x.cuda(), d, info, tables, bias=bias.cuda() if bias is not None else None, status=status)
+    work = torch.zeros(B.linear_fused_workspace(info, m), dtype=torch.uint8, device="cuda")
+    y = B.linear_fused(x.cuda(), d, info, tables, bias=bias.cuda() if bias is not None else None, work=work,
+                       status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     ref, tol = reference(oracle, blob, x, bias)
@@ -84,9 +86,12 @@ def test_fused_equals_gemm_on_decoded_weight(oracle, shape, m, coding, with_bias
     assert got.shape == ref.shape
     bad = (got - ref).abs() > tol
     assert not bad.any(), (float((got - ref).abs().max()), int(bad.sum()))
-    # a second call on the same tables gives the same bits
-    y2 = B.linear_fused(x.cuda(), d, info, tables, bias=bias.cuda() if bias is not None else None)
+    # a second call on the same tables and scratch gives the same bits (the band counters in the
+    # scratch are back at zero after every call)
+    y2 = B.linear_fused(x.cuda(), d, info, tables, bias=bias.cuda() if bias is not None else None, work=work)
     assert torch.equal(y2, y)
+    nb = info.rows // 128
+    assert int(work[-4 * nb:].view(torch.int32).abs().sum()) == 0
 
 
 def test_layer_takes_the_fused_path_only_where_it_applies():
