@@ -887,6 +887,28 @@ def run_ours_linear(a, rank, world, local_rank):
     assert int(status.item()) == 0
     unfused_ms, _ = timed(unfused, a.steps)
     dense_ms, _ = timed(dense, a.steps)
+    # each layer alone, the same three ways (fewer steps: context, not the metric)
+    per_layer = {}
+    n_layer = max(a.warmup + 1, min(a.steps, 100))
+    for L in layers:
+        one = [L]
+
+        def f1(r, one=one):
+            for L_ in one:
+                B.linear_fused(L_["x"], L_["blobs"][r], L_["info"], L_["tables"], out=L_["y"], work=L_["work"],
+                               status=status, stream=stream)
+
+        def u1(r, one=one):
+            for L_ in one:
+                F.linear(L_["x"], B.decompress(L_["rblobs"][r], L_["rinfo"], workspace=L_["rtables"],
+                                               out=L_["wbuf"], stream=stream))
+
+        def d1(r, one=one):
+            for L_ in one:
+                F.linear(L_["x"], L_["w"])
+
+        per_layer[f'{L["info"].rows}x{L["info"].cols}'] = [round(1e3 * timed(fn, n_layer)[0] / n_layer, 2)
+                                                          for fn in (f1, u1, d1)]
     nweights = sum(L["info"].rows * L["info"].cols for L in layers)
     stream_bytes = sum(L["info"].storage_nbytes for L in layers)
     act_bytes = sum(2 * m * (L["info"].cols + L["info"].rows) for L in layers)
@@ -924,7 +946,8 @@ def run_ours_linear(a, rank, world, local_rank):
                    "layout": "gemm"},
         "step_us": {"fused": round(1e3 * fused_ms / a.steps, 2),
                     "decode_row_stream_then_library_gemm": round(1e3 * unfused_ms / a.steps, 2),
-                    "library_gemm_bf16_weights": round(1e3 * dense_ms / a.steps, 2)},
+                    "library_gemm_bf16_weights": round(1e3 * dense_ms / a.steps, 2),
+                    "per_layer_fused_unfused_bf16": per_layer},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic_for_kernel("linear_kernel", traffic_key(a)),
                      "peak_kind": peak_kind, "algorithmic_bytes_per_step": stream_bytes + act_bytes,

@@ -80,7 +80,7 @@ __device__ __forceinline__ void store_element(const Params &p, uint64_t i, uint3
 }
 
 // the raw bytes of whole chunk c (8 for 16-bit types, 24 for FP32; none for 8-bit types), loaded
-// before the chunk's symbols are decoded so that the load's latency hides behind the rANS chain
+// two chunks ahead of their use so that the load's latency hides behind the rANS chain
 template <int ESZ>
 struct RawChunk {
     uint2 r[ESZ == 1 ? 1 : ESZ - 1];
@@ -155,6 +155,11 @@ __device__ __forceinline__ uint32_t decode_tile(const Params &p, uint32_t lut, u
     const uint32_t wlim = area + 2u * capacity;
     uint32_t err = 0;
     uint64_t c = uint64_t(t) * 32u * p.K + lane;
+    // the raw bytes of the lane's chunk at step k + j, j = 0, 1 (zero past the lane's chunks)
+    auto raw_at = [&](uint32_t k, uint64_t ck) {
+        return k < p.K && ck < p.nc ? load_raw<ESZ>(p, ck, 8 * ck + 8 <= p.n) : RawChunk<ESZ>{};
+    };
+    RawChunk<ESZ> R0 = raw_at(0, c), R1 = raw_at(1, c + 32u);
     for (uint32_t k = 0; k < p.K; ++k, c += 32u) {
         const bool act = c < p.nc;
         if (!__any_sync(0xffffffffu, act)) break;
@@ -164,13 +169,15 @@ __device__ __forceinline__ uint32_t decode_tile(const Params &p, uint32_t lut, u
             err |= EP_DEC_WORD_OVERRUN;
             break;
         }
+        const RawChunk<ESZ> R2 = raw_at(k + 2, c + 64u);
         if (act) {
-            const RawChunk<ESZ> R = load_raw<ESZ>(p, c, 8 * c + 8 <= p.n);
             uint32_t e[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) e[j] = ans_step(x, wp, w, lut);
-            store_chunk<ESZ>(p, c, e, R);
+            store_chunk<ESZ>(p, c, e, R0);
         }
+        R0 = R1;
+        R1 = R2;
     }
     if (err) return err;
     if (x != kStateLow) err |= EP_DEC_BAD_END;
