@@ -412,15 +412,15 @@ def ans_decompress(d_blob, info, workspace=None, out=None, status=None, stream=N
 
 # ---------------------------------------------------------------- the decode fused into a GEMM
 def linear_fused_workspace(info, m):
-    """bytes of the fp32 partial sums ep_linear_fused needs for m tokens (0: the stream or m is not
-    one it takes)"""
+    """bytes of scratch ep_linear_fused needs for m tokens (0: the stream or m is not one it takes)"""
     return int(lib().ep_linear_fused_workspace(C.byref(info), m))
 
 
 def linear_fused(x, d_blob, info, tables, bias=None, out=None, work=None, status=None, stream=None):
     """Y = X W^T (+ bias) with W decoded inside the tcgen05 GEMM (ep_linear_fused).  ``x``: CUDA
-    BF16 (m, K) with 1 <= m <= 128; ``d_blob``: a GEMM-ordered (LAYOUT_GEMM) BF16 stream on the
-    device; ``tables``: from ``prepare``; ``work``: scratch of linear_fused_workspace bytes,
+    BF16 (m, K) with 1 <= m <= 128; ``d_blob``: a GEMM-ordered (LAYOUT_GEMM) BF16, INT8 or FP8
+    stream on the device (INT8 / FP8: the activations are quantized per token and the codes
+    multiplied); ``tables``: from ``prepare``; ``work``: scratch of linear_fused_workspace bytes,
     zero-filled before its first use (the call leaves it reusable; a new one is zero-allocated
     when absent or too small).  Returns the BF16 (m, N) output."""
     if not (x.is_cuda and d_blob.is_cuda and tables.is_cuda):
@@ -432,7 +432,7 @@ def linear_fused(x, d_blob, info, tables, bias=None, out=None, work=None, status
     L = lib()
     need = linear_fused_workspace(info, m)
     if need == 0:
-        raise EpError(-1, "ep_linear_fused takes a GEMM-ordered BF16 stream and 1 <= m <= 128")
+        raise EpError(-1, "ep_linear_fused takes a GEMM-ordered BF16 / INT8 / FP8 stream and 1 <= m <= 128")
     if work is None or work.numel() * work.element_size() < need:
         work = torch.zeros(need, dtype=torch.uint8, device=x.device)
     elif not (work.is_cuda and work.is_contiguous()):

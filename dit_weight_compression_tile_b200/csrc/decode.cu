@@ -209,10 +209,16 @@ struct Packer<EP_INT8> {
         b[i] = uint32_t(r);
         b[i + 1] = uint32_t(r >> 32);
     }
-    __device__ __forceinline__ void store(void *out, uint32_t blk) {
+    __device__ __forceinline__ uint2 packed() const {
         uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
         uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
-        reinterpret_cast<uint2 *>(out)[blk] = make_uint2(lo, hi);
+        return make_uint2(lo, hi);
+    }
+    __device__ __forceinline__ void store(void *out, uint32_t blk) { reinterpret_cast<uint2 *>(out)[blk] = packed(); }
+    // the 8 codes as 8 bytes at a shared-memory address (an operand slice of the fused GEMM)
+    __device__ __forceinline__ void store_shared(uint32_t a) {
+        const uint2 v = packed();
+        asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(v.x), "r"(v.y) : "memory");
     }
     __device__ __forceinline__ void store_n(void *out, uint64_t e, uint32_t n) {
         for (uint32_t i = 0; i < n; ++i) reinterpret_cast<uint8_t *>(out)[e + i] = uint8_t(b[i]);
@@ -236,6 +242,9 @@ struct Packer<EP_FP8_E4M3> {
     }
     __device__ __forceinline__ void store(void *out, uint32_t b) {
         reinterpret_cast<uint2 *>(out)[b] = make_uint2(o[0], o[1]);
+    }
+    __device__ __forceinline__ void store_shared(uint32_t a) {
+        asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(o[0]), "r"(o[1]) : "memory");
     }
     __device__ __forceinline__ void store_n(void *out, uint64_t e, uint32_t n) {
         for (uint32_t i = 0; i < n; ++i) reinterpret_cast<uint8_t *>(out)[e + i] = uint8_t(o[i >> 2] >> (8 * (i & 3)));
@@ -421,8 +430,8 @@ __device__ __forceinline__ uint32_t resolve_pair(const Params &p, uint32_t h, ui
 // ------------------------------------------------------------------ the blocks of one tile
 // Lane l decodes blocks t*32K + 32k + l, k = 0..K-1.  ACT: the last tile, where lanes run out
 // of blocks.  ROWS: the launch's RowLayout.  Returns EP_DEC_* bits.
-// Sink (BF16 GEMM-ordered tiles only; NoSink otherwise): the blocks go to shared-memory operand
-// tiles of the fused GEMM instead of global memory.  sink.begin(k) runs before step k (it may
+// Sink (GEMM-ordered BF16 / INT8 / FP8 tiles only; NoSink otherwise): the blocks go to shared-memory
+// operand slices of the fused GEMM instead of global memory.  sink.begin(k) runs before step k (it may
 // wait for a buffer; false gives up), sink.put(k, lane, pk) stores the step's 8 weights and
 // sink.end(k, lane) runs after the store.
 struct NoSink {};
@@ -565,7 +574,8 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
                 const uint64_t c0 = 8ull * col;
                 if (act) pk.store_n(p.out, uint64_t(row) * p.cols + c0, uint32_t(min(p.cols - c0, uint64_t(8))));
             } else if constexpr (TO_SMEM) {
-                static_assert(DT == EP_BF16 && ROWS == kRowsGemm, "operand tiles are BF16 GEMM tiles");
+                static_assert((DT == EP_BF16 || DT == EP_INT8 || DT == EP_FP8_E4M3) && ROWS == kRowsGemm,
+                              "operand slices come from GEMM-ordered BF16 / INT8 / FP8 tiles");
                 sink->put(k, lane, pk);
                 sink->end(k, lane);
             } else if (act) {
@@ -912,6 +922,9 @@ struct LinParams {
     const uint16_t *bias;      // nullable, BF16, N
     uint16_t *y;               // BF16, M x N
     uint32_t splits;
+    const uint8_t *xq;         // code containers: the activations' 8-bit codes, M x cols
+    const float *xscale;       // code containers: the activations' per-token scales
+    const float *wscale;       // code containers: the weight's per-row scales (from the stream)
     uint32_t M, N;             // tokens, output features (rows of W)
     uint32_t npad;             // tokens padded to a multiple of 16 (the MMA's N)
     uint32_t idesc;            // the MMA's instruction descriptor
@@ -935,36 +948,56 @@ __device__ __forceinline__ uint64_t umma_desc_plain(uint32_t a, uint32_t lbo, ui
            (uint64_t((sbo >> 4) & 0x3fffu) << 32) | (uint64_t(1) << 46);
 }
 
-// where a decoding warp's steps go: step k writes rows 32 (k mod 4) + lane, columns 8 (k / 4) .. + 7
-// of the tile, i.e. K-slice k / 8, which lives in ring buffer (k / 8) mod 2; inside a slice, row r's
-// 16-byte chunk c (columns 8c .. 8c + 7 of the slice) sits at (r / 8) 256 + 128 c + 16 (r mod 8)
+// where a decoding warp's steps go.  A K-slice is 128 rows x 32 bytes of the tile (16 BF16 weights or
+// 32 8-bit codes: the K extent of one MMA), stored as no-swizzle K-major core matrices: row r's
+// 16-byte chunk c at (r / 8) 256 + 128 c + 16 (r mod 8).  Step k writes 8 weights of row
+// 32 (k mod 4) + lane at column block k / 4, so BF16 tiles complete a slice every 8 steps (4 slices
+// per tile), 8-bit tiles every 16 (2 slices); slice j of the warp's round-th tile is its use
+// U round + j (U slices per tile) and lives in ring buffer j mod 2.
+template <int DT>
 struct SliceSink {
+    static constexpr uint32_t kSteps = DT == EP_BF16 ? 8u : 16u;  // steps per slice
+    static constexpr uint32_t kUses = 32u / kSteps;                // slices per tile
     uint32_t ring;   // shared address of the warp's two slice buffers
     uint32_t full;   // full[0]; full[1] = full + 8, empty[j] = full + 16 + 8 j
-    uint32_t round;  // the warp's tile number: slice j of this tile is the warp's use 4 round + j
+    uint32_t round;  // the warp's tile number
     __device__ __forceinline__ bool begin(uint32_t k) const {
-        // slices 2 and 3 reuse the buffers of slices 0 and 1: wait for their MMAs (use u - 2); the
-        // buffers of slices 0 and 1 were freed before the tile started
-        if ((k & 7u) != 0 || k < 16u) return true;
-        const uint32_t u = 4u * round + (k >> 3);
+        // BF16 slices 2 and 3 reuse the buffers of slices 0 and 1: wait for their MMAs (use u - 2);
+        // the buffers of a tile's first two slices were freed before the tile started
+        if (k % kSteps != 0 || k < 2u * kSteps) return true;
+        const uint32_t u = kUses * round + k / kSteps;
         return mbar_wait(full + 16u + 8u * (u & 1u), ((u - 2u) >> 1) & 1u);
     }
-    __device__ __forceinline__ void put(uint32_t k, uint32_t lane, Packer<EP_BF16> &pk) const {
-        const uint32_t r = 32u * (k & 3u) + lane, c = (k >> 2) & 1u;
-        pk.store_shared(ring + ((k >> 3) & 1u) * kLinSlice + (r >> 3) * 256u + c * 128u + (r & 7u) * 16u);
+    __device__ __forceinline__ void put(uint32_t k, uint32_t lane, Packer<DT> &pk) const {
+        const uint32_t r = 32u * (k & 3u) + lane, slot = (k / kSteps) & 1u;
+        uint32_t off;
+        if constexpr (DT == EP_BF16)
+            off = ((k >> 2) & 1u) * 128u;  // 16 bytes per step: chunk (k / 4) mod 2
+        else
+            off = ((k >> 3) & 1u) * 128u + ((k >> 2) & 1u) * 8u;  // 8 bytes per step
+        pk.store_shared(ring + slot * kLinSlice + (r >> 3) * 256u + (r & 7u) * 16u + off);
     }
     __device__ __forceinline__ void end(uint32_t k, uint32_t lane) const {
-        if ((k & 7u) != 7u) return;
+        if (k % kSteps != kSteps - 1u) return;
         // the slice, written through the generic proxy, becomes visible to the tensor cores
         fence_proxy_async();
         __syncwarp();
-        if (lane == 0) mbar_arrive(full + 8u * ((k >> 3) & 1u));
+        if (lane == 0) mbar_arrive(full + 8u * ((k / kSteps) & 1u));
     }
 };
 
-template <int MODE>
+// the X operand: BF16 (K = 16 per MMA) or the 8-bit codes of the quantized activations (K = 32);
+// either way 32 bytes of a row per MMA, row n's 16-byte chunk c of a K tile at
+// (n / 8) 8 XB + 128 c + 16 (n mod 8), XB the row's bytes per K tile
+template <int DT>
+struct XOperand {
+    static constexpr uint32_t kRowBytes = DT == EP_BF16 ? 128u : 64u;  // one K tile (64 inputs) of a row
+};
+
+template <int DT, int MODE>
 __global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(const __grid_constant__ LinParams P) {
     extern __shared__ __align__(128) uint8_t smem[];
+    constexpr uint32_t XB = XOperand<DT>::kRowBytes;
     const Params &p = P.dp;
     constexpr uint32_t kTables = uint32_t(MODE == kPaired ? kPairedTableBytes : kLutBytes);
     const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5, S = P.S;
@@ -973,7 +1006,7 @@ __global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(cons
     auto wbar = [&](uint32_t w) { return base + P.off_bars + kLinBarBytes * w; };  // full[2], empty[2], copy
     const uint32_t tbar = base + P.off_bars + kLinBarBytes * S, done = tbar + 8u, tmem_slot = tbar + 16u;
     auto ring = [&](uint32_t w) { return base + P.off_w + 2u * kLinSlice * w; };
-    auto xbuf = [&](uint32_t w) { return base + P.off_x + P.npad * 128u * w; };
+    auto xbuf = [&](uint32_t w) { return base + P.off_x + P.npad * XB * w; };
     auto tbuf = [&](uint32_t w) { return base + P.off_tile + P.tile_buf * w; };
     const uint32_t band = blockIdx.x;
     const uint32_t kt0 = blockIdx.y * P.kt_per_split;
@@ -1006,13 +1039,13 @@ __global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(cons
 
     if (warp < S) {
         // ---- decoding warps: tiles j = warp, warp + S, ... of the CTA's K range
-        SliceSink sink{ring(warp), wbar(warp), 0u};
+        SliceSink<DT> sink{ring(warp), wbar(warp), 0u};
         const uint32_t copyb = wbar(warp) + 32u;
         for (uint32_t j = warp; j < nkt && ok; j += S, ++sink.round) {
             const uint32_t kt = kt0 + j, t = band * P.KT + kt;
-            // the MMAs of the previous tile (its last slice, use 4 round - 1, and so all before it)
-            // are done: the X buffer and both slice buffers are free
-            if (sink.round > 0 && !mbar_wait(wbar(warp) + 24u, 1u)) {
+            // the MMAs of the previous tile (its last slice, use U round - 1, in ring buffer 1, and
+            // so all before it) are done: the X buffer and both slice buffers are free
+            if (sink.round > 0 && !mbar_wait(wbar(warp) + 24u, ((SliceSink<DT>::kUses * sink.round - 1u) >> 1) & 1u)) {
                 err |= EP_DEC_TIMEOUT;
                 break;
             }
@@ -1026,13 +1059,16 @@ __global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(cons
                 mbar_expect(copyb, bytes);
                 bulk_g2s(tbuf(warp), p.tiles + size_t(beg) * 16, bytes, copyb);
             }
-            // X rows n < npad, columns 64 kt .. + 63 (zero for n >= M): 8 lanes per row, 16 bytes
-            // each; row n's chunk c at (n / 8) 1024 + 128 c + 16 (n mod 8)
-            const uint32_t xb = xbuf(warp), c = lane & 7u;
-            for (uint32_t n = lane >> 3; n < P.npad; n += 4u) {
+            // X rows n < npad, inputs 64 kt .. + 63 (zero for n >= M): XB / 16 lanes per row, 16 bytes
+            // each (BF16 activations, or their 8-bit codes quantized by the launch before this one)
+            constexpr uint32_t kLanesPerRow = XB / 16u;
+            const uint32_t xb = xbuf(warp), c = lane % kLanesPerRow;
+            const uint8_t *xrow = DT == EP_BF16 ? reinterpret_cast<const uint8_t *>(P.x) + 128u * kt : P.xq + 64u * kt;
+            const size_t xstride = DT == EP_BF16 ? 2u * p.cols : p.cols;
+            for (uint32_t n = lane / kLanesPerRow; n < P.npad; n += 32u / kLanesPerRow) {
                 uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (n < P.M) v = __ldg(reinterpret_cast<const uint4 *>(P.x + size_t(n) * p.cols + 64u * kt) + c);
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(xb + (n >> 3) * 1024u + c * 128u +
+                if (n < P.M) v = __ldg(reinterpret_cast<const uint4 *>(xrow + size_t(n) * xstride) + c);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(xb + (n >> 3) * 8u * XB + c * 128u +
                                                                               (n & 7u) * 16u),
                              "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                              : "memory");
@@ -1041,19 +1077,20 @@ __global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(cons
                 err |= EP_DEC_TIMEOUT;
                 break;
             }
-            const uint32_t e = decode_tile<EP_BF16, kRowsGemm, MODE, true, uint32_t, SliceSink>(
+            const uint32_t e = decode_tile<DT, kRowsGemm, MODE, true, uint32_t, SliceSink<DT>>(
                 p, lut, tbuf(warp), bytes, t, lane, &sink);
             err |= e;
             if (__any_sync(0xffffffffu, e != 0)) break;  // the tile's slices may be missing: stop here
         }
     } else if (warp == S) {
         // ---- the MMA issuer: round by round, slice by slice, warp by warp
+        constexpr uint32_t U = SliceSink<DT>::kUses;
         const uint32_t rounds = (nkt + S - 1) / S;
         bool first = true;
         for (uint32_t r = 0; r < rounds && ok; ++r)
-            for (uint32_t sl = 0; sl < 4u && ok; ++sl)
+            for (uint32_t sl = 0; sl < U && ok; ++sl)
                 for (uint32_t w = 0; w < S && r * S + w < nkt; ++w) {
-                    const uint32_t u = 4u * r + sl, fb = wbar(w) + 8u * (u & 1u);
+                    const uint32_t u = U * r + sl, fb = wbar(w) + 8u * (u & 1u);
                     if (!mbar_wait(fb, (u >> 1) & 1u)) {
                         err |= EP_DEC_TIMEOUT;
                         ok = false;
@@ -1062,13 +1099,26 @@ __global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(cons
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                     if (lane == 0) {
                         const uint64_t da = umma_desc_plain(ring(w) + (u & 1u) * kLinSlice, 128u, 256u);
-                        const uint64_t db = umma_desc_plain(xbuf(w) + 256u * sl, 128u, 1024u);
+                        const uint64_t db = umma_desc_plain(xbuf(w) + 256u * sl, 128u, 8u * XB);
                         const uint32_t acc = first ? 0u : 1u;
-                        asm volatile(
-                            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
-                            "l"(da), "l"(db), "r"(P.idesc), "r"(acc)
-                            : "memory");
+                        if constexpr (DT == EP_BF16)
+                            asm volatile(
+                                "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                                "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+                                "l"(da), "l"(db), "r"(P.idesc), "r"(acc)
+                                : "memory");
+                        else if constexpr (DT == EP_INT8)
+                            asm volatile(
+                                "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                                "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+                                "l"(da), "l"(db), "r"(P.idesc), "r"(acc)
+                                : "memory");
+                        else
+                            asm volatile(
+                                "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                                "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+                                "l"(da), "l"(db), "r"(P.idesc), "r"(acc)
+                                : "memory");
                         asm volatile(
                             "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                                 fb + 16u)
@@ -1099,8 +1149,8 @@ __global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(cons
                 : "r"(tmem + ((32u * warp) << 16) + c0));
             asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-            for (uint32_t i = 0; i < 16u; ++i)
-                if (c0 + i < P.M) dst[size_t(c0 + i) * P.N] = __uint_as_float(r[i]);
+            for (uint32_t i = 0; i < 16u; ++i)  // fp32 sums, or the int32 sums of the INT8 MMA, as bits
+                if (c0 + i < P.M) reinterpret_cast<uint32_t *>(dst)[size_t(c0 + i) * P.N] = r[i];
         }
     }
     if (err && p.status && lane == 0) atomicOr(p.status, err);
@@ -1123,41 +1173,77 @@ __global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(cons
     if (lds32(tmem_slot) == 0u) return;
     __threadfence();
     // four features per thread and step; the loads of up to eight splits are issued before their
-    // additions, which stay in split order
+    // additions, which stay in split order (INT8: exact int32 sums).  BF16: y = RNE(sum + bias).
+    // Codes: y = RNE(fp32(fp32(sum) s_x) s_w), then with a bias RNE(y + bias): the order of the
+    // per-row-quantized layers' own arithmetic
+    using Acc = typename std::conditional<DT == EP_INT8, int32_t, float>::type;
+    using Acc4 = typename std::conditional<DT == EP_INT8, int4, float4>::type;
     const size_t MN4 = size_t(P.M) * P.N / 4u;
     for (uint32_t i = threadIdx.x; i < P.M * 32u; i += blockDim.x) {
         const uint32_t m = i >> 5, n = 128u * band + 4u * (i & 31u);
-        const float4 *src = reinterpret_cast<const float4 *>(P.part + size_t(m) * P.N + n);
-        float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+        const Acc4 *src = reinterpret_cast<const Acc4 *>(P.part + size_t(m) * P.N + n);
+        Acc a[4] = {Acc(0), Acc(0), Acc(0), Acc(0)};
         for (uint32_t s0 = 0; s0 < P.splits; s0 += 8u) {
-            float4 v[8];
+            Acc4 v[8];
 #pragma unroll
             for (uint32_t j = 0; j < 8u; ++j)
                 if (s0 + j < P.splits) v[j] = __ldcg(src + (s0 + j) * MN4);
 #pragma unroll
             for (uint32_t j = 0; j < 8u; ++j)
                 if (s0 + j < P.splits) {
-                    a0 += v[j].x;
-                    a1 += v[j].y;
-                    a2 += v[j].z;
-                    a3 += v[j].w;
+                    a[0] += v[j].x;
+                    a[1] += v[j].y;
+                    a[2] += v[j].z;
+                    a[3] += v[j].w;
                 }
         }
-        if (P.bias) {
-            a0 += __uint_as_float(uint32_t(P.bias[n]) << 16);
-            a1 += __uint_as_float(uint32_t(P.bias[n + 1]) << 16);
-            a2 += __uint_as_float(uint32_t(P.bias[n + 2]) << 16);
-            a3 += __uint_as_float(uint32_t(P.bias[n + 3]) << 16);
-        }
         uint16_t *dst = P.y + size_t(m) * P.N + n;
-        const float a[4] = {a0, a1, a2, a3};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const __nv_bfloat16 h = __float2bfloat16_rn(a[j]);
+            float yv;
+            if constexpr (DT == EP_BF16) {
+                yv = a[j];
+                if (P.bias) yv += __uint_as_float(uint32_t(P.bias[n + j]) << 16);
+            } else {
+                const float f = DT == EP_INT8 ? __int2float_rn(int32_t(a[j])) : float(a[j]);
+                yv = __fmul_rn(__fmul_rn(f, P.xscale[m]), __ldg(P.wscale + n + j));
+                if (P.bias)
+                    yv = __bfloat162float(__float2bfloat16_rn(yv)) + __uint_as_float(uint32_t(P.bias[n + j]) << 16);
+            }
+            const __nv_bfloat16 h = __float2bfloat16_rn(yv);
             dst[j] = *reinterpret_cast<const uint16_t *>(&h);
         }
     }
     if (threadIdx.x == 0) P.count[band] = 0u;  // ready for the next call
+}
+
+// The activations of a per-row-quantized layer: per token, scale = amax / 127 (INT8) or / 448 (FP8
+// E4M3), 1 for an all-zero row; codes = x / scale rounded to nearest even and clamped to [-127, 127]
+// (INT8), or clamped to [-448, 448] and rounded to E4M3 (FP8).  One CTA per token.
+template <int DT>
+__global__ void __launch_bounds__(256) quantize_x_kernel(const uint16_t *x, uint32_t K, uint8_t *xq, float *xscale) {
+    __shared__ float part[8];
+    const uint32_t m = blockIdx.x;
+    const uint16_t *row = x + size_t(m) * K;
+    float amax = 0.0f;
+    for (uint32_t k = threadIdx.x; k < K; k += blockDim.x) amax = fmaxf(amax, fabsf(__uint_as_float(uint32_t(row[k]) << 16)));
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+    if ((threadIdx.x & 31u) == 0) part[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = part[0];
+    for (uint32_t w = 1; w < (blockDim.x >> 5); ++w) amax = fmaxf(amax, part[w]);
+    const float scale = amax > 0.0f ? __fdiv_rn(amax, DT == EP_INT8 ? 127.0f : 448.0f) : 1.0f;
+    if (threadIdx.x == 0) xscale[m] = scale;
+    uint8_t *out = xq + size_t(m) * K;
+    for (uint32_t k = threadIdx.x; k < K; k += blockDim.x) {
+        const float v = __fdiv_rn(__uint_as_float(uint32_t(row[k]) << 16), scale);
+        if constexpr (DT == EP_INT8)
+            out[k] = uint8_t(int8_t(__float2int_rn(fminf(fmaxf(rintf(v), -127.0f), 127.0f))));
+        else
+            out[k] = uint8_t(__nv_cvt_float_to_fp8(fminf(fmaxf(v, -448.0f), 448.0f), __NV_SATFINITE, __NV_E4M3));
+    }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ host side
@@ -1328,6 +1414,8 @@ Params params_of(const ep_info *info, const void *d_blob, const void *d_tables, 
 // few as give the same number of rounds of tiles.
 struct LinPlan {
     uint32_t nbands, KT, splits, kt_per_split, S, npad, tmem_cols, tile_buf, off_bars, off_tile, off_w, off_x;
+    uint32_t xrow;  // bytes of one token's K tile in the X buffer: 128 (BF16) or 64 (8-bit codes)
+    bool codes;     // an INT8 / FP8 container: the activations are quantized per token first
     size_t smem;
 };
 
@@ -1340,6 +1428,8 @@ LinPlan lin_plan(const ep_info *info, int sms, int64_t m) {
     L.kt_per_split = (L.KT + splits_max - 1) / splits_max;
     L.splits = (L.KT + L.kt_per_split - 1) / L.kt_per_split;
     L.npad = uint32_t((m + 15) / 16 * 16);
+    L.codes = info->container_dtype != EP_BF16;
+    L.xrow = L.codes ? 64u : 128u;
     L.tile_buf = uint32_t((info->max_tile_nbytes + kSlack + 15) & ~uint64_t(15));
     const uint32_t tables = uint32_t(info->paired ? kPairedTableBytes : kLutBytes);
     auto layout = [&](uint32_t S) {
@@ -1348,7 +1438,7 @@ LinPlan lin_plan(const ep_info *info, int sms, int64_t m) {
         L.off_tile = (L.off_bars + kLinBarBytes * S + 24u + 15u) & ~15u;
         L.off_w = (L.off_tile + S * L.tile_buf + 127u) & ~127u;
         L.off_x = L.off_w + S * 2u * kLinSlice;
-        L.smem = size_t(L.off_x) + size_t(S) * L.npad * 128u;
+        L.smem = size_t(L.off_x) + size_t(S) * L.npad * L.xrow;
     };
     uint32_t S = std::min(kLinMaxWarps, L.kt_per_split);
     for (layout(S); S > 1 && L.smem > kSmemLimit; layout(--S)) {
@@ -1362,11 +1452,20 @@ LinPlan lin_plan(const ep_info *info, int sms, int64_t m) {
     return L;
 }
 
-// the caller's scratch: the fp32 partial sums (splits x m x N), then one counter per band
+// the caller's scratch: the partial sums (splits x m x N, fp32 or int32), one counter per band, and
+// for code containers the activations' codes (m x K bytes) and per-token scales (m floats)
 size_t lin_count_offset(const LinPlan &L, int64_t m) {
     return (size_t(L.splits) * size_t(m) * size_t(L.nbands) * 128u * sizeof(float) + 15u) & ~size_t(15);
 }
-size_t lin_work_bytes(const LinPlan &L, int64_t m) { return lin_count_offset(L, m) + size_t(L.nbands) * 4u; }
+size_t lin_xq_offset(const LinPlan &L, int64_t m) {
+    return (lin_count_offset(L, m) + size_t(L.nbands) * 4u + 15u) & ~size_t(15);
+}
+size_t lin_xscale_offset(const LinPlan &L, int64_t m) {
+    return (lin_xq_offset(L, m) + size_t(m) * L.KT * 64u + 15u) & ~size_t(15);
+}
+size_t lin_work_bytes(const LinPlan &L, int64_t m) {
+    return L.codes ? lin_xscale_offset(L, m) + size_t(m) * 4u : lin_count_offset(L, m) + size_t(L.nbands) * 4u;
+}
 
 }  // namespace
 }  // namespace ep
@@ -1441,13 +1540,15 @@ int device_sms(int *device, int *sms) {
 }
 
 bool linear_ok(const ep_info *info, int64_t m) {
-    return info && info->layout == 1 && info->container_dtype == EP_BF16 && m >= 1 && m <= 128 &&
-           check_info(info) == EP_OK;
+    return info && info->layout == 1 &&
+           (info->container_dtype == EP_BF16 || info->container_dtype == EP_INT8 ||
+            info->container_dtype == EP_FP8_E4M3) &&
+           m >= 1 && m <= 128 && check_info(info) == EP_OK;
 }
 
 struct LinCache {
     std::mutex mu;
-    size_t smem_set[64][2] = {};
+    size_t smem_set[64][9] = {};  // [device][3 container + coding mode]
 };
 LinCache g_lin;
 
@@ -1488,9 +1589,14 @@ extern "C" int ep_linear_fused(const ep_info *info, const void *d_blob, const vo
     P.M = uint32_t(m);
     P.N = uint32_t(info->rows);
     P.npad = L.npad;
-    // the MMA: fp32 accumulator, BF16 A and B, both K-major, N = npad (bits 17..22: N / 8),
-    // M = 128 (bits 24..28: M / 16)
-    P.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((L.npad >> 3) << 17) | ((128u >> 4) << 24);
+    // the MMA's instruction descriptor: accumulator type (bits 4..5: 1 fp32, 2 int32), A and B types
+    // (bits 7..9, 10..12: BF16 = 1 for kind::f16, signed = 1 for kind::i8, E4M3 = 0 for
+    // kind::f8f6f4), both K-major, N = npad (bits 17..22: N / 8), M = 128 (bits 24..28: M / 16)
+    const int dt = info->container_dtype;
+    const uint32_t types = dt == EP_BF16 ? (1u << 4) | (1u << 7) | (1u << 10)
+                           : dt == EP_INT8 ? (2u << 4) | (1u << 7) | (1u << 10)
+                                           : (1u << 4);
+    P.idesc = types | ((L.npad >> 3) << 17) | ((128u >> 4) << 24);
     P.tmem_cols = L.tmem_cols;
     P.KT = L.KT;
     P.kt_per_split = L.kt_per_split;
@@ -1500,22 +1606,40 @@ extern "C" int ep_linear_fused(const ep_info *info, const void *d_blob, const vo
     P.off_tile = L.off_tile;
     P.off_w = L.off_w;
     P.off_x = L.off_x;
-    const bool paired = info->paired != 0;
-    auto kern = paired ? linear_kernel<kPaired> : (wide_fields(info) ? linear_kernel<kWide> : linear_kernel<kNarrow>);
+    uint8_t *work = static_cast<uint8_t *>(d_work);
+    P.xq = L.codes ? work + lin_xq_offset(L, m) : nullptr;
+    P.xscale = L.codes ? reinterpret_cast<const float *>(work + lin_xscale_offset(L, m)) : nullptr;
+    P.wscale = L.codes ? reinterpret_cast<const float *>(static_cast<const uint8_t *>(d_blob) + info->off_scales)
+                       : nullptr;
+    const int mode = info->paired ? kPaired : (wide_fields(info) ? kWide : kNarrow);
+    using Kern = void (*)(LinParams);
+    // [container: BF16, INT8, FP8][coding mode]
+    static const Kern kerns[3][3] = {
+        {linear_kernel<EP_BF16, kNarrow>, linear_kernel<EP_BF16, kWide>, linear_kernel<EP_BF16, kPaired>},
+        {linear_kernel<EP_INT8, kNarrow>, linear_kernel<EP_INT8, kWide>, linear_kernel<EP_INT8, kPaired>},
+        {linear_kernel<EP_FP8_E4M3, kNarrow>, linear_kernel<EP_FP8_E4M3, kWide>, linear_kernel<EP_FP8_E4M3, kPaired>}};
+    const int ci = dt == EP_BF16 ? 0 : (dt == EP_INT8 ? 1 : 2);
+    const Kern kern = kerns[ci][mode];
     {
         std::lock_guard<std::mutex> g(g_lin.mu);
-        size_t &set = g_lin.smem_set[device][paired ? 1 : 0];
+        size_t &set = g_lin.smem_set[device][3 * ci + mode];
         if (set < L.smem) {
-            // one attribute for the coding modes of a table size
-            decltype(kern) ks[2] = {linear_kernel<kNarrow>, linear_kernel<kWide>};
-            if (paired) ks[0] = ks[1] = linear_kernel<kPaired>;
-            for (auto k : ks)
-                if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(L.smem)) != cudaSuccess)
-                    return EP_ERR_CUDA;
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(L.smem)) != cudaSuccess)
+                return EP_ERR_CUDA;
             set = L.smem;
         }
     }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (L.codes) {  // the activations' codes and scales, into the scratch
+        float *xs = reinterpret_cast<float *>(work + lin_xscale_offset(L, m));
+        uint8_t *xq = work + lin_xq_offset(L, m);
+        const uint16_t *x = static_cast<const uint16_t *>(d_x);
+        if (dt == EP_INT8)
+            quantize_x_kernel<EP_INT8><<<unsigned(m), 256, 0, s>>>(x, uint32_t(info->cols), xq, xs);
+        else
+            quantize_x_kernel<EP_FP8_E4M3><<<unsigned(m), 256, 0, s>>>(x, uint32_t(info->cols), xq, xs);
+        if (cudaGetLastError() != cudaSuccess) return EP_ERR_CUDA;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(L.nbands, L.splits);
     cfg.blockDim = dim3(std::max(L.S + 1, 4u) * 32);  // the epilogue needs warps 0..3

@@ -5,7 +5,8 @@ call.  The reconstruction is the fused decode kernel (ep_decompress) into a buff
 keeps; the product is the library GEMM (cuBLAS through torch: F.linear, torch._scaled_mm for
 FP8, torch._int_mm for INT8).  A BF16 layer whose stream is GEMM-ordered (LatticeRANSConfig(layout=
 "gemm")) instead decodes inside its own tcgen05 GEMM (ep_linear_fused) when the call has at most
-FUSED_MAX_TOKENS tokens: the weight then never passes through memory in BF16.  Above that the decode
+FUSED_MAX_TOKENS BF16 tokens: the weight then never passes through memory (the FP8 / INT8 layers
+quantize the activations per token the same way and multiply codes with kind::f8f6f4 / kind::i8).  Above that the decode
 into a buffer plus the library GEMM is faster (the fused kernel's decoding warps share each SM with
 the operand buffers and go no faster with more tokens, while its X slices grow).
 
@@ -110,21 +111,26 @@ class CompressedLinear(nn.Module):
             return False
         info = w.info
         tokens = x.numel() // self.in_features if x.dim() else 0
-        return (info.layout == B.LAYOUT_GEMM and info.container_dtype == B.BF16 and w.device == x.device
-                and 1 <= tokens <= FUSED_MAX_TOKENS)
+        return (info.layout == B.LAYOUT_GEMM and info.container_dtype in (B.BF16, B.INT8, B.FP8E4M3)
+                and w.device == x.device and 1 <= tokens <= FUSED_MAX_TOKENS)
+
+    def _fused_forward(self, x):
+        """the weight decoded inside the tcgen05 GEMM (ep_linear_fused); the FP8 / INT8 layers'
+        activations are quantized per token inside the same call"""
+        w = self._weight
+        s = torch.cuda.current_stream(x.device)
+        tables = _tables(w, s)
+        bias = None if self.bias is None else self.bias.to(torch.bfloat16)
+        if self._work is None or self._work.device != x.device:
+            self._work = torch.zeros(B.linear_fused_workspace(w.info, FUSED_MAX_TOKENS), dtype=torch.uint8,
+                                     device=x.device)
+        y = B.linear_fused(x.reshape(-1, self.in_features), w.blob, w.info, tables, bias=bias, work=self._work,
+                           stream=s)
+        return y.reshape(*x.shape[:-1], self.out_features)
 
     def forward(self, x):
         if self.fused_for(x):
-            w = self._weight
-            s = torch.cuda.current_stream(x.device)
-            tables = _tables(w, s)
-            bias = None if self.bias is None else self.bias.to(torch.bfloat16)
-            if self._work is None or self._work.device != x.device:
-                self._work = torch.zeros(B.linear_fused_workspace(w.info, FUSED_MAX_TOKENS), dtype=torch.uint8,
-                                         device=x.device)
-            y = B.linear_fused(x.reshape(-1, self.in_features), w.blob, w.info, tables, bias=bias, work=self._work,
-                               stream=s)
-            return y.reshape(*x.shape[:-1], self.out_features)
+            return self._fused_forward(x)
         w = self._decoded()
         return F.linear(x, w.to(x.dtype) if w.dtype != x.dtype else w, self.bias)
 
@@ -203,6 +209,8 @@ class CompressedFP8Linear(_CodeLinear):
     code_dtype = torch.float8_e4m3fn
 
     def forward(self, x):
+        if self.fused_for(x):
+            return self._fused_forward(x)
         shape = x.shape
         x2 = x.reshape(-1, self.in_features)
         q, sx = self._quantize_x(x2)
@@ -219,6 +227,8 @@ class CompressedINT8Linear(_CodeLinear):
     code_dtype = torch.int8
 
     def forward(self, x):
+        if self.fused_for(x):
+            return self._fused_forward(x)
         shape = x.shape
         x2 = x.reshape(-1, self.in_features)
         q, sx = self._quantize_x(x2)

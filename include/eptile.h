@@ -213,8 +213,16 @@ int ep_decompress(const ep_info *info, const void *d_blob, const void *d_workspa
                   uint32_t *d_status, ep_stream_t stream);
 
 /* A linear layer's forward with the weight decoded inside the GEMM ("EntroPack API reference",
- * CompressedLinear: the weight is reconstructed for every forward call; here it never reaches
- * global memory): Y = X W^T (+ bias) for a stream written with EP_LAYOUT_GEMM and a BF16 container.
+ * CompressedLinear and CompressedFP8Linear / CompressedINT8Linear: the weight is reconstructed for
+ * every forward call; here it never reaches global memory): Y = X W^T (+ bias) for a stream written
+ * with EP_LAYOUT_GEMM and a BF16, INT8 or FP8 E4M3 container.
+ *   BF16:       the fp32 sum of the BF16 products, plus the bias, rounded once to BF16.
+ *   INT8 / FP8: W8A8, as "Compressed Linear usage", Combine compression with FP8 or INT8
+ *               computation: the activations are quantized per token (scale s_x = amax / 127 or
+ *               / 448, 1 for an all-zero row; codes x / s_x rounded to nearest even and clamped to
+ *               [-127, 127], or clamped to [-448, 448] and rounded to E4M3), the codes multiplied
+ *               (INT8: exact int32 sums; FP8: fp32 sums), then y = RNE_bf16(fp32(fp32(sum) s_x) s_w)
+ *               with s_w the stream's row scale, and with a bias RNE_bf16(y + bias).
  *   info        from ep_stream_info; W is info->rows (N, output features) x info->cols (K).
  *   d_blob      the stream in device memory (16-byte aligned); d_tables the slot tables
  *               ep_prepare built from it.
@@ -222,17 +230,19 @@ int ep_decompress(const ep_info *info, const void *d_blob, const void *d_workspa
  *   d_bias      nullable BF16 bias of N elements.
  *   d_y         BF16 output, m x N row-major: the fp32 sum rounded once to nearest even.
  *   d_work      caller-owned device scratch of ep_linear_fused_workspace(info, m) bytes, 16-byte
- *               aligned: the fp32 partial sums of the K splits and one counter per band of 128
- *               output features.  It must be zero-filled before its first use; every call leaves
- *               the counters at zero again.  One call at a time per scratch buffer.
+ *               aligned: the partial sums of the K splits, one counter per band of 128 output
+ *               features and, for INT8 / FP8, the activations' codes and scales.  It must be
+ *               zero-filled before its first use; every call leaves the counters at zero again.
+ *               One call at a time per scratch buffer.
  *   d_status    nullable device uint32: EP_DEC_* bits of stream damage.
- * One launch: a CTA per band of 128 output features and range of K tiles.  Its warps bulk-copy
- * stream tiles into shared memory and decode them straight into BF16 operand slices (128 features
- * x 16 inputs) beside the matching slices of X; one warp issues tcgen05.mma (M = 128 features,
- * N = m padded to 16) into an fp32 accumulator in tensor memory, read out with tcgen05.ld into the
- * partial sums; the band's last CTA adds the splits in order and the bias.  Asynchronous;
- * allocates nothing.  EP_ERR_INVALID_ARG for another layout, container or m out of range,
- * EP_ERR_UNSUPPORTED when a tile is too large for the shared memory of one decoding warp. */
+ * One launch (INT8 / FP8: after one launch that quantizes X): a CTA per band of 128 output features
+ * and range of K tiles.  Its warps bulk-copy stream tiles into shared memory and decode them
+ * straight into operand slices (128 features x 32 bytes: 16 BF16 weights or 32 codes) beside the
+ * matching slices of X; one warp issues tcgen05.mma (kind::f16, kind::i8 or kind::f8f6f4; M = 128
+ * features, N = m padded to 16) into an accumulator in tensor memory, read out with tcgen05.ld into
+ * the partial sums; the band's last CTA adds the splits in order, scales and adds the bias.
+ * Asynchronous; allocates nothing.  EP_ERR_INVALID_ARG for another layout, container or m out of
+ * range, EP_ERR_UNSUPPORTED when a tile is too large for the shared memory of one decoding warp. */
 size_t ep_linear_fused_workspace(const ep_info *info, int64_t m);
 int ep_linear_fused(const ep_info *info, const void *d_blob, const void *d_tables, const void *d_x, int64_t m,
                     const void *d_bias, void *d_y, void *d_work, size_t work_nbytes, uint32_t *d_status,
