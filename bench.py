@@ -72,6 +72,22 @@ WORKLOADS = {
         shape="block 0 linears {3072x9216, 3072x3072, 3072x12288, 12288x3072} (out x in), 16 tokens",
         distribution="DiT block 0 weights (as dit_28blocks_hidden3072_bf16), GEMM block order; "
                      "x = 0.5 N(0, 1) BF16, seed 5"),
+    "linear_fused_dit_block_16tok_int8": dict(
+        layers=lambda: [(f"block0.{n}", (lambda l=l: _synth().dit_layer(0, l)))
+                        for l, n in enumerate(("qkv", "out", "mlp_up", "mlp_down"))],
+        target=4.0, container="int8", scheme="linear_fused", tokens=16,
+        dims=[(3072, 9216), (3072, 3072), (3072, 12288), (12288, 3072)],
+        shape="block 0 linears {3072x9216, 3072x3072, 3072x12288, 12288x3072} (out x in), 16 tokens",
+        distribution="DiT block 0 weights as per-row absmax INT8 codes, GEMM block order; x = 0.5 N(0, 1) BF16, "
+                     "seed 5, quantized per token (W8A8)"),
+    "linear_fused_dit_block_16tok_fp8": dict(
+        layers=lambda: [(f"block0.{n}", (lambda l=l: _synth().dit_layer(0, l)))
+                        for l, n in enumerate(("qkv", "out", "mlp_up", "mlp_down"))],
+        target=4.0, container="fp8_e4m3", scheme="linear_fused", tokens=16,
+        dims=[(3072, 9216), (3072, 3072), (3072, 12288), (12288, 3072)],
+        shape="block 0 linears {3072x9216, 3072x3072, 3072x12288, 12288x3072} (out x in), 16 tokens",
+        distribution="DiT block 0 weights as per-row absmax FP8 E4M3 codes, GEMM block order; x = 0.5 N(0, 1) "
+                     "BF16, seed 5, quantized per token (W8A8)"),
     "outliers_8192x28672_bf16": dict(
         layers=lambda: [("w", lambda: _synth().gaussian_outliers(8192, 28672, 3))], target=4.0, container=0,
         dims=[(8192, 28672)],
@@ -796,17 +812,18 @@ def run_ours_linear(a, rank, world, local_rank):
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     g = torch.Generator().manual_seed(5)
     layers, t_enc = [], 0.0
+    code_dtype = {"int8": torch.int8, "fp8_e4m3": torch.float8_e4m3fn}.get(wl["container"])
     for name, make in wl["layers"]():
         w = make().to(dev)
         torch.cuda.synchronize(dev)
         t0 = time.perf_counter()
-        blob = B.compress_device(w, a.target, layout=B.LAYOUT_GEMM)
+        blob = B.compress_device(w, a.target, container=wl["container"], layout=B.LAYOUT_GEMM)
         torch.cuda.synchronize(dev)
         t_enc += time.perf_counter() - t0
         info = B.stream_info(blob.cpu())
         # the same weights in the row order, for the decode-then-GEMM comparison (its decode stores
         # whole rows, the faster order for a decode into memory)
-        rblob = B.compress_device(w, a.target)
+        rblob = B.compress_device(w, a.target, container=wl["container"])
         rinfo = B.stream_info(rblob.cpu())
         x = (torch.randn(m, info.cols, generator=g) * 0.5).to(torch.bfloat16)
         with torch.cuda.stream(stream):
@@ -818,7 +835,9 @@ def run_ours_linear(a, rank, world, local_rank):
                            rtables=rtables, x_host=x, x=x.to(dev),
                            y=torch.empty(m, info.rows, dtype=torch.bfloat16, device=dev),
                            work=torch.zeros(B.linear_fused_workspace(info, m), dtype=torch.uint8, device=dev),
-                           wbuf=torch.empty(info.rows, info.cols, dtype=torch.bfloat16, device=dev)))
+                           wbuf=torch.empty(info.rows, info.cols, dtype=code_dtype or torch.bfloat16, device=dev),
+                           sw=rblob[rinfo.off_scales: rinfo.off_scales + 4 * rinfo.rows].view(torch.float32)
+                           if code_dtype else None))
     torch.cuda.synchronize(dev)
 
     def fused(r, s_=stream):
@@ -826,10 +845,31 @@ def run_ours_linear(a, rank, world, local_rank):
             B.linear_fused(L["x"], L["blobs"][r], L["info"], L["tables"], out=L["y"], work=L["work"],
                            status=status, stream=s_)
 
+    def library_w8a8(L, codes):
+        """what the per-row-quantized layers do unfused: the activations quantized per token with
+        torch ops, then torch._int_mm (INT8, tokens padded to 32: it takes more than 16 rows) or
+        torch._scaled_mm (FP8), and the two scales"""
+        x2 = L["x"]
+        amax = x2.abs().amax(dim=1, keepdim=True).float()
+        bound = 127.0 if code_dtype == torch.int8 else 448.0
+        sx = torch.where(amax > 0, amax / bound, torch.ones_like(amax))
+        q = x2.float() / sx
+        if code_dtype == torch.int8:
+            qp = torch.zeros(32, x2.shape[1], dtype=torch.int8, device=x2.device)
+            qp[:m] = q.round().clamp(-127, 127).to(torch.int8)
+            acc = torch._int_mm(qp, codes.t())[:m]
+            return (acc.float() * sx * L["sw"][None, :]).to(torch.bfloat16)
+        q = q.clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+        return torch._scaled_mm(q, codes.t(), scale_a=sx, scale_b=L["sw"][None, :].contiguous(),
+                                out_dtype=torch.bfloat16)
+
     def unfused(r):
         for L in layers:
-            F.linear(L["x"], B.decompress(L["rblobs"][r], L["rinfo"], workspace=L["rtables"], out=L["wbuf"],
-                                          stream=stream))
+            wd = B.decompress(L["rblobs"][r], L["rinfo"], workspace=L["rtables"], out=L["wbuf"], stream=stream)
+            if code_dtype is None:
+                F.linear(L["x"], wd)
+            else:
+                library_w8a8(L, wd)
 
     def dense(r):
         for L in layers:
@@ -842,7 +882,17 @@ def run_ours_linear(a, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     assert int(status.item()) == 0, "fused GEMM status"
     for L in layers:
-        wd = B.decompress(L["blobs"][0], L["info"], workspace=L["tables"]).float()
+        wd = B.decompress(L["blobs"][0], L["info"], workspace=L["tables"])
+        if code_dtype is not None:
+            # INT8: the same bits as the layer's unfused arithmetic; FP8: the same up to the order
+            # of the fp32 sums
+            lib_y = library_w8a8(L, wd)
+            if code_dtype == torch.int8:
+                assert torch.equal(L["y"], lib_y), L["name"]
+            else:
+                assert torch.allclose(L["y"].float(), lib_y.float(), rtol=2 ** -6, atol=1e-3), L["name"]
+            continue
+        wd = wd.float()
         ref = L["x"].float() @ wd.T
         mag = L["x"].float().abs() @ wd.abs().T
         tol = L["info"].cols * 2.0 ** -24 * mag + 2.0 ** -8 * ref.abs()
@@ -900,8 +950,12 @@ def run_ours_linear(a, rank, world, local_rank):
 
         def u1(r, one=one):
             for L_ in one:
-                F.linear(L_["x"], B.decompress(L_["rblobs"][r], L_["rinfo"], workspace=L_["rtables"],
-                                               out=L_["wbuf"], stream=stream))
+                wd = B.decompress(L_["rblobs"][r], L_["rinfo"], workspace=L_["rtables"], out=L_["wbuf"],
+                                  stream=stream)
+                if code_dtype is None:
+                    F.linear(L_["x"], wd)
+                else:
+                    library_w8a8(L_, wd)
 
         def d1(r, one=one):
             for L_ in one:
@@ -945,7 +999,8 @@ def run_ours_linear(a, rank, world, local_rank):
         "stream": {"bpp": [round(L["info"].actual_bpp, 4) for L in layers], "paired": [L["info"].paired for L in layers],
                    "layout": "gemm"},
         "step_us": {"fused": round(1e3 * fused_ms / a.steps, 2),
-                    "decode_row_stream_then_library_gemm": round(1e3 * unfused_ms / a.steps, 2),
+                    ("decode_row_stream_then_library_gemm" if code_dtype is None else
+                     "decode_row_stream_then_library_w8a8"): round(1e3 * unfused_ms / a.steps, 2),
                     "library_gemm_bf16_weights": round(1e3 * dense_ms / a.steps, 2),
                     "per_layer_fused_unfused_bf16": per_layer},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -967,6 +1022,20 @@ def run_ours_linear(a, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def _oracle_weights_f32(O, blob_np, wd):
+    """the oracle's decoded container as fp32 weights: BF16 as it is, INT8 / FP8 codes times the
+    stream's row scales"""
+    rc, info = O.parse(blob_np)
+    if info.container_dtype == O.BF16:
+        return (wd.view(np.uint16).astype(np.uint32) << 16).view(np.float32)
+    scales = np.frombuffer(blob_np.tobytes(), np.float32, count=info.rows, offset=info.off_scales)
+    if info.container_dtype == O.INT8:
+        codes = wd.astype(np.float32)
+    else:
+        codes = torch.from_numpy(wd.view(np.uint8).copy()).view(torch.float8_e4m3fn).float().numpy()
+    return codes * scales[:, None]
+
+
 def cpu_linear_baseline(a, layers, m):
     """the oracle (tile-parallel decode on every host core) plus a numpy fp32 GEMM, on a bounded
     sample: the 3072x3072 layer's stream, whole, repeated for about --cpu-seconds"""
@@ -982,7 +1051,7 @@ def cpu_linear_baseline(a, layers, m):
     while time.perf_counter() - t0 < a.cpu_seconds:
         rc, st, _, wd = O.decode_parallel(blob_np, threads=ncores, want_v=False)
         assert rc == 0 and st == 0
-        _ = x_np @ (wd.view(np.uint16).astype(np.uint32) << 16).view(np.float32).T
+        _ = x_np @ _oracle_weights_f32(O, blob_np, wd).T
         done += 1
     el = time.perf_counter() - t0
     n = oinfo.rows * oinfo.cols
@@ -1001,7 +1070,8 @@ def run_reference_linear(a, rank, world):
     m = wl["tokens"]
     name, make = [(n, f) for n, f in wl["layers"]() if n.endswith(".out")][0]
     w = make()
-    rc, blob = O.compress(w, a.target, layout=1)
+    rc, blob = O.compress(w, a.target, container={0: 0, "int8": O.INT8, "fp8_e4m3": O.FP8E4M3}[wl["container"]],
+                          layout=1)
     assert rc == 0
     rc, oinfo = O.parse(blob)
     g = torch.Generator().manual_seed(5)
@@ -1011,7 +1081,7 @@ def run_reference_linear(a, rank, world):
     def step():
         rc_, st_, _, wd = O.decode_parallel(blob, threads=ncores, want_v=False)
         assert rc_ == 0 and st_ == 0
-        return x_np @ (wd.view(np.uint16).astype(np.uint32) << 16).view(np.float32).T
+        return x_np @ _oracle_weights_f32(O, blob, wd).T
 
     for _ in range(a.warmup):
         step()
@@ -1027,7 +1097,8 @@ def run_reference_linear(a, rank, world):
             "data": "synthetic", "config": bench_config(a, world),
             "cpu_baseline": {"value": round(rate, 4), "unit": "Gweights/s", "cores": ncores, "kind": "oracle",
                              "sample": f"the {oinfo.rows}x{oinfo.cols} layer's stream per step, decoded by the C oracle "
-                                       f"on {ncores} threads, then x W^T in numpy fp32 ({m} tokens)"},
+                                       f"on {ncores} threads, then x W^T in numpy fp32 with the decoded weights "
+                                       f"({m} tokens)"},
             "e2e": {"value": round(rate, 4), "unit": "Gweights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
