@@ -34,8 +34,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "fused decode GB/s (container out) & Gweights/s at 4 bpp; % of HBM roofline"
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
-KERNEL_SRCS = {"decode_kernel": ("decode.cu", "device_util.cuh", "format.h"),
-               "linear_kernel": ("decode.cu", "device_util.cuh", "format.h"),
+KERNEL_SRCS = {"decode_kernel": ("decode.cu", "decode_core.cuh", "device_util.cuh", "format.h"),
+               "linear_kernel": ("linear.cu", "decode_core.cuh", "device_util.cuh", "format.h"),
                "ans_decode_kernel": ("tile_ans.cu", "device_util.cuh", "tile_ans.h")}
 L2_BYTES = 126 * 2 ** 20
 
@@ -852,7 +852,7 @@ def run_ours_linear(a, rank, world, local_rank):
         x2 = L["x"]
         amax = x2.abs().amax(dim=1, keepdim=True).float()
         bound = 127.0 if code_dtype == torch.int8 else 448.0
-        sx = torch.where(amax > 0, amax / bound, torch.ones_like(amax))
+        sx = torch.where(amax > 0, amax / torch.full_like(amax, bound), torch.ones_like(amax))  # rounded division
         q = x2.float() / sx
         if code_dtype == torch.int8:
             qp = torch.zeros(32, x2.shape[1], dtype=torch.int8, device=x2.device)
@@ -899,6 +899,11 @@ def run_ours_linear(a, rank, world, local_rank):
         assert bool(((L["y"].float() - ref).abs() <= tol + 2.0 ** -8 * L["y"].float().abs()).all()), L["name"]
 
     def timed(body, steps):
+        # once outside the capture: libraries create their per-stream handles on first use, which a
+        # capture does not allow
+        with torch.cuda.stream(stream):
+            body(0)
+        torch.cuda.synchronize(dev)
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=stream):
             for r in range(rot):

@@ -123,6 +123,8 @@ def lib():
         L.ep_decompress_host.argtypes = [C.POINTER(StreamInfo), p, p, C.c_int32, p, C.c_size_t, p, p]
         L.ep_linear_fused_workspace.restype = C.c_size_t
         L.ep_linear_fused_workspace.argtypes = [C.POINTER(StreamInfo), C.c_int64]
+        L.ep_linear_fused_plan.restype = C.c_int
+        L.ep_linear_fused_plan.argtypes = [C.POINTER(StreamInfo), C.c_int64, C.c_int32, C.POINTER(LinearPlan)]
         L.ep_linear_fused.restype = C.c_int
         L.ep_linear_fused.argtypes = [C.POINTER(StreamInfo), p, p, p, C.c_int64, p, p, p, C.c_size_t, p, p]
         L.ep_ans_compress_bound.restype = C.c_size_t
@@ -411,6 +413,23 @@ def ans_decompress(d_blob, info, workspace=None, out=None, status=None, stream=N
 
 
 # ---------------------------------------------------------------- the decode fused into a GEMM
+class LinearPlan(C.Structure):
+    """ep_linear_plan: the launch ep_linear_fused would make (grid, warps, shared-memory layout)"""
+    _fields_ = [(n, C.c_uint32) for n in ("bands", "splits", "k_tiles_per_split", "decoding_warps", "threads",
+                                          "tokens_padded", "tmem_columns", "tile_buffer_bytes", "smem_tables_bytes",
+                                          "smem_barriers_offset", "smem_tiles_offset", "smem_slices_offset",
+                                          "smem_x_offset", "smem_x_bytes_per_warp")] + \
+               [("smem_bytes", C.c_uint64), ("work_bytes", C.c_uint64)]
+
+
+def linear_fused_plan(info, m, sms):
+    """(status, LinearPlan) of ep_linear_fused for m tokens on a GPU with `sms` multiprocessors,
+    computed on the host"""
+    plan = LinearPlan()
+    rc = lib().ep_linear_fused_plan(C.byref(info), m, sms, C.byref(plan))
+    return rc, plan
+
+
 def linear_fused_workspace(info, m):
     """bytes of scratch ep_linear_fused needs for m tokens (0: the stream or m is not one it takes)"""
     return int(lib().ep_linear_fused_workspace(C.byref(info), m))

@@ -12,9 +12,10 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libeptile.so")
-SOURCES = ["decode.cu", "device_encode.cu", "host_encode.cpp", "host_stream.cpp", "tile_ans.cu", "tile_ans_host.cpp"]
+SOURCES = ["decode.cu", "linear.cu", "device_encode.cu", "host_encode.cpp", "host_stream.cpp", "tile_ans.cu",
+           "tile_ans_host.cpp"]
 HEADERS = [os.path.join(CSRC, h) for h in ("format.h", "encode_math.h", "encode_host.h", "device_util.cuh",
-                                           "tile_ans.h")] + \
+                                           "decode_core.cuh", "tile_ans.h")] + \
     [os.path.join(ROOT, "include", "eptile.h")]
 
 

@@ -196,7 +196,9 @@ class _CodeLinear(CompressedLinear):
     def _quantize_x(self, x2):
         amax = x2.abs().amax(dim=1, keepdim=True).float()
         bound = 448.0 if self.code_dtype == torch.float8_e4m3fn else 127.0
-        scale = torch.where(amax > 0, amax / bound, torch.ones_like(amax))
+        # a correctly rounded division (tensor by tensor: torch divides by a Python number as a
+        # multiplication by its reciprocal, which can differ in the last bit)
+        scale = torch.where(amax > 0, amax / torch.full_like(amax, bound), torch.ones_like(amax))
         q = x2.float() / scale
         if self.code_dtype == torch.int8:
             q = q.round().clamp(-127, 127).to(torch.int8)

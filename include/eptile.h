@@ -244,6 +244,21 @@ int ep_decompress(const ep_info *info, const void *d_blob, const void *d_workspa
  * Asynchronous; allocates nothing.  EP_ERR_INVALID_ARG for another layout, container or m out of
  * range, EP_ERR_UNSUPPORTED when a tile is too large for the shared memory of one decoding warp. */
 size_t ep_linear_fused_workspace(const ep_info *info, int64_t m);
+
+/* The launch ep_linear_fused would make for this stream and m on a GPU with `sms` multiprocessors,
+ * computed on the host without touching a device (for tests and capacity planning): the grid
+ * (bands of 128 output features x K splits, one wave), the decoding warps per CTA, the padded
+ * token count, the tensor-memory columns, the shared-memory layout (tables from offset 0, then the
+ * barriers, the per-warp stream-tile buffers, the per-warp pairs of 4 KB W slices and the per-warp
+ * X buffers) and the scratch bytes.  EP_ERR_INVALID_ARG as ep_linear_fused refuses the stream or m,
+ * EP_ERR_UNSUPPORTED when even one decoding warp's buffers do not fit (*out is filled either way). */
+typedef struct {
+    uint32_t bands, splits, k_tiles_per_split, decoding_warps, threads, tokens_padded, tmem_columns;
+    uint32_t tile_buffer_bytes, smem_tables_bytes, smem_barriers_offset, smem_tiles_offset, smem_slices_offset;
+    uint32_t smem_x_offset, smem_x_bytes_per_warp;
+    uint64_t smem_bytes, work_bytes;
+} ep_linear_plan;
+int ep_linear_fused_plan(const ep_info *info, int64_t m, int32_t sms, ep_linear_plan *out);
 int ep_linear_fused(const ep_info *info, const void *d_blob, const void *d_tables, const void *d_x, int64_t m,
                     const void *d_bias, void *d_y, void *d_work, size_t work_nbytes, uint32_t *d_status,
                     ep_stream_t stream);

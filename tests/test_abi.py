@@ -16,7 +16,7 @@ def test_exports_every_declared_symbol():
                           "ep_compress_device", "ep_stream_info", "ep_prepare", "ep_decompress",
                           "ep_decompress_noalloc", "ep_decompress_host_scratch", "ep_decompress_host",
                           "ep_ans_compress_bound", "ep_ans_compress_host", "ep_ans_stream_info",
-                          "ep_ans_prepare", "ep_ans_decompress", "ep_linear_fused_workspace", "ep_linear_fused",
+                          "ep_ans_prepare", "ep_ans_decompress", "ep_linear_fused_workspace", "ep_linear_fused", "ep_linear_fused_plan",
                           "ep_status_string"}
     lib = B.lib()
     for n in names:

@@ -66,7 +66,7 @@ def test_checkpoint_on_the_gpu(oracle):
 
 def quantized_x(x, bound, dtype):
     amax = x.abs().amax(dim=1, keepdim=True).float()
-    sx = torch.where(amax > 0, amax / bound, torch.ones_like(amax))
+    sx = torch.where(amax > 0, amax / torch.full_like(amax, bound), torch.ones_like(amax))  # rounded division
     q = x.float() / sx
     q = q.round().clamp(-127, 127).to(torch.int8) if dtype == torch.int8 else q.clamp(-448, 448).to(dtype)
     return q, sx

@@ -144,7 +144,7 @@ def w8a8_reference(oracle, blob, x, bias, container):
     xf = x.float().cpu()
     bound = 127.0 if container == B.INT8 else 448.0
     amax = xf.abs().amax(dim=1, keepdim=True)
-    sx = torch.where(amax > 0, amax / bound, torch.ones_like(amax))
+    sx = torch.where(amax > 0, amax / torch.full_like(amax, bound), torch.ones_like(amax))  # rounded division
     q = xf / sx
     if container == B.INT8:
         xq = q.round().clamp(-127, 127).to(torch.int64)
@@ -172,7 +172,10 @@ def w8a8_reference(oracle, blob, x, bias, container):
                                                                 ((3072, 3072), 16, B.INT8, B.CODING_AUTO, True),
                                                                 ((384, 1024), 7, B.FP8E4M3, B.CODING_SINGLE, True),
                                                                 ((3072, 9216), 16, B.FP8E4M3, B.CODING_AUTO, False),
-                                                                ((128, 1024), 128, B.INT8, B.CODING_SINGLE, True)])
+                                                                ((128, 1024), 128, B.INT8, B.CODING_SINGLE, True),
+                                                                # 2 and 3 rounds of tiles per decoding warp
+                                                                ((3072, 9216), 16, B.INT8, B.CODING_AUTO, True),
+                                                                ((3072, 12288), 3, B.INT8, B.CODING_SINGLE, False)])
 def test_fused_w8a8(oracle, shape, m, container, coding, with_bias):
     """INT8: every output bit equals the CPU arithmetic on the oracle's codes; FP8: within the bound"""
     w = synth.row_lognormal(*shape, seed=shape[0] + m)
