@@ -452,6 +452,9 @@ __device__ __forceinline__ uint32_t decode_blocks(const Params &p, Lane<SMEM> &L
             uint32_t left = (p.cb - (col - lane)) >> 5;
             kseg = k + left < p.K ? k + left : p.K;
         }
+        // GEMM-ordered tiles: four steps per unrolled iteration, so that the step's row of the
+        // group of four (its factor, its place in the operand slice) is known when compiled
+#pragma unroll (GEMM ? 4 : 1)
         for (; k < kseg; ++k, b += 32u) {
             if constexpr (GEMM) {
                 b = gbase + (k & 3u) * 32u * p.cb + (k >> 2);
