@@ -415,7 +415,8 @@ def ans_decompress(d_blob, info, workspace=None, out=None, status=None, stream=N
 # ---------------------------------------------------------------- the decode fused into a GEMM
 class LinearPlan(C.Structure):
     """ep_linear_plan: the launch ep_linear_fused would make (grid, warps, shared-memory layout)"""
-    _fields_ = [(n, C.c_uint32) for n in ("bands", "splits", "k_tiles_per_split", "decoding_warps", "threads",
+    _fields_ = [(n, C.c_uint32) for n in ("bands", "ctas", "tiles_per_cta", "accumulators", "spread", "splits",
+                                          "decoding_warps", "threads",
                                           "tokens_padded", "tmem_columns", "tile_buffer_bytes", "smem_tables_bytes",
                                           "smem_barriers_offset", "smem_tiles_offset", "smem_slices_offset",
                                           "smem_x_offset", "smem_x_bytes_per_warp")] + \

@@ -12,30 +12,50 @@ namespace {
 
 // ------------------------------------------------------------------ the decode fused into a GEMM
 // Y^T = W X^T for a weight W (N x K) held as a GEMM-ordered stream (EP_LAYOUT_GEMM): each stream tile
-// is one 128 x 64 tile of W.  One CTA per (band of 128 output features, range of K tiles); warps
-// 0 .. S-1 decode, one tile at a time each: a bulk copy of the stream tile into the warp's buffer,
+// is one 128 x 64 tile of W, tiles in band-major order (a band: 128 output features, all K tiles).
+// The tiles are spread evenly over one wave of CTAs, one per SM: CTA c takes tiles
+// [c T / C, (c + 1) T / C), which may span two or more bands.  Warps 0 .. S-1 decode, one tile at a
+// time each: a bulk copy of the stream tile into the warp's buffer,
 // the matching slice of X (tokens padded to a multiple of 16) into the warp's X buffer, then the
 // tile's 32 steps.  Every 8 steps complete a 128 x 16 K-slice of the tile, which goes to one of the
 // warp's two 4 KB slice buffers (a ring) and is announced on that buffer's `full` barrier.  Warp S
 // issues the tensor-core work: for each round of tiles, slice by slice, warp by warp (a fixed
 // order, so the fp32 sums are the same on every call), one tcgen05.mma (M = 128 features,
-// N = tokens, K = 16, A = the W slice, B = the X slice, both K-major) accumulating in tensor
-// memory, committed to the slice buffer's `empty` barrier.  After the last MMA, warps 0..3 read
-// the 128 x N fp32 accumulator out of tensor memory into the CTA's slice of the partial sums; the
-// band's last CTA to finish adds the splits' partial sums in split order (the same sums on every
-// call), adds the bias, rounds once to BF16 and writes Y.
+// N = tokens, K = 16, A = the W slice, B = the X slice, both K-major) into the tensor-memory
+// accumulator of the tile's band (one per band the CTA touches), committed to the slice buffer's
+// `empty` barrier.  After the last MMA, warps 0..3 read the accumulators out of tensor memory into
+// the CTA's partial sums; the last CTA to finish a band adds the partial sums of the CTAs that
+// touched it in CTA order (the same sums on every call), scales, adds the bias, rounds once to BF16
+// and writes the band's part of Y.
 constexpr uint32_t kLinMaxWarps = 15;       // decoding warps per CTA
 constexpr uint32_t kLinSlice = 128u * 16u * 2u;  // one 128 x 16 BF16 K-slice of a W tile
 constexpr uint32_t kLinBarBytes = 40;       // per decoding warp: full[2], empty[2], copy
 
+// Which tiles each CTA takes (tiles in band-major order, KT per band): either band-aligned (each
+// band's K tiles split into `splits` ranges of ktps, CTA c = band * splits + split) or spread evenly
+// (CTA c takes [c T / C, (c + 1) T / C), which may span bands).  first(c): CTA c's first tile
+// (first(C) = T); cta_of(t): the CTA holding tile t.
+struct TileMap {
+    uint32_t T, C, KT, splits, ktps, aligned;
+    __host__ __device__ __forceinline__ uint32_t first(uint32_t c) const {
+        if (aligned) return (c / splits) * KT + min((c % splits) * ktps, KT);
+        return uint32_t(uint64_t(c) * T / C);
+    }
+    __host__ __device__ __forceinline__ uint32_t cta_of(uint32_t t) const {
+        if (aligned) return (t / KT) * splits + (t % KT) / ktps;
+        return uint32_t((uint64_t(t + 1) * C - 1) / T);  // the largest c with first(c) <= t
+    }
+};
+
 struct LinParams {
     Params dp;                 // the stream (tiles, tables, row factors, status)
     const uint16_t *x;         // activations, BF16, M x cols row-major
-    float *part;               // fp32 partial sums, splits x M x N
+    float *part;               // partial sums (fp32, int32 for INT8): C x nacc slots of M x 128
     uint32_t *count;           // per band: CTAs done (zero between calls)
     const uint16_t *bias;      // nullable, BF16, N
     uint16_t *y;               // BF16, M x N
-    uint32_t splits;
+    TileMap map;               // the CTAs' tile ranges (map.C CTAs: the grid)
+    uint32_t nacc;             // partial-sum slots per CTA (most bands a CTA touches)
     const uint8_t *xq;         // code containers: the activations' 8-bit codes, M x cols
     const float *xscale;       // code containers: the activations' per-token scales
     const float *wscale;       // code containers: the weight's per-row scales (from the stream)
@@ -44,7 +64,6 @@ struct LinParams {
     uint32_t idesc;            // the MMA's instruction descriptor
     uint32_t tmem_cols;        // tensor-memory columns of the accumulator (a power of 2, >= 32)
     uint32_t KT;               // K tiles per band (cols / 64)
-    uint32_t kt_per_split;
     uint32_t S;                // decoding warps
     uint32_t tile_buf;         // bytes of a stream-tile buffer
     uint32_t off_bars, off_tile, off_w, off_x;  // shared-memory layout (offsets from the dynamic base)
@@ -122,9 +141,10 @@ __global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(cons
     auto ring = [&](uint32_t w) { return base + P.off_w + 2u * kLinSlice * w; };
     auto xbuf = [&](uint32_t w) { return base + P.off_x + P.npad * XB * w; };
     auto tbuf = [&](uint32_t w) { return base + P.off_tile + P.tile_buf * w; };
-    const uint32_t band = blockIdx.x;
-    const uint32_t kt0 = blockIdx.y * P.kt_per_split;
-    const uint32_t nkt = min(P.KT, kt0 + P.kt_per_split) - kt0;  // >= 1: the plan leaves no split empty
+    const uint32_t cta = blockIdx.x;
+    const uint32_t t0 = P.map.first(cta);
+    const uint32_t nkt = P.map.first(cta + 1) - t0;  // >= 1: the plan leaves no CTA without tiles
+    const uint32_t b0 = t0 / P.KT, nband = (t0 + nkt - 1) / P.KT - b0 + 1;  // bands touched, <= P.nacc
 
     if (threadIdx.x == 0) {
         for (uint32_t w = 0; w < S; ++w)
@@ -152,11 +172,11 @@ __global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(cons
     uint32_t err = ok ? 0u : uint32_t(EP_DEC_TIMEOUT);
 
     if (warp < S) {
-        // ---- decoding warps: tiles j = warp, warp + S, ... of the CTA's K range
+        // ---- decoding warps: tiles t0 + j, j = warp, warp + S, ... of the CTA's range
         SliceSink<DT> sink{ring(warp), wbar(warp), 0u};
         const uint32_t copyb = wbar(warp) + 32u;
         for (uint32_t j = warp; j < nkt && ok; j += S, ++sink.round) {
-            const uint32_t kt = kt0 + j, t = band * P.KT + kt;
+            const uint32_t t = t0 + j, kt = t % P.KT;
             // the MMAs of the previous tile (its last slice, use U round - 1, in ring buffer 1, and
             // so all before it) are done: the X buffer and both slice buffers are free
             if (sink.round > 0 && !mbar_wait(wbar(warp) + 24u, ((SliceSink<DT>::kUses * sink.round - 1u) >> 1) & 1u)) {
@@ -200,10 +220,17 @@ __global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(cons
         // ---- the MMA issuer: round by round, slice by slice, warp by warp
         constexpr uint32_t U = SliceSink<DT>::kUses;
         const uint32_t rounds = (nkt + S - 1) / S;
-        bool first = true;
-        for (uint32_t r = 0; r < rounds && ok; ++r)
-            for (uint32_t sl = 0; sl < U && ok; ++sl)
-                for (uint32_t w = 0; w < S && r * S + w < nkt; ++w) {
+        uint32_t started = 0;  // the accumulators (bands) that have had their first MMA
+        for (uint32_t r = 0; r < rounds && ok; ++r) {
+            // the band (accumulator) of the round's first tile, and the tile's place in it
+            const uint32_t ar = (t0 + r * S) / P.KT - b0, kr = (t0 + r * S) % P.KT;
+            for (uint32_t sl = 0; sl < U && ok; ++sl) {
+                uint32_t a = ar, kin = kr;
+                for (uint32_t w = 0; w < S && r * S + w < nkt; ++w, ++kin) {
+                    if (kin == P.KT) {  // this warp's tile starts the next band
+                        kin = 0;
+                        ++a;
+                    }
                     const uint32_t u = U * r + sl, fb = wbar(w) + 8u * (u & 1u);
                     if (!mbar_wait(fb, (u >> 1) & 1u)) {
                         err |= EP_DEC_TIMEOUT;
@@ -211,26 +238,27 @@ __global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(cons
                         break;
                     }
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    const uint32_t d = tmem + a * P.npad;  // the accumulator of the tile's band
                     if (lane == 0) {
                         const uint64_t da = umma_desc_plain(ring(w) + (u & 1u) * kLinSlice, 128u, 256u);
                         const uint64_t db = umma_desc_plain(xbuf(w) + 256u * sl, 128u, 8u * XB);
-                        const uint32_t acc = first ? 0u : 1u;
+                        const uint32_t acc = (started >> a) & 1u;
                         if constexpr (DT == EP_BF16)
                             asm volatile(
                                 "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                                "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+                                "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
                                 "l"(da), "l"(db), "r"(P.idesc), "r"(acc)
                                 : "memory");
                         else if constexpr (DT == EP_INT8)
                             asm volatile(
                                 "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                                "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+                                "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
                                 "l"(da), "l"(db), "r"(P.idesc), "r"(acc)
                                 : "memory");
                         else
                             asm volatile(
                                 "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                                "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+                                "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
                                 "l"(da), "l"(db), "r"(P.idesc), "r"(acc)
                                 : "memory");
                         asm volatile(
@@ -238,33 +266,39 @@ __global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(cons
                                 fb + 16u)
                             : "memory");
                     }
-                    first = false;
+                    started |= 1u << a;
                     __syncwarp();
                 }
+            }
+        }
         if (lane == 0)
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(done)
                          : "memory");
         __syncwarp();
     }
-    // ---- epilogue: warp q < 4 reads tensor-memory lanes 32 q .. 32 q + 31 (features), one column per
-    // token, and writes each token's 32 features (128 contiguous bytes) of the partial sums
+    // ---- epilogue: warp q < 4 reads tensor-memory lanes 32 q .. 32 q + 31 (features) of each band's
+    // accumulator, one column per token, into the CTA's partial-sum slot of that band: M rows of the
+    // band's 128 features (each warp writes 128 contiguous bytes per token)
     if (warp < 4) {
         if (!mbar_wait(done, 0)) err |= EP_DEC_TIMEOUT;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        float *dst = P.part + size_t(blockIdx.y) * P.M * P.N + 128u * band + 32u * warp + lane;
-        for (uint32_t c0 = 0; c0 < P.npad; c0 += 16u) {
-            uint32_t r[16];
-            asm volatile(
-                "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-                "%14, %15}, [%16];"
-                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-                  "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-                  "=r"(r[15])
-                : "r"(tmem + ((32u * warp) << 16) + c0));
-            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        for (uint32_t a = 0; a < nband; ++a) {
+            uint32_t *dst = reinterpret_cast<uint32_t *>(P.part) + size_t(cta * P.nacc + a) * P.M * 128u + 32u * warp +
+                            lane;
+            for (uint32_t c0 = 0; c0 < P.npad; c0 += 16u) {
+                uint32_t r[16];
+                asm volatile(
+                    "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+                    "%13, %14, %15}, [%16];"
+                    : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                      "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                      "=r"(r[15])
+                    : "r"(tmem + ((32u * warp) << 16) + a * P.npad + c0));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-            for (uint32_t i = 0; i < 16u; ++i)  // fp32 sums, or the int32 sums of the INT8 MMA, as bits
-                if (c0 + i < P.M) reinterpret_cast<uint32_t *>(dst)[size_t(c0 + i) * P.N] = r[i];
+                for (uint32_t i = 0; i < 16u; ++i)  // fp32 sums, or the int32 sums of the INT8 MMA, as bits
+                    if (c0 + i < P.M) dst[size_t(c0 + i) * 128u] = r[i];
+            }
         }
     }
     if (err && p.status && lane == 0) atomicOr(p.status, err);
@@ -278,57 +312,75 @@ __global__ void __launch_bounds__((kLinMaxWarps + 1) * 32, 1) linear_kernel(cons
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(P.tmem_cols)
                      : "memory");
     }
-    // ---- the band's last CTA: Y = the splits' partial sums in split order, plus the bias
+    // ---- count this CTA in each band it touched; the band's last CTA (the one that completes its
+    // count: every CTA from the one holding the band's first tile to the one holding its last) adds
+    // the band's partial sums
     if (threadIdx.x == 0) {
-        const uint32_t ticket = atomicAdd(P.count + band, 1u);
-        asm volatile("st.shared.u32 [%0], %1;" ::"r"(tmem_slot), "r"(ticket == P.splits - 1u ? 1u : 0u) : "memory");
+        uint32_t last = 0;
+        for (uint32_t a = 0; a < nband; ++a) {
+            const uint32_t b = b0 + a;
+            const uint32_t lo = P.map.cta_of(b * P.KT), hi = P.map.cta_of((b + 1) * P.KT - 1u);
+            if (atomicAdd(P.count + b, 1u) == hi - lo) last |= 1u << a;
+        }
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(tmem_slot), "r"(last) : "memory");
     }
     __syncthreads();
-    if (lds32(tmem_slot) == 0u) return;
+    const uint32_t last = lds32(tmem_slot);
+    if (last == 0u) return;
     __threadfence();
-    // four features per thread and step; the loads of up to eight splits are issued before their
-    // additions, which stay in split order (INT8: exact int32 sums).  BF16: y = RNE(sum + bias).
+    // four features per thread and step; the loads of up to eight CTAs' partials are issued before
+    // their additions, which stay in CTA order (INT8: exact int32 sums).  BF16: y = RNE(sum + bias).
     // Codes: y = RNE(fp32(fp32(sum) s_x) s_w), then with a bias RNE(y + bias): the order of the
     // per-row-quantized layers' own arithmetic
     using Acc = typename std::conditional<DT == EP_INT8, int32_t, float>::type;
     using Acc4 = typename std::conditional<DT == EP_INT8, int4, float4>::type;
-    const size_t MN4 = size_t(P.M) * P.N / 4u;
-    for (uint32_t i = threadIdx.x; i < P.M * 32u; i += blockDim.x) {
-        const uint32_t m = i >> 5, n = 128u * band + 4u * (i & 31u);
-        const Acc4 *src = reinterpret_cast<const Acc4 *>(P.part + size_t(m) * P.N + n);
-        Acc a[4] = {Acc(0), Acc(0), Acc(0), Acc(0)};
-        for (uint32_t s0 = 0; s0 < P.splits; s0 += 8u) {
-            Acc4 v[8];
+    for (uint32_t a = 0; a < nband; ++a) {
+        if (!((last >> a) & 1u)) continue;
+        const uint32_t b = b0 + a;
+        const uint32_t lo = P.map.cta_of(b * P.KT), hi = P.map.cta_of((b + 1) * P.KT - 1u);
+        // CTA lo may start in an earlier band (its slot for b is further on); every later contributor
+        // starts inside band b, so band b is its first slot
+        const uint32_t slot_lo = lo * P.nacc + (b - P.map.first(lo) / P.KT);
+        for (uint32_t i = threadIdx.x; i < P.M * 32u; i += blockDim.x) {
+            const uint32_t m = i >> 5, f = 4u * (i & 31u), n = 128u * b + f;
+            Acc acc[4] = {Acc(0), Acc(0), Acc(0), Acc(0)};
+            for (uint32_t c0 = lo; c0 <= hi; c0 += 8u) {
+                Acc4 v[8];
 #pragma unroll
-            for (uint32_t j = 0; j < 8u; ++j)
-                if (s0 + j < P.splits) v[j] = __ldcg(src + (s0 + j) * MN4);
+                for (uint32_t j = 0; j < 8u; ++j)
+                    if (c0 + j <= hi) {
+                        const uint32_t c = c0 + j;
+                        const uint32_t slot = c == lo ? slot_lo : c * P.nacc;
+                        v[j] = __ldcg(reinterpret_cast<const Acc4 *>(P.part + (size_t(slot) * P.M + m) * 128u + f));
+                    }
 #pragma unroll
-            for (uint32_t j = 0; j < 8u; ++j)
-                if (s0 + j < P.splits) {
-                    a[0] += v[j].x;
-                    a[1] += v[j].y;
-                    a[2] += v[j].z;
-                    a[3] += v[j].w;
-                }
-        }
-        uint16_t *dst = P.y + size_t(m) * P.N + n;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float yv;
-            if constexpr (DT == EP_BF16) {
-                yv = a[j];
-                if (P.bias) yv += __uint_as_float(uint32_t(P.bias[n + j]) << 16);
-            } else {
-                const float f = DT == EP_INT8 ? __int2float_rn(int32_t(a[j])) : float(a[j]);
-                yv = __fmul_rn(__fmul_rn(f, P.xscale[m]), __ldg(P.wscale + n + j));
-                if (P.bias)
-                    yv = __bfloat162float(__float2bfloat16_rn(yv)) + __uint_as_float(uint32_t(P.bias[n + j]) << 16);
+                for (uint32_t j = 0; j < 8u; ++j)
+                    if (c0 + j <= hi) {
+                        acc[0] += v[j].x;
+                        acc[1] += v[j].y;
+                        acc[2] += v[j].z;
+                        acc[3] += v[j].w;
+                    }
             }
-            const __nv_bfloat16 h = __float2bfloat16_rn(yv);
-            dst[j] = *reinterpret_cast<const uint16_t *>(&h);
+            uint16_t *dst = P.y + size_t(m) * P.N + n;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float yv;
+                if constexpr (DT == EP_BF16) {
+                    yv = acc[j];
+                    if (P.bias) yv += __uint_as_float(uint32_t(P.bias[n + j]) << 16);
+                } else {
+                    const float fa = DT == EP_INT8 ? __int2float_rn(int32_t(acc[j])) : float(acc[j]);
+                    yv = __fmul_rn(__fmul_rn(fa, P.xscale[m]), __ldg(P.wscale + n + j));
+                    if (P.bias)
+                        yv = __bfloat162float(__float2bfloat16_rn(yv)) + __uint_as_float(uint32_t(P.bias[n + j]) << 16);
+                }
+                const __nv_bfloat16 h = __float2bfloat16_rn(yv);
+                dst[j] = *reinterpret_cast<const uint16_t *>(&h);
+            }
         }
+        if (threadIdx.x == 0) P.count[b] = 0u;  // ready for the next call
     }
-    if (threadIdx.x == 0) P.count[band] = 0u;  // ready for the next call
 }
 
 // The activations of a per-row-quantized layer: per token, scale = amax / 127 (INT8) or / 448 (FP8
@@ -360,63 +412,105 @@ __global__ void __launch_bounds__(256) quantize_x_kernel(const uint16_t *x, uint
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// ---- the fused GEMM's launch plan: bands of 128 output features, K tiles split across CTAs so that
-// all CTAs run in one wave (one per SM); shared memory = tables, barriers, then per decoding warp a
-// stream-tile buffer, two W slice buffers and an X buffer.  Decoding warps: as many as fit, then as
-// few as give the same number of rounds of tiles.
+// ---- the fused GEMM's launch plan.  The T = bands x KT tiles go to CTAs (one per SM) either
+// band-aligned (each band's K tiles split so that about one wave of CTAs runs) or spread evenly over
+// one wave (more CTAs when one would touch more bands than tensor memory holds accumulators for);
+// the plan takes the even spread only when it needs fewer rounds of tiles per decoding warp (times
+// waves), since aligned CTAs have one accumulator and fewer contributors per band.  Shared memory =
+// tables, barriers, then per decoding warp a stream-tile buffer, two W slice buffers and an X
+// buffer; decoding warps: as many as fit, then as few as give the same number of rounds.
 struct LinPlan {
-    uint32_t nbands, KT, splits, kt_per_split, S, npad, tmem_cols, tile_buf, off_bars, off_tile, off_w, off_x;
+    TileMap map;
+    uint32_t nbands, KT, L, nacc, S, npad, tmem_cols, tile_buf, off_bars, off_tile, off_w, off_x;
     uint32_t xrow;  // bytes of one token's K tile in the X buffer: 128 (BF16) or 64 (8-bit codes)
     bool codes;     // an INT8 / FP8 container: the activations are quantized per token first
     size_t smem;
 };
 
 LinPlan lin_plan(const ep_info *info, int sms, int64_t m) {
-    LinPlan L{};
-    L.nbands = uint32_t(info->rows / 128);
-    L.KT = uint32_t(info->cols / 64);
-    uint32_t splits_max = L.nbands < uint32_t(sms) ? uint32_t(sms) / L.nbands : 1u;
-    splits_max = std::max(1u, std::min(splits_max, L.KT));
-    L.kt_per_split = (L.KT + splits_max - 1) / splits_max;
-    L.splits = (L.KT + L.kt_per_split - 1) / L.kt_per_split;
-    L.npad = uint32_t((m + 15) / 16 * 16);
-    L.codes = info->container_dtype != EP_BF16;
-    L.xrow = L.codes ? 64u : 128u;
-    L.tile_buf = uint32_t((info->max_tile_nbytes + kSlack + 15) & ~uint64_t(15));
+    LinPlan P{};
+    P.nbands = uint32_t(info->rows / 128);
+    P.KT = uint32_t(info->cols / 64);
+    const uint32_t T = P.nbands * P.KT;
+    P.npad = uint32_t((m + 15) / 16 * 16);
+    P.codes = info->container_dtype != EP_BF16;
+    P.xrow = P.codes ? 64u : 128u;
+    P.tile_buf = uint32_t((info->max_tile_nbytes + kSlack + 15) & ~uint64_t(15));
     const uint32_t tables = uint32_t(info->paired ? kPairedTableBytes : kLutBytes);
     auto layout = [&](uint32_t S) {
-        L.S = S;
-        L.off_bars = tables;
-        L.off_tile = (L.off_bars + kLinBarBytes * S + 24u + 15u) & ~15u;
-        L.off_w = (L.off_tile + S * L.tile_buf + 127u) & ~127u;
-        L.off_x = L.off_w + S * 2u * kLinSlice;
-        L.smem = size_t(L.off_x) + size_t(S) * L.npad * L.xrow;
+        P.S = S;
+        P.off_bars = tables;
+        P.off_tile = (P.off_bars + kLinBarBytes * S + 24u + 15u) & ~15u;
+        P.off_w = (P.off_tile + S * P.tile_buf + 127u) & ~127u;
+        P.off_x = P.off_w + S * 2u * kLinSlice;
+        P.smem = size_t(P.off_x) + size_t(S) * P.npad * P.xrow;
     };
-    uint32_t S = std::min(kLinMaxWarps, L.kt_per_split);
-    for (layout(S); S > 1 && L.smem > kSmemLimit; layout(--S)) {
+    uint32_t smax = kLinMaxWarps;  // decoding warps that fit beside the tables
+    for (layout(smax); smax > 1 && P.smem > kSmemLimit; layout(--smax)) {
     }
-    const uint32_t rounds = (L.kt_per_split + S - 1) / S;
-    layout((L.kt_per_split + rounds - 1) / rounds);
-    L.tmem_cols = 32;
-    while (L.tmem_cols < L.npad) L.tmem_cols *= 2;
+    auto warps_for = [&](uint32_t L) {  // as few warps as give the fewest rounds
+        const uint32_t S = std::min(smax, L), rounds = (L + S - 1) / S;
+        return (L + rounds - 1) / rounds;
+    };
+    auto most_bands = [&](const TileMap &M) {
+        uint32_t n = 0;
+        for (uint32_t c = 0; c < M.C; ++c) n = std::max(n, (M.first(c + 1) - 1) / P.KT - M.first(c) / P.KT + 1);
+        return n;
+    };
+    const uint32_t waves_sm = uint32_t(std::max(sms, 1));
+    // band-aligned
+    TileMap A{T, 0, P.KT, 0, 0, 1};
+    uint32_t splits_max = P.nbands < waves_sm ? waves_sm / P.nbands : 1u;
+    splits_max = std::max(1u, std::min(splits_max, P.KT));
+    A.ktps = (P.KT + splits_max - 1) / splits_max;
+    A.splits = (P.KT + A.ktps - 1) / A.ktps;
+    A.C = P.nbands * A.splits;
+    const uint32_t SA = warps_for(A.ktps);
+    const uint32_t cost_a = ((A.ktps + SA - 1) / SA) * ((A.C + waves_sm - 1) / waves_sm);
+    // spread evenly
+    TileMap E{T, std::min(waves_sm, T), P.KT, 1, P.KT, 0};
+    uint32_t nacc_e = most_bands(E);
+    while (nacc_e * P.npad > 512u && E.C < T) {
+        E.C = std::min(T, 2u * E.C);
+        nacc_e = most_bands(E);
+    }
+    const uint32_t LE = (T + E.C - 1) / E.C;
+    const uint32_t SE = warps_for(LE);
+    const uint32_t cost_e = ((LE + SE - 1) / SE) * ((E.C + waves_sm - 1) / waves_sm);
+    if (cost_e < cost_a) {
+        P.map = E;
+        P.L = LE;
+        P.nacc = nacc_e;
+        layout(SE);
+    } else {
+        P.map = A;
+        P.L = A.ktps;
+        P.nacc = 1;
+        layout(SA);
+    }
+    P.tmem_cols = 32;
+    while (P.tmem_cols < P.nacc * P.npad) P.tmem_cols *= 2;
     // more than half an SM's shared memory: one CTA per SM, so no CTA waits for another's tensor memory
-    L.smem = std::max(L.smem, kSmemLimit / 2 + 1024);
-    return L;
+    P.smem = std::max(P.smem, kSmemLimit / 2 + 1024);
+    return P;
 }
+// the plan fits the shared memory (the accumulators fit the 512 columns of tensor memory by the
+// choice of C)
+bool lin_fits(const LinPlan &P) { return P.smem <= kSmemLimit && P.tmem_cols <= 512u; }
 
-// the caller's scratch: the partial sums (splits x m x N, fp32 or int32), one counter per band, and
-// for code containers the activations' codes (m x K bytes) and per-token scales (m floats)
-size_t lin_count_offset(const LinPlan &L, int64_t m) {
-    return (size_t(L.splits) * size_t(m) * size_t(L.nbands) * 128u * sizeof(float) + 15u) & ~size_t(15);
+// the caller's scratch: the partial sums (CTAs x nacc slots of m x 128, fp32 or int32), one counter per
+// band, and for code containers the activations' codes (m x K bytes) and per-token scales (m floats)
+size_t lin_count_offset(const LinPlan &P, int64_t m) {
+    return (size_t(P.map.C) * P.nacc * size_t(m) * 128u * sizeof(float) + 15u) & ~size_t(15);
 }
-size_t lin_xq_offset(const LinPlan &L, int64_t m) {
-    return (lin_count_offset(L, m) + size_t(L.nbands) * 4u + 15u) & ~size_t(15);
+size_t lin_xq_offset(const LinPlan &P, int64_t m) {
+    return (lin_count_offset(P, m) + size_t(P.nbands) * 4u + 15u) & ~size_t(15);
 }
-size_t lin_xscale_offset(const LinPlan &L, int64_t m) {
-    return (lin_xq_offset(L, m) + size_t(m) * L.KT * 64u + 15u) & ~size_t(15);
+size_t lin_xscale_offset(const LinPlan &P, int64_t m) {
+    return (lin_xq_offset(P, m) + size_t(m) * P.KT * 64u + 15u) & ~size_t(15);
 }
-size_t lin_work_bytes(const LinPlan &L, int64_t m) {
-    return L.codes ? lin_xscale_offset(L, m) + size_t(m) * 4u : lin_count_offset(L, m) + size_t(L.nbands) * 4u;
+size_t lin_work_bytes(const LinPlan &P, int64_t m) {
+    return P.codes ? lin_xscale_offset(P, m) + size_t(m) * 4u : lin_count_offset(P, m) + size_t(P.nbands) * 4u;
 }
 
 }  // namespace
@@ -463,8 +557,11 @@ extern "C" int ep_linear_fused_plan(const ep_info *info, int64_t m, int32_t sms,
     if (!out || sms < 1 || !linear_ok(info, m)) return EP_ERR_INVALID_ARG;
     const LinPlan L = lin_plan(info, sms, m);
     out->bands = L.nbands;
-    out->splits = L.splits;
-    out->k_tiles_per_split = L.kt_per_split;
+    out->ctas = L.map.C;
+    out->tiles_per_cta = L.L;
+    out->accumulators = L.nacc;
+    out->spread = L.map.aligned ? 0u : 1u;
+    out->splits = L.map.aligned ? L.map.splits : 0u;
     out->decoding_warps = L.S;
     out->threads = std::max(L.S + 1, 4u) * 32u;
     out->tokens_padded = L.npad;
@@ -478,7 +575,7 @@ extern "C" int ep_linear_fused_plan(const ep_info *info, int64_t m, int32_t sms,
     out->smem_x_bytes_per_warp = L.npad * L.xrow;
     out->smem_bytes = L.smem;
     out->work_bytes = lin_work_bytes(L, m);
-    return L.smem > kSmemLimit ? EP_ERR_UNSUPPORTED : EP_OK;
+    return lin_fits(L) ? EP_OK : EP_ERR_UNSUPPORTED;
 }
 
 extern "C" size_t ep_linear_fused_workspace(const ep_info *info, int64_t m) {
@@ -503,7 +600,9 @@ extern "C" int ep_linear_fused(const ep_info *info, const void *d_blob, const vo
     if (device_sms(&device, &sms) != EP_OK) return EP_ERR_CUDA;
     const LinPlan L = lin_plan(info, sms, m);
     if (work_nbytes < lin_work_bytes(L, m)) return EP_ERR_INVALID_ARG;
-    if (L.smem > kSmemLimit) return EP_ERR_UNSUPPORTED;  // tiles too large for one warp's buffers beside the tables
+    // tiles too large for one warp's buffers beside the tables, or too many bands per CTA for the
+    // accumulators of a large token count
+    if (!lin_fits(L)) return EP_ERR_UNSUPPORTED;
     LinParams P;
     P.dp = params_of(info, d_blob, d_tables, nullptr, d_status);
     P.x = static_cast<const uint16_t *>(d_x);
@@ -511,7 +610,8 @@ extern "C" int ep_linear_fused(const ep_info *info, const void *d_blob, const vo
     P.count = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(d_work) + lin_count_offset(L, m));
     P.bias = static_cast<const uint16_t *>(d_bias);
     P.y = static_cast<uint16_t *>(d_y);
-    P.splits = L.splits;
+    P.map = L.map;
+    P.nacc = L.nacc;
     P.M = uint32_t(m);
     P.N = uint32_t(info->rows);
     P.npad = L.npad;
@@ -525,7 +625,6 @@ extern "C" int ep_linear_fused(const ep_info *info, const void *d_blob, const vo
     P.idesc = types | ((L.npad >> 3) << 17) | ((128u >> 4) << 24);
     P.tmem_cols = L.tmem_cols;
     P.KT = L.KT;
-    P.kt_per_split = L.kt_per_split;
     P.S = L.S;
     P.tile_buf = L.tile_buf;
     P.off_bars = L.off_bars;
@@ -567,7 +666,7 @@ extern "C" int ep_linear_fused(const ep_info *info, const void *d_blob, const vo
         if (cudaGetLastError() != cudaSuccess) return EP_ERR_CUDA;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(L.nbands, L.splits);
+    cfg.gridDim = dim3(L.map.C);
     cfg.blockDim = dim3(std::max(L.S + 1, 4u) * 32);  // the epilogue needs warps 0..3
     cfg.dynamicSmemBytes = L.smem;
     cfg.stream = s;

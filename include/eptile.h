@@ -235,25 +235,33 @@ int ep_decompress(const ep_info *info, const void *d_blob, const void *d_workspa
  *               zero-filled before its first use; every call leaves the counters at zero again.
  *               One call at a time per scratch buffer.
  *   d_status    nullable device uint32: EP_DEC_* bits of stream damage.
- * One launch (INT8 / FP8: after one launch that quantizes X): a CTA per band of 128 output features
- * and range of K tiles.  Its warps bulk-copy stream tiles into shared memory and decode them
+ * One launch (INT8 / FP8: after one launch that quantizes X): the stream's tiles in ranges over about
+ * one wave of CTAs.  Their warps bulk-copy stream tiles into shared memory and decode them
  * straight into operand slices (128 features x 32 bytes: 16 BF16 weights or 32 codes) beside the
  * matching slices of X; one warp issues tcgen05.mma (kind::f16, kind::i8 or kind::f8f6f4; M = 128
- * features, N = m padded to 16) into an accumulator in tensor memory, read out with tcgen05.ld into
- * the partial sums; the band's last CTA adds the splits in order, scales and adds the bias.
+ * features, N = m padded to 16) into the accumulator of the tile's band in tensor memory, read out
+ * with tcgen05.ld into partial sums; a band's last CTA adds its CTAs' sums in order, scales and adds
+ * the bias.
  * Asynchronous; allocates nothing.  EP_ERR_INVALID_ARG for another layout, container or m out of
  * range, EP_ERR_UNSUPPORTED when a tile is too large for the shared memory of one decoding warp. */
 size_t ep_linear_fused_workspace(const ep_info *info, int64_t m);
 
 /* The launch ep_linear_fused would make for this stream and m on a GPU with `sms` multiprocessors,
- * computed on the host without touching a device (for tests and capacity planning): the grid
- * (bands of 128 output features x K splits, one wave), the decoding warps per CTA, the padded
- * token count, the tensor-memory columns, the shared-memory layout (tables from offset 0, then the
- * barriers, the per-warp stream-tile buffers, the per-warp pairs of 4 KB W slices and the per-warp
- * X buffers) and the scratch bytes.  EP_ERR_INVALID_ARG as ep_linear_fused refuses the stream or m,
- * EP_ERR_UNSUPPORTED when even one decoding warp's buffers do not fit (*out is filled either way). */
+ * computed on the host without touching a device (for tests and capacity planning): the grid (each
+ * band's K tiles split into ranges, about one wave of CTAs, or all tiles spread evenly over one wave
+ * when that gives each decoding warp fewer rounds of tiles, more CTAs when one would touch more
+ * bands than tensor memory holds accumulators for; the most tiles and the most bands of 128 output
+ * features one CTA holds), the decoding warps per CTA, the padded token
+ * count, the tensor-memory columns (one accumulator per band a CTA touches), the shared-memory
+ * layout (tables from offset 0, then the barriers, the per-warp stream-tile buffers, the per-warp
+ * pairs of 4 KB W slices and the per-warp X buffers) and the scratch bytes.  EP_ERR_INVALID_ARG as
+ * ep_linear_fused refuses the stream or m, EP_ERR_UNSUPPORTED when even one decoding warp's buffers
+ * do not fit (*out is filled either way). */
 typedef struct {
-    uint32_t bands, splits, k_tiles_per_split, decoding_warps, threads, tokens_padded, tmem_columns;
+    uint32_t bands, ctas, tiles_per_cta, accumulators;
+    uint32_t spread;  /* 1: tiles spread evenly over the CTAs; 0: each band's K tiles in `splits` ranges */
+    uint32_t splits;
+    uint32_t decoding_warps, threads, tokens_padded, tmem_columns;
     uint32_t tile_buffer_bytes, smem_tables_bytes, smem_barriers_offset, smem_tiles_offset, smem_slices_offset;
     uint32_t smem_x_offset, smem_x_bytes_per_warp;
     uint64_t smem_bytes, work_bytes;
