@@ -125,7 +125,7 @@ struct Packer<EP_BF16> {
     __device__ __forceinline__ void store(void *out, uint32_t b) {
         reinterpret_cast<uint4 *>(out)[b] = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    // the 8 values as 16 bytes at a shared-memory address (an operand tile of the fused GEMM)
+    // the 8 values as 16 bytes at a shared-memory address (an operand slice of the fused GEMM)
     __device__ __forceinline__ void store_shared(uint32_t a) {
         asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
                      : "memory");

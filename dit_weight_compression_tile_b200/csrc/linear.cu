@@ -13,17 +13,18 @@ namespace {
 // ------------------------------------------------------------------ the decode fused into a GEMM
 // Y^T = W X^T for a weight W (N x K) held as a GEMM-ordered stream (EP_LAYOUT_GEMM): each stream tile
 // is one 128 x 64 tile of W, tiles in band-major order (a band: 128 output features, all K tiles).
-// The tiles are spread evenly over one wave of CTAs, one per SM: CTA c takes tiles
-// [c T / C, (c + 1) T / C), which may span two or more bands.  Warps 0 .. S-1 decode, one tile at a
-// time each: a bulk copy of the stream tile into the warp's buffer,
-// the matching slice of X (tokens padded to a multiple of 16) into the warp's X buffer, then the
-// tile's 32 steps.  Every 8 steps complete a 128 x 16 K-slice of the tile, which goes to one of the
-// warp's two 4 KB slice buffers (a ring) and is announced on that buffer's `full` barrier.  Warp S
-// issues the tensor-core work: for each round of tiles, slice by slice, warp by warp (a fixed
-// order, so the fp32 sums are the same on every call), one tcgen05.mma (M = 128 features,
-// N = tokens, K = 16, A = the W slice, B = the X slice, both K-major) into the tensor-memory
-// accumulator of the tile's band (one per band the CTA touches), committed to the slice buffer's
-// `empty` barrier.  After the last MMA, warps 0..3 read the accumulators out of tensor memory into
+// Each CTA (one per SM) takes a range of tiles (TileMap): a range of one band's K tiles, or, where
+// whole bands would leave SMs idle, an even share of all tiles that may span two or more bands.
+// Warps 0 .. S-1 decode, one tile at a time each: a bulk copy of the stream tile into the warp's
+// buffer, the matching slice of X (tokens padded to a multiple of 16: BF16 activations, or their
+// 8-bit codes) into the warp's X buffer, then the tile's 32 steps.  Every 8 steps (16 for 8-bit
+// codes) complete a K-slice of the tile, 128 features x 32 bytes, which goes to one of the warp's
+// two 4 KB slice buffers (a ring) and is announced on that buffer's `full` barrier.  Warp S issues
+// the tensor-core work: for each round of tiles, slice by slice, warp by warp (a fixed order, so
+// the sums are the same on every call), one tcgen05.mma (M = 128 features, N = tokens, K = 16 BF16
+// or 32 codes, A = the W slice, B = the X slice, both K-major) into the tensor-memory accumulator
+// of the tile's band (one per band the CTA touches), committed to the slice buffer's `empty`
+// barrier.  After the last MMA, warps 0..3 read the accumulators out of tensor memory into
 // the CTA's partial sums; the last CTA to finish a band adds the partial sums of the CTAs that
 // touched it in CTA order (the same sums on every call), scales, adds the bias, rounds once to BF16
 // and writes the band's part of Y.
