@@ -2,7 +2,7 @@
 instance a plugin inside an inference engine that owns all device memory, or code that must
 avoid the synchronisation a cudaMalloc can cause): it keeps the decoder's tables in a static
 device array instead of a caller workspace.  Called through the C ABI, its output must equal
-the workspace path's (ep_prepare + ep_decompress) bit for bit, on calls in a row with
+the workspace path's (ep_prepare + ep_decompress) and the oracle's bit for bit, on calls in a row with
 different streams and table layouts (paired, single-coded, paired), so each call must replace
 the previous call's tables.
 
@@ -36,7 +36,7 @@ def workspace_decode(d_blob, info, stream):
     return out, status
 
 
-def test_noalloc_matches_workspace_path_twice():
+def test_noalloc_matches_workspace_path_twice(oracle):
     # a paired stream (108,544 bytes of tables) then a single-coded one (57,344 bytes) and a paired
     # one again: each call must leave its own tables in the shared array, whatever the one before
     cases = [(synth.row_lognormal(512, 2048, 21), 4.0, 0, B.CODING_PAIRED),
@@ -56,6 +56,11 @@ def test_noalloc_matches_workspace_path_twice():
         assert int(st_got.item()) == 0 and int(st_ref.item()) == 0
         assert got.dtype == ref.dtype and got.shape == ref.shape
         assert np.array_equal(got.view(torch.uint8).cpu().numpy(), ref.view(torch.uint8).cpu().numpy())
+        # and both equal the oracle's decode of the same stream, byte for byte
+        rc, st, _, out_ref = oracle.decode(blob.numpy())
+        assert rc == 0 and st == 0
+        assert np.array_equal(got.contiguous().view(torch.uint8).cpu().numpy().reshape(-1),
+                              out_ref.view(np.uint8).reshape(-1))
     assert layouts == [(1, 108544), (0, 57344), (1, 108544)]
 
 
